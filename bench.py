@@ -1,0 +1,431 @@
+"""Benchmark of the S3R per-round hot path on B200 (one process per GPU).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config 2]
+
+A step is one whole S3R round over the batch of the chosen synthetic workload (default:
+the Qwen3-8B-shaped single attention layer, 32 requests with contexts uniform in
+[8192, 24576], k = 6, s = 0.05, vocabulary 151936): select, k x (sparse draft attention +
+draft sampling), dense verify with score capture, speculative sampling and commit, every
+step in libs3r.so. Each step starts from the workload's committed lengths (the lengths are
+restored by a 4-byte-per-request device copy), so every timed step is the same workload.
+Inputs (KV cache 2.1 GB, logits 0.25 GB per round) are larger than the 126 MB L2.
+
+Rank 0 prints one JSON line. `--impl reference` times the CPU oracle instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "accepted tokens/s per draft+verify round"
+UNIT = "tokens/s"
+
+
+# ------------------------------------------------------------------------ helpers -------
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(
+        os.environ.get("LOCAL_RANK", 0))
+
+
+def reduce_results(elapsed_ms: float, tokens: int, group=None):
+    """Max of elapsed time and sum of tokens over ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return elapsed_ms, tokens
+    dev = "cuda" if dist.get_backend(group) == "nccl" else "cpu"
+    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+    n = torch.tensor([tokens], dtype=torch.int64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX, group=group)
+    dist.all_reduce(n, op=dist.ReduceOp.SUM, group=group)
+    return float(t.item()), int(n.item())
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_source_hash(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+VERIFY_SOURCES = ["sparse_dense_kv_b200/csrc/verify.cu", "sparse_dense_kv_b200/csrc/attention.cuh",
+                  "sparse_dense_kv_b200/csrc/common.cuh"]
+
+
+def verify_traffic_per_launch(workload: str):
+    """DRAM bytes per verify launch from the committed ncu summary, if it was taken on the
+    current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "verify_attn_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    if d.get("source_hash") != kernel_source_hash(VERIFY_SOURCES):
+        return None
+    return d.get("per_launch_bytes", {}).get(workload)
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 100 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.rows = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append((time.time(), [x.strip() for x in line.split(",")]))
+
+    def stop(self, t0, t1):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = [r for t, r in self.rows if t0 - 0.15 <= t <= t1 + 0.15] or [r for _, r in self.rows]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if len(r) > 5 + i and r[5 + i] == "Active"})
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+# -------------------------------------------------------------------- GPU workload ------
+def build_workload(spec, rank, device):
+    import torch
+    lens = synth.make_lengths(spec)
+    k = spec.k
+    cache = synth.build_cache(spec, lens, extra_tokens=k + 1 + 16, device=device,
+                              seed=spec.data_seed + 7919 * rank)
+    NR, Hq, Hkv, d, V = spec.num_requests, spec.num_q_heads, spec.num_kv_heads, spec.head_dim, spec.vocab
+    s = 100 + 13 * rank
+    inp = dict(
+        q=synth.randn_bf16((NR, k + 1, Hq, d), s, device),
+        k=synth.randn_bf16((NR, k + 1, Hkv, d), s + 1, device),
+        v=synth.randn_bf16((NR, k + 1, Hkv, d), s + 2, device),
+        p=synth.randn_f32((NR, k + 1, V), s + 3, device, scale=spec.logit_std),
+    )
+    inp["qlog"] = (inp["p"][:, :k] + synth.randn_f32((NR, k, V), s + 4, device,
+                                                      scale=spec.draft_noise_std)).contiguous()
+    seq = torch.as_tensor(lens, dtype=torch.int32, device=device)
+    return lens, cache, seq, inp
+
+
+def algorithmic_bytes(spec, lens):
+    """KV bytes per launch: verify reads (L+k+1) positions, draft step i reads n+i+1 positions
+    (+4 B per selected index), 2*d*2 bytes per position and KV head."""
+    from sparse_dense_kv_b200.engine import budget_count
+    Hkv, d, k = spec.num_kv_heads, spec.head_dim, spec.k
+    per_pos = 2 * d * 2 * Hkv
+    verify = int(sum((L + k + 1) for L in lens)) * per_pos
+    draft = []
+    for i in range(k):
+        tot = 0
+        for L in lens:
+            n = budget_count(int(L), spec.budget_bp, spec.window)
+            tot += (n + i + 1) * per_pos + 4 * n * Hkv
+        draft.append(tot)
+    G = spec.num_q_heads // Hkv
+    scores = int(sum(lens)) * Hkv * G * (k + 1) * 4
+    return verify, draft, scores
+
+
+def run_ours(args, spec):
+    import torch
+    import torch.distributed as dist
+    import sparse_dense_kv_b200 as s3r
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1 and not dist.is_initialized():
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    lens, cache, seq, inp = build_workload(spec, rank, dev)
+    k = spec.k
+    eng = s3r.S3REngine(cache.k_pool, cache.v_pool, cache.page_table, seq, spec.num_q_heads,
+                        k=k, budget_bp=spec.budget_bp, window=spec.window, vocab=spec.vocab,
+                        seed=spec.sample_seed + rank)
+    seq0 = seq.clone()
+    eng.prefill(inp["q"][:, :1].contiguous(), inp["k"][:, :1].contiguous(), inp["v"][:, :1].contiguous())
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        seq.copy_(seq0, non_blocking=True)
+        eng.select()
+        for i in range(k):
+            if ev is not None:
+                ev["d0"][i].record(stream)
+            eng.draft_step(i, inp["q"], inp["k"], inp["v"], inp["qlog"])
+            if ev is not None:
+                ev["d1"][i].record(stream)
+        if ev is not None:
+            ev["v0"].record(stream)
+        eng.verify(inp["q"], inp["k"], inp["v"])
+        if ev is not None:
+            ev["v1"].record(stream)
+        eng.sample_and_commit(inp["p"], inp["qlog"])
+
+    for _ in range(args.warmup):
+        step()
+    assert eng.check_errors() == 0, "device error during warm-up"
+
+    E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    evs = [dict(d0=[E() for _ in range(k)], d1=[E() for _ in range(k)], v0=E(), v1=E())
+           for _ in range(args.steps)]
+    start, end = E(), E()
+    tok0 = int(eng.buf.stats[0].item())
+    launches0 = s3r.s3r_launch_count()
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = time.time()
+    start.record(stream)
+    for s in range(args.steps):
+        step(evs[s])
+    end.record(stream)
+    torch.cuda.synchronize()
+    t1 = time.time()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop(t0, t1)
+    launches = s3r.s3r_launch_count() - launches0
+    ms = start.elapsed_time(end)
+    tokens = int(eng.buf.stats[0].item()) - tok0
+    assert eng.check_errors() == 0, "device error in the timed region"
+    ms_max, tokens_all = reduce_results(ms, tokens)
+
+    # per-kernel device times (same stream) and roofline of the dominant kernel (verify)
+    v_ms = sum(e["v0"].elapsed_time(e["v1"]) for e in evs) / args.steps
+    d_ms = [sum(e["d0"][i].elapsed_time(e["d1"][i]) for e in evs) / args.steps for i in range(k)]
+    vb, db, sb = algorithmic_bytes(spec, lens)
+    peak, peak_kind = measured_peaks()
+    v_gbs = vb / (v_ms * 1e-3) / 1e9
+    d_gbs = sum(db) / (sum(d_ms) * 1e-3) / 1e9
+
+    # end to end through the public API: pinned host inputs in, tokens out, every round
+    e2e = None
+    if args.e2e_steps > 0:
+        host = {n: t.cpu().pin_memory() for n, t in inp.items()}
+        out_h = torch.empty((spec.num_requests, k + 1), dtype=torch.int32).pin_memory()
+        n_h = torch.empty((spec.num_requests,), dtype=torch.int32).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = out_h.numel() * 4 + n_h.numel() * 4
+        e0, e1 = E(), E()
+        tok_e = int(eng.buf.stats[0].item())
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            for n_, t in host.items():
+                inp[n_].copy_(t, non_blocking=True)
+            step()
+            out_h.copy_(eng.buf.out_tokens, non_blocking=True)
+            n_h.copy_(eng.buf.n_out, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        tok_e = int(eng.buf.stats[0].item()) - tok_e
+        ems, etok = reduce_results(e0.elapsed_time(e1), tok_e)
+        e2e = {"value": etok / (ems * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
+
+    st = eng.buf.stats.cpu().numpy()
+    acc = [float(st[2 + j] / max(st[2 + k + j], 1)) for j in range(k)]
+    result = {
+        "metric": METRIC, "value": tokens_all / (ms_max * 1e-3), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{spec.name} (config {args.config}): {spec.num_requests} requests, "
+                               f"L {spec.lengths}, {spec.num_q_heads}/{spec.num_kv_heads} heads, "
+                               f"d {spec.head_dim}, k {k}, s {spec.budget_bp / 1e4}, window {spec.window}, "
+                               f"vocab {spec.vocab}",
+                   "requests_per_gpu": spec.num_requests, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (KV 2.1 GB, logits 0.25 GB per round)"},
+        "roofline": {"bound": "hbm", "achieved": v_gbs, "peak": peak, "unit": "GB/s",
+                     "frac": v_gbs / peak, "traffic": verify_traffic_per_launch(spec.name),
+                     "kernel": "s3r_verify_attn", "peak_kind": peak_kind,
+                     "algorithmic_bytes_per_launch": vb},
+        "kernels": {"verify_ms": v_ms, "verify_kv_gbs": v_gbs,
+                    "verify_gbs_with_scores": (vb + sb) / (v_ms * 1e-3) / 1e9,
+                    "draft_ms_per_step": sum(d_ms) / k, "draft_kv_gbs": d_gbs,
+                    "frac_of_8tbs": {"verify": v_gbs / 8000.0, "draft": d_gbs / 8000.0}},
+        "tau": float(st[0] / max(st[1], 1)), "acceptance_by_position": acc,
+        "gpu_launches": int(launches), "clocks": clocks, "e2e": e2e,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(spec, lens, cache, inp, budget_s=args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------------- oracle -------
+def oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        return 1
+
+
+def oracle_round_sample(spec, lens, pools, page_table, inp_host, reqs):
+    """Oracle rounds for the requests `reqs` (dense copies built outside the timing)."""
+    from oracle import s3r_oracle as O
+    k = spec.k
+    kp, vp = pools
+    prepared = []
+    for r in reqs:
+        L = int(lens[r])
+        H = spec.num_kv_heads
+        K = np.stack([O.gather_positions(kp, page_table[r], h, np.arange(L + k + 1)) for h in range(H)])
+        V = np.stack([O.gather_positions(vp, page_table[r], h, np.arange(L + k + 1)) for h in range(H)])
+        st = O.RequestState(K, V, L)
+        q = inp_host["q"][r].astype(np.float64)
+        O.prefill_scores(st, q[0], inp_host["k"][r][0], inp_host["v"][r][0])
+        prepared.append((r, st))
+    t0 = time.perf_counter()
+    tokens = 0
+    for r, st in prepared:
+        res = O.run_round(st, r, spec.sample_seed, k, spec.budget_bp, spec.window,
+                          inp_host["q"][r], inp_host["k"][r], inp_host["v"][r],
+                          inp_host["qlog"][r], inp_host["p"][r])
+        tokens += res["n_out"]
+    return tokens, time.perf_counter() - t0
+
+
+def host_inputs(inp, reqs):
+    return {n: {r: t[r].float().cpu().numpy() for r in reqs} for n, t in inp.items()}
+
+
+def cpu_baseline(spec, lens, cache, inp, budget_s=15.0):
+    """The oracle on this host's cores on a bounded sample of the same workload."""
+    reqs, tokens, secs = [], 0, 0.0
+    pools = (cache.k_pool.float().cpu().numpy(), cache.v_pool.float().cpu().numpy())
+    pt = cache.page_table.cpu().numpy()
+    r = 0
+    while secs < budget_s and r < spec.num_requests:
+        hi = host_inputs(inp, [r])
+        t, s = oracle_round_sample(spec, lens, pools, pt, hi, [r])
+        tokens, secs = tokens + t, secs + s
+        reqs.append(r)
+        r += 1
+    return {"value": tokens / secs, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+            "sample": f"one round of requests {reqs[0]}..{reqs[-1]} ({len(reqs)} of "
+                      f"{spec.num_requests}), float64 numpy, {secs:.1f} s"}
+
+
+def run_reference(args, spec):
+    """The CPU oracle as the reference arm: each step = one round of one request."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import torch
+    sub = spec.with_(num_requests=max(1, min(spec.num_requests, 4)))
+    lens = synth.make_lengths(spec)[: sub.num_requests]
+    cache = synth.build_cache(sub.with_(lengths=("fixed", tuple(int(x) for x in lens))), lens,
+                              extra_tokens=spec.k + 1 + 16, device="cpu")
+    k = spec.k
+    NR = sub.num_requests
+    inp = dict(q=synth.randn_bf16((NR, k + 1, spec.num_q_heads, spec.head_dim), 100),
+               k=synth.randn_bf16((NR, k + 1, spec.num_kv_heads, spec.head_dim), 101),
+               v=synth.randn_bf16((NR, k + 1, spec.num_kv_heads, spec.head_dim), 102),
+               p=synth.randn_f32((NR, k + 1, spec.vocab), 103, scale=spec.logit_std))
+    inp["qlog"] = inp["p"][:, :k] + synth.randn_f32((NR, k, spec.vocab), 104, scale=spec.draft_noise_std)
+    pools = (cache.k_pool.float().numpy(), cache.v_pool.float().numpy())
+    pt = cache.page_table.numpy()
+    tok, secs = 0, 0.0
+    for s in range(args.warmup + args.steps):
+        r = s % NR
+        hi = host_inputs(inp, [r])
+        t, dt = oracle_round_sample(spec, lens, pools, pt, hi, [r])
+        if s >= args.warmup:
+            tok, secs = tok + t, secs + dt
+    v = tok / secs
+    out = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic",
+           "config": {"workload": f"{spec.name} (config {args.config}), one request-round per step",
+                      "requests_sampled": NR},
+           "cpu_baseline": {"value": v, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+                            "sample": f"{args.steps} request-rounds over {NR} requests of the workload"},
+           "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+    del torch
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", type=int, default=2)
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    spec = synth.CONFIGS[args.config]
+    if spec.projection_logits or spec.mixed_phases:
+        raise SystemExit("config 3 (mixed phases) and 4 (sweep) are parity / sweep cases, not bench lines")
+    if args.impl == "reference":
+        run_reference(args, spec)
+    else:
+        run_ours(args, spec)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,218 @@
+/*
+ * s3r.h - C ABI of libs3r.so: the per-round hot path of Self-Sparse Speculative Rollouts
+ * (S3R) over a paged bf16 GQA KV cache, as hand-written CUDA kernels for sm_100a (B200).
+ *
+ * Sources (by page title and section):
+ *   [News]      "Long-context RL training stops waiting on autoregressive rollouts: sparse
+ *               self-drafting plus full-attention verification lifts throughput 1.39x",
+ *               Interpretation and Perspective.
+ *   [Listing]   "S^3R: Fast and Faithful RL Rollouts via Self-Sparse Speculative Decoding",
+ *               Abstract; appendix Tables 4-7.
+ *   [Explainer] "S3R - Self-sparse speculative rollouts for RL - What does it mean?",
+ *               Jargon, walkthrough, "Where it earns its keep".
+ *
+ * One round of one request with committed length L and pending token x at position L:
+ *   s3r_select_kv          sparse set S (n = ceil(s*L) positions) from the last verify's scores
+ *   k x s3r_sparse_draft_attn + s3r_draft_sample     draft tokens d_1..d_k
+ *   s3r_verify_attn        dense attention of the k+1 rows at L..L+k, with score capture
+ *   s3r_spec_sample        exact speculative sampling -> a accepted drafts + 1 token
+ *   s3r_commit             L <- L + a + 1, acceptance counters
+ *
+ * Conventions shared by every call
+ *   - Every pointer argument is a DEVICE pointer owned by the caller, unless it is marked
+ *     "host". The library keeps no pointer after a call returns and allocates no memory.
+ *   - Every call is asynchronous on the given stream (NULL = legacy default stream) and
+ *     returns an s3r_status. Arguments are validated on the host before anything is
+ *     launched; a non-OK status means nothing was launched.
+ *   - Faults the host cannot see (a page id outside the pool, a selected index >= L, a
+ *     context longer than the page table, a non-finite logit, an expired wait) are
+ *     recorded in the workspace's error word as bit (1 << S3R_ERR_*) and the offending
+ *     access is skipped; kernels never trap. s3r_get_error() reads and clears the word.
+ *   - KV pools: bf16 [num_pages][num_kv_heads][16][head_dim]; head_dim is 64 or 128.
+ *     Query head h reads KV head h / G, G = num_q_heads / num_kv_heads <= 8.
+ *   - Requests: a launch covers `batch` requests; with req_ids == NULL they are requests
+ *     0..batch-1, else req_ids[0..batch-1]. Every per-request array is indexed by the
+ *     request id (size num_requests), so a launch can cover a subset of a larger batch
+ *     (mixed round phases).
+ *     Attention and selection calls cover at most 65535 requests per launch.
+ *   - Page table: int32 [num_requests][max_pages_per_req]; position j of request r is
+ *     slot j % 16 of page page_table[r][j / 16]. capacity = 16 * max_pages_per_req.
+ *   - A workspace serves one stream at a time. It must be zeroed once by
+ *     s3r_workspace_init before first use; every call leaves it ready for the next.
+ */
+#ifndef S3R_H_
+#define S3R_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define S3R_API __attribute__((visibility("default")))
+#else
+#define S3R_API
+#endif
+
+typedef struct CUstream_st* s3r_stream_t; /* same handle as cudaStream_t */
+
+typedef enum {
+  S3R_OK = 0,
+  S3R_ERR_INVALID_ARG = 1,   /* a NULL/misaligned pointer or a size out of range */
+  S3R_ERR_UNSUPPORTED = 2,   /* head_dim, page size, group or k outside what is built */
+  S3R_ERR_CUDA = 3,          /* a CUDA runtime call failed (launch, copy, attribute) */
+  S3R_ERR_WORKSPACE = 4,     /* workspace NULL, misaligned or smaller than needed */
+  S3R_ERR_DEVICE_BOUNDS = 5, /* device: page id / index / length outside its range */
+  S3R_ERR_NONFINITE = 6,     /* device: NaN or Inf in logits or scores */
+  S3R_ERR_TIMEOUT = 7        /* device: a bounded wait on a copy expired */
+} s3r_status;
+
+#define S3R_PAGE_SIZE 16
+#define S3R_MAX_K 8          /* draft length k <= 8 */
+#define S3R_MAX_GROUP 8      /* query heads per KV head */
+#define S3R_MAX_ROWS 64      /* G * (k + 1) rows of one KV head in a verify */
+
+typedef struct {
+  int32_t num_q_heads;
+  int32_t num_kv_heads;
+  int32_t head_dim;          /* 64 or 128 */
+  int32_t page_size;         /* must be 16 */
+  int64_t num_pages;
+  void* k_pool;              /* bf16 [num_pages][num_kv_heads][16][head_dim], 16-byte aligned */
+  void* v_pool;              /* same layout */
+} s3r_kv_cache;
+
+typedef struct {
+  int32_t batch;             /* requests covered by this launch (0 = nothing to do) */
+  int32_t num_requests;      /* size of every per-request array */
+  const int32_t* req_ids;    /* [batch] request ids, or NULL for 0..batch-1 */
+  const int32_t* seq_lens;   /* [num_requests] committed length L per request */
+  const int32_t* page_table; /* [num_requests][max_pages_per_req] */
+  int32_t max_pages_per_req;
+} s3r_batch;
+
+/* Bytes of workspace that every call below needs for a cache with this shape, up to
+ * num_requests requests, page tables of max_pages_per_req pages, draft length <= max_k,
+ * vocabularies <= vocab and selections of <= sel_stride positions. Pure host function. */
+S3R_API size_t s3r_workspace_size(const s3r_kv_cache* cache, int32_t num_requests,
+                          int32_t max_pages_per_req, int32_t max_k, int32_t vocab,
+                          int32_t sel_stride);
+
+/* Zero a workspace (256-byte aligned device buffer of ws_bytes bytes). */
+S3R_API int s3r_workspace_init(void* ws, size_t ws_bytes, s3r_stream_t stream);
+
+/* Dense verify attention with score capture ([News] Interpretation: verification recomputes
+ * the proposed block against the complete historical KV; [Explainer] walkthrough: the
+ * sparse set is refreshed from the verifier's last attention pass).
+ *   k          draft length; the block has T = k+1 rows at positions L..L+k (0 <= k <= 8;
+ *              k = 0 is the one-row pass of a prefill's last token).
+ *   q          bf16 [num_requests][T][H_q][d]; row t of head h attends positions 0..L+t.
+ *   k_new,v_new bf16 [num_requests][T][H_kv][d]: K/V of the block; written into the pages
+ *              of positions L..L+k (which must be allocated) and used for the block.
+ *   out        bf16 [num_requests][T][H_q][d], softmax(q K^T / sqrt(d)) V rounded once.
+ *   lse        fp32 [num_requests][T][H_q], natural-log log-sum-exp of the logits.
+ *   score_logits fp32 [num_requests][H_kv][G*T][capacity] or NULL: logit q.k/sqrt(d) of
+ *              row t*G+g of each KV head at every committed position j < L (entries at
+ *              j >= L are not written). With lse it defines the scores of s3r_select_kv.
+ * Needs L + T <= capacity (device check). */
+S3R_API int s3r_verify_attn(const s3r_kv_cache* cache, const s3r_batch* batch, int32_t k,
+                    const void* q, const void* k_new, const void* v_new, void* out,
+                    float* lse, float* score_logits, void* ws, size_t ws_bytes,
+                    s3r_stream_t stream);
+
+/* Sparse KV selection ([Explainer] Jargon, sparse attention budget: a fraction s of the
+ * cached positions, the newest ones plus those the verifier attended to most).
+ * For request r at committed length L (seq_lens, already advanced by s3r_commit) and KV
+ * head h: W' = min(window, L), n = clamp(ceil(L * budget_bp / 10000), W', L), and the set
+ * is the W' newest positions plus the n - W' positions j < L - W' of highest score
+ *   sigma_j = sum over the G*(k_prev+1) rows of exp(score_logits[row][j] - lse[row]),
+ * ties to the lower j, written ascending to sel_idx[r][h][0..n-1]; sel_count[r][h] = n.
+ *   score_logits, lse  as written by the previous s3r_verify_attn with k = k_prev.
+ *   sel_idx    int32 [num_requests][H_kv][sel_stride]; n > sel_stride is a device bounds
+ *              error. sel_count int32 [num_requests][H_kv].
+ * Needs 1 <= budget_bp <= 10000 and window >= k_prev + 1 (so that every scored non-window
+ * position is committed), L - W' <= 49152. */
+S3R_API int s3r_select_kv(const s3r_kv_cache* cache, const s3r_batch* batch, const float* score_logits,
+                  const float* lse, int32_t k_prev, int32_t budget_bp, int32_t window,
+                  int32_t* sel_idx, int32_t sel_stride, int32_t* sel_count, void* ws,
+                  size_t ws_bytes, s3r_stream_t stream);
+
+/* The same selection from caller-given scores: scores fp32 [num_requests][H_kv][score_stride],
+ * sigma_j = scores[r][h][j] (any finite float; order by value, ties to the lower j). */
+S3R_API int s3r_select_from_scores(const s3r_kv_cache* cache, const s3r_batch* batch,
+                           const float* scores, int32_t score_stride, int32_t budget_bp,
+                           int32_t window, int32_t* sel_idx, int32_t sel_stride,
+                           int32_t* sel_count, void* ws, size_t ws_bytes, s3r_stream_t stream);
+
+/* Sparse self-draft attention ([News] Interpretation; [Explainer] "How is this different":
+ * the same weights reading a sparse subset of the KV cache). Draft step i = draft_step[r]
+ * handles the token at position L+i: its K/V (k_new, v_new) are written to that position's
+ * page, and its query rows attend S (sel_idx[r][h][0..n-1], every index < L) plus the block
+ * positions L..L+i (the earlier ones written by the earlier steps of the round).
+ *   q      bf16, request r's [H_q][d] rows at q + r * q_stride (elements; 0 means H_q * d)
+ *   k_new, v_new bf16, request r's [H_kv][d] rows at k_new + r * kv_stride (0 means H_kv * d)
+ *          (strides let a caller pass step i of a [num_requests][k+1][...] block in place)
+ *   out    bf16 [num_requests][H_q][d];  lse fp32 [num_requests][H_q] or NULL. */
+S3R_API int s3r_sparse_draft_attn(const s3r_kv_cache* cache, const s3r_batch* batch,
+                          const int32_t* draft_step, const void* q, int32_t q_stride,
+                          const void* k_new, const void* v_new, int32_t kv_stride,
+                          const int32_t* sel_idx, int32_t sel_stride,
+                          const int32_t* sel_count, void* out, float* lse, void* ws,
+                          size_t ws_bytes, s3r_stream_t stream);
+
+/* Draft-token sampling (temperature 1). For request r at step i = draft_step[r]:
+ * q_i = softmax(q_logits[r][i][0..vocab-1]); u = Philox4x32-10(key = seed,
+ * counter = (L+i+1, r, 0, 0)) word 0 >> 8, times 2^-24; the token is the smallest v with
+ * u * Z < C_v (C inclusive cumulative sum of exp(x - max), Z its total), written to
+ * draft_tokens[r][i].  q_logits fp32 [num_requests][k][vocab]; draft_tokens int32
+ * [num_requests][k]. */
+S3R_API int s3r_draft_sample(const s3r_batch* batch, const int32_t* draft_step, int32_t k,
+                     const float* q_logits, int32_t vocab, uint64_t seed, int32_t* draft_tokens,
+                     void* ws, size_t ws_bytes, s3r_stream_t stream);
+
+/* Exact speculative sampling ([News] Interpretation; [Explainer] Jargon, exact speculative
+ * sampling). p_j = softmax(p_logits[r][j]) (j = 0..k), q_j = softmax(q_logits[r][j])
+ * (j < k) are the target / draft distributions of the token at position L+j+1.
+ * Draft j is accepted iff u1 * q_j(d) < p_j(d), u1 from counter (L+j+1, r, 1, 0). At the
+ * first rejection the token is drawn from max(0, p_j - q_j) normalised (from p_j if that is
+ * all zero) with u2 from counter (L+j+1, r, 2, 0); if all k pass, from p_k with
+ * counter (L+k+1, r, 2, 0).  out_tokens int32 [num_requests][k+1] receives the a accepted
+ * drafts and the drawn token (entries after them untouched); n_out[r] = a + 1. */
+S3R_API int s3r_spec_sample(const s3r_batch* batch, int32_t k, const float* p_logits,
+                    const float* q_logits, const int32_t* draft_tokens, int32_t vocab,
+                    uint64_t seed, int32_t* out_tokens, int32_t* n_out, void* ws,
+                    size_t ws_bytes, s3r_stream_t stream);
+
+/* Commit a round ([Explainer] Jargon, block efficiency: tokens per round): for each
+ * request of the batch, seq_lens[r] += n_out[r]. stats (int64, may be NULL) accumulates
+ * [0] tokens emitted, [1] request-rounds, [2+j] drafts accepted at position j and
+ * [2+k+j] drafts decided at position j (j < k); it has 2 + 2k entries. */
+S3R_API int s3r_commit(const s3r_batch* batch, int32_t k, const int32_t* n_out, int32_t* seq_lens,
+               int64_t* stats, s3r_stream_t stream);
+
+/* Philox4x32-10 words and uniforms for n counters (position[i], request[i], stream_id, 0)
+ * under key = seed: words uint32 [n][4] (may be NULL), u fp32 [n] (may be NULL). */
+S3R_API int s3r_philox(uint64_t seed, int32_t stream_id, const int32_t* request, const int32_t* position,
+               int64_t n, uint32_t* words, float* u, s3r_stream_t stream);
+
+/* Synchronise `stream`, copy the workspace error word to *device_error (host pointer; a
+ * bitmask of (1 << S3R_ERR_*)) and clear it. Returns S3R_ERR_CUDA if the stream failed. */
+S3R_API int s3r_get_error(void* ws, int32_t* device_error, s3r_stream_t stream);
+
+/* Static text for a status code. */
+S3R_API const char* s3r_status_string(int status);
+
+/* Number of kernels this library has launched in the process (all calls, all streams). */
+S3R_API uint64_t s3r_launch_count(void);
+
+/* Text of the CUDA error behind the last S3R_ERR_CUDA status returned on this thread
+ * ("" if none). */
+S3R_API const char* s3r_last_error_message(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* S3R_H_ */

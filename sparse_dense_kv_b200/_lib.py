@@ -1,0 +1,262 @@
+"""ctypes binding of libs3r.so: argument marshalling only.
+
+Every function has the name of the C entry point it calls and takes torch tensors where
+the C function takes device pointers. Tensors must already live on the GPU with the dtype
+and layout the header states; the binding checks dtype/device/contiguity, passes
+`data_ptr()` and the current CUDA stream, and raises S3RError on any non-OK status. No
+step of the hot path runs in Python.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libs3r.so")
+
+S3R_OK = 0
+STATUS_NAMES = {
+    0: "S3R_OK", 1: "S3R_ERR_INVALID_ARG", 2: "S3R_ERR_UNSUPPORTED", 3: "S3R_ERR_CUDA",
+    4: "S3R_ERR_WORKSPACE", 5: "S3R_ERR_DEVICE_BOUNDS", 6: "S3R_ERR_NONFINITE",
+    7: "S3R_ERR_TIMEOUT",
+}
+PAGE_SIZE = 16
+MAX_K = 8
+
+
+class S3RError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)}")
+
+
+class KVCacheDesc(ctypes.Structure):
+    _fields_ = [("num_q_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("page_size", ctypes.c_int32),
+                ("num_pages", ctypes.c_int64), ("k_pool", ctypes.c_void_p),
+                ("v_pool", ctypes.c_void_p)]
+
+
+class BatchDesc(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("num_requests", ctypes.c_int32),
+                ("req_ids", ctypes.c_void_p), ("seq_lens", ctypes.c_void_p),
+                ("page_table", ctypes.c_void_p), ("max_pages_per_req", ctypes.c_int32)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libs3r.so is not built ({LIB_PATH}); run python sparse_dense_kv_b200/build.py")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I32, I64, U64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64, ctypes.c_size_t
+    C, B = ctypes.POINTER(KVCacheDesc), ctypes.POINTER(BatchDesc)
+    sig = {
+        "s3r_workspace_size": (SZ, [C, I32, I32, I32, I32, I32]),
+        "s3r_workspace_init": (ctypes.c_int, [P, SZ, P]),
+        "s3r_verify_attn": (ctypes.c_int, [C, B, I32, P, P, P, P, P, P, P, SZ, P]),
+        "s3r_select_kv": (ctypes.c_int, [C, B, P, P, I32, I32, I32, P, I32, P, P, SZ, P]),
+        "s3r_select_from_scores": (ctypes.c_int, [C, B, P, I32, I32, I32, P, I32, P, P, SZ, P]),
+        "s3r_sparse_draft_attn": (ctypes.c_int, [C, B, P, P, I32, P, P, I32, P, I32, P, P, P, P, SZ, P]),
+        "s3r_draft_sample": (ctypes.c_int, [B, P, I32, P, I32, U64, P, P, SZ, P]),
+        "s3r_spec_sample": (ctypes.c_int, [B, I32, P, P, P, I32, U64, P, P, P, SZ, P]),
+        "s3r_commit": (ctypes.c_int, [B, I32, P, P, P, P]),
+        "s3r_philox": (ctypes.c_int, [U64, I32, P, P, I64, P, P, P]),
+        "s3r_get_error": (ctypes.c_int, [P, P, P]),
+        "s3r_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "s3r_launch_count": (U64, []),
+        "s3r_last_error_message": (ctypes.c_char_p, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = _load()
+lib = _lib
+
+
+def _check(status: int, what: str):
+    if status != S3R_OK:
+        if status == 3:
+            what = f"{what} ({_lib.s3r_last_error_message().decode()})"
+        raise S3RError(status, what)
+
+
+def _stream(stream=None):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t, dtype=None, what="tensor", allow_none=False):
+    if t is None:
+        if allow_none:
+            return None
+        raise ValueError(f"{what} is required")
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{what} must be a torch.Tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{what} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{what} must be contiguous")
+    if t.device.type != "cuda":
+        raise ValueError(f"{what} must be a CUDA tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def make_cache(k_pool: torch.Tensor, v_pool: torch.Tensor, num_q_heads: int) -> KVCacheDesc:
+    """Descriptor of bf16 pools [num_pages][num_kv_heads][16][head_dim]."""
+    P, H, S, D = k_pool.shape
+    if v_pool.shape != k_pool.shape or S != PAGE_SIZE:
+        raise ValueError("pools must be [num_pages][num_kv_heads][16][head_dim] and equal")
+    desc = KVCacheDesc(num_q_heads, H, D, S, P, _ptr(k_pool, torch.bfloat16, "k_pool").value,
+                       _ptr(v_pool, torch.bfloat16, "v_pool").value)
+    desc._refs = (k_pool, v_pool)          # the descriptor keeps its tensors alive
+    return desc
+
+
+def make_batch(seq_lens: torch.Tensor, page_table: torch.Tensor | None = None,
+               req_ids: torch.Tensor | None = None, batch: int | None = None) -> BatchDesc:
+    """Batch descriptor; covers req_ids (or all requests) of int32 seq_lens / page_table."""
+    nr = seq_lens.numel()
+    if batch is None:
+        batch = req_ids.numel() if req_ids is not None else nr
+    pt = _ptr(page_table, torch.int32, "page_table", allow_none=True)
+    mp = page_table.shape[1] if page_table is not None else 0
+    rid = _ptr(req_ids, torch.int32, "req_ids", allow_none=True)
+    desc = BatchDesc(batch, nr, rid.value if rid is not None else None,
+                     _ptr(seq_lens, torch.int32, "seq_lens").value,
+                     pt.value if pt is not None else None, mp)
+    desc._refs = (seq_lens, page_table, req_ids)
+    return desc
+
+
+def s3r_workspace_size(cache: KVCacheDesc, num_requests: int, max_pages_per_req: int,
+                       max_k: int, vocab: int, sel_stride: int) -> int:
+    n = _lib.s3r_workspace_size(ctypes.byref(cache), num_requests, max_pages_per_req, max_k,
+                                vocab, sel_stride)
+    if n == 0:
+        raise S3RError(1, "s3r_workspace_size")
+    return int(n)
+
+
+def s3r_workspace_init(ws: torch.Tensor, stream=None):
+    _check(_lib.s3r_workspace_init(_ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)),
+           "s3r_workspace_init")
+
+
+def new_workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    """A zeroed workspace (uint8 CUDA tensor, 256-byte aligned by the caching allocator)."""
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    if ws.data_ptr() % 256:
+        raise RuntimeError("workspace allocation is not 256-byte aligned")
+    s3r_workspace_init(ws)
+    return ws
+
+
+def s3r_verify_attn(cache, batch, k, q, k_new, v_new, out, lse, score_logits, ws, stream=None):
+    bf, f32 = torch.bfloat16, torch.float32
+    _check(_lib.s3r_verify_attn(
+        ctypes.byref(cache), ctypes.byref(batch), k, _ptr(q, bf, "q"), _ptr(k_new, bf, "k_new"),
+        _ptr(v_new, bf, "v_new"), _ptr(out, bf, "out"), _ptr(lse, f32, "lse"),
+        _ptr(score_logits, f32, "score_logits", allow_none=True), _ptr(ws, torch.uint8, "ws"),
+        ws.numel(), _stream(stream)), "s3r_verify_attn")
+
+
+def s3r_select_kv(cache, batch, score_logits, lse, k_prev, budget_bp, window, sel_idx,
+                  sel_count, ws, stream=None):
+    f32, i32 = torch.float32, torch.int32
+    _check(_lib.s3r_select_kv(
+        ctypes.byref(cache), ctypes.byref(batch), _ptr(score_logits, f32, "score_logits"),
+        _ptr(lse, f32, "lse"), k_prev, budget_bp, window, _ptr(sel_idx, i32, "sel_idx"),
+        sel_idx.shape[-1], _ptr(sel_count, i32, "sel_count"), _ptr(ws, torch.uint8, "ws"),
+        ws.numel(), _stream(stream)), "s3r_select_kv")
+
+
+def s3r_select_from_scores(cache, batch, scores, budget_bp, window, sel_idx, sel_count, ws,
+                           stream=None):
+    f32, i32 = torch.float32, torch.int32
+    _check(_lib.s3r_select_from_scores(
+        ctypes.byref(cache), ctypes.byref(batch), _ptr(scores, f32, "scores"), scores.shape[-1],
+        budget_bp, window, _ptr(sel_idx, i32, "sel_idx"), sel_idx.shape[-1],
+        _ptr(sel_count, i32, "sel_count"), _ptr(ws, torch.uint8, "ws"), ws.numel(),
+        _stream(stream)), "s3r_select_from_scores")
+
+
+def _rows(t, inner, what):
+    """Pointer and request stride (elements) of a [num_requests][...] view whose per-request
+    part of `inner` elements is contiguous (e.g. block[:, i] of a [R][k+1][H][d] tensor)."""
+    if not isinstance(t, torch.Tensor) or t.device.type != "cuda" or t.dtype != torch.bfloat16:
+        raise TypeError(f"{what} must be a bf16 CUDA tensor")
+    if t[0].numel() != inner or not t[0].is_contiguous():
+        raise ValueError(f"{what}: each request's rows must be contiguous ({inner} elements)")
+    return ctypes.c_void_p(t.data_ptr()), int(t.stride(0)) if t.shape[0] > 1 else inner
+
+
+def s3r_sparse_draft_attn(cache, batch, draft_step, q, k_new, v_new, sel_idx, sel_count, out,
+                          lse, ws, stream=None):
+    """q [NR][H_q][d] and k_new / v_new [NR][H_kv][d], each possibly a strided view."""
+    bf, i32 = torch.bfloat16, torch.int32
+    qp, qs = _rows(q, cache.num_q_heads * cache.head_dim, "q")
+    kp, ks = _rows(k_new, cache.num_kv_heads * cache.head_dim, "k_new")
+    vp, vs = _rows(v_new, cache.num_kv_heads * cache.head_dim, "v_new")
+    if ks != vs:
+        raise ValueError("k_new and v_new must share a request stride")
+    _check(_lib.s3r_sparse_draft_attn(
+        ctypes.byref(cache), ctypes.byref(batch), _ptr(draft_step, i32, "draft_step"),
+        qp, qs, kp, vp, ks,
+        _ptr(sel_idx, i32, "sel_idx"), sel_idx.shape[-1], _ptr(sel_count, i32, "sel_count"),
+        _ptr(out, bf, "out"), _ptr(lse, torch.float32, "lse", allow_none=True),
+        _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)), "s3r_sparse_draft_attn")
+
+
+def s3r_draft_sample(batch, draft_step, k, q_logits, vocab, seed, draft_tokens, ws, stream=None):
+    _check(_lib.s3r_draft_sample(
+        ctypes.byref(batch), _ptr(draft_step, torch.int32, "draft_step"), k,
+        _ptr(q_logits, torch.float32, "q_logits"), vocab, seed,
+        _ptr(draft_tokens, torch.int32, "draft_tokens"), _ptr(ws, torch.uint8, "ws"), ws.numel(),
+        _stream(stream)), "s3r_draft_sample")
+
+
+def s3r_spec_sample(batch, k, p_logits, q_logits, draft_tokens, vocab, seed, out_tokens, n_out,
+                    ws, stream=None):
+    f32, i32 = torch.float32, torch.int32
+    _check(_lib.s3r_spec_sample(
+        ctypes.byref(batch), k, _ptr(p_logits, f32, "p_logits"),
+        _ptr(q_logits, f32, "q_logits", allow_none=(k == 0)),
+        _ptr(draft_tokens, i32, "draft_tokens", allow_none=(k == 0)), vocab, seed,
+        _ptr(out_tokens, i32, "out_tokens"), _ptr(n_out, i32, "n_out"),
+        _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)), "s3r_spec_sample")
+
+
+def s3r_commit(batch, k, n_out, seq_lens, stats=None, stream=None):
+    _check(_lib.s3r_commit(
+        ctypes.byref(batch), k, _ptr(n_out, torch.int32, "n_out"),
+        _ptr(seq_lens, torch.int32, "seq_lens"), _ptr(stats, torch.int64, "stats", allow_none=True),
+        _stream(stream)), "s3r_commit")
+
+
+def s3r_philox(seed, stream_id, request, position, words=None, u=None, stream=None):
+    _check(_lib.s3r_philox(
+        seed, stream_id, _ptr(request, torch.int32, "request"),
+        _ptr(position, torch.int32, "position"), request.numel(),
+        _ptr(words, torch.int32, "words", allow_none=True),
+        _ptr(u, torch.float32, "u", allow_none=True), _stream(stream)), "s3r_philox")
+
+
+def s3r_get_error(ws, stream=None) -> int:
+    v = ctypes.c_int32(0)
+    _check(_lib.s3r_get_error(_ptr(ws, torch.uint8, "ws"), ctypes.byref(v), _stream(stream)),
+           "s3r_get_error")
+    return int(v.value)
+
+
+def s3r_status_string(status: int) -> str:
+    return _lib.s3r_status_string(status).decode()
+
+
+def s3r_launch_count() -> int:
+    return int(_lib.s3r_launch_count())

@@ -1,0 +1,195 @@
+// Sparse self-draft attention.
+//
+// What it computes ([News] Interpretation; [Explainer] "How is this different": the draft
+// reads a sparse subset of the same KV cache with the same weights): draft step i of
+// request r (token at position L+i) writes that token's K/V into its page and lets the G
+// query rows of each KV head attend A_i = S ∪ {L, .., L+i}, S the selected positions.
+//
+// Layout of the work: grid (chunk of A_i, kv_head, request), 128 threads. The CTA first
+// resolves the element offsets of its <= 256 positions (index -> page -> slot), then
+// gathers 256-byte K and V rows with 16-byte cp.async (16 lanes per row, coalesced) into a
+// 3-stage pipeline laid out like the TMA tiles of the verify (128-byte swizzle), so the
+// same tensor-core step (one n-tile of 8 rows per warp) serves both. Chunks merge through
+// the workspace in the last CTA of the (request, head).
+#include "attention.cuh"
+#include "kernels.h"
+
+namespace s3r {
+
+constexpr int kDraftStages = 3;
+
+template <int D>
+__global__ void __launch_bounds__(128) draft_kernel(const DraftParams p) {
+  constexpr int NTW = 1, RW = 8, STAGE = 2 * kTile * D * 2, CPR = D / 8;
+  extern __shared__ uint8_t smem_dyn[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) &
+                                             ~uintptr_t(1023));
+  int64_t* rowoff = reinterpret_cast<int64_t*>(smem + kDraftStages * STAGE);
+  __shared__ int s_flag_mem;
+  int* s_flag = &s_flag_mem;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int bl = blockIdx.z, kvh = blockIdx.y, c = blockIdx.x;
+  const int r = p.req_ids ? p.req_ids[bl] : bl;
+  const int L = p.seq_lens[r];
+  const int i = p.draft_step[r];
+  const int Hkv = p.Hkv, G = p.G;
+  const int n = p.sel_count[(size_t)r * Hkv + kvh];
+  if (L < 0 || i < 0 || L + i >= p.cap || n < 0 || n > p.sel_stride) {
+    if (c == 0 && tid == 0) set_error(p.err, S3R_ERR_DEVICE_BOUNDS);
+    return;
+  }
+  const int A = n + i + 1;
+  const int start = c * kDraftChunk;
+  if (start >= A) return;
+  const int end = min(start + kDraftChunk, A);
+  const int nch = (A + kDraftChunk - 1) / kDraftChunk;
+  const int* ptab = p.page_table + (size_t)r * p.max_pages;
+  const int* sel = p.sel_idx + ((size_t)r * Hkv + kvh) * p.sel_stride;
+  const int64_t npages = p.num_pages;
+  const size_t new_off = (size_t)r * p.kv_stride + (size_t)kvh * D;   // this token in k_new / v_new
+
+  // This step's token enters the cache at position L+i (read below from k_new / v_new).
+  if (c == 0 && tid < CPR) {
+    const int pos = L + i;
+    const int page = ptab[pos >> 4];
+    if (page < 0 || page >= npages) {
+      set_error(p.err, S3R_ERR_DEVICE_BOUNDS);
+    } else {
+      const size_t dst = (((size_t)page * Hkv + kvh) * kPage + (pos & 15)) * D + tid * 8;
+      *reinterpret_cast<uint4*>(p.k_pool + dst) =
+          *reinterpret_cast<const uint4*>(p.k_new + new_off + tid * 8);
+      *reinterpret_cast<uint4*>(p.v_pool + dst) =
+          *reinterpret_cast<const uint4*>(p.v_new + new_off + tid * 8);
+    }
+  }
+
+  // Element offsets of the chunk's rows: >= 0 pool offset, -1 zeros, -2 this step's token.
+  for (int e = tid; e < kDraftChunk; e += blockDim.x) {
+    const int a = start + e;
+    int64_t off = -1;
+    if (a < end) {
+      int pos;
+      bool ok = true;
+      if (a < n) {
+        pos = sel[a];
+        ok = pos >= 0 && pos < L;
+      } else {
+        pos = L + (a - n);
+      }
+      if (!ok) {
+        set_error(p.err, S3R_ERR_DEVICE_BOUNDS);
+      } else if (pos == L + i) {
+        off = -2;
+      } else {
+        const int page = ptab[pos >> 4];
+        if (page < 0 || page >= npages) set_error(p.err, S3R_ERR_DEVICE_BOUNDS);
+        else off = (((int64_t)page * Hkv + kvh) * kPage + (pos & 15)) * D;
+      }
+    }
+    rowoff[e] = off;
+  }
+
+  WarpAttn<D, NTW> wa;
+  wa.init();
+  wa.load_q(0, lane, [&](int rr) -> const __nv_bfloat16* {
+    return rr < G ? p.q + (size_t)r * p.q_stride + (size_t)(kvh * G + rr) * D : nullptr;
+  });
+  __syncthreads();
+
+  const int ntiles = (end - start + kTile - 1) / kTile;
+  const uint32_t sbase = smem_u32(smem);
+  auto load_tile = [&](int it) {
+    const uint32_t kdst = sbase + (it % kDraftStages) * STAGE, vdst = kdst + kTile * D * 2;
+    for (int idx = tid; idx < kTile * CPR; idx += blockDim.x) {
+      const int row = idx / CPR, ch = idx - row * CPR;
+      const int64_t off = rowoff[it * kTile + row];
+      const __nv_bfloat16 *ks, *vs;
+      int bytes = 16;
+      if (off >= 0) {
+        ks = p.k_pool + off + ch * 8;
+        vs = p.v_pool + off + ch * 8;
+      } else if (off == -2) {
+        ks = p.k_new + new_off + ch * 8;
+        vs = p.v_new + new_off + ch * 8;
+      } else {
+        ks = p.k_new + new_off;   // any valid address; nothing is read
+        vs = p.v_new + new_off;
+        bytes = 0;
+      }
+      cp_async16(kdst + swz(row, ch), ks, bytes);
+      cp_async16(vdst + swz(row, ch), vs, bytes);
+    }
+  };
+
+#pragma unroll
+  for (int s = 0; s < kDraftStages - 1; ++s) {
+    if (s < ntiles) load_tile(s);
+    cp_async_commit();
+  }
+  for (int it = 0; it < ntiles; ++it) {
+    if (it + kDraftStages - 1 < ntiles) load_tile(it + kDraftStages - 1);
+    cp_async_commit();
+    cp_async_wait<kDraftStages - 1>();
+    __syncthreads();
+    const int t0 = start + it * kTile;
+    const uint32_t kb = sbase + (it % kDraftStages) * STAGE, vb = kb + kTile * D * 2;
+    const int row0 = warp * 16;
+    if (t0 + row0 < end) {
+      wa.step(
+          kb, vb, row0, lane, p.scale,
+          [&](int tr, int, int) -> bool { return t0 + tr < end; },
+          [](int, int, int, float) {});
+    }
+    __syncthreads();
+  }
+  cp_async_wait<0>();
+
+  wa.finish_sums();
+  float* redO = reinterpret_cast<float*>(smem);
+  float* redM = redO + 4 * RW * (D + 4);
+  float* redL = redM + 4 * RW;
+  wa.store_shared(redO, redM, redL, warp, lane);
+  __syncthreads();
+  const size_t rec_floats = (size_t)RW * (D + 2);
+  float* recs = p.part + ((size_t)r * Hkv + kvh) * p.nchunk_max * rec_floats;
+  merge_slices_to_record<D, RW>(redO, redM, redL, 1, recs + c * rec_floats, RW);
+
+  if (!last_of(p.tickets + (size_t)r * Hkv + kvh, nch, s_flag)) return;
+  combine_records<D>(
+      recs, rec_floats, nch, G, RW,
+      [&](int row) { return p.out + ((size_t)r * p.Hq + kvh * G + row) * D; },
+      [&](int row) -> float* {
+        return p.lse ? p.lse + (size_t)r * p.Hq + kvh * G + row : nullptr;
+      });
+}
+
+template <int D>
+static int launch_draft_d(const DraftParams& p, int batch, cudaStream_t stream) {
+  const size_t smem = 1024 + kDraftStages * 2 * kTile * D * 2 + kDraftChunk * 8 + 64;
+  static bool attr_done = false;
+  if (!attr_done) {
+    if (cuda_status(cudaFuncSetAttribute(draft_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem), "cudaFuncSetAttribute") != S3R_OK)
+
+      return S3R_ERR_CUDA;
+    attr_done = true;
+  }
+  dim3 grid(p.nchunk_max, p.Hkv, batch);
+  draft_kernel<D><<<grid, 128, smem, stream>>>(p);
+  return cuda_status(cudaGetLastError(), __func__);
+}
+
+int launch_draft(const DraftParams& p, int D, int batch, cudaStream_t stream) {
+  if (D == 128) return launch_draft_d<128>(p, batch, stream);
+  if (D == 64) return launch_draft_d<64>(p, batch, stream);
+  return S3R_ERR_UNSUPPORTED;
+}
+
+int draft_chunks(int sel_stride) { return (sel_stride + S3R_MAX_K + 1 + kDraftChunk - 1) / kDraftChunk; }
+
+size_t draft_partial_bytes(int num_requests, int Hkv, int sel_stride, int D) {
+  return align_up((size_t)num_requests * Hkv * draft_chunks(sel_stride) * 8 * (D + 2) * 4, 256);
+}
+
+}  // namespace s3r

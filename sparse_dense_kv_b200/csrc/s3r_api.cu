@@ -1,0 +1,470 @@
+// The extern "C" boundary of libs3r.so: host-side validation, workspace carving, TMA
+// descriptors and kernel launches. Nothing here allocates device memory.
+#include <atomic>
+#include <cstdio>
+#include <cstring>
+
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace s3r;
+
+thread_local char g_last_error[256] = "";
+
+namespace s3r {
+int cuda_status(cudaError_t e, const char* where) {
+  if (e == cudaSuccess) return S3R_OK;
+  std::snprintf(g_last_error, sizeof(g_last_error), "%s: %s", where, cudaGetErrorString(e));
+  return S3R_ERR_CUDA;
+}
+}  // namespace s3r
+
+namespace {
+
+std::atomic<uint64_t> g_launches{0};
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+int check_cache(const s3r_kv_cache* c) {
+  if (!c) return S3R_ERR_INVALID_ARG;
+  if (c->page_size != S3R_PAGE_SIZE) return S3R_ERR_UNSUPPORTED;
+  if (c->head_dim != 64 && c->head_dim != 128) return S3R_ERR_UNSUPPORTED;
+  if (c->num_kv_heads <= 0 || c->num_q_heads <= 0 || c->num_q_heads % c->num_kv_heads)
+    return S3R_ERR_INVALID_ARG;
+  if (c->num_q_heads / c->num_kv_heads > S3R_MAX_GROUP) return S3R_ERR_UNSUPPORTED;
+  if (c->num_kv_heads > kMaxKvHeads) return S3R_ERR_UNSUPPORTED;
+  if (c->num_pages <= 0 || !c->k_pool || !c->v_pool) return S3R_ERR_INVALID_ARG;
+  if (!aligned16(c->k_pool) || !aligned16(c->v_pool)) return S3R_ERR_INVALID_ARG;
+  if ((int64_t)c->num_pages * c->num_kv_heads * S3R_PAGE_SIZE >= ((int64_t)1 << 31))
+    return S3R_ERR_UNSUPPORTED;   // TMA row coordinate is a signed 32-bit integer
+  return S3R_OK;
+}
+
+// need_pages: the call reads the page table (attention, selection); those kernels put the
+// request in grid.y / grid.z, which limits a launch to 65535 requests.
+int check_batch(const s3r_batch* b, bool need_pages) {
+  if (!b) return S3R_ERR_INVALID_ARG;
+  if (b->batch < 0 || b->num_requests < 0) return S3R_ERR_INVALID_ARG;
+  if (b->batch == 0) return S3R_OK;
+  if (!b->req_ids && b->batch > b->num_requests) return S3R_ERR_INVALID_ARG;
+  if (!b->seq_lens || !aligned4(b->seq_lens)) return S3R_ERR_INVALID_ARG;
+  if (b->req_ids && !aligned4(b->req_ids)) return S3R_ERR_INVALID_ARG;
+  if (need_pages) {
+    if (b->batch > 65535) return S3R_ERR_UNSUPPORTED;
+    if (!b->page_table || !aligned4(b->page_table) || b->max_pages_per_req <= 0)
+      return S3R_ERR_INVALID_ARG;
+    if ((int64_t)b->max_pages_per_req * S3R_PAGE_SIZE >= ((int64_t)1 << 30))
+      return S3R_ERR_UNSUPPORTED;
+  }
+  return S3R_OK;
+}
+
+int check_ws(void* ws, size_t ws_bytes, size_t need) {
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return S3R_ERR_WORKSPACE;
+  if (ws_bytes < need) return S3R_ERR_WORKSPACE;
+  return S3R_OK;
+}
+
+struct Carve {
+  int* err;
+  int* tickets;
+  uint8_t* part;
+};
+
+Carve carve(void* ws, int num_requests) {
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  Carve c;
+  c.err = reinterpret_cast<int*>(b);
+  c.tickets = reinterpret_cast<int*>(b + kWsHeader);
+  c.part = b + kWsHeader + ws_tickets_bytes(num_requests);
+  return c;
+}
+
+size_t head_bytes(int num_requests) { return kWsHeader + ws_tickets_bytes(num_requests); }
+
+int nvch_of(int vocab) { return (vocab + kVocabChunk - 1) / kVocabChunk; }
+
+int finish(int st, int launches) {
+  if (st == S3R_OK) g_launches.fetch_add((uint64_t)launches, std::memory_order_relaxed);
+  return st;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2-D view of a pool: rows of head_dim bf16 (one per (page, head, slot)), boxes of 16 rows
+// x 64 columns with the 128-byte swizzle.
+int make_pool_map(CUtensorMap* map, void* pool, const s3r_kv_cache* c) {
+  auto fn = encode_fn();
+  if (!fn) {
+    std::snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled unavailable");
+    return S3R_ERR_CUDA;
+  }
+  cuuint64_t dims[2] = {(cuuint64_t)c->head_dim,
+                        (cuuint64_t)c->num_pages * c->num_kv_heads * S3R_PAGE_SIZE};
+  cuuint64_t strides[1] = {(cuuint64_t)c->head_dim * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)S3R_PAGE_SIZE};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pool, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    std::snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled: error %d", (int)r);
+    return S3R_ERR_CUDA;
+  }
+  return S3R_OK;
+}
+
+size_t verify_need(const s3r_kv_cache* c, int num_requests, int cap, int k) {
+  const int G = c->num_q_heads / c->num_kv_heads;
+  return head_bytes(num_requests) +
+         verify_partial_bytes(num_requests, c->num_kv_heads, cap, G * (k + 1), c->head_dim,
+                              kVerifyChunk);
+}
+
+size_t draft_need(const s3r_kv_cache* c, int num_requests, int sel_stride) {
+  return head_bytes(num_requests) +
+         draft_partial_bytes(num_requests, c->num_kv_heads, sel_stride, c->head_dim);
+}
+
+size_t sample_need(int num_requests, int hkv, int k, int vocab) {
+  return head_bytes(num_requests) + sample_partial_bytes(num_requests, k, vocab);
+}
+
+#define S3R_TRY(x)              \
+  do {                          \
+    const int _st = (x);        \
+    if (_st != S3R_OK) return _st; \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+size_t s3r_workspace_size(const s3r_kv_cache* cache, int32_t num_requests,
+                          int32_t max_pages_per_req, int32_t max_k, int32_t vocab,
+                          int32_t sel_stride) {
+  if (check_cache(cache) != S3R_OK || num_requests < 0 || max_pages_per_req <= 0 || max_k < 0 ||
+      max_k > S3R_MAX_K || vocab < 0 || sel_stride < 0)
+    return 0;
+  const int cap = max_pages_per_req * S3R_PAGE_SIZE;
+  size_t need = head_bytes(num_requests);
+  size_t a = verify_need(cache, num_requests, cap, max_k);
+  size_t b = draft_need(cache, num_requests, sel_stride);
+  size_t c = sample_need(num_requests, cache->num_kv_heads, max_k, vocab > 0 ? vocab : 1);
+  if (a > need) need = a;
+  if (b > need) need = b;
+  if (c > need) need = c;
+  return need;
+}
+
+int s3r_workspace_init(void* ws, size_t ws_bytes, s3r_stream_t stream) {
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < kWsHeader)
+    return S3R_ERR_WORKSPACE;
+  return cuda_status(cudaMemsetAsync(ws, 0, ws_bytes, (cudaStream_t)stream), "cudaMemsetAsync");
+}
+
+int s3r_verify_attn(const s3r_kv_cache* cache, const s3r_batch* batch, int32_t k,
+                    const void* q, const void* k_new, const void* v_new, void* out, float* lse,
+                    float* score_logits, void* ws, size_t ws_bytes, s3r_stream_t stream) {
+  S3R_TRY(check_cache(cache));
+  S3R_TRY(check_batch(batch, true));
+  if (k < 0 || k > S3R_MAX_K) return S3R_ERR_UNSUPPORTED;
+  const int G = cache->num_q_heads / cache->num_kv_heads;
+  const int R = G * (k + 1);
+  if (R > S3R_MAX_ROWS) return S3R_ERR_UNSUPPORTED;
+  if (!q || !k_new || !v_new || !out || !lse) return S3R_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(out) ||
+      !aligned4(lse) || (score_logits && !aligned4(score_logits)))
+    return S3R_ERR_INVALID_ARG;
+  if (batch->batch == 0) return S3R_OK;
+  const int cap = batch->max_pages_per_req * S3R_PAGE_SIZE;
+  S3R_TRY(check_ws(ws, ws_bytes, verify_need(cache, batch->num_requests, cap, k)));
+  CUtensorMap tk, tv;
+  S3R_TRY(make_pool_map(&tk, cache->k_pool, cache));
+  S3R_TRY(make_pool_map(&tv, cache->v_pool, cache));
+  const Carve w = carve(ws, batch->num_requests);
+  VerifyParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.req_ids = batch->req_ids;
+  p.seq_lens = batch->seq_lens;
+  p.page_table = batch->page_table;
+  p.max_pages = batch->max_pages_per_req;
+  p.cap = cap;
+  p.Hq = cache->num_q_heads;
+  p.Hkv = cache->num_kv_heads;
+  p.G = G;
+  p.T = k + 1;
+  p.R = R;
+  p.Rp = ((R + 15) / 16) * 16;
+  p.num_pages = cache->num_pages;
+  p.k_pool = static_cast<__nv_bfloat16*>(cache->k_pool);
+  p.v_pool = static_cast<__nv_bfloat16*>(cache->v_pool);
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k_new = static_cast<const __nv_bfloat16*>(k_new);
+  p.v_new = static_cast<const __nv_bfloat16*>(v_new);
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.scores = score_logits;
+  p.scale = 1.0f / sqrtf((float)cache->head_dim);
+  p.chunk = kVerifyChunk;
+  p.nchunk_max = (cap + kVerifyChunk - 1) / kVerifyChunk;
+  p.err = w.err;
+  p.tickets = w.tickets;
+  p.part = reinterpret_cast<float*>(w.part);
+  return finish(launch_verify(tk, tv, p, cache->head_dim, batch->batch, (cudaStream_t)stream), 1);
+}
+
+static int select_common(const s3r_kv_cache* cache, const s3r_batch* batch, SelectParams& p,
+                         int32_t budget_bp, int32_t window, int32_t* sel_idx, int32_t sel_stride,
+                         int32_t* sel_count, void* ws, size_t ws_bytes, s3r_stream_t stream) {
+  if (budget_bp < 1 || budget_bp > 10000 || window < 1) return S3R_ERR_INVALID_ARG;
+  if (!sel_idx || !sel_count || sel_stride < 1 || !aligned4(sel_idx) || !aligned4(sel_count))
+    return S3R_ERR_INVALID_ARG;
+  if (batch->batch > 65535) return S3R_ERR_UNSUPPORTED;   // grid.y
+  if (batch->batch == 0) return S3R_OK;
+  S3R_TRY(check_ws(ws, ws_bytes, head_bytes(batch->num_requests)));
+  const Carve w = carve(ws, batch->num_requests);
+  p.req_ids = batch->req_ids;
+  p.seq_lens = batch->seq_lens;
+  p.Hq = cache->num_q_heads;
+  p.Hkv = cache->num_kv_heads;
+  p.G = cache->num_q_heads / cache->num_kv_heads;
+  p.budget_bp = budget_bp;
+  p.window = window;
+  p.sel_idx = sel_idx;
+  p.sel_stride = sel_stride;
+  p.sel_count = sel_count;
+  p.err = w.err;
+  return finish(launch_select(p, batch->batch, (cudaStream_t)stream), 1);
+}
+
+int s3r_select_kv(const s3r_kv_cache* cache, const s3r_batch* batch, const float* score_logits,
+                  const float* lse, int32_t k_prev, int32_t budget_bp, int32_t window,
+                  int32_t* sel_idx, int32_t sel_stride, int32_t* sel_count, void* ws,
+                  size_t ws_bytes, s3r_stream_t stream) {
+  S3R_TRY(check_cache(cache));
+  S3R_TRY(check_batch(batch, true));
+  if (k_prev < 0 || k_prev > S3R_MAX_K) return S3R_ERR_UNSUPPORTED;
+  if (window < k_prev + 1) return S3R_ERR_INVALID_ARG;
+  if (!score_logits || !lse || !aligned4(score_logits) || !aligned4(lse))
+    return S3R_ERR_INVALID_ARG;
+  const int G = cache->num_q_heads / cache->num_kv_heads;
+  if (G * (k_prev + 1) > S3R_MAX_ROWS) return S3R_ERR_UNSUPPORTED;
+  SelectParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.cap = batch->max_pages_per_req * S3R_PAGE_SIZE;
+  p.logits = score_logits;
+  p.lse = lse;
+  p.T = k_prev + 1;
+  p.R = G * (k_prev + 1);
+  return select_common(cache, batch, p, budget_bp, window, sel_idx, sel_stride, sel_count, ws,
+                       ws_bytes, stream);
+}
+
+int s3r_select_from_scores(const s3r_kv_cache* cache, const s3r_batch* batch,
+                           const float* scores, int32_t score_stride, int32_t budget_bp,
+                           int32_t window, int32_t* sel_idx, int32_t sel_stride,
+                           int32_t* sel_count, void* ws, size_t ws_bytes, s3r_stream_t stream) {
+  S3R_TRY(check_cache(cache));
+  S3R_TRY(check_batch(batch, false));
+  if (!scores || !aligned4(scores) || score_stride < 1) return S3R_ERR_INVALID_ARG;
+  SelectParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.scores = scores;
+  p.score_stride = score_stride;
+  return select_common(cache, batch, p, budget_bp, window, sel_idx, sel_stride, sel_count, ws,
+                       ws_bytes, stream);
+}
+
+int s3r_sparse_draft_attn(const s3r_kv_cache* cache, const s3r_batch* batch,
+                          const int32_t* draft_step, const void* q, int32_t q_stride,
+                          const void* k_new, const void* v_new, int32_t kv_stride,
+                          const int32_t* sel_idx, int32_t sel_stride,
+                          const int32_t* sel_count, void* out, float* lse, void* ws,
+                          size_t ws_bytes, s3r_stream_t stream) {
+  S3R_TRY(check_cache(cache));
+  S3R_TRY(check_batch(batch, true));
+  if (!draft_step || !q || !k_new || !v_new || !sel_idx || !sel_count || !out)
+    return S3R_ERR_INVALID_ARG;
+  if (!aligned4(draft_step) || !aligned16(q) || !aligned16(k_new) || !aligned16(v_new) ||
+      !aligned4(sel_idx) || !aligned4(sel_count) || !aligned16(out) || (lse && !aligned4(lse)))
+    return S3R_ERR_INVALID_ARG;
+  if (sel_stride < 1) return S3R_ERR_INVALID_ARG;
+  const int64_t qrow = (int64_t)cache->num_q_heads * cache->head_dim;
+  const int64_t kvrow = (int64_t)cache->num_kv_heads * cache->head_dim;
+  if (q_stride == 0) q_stride = (int32_t)qrow;
+  if (kv_stride == 0) kv_stride = (int32_t)kvrow;
+  if (q_stride < qrow || kv_stride < kvrow || (q_stride % 8) || (kv_stride % 8))
+    return S3R_ERR_INVALID_ARG;
+  if (batch->batch == 0) return S3R_OK;
+  S3R_TRY(check_ws(ws, ws_bytes, draft_need(cache, batch->num_requests, sel_stride)));
+  const Carve w = carve(ws, batch->num_requests);
+  DraftParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.req_ids = batch->req_ids;
+  p.seq_lens = batch->seq_lens;
+  p.page_table = batch->page_table;
+  p.max_pages = batch->max_pages_per_req;
+  p.cap = batch->max_pages_per_req * S3R_PAGE_SIZE;
+  p.Hq = cache->num_q_heads;
+  p.Hkv = cache->num_kv_heads;
+  p.G = cache->num_q_heads / cache->num_kv_heads;
+  p.num_pages = cache->num_pages;
+  p.k_pool = static_cast<__nv_bfloat16*>(cache->k_pool);
+  p.v_pool = static_cast<__nv_bfloat16*>(cache->v_pool);
+  p.draft_step = draft_step;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k_new = static_cast<const __nv_bfloat16*>(k_new);
+  p.v_new = static_cast<const __nv_bfloat16*>(v_new);
+  p.q_stride = q_stride;
+  p.kv_stride = kv_stride;
+  p.sel_idx = sel_idx;
+  p.sel_stride = sel_stride;
+  p.sel_count = sel_count;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.scale = 1.0f / sqrtf((float)cache->head_dim);
+  p.nchunk_max = (sel_stride + S3R_MAX_K + 1 + kDraftChunk - 1) / kDraftChunk;
+  p.err = w.err;
+  p.tickets = w.tickets;
+  p.part = reinterpret_cast<float*>(w.part);
+  return finish(launch_draft(p, cache->head_dim, batch->batch, (cudaStream_t)stream), 1);
+}
+
+int s3r_draft_sample(const s3r_batch* batch, const int32_t* draft_step, int32_t k,
+                     const float* q_logits, int32_t vocab, uint64_t seed, int32_t* draft_tokens,
+                     void* ws, size_t ws_bytes, s3r_stream_t stream) {
+  S3R_TRY(check_batch(batch, false));
+  if (k < 1 || k > S3R_MAX_K) return S3R_ERR_UNSUPPORTED;
+  if (vocab < 1 || vocab > 64 * kVocabChunk) return S3R_ERR_UNSUPPORTED;
+  if (!draft_step || !q_logits || !draft_tokens || !aligned4(draft_step) ||
+      !aligned4(q_logits) || !aligned4(draft_tokens))
+    return S3R_ERR_INVALID_ARG;
+  if (batch->batch == 0) return S3R_OK;
+  S3R_TRY(check_ws(ws, ws_bytes, sample_need(batch->num_requests, 1, k, vocab)));
+  const Carve w = carve(ws, batch->num_requests);
+  SampleParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.req_ids = batch->req_ids;
+  p.seq_lens = batch->seq_lens;
+  p.draft_step = draft_step;
+  p.k = k;
+  p.vocab = vocab;
+  p.nvch = nvch_of(vocab);
+  p.q_logits = q_logits;
+  p.draft_out = draft_tokens;
+  p.seed = seed;
+  p.err = w.err;
+  p.tickets = w.tickets;
+  p.part = w.part;
+  return finish(launch_draft_sample(p, batch->batch, (cudaStream_t)stream), 1);
+}
+
+int s3r_spec_sample(const s3r_batch* batch, int32_t k, const float* p_logits,
+                    const float* q_logits, const int32_t* draft_tokens, int32_t vocab,
+                    uint64_t seed, int32_t* out_tokens, int32_t* n_out, void* ws,
+                    size_t ws_bytes, s3r_stream_t stream) {
+  S3R_TRY(check_batch(batch, false));
+  if (k < 0 || k > S3R_MAX_K) return S3R_ERR_UNSUPPORTED;
+  if (vocab < 1 || vocab > 64 * kVocabChunk) return S3R_ERR_UNSUPPORTED;
+  if (!p_logits || !out_tokens || !n_out || !aligned4(p_logits) || !aligned4(out_tokens) ||
+      !aligned4(n_out))
+    return S3R_ERR_INVALID_ARG;
+  if (k > 0 && (!q_logits || !draft_tokens || !aligned4(q_logits) || !aligned4(draft_tokens)))
+    return S3R_ERR_INVALID_ARG;
+  if (batch->batch == 0) return S3R_OK;
+  S3R_TRY(check_ws(ws, ws_bytes, sample_need(batch->num_requests, 1, k, vocab)));
+  const Carve w = carve(ws, batch->num_requests);
+  SampleParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.req_ids = batch->req_ids;
+  p.seq_lens = batch->seq_lens;
+  p.k = k;
+  p.vocab = vocab;
+  p.nvch = nvch_of(vocab);
+  p.p_logits = p_logits;
+  p.q_logits = q_logits;
+  p.draft_tokens = draft_tokens;
+  p.out_tokens = out_tokens;
+  p.n_out = n_out;
+  p.seed = seed;
+  p.err = w.err;
+  p.tickets = w.tickets;
+  p.part = w.part;
+  spec_offsets(batch->num_requests, k, vocab, &p.plan_off, &p.draw_off);
+  int launches = 0;
+  const int st = launch_spec_sample(p, batch->batch, (cudaStream_t)stream, &launches);
+  if (st != S3R_OK && launches == 0) return st;
+  g_launches.fetch_add((uint64_t)(st == S3R_OK ? launches : 1), std::memory_order_relaxed);
+  return st;
+}
+
+int s3r_commit(const s3r_batch* batch, int32_t k, const int32_t* n_out, int32_t* seq_lens,
+               int64_t* stats, s3r_stream_t stream) {
+  S3R_TRY(check_batch(batch, false));
+  if (k < 0 || k > S3R_MAX_K) return S3R_ERR_UNSUPPORTED;
+  if (!n_out || !seq_lens || !aligned4(n_out) || !aligned4(seq_lens)) return S3R_ERR_INVALID_ARG;
+  if (stats && (reinterpret_cast<uintptr_t>(stats) & 7u)) return S3R_ERR_INVALID_ARG;
+  if (batch->batch == 0) return S3R_OK;
+  return finish(launch_commit(batch->req_ids, batch->batch, k, n_out, seq_lens, stats,
+                              (cudaStream_t)stream),
+                1);
+}
+
+int s3r_philox(uint64_t seed, int32_t stream_id, const int32_t* request, const int32_t* position,
+               int64_t n, uint32_t* words, float* u, s3r_stream_t stream) {
+  if (n < 0 || (n > 0 && (!request || !position))) return S3R_ERR_INVALID_ARG;
+  if (n == 0) return S3R_OK;
+  if (n > ((int64_t)1 << 31) * 255) return S3R_ERR_UNSUPPORTED;
+  return finish(launch_philox(seed, stream_id, request, position, n, words, u,
+                              (cudaStream_t)stream),
+                1);
+}
+
+int s3r_get_error(void* ws, int32_t* device_error, s3r_stream_t stream) {
+  if (!ws || !device_error) return S3R_ERR_INVALID_ARG;
+  int32_t v = 0;
+  const cudaStream_t st = (cudaStream_t)stream;
+  S3R_TRY(cuda_status(cudaMemcpyAsync(&v, ws, sizeof(v), cudaMemcpyDeviceToHost, st), "cudaMemcpyAsync"));
+  S3R_TRY(cuda_status(cudaStreamSynchronize(st), "cudaStreamSynchronize"));
+  *device_error = v;
+  if (v) S3R_TRY(cuda_status(cudaMemsetAsync(ws, 0, sizeof(v), st), "cudaMemsetAsync"));
+  S3R_TRY(cuda_status(cudaStreamSynchronize(st), "cudaStreamSynchronize"));
+  return S3R_OK;
+}
+
+const char* s3r_status_string(int status) {
+  switch (status) {
+    case S3R_OK: return "ok";
+    case S3R_ERR_INVALID_ARG: return "invalid argument";
+    case S3R_ERR_UNSUPPORTED: return "unsupported shape or parameter";
+    case S3R_ERR_CUDA: return "CUDA runtime error";
+    case S3R_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case S3R_ERR_DEVICE_BOUNDS: return "device: index, page id or length out of range";
+    case S3R_ERR_NONFINITE: return "device: non-finite logit or score";
+    case S3R_ERR_TIMEOUT: return "device: bounded wait expired";
+    default: return "unknown status";
+  }
+}
+
+uint64_t s3r_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char* s3r_last_error_message(void) { return g_last_error; }
+
+}  // extern "C"

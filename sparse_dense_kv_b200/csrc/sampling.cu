@@ -1,0 +1,456 @@
+// Draft-token sampling, exact speculative sampling, round commit and Philox uniforms.
+//
+// What they compute ([News] Interpretation and [Explainer] Jargon, exact speculative
+// sampling: accept a draft or draw from the residual distribution so that emitted tokens
+// follow the dense policy): softmax normalisers of the draft / target rows, the accept
+// tests u * q(d) < p(d), and inverse-CDF draws from q, from max(0, p - q) or from p.
+//
+// The vocabulary is split into chunks of 8192 entries. A pass over (chunk, row, request)
+// produces (max, sum exp(x - max)) per chunk with fp32 exponentials and fp64 sums; the last
+// CTA of a request merges the chunks (ticket, no spinning) and decides. A draw first finds
+// the chunk holding u * Z from the chunk sums, then splits that chunk into 256 segments of
+// 32 entries, one per thread, scans the segment sums and lets the owning thread walk its
+// 32 entries.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace s3r {
+
+constexpr int kSampThreads = 256;
+constexpr int kSeg = kVocabChunk / kSampThreads;   // 32 entries per thread in a draw
+
+struct MS {
+  float m;
+  float pad;
+  double s;
+};
+
+struct SpecPlan {
+  int type;      // 0: residual of row j, 1: target row j
+  int row;
+  int a;         // accepted drafts
+  int pad;
+  float mp, mq;
+  double zp, zq, u;
+};
+
+// Block reduction of (max, sum) pairs; result valid in thread 0.
+__device__ MS block_ms(float m, double s) {
+  __shared__ float sm[kSampThreads / 32];
+  __shared__ double ss[kSampThreads / 32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    const float m2 = __shfl_xor_sync(kFull, m, o);
+    const double s2 = __shfl_xor_sync(kFull, s, o);
+    merge_ms(m, s, m2, s2);
+  }
+  if (lane == 0) {
+    sm[warp] = m;
+    ss[warp] = s;
+  }
+  __syncthreads();
+  MS r{-INFINITY, 0.f, 0.0};
+  if (threadIdx.x == 0)
+    for (int w = 0; w < kSampThreads / 32; ++w) merge_ms(r.m, r.s, sm[w], ss[w]);
+  return r;
+}
+
+// (max, sum exp(x - max)) of row[v0 .. v1) by this thread (strided), fp64 sum.
+__device__ __forceinline__ void chunk_ms(const float* row, int v0, int v1, float& m, double& s,
+                                         bool& bad) {
+  m = -INFINITY;
+  s = 0.0;
+  for (int v = v0 + threadIdx.x; v < v1; v += blockDim.x) {
+    const float x = __ldg(row + v);
+    if (!isfinite(x)) {
+      bad = true;
+      continue;
+    }
+    if (x > m) {
+      s = s * (double)expf(m - x) + 1.0;
+      m = x;
+    } else {
+      s += (double)expf(x - m);
+    }
+  }
+}
+
+__device__ double block_sum_d(double v) {
+  __shared__ double sd[kSampThreads / 32];
+  __shared__ double tot;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  v = warp_sum_d(v);
+  if (lane == 0) sd[warp] = v;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int w = 0; w < kSampThreads / 32; ++w) t += sd[w];
+    tot = t;
+  }
+  __syncthreads();
+  const double r = tot;
+  __syncthreads();
+  return r;
+}
+
+// Exclusive block scan of doubles (fixed order: warp shuffles, then warps in order).
+__device__ double block_excl_scan_d(double v, double& total) {
+  __shared__ double sd[kSampThreads / 32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  double incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const double t = __shfl_up_sync(kFull, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) sd[warp] = incl;
+  __syncthreads();
+  double before = 0.0, tot = 0.0;
+  for (int w = 0; w < kSampThreads / 32; ++w) {
+    before += (w < warp) ? sd[w] : 0.0;
+    tot += sd[w];
+  }
+  __syncthreads();
+  total = tot;
+  return before + incl - v;
+}
+
+// Inverse-CDF search inside [v0, v1): smallest v with target < base + C_v, C the inclusive
+// running sum of weight(v). The chunk is cut into one 32-entry segment per thread; segment
+// bounds come from one block scan and are shared through shared memory, so the segments
+// partition [base, base + total) exactly and at most one thread owns the target.
+// Returns -1 if the target lies past the chunk; `base` then moves to the chunk's end.
+template <class W>
+__device__ int chunk_search(int v0, int v1, double target, double& base, W weight) {
+  __shared__ double hi_s[kSampThreads];
+  __shared__ int s_tok;
+  const int t = threadIdx.x;
+  const int a = v0 + t * kSeg;
+  const int b = min(a + kSeg, v1);
+  double seg = 0.0;
+  for (int v = a; v < b; ++v) seg += weight(v);
+  double total;
+  const double excl = block_excl_scan_d(seg, total);
+  hi_s[t] = base + (excl + seg);
+  if (t == 0) s_tok = -1;
+  __syncthreads();
+  const double lo = t ? hi_s[t - 1] : base;
+  const double hi = hi_s[t];
+  if (seg > 0.0 && target >= lo && target < hi) {
+    double c = lo;
+    int tok = -1, last_nz = -1;
+    for (int v = a; v < b; ++v) {
+      const double wv = weight(v);
+      if (wv > 0.0) last_nz = v;
+      c += wv;
+      if (target < c) {
+        tok = v;
+        break;
+      }
+    }
+    atomicMax(&s_tok, tok < 0 ? last_nz : tok);
+  }
+  __syncthreads();
+  const int tok = s_tok;
+  base = hi_s[kSampThreads - 1];
+  __syncthreads();
+  return tok;
+}
+
+// Last entry with non-zero weight in [0, V) (rounding fallback of a draw).
+template <class W>
+__device__ int last_nonzero(int V, W weight) {
+  __shared__ int s_last;
+  if (threadIdx.x == 0) s_last = -1;
+  __syncthreads();
+  for (int v = threadIdx.x; v < V; v += blockDim.x)
+    if (weight(v) > 0.0) atomicMax(&s_last, v);
+  __syncthreads();
+  const int r = s_last;
+  __syncthreads();
+  return r < 0 ? V - 1 : r;
+}
+
+// Draw with target u * Z over weights whose chunk sums are csum[0..nvch).
+template <class W>
+__device__ int draw_token(int V, int nvch, const double* csum, double target, W weight) {
+  __shared__ int s_c;
+  __shared__ double s_base;
+  if (threadIdx.x == 0) {
+    double cum = 0.0;
+    int c = nvch;
+    for (int i = 0; i < nvch; ++i) {
+      if (target < cum + csum[i]) {
+        c = i;
+        break;
+      }
+      cum += csum[i];
+    }
+    s_c = c;
+    s_base = cum;
+  }
+  __syncthreads();
+  int c = s_c;
+  double base = s_base;
+  __syncthreads();
+  for (; c < nvch; ++c) {
+    const int tok = chunk_search(c * kVocabChunk, min(V, (c + 1) * kVocabChunk), target, base, weight);
+    if (tok >= 0) return tok;
+  }
+  return last_nonzero(V, weight);
+}
+
+// ------------------------------------------------------------------ draft sampling ----
+__global__ void __launch_bounds__(kSampThreads) draft_sample_kernel(const SampleParams p) {
+  __shared__ int s_flag;
+  __shared__ double csum[64];
+  __shared__ float s_M;
+  const int c = blockIdx.y, bl = blockIdx.x;
+  const int r = p.req_ids ? p.req_ids[bl] : bl;
+  const int i = p.draft_step[r];
+  const int V = p.vocab;
+  if (i < 0 || i >= p.k) {
+    if (c == 0 && threadIdx.x == 0) set_error(p.err, S3R_ERR_DEVICE_BOUNDS);
+    return;
+  }
+  const float* row = p.q_logits + ((size_t)r * p.k + i) * V;
+  MS* part = reinterpret_cast<MS*>(p.part) + (size_t)r * p.nvch;
+
+  float m;
+  double s;
+  bool bad = false;
+  chunk_ms(row, c * kVocabChunk, min(V, (c + 1) * kVocabChunk), m, s, bad);
+  if (bad) set_error(p.err, S3R_ERR_NONFINITE);
+  const MS tot = block_ms(m, s);
+  if (threadIdx.x == 0) part[c] = tot;
+  if (!last_of(p.tickets + r, p.nvch, &s_flag)) return;
+
+  if (threadIdx.x == 0) {
+    float M = -INFINITY;
+    for (int q = 0; q < p.nvch; ++q) M = fmaxf(M, __ldcg(&part[q].m));
+    for (int q = 0; q < p.nvch; ++q) {
+      const float mq = __ldcg(&part[q].m);
+      csum[q] = (mq == -INFINITY) ? 0.0 : __ldcg(&part[q].s) * exp((double)mq - (double)M);
+    }
+    s_M = M;
+  }
+  __syncthreads();
+  const float M = s_M;
+  double Z = 0.0;
+  for (int q = 0; q < p.nvch; ++q) Z += csum[q];
+  const int L = p.seq_lens[r];
+  const double u = philox_u(p.seed, (uint32_t)(L + i + 1), (uint32_t)r, 0u);
+  const int tok = draw_token(V, p.nvch, csum, u * Z, [&](int v) -> double {
+    const float x = row[v];
+    return isfinite(x) ? (double)expf(x - M) : 0.0;
+  });
+  if (threadIdx.x == 0) p.draft_out[(size_t)r * p.k + i] = tok;
+}
+
+// ------------------------------------------------------- speculative sampling: pass 1 --
+__global__ void __launch_bounds__(kSampThreads) spec_norm_kernel(const SampleParams p) {
+  __shared__ int s_flag;
+  __shared__ float sM[2 * S3R_MAX_K + 1];
+  __shared__ double sZ[2 * S3R_MAX_K + 1];
+  const int bl = blockIdx.x, rw = blockIdx.y, c = blockIdx.z;
+  const int r = p.req_ids ? p.req_ids[bl] : bl;
+  const int k = p.k, V = p.vocab, nrows = 2 * k + 1;
+  const float* row = (rw <= k) ? p.p_logits + ((size_t)r * (k + 1) + rw) * V
+                               : p.q_logits + ((size_t)r * k + (rw - k - 1)) * V;
+  MS* part = reinterpret_cast<MS*>(p.part) + (size_t)r * nrows * p.nvch;
+
+  float m;
+  double s;
+  bool bad = false;
+  chunk_ms(row, c * kVocabChunk, min(V, (c + 1) * kVocabChunk), m, s, bad);
+  if (bad) set_error(p.err, S3R_ERR_NONFINITE);
+  const MS tot = block_ms(m, s);
+  if (threadIdx.x == 0) part[rw * p.nvch + c] = tot;
+  if (!last_of(p.tickets + r, nrows * p.nvch, &s_flag)) return;
+
+  // normalisers of every row
+  if (threadIdx.x < nrows) {
+    const MS* pr = part + threadIdx.x * p.nvch;
+    float M = -INFINITY;
+    for (int q = 0; q < p.nvch; ++q) M = fmaxf(M, __ldcg(&pr[q].m));
+    double Z = 0.0;
+    for (int q = 0; q < p.nvch; ++q) {
+      const float mq = __ldcg(&pr[q].m);
+      if (mq != -INFINITY) Z += __ldcg(&pr[q].s) * exp((double)mq - (double)M);
+    }
+    sM[threadIdx.x] = M;
+    sZ[threadIdx.x] = Z;
+  }
+  __syncthreads();
+  if (threadIdx.x != 0) return;
+
+  const int L = p.seq_lens[r];
+  const size_t pbase = (size_t)r * (k + 1) * V, qbase = (size_t)r * k * V;
+  int a = 0, type = 1, jrow = k;
+  for (int j = 0; j < k; ++j) {
+    const int d = p.draft_tokens[(size_t)r * k + j];
+    bool accept = false;
+    if (d < 0 || d >= V) {
+      set_error(p.err, S3R_ERR_DEVICE_BOUNDS);
+    } else {
+      const double pj = exp((double)p.p_logits[pbase + (size_t)j * V + d] - (double)sM[j]) / sZ[j];
+      const double qj =
+          exp((double)p.q_logits[qbase + (size_t)j * V + d] - (double)sM[k + 1 + j]) / sZ[k + 1 + j];
+      const double u = philox_u(p.seed, (uint32_t)(L + j + 1), (uint32_t)r, 1u);
+      accept = u * qj < pj;
+    }
+    if (!accept) {
+      type = 0;
+      jrow = j;
+      break;
+    }
+    p.out_tokens[(size_t)r * (k + 1) + j] = d;
+    ++a;
+  }
+  SpecPlan* plan = reinterpret_cast<SpecPlan*>(p.part + p.plan_off) + r;
+  SpecPlan pl;
+  pl.type = type;
+  pl.row = jrow;
+  pl.a = a;
+  pl.pad = 0;
+  pl.mp = sM[jrow];
+  pl.zp = sZ[jrow];
+  pl.mq = (type == 0) ? sM[k + 1 + jrow] : 0.f;
+  pl.zq = (type == 0) ? sZ[k + 1 + jrow] : 1.0;
+  pl.u = philox_u(p.seed, (uint32_t)(L + jrow + 1), (uint32_t)r, 2u);
+  *plan = pl;
+  p.n_out[r] = a + 1;
+}
+
+// ------------------------------------------------------- speculative sampling: pass 2 --
+__global__ void __launch_bounds__(kSampThreads) spec_draw_kernel(const SampleParams p) {
+  __shared__ int s_flag;
+  __shared__ double csum[64];
+  __shared__ int s_use_res;
+  const int c = blockIdx.y, bl = blockIdx.x;
+  const int r = p.req_ids ? p.req_ids[bl] : bl;
+  const int k = p.k, V = p.vocab;
+  const SpecPlan pl = reinterpret_cast<const SpecPlan*>(p.part + p.plan_off)[r];
+  const float* prow = p.p_logits + ((size_t)r * (k + 1) + pl.row) * V;
+  const float* qrow = p.q_logits + ((size_t)r * k + (pl.type == 0 ? pl.row : 0)) * V;
+  double2* part = reinterpret_cast<double2*>(p.part + p.draw_off) + (size_t)r * p.nvch;
+  const bool resid = pl.type == 0;
+  auto w_p = [&](int v) -> double {
+    const float x = prow[v];
+    return isfinite(x) ? (double)expf(x - pl.mp) : 0.0;
+  };
+  auto w_res = [&](int v) -> double {
+    const float x = prow[v], y = qrow[v];
+    const double pv = isfinite(x) ? (double)expf(x - pl.mp) / pl.zp : 0.0;
+    const double qv = isfinite(y) ? (double)expf(y - pl.mq) / pl.zq : 0.0;
+    return pv > qv ? pv - qv : 0.0;
+  };
+
+  const int v0 = c * kVocabChunk, v1 = min(V, (c + 1) * kVocabChunk);
+  double sr = 0.0, sp = 0.0;
+  for (int v = v0 + threadIdx.x; v < v1; v += blockDim.x) {
+    sp += w_p(v);
+    if (resid) sr += w_res(v);
+  }
+  sp = block_sum_d(sp);
+  sr = block_sum_d(sr);
+  if (threadIdx.x == 0) part[c] = make_double2(sr, sp);
+  if (!last_of(p.tickets + r, p.nvch, &s_flag)) return;
+
+  if (threadIdx.x == 0) {
+    double zr = 0.0;
+    for (int q = 0; q < p.nvch; ++q) zr += __ldcg(&part[q].x);
+    const int use_res = resid && zr > 0.0;
+    for (int q = 0; q < p.nvch; ++q) csum[q] = use_res ? __ldcg(&part[q].x) : __ldcg(&part[q].y);
+    s_use_res = use_res;
+  }
+  __syncthreads();
+  double Z = 0.0;
+  for (int q = 0; q < p.nvch; ++q) Z += csum[q];
+  const double target = pl.u * Z;
+  int tok;
+  if (s_use_res) tok = draw_token(V, p.nvch, csum, target, w_res);
+  else tok = draw_token(V, p.nvch, csum, target, w_p);
+  if (threadIdx.x == 0) p.out_tokens[(size_t)r * (k + 1) + pl.a] = tok;
+}
+
+// ------------------------------------------------------------------------- commit ----
+__global__ void commit_kernel(const int32_t* req_ids, int batch, int k, const int32_t* n_out,
+                              int32_t* seq_lens, long long* stats) {
+  const int bl = blockIdx.x * blockDim.x + threadIdx.x;
+  if (bl >= batch) return;
+  const int r = req_ids ? req_ids[bl] : bl;
+  const int n = n_out[r];
+  seq_lens[r] += n;
+  if (stats) {
+    atomicAdd(reinterpret_cast<unsigned long long*>(&stats[0]), (unsigned long long)n);
+    atomicAdd(reinterpret_cast<unsigned long long*>(&stats[1]), 1ull);
+    for (int j = 0; j < k && j < n; ++j) {
+      atomicAdd(reinterpret_cast<unsigned long long*>(&stats[2 + k + j]), 1ull);
+      if (j < n - 1) atomicAdd(reinterpret_cast<unsigned long long*>(&stats[2 + j]), 1ull);
+    }
+  }
+}
+
+__global__ void philox_kernel(uint64_t seed, int stream_id, const int32_t* request,
+                              const int32_t* position, int64_t n, uint32_t* words, float* u) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  uint32_t c[4] = {(uint32_t)position[i], (uint32_t)request[i], (uint32_t)stream_id, 0u};
+  philox4x32_10(c, (uint32_t)seed, (uint32_t)(seed >> 32));
+  if (words) {
+    words[4 * i + 0] = c[0];
+    words[4 * i + 1] = c[1];
+    words[4 * i + 2] = c[2];
+    words[4 * i + 3] = c[3];
+  }
+  if (u) u[i] = (float)(c[0] >> 8) * (1.0f / 16777216.0f);
+}
+
+// ------------------------------------------------------------------------ launchers ----
+int launch_draft_sample(const SampleParams& p, int batch, cudaStream_t stream) {
+  dim3 grid(batch, p.nvch);
+  draft_sample_kernel<<<grid, kSampThreads, 0, stream>>>(p);
+  return cuda_status(cudaGetLastError(), __func__);
+}
+
+int launch_spec_sample(const SampleParams& p, int batch, cudaStream_t stream, int* launches) {
+  dim3 g1(batch, 2 * p.k + 1, p.nvch);
+  spec_norm_kernel<<<g1, kSampThreads, 0, stream>>>(p);
+  if (cuda_status(cudaGetLastError(), __func__) != S3R_OK) return S3R_ERR_CUDA;
+  dim3 g2(batch, p.nvch);
+  spec_draw_kernel<<<g2, kSampThreads, 0, stream>>>(p);
+  *launches = 2;
+  return cuda_status(cudaGetLastError(), __func__);
+}
+
+size_t sample_partial_bytes(int num_requests, int k, int vocab) {
+  const size_t nvch = (size_t)((vocab + kVocabChunk - 1) / kVocabChunk);
+  const size_t a = align_up((size_t)num_requests * (2 * k + 1) * nvch * sizeof(MS), 256);
+  const size_t b = align_up((size_t)num_requests * sizeof(SpecPlan), 256);
+  const size_t c = align_up((size_t)num_requests * nvch * sizeof(double2), 256);
+  return a + b + c;
+}
+
+void spec_offsets(int num_requests, int k, int vocab, size_t* plan_off, size_t* draw_off) {
+  const size_t nvch = (size_t)((vocab + kVocabChunk - 1) / kVocabChunk);
+  *plan_off = align_up((size_t)num_requests * (2 * k + 1) * nvch * sizeof(MS), 256);
+  *draw_off = *plan_off + align_up((size_t)num_requests * sizeof(SpecPlan), 256);
+}
+
+int launch_commit(const int32_t* req_ids, int batch, int k, const int32_t* n_out,
+                  int32_t* seq_lens, int64_t* stats, cudaStream_t stream) {
+  commit_kernel<<<(batch + 255) / 256, 256, 0, stream>>>(req_ids, batch, k, n_out, seq_lens,
+                                                        reinterpret_cast<long long*>(stats));
+  return cuda_status(cudaGetLastError(), __func__);
+}
+
+int launch_philox(uint64_t seed, int stream_id, const int32_t* request, const int32_t* position,
+                  int64_t n, uint32_t* words, float* u, cudaStream_t stream) {
+  philox_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(seed, stream_id, request, position,
+                                                                 n, words, u);
+  return cuda_status(cudaGetLastError(), __func__);
+}
+
+}  // namespace s3r

@@ -1,0 +1,131 @@
+"""A round driver over the C ABI: owns the per-batch device buffers and issues, per round,
+select -> k x (sparse draft attention, [draft logits], draft sampling) -> dense verify ->
+[target logits] -> speculative sampling -> commit, all on one stream and all in libs3r.so.
+
+The logits between attention and sampling belong to the rest of the model; callers pass
+them in (synthetic workloads) or fill them from the attention outputs through the
+optional callbacks (a projection, as in the budget sweep).
+"""
+from __future__ import annotations
+
+import torch
+
+from . import _lib as L
+
+
+def budget_count(length: int, budget_bp: int, window: int) -> int:
+    """Size n of the sparse set at committed length `length` (host-side mirror for sizing)."""
+    n = -(-(length * budget_bp) // 10000)
+    w = min(window, length)
+    return min(max(n, w), length)
+
+
+class RoundBuffers:
+    """Device buffers of one batch: selection, attention outputs, tokens and statistics."""
+
+    def __init__(self, num_requests, num_q_heads, num_kv_heads, head_dim, cap, k, vocab,
+                 sel_stride, device="cuda"):
+        G = num_q_heads // num_kv_heads
+        f32, bf, i32 = torch.float32, torch.bfloat16, torch.int32
+        self.scores = torch.empty((num_requests, num_kv_heads, G * (k + 1), cap), dtype=f32, device=device)
+        self.lse = torch.empty((num_requests, k + 1, num_q_heads), dtype=f32, device=device)
+        self.prefill_lse = torch.empty((num_requests, 1, num_q_heads), dtype=f32, device=device)
+        self.sel_idx = torch.zeros((num_requests, num_kv_heads, sel_stride), dtype=i32, device=device)
+        self.sel_count = torch.zeros((num_requests, num_kv_heads), dtype=i32, device=device)
+        self.steps = [torch.full((num_requests,), i, dtype=i32, device=device) for i in range(max(k, 1))]
+        self.draft_out = torch.empty((num_requests, num_q_heads, head_dim), dtype=bf, device=device)
+        self.draft_lse = torch.empty((num_requests, num_q_heads), dtype=f32, device=device)
+        self.verify_out = torch.empty((num_requests, k + 1, num_q_heads, head_dim), dtype=bf, device=device)
+        self.draft_tokens = torch.zeros((num_requests, max(k, 1)), dtype=i32, device=device)
+        self.out_tokens = torch.full((num_requests, k + 1), -1, dtype=i32, device=device)
+        self.n_out = torch.zeros((num_requests,), dtype=i32, device=device)
+        self.stats = torch.zeros((2 + 2 * k,), dtype=torch.int64, device=device)
+
+
+class S3REngine:
+    """S3R rounds for a batch of requests over one paged KV cache on one GPU."""
+
+    def __init__(self, k_pool, v_pool, page_table, seq_lens, num_q_heads, *, k, budget_bp,
+                 window, vocab, seed, sel_stride=None):
+        if not (1 <= k <= L.MAX_K):
+            raise ValueError("k must be in 1..8")
+        self.k, self.budget_bp, self.window, self.vocab, self.seed = k, budget_bp, window, vocab, seed
+        self.k_pool, self.v_pool = k_pool, v_pool
+        self.page_table = page_table
+        self.seq_lens = seq_lens
+        self.cache = L.make_cache(k_pool, v_pool, num_q_heads)
+        self.num_requests, self.max_pages = page_table.shape
+        self.cap = self.max_pages * L.PAGE_SIZE
+        self.sel_stride = sel_stride or budget_count(self.cap, budget_bp, window)
+        self.buf = RoundBuffers(self.num_requests, num_q_heads, self.cache.num_kv_heads,
+                                self.cache.head_dim, self.cap, k, vocab, self.sel_stride,
+                                k_pool.device)
+        nbytes = L.s3r_workspace_size(self.cache, self.num_requests, self.max_pages, k, vocab,
+                                      self.sel_stride)
+        self.ws = L.new_workspace(nbytes, k_pool.device)
+        self.batch = L.make_batch(seq_lens, page_table)
+        self.k_prev = None
+
+    @property
+    def launches_per_round(self) -> int:
+        return 1 + 2 * self.k + 1 + 2 + 1
+
+    def prefill(self, q_x, k_x, v_x):
+        """One-row dense pass of each request's pending token at position L (the last step of
+        a prefill): writes its K/V and the scores the first selection reads.
+        q_x [NR][1][H_q][d], k_x / v_x [NR][1][H_kv][d]."""
+        b = self.buf
+        out = torch.empty_like(q_x)
+        L.s3r_verify_attn(self.cache, self.batch, 0, q_x, k_x, v_x, out, b.prefill_lse, b.scores,
+                          self.ws)
+        self.k_prev = 0
+        return out
+
+    def select(self):
+        b = self.buf
+        lse = b.prefill_lse if self.k_prev == 0 else b.lse
+        L.s3r_select_kv(self.cache, self.batch, b.scores, lse, self.k_prev, self.budget_bp,
+                        self.window, b.sel_idx, b.sel_count, self.ws)
+
+    def draft_step(self, i, q_block, k_block, v_block, q_logits, draft_logits_fn=None):
+        b = self.buf
+        L.s3r_sparse_draft_attn(self.cache, self.batch, b.steps[i], q_block[:, i], k_block[:, i],
+                                v_block[:, i], b.sel_idx, b.sel_count, b.draft_out, b.draft_lse,
+                                self.ws)
+        if draft_logits_fn is not None:
+            draft_logits_fn(i, b.draft_out, q_logits)
+        L.s3r_draft_sample(self.batch, b.steps[i], self.k, q_logits, self.vocab, self.seed,
+                           b.draft_tokens, self.ws)
+
+    def verify(self, q_block, k_block, v_block):
+        b = self.buf
+        L.s3r_verify_attn(self.cache, self.batch, self.k, q_block, k_block, v_block, b.verify_out,
+                          b.lse, b.scores, self.ws)
+        self.k_prev = self.k
+
+    def sample_and_commit(self, p_logits, q_logits):
+        b = self.buf
+        L.s3r_spec_sample(self.batch, self.k, p_logits, q_logits, b.draft_tokens, self.vocab,
+                          self.seed, b.out_tokens, b.n_out, self.ws)
+        L.s3r_commit(self.batch, self.k, b.n_out, self.seq_lens, b.stats)
+
+    def round(self, q_block, k_block, v_block, p_logits, q_logits, draft_logits_fn=None,
+              target_logits_fn=None):
+        """One draft+verify round for every request.
+
+        q_block [NR][k+1][H_q][d], k_block / v_block [NR][k+1][H_kv][d]: projections of the
+        tokens at positions L..L+k; p_logits [NR][k+1][V], q_logits [NR][k][V] (filled by the
+        callbacks when given)."""
+        if self.k_prev is None:
+            raise RuntimeError("call prefill() before the first round")
+        self.select()
+        for i in range(self.k):
+            self.draft_step(i, q_block, k_block, v_block, q_logits, draft_logits_fn)
+        self.verify(q_block, k_block, v_block)
+        if target_logits_fn is not None:
+            target_logits_fn(self.buf.verify_out, p_logits)
+        self.sample_and_commit(p_logits, q_logits)
+
+    def check_errors(self) -> int:
+        """Synchronise and return (and clear) the device error bitmask."""
+        return L.s3r_get_error(self.ws)

@@ -13,4 +13,8 @@ from .workload import (  # noqa: F401
     token_qkv,
     token_logits,
     bf16_round,
+    initial_phases,
+    projection_matrix,
+    randn_bf16,
+    randn_f32,
 )

@@ -1,0 +1,59 @@
+"""Shared helpers of the GPU parity tests: seeded cases on the device and their dense
+float64 copies for the oracle. Inputs come from `synth`; expected values from `oracle`."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import synth
+from oracle import s3r_oracle as O
+
+ATOL, RTOL = 2e-2, 1e-2          # attention outputs: bf16 out, fp32 accumulation
+MARGIN = 1e-5                     # decisions closer than this to a boundary are not compared
+
+
+def spec_for(H_q, H_kv, d, lens, k=6, budget_bp=500, window=64, vocab=64, seed=0, heavy=0,
+             shuffle=False):
+    return synth.CONFIGS[0].with_(num_requests=len(lens), num_q_heads=H_q, num_kv_heads=H_kv,
+                                  head_dim=d, lengths=("fixed", tuple(int(x) for x in lens)),
+                                  k=k, budget_bp=budget_bp, window=window, vocab=vocab,
+                                  data_seed=seed, heavy_hitters=heavy, shuffle_pages=shuffle)
+
+
+class Case:
+    """A paged cache generated on the host, copied to the GPU, plus host float copies."""
+
+    def __init__(self, spec, extra_tokens, seed=None):
+        self.spec = spec
+        self.cache = synth.build_cache(spec, synth.make_lengths(spec), extra_tokens, "cpu", seed)
+        self.k_pool = self.cache.k_pool.cuda()
+        self.v_pool = self.cache.v_pool.cuda()
+        self.page_table = self.cache.page_table.cuda()
+        self.lens = self.cache.lengths.copy()
+        self.seq_lens = torch.as_tensor(self.lens, dtype=torch.int32).cuda()
+
+    def host_pools(self):
+        """Current device pools as float32 numpy arrays."""
+        return self.k_pool.float().cpu().numpy(), self.v_pool.float().cpu().numpy()
+
+    def dense(self, r, upto, pools=None):
+        """K, V [H_kv][upto][d] float64 of request r from the (device) pools."""
+        kp, vp = pools if pools is not None else self.host_pools()
+        pt = self.cache.page_table.numpy()[r]
+        H = self.spec.num_kv_heads
+        K = np.stack([O.gather_positions(kp, pt, h, np.arange(upto)) for h in range(H)])
+        V = np.stack([O.gather_positions(vp, pt, h, np.arange(upto)) for h in range(H)])
+        return K, V
+
+
+def f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def assert_attention_close(gpu, ref, what=""):
+    gpu = np.asarray(gpu, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    err = np.abs(gpu - ref)
+    bound = ATOL + RTOL * np.abs(ref)
+    bad = err > bound
+    assert not bad.any(), f"{what}: {bad.sum()} of {bad.size} outside tolerance, max err {err.max():.3g}"

@@ -1,0 +1,92 @@
+"""CPU checks of the C ABI: the library loads, exports every entry point include/s3r.h
+declares, and rejects bad arguments on the host (nothing is launched without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "s3r.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^S3R_API\s+[\w\s\*]+?\b(s3r_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_hot_path():
+    syms = declared_symbols()
+    for name in ("s3r_select_kv", "s3r_sparse_draft_attn", "s3r_verify_attn", "s3r_spec_sample",
+                 "s3r_draft_sample", "s3r_commit", "s3r_workspace_size", "s3r_get_error"):
+        assert name in syms
+
+
+def test_library_exports_every_declared_symbol():
+    import sparse_dense_kv_b200 as s3r
+    raw = ctypes.CDLL(s3r.LIB_PATH)
+    missing = [n for n in declared_symbols() if not hasattr(raw, n)]
+    assert not missing, missing
+
+
+def test_status_strings_and_counter():
+    import sparse_dense_kv_b200 as s3r
+    for code, name in s3r.STATUS_NAMES.items():
+        assert s3r.s3r_status_string(code)
+    assert s3r.s3r_status_string(99) == "unknown status"
+    assert s3r.s3r_launch_count() >= 0
+
+
+def _cache(**kw):
+    import sparse_dense_kv_b200 as s3r
+    d = dict(num_q_heads=32, num_kv_heads=8, head_dim=128, page_size=16, num_pages=1000,
+             k_pool=0x100000, v_pool=0x200000)
+    d.update(kw)
+    return s3r.KVCacheDesc(**d)
+
+
+def test_workspace_size_is_host_only_and_monotone():
+    import sparse_dense_kv_b200 as s3r
+    c = _cache()
+    a = s3r.s3r_workspace_size(c, 32, 1540, 6, 151936, 1232)
+    b = s3r.s3r_workspace_size(c, 64, 1540, 6, 151936, 1232)
+    assert 0 < a < b
+    assert s3r.s3r_workspace_size(c, 32, 1540, 8, 151936, 1232) >= a
+    with pytest.raises(s3r.S3RError):
+        s3r.s3r_workspace_size(_cache(head_dim=96), 32, 1540, 6, 151936, 1232)
+
+
+def test_host_validation_rejects_before_launch():
+    import sparse_dense_kv_b200 as s3r
+    L = s3r.lib
+    null = ctypes.c_void_p(0)
+    # NULL descriptors
+    assert L.s3r_verify_attn(None, None, 6, null, null, null, null, null, null, null, 0, null) == 1
+    b = s3r.BatchDesc(1, 1, None, 0x1000, 0x2000, 10)
+    # unsupported head_dim / page size / group / k
+    for bad in (_cache(head_dim=96), _cache(page_size=32), _cache(num_q_heads=72, num_kv_heads=8)):
+        assert L.s3r_verify_attn(ctypes.byref(bad), ctypes.byref(b), 6, 0x10, 0x10, 0x10, 0x10,
+                                 0x10, None, 0x100, 1 << 20, null) == 2
+    c = _cache()
+    assert L.s3r_verify_attn(ctypes.byref(c), ctypes.byref(b), 9, 0x10, 0x10, 0x10, 0x10, 0x10,
+                             None, 0x100, 1 << 20, null) == 2
+    # misaligned q
+    assert L.s3r_verify_attn(ctypes.byref(c), ctypes.byref(b), 6, 0x18, 0x10, 0x10, 0x10, 0x10,
+                             None, 0x100, 1 << 20, null) == 1
+    # workspace too small / misaligned
+    assert L.s3r_verify_attn(ctypes.byref(c), ctypes.byref(b), 6, 0x10, 0x10, 0x10, 0x10, 0x10,
+                             None, 0x100, 16, null) == 4
+    assert L.s3r_verify_attn(ctypes.byref(c), ctypes.byref(b), 6, 0x10, 0x10, 0x10, 0x10, 0x10,
+                             None, 0x180, 1 << 30, null) == 4
+    # selection: budget and window
+    assert L.s3r_select_kv(ctypes.byref(c), ctypes.byref(b), 0x10, 0x10, 6, 0, 64, 0x10, 100,
+                           0x10, 0x100, 1 << 30, null) == 1
+    assert L.s3r_select_kv(ctypes.byref(c), ctypes.byref(b), 0x10, 0x10, 6, 500, 6, 0x10, 100,
+                           0x10, 0x100, 1 << 30, null) == 1
+    # sampling: vocabulary and k
+    assert L.s3r_spec_sample(ctypes.byref(b), 9, 0x10, 0x10, 0x10, 64, 1, 0x10, 0x10, 0x100,
+                             1 << 30, null) == 2
+    assert L.s3r_draft_sample(ctypes.byref(b), 0x10, 6, 0x10, 0, 1, 0x10, 0x100, 1 << 30, null) == 2
+    # an empty batch is a no-op that succeeds
+    e = s3r.BatchDesc(0, 0, None, None, None, 0)
+    assert L.s3r_commit(ctypes.byref(e), 6, 0x10, 0x10, None, null) == 0

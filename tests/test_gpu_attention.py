@@ -1,0 +1,134 @@
+"""GPU parity of the verify and sparse draft attention kernels against the oracle."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+import sparse_dense_kv_b200 as s3r
+from oracle import s3r_oracle as O
+from tests.s3r_testlib import Case, assert_attention_close, f64, spec_for
+
+pytestmark = pytest.mark.gpu
+
+
+def run_verify(case, k, seed, scores=True):
+    spec = case.spec
+    NR, Hq, Hkv, d = spec.num_requests, spec.num_q_heads, spec.num_kv_heads, spec.head_dim
+    T = k + 1
+    q = synth.randn_bf16((NR, T, Hq, d), seed, "cuda")
+    kn = synth.randn_bf16((NR, T, Hkv, d), seed + 1, "cuda")
+    vn = synth.randn_bf16((NR, T, Hkv, d), seed + 2, "cuda")
+    out = torch.empty_like(q)
+    lse = torch.empty((NR, T, Hq), dtype=torch.float32, device="cuda")
+    cap = case.cache.capacity
+    G = Hq // Hkv
+    sc = torch.full((NR, Hkv, G * T, cap), float("nan"), device="cuda") if scores else None
+    cache = s3r.make_cache(case.k_pool, case.v_pool, Hq)
+    batch = s3r.make_batch(case.seq_lens, case.page_table)
+    ws = s3r.new_workspace(s3r.s3r_workspace_size(cache, NR, case.cache.max_pages, k, 64, 64))
+    s3r.s3r_verify_attn(cache, batch, k, q, kn, vn, out, lse, sc, ws)
+    assert s3r.s3r_get_error(ws) == 0
+    return q, kn, vn, out, lse, sc
+
+
+@pytest.mark.parametrize("Hq,Hkv,d,k,lens", [
+    (2, 1, 64, 6, [256, 300]),                 # tiny workload shape
+    (32, 8, 128, 6, [1000, 2049, 3071, 64]),   # GQA 4, ragged, several chunks, 28 rows
+    (16, 8, 128, 0, [700, 1500]),              # one-row pass (prefill scores)
+    (32, 8, 128, 8, [1030, 2000]),             # 36 rows: three row groups
+    (8, 1, 128, 2, [5, 17, 0, 33]),            # short / empty contexts, G = 8
+])
+def test_verify_matches_oracle(Hq, Hkv, d, k, lens):
+    spec = spec_for(Hq, Hkv, d, lens, k=k, seed=11)
+    case = Case(spec, extra_tokens=k + 1 + 20)
+    q, kn, vn, out, lse, sc = run_verify(case, k, seed=100)
+    kp, vp = case.host_pools()
+    T, G = k + 1, Hq // Hkv
+    for r, L in enumerate(case.lens):
+        K, V = case.dense(r, L + T, (kp, vp))
+        # the block rows now in the pool are the caller's k_new / v_new
+        np.testing.assert_array_equal(K[:, L:], f64(kn[r]).transpose(1, 0, 2))
+        np.testing.assert_array_equal(V[:, L:], f64(vn[r]).transpose(1, 0, 2))
+        o, l, sigma, logits = O.verify_attention(f64(q[r]), K, V, int(L))
+        assert_attention_close(f64(out[r]), o, f"out r={r}")
+        np.testing.assert_allclose(f64(lse[r]), l, rtol=0, atol=2e-4)
+        got = f64(sc[r][:, :, :L])
+        np.testing.assert_allclose(got, logits[:, :, :L], rtol=1e-5, atol=1e-4)
+
+
+def test_verify_without_score_capture_and_full_capacity():
+    k = 6
+    spec = spec_for(32, 8, 128, [1017, 64], k=k, seed=3)
+    case = Case(spec, extra_tokens=k + 1)          # L + k + 1 reaches the page-table capacity
+    q, kn, vn, out, lse, _ = run_verify(case, k, seed=7, scores=False)
+    kp, vp = case.host_pools()
+    for r, L in enumerate(case.lens):
+        K, V = case.dense(r, L + k + 1, (kp, vp))
+        o, l, _, _ = O.verify_attention(f64(q[r]), K, V, int(L))
+        assert_attention_close(f64(out[r]), o, f"out r={r}")
+
+
+def draft_case(Hq, Hkv, d, lens, steps, budget_bp, window, seed):
+    spec = spec_for(Hq, Hkv, d, lens, budget_bp=budget_bp, window=window, seed=seed)
+    case = Case(spec, extra_tokens=16)
+    NR = len(lens)
+    rng = np.random.default_rng(seed)
+    sels = [[O.select_positions(rng.exponential(size=L), int(L), budget_bp, window)
+             for _ in range(Hkv)] for L in case.lens]
+    stride = max(len(s) for ss in sels for s in ss)
+    sel_idx = torch.zeros((NR, Hkv, stride), dtype=torch.int32)
+    sel_cnt = torch.zeros((NR, Hkv), dtype=torch.int32)
+    for r in range(NR):
+        for h in range(Hkv):
+            sel_idx[r, h, : len(sels[r][h])] = torch.as_tensor(sels[r][h])
+            sel_cnt[r, h] = len(sels[r][h])
+    q = synth.randn_bf16((NR, Hq, d), seed + 1, "cuda")
+    kn = synth.randn_bf16((NR, Hkv, d), seed + 2, "cuda")
+    vn = synth.randn_bf16((NR, Hkv, d), seed + 3, "cuda")
+    step = torch.as_tensor(steps, dtype=torch.int32).cuda()
+    out = torch.empty_like(q)
+    lse = torch.empty((NR, Hq), dtype=torch.float32, device="cuda")
+    cache = s3r.make_cache(case.k_pool, case.v_pool, Hq)
+    batch = s3r.make_batch(case.seq_lens, case.page_table)
+    ws = s3r.new_workspace(s3r.s3r_workspace_size(cache, NR, case.cache.max_pages, 8, 64, stride))
+    s3r.s3r_sparse_draft_attn(cache, batch, step, q, kn, vn, sel_idx.cuda(), sel_cnt.cuda(), out,
+                              lse, ws)
+    assert s3r.s3r_get_error(ws) == 0
+    return case, sels, q, kn, vn, out, lse
+
+
+@pytest.mark.parametrize("Hq,Hkv,d,lens,steps,bp,W", [
+    (2, 1, 64, [256, 300], [0, 5], 2500, 16),
+    (32, 8, 128, [4100, 9000, 700], [3, 0, 5], 500, 64),
+    (16, 8, 128, [2000, 3000], [1, 2], 2000, 64),       # several draft chunks
+    (32, 8, 128, [1500, 600], [2, 4], 10000, 64),       # s = 1: every committed position
+])
+def test_sparse_draft_matches_oracle(Hq, Hkv, d, lens, steps, bp, W):
+    case, sels, q, kn, vn, out, lse = draft_case(Hq, Hkv, d, lens, steps, bp, W, seed=21)
+    kp, vp = case.host_pools()
+    for r, L in enumerate(case.lens):
+        i = steps[r]
+        K, V = case.dense(r, L + i + 1, (kp, vp))
+        np.testing.assert_array_equal(K[:, L + i], f64(kn[r]))   # this step's token was appended
+        np.testing.assert_array_equal(V[:, L + i], f64(vn[r]))
+        o, l = O.sparse_draft_attention(f64(q[r]), K, V, sels[r], int(L), i)
+        assert_attention_close(f64(out[r]), o, f"draft r={r}")
+        np.testing.assert_allclose(f64(lse[r]), l, rtol=0, atol=2e-4)
+
+
+def test_sparse_draft_full_budget_equals_verify_row():
+    """With s = 1 the draft of step 0 reads every committed position plus its own token:
+    the verify's first row on the same cache and token."""
+    Hq, Hkv, d, lens = 32, 8, 128, [1300, 517]
+    case, sels, q, kn, vn, out, lse = draft_case(Hq, Hkv, d, lens, [0, 0], 10000, 64, seed=5)
+    cache = s3r.make_cache(case.k_pool, case.v_pool, Hq)
+    batch = s3r.make_batch(case.seq_lens, case.page_table)
+    NR = len(lens)
+    vq = q[:, None].contiguous()
+    vo = torch.empty_like(vq)
+    vl = torch.empty((NR, 1, Hq), dtype=torch.float32, device="cuda")
+    ws = s3r.new_workspace(s3r.s3r_workspace_size(cache, NR, case.cache.max_pages, 0, 64, 64))
+    s3r.s3r_verify_attn(cache, batch, 0, vq, kn[:, None].contiguous(), vn[:, None].contiguous(),
+                        vo, vl, None, ws)
+    torch.cuda.synchronize()
+    assert_attention_close(f64(out), f64(vo[:, 0]), "draft vs verify row")
