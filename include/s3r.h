@@ -113,9 +113,10 @@ S3R_API int s3r_workspace_init(void* ws, size_t ws_bytes, s3r_stream_t stream);
  *              of positions L..L+k (which must be allocated) and used for the block.
  *   out        bf16 [num_requests][T][H_q][d], softmax(q K^T / sqrt(d)) V rounded once.
  *   lse        fp32 [num_requests][T][H_q], natural-log log-sum-exp of the logits.
- *   score_logits fp32 [num_requests][H_kv][G*T][capacity] or NULL: logit q.k/sqrt(d) of
- *              row t*G+g of each KV head at every committed position j < L (entries at
- *              j >= L are not written). With lse it defines the scores of s3r_select_kv.
+ *   score_logits fp32 [num_requests][H_kv][capacity][G*T] or NULL: logit q.k/sqrt(d) of
+ *              row t*G+g of each KV head at every committed position j < L, the G*T logits
+ *              of one position contiguous (entries at j >= L are not written). With lse it
+ *              defines the scores of s3r_select_kv.
  * Needs L + T <= capacity (device check). */
 S3R_API int s3r_verify_attn(const s3r_kv_cache* cache, const s3r_batch* batch, int32_t k,
                     const void* q, const void* k_new, const void* v_new, void* out,

@@ -50,10 +50,15 @@ struct WarpAttn {
   }
 
   // One 16-position m-tile starting at tile row `row0` of the stage at kb / vb (shared
-  // addresses). `visible(tile_row, nt, j)` says whether the lane's row j (0/1) of n-tile nt
-  // sees the position in tile row `tile_row`; `capture(tile_row, nt, j, logit)` receives the
-  // natural-log logit of every pair (visible or not).
-  template <class Visible, class Capture>
+  // addresses). With MASKED, `visible(tile_row, nt, j)` says whether the lane's row j (0/1)
+  // of n-tile nt sees the position in tile row `tile_row` (without it every pair is
+  // visible). `capture(tile_row, nt, logit_j0, logit_j1)` receives the natural-log logits
+  // of the lane's two rows at each of its two positions.
+  //
+  // The running max is lazy: P = 2^(x - m) is formed against a reference max m that is
+  // raised only when a tile exceeds it by more than 8 (log2 units), so P <= 256 stays exact
+  // enough in bf16 and the O / l rescale is skipped for almost every tile.
+  template <bool MASKED, class Visible, class Capture>
   __device__ __forceinline__ void step(uint32_t kb, uint32_t vb, int row0, int lane,
                                        float scale, Visible visible, Capture capture) {
     const int mi = lane >> 3, rr = lane & 7;
@@ -73,15 +78,17 @@ struct WarpAttn {
     const int p0 = row0 + (lane >> 2), p1 = p0 + 8;
     const float scale2 = scale * kLog2e;
     uint32_t b[NTW][2];
+    float al[NTW][2];
+    bool any_rescale = false;
 #pragma unroll
     for (int nt = 0; nt < NTW; ++nt) {
+      capture(p0, nt, s[nt][0] * scale, s[nt][1] * scale);
+      capture(p1, nt, s[nt][2] * scale, s[nt][3] * scale);
       float x[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const int pr = (i < 2) ? p0 : p1;
-        const int j = i & 1;
-        capture(pr, nt, j, s[nt][i] * scale);
-        x[i] = visible(pr, nt, j) ? s[nt][i] * scale2 : -INFINITY;
+        x[i] = s[nt][i] * scale2;
+        if (MASKED && !visible((i < 2) ? p0 : p1, nt, i & 1)) x[i] = -INFINITY;
       }
       float mx0 = fmaxf(x[0], x[2]), mx1 = fmaxf(x[1], x[3]);
 #pragma unroll
@@ -89,26 +96,37 @@ struct WarpAttn {
         mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, off));
         mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, off));
       }
-      const float mn0 = fmaxf(m[nt][0], mx0), mn1 = fmaxf(m[nt][1], mx1);
-      const float al0 = (mn0 == -INFINITY) ? 1.f : ex2(m[nt][0] - mn0);
-      const float al1 = (mn1 == -INFINITY) ? 1.f : ex2(m[nt][1] - mn1);
-      m[nt][0] = mn0;
-      m[nt][1] = mn1;
-      const float e0 = (mn0 == -INFINITY) ? 0.f : ex2(x[0] - mn0);
-      const float e1 = (mn1 == -INFINITY) ? 0.f : ex2(x[1] - mn1);
-      const float e2 = (mn0 == -INFINITY) ? 0.f : ex2(x[2] - mn0);
-      const float e3 = (mn1 == -INFINITY) ? 0.f : ex2(x[3] - mn1);
-      l[nt][0] = l[nt][0] * al0 + e0 + e2;
-      l[nt][1] = l[nt][1] * al1 + e1 + e3;
-#pragma unroll
-      for (int dm = 0; dm < D / 16; ++dm) {
-        o[dm][nt][0] *= al0;
-        o[dm][nt][1] *= al1;
-        o[dm][nt][2] *= al0;
-        o[dm][nt][3] *= al1;
+      al[nt][0] = al[nt][1] = 1.f;
+      if (mx0 > m[nt][0] + 8.f) {
+        al[nt][0] = ex2(m[nt][0] - mx0);   // 0 when m was -inf
+        m[nt][0] = mx0;
+        any_rescale = true;
       }
+      if (mx1 > m[nt][1] + 8.f) {
+        al[nt][1] = ex2(m[nt][1] - mx1);
+        m[nt][1] = mx1;
+        any_rescale = true;
+      }
+      const float r0 = m[nt][0], r1 = m[nt][1];
+      const float e0 = (r0 == -INFINITY) ? 0.f : ex2(x[0] - r0);
+      const float e1 = (r1 == -INFINITY) ? 0.f : ex2(x[1] - r1);
+      const float e2 = (r0 == -INFINITY) ? 0.f : ex2(x[2] - r0);
+      const float e3 = (r1 == -INFINITY) ? 0.f : ex2(x[3] - r1);
+      l[nt][0] = l[nt][0] * al[nt][0] + e0 + e2;
+      l[nt][1] = l[nt][1] * al[nt][1] + e1 + e3;
       b[nt][0] = movm_t(pack_bf16(e0, e1));
       b[nt][1] = movm_t(pack_bf16(e2, e3));
+    }
+    if (__any_sync(kFull, any_rescale)) {
+#pragma unroll
+      for (int dm = 0; dm < D / 16; ++dm)
+#pragma unroll
+        for (int nt = 0; nt < NTW; ++nt) {
+          o[dm][nt][0] *= al[nt][0];
+          o[dm][nt][1] *= al[nt][1];
+          o[dm][nt][2] *= al[nt][0];
+          o[dm][nt][3] *= al[nt][1];
+        }
     }
     const int vrow = row0 + rr + 8 * (mi >> 1);
 #pragma unroll
@@ -197,26 +215,65 @@ __device__ __forceinline__ void merge_slices_to_record(const float* redO, const 
 
 // Combine `nch` chunk records of `R` rows into normalised outputs: for row < R and d < D,
 // out = sum_c O_c exp2(m_c - M) / sum_c l_c exp2(m_c - M); lse (natural) per row.
+// The per-(chunk, row) weights are formed once in shared memory (`wts`, >= 32*R floats),
+// then every thread sums 4 consecutive d of one row over the chunks with 16-byte loads
+// (R * D / 4 <= 4 * nthreads: R <= 16 rows per 128 threads).
 template <int D, class OutPtr, class LsePtr>
 __device__ __forceinline__ void combine_records(const float* recs, size_t rec_floats, int nch,
-                                                int R, int Rp, OutPtr out_row, LsePtr lse_row) {
-  for (int idx = threadIdx.x; idx < R * D; idx += blockDim.x) {
-    const int row = idx / D, d = idx - row * D;
-    float M = -INFINITY;
-    for (int c = 0; c < nch; ++c) M = fmaxf(M, __ldcg(recs + c * rec_floats + row));
-    float acc = 0.f, lsum = 0.f;
-    for (int c = 0; c < nch; ++c) {
-      const float* rc = recs + c * rec_floats;
-      const float mc = __ldcg(rc + row);
-      const float f = (mc == -INFINITY) ? 0.f : exp2f(mc - M);
-      acc += f * __ldcg(rc + 2 * Rp + (size_t)row * D + d);
-      lsum += f * __ldcg(rc + Rp + row);
+                                                int R, int Rp, float* wts, OutPtr out_row,
+                                                LsePtr lse_row, int tid, int nthreads) {
+  float4 acc[4];
+  const int nvec = R * (D / 4);
+  for (int c0 = 0; c0 < nch; c0 += 32) {
+    const int cn = min(32, nch - c0);
+    // weights of this batch of chunks, relative to the max over all chunks
+    for (int row = tid; row < R; row += nthreads) {
+      float M = -INFINITY;
+      for (int c = 0; c < nch; ++c) M = fmaxf(M, __ldcg(recs + c * rec_floats + row));
+      float lsum = 0.f;
+      for (int c = 0; c < nch; ++c) {
+        const float mc = __ldcg(recs + c * rec_floats + row);
+        lsum += (mc == -INFINITY) ? 0.f : exp2f(mc - M) * __ldcg(recs + c * rec_floats + Rp + row);
+      }
+      for (int c = 0; c < cn; ++c) {
+        const float mc = __ldcg(recs + (c0 + c) * rec_floats + row);
+        wts[c * R + row] = (mc == -INFINITY) ? 0.f : exp2f(mc - M) / lsum;
+      }
+      if (c0 == 0 && tid < R) {
+        float* lp = lse_row(row);
+        if (lp) *lp = (M + log2f(lsum)) * kLn2;
+      }
     }
-    out_row(row)[d] = __float2bfloat16_rn(acc / lsum);
-    if (d == 0) {
-      float* lp = lse_row(row);
-      if (lp) *lp = (M + log2f(lsum)) * kLn2;
+    __syncthreads();
+#pragma unroll
+    for (int slot = 0; slot < 4; ++slot) {
+      const int v = tid + slot * nthreads;
+      if (v >= nvec) break;
+      const int row = v / (D / 4), d4 = v - row * (D / 4);
+      float4 a = (c0 == 0) ? make_float4(0.f, 0.f, 0.f, 0.f) : acc[slot];
+#pragma unroll 4
+      for (int c = 0; c < cn; ++c) {
+        const float w = wts[c * R + row];
+        const float4 x = __ldcg(reinterpret_cast<const float4*>(
+            recs + (c0 + c) * rec_floats + 2 * Rp + (size_t)row * D) + d4);
+        a.x += w * x.x;
+        a.y += w * x.y;
+        a.z += w * x.z;
+        a.w += w * x.w;
+      }
+      acc[slot] = a;
     }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int slot = 0; slot < 4; ++slot) {
+    const int v = tid + slot * nthreads;
+    if (v >= nvec) break;
+    const int row = v / (D / 4), d4 = v - row * (D / 4);
+    const float4 a = acc[slot];
+    __nv_bfloat162* o = reinterpret_cast<__nv_bfloat162*>(out_row(row) + d4 * 4);
+    o[0] = __floats2bfloat162_rn(a.x, a.y);
+    o[1] = __floats2bfloat162_rn(a.z, a.w);
   }
 }
 

@@ -136,10 +136,12 @@ __global__ void __launch_bounds__(128) draft_kernel(const DraftParams p) {
     const uint32_t kb = sbase + (it % kDraftStages) * STAGE, vb = kb + kTile * D * 2;
     const int row0 = warp * 16;
     if (t0 + row0 < end) {
-      wa.step(
-          kb, vb, row0, lane, p.scale,
-          [&](int tr, int, int) -> bool { return t0 + tr < end; },
-          [](int, int, int, float) {});
+      auto vis = [&](int tr, int, int) -> bool { return t0 + tr < end; };
+      auto nocap = [](int, int, float, float) {};
+      if (t0 + kTile <= end)
+        wa.template step<false>(kb, vb, row0, lane, p.scale, vis, nocap);
+      else
+        wa.template step<true>(kb, vb, row0, lane, p.scale, vis, nocap);
     }
     __syncthreads();
   }
@@ -156,12 +158,14 @@ __global__ void __launch_bounds__(128) draft_kernel(const DraftParams p) {
   merge_slices_to_record<D, RW>(redO, redM, redL, 1, recs + c * rec_floats, RW);
 
   if (!last_of(p.tickets + (size_t)r * Hkv + kvh, nch, s_flag)) return;
+  __shared__ float wts[32 * RW];
   combine_records<D>(
-      recs, rec_floats, nch, G, RW,
+      recs, rec_floats, nch, G, RW, wts,
       [&](int row) { return p.out + ((size_t)r * p.Hq + kvh * G + row) * D; },
       [&](int row) -> float* {
         return p.lse ? p.lse + (size_t)r * p.Hq + kvh * G + row : nullptr;
-      });
+      },
+      tid, blockDim.x);
 }
 
 template <int D>

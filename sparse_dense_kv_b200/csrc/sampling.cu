@@ -34,46 +34,70 @@ struct SpecPlan {
   double zp, zq, u;
 };
 
-// Block reduction of (max, sum) pairs; result valid in thread 0.
-__device__ MS block_ms(float m, double s) {
-  __shared__ float sm[kSampThreads / 32];
-  __shared__ double ss[kSampThreads / 32];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+// (max, sum 2^((x - max) log2 e)) of this thread's share of row[v0 .. v1): up to 32 entries,
+// as eight 16-byte loads (v0 + 4 (t + 256 j)) when the range is 16-byte aligned, else as
+// strided scalars. NaN and +inf are flagged and count as probability 0; -inf is a valid
+// zero-probability logit.
+__device__ __forceinline__ void thread_ms(const float* row, int v0, int v1, float& m, float& s,
+                                          bool& bad) {
+  float x[32];
+  const bool vec = ((reinterpret_cast<uintptr_t>(row + v0) & 15u) == 0) && (((v1 - v0) & 3) == 0);
+  if (vec) {
 #pragma unroll
-  for (int o = 16; o; o >>= 1) {
-    const float m2 = __shfl_xor_sync(kFull, m, o);
-    const double s2 = __shfl_xor_sync(kFull, s, o);
-    merge_ms(m, s, m2, s2);
+    for (int j = 0; j < 8; ++j) {
+      const int v = v0 + 4 * ((int)threadIdx.x + kSampThreads * j);
+      float4 q = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+      if (v < v1) q = __ldg(reinterpret_cast<const float4*>(row + v));
+      x[4 * j] = q.x;
+      x[4 * j + 1] = q.y;
+      x[4 * j + 2] = q.z;
+      x[4 * j + 3] = q.w;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const int v = v0 + (int)threadIdx.x + kSampThreads * j;
+      x[j] = v < v1 ? __ldg(row + v) : -INFINITY;
+    }
   }
+  m = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    if (isnan(x[j]) || x[j] == INFINITY) {
+      bad = true;
+      x[j] = -INFINITY;
+    }
+    m = fmaxf(m, x[j]);
+  }
+  s = 0.f;
+  if (m != -INFINITY) {
+    const float mb = m * kLog2e;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) s += ex2(fmaf(x[j], kLog2e, -mb));
+  }
+}
+
+// Block reduction of per-thread (max, sum) pairs; the result is valid in thread 0.
+__device__ MS block_ms(float m, float s) {
+  __shared__ float sm[kSampThreads / 32];
+  __shared__ float ss[kSampThreads / 32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const float mw = warp_max(m);
+  float sw = (m == -INFINITY) ? 0.f : s * ex2((m - mw) * kLog2e);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) sw += __shfl_xor_sync(kFull, sw, o);
   if (lane == 0) {
-    sm[warp] = m;
-    ss[warp] = s;
+    sm[warp] = mw;
+    ss[warp] = sw;
   }
   __syncthreads();
   MS r{-INFINITY, 0.f, 0.0};
-  if (threadIdx.x == 0)
-    for (int w = 0; w < kSampThreads / 32; ++w) merge_ms(r.m, r.s, sm[w], ss[w]);
-  return r;
-}
-
-// (max, sum exp(x - max)) of row[v0 .. v1) by this thread (strided), fp64 sum.
-__device__ __forceinline__ void chunk_ms(const float* row, int v0, int v1, float& m, double& s,
-                                         bool& bad) {
-  m = -INFINITY;
-  s = 0.0;
-  for (int v = v0 + threadIdx.x; v < v1; v += blockDim.x) {
-    const float x = __ldg(row + v);
-    if (!isfinite(x)) {
-      bad = true;
-      continue;
-    }
-    if (x > m) {
-      s = s * (double)expf(m - x) + 1.0;
-      m = x;
-    } else {
-      s += (double)expf(x - m);
-    }
+  if (threadIdx.x == 0) {
+    for (int w = 0; w < kSampThreads / 32; ++w) r.m = fmaxf(r.m, sm[w]);
+    for (int w = 0; w < kSampThreads / 32; ++w)
+      if (sm[w] != -INFINITY) r.s += (double)ss[w] * (double)ex2((sm[w] - r.m) * kLog2e);
   }
+  return r;
 }
 
 __device__ double block_sum_d(double v) {
@@ -128,8 +152,9 @@ __device__ int chunk_search(int v0, int v1, double target, double& base, W weigh
   const int t = threadIdx.x;
   const int a = v0 + t * kSeg;
   const int b = min(a + kSeg, v1);
-  double seg = 0.0;
-  for (int v = a; v < b; ++v) seg += weight(v);
+  float segf = 0.f;
+  for (int v = a; v < b; ++v) segf += weight(v);
+  const double seg = segf;
   double total;
   const double excl = block_excl_scan_d(seg, total);
   hi_s[t] = base + (excl + seg);
@@ -165,7 +190,7 @@ __device__ int last_nonzero(int V, W weight) {
   if (threadIdx.x == 0) s_last = -1;
   __syncthreads();
   for (int v = threadIdx.x; v < V; v += blockDim.x)
-    if (weight(v) > 0.0) atomicMax(&s_last, v);
+    if (weight(v) > 0.f) atomicMax(&s_last, v);
   __syncthreads();
   const int r = s_last;
   __syncthreads();
@@ -217,10 +242,9 @@ __global__ void __launch_bounds__(kSampThreads) draft_sample_kernel(const Sample
   const float* row = p.q_logits + ((size_t)r * p.k + i) * V;
   MS* part = reinterpret_cast<MS*>(p.part) + (size_t)r * p.nvch;
 
-  float m;
-  double s;
+  float m, s;
   bool bad = false;
-  chunk_ms(row, c * kVocabChunk, min(V, (c + 1) * kVocabChunk), m, s, bad);
+  thread_ms(row, c * kVocabChunk, min(V, (c + 1) * kVocabChunk), m, s, bad);
   if (bad) set_error(p.err, S3R_ERR_NONFINITE);
   const MS tot = block_ms(m, s);
   if (threadIdx.x == 0) part[c] = tot;
@@ -231,7 +255,7 @@ __global__ void __launch_bounds__(kSampThreads) draft_sample_kernel(const Sample
     for (int q = 0; q < p.nvch; ++q) M = fmaxf(M, __ldcg(&part[q].m));
     for (int q = 0; q < p.nvch; ++q) {
       const float mq = __ldcg(&part[q].m);
-      csum[q] = (mq == -INFINITY) ? 0.0 : __ldcg(&part[q].s) * exp((double)mq - (double)M);
+      csum[q] = (mq == -INFINITY) ? 0.0 : __ldcg(&part[q].s) * (double)exp2f((mq - M) * kLog2e);
     }
     s_M = M;
   }
@@ -241,9 +265,10 @@ __global__ void __launch_bounds__(kSampThreads) draft_sample_kernel(const Sample
   for (int q = 0; q < p.nvch; ++q) Z += csum[q];
   const int L = p.seq_lens[r];
   const double u = philox_u(p.seed, (uint32_t)(L + i + 1), (uint32_t)r, 0u);
-  const int tok = draw_token(V, p.nvch, csum, u * Z, [&](int v) -> double {
+  const float Mb = M * kLog2e;
+  const int tok = draw_token(V, p.nvch, csum, u * Z, [&](int v) -> float {
     const float x = row[v];
-    return isfinite(x) ? (double)expf(x - M) : 0.0;
+    return (isnan(x) || x == INFINITY) ? 0.f : ex2(fmaf(x, kLog2e, -Mb));
   });
   if (threadIdx.x == 0) p.draft_out[(size_t)r * p.k + i] = tok;
 }
@@ -260,10 +285,9 @@ __global__ void __launch_bounds__(kSampThreads) spec_norm_kernel(const SamplePar
                                : p.q_logits + ((size_t)r * k + (rw - k - 1)) * V;
   MS* part = reinterpret_cast<MS*>(p.part) + (size_t)r * nrows * p.nvch;
 
-  float m;
-  double s;
+  float m, s;
   bool bad = false;
-  chunk_ms(row, c * kVocabChunk, min(V, (c + 1) * kVocabChunk), m, s, bad);
+  thread_ms(row, c * kVocabChunk, min(V, (c + 1) * kVocabChunk), m, s, bad);
   if (bad) set_error(p.err, S3R_ERR_NONFINITE);
   const MS tot = block_ms(m, s);
   if (threadIdx.x == 0) part[rw * p.nvch + c] = tot;
@@ -277,7 +301,7 @@ __global__ void __launch_bounds__(kSampThreads) spec_norm_kernel(const SamplePar
     double Z = 0.0;
     for (int q = 0; q < p.nvch; ++q) {
       const float mq = __ldcg(&pr[q].m);
-      if (mq != -INFINITY) Z += __ldcg(&pr[q].s) * exp((double)mq - (double)M);
+      if (mq != -INFINITY) Z += __ldcg(&pr[q].s) * (double)exp2f((mq - M) * kLog2e);
     }
     sM[threadIdx.x] = M;
     sZ[threadIdx.x] = Z;
@@ -336,23 +360,26 @@ __global__ void __launch_bounds__(kSampThreads) spec_draw_kernel(const SamplePar
   const float* qrow = p.q_logits + ((size_t)r * k + (pl.type == 0 ? pl.row : 0)) * V;
   double2* part = reinterpret_cast<double2*>(p.part + p.draw_off) + (size_t)r * p.nvch;
   const bool resid = pl.type == 0;
-  auto w_p = [&](int v) -> double {
+  const float mpb = pl.mp * kLog2e, mqb = pl.mq * kLog2e;
+  const float izp = (float)(1.0 / pl.zp), izq = (float)(1.0 / pl.zq);
+  auto w_p = [&](int v) -> float {
     const float x = prow[v];
-    return isfinite(x) ? (double)expf(x - pl.mp) : 0.0;
+    return (isnan(x) || x == INFINITY) ? 0.f : ex2(fmaf(x, kLog2e, -mpb));
   };
-  auto w_res = [&](int v) -> double {
+  auto w_res = [&](int v) -> float {
     const float x = prow[v], y = qrow[v];
-    const double pv = isfinite(x) ? (double)expf(x - pl.mp) / pl.zp : 0.0;
-    const double qv = isfinite(y) ? (double)expf(y - pl.mq) / pl.zq : 0.0;
-    return pv > qv ? pv - qv : 0.0;
+    const float pv = (isnan(x) || x == INFINITY) ? 0.f : ex2(fmaf(x, kLog2e, -mpb)) * izp;
+    const float qv = (isnan(y) || y == INFINITY) ? 0.f : ex2(fmaf(y, kLog2e, -mqb)) * izq;
+    return fmaxf(pv - qv, 0.f);
   };
 
   const int v0 = c * kVocabChunk, v1 = min(V, (c + 1) * kVocabChunk);
-  double sr = 0.0, sp = 0.0;
+  float srf = 0.f, spf = 0.f;
   for (int v = v0 + threadIdx.x; v < v1; v += blockDim.x) {
-    sp += w_p(v);
-    if (resid) sr += w_res(v);
+    spf += w_p(v);
+    if (resid) srf += w_res(v);
   }
+  double sr = srf, sp = spf;
   sp = block_sum_d(sp);
   sr = block_sum_d(sr);
   if (threadIdx.x == 0) part[c] = make_double2(sr, sp);

@@ -90,9 +90,23 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const SelectPara
   for (int j = tid; j < N; j += blockDim.x) {
     float sigma;
     if (p.logits) {
-      const float* lg = p.logits + ((size_t)r * p.Hkv + kvh) * (size_t)p.R * p.cap + j;
+      // the G*(k+1) logits of position j are contiguous: [..][cap][R]
+      const float* lg = p.logits + (((size_t)r * p.Hkv + kvh) * p.cap + j) * p.R;
       float acc = 0.f;
-      for (int row = 0; row < p.R; ++row) acc += expf(__ldg(lg + (size_t)row * p.cap) - lse_s[row]);
+      if ((p.R & 3) == 0) {
+        for (int row = 0; row < p.R; row += 4) {
+          const float4 x = __ldg(reinterpret_cast<const float4*>(lg + row));
+          acc += expf(x.x - lse_s[row]) + expf(x.y - lse_s[row + 1]) +
+                 expf(x.z - lse_s[row + 2]) + expf(x.w - lse_s[row + 3]);
+        }
+      } else if ((p.R & 1) == 0) {
+        for (int row = 0; row < p.R; row += 2) {
+          const float2 x = __ldg(reinterpret_cast<const float2*>(lg + row));
+          acc += expf(x.x - lse_s[row]) + expf(x.y - lse_s[row + 1]);
+        }
+      } else {
+        for (int row = 0; row < p.R; ++row) acc += expf(__ldg(lg + row) - lse_s[row]);
+      }
       sigma = acc;
     } else {
       sigma = p.scores[((size_t)r * p.Hkv + kvh) * p.score_stride + j];

@@ -136,7 +136,7 @@ __global__ void __launch_bounds__(MAXT) verify_kernel(const __grid_constant__ CU
 
   float* scores = p.scores;
   const int R = p.R;
-  const size_t score_base = ((size_t)r * Hkv + kvh) * (size_t)R * p.cap;
+  const size_t score_base = ((size_t)r * Hkv + kvh) * (size_t)p.cap * R;
   bool timed_out = false;
 
   for (int it = 0; it < ntiles; ++it) {
@@ -175,19 +175,28 @@ __global__ void __launch_bounds__(MAXT) verify_kernel(const __grid_constant__ CU
 
     const int row0 = slice * 16;
     if (t0 + row0 < end) {
-      wa.step(
-          kb, vb, row0, lane, p.scale,
-          [&](int tr, int nt, int j) -> bool {
-            const int pos = t0 + tr;
-            const int row = grp * RW + nt * 8 + 2 * (lane & 3) + j;
-            return pos < end && (pos < L || pos - L <= row / G);
-          },
-          [&](int tr, int nt, int j, float logit) {
-            const int pos = t0 + tr;
-            const int row = grp * RW + nt * 8 + 2 * (lane & 3) + j;
-            if (scores && row < R && pos < L && pos < end)
-              scores[score_base + (size_t)row * p.cap + pos] = logit;
-          });
+      auto vis = [&](int tr, int nt, int j) -> bool {
+        const int pos = t0 + tr;
+        const int row = grp * RW + nt * 8 + 2 * (lane & 3) + j;
+        return pos < end && (pos < L || pos - L <= row / G);
+      };
+      auto cap_fn = [&](int tr, int nt, float lg0, float lg1) {
+        const int pos = t0 + tr;
+        const int row = grp * RW + nt * 8 + 2 * (lane & 3);
+        if (scores && row < R && pos < L) {
+          float* dst = scores + score_base + (size_t)pos * R + row;
+          if (!(R & 1)) {
+            *reinterpret_cast<float2*>(dst) = make_float2(lg0, lg1);
+          } else {
+            dst[0] = lg0;
+            if (row + 1 < R) dst[1] = lg1;
+          }
+        }
+      };
+      if (t0 + kTile <= L && t0 + kTile <= end)
+        wa.template step<false>(kb, vb, row0, lane, p.scale, vis, cap_fn);
+      else
+        wa.template step<true>(kb, vb, row0, lane, p.scale, vis, cap_fn);
     }
     if (__syncthreads_or(timed_out)) {
       if (tid == 0) set_error(p.err, S3R_ERR_TIMEOUT);
@@ -211,8 +220,9 @@ __global__ void __launch_bounds__(MAXT) verify_kernel(const __grid_constant__ CU
   merge_slices_to_record<D, RW>(redO, redM, redL, nwarps / 4, recs + c * rec_floats, p.Rp);
 
   if (!last_of(p.tickets + (size_t)r * Hkv + kvh, nch, s_flag)) return;
+  __shared__ float wts[32 * S3R_MAX_ROWS];
   combine_records<D>(
-      recs, rec_floats, nch, R, p.Rp,
+      recs, rec_floats, nch, R, p.Rp, wts,
       [&](int row) {
         const int t = row / G, g = row - t * G;
         return p.out + (((size_t)r * T + t) * p.Hq + kvh * G + g) * D;
@@ -220,7 +230,8 @@ __global__ void __launch_bounds__(MAXT) verify_kernel(const __grid_constant__ CU
       [&](int row) -> float* {
         const int t = row / G, g = row - t * G;
         return p.lse + ((size_t)r * T + t) * p.Hq + kvh * G + g;
-      });
+      },
+      tid, blockDim.x);
 }
 
 template <int D, int MAXT>

@@ -27,7 +27,7 @@ class RoundBuffers:
                  sel_stride, device="cuda"):
         G = num_q_heads // num_kv_heads
         f32, bf, i32 = torch.float32, torch.bfloat16, torch.int32
-        self.scores = torch.empty((num_requests, num_kv_heads, G * (k + 1), cap), dtype=f32, device=device)
+        self.scores = torch.empty((num_requests, num_kv_heads, cap, G * (k + 1)), dtype=f32, device=device)
         self.lse = torch.empty((num_requests, k + 1, num_q_heads), dtype=f32, device=device)
         self.prefill_lse = torch.empty((num_requests, 1, num_q_heads), dtype=f32, device=device)
         self.sel_idx = torch.zeros((num_requests, num_kv_heads, sel_stride), dtype=i32, device=device)

@@ -22,7 +22,7 @@ def run_verify(case, k, seed, scores=True):
     lse = torch.empty((NR, T, Hq), dtype=torch.float32, device="cuda")
     cap = case.cache.capacity
     G = Hq // Hkv
-    sc = torch.full((NR, Hkv, G * T, cap), float("nan"), device="cuda") if scores else None
+    sc = torch.full((NR, Hkv, cap, G * T), float("nan"), device="cuda") if scores else None
     cache = s3r.make_cache(case.k_pool, case.v_pool, Hq)
     batch = s3r.make_batch(case.seq_lens, case.page_table)
     ws = s3r.new_workspace(s3r.s3r_workspace_size(cache, NR, case.cache.max_pages, k, 64, 64))
@@ -52,8 +52,8 @@ def test_verify_matches_oracle(Hq, Hkv, d, k, lens):
         o, l, sigma, logits = O.verify_attention(f64(q[r]), K, V, int(L))
         assert_attention_close(f64(out[r]), o, f"out r={r}")
         np.testing.assert_allclose(f64(lse[r]), l, rtol=0, atol=2e-4)
-        got = f64(sc[r][:, :, :L])
-        np.testing.assert_allclose(got, logits[:, :, :L], rtol=1e-5, atol=1e-4)
+        got = f64(sc[r][:, :L, :])                      # [H_kv][position][row]
+        np.testing.assert_allclose(got, logits[:, :, :L].transpose(0, 2, 1), rtol=1e-5, atol=1e-4)
 
 
 def test_verify_without_score_capture_and_full_capacity():
