@@ -208,6 +208,12 @@ S3R_API const char* s3r_status_string(int status);
 /* Number of kernels this library has launched in the process (all calls, all streams). */
 S3R_API uint64_t s3r_launch_count(void);
 
+/* Choose the kernel behind s3r_verify_attn for later calls (process-wide): 0 = automatic
+ * (the tcgen05 tensor-memory kernel for head_dim 128 with G*(k+1) <= 32 and <= 2048
+ * requests, otherwise the mma.sync kernel), 1 = always the mma.sync kernel. Both compute
+ * the same function. */
+S3R_API int s3r_set_verify_kernel(int32_t which);
+
 /* Text of the CUDA error behind the last S3R_ERR_CUDA status returned on this thread
  * ("" if none). */
 S3R_API const char* s3r_last_error_message(void);

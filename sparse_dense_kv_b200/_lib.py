@@ -66,6 +66,7 @@ def _load():
         "s3r_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "s3r_launch_count": (U64, []),
         "s3r_last_error_message": (ctypes.c_char_p, []),
+        "s3r_set_verify_kernel": (ctypes.c_int, [I32]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -256,6 +257,11 @@ def s3r_get_error(ws, stream=None) -> int:
 
 def s3r_status_string(status: int) -> str:
     return _lib.s3r_status_string(status).decode()
+
+
+def s3r_set_verify_kernel(which: int):
+    """0: automatic (tcgen05 kernel where supported), 1: mma.sync kernel."""
+    _check(_lib.s3r_set_verify_kernel(which), "s3r_set_verify_kernel")
 
 
 def s3r_launch_count() -> int:

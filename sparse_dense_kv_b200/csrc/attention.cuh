@@ -215,66 +215,71 @@ __device__ __forceinline__ void merge_slices_to_record(const float* redO, const 
 
 // Combine `nch` chunk records of `R` rows into normalised outputs: for row < R and d < D,
 // out = sum_c O_c exp2(m_c - M) / sum_c l_c exp2(m_c - M); lse (natural) per row.
-// The per-(chunk, row) weights are formed once in shared memory (`wts`, >= 32*R floats),
-// then every thread sums 4 consecutive d of one row over the chunks with 16-byte loads
-// (R * D / 4 <= 4 * nthreads: R <= 16 rows per 128 threads).
-template <int D, class OutPtr, class LsePtr>
-__device__ __forceinline__ void combine_records(const float* recs, size_t rec_floats, int nch,
-                                                int R, int Rp, float* wts, OutPtr out_row,
-                                                LsePtr lse_row, int tid, int nthreads) {
-  float4 acc[4];
-  const int nvec = R * (D / 4);
-  for (int c0 = 0; c0 < nch; c0 += 32) {
-    const int cn = min(32, nch - c0);
-    // weights of this batch of chunks, relative to the max over all chunks
-    for (int row = tid; row < R; row += nthreads) {
-      float M = -INFINITY;
-      for (int c = 0; c < nch; ++c) M = fmaxf(M, __ldcg(recs + c * rec_floats + row));
-      float lsum = 0.f;
+// Per-(chunk, row) weights go to shared memory (`wts`, capacity `wcap` floats) when they fit;
+// otherwise each weight is recomputed from the record. Every thread then sums 4 consecutive
+// d of one row over the chunks with 16-byte loads and writes them as bf16.
+template <int D, class OutPtr, class LsePtr, class Sync>
+__device__ __forceinline__ void combine_records_sync(const float* recs, size_t rec_floats,
+                                                     int nch, int R, int Rp, float* wts, int wcap,
+                                                     OutPtr out_row, LsePtr lse_row, int tid,
+                                                     int nthreads, Sync sync) {
+  float* Ms = wts;            // [R] row max
+  float* iLs = wts + R;       // [R] 1 / row sum
+  float* W = wts + 2 * R;     // [nch][R] weights, if they fit
+  const bool table = (size_t)(2 + nch) * R <= (size_t)wcap;
+  for (int row = tid; row < R; row += nthreads) {
+    float M = -INFINITY;
+    for (int c = 0; c < nch; ++c) M = fmaxf(M, __ldcg(recs + c * rec_floats + row));
+    float lsum = 0.f;
+    for (int c = 0; c < nch; ++c) {
+      const float mc = __ldcg(recs + c * rec_floats + row);
+      lsum += (mc == -INFINITY) ? 0.f : exp2f(mc - M) * __ldcg(recs + c * rec_floats + Rp + row);
+    }
+    Ms[row] = M;
+    iLs[row] = 1.f / lsum;
+    if (table)
       for (int c = 0; c < nch; ++c) {
         const float mc = __ldcg(recs + c * rec_floats + row);
-        lsum += (mc == -INFINITY) ? 0.f : exp2f(mc - M) * __ldcg(recs + c * rec_floats + Rp + row);
+        W[c * R + row] = (mc == -INFINITY) ? 0.f : exp2f(mc - M) / lsum;
       }
-      for (int c = 0; c < cn; ++c) {
-        const float mc = __ldcg(recs + (c0 + c) * rec_floats + row);
-        wts[c * R + row] = (mc == -INFINITY) ? 0.f : exp2f(mc - M) / lsum;
-      }
-      if (c0 == 0 && tid < R) {
-        float* lp = lse_row(row);
-        if (lp) *lp = (M + log2f(lsum)) * kLn2;
-      }
-    }
-    __syncthreads();
-#pragma unroll
-    for (int slot = 0; slot < 4; ++slot) {
-      const int v = tid + slot * nthreads;
-      if (v >= nvec) break;
-      const int row = v / (D / 4), d4 = v - row * (D / 4);
-      float4 a = (c0 == 0) ? make_float4(0.f, 0.f, 0.f, 0.f) : acc[slot];
-#pragma unroll 4
-      for (int c = 0; c < cn; ++c) {
-        const float w = wts[c * R + row];
-        const float4 x = __ldcg(reinterpret_cast<const float4*>(
-            recs + (c0 + c) * rec_floats + 2 * Rp + (size_t)row * D) + d4);
-        a.x += w * x.x;
-        a.y += w * x.y;
-        a.z += w * x.z;
-        a.w += w * x.w;
-      }
-      acc[slot] = a;
-    }
-    __syncthreads();
+    float* lp = lse_row(row);
+    if (lp) *lp = (M + log2f(lsum)) * kLn2;
   }
-#pragma unroll
-  for (int slot = 0; slot < 4; ++slot) {
-    const int v = tid + slot * nthreads;
-    if (v >= nvec) break;
+  sync();
+  const int nvec = R * (D / 4);
+  for (int v = tid; v < nvec; v += nthreads) {
     const int row = v / (D / 4), d4 = v - row * (D / 4);
-    const float4 a = acc[slot];
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int c = 0; c < nch; ++c) {
+      float w;
+      if (table) {
+        w = W[c * R + row];
+      } else {
+        const float mc = __ldcg(recs + c * rec_floats + row);
+        w = (mc == -INFINITY) ? 0.f : exp2f(mc - Ms[row]) * iLs[row];
+      }
+      const float4 x = __ldcg(reinterpret_cast<const float4*>(
+          recs + c * rec_floats + 2 * Rp + (size_t)row * D) + d4);
+      a.x += w * x.x;
+      a.y += w * x.y;
+      a.z += w * x.z;
+      a.w += w * x.w;
+    }
     __nv_bfloat162* o = reinterpret_cast<__nv_bfloat162*>(out_row(row) + d4 * 4);
     o[0] = __floats2bfloat162_rn(a.x, a.y);
     o[1] = __floats2bfloat162_rn(a.z, a.w);
   }
+}
+
+// combine_records_sync for a whole CTA (block-wide barriers).
+template <int D, class OutPtr, class LsePtr>
+__device__ __forceinline__ void combine_records(const float* recs, size_t rec_floats, int nch,
+                                                int R, int Rp, float* wts, int wcap,
+                                                OutPtr out_row, LsePtr lse_row, int tid,
+                                                int nthreads) {
+  combine_records_sync<D>(recs, rec_floats, nch, R, Rp, wts, wcap, out_row, lse_row, tid,
+                          nthreads, [] { __syncthreads(); });
 }
 
 }  // namespace s3r

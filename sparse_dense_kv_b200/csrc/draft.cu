@@ -160,7 +160,7 @@ __global__ void __launch_bounds__(128) draft_kernel(const DraftParams p) {
   if (!last_of(p.tickets + (size_t)r * Hkv + kvh, nch, s_flag)) return;
   __shared__ float wts[32 * RW];
   combine_records<D>(
-      recs, rec_floats, nch, G, RW, wts,
+      recs, rec_floats, nch, G, RW, wts, 32 * RW,
       [&](int row) { return p.out + ((size_t)r * p.Hq + kvh * G + row) * D; },
       [&](int row) -> float* {
         return p.lse ? p.lse + (size_t)r * p.Hq + kvh * G + row : nullptr;

@@ -105,6 +105,14 @@ int cuda_status(cudaError_t e, const char* where);
 int launch_verify(const CUtensorMap& tk, const CUtensorMap& tv, const VerifyParams& p, int D,
                   int batch, cudaStream_t stream);
 size_t verify_partial_bytes(int num_requests, int Hkv, int cap, int R, int D, int chunk);
+int launch_verify_combine(const VerifyParams& p, int D, int batch, cudaStream_t stream);
+
+// tcgen05 verify (head_dim 128, G*(k+1) <= 32 rows, <= 2048 requests per launch)
+bool verify_tc_supported(int D, int R, int batch);
+int verify_tc_npad(int R);
+int verify_tc_chunk();
+int launch_verify_tc(const CUtensorMap& tk, const CUtensorMap& tv, const VerifyParams& p,
+                     int batch, int num_sms, cudaStream_t stream);
 
 int launch_draft(const DraftParams& p, int D, int batch, cudaStream_t stream);
 size_t draft_partial_bytes(int num_requests, int Hkv, int sel_stride, int D);

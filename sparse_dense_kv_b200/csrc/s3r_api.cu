@@ -24,6 +24,15 @@ int cuda_status(cudaError_t e, const char* where) {
 namespace {
 
 std::atomic<uint64_t> g_launches{0};
+std::atomic<int> g_verify_kernel{0};   // 0 auto, 1 CUDA-core mma.sync kernel
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    return 148;
+  return n;
+}
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
@@ -227,7 +236,18 @@ int s3r_verify_attn(const s3r_kv_cache* cache, const s3r_batch* batch, int32_t k
   p.err = w.err;
   p.tickets = w.tickets;
   p.part = reinterpret_cast<float*>(w.part);
-  return finish(launch_verify(tk, tv, p, cache->head_dim, batch->batch, (cudaStream_t)stream), 1);
+  int st;
+  if (g_verify_kernel.load() == 0 && verify_tc_supported(cache->head_dim, R, batch->batch)) {
+    p.Rp = verify_tc_npad(R);
+    p.chunk = verify_tc_chunk();
+    p.nchunk_max = (cap + p.chunk - 1) / p.chunk;
+    st = launch_verify_tc(tk, tv, p, batch->batch, sm_count(), (cudaStream_t)stream);
+  } else {
+    st = launch_verify(tk, tv, p, cache->head_dim, batch->batch, (cudaStream_t)stream);
+  }
+  if (st != S3R_OK) return st;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return finish(launch_verify_combine(p, cache->head_dim, batch->batch, (cudaStream_t)stream), 1);
 }
 
 static int select_common(const s3r_kv_cache* cache, const s3r_batch* batch, SelectParams& p,
@@ -466,5 +486,11 @@ const char* s3r_status_string(int status) {
 uint64_t s3r_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 const char* s3r_last_error_message(void) { return g_last_error; }
+
+int s3r_set_verify_kernel(int32_t which) {
+  if (which < 0 || which > 1) return S3R_ERR_INVALID_ARG;
+  g_verify_kernel.store(which);
+  return S3R_OK;
+}
 
 }  // extern "C"

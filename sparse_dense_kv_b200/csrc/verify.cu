@@ -11,8 +11,8 @@
 // 64-column half, 128-byte swizzle) into a 3-stage mbarrier pipeline; the block's own K/V
 // (positions >= L) are patched into the tile from the caller's k_new / v_new. Warp
 // (group, slice) computes 16 rows x 16 positions per tile on the tensor cores. Chunk
-// results go to the workspace; the last CTA of the (request, head) merges them in chunk
-// order (deterministic) and writes out / lse.
+// results go to the workspace; verify_combine_kernel merges them in chunk order
+// (deterministic) and writes out / lse.
 #include "attention.cuh"
 #include "kernels.h"
 
@@ -32,8 +32,6 @@ __global__ void __launch_bounds__(MAXT) verify_kernel(const __grid_constant__ CU
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) &
                                              ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kVerifyStages * STAGE);
-  __shared__ int s_flag_mem;
-  int* s_flag = &s_flag_mem;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int grp = warp >> 2, slice = warp & 3;
@@ -48,7 +46,6 @@ __global__ void __launch_bounds__(MAXT) verify_kernel(const __grid_constant__ CU
   const int start = c * p.chunk;
   if (start >= Lc) return;
   const int end = min(start + p.chunk, Lc);
-  const int nch = (Lc + p.chunk - 1) / p.chunk;
   const int* ptab = p.page_table + (size_t)r * p.max_pages;
   const int64_t npages = p.num_pages;
   const int Hkv = p.Hkv;
@@ -219,19 +216,117 @@ __global__ void __launch_bounds__(MAXT) verify_kernel(const __grid_constant__ CU
   float* recs = p.part + ((size_t)r * Hkv + kvh) * p.nchunk_max * rec_floats;
   merge_slices_to_record<D, RW>(redO, redM, redL, nwarps / 4, recs + c * rec_floats, p.Rp);
 
-  if (!last_of(p.tickets + (size_t)r * Hkv + kvh, nch, s_flag)) return;
-  __shared__ float wts[32 * S3R_MAX_ROWS];
-  combine_records<D>(
-      recs, rec_floats, nch, R, p.Rp, wts,
-      [&](int row) {
-        const int t = row / G, g = row - t * G;
-        return p.out + (((size_t)r * T + t) * p.Hq + kvh * G + g) * D;
-      },
-      [&](int row) -> float* {
-        const int t = row / G, g = row - t * G;
-        return p.lse + ((size_t)r * T + t) * p.Hq + kvh * G + g;
-      },
-      tid, blockDim.x);
+}
+
+// Merge the chunk records of every (request, KV head) of a verify launch into out / lse:
+// one CTA per (KV head, request), weights from all chunk maxima / sums, then 16-byte loads
+// of the chunk outputs with several independent accumulators per thread.
+template <int D>
+__global__ void __launch_bounds__(256) verify_combine_kernel(const VerifyParams p) {
+  extern __shared__ float cw[];   // [nchunk_max][R] m, then l, then weights
+  const int kvh = blockIdx.x, bl = blockIdx.y;
+  const int r = p.req_ids ? p.req_ids[bl] : bl;
+  const int L = p.seq_lens[r];
+  const int T = p.T, G = p.G, R = p.R, Rp = p.Rp, Lc = L + T;
+  if (L < 0 || Lc > p.cap) return;   // reported by the attention kernel
+  const int nch = (Lc + p.chunk - 1) / p.chunk;
+  const size_t rec_floats = (size_t)Rp * (D + 2);
+  const float* recs = p.part + ((size_t)r * p.Hkv + kvh) * p.nchunk_max * rec_floats;
+  float* mm = cw;
+  float* ll = cw + (size_t)nch * R;
+  float* ww = ll + (size_t)nch * R;
+  float* Ms = ww + (size_t)nch * R;
+  for (int i = threadIdx.x; i < nch * R; i += blockDim.x) {
+    const int c = i / R, row = i - c * R;
+    mm[i] = __ldcg(recs + c * rec_floats + row);
+    ll[i] = __ldcg(recs + c * rec_floats + Rp + row);
+  }
+  __syncthreads();
+  for (int row = threadIdx.x; row < R; row += blockDim.x) {
+    float M = -INFINITY;
+    for (int c = 0; c < nch; ++c) M = fmaxf(M, mm[c * R + row]);
+    float lsum = 0.f;
+    for (int c = 0; c < nch; ++c) {
+      const float mc = mm[c * R + row];
+      lsum += (mc == -INFINITY) ? 0.f : exp2f(mc - M) * ll[c * R + row];
+    }
+    const float inv = 1.f / lsum;
+    for (int c = 0; c < nch; ++c) {
+      const float mc = mm[c * R + row];
+      ww[c * R + row] = (mc == -INFINITY) ? 0.f : exp2f(mc - M) * inv;
+    }
+    const int t = row / G, g = row - t * G;
+    p.lse[((size_t)r * T + t) * p.Hq + kvh * G + g] = (M + log2f(lsum)) * kLn2;
+    Ms[row] = M;
+  }
+  __syncthreads();
+  constexpr int kV = 4;   // (row, 4 d) items per thread per pass
+  const int nvec = R * (D / 4);
+  for (int v0 = threadIdx.x; v0 < nvec; v0 += kV * blockDim.x) {
+    float4 acc[kV];
+    int rows[kV];
+#pragma unroll
+    for (int s = 0; s < kV; ++s) {
+      acc[s] = make_float4(0.f, 0.f, 0.f, 0.f);
+      const int v = v0 + s * blockDim.x;
+      rows[s] = v < nvec ? v / (D / 4) : 0;
+    }
+    for (int c = 0; c < nch; ++c) {
+      const float* oc = recs + c * rec_floats + 2 * Rp;
+#pragma unroll
+      for (int s = 0; s < kV; ++s) {
+        const int v = v0 + s * blockDim.x;
+        if (v < nvec) {
+          const float w = ww[c * R + rows[s]];
+          const float4 x = __ldcg(reinterpret_cast<const float4*>(oc) + v);
+          acc[s].x += w * x.x;
+          acc[s].y += w * x.y;
+          acc[s].z += w * x.z;
+          acc[s].w += w * x.w;
+        }
+      }
+    }
+#pragma unroll
+    for (int s = 0; s < kV; ++s) {
+      const int v = v0 + s * blockDim.x;
+      if (v >= nvec) continue;
+      const int row = rows[s], d4 = v - row * (D / 4);
+      const int t = row / G, g = row - t * G;
+      __nv_bfloat162* o = reinterpret_cast<__nv_bfloat162*>(
+          p.out + (((size_t)r * T + t) * p.Hq + kvh * G + g) * D + d4 * 4);
+      o[0] = __floats2bfloat162_rn(acc[s].x, acc[s].y);
+      o[1] = __floats2bfloat162_rn(acc[s].z, acc[s].w);
+    }
+  }
+  (void)Ms;
+}
+
+int launch_verify_combine(const VerifyParams& p, int D, int batch, cudaStream_t stream) {
+  const size_t smem = ((size_t)3 * p.nchunk_max * p.R + p.R) * 4;
+  if (smem > 200 * 1024) return S3R_ERR_UNSUPPORTED;
+  dim3 grid(p.Hkv, batch);
+  if (D == 128) {
+    static size_t attr = 0;
+    if (smem > 48 * 1024 && smem > attr) {
+      if (cuda_status(cudaFuncSetAttribute(verify_combine_kernel<128>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem),
+                      "cudaFuncSetAttribute") != S3R_OK)
+        return S3R_ERR_CUDA;
+      attr = smem;
+    }
+    verify_combine_kernel<128><<<grid, 256, smem, stream>>>(p);
+  } else {
+    static size_t attr = 0;
+    if (smem > 48 * 1024 && smem > attr) {
+      if (cuda_status(cudaFuncSetAttribute(verify_combine_kernel<64>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem),
+                      "cudaFuncSetAttribute") != S3R_OK)
+        return S3R_ERR_CUDA;
+      attr = smem;
+    }
+    verify_combine_kernel<64><<<grid, 256, smem, stream>>>(p);
+  }
+  return cuda_status(cudaGetLastError(), __func__);
 }
 
 template <int D, int MAXT>

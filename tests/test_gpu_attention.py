@@ -56,6 +56,36 @@ def test_verify_matches_oracle(Hq, Hkv, d, k, lens):
         np.testing.assert_allclose(got, logits[:, :, :L].transpose(0, 2, 1), rtol=1e-5, atol=1e-4)
 
 
+@pytest.mark.parametrize("Hq,Hkv,k,lens", [
+    (32, 8, 6, [2500, 1025, 4000]),     # 28 rows
+    (16, 8, 6, [3000, 900]),            # 14 rows
+    (32, 8, 0, [1200, 2100]),           # 4 rows (prefill pass)
+])
+def test_verify_kernels_agree_with_oracle(Hq, Hkv, k, lens):
+    """The tcgen05 tensor-memory kernel and the mma.sync kernel on the same case."""
+    spec = spec_for(Hq, Hkv, 128, lens, k=k, seed=17)
+    outs = []
+    for which in (1, 0):
+        case = Case(spec, extra_tokens=k + 1 + 20)
+        s3r.s3r_set_verify_kernel(which)
+        try:
+            q, kn, vn, out, lse, sc = run_verify(case, k, seed=300)
+        finally:
+            s3r.s3r_set_verify_kernel(0)
+        outs.append((out, lse, sc))
+        kp, vp = case.host_pools()
+        for r, L in enumerate(case.lens):
+            K, V = case.dense(r, L + k + 1, (kp, vp))
+            o, l, _, logits = O.verify_attention(f64(q[r]), K, V, int(L))
+            assert_attention_close(f64(out[r]), o, f"kernel {which} out r={r}")
+            np.testing.assert_allclose(f64(lse[r]), l, rtol=0, atol=2e-4)
+            np.testing.assert_allclose(f64(sc[r][:, :L, :]), logits[:, :, :L].transpose(0, 2, 1),
+                                       rtol=1e-5, atol=1e-4)
+    (o1, l1, s1), (o0, l0, s0) = outs
+    assert (o1.float() - o0.float()).abs().max().item() < 2e-2
+    assert (l1 - l0).abs().max().item() < 1e-3
+
+
 def test_verify_without_score_capture_and_full_capacity():
     k = 6
     spec = spec_for(32, 8, 128, [1017, 64], k=k, seed=3)
