@@ -9,6 +9,7 @@
 namespace s3r {
 
 constexpr int kVerifyChunk = 1024;   // positions per verify CTA (multiple of 64)
+constexpr int kVerifyChunkMin = 896; // smallest verify chunk of any kernel (workspace sizing)
 constexpr int kDraftChunk = 256;     // positions per draft CTA (multiple of 64)
 constexpr int kVocabChunk = 8192;    // vocabulary entries per sampler CTA
 
@@ -110,7 +111,7 @@ int launch_verify_combine(const VerifyParams& p, int D, int batch, cudaStream_t 
 // tcgen05 verify (head_dim 128, G*(k+1) <= 32 rows, <= 2048 requests per launch)
 bool verify_tc_supported(int D, int R, int batch);
 int verify_tc_npad(int R);
-int verify_tc_chunk();
+int verify_tc_chunk(int R);
 int launch_verify_tc(const CUtensorMap& tk, const CUtensorMap& tv, const VerifyParams& p,
                      int batch, int num_sms, cudaStream_t stream);
 

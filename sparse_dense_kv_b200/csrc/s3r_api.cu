@@ -143,7 +143,7 @@ size_t verify_need(const s3r_kv_cache* c, int num_requests, int cap, int k) {
   const int G = c->num_q_heads / c->num_kv_heads;
   return head_bytes(num_requests) +
          verify_partial_bytes(num_requests, c->num_kv_heads, cap, G * (k + 1), c->head_dim,
-                              kVerifyChunk);
+                              kVerifyChunkMin);
 }
 
 size_t draft_need(const s3r_kv_cache* c, int num_requests, int sel_stride) {
@@ -239,7 +239,7 @@ int s3r_verify_attn(const s3r_kv_cache* cache, const s3r_batch* batch, int32_t k
   int st;
   if (g_verify_kernel.load() == 0 && verify_tc_supported(cache->head_dim, R, batch->batch)) {
     p.Rp = verify_tc_npad(R);
-    p.chunk = verify_tc_chunk();
+    p.chunk = verify_tc_chunk(R);
     p.nchunk_max = (cap + p.chunk - 1) / p.chunk;
     st = launch_verify_tc(tk, tv, p, batch->batch, sm_count(), (cudaStream_t)stream);
   } else {

@@ -34,9 +34,8 @@ namespace tc {
 constexpr int kPos = 128;                   // positions per tile (MMA M)
 constexpr int kD = 128;                     // head_dim of this path
 constexpr int kStages = 4;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;          // producer, MMA, 8 softmax warps
 constexpr int kTileBytes = kPos * kD * 2;   // 32 KB: [2 halves][128 rows][128 B]
-constexpr int kMaxTiles = 8;                // tiles per chunk
 constexpr int kMaxBatch = 2048;             // requests per launch on this path
 
 // --------------------------------------------------------------- tcgen05 wrappers -------
@@ -115,31 +114,36 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool 
 
 template <int NP>
 struct Cfg {
-  static constexpr int kTiles = kMaxTiles;                   // tiles per chunk
+  static constexpr int kTiles = NP == 32 ? 7 : 8;            // tiles per chunk
   static constexpr int kChunk = kTiles * kPos;
   static constexpr int kQBytes = 2 * NP * 128;               // [2 halves][NP rows][128 B]
   static constexpr int kPTile = kPos * NP * 2;               // P^T tile: [128 pos][NP rows] bf16
-  static constexpr uint32_t kPSwz = NP == 16 ? 6u : 4u;      // 32- / 64-byte swizzle
   static constexpr int kPBytes = kTiles * kPTile;
+  static constexpr uint32_t kPSwz = NP == 16 ? 6u : 4u;      // 32- / 64-byte swizzle
   static constexpr int kTmemCols = 512;
-  static constexpr int kOCol = kTiles * NP;                  // O^T columns
-  static_assert(kOCol + NP <= kTmemCols, "tensor memory budget");
+  static constexpr int kSCols = kTiles * NP;                 // one S buffer
+  static constexpr int kOCol = 2 * kSCols;                   // two O buffers after two S buffers
+  static_assert(kOCol + 2 * NP <= kTmemCols, "tensor memory budget");
   static constexpr int kRingOff = 0;
   static constexpr int kQOff = kStages * kTileBytes;
   static constexpr int kPOff = kQOff + kQBytes;
-  static constexpr int kRedOff = kPOff + kPBytes;            // [4 warps][NP] floats x 2
-  static constexpr int kPrefOff = kRedOff + 2 * 4 * NP * 4;  // request prefix [kMaxBatch+1]
+  static constexpr int kRedOff = kPOff + kPBytes;            // redM, redL [8 warps][NP]; cm, cl [2][NP]
+  static constexpr int kRedBytes = (2 * 8 * NP + 4 * NP) * 4;
+  static constexpr int kPrefOff = kRedOff + kRedBytes;       // request prefix [kMaxBatch+1]
   static constexpr int kBarOff = (kPrefOff + (kMaxBatch + 1) * 4 + 63) / 64 * 64;
   static constexpr int kSmem = kBarOff + 256 + 1024;         // + barriers + alignment slack
 };
 
 struct Bars {
   uint64_t full[kStages], empty[kStages], tma[kStages];
-  uint64_t q_full, q_empty, s_full, s_empty, p_full, o_full, o_empty, fin;
+  // one barrier pair per tensor-memory buffer (chunk parity), so that no barrier ever runs
+  // two phases ahead of a waiter
+  uint64_t q_full, q_empty, p_full, fin;
+  uint64_t s_full[2], s_empty[2], o_full[2], o_empty[2];
   uint32_t tmem_base;
   int abort_flag;
-  int last_flag;
 };
+static_assert(sizeof(Bars) <= 256, "barrier block");
 
 // Warp-uniform bounded wait on an mbarrier phase (every lane observes the phase itself).
 // Gives up when another role raised the abort flag, or after kWaitLimit polls (then raises
@@ -165,7 +169,7 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
 }
 __device__ __forceinline__ void named_sync_softmax() {
-  asm volatile("bar.sync 1, 128;\n" ::: "memory");
+  asm volatile("bar.sync 1, 256;\n" ::: "memory");
 }
 
 // Work item i of the launch -> (launch-local request, KV head, chunk), from the prefix of
@@ -185,6 +189,24 @@ __device__ __forceinline__ void item_of(int i, const int* pref, int batch, int H
   c = rem - kvh * nch;
 }
 
+struct Item {
+  int r, kvh, c, L, Lc, start, end, ntile;
+};
+
+template <int NP>
+__device__ __forceinline__ Item make_item(int it, const int* pref, int batch, const VerifyParams& p) {
+  Item x;
+  int bl;
+  item_of(it, pref, batch, p.Hkv, bl, x.kvh, x.c);
+  x.r = p.req_ids ? p.req_ids[bl] : bl;
+  x.L = p.seq_lens[x.r];
+  x.Lc = x.L + p.T;
+  x.start = x.c * Cfg<NP>::kChunk;
+  x.end = min(x.start + Cfg<NP>::kChunk, x.Lc);
+  x.ntile = (x.end - x.start + kPos - 1) / kPos;
+  return x;
+}
+
 template <int NP>
 __global__ void __launch_bounds__(kThreads, 1)
     verify_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -194,10 +216,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) &
                                              ~uintptr_t(1023));
   int* pref = reinterpret_cast<int*>(smem + C::kPrefOff);
-  float* red = reinterpret_cast<float*>(smem + C::kRedOff);
-  __shared__ int trow[NP];   // block row t of query row j (j / G)
+  float* redM = reinterpret_cast<float*>(smem + C::kRedOff);   // [8][NP]
+  float* redL = redM + 8 * NP;                                  // [8][NP]
+  float* cm = redL + 8 * NP;                                    // [2][NP] chunk max (log2)
+  float* cl = cm + 2 * NP;                                      // [2][NP] chunk sum
   Bars* B = reinterpret_cast<Bars*>(smem + C::kBarOff);
   volatile int* abort_flag = &B->abort_flag;
+  __shared__ int trow[NP];   // block row t of query row j (j / G)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int T = p.T, G = p.G, R = p.R, Hkv = p.Hkv, Hq = p.Hq;
@@ -234,7 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (lane == 0) pref[0] = 0;
   }
-  if (tid < NP) trow[tid] = tid / p.G;
+  if (tid < NP) trow[tid] = tid / G;
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(smem_u32(&B->full[s]), 1);
@@ -243,11 +268,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(smem_u32(&B->q_full), 1);
     mbar_init(smem_u32(&B->q_empty), 1);
-    mbar_init(smem_u32(&B->s_full), 1);
-    mbar_init(smem_u32(&B->s_empty), 4);
-    mbar_init(smem_u32(&B->p_full), 4);
-    mbar_init(smem_u32(&B->o_full), 1);
-    mbar_init(smem_u32(&B->o_empty), 4);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&B->s_full[b]), 1);
+      mbar_init(smem_u32(&B->s_empty[b]), 8);
+      mbar_init(smem_u32(&B->o_full[b]), 1);
+      mbar_init(smem_u32(&B->o_empty[b]), 8);
+    }
+    mbar_init(smem_u32(&B->p_full), 8);
     mbar_init(smem_u32(&B->fin), 1);
     B->abort_flag = 0;
     fence_mbar_init();
@@ -262,152 +289,157 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = B->tmem_base;
   const int nitems = pref[batch];
+  const int my_items = nitems > (int)blockIdx.x ? (nitems - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
   const uint32_t qbuf = sbase + C::kQOff, pbuf = sbase + C::kPOff;
 
   if (warp == 0) {
     // ===================================================================== producer ====
-    int g = 0;           // ring tile counter
-    int n = 0;           // items done by this CTA
-    uint32_t tma_phase[kStages] = {0, 0, 0, 0};
-    for (int it = blockIdx.x; it < nitems && !aborted(abort_flag); it += gridDim.x, ++n) {
-      int bl, kvh, c;
-      item_of(it, pref, batch, Hkv, bl, kvh, c);
-      const int r = p.req_ids ? p.req_ids[bl] : bl;
-      const int L = p.seq_lens[r], Lc = L + T;
-      const int start = c * chunk, end = min(start + chunk, Lc);
-      const int ntile = (end - start + kPos - 1) / kPos;
-      const int* ptab = p.page_table + (size_t)r * p.max_pages;
-      // block K/V into the cache (chunk 0 of each (request, head))
-      if (c == 0) {
+    // ring order: K(0), then per item n: K(n+1), V(n) -- the MMA warp consumes in this order
+    int g = 0;
+    uint32_t tma_phase = 0;   // bit s: phase of tma[s]
+    bool stop = false;
+    auto load_tiles = [&](const Item& x, bool is_v) {
+      const CUtensorMap* map = is_v ? &tmV : &tmK;
+      const __nv_bfloat16* blk = is_v ? p.v_new : p.k_new;
+      const int* ptab = p.page_table + (size_t)x.r * p.max_pages;
+      for (int t = 0; t < x.ntile && !stop; ++t, ++g) {
+        const int s = g % kStages;
+        if (g >= kStages &&
+            !wait_bar(smem_u32(&B->empty[s]), ((g / kStages) - 1) & 1, abort_flag, p.err)) {
+          stop = true;
+          break;
+        }
+        const int t0 = x.start + t * kPos;
+        const uint32_t dst = sbase + C::kRingOff + s * kTileBytes;
+        uint32_t okmask = 0;
+        int nload = 0;
+        bool tail = (t0 + kPos > x.L);
+        int ids[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int pg = (t0 >> 4) + i;
+          ids[i] = -1;
+          if (pg * kPage < x.L) ids[i] = ptab[pg];
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int pg = (t0 >> 4) + i;
+          if (pg * kPage < x.L) {
+            if (ids[i] >= 0 && ids[i] < p.num_pages) {
+              okmask |= 1u << i;
+              ++nload;
+            } else {
+              tail = true;
+              if (lane == 0) set_error(p.err, S3R_ERR_DEVICE_BOUNDS);
+            }
+          }
+        }
+        const uint32_t landing = smem_u32(tail ? &B->tma[s] : &B->full[s]);
+        if (lane == 0) {
+          mbar_arrive_expect_tx(landing, (uint32_t)(nload * kPage * kD * 2));
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            if (!(okmask & (1u << i))) continue;
+            const int y = (int)(((int64_t)ids[i] * Hkv + x.kvh) * kPage);
+            tma_load_2d(dst + i * kPage * 128, map, 0, y, landing);
+            tma_load_2d(dst + kPos * 128 + i * kPage * 128, map, 64, y, landing);
+          }
+        }
+        if (tail) {
+          // wait for the committed rows, then write block rows / zeros over the rest
+          if (!wait_bar(smem_u32(&B->tma[s]), (tma_phase >> s) & 1, abort_flag, p.err)) {
+            stop = true;
+            break;
+          }
+          tma_phase ^= 1u << s;
+          for (int idx = lane; idx < kPos * (kD / 8); idx += 32) {
+            const int row = idx / (kD / 8), ch = idx - row * (kD / 8);
+            const int pos = t0 + row;
+            if (pos < x.L && (okmask & (1u << (row >> 4)))) continue;
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (pos >= x.L && pos < x.Lc)
+              v = *reinterpret_cast<const uint4*>(blk + (((size_t)x.r * T + (pos - x.L)) * Hkv + x.kvh) * kD + ch * 8);
+            const uint32_t off = (ch >> 3) * (kPos * 128) + row * 128 + (((ch & 7) ^ (row & 7)) << 4);
+            *reinterpret_cast<uint4*>(smem + C::kRingOff + s * kTileBytes + off) = v;
+          }
+          fence_proxy_async();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&B->full[s]));
+        }
+        __syncwarp();
+      }
+    };
+    auto load_q_and_k = [&](int m) {
+      const Item x = make_item<NP>(blockIdx.x + m * gridDim.x, pref, batch, p);
+      const int* ptab = p.page_table + (size_t)x.r * p.max_pages;
+      if (x.c == 0) {   // the block's K/V enter the cache once per (request, head)
         for (int idx = lane; idx < T * (kD / 8); idx += 32) {
           const int t = idx / (kD / 8), ch = idx - t * (kD / 8);
-          const int pos = L + t;
+          const int pos = x.L + t;
           const int page = ptab[pos >> 4];
           if (page < 0 || page >= p.num_pages) {
             set_error(p.err, S3R_ERR_DEVICE_BOUNDS);
             continue;
           }
-          const size_t dst = (((size_t)page * Hkv + kvh) * kPage + (pos & 15)) * kD + ch * 8;
-          const size_t src = (((size_t)r * T + t) * Hkv + kvh) * kD + ch * 8;
+          const size_t dst = (((size_t)page * Hkv + x.kvh) * kPage + (pos & 15)) * kD + ch * 8;
+          const size_t src = (((size_t)x.r * T + t) * Hkv + x.kvh) * kD + ch * 8;
           *reinterpret_cast<uint4*>(p.k_pool + dst) = *reinterpret_cast<const uint4*>(p.k_new + src);
           *reinterpret_cast<uint4*>(p.v_pool + dst) = *reinterpret_cast<const uint4*>(p.v_new + src);
         }
       }
-      // Q rows of this (request, head) -> qbuf, K-major, 128-byte swizzle; padding rows zero
-      if (n > 0 && !wait_bar(smem_u32(&B->q_empty), (n - 1) & 1, abort_flag, p.err)) break;
-      {
-        constexpr int kPer = NP * (kD / 8) / 32;   // 16-byte chunks per lane
-        uint4 qv[kPer];
+      // Q rows -> qbuf (K-major, 128-byte swizzle, zero padding rows), once QK(m-1) is done
+      constexpr int kPer = NP * (kD / 8) / 32;
+      uint4 qv[kPer];
 #pragma unroll
-        for (int i = 0; i < kPer; ++i) {   // all loads first, then the stores
-          const int idx = lane + 32 * i;
-          const int row = idx / (kD / 8), ch = idx - row * (kD / 8);
-          qv[i] = make_uint4(0, 0, 0, 0);
-          if (row < R) {
-            const int t = row / G, gg = row - t * G;
-            qv[i] = __ldg(reinterpret_cast<const uint4*>(p.q + (((size_t)r * T + t) * Hq + kvh * G + gg) * kD + ch * 8));
-          }
+      for (int i = 0; i < kPer; ++i) {
+        const int idx = lane + 32 * i;
+        const int row = idx / (kD / 8), ch = idx - row * (kD / 8);
+        qv[i] = make_uint4(0, 0, 0, 0);
+        if (row < R) {
+          const int t = row / G, gg = row - t * G;
+          qv[i] = __ldg(reinterpret_cast<const uint4*>(
+              p.q + (((size_t)x.r * T + t) * Hq + x.kvh * G + gg) * kD + ch * 8));
         }
+      }
+      if (m > 0 && !wait_bar(smem_u32(&B->q_empty), (m - 1) & 1, abort_flag, p.err)) {
+        stop = true;
+        return;
+      }
 #pragma unroll
-        for (int i = 0; i < kPer; ++i) {
-          const int idx = lane + 32 * i;
-          const int row = idx / (kD / 8), ch = idx - row * (kD / 8);
-          const uint32_t off = (ch >> 3) * (NP * 128) + row * 128 + (((ch & 7) ^ (row & 7)) << 4);
-          *reinterpret_cast<uint4*>(smem + C::kQOff + off) = qv[i];
-        }
+      for (int i = 0; i < kPer; ++i) {
+        const int idx = lane + 32 * i;
+        const int row = idx / (kD / 8), ch = idx - row * (kD / 8);
+        const uint32_t off = (ch >> 3) * (NP * 128) + row * 128 + (((ch & 7) ^ (row & 7)) << 4);
+        *reinterpret_cast<uint4*>(smem + C::kQOff + off) = qv[i];
       }
       fence_proxy_async();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&B->q_full));
-
-      // K tiles then V tiles of the chunk
-      bool stop = false;
-      for (int phase = 0; phase < 2 && !stop; ++phase) {
-        const CUtensorMap* map = phase ? &tmV : &tmK;
-        const __nv_bfloat16* blk = phase ? p.v_new : p.k_new;
-        for (int t = 0; t < ntile; ++t, ++g) {
-          const int s = g % kStages;
-          if (g >= kStages &&
-              !wait_bar(smem_u32(&B->empty[s]), ((g / kStages) - 1) & 1, abort_flag, p.err)) {
-            stop = true;
-            break;
-          }
-          const int t0 = start + t * kPos;
-          const uint32_t dst = sbase + C::kRingOff + s * kTileBytes;
-          // pages of committed positions that exist in the pool
-          uint32_t okmask = 0;
-          int nload = 0;
-          bool tail = (t0 + kPos > L);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int pg = (t0 >> 4) + i;
-            if (pg * kPage < L) {
-              const int id = ptab[pg];
-              if (id >= 0 && id < p.num_pages) {
-                okmask |= 1u << i;
-                ++nload;
-              } else {
-                tail = true;
-                if (lane == 0) set_error(p.err, S3R_ERR_DEVICE_BOUNDS);
-              }
-            }
-          }
-          const uint32_t landing = smem_u32(tail ? &B->tma[s] : &B->full[s]);
-          if (lane == 0) {
-            mbar_arrive_expect_tx(landing, (uint32_t)(nload * kPage * kD * 2));
-            for (int i = 0; i < 8; ++i) {
-              if (!(okmask & (1u << i))) continue;
-              const int y = (int)(((int64_t)ptab[(t0 >> 4) + i] * Hkv + kvh) * kPage);
-              tma_load_2d(dst + i * kPage * 128, map, 0, y, landing);
-              tma_load_2d(dst + kPos * 128 + i * kPage * 128, map, 64, y, landing);
-            }
-          }
-          if (tail) {
-            // wait for the committed rows, then write block rows / zeros over the rest
-            if (!wait_bar(smem_u32(&B->tma[s]), tma_phase[s], abort_flag, p.err)) {
-              stop = true;
-              break;
-            }
-            tma_phase[s] ^= 1;
-            for (int idx = lane; idx < kPos * (kD / 8); idx += 32) {
-              const int row = idx / (kD / 8), ch = idx - row * (kD / 8);
-              const int pos = t0 + row;
-              if (pos < L && (okmask & (1u << (row >> 4)))) continue;
-              uint4 v = make_uint4(0, 0, 0, 0);
-              if (pos >= L && pos < Lc)
-                v = *reinterpret_cast<const uint4*>(blk + (((size_t)r * T + (pos - L)) * Hkv + kvh) * kD + ch * 8);
-              const uint32_t off = (ch >> 3) * (kPos * 128) + row * 128 + (((ch & 7) ^ (row & 7)) << 4);
-              *reinterpret_cast<uint4*>(smem + C::kRingOff + s * kTileBytes + off) = v;
-            }
-            fence_proxy_async();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&B->full[s]));
-          }
-          __syncwarp();
-        }
-      }
+      load_tiles(x, false);
+    };
+    if (my_items > 0) load_q_and_k(0);
+    for (int n = 0; n < my_items && !stop && !aborted(abort_flag); ++n) {
+      if (n + 1 < my_items) load_q_and_k(n + 1);
       if (stop) break;
+      load_tiles(make_item<NP>(blockIdx.x + n * gridDim.x, pref, batch, p), true);
     }
   } else if (warp == 1) {
     // ====================================================================== MMA warp ===
     constexpr uint32_t kIdQK = idesc_bf16(kPos, NP, false, false);
     constexpr uint32_t kIdPV = idesc_bf16(kD, NP, true, true);
-    int g = 0, n = 0;
-    for (int it = blockIdx.x; it < nitems && !aborted(abort_flag); it += gridDim.x, ++n) {
-      int bl, kvh, c;
-      item_of(it, pref, batch, Hkv, bl, kvh, c);
-      const int r = p.req_ids ? p.req_ids[bl] : bl;
-      const int L = p.seq_lens[r], Lc = L + T;
-      const int start = c * chunk, end = min(start + chunk, Lc);
-      const int ntile = (end - start + kPos - 1) / kPos;
-      bool ok = wait_bar(smem_u32(&B->q_full), n & 1, abort_flag, p.err);
-      if (ok && n > 0) ok = wait_bar(smem_u32(&B->s_empty), (n - 1) & 1, abort_flag, p.err);
-      if (!ok) break;
+    int g = 0;
+    bool ok = true;
+    auto qk = [&](int m) {
+      const Item x = make_item<NP>(blockIdx.x + m * gridDim.x, pref, batch, p);
+      ok = wait_bar(smem_u32(&B->q_full), m & 1, abort_flag, p.err);
+      if (ok && m >= 2) ok = wait_bar(smem_u32(&B->s_empty[m & 1]), ((m - 2) >> 1) & 1, abort_flag, p.err);
+      if (!ok) return;
       tc_fence_after();
-      for (int t = 0; t < ntile && ok; ++t, ++g) {
+      const uint32_t sd = tmem + (m & 1) * C::kSCols;
+      for (int t = 0; t < x.ntile; ++t, ++g) {
         const int s = g % kStages;
         ok = wait_bar(smem_u32(&B->full[s]), (g / kStages) & 1, abort_flag, p.err);
-        if (!ok) break;
+        if (!ok) return;
         tc_fence_after();
         if (lane == 0) {
           const uint32_t kt = sbase + C::kRingOff + s * kTileBytes;
@@ -415,26 +447,29 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kk = 0; kk < kD / 16; ++kk) {
             const uint64_t ad = sdesc(kt + (kk >> 2) * (kPos * 128) + (kk & 3) * 32, 16, 1024, 2);
             const uint64_t bd = sdesc(qbuf + (kk >> 2) * (NP * 128) + (kk & 3) * 32, 16, 1024, 2);
-            tc_mma(tmem + t * NP, ad, bd, kIdQK, kk > 0 ? 1u : 0u);
+            tc_mma(sd + t * NP, ad, bd, kIdQK, kk > 0 ? 1u : 0u);
           }
           tc_commit(smem_u32(&B->empty[s]));
         }
         __syncwarp();
       }
-      if (!ok) break;
       if (lane == 0) {
-        tc_commit(smem_u32(&B->s_full));
+        tc_commit(smem_u32(&B->s_full[m & 1]));
         tc_commit(smem_u32(&B->q_empty));
       }
       __syncwarp();
+    };
+    auto pv = [&](int n) {
+      const Item x = make_item<NP>(blockIdx.x + n * gridDim.x, pref, batch, p);
       ok = wait_bar(smem_u32(&B->p_full), n & 1, abort_flag, p.err);
-      if (ok && n > 0) ok = wait_bar(smem_u32(&B->o_empty), (n - 1) & 1, abort_flag, p.err);
-      if (!ok) break;
+      if (ok && n >= 2) ok = wait_bar(smem_u32(&B->o_empty[n & 1]), ((n - 2) >> 1) & 1, abort_flag, p.err);
+      if (!ok) return;
       tc_fence_after();
-      for (int t = 0; t < ntile && ok; ++t, ++g) {
+      const uint32_t od = tmem + C::kOCol + (n & 1) * NP;
+      for (int t = 0; t < x.ntile; ++t, ++g) {
         const int s = g % kStages;
         ok = wait_bar(smem_u32(&B->full[s]), (g / kStages) & 1, abort_flag, p.err);
-        if (!ok) break;
+        if (!ok) return;
         tc_fence_after();
         if (lane == 0) {
           const uint32_t vt = sbase + C::kRingOff + s * kTileBytes;
@@ -443,15 +478,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kk = 0; kk < kPos / 16; ++kk) {
             const uint64_t ad = sdesc(vt + kk * 2048, kPos * 128, 1024, 2);
             const uint64_t bd = sdesc(pt + kk * 16 * NP * 2, NP * 2 * 8, 8 * NP * 2, C::kPSwz);
-            tc_mma(tmem + C::kOCol, ad, bd, kIdPV, (t > 0 || kk > 0) ? 1u : 0u);
+            tc_mma(od, ad, bd, kIdPV, (t > 0 || kk > 0) ? 1u : 0u);
           }
           tc_commit(smem_u32(&B->empty[s]));
         }
         __syncwarp();
       }
-      if (!ok) break;
-      if (lane == 0) tc_commit(smem_u32(&B->o_full));
+      if (lane == 0) tc_commit(smem_u32(&B->o_full[n & 1]));
       __syncwarp();
+    };
+    if (my_items > 0) qk(0);
+    for (int n = 0; n < my_items && ok && !aborted(abort_flag); ++n) {
+      if (n + 1 < my_items) qk(n + 1);
+      if (!ok) break;
+      pv(n);
     }
     // make sure nothing issued is still running before the tensor memory goes away
     if (lane == 0) tc_commit(smem_u32(&B->fin));
@@ -459,35 +499,59 @@ __global__ void __launch_bounds__(kThreads, 1)
     wait_bar(smem_u32(&B->fin), 0, abort_flag, p.err);
   } else {
     // ================================================================ softmax warps ===
+    const int sw8 = warp - 2;                // 0..7
+    const int sg = sw8 >> 2;                 // warpgroup: tiles t with t % 2 == sg
     const int q4 = warp & 3;                 // tensor-memory lane quarter of this warp
-    const int st = tid - 64;                 // 0..127 within the softmax group
+    const int st = tid - 64;                 // 0..255 within the softmax warps
     const int lrow = q4 * 32 + lane;         // tile position (S) or d (O) of this thread
     const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
     const float scale = p.scale, scale2 = p.scale * kLog2e;
-    float* redM = red;
-    float* redL = red + 4 * NP;
-    int n = 0;
-    for (int it = blockIdx.x; it < nitems && !aborted(abort_flag); it += gridDim.x, ++n) {
-      int bl, kvh, c;
-      item_of(it, pref, batch, Hkv, bl, kvh, c);
-      const int r = p.req_ids ? p.req_ids[bl] : bl;
-      const int L = p.seq_lens[r], Lc = L + T;
-      const int start = c * chunk, end = min(start + chunk, Lc);
-      const int ntile = (end - start + kPos - 1) / kPos;
-      const int nch = (Lc + chunk - 1) / chunk;
-      float* scores = p.scores ? p.scores + ((size_t)r * Hkv + kvh) * (size_t)p.cap * R : nullptr;
-      if (!wait_bar(smem_u32(&B->s_full), n & 1, abort_flag, p.err)) break;
-      tc_fence_after();
+    const int swz_row = (NP == 16) ? ((lrow >> 2) & 1) : ((lrow >> 1) & 3);
 
-      // pass 1: committed logits out, chunk max per row (raw q.k units until the end).
-      // Tiles entirely inside [0, min(L, end)) need no mask: every row sees every position
-      // (padding rows have zero queries and are discarded later).
+    // record of chunk m: O^T buffer m&1 -> workspace, with its row max / sum from cm / cl
+    auto epilogue = [&](int m) -> bool {
+      const Item x = make_item<NP>(blockIdx.x + m * gridDim.x, pref, batch, p);
+      if (!wait_bar(smem_u32(&B->o_full[m & 1]), (m >> 1) & 1, abort_flag, p.err)) return false;
+      tc_fence_after();
+      const size_t rec_floats = (size_t)p.Rp * (kD + 2);
+      float* rec = p.part + (((size_t)x.r * Hkv + x.kvh) * p.nchunk_max + x.c) * rec_floats;
+      constexpr int kHalf = NP / 2 >= 16 ? NP / 2 : 16;    // columns per warpgroup
+      if (sg * kHalf < NP) {
+        float o[16];
+        tmem_ld16(tl + C::kOCol + (m & 1) * NP + sg * kHalf, o);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) rec[2 * p.Rp + (size_t)(sg * kHalf + j) * kD + lrow] = o[j];
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&B->o_empty[m & 1]));
+      if (st < NP) {
+        rec[st] = cm[(m & 1) * NP + st];
+        rec[p.Rp + st] = cl[(m & 1) * NP + st];
+      }
+      return true;
+    };
+
+    bool ok = true;
+    for (int n = 0; n < my_items && !aborted(abort_flag); ++n) {
+      const Item x = make_item<NP>(blockIdx.x + n * gridDim.x, pref, batch, p);
+      const int L = x.L, start = x.start, end = x.end;
+      float* scores = p.scores ? p.scores + ((size_t)x.r * Hkv + x.kvh) * (size_t)p.cap * R : nullptr;
+      if (!wait_bar(smem_u32(&B->s_full[n & 1]), (n >> 1) & 1, abort_flag, p.err)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t sbuf = tl + (n & 1) * C::kSCols;
+
+      // pass 1 over this warpgroup's tiles: committed logits out, max per row (raw units)
       float mrow[NP];
 #pragma unroll
       for (int j = 0; j < NP; ++j) mrow[j] = -INFINITY;
-      for (int t = 0; t < ntile; ++t) {
+      for (int t = sg; t < x.ntile; t += 2) {
         float v[NP];
-        tmem_ld<NP>(tl + t * NP, v);
+        tmem_ld<NP>(sbuf + t * NP, v);
         tmem_wait_ld();
         const int t0 = start + t * kPos;
         const int pos = t0 + lrow;
@@ -521,29 +585,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         float m = mrow[j];
 #pragma unroll
         for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
-        mrow[j] = m;
+        if (lane == j) redM[sw8 * NP + j] = m;
       }
-      if (lane < NP) {
-        float mine = -INFINITY;
+      named_sync_softmax();
+      if (st < NP) {
+        float m = redM[st];
 #pragma unroll
-        for (int j = 0; j < NP; ++j)
-          if (j == lane) mine = mrow[j];
-        redM[q4 * NP + lane] = mine;
+        for (int w = 1; w < 8; ++w) m = fmaxf(m, redM[w * NP + st]);
+        cm[(n & 1) * NP + st] = scale2 * m;
       }
       named_sync_softmax();
 #pragma unroll
-      for (int j = 0; j < NP; ++j)
-        mrow[j] = scale2 * fmaxf(fmaxf(redM[j], redM[NP + j]), fmaxf(redM[2 * NP + j], redM[3 * NP + j]));
+      for (int j = 0; j < NP; ++j) mrow[j] = cm[(n & 1) * NP + j];
 
-      // pass 2: P = 2^(s - max) as bf16 P^T tiles, MN-major (the NP values of a position are
-      // contiguous, NP*2 bytes per row, swizzled in 16-byte chunks), and the row sums
+      // the previous chunk's output leaves tensor memory before P^T is overwritten
+      if (n > 0 && !epilogue(n - 1)) {
+        ok = false;
+        break;
+      }
+
+      // pass 2: P = 2^(s - max) as bf16 P^T tiles (MN-major, NP values per position) + sums
       float lsum[NP];
 #pragma unroll
       for (int j = 0; j < NP; ++j) lsum[j] = 0.f;
-      const int sw = (NP == 16) ? ((lrow >> 2) & 1) : ((lrow >> 1) & 3);
-      for (int t = 0; t < ntile; ++t) {
+      for (int t = sg; t < x.ntile; t += 2) {
         float v[NP];
-        tmem_ld<NP>(tl + t * NP, v);
+        tmem_ld<NP>(sbuf + t * NP, v);
         tmem_wait_ld();
         const int t0 = start + t * kPos;
         const int pos = t0 + lrow;
@@ -567,14 +634,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* prow = smem + C::kPOff + t * C::kPTile + lrow * (NP * 2);
 #pragma unroll
         for (int cc = 0; cc < NP / 8; ++cc)
-          *reinterpret_cast<uint4*>(prow + ((cc ^ sw) << 4)) =
+          *reinterpret_cast<uint4*>(prow + ((cc ^ swz_row) << 4)) =
               make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
       }
       fence_proxy_async();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(smem_u32(&B->s_empty));
+        mbar_arrive(smem_u32(&B->s_empty[n & 1]));
         mbar_arrive(smem_u32(&B->p_full));
       }
 #pragma unroll
@@ -582,41 +649,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         float sacc = lsum[j];
 #pragma unroll
         for (int o = 16; o; o >>= 1) sacc += __shfl_xor_sync(kFull, sacc, o);
-        lsum[j] = sacc;
+        if (lane == j) redL[sw8 * NP + j] = sacc;
       }
-      if (lane < NP) {
-        float mine = 0.f;
-#pragma unroll
-        for (int j = 0; j < NP; ++j)
-          if (j == lane) mine = lsum[j];
-        redL[q4 * NP + lane] = mine;
-      }
-
-      // epilogue: O^T (d = lrow, NP rows) -> chunk record
-      if (!wait_bar(smem_u32(&B->o_full), n & 1, abort_flag, p.err)) break;
-      tc_fence_after();
-      float o[NP];
-      tmem_ld<NP>(tl + C::kOCol, o);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&B->o_empty));
-      named_sync_softmax();   // redL complete
-      const size_t rec_floats = (size_t)p.Rp * (kD + 2);
-      float* recs = p.part + ((size_t)r * Hkv + kvh) * p.nchunk_max * rec_floats;
-      float* rec = recs + c * rec_floats;
+      named_sync_softmax();
       if (st < NP) {
-        float mm = -INFINITY;
+        float l = 0.f;
 #pragma unroll
-        for (int j = 0; j < NP; ++j)
-          if (j == st) mm = mrow[j];
-        rec[st] = mm;
-        rec[p.Rp + st] = redL[st] + redL[NP + st] + redL[2 * NP + st] + redL[3 * NP + st];
+        for (int w = 0; w < 8; ++w) l += redL[w * NP + st];
+        cl[(n & 1) * NP + st] = l;
       }
-#pragma unroll
-      for (int j = 0; j < NP; ++j) rec[2 * p.Rp + (size_t)j * kD + lrow] = o[j];
-
-      (void)nch;
+      // (cl / redL reuse is ordered by the barriers of the next chunk)
+    }
+    if (ok && my_items > 0 && !aborted(abort_flag)) {
+      named_sync_softmax();   // cl of the last chunk complete
+      epilogue(my_items - 1);
     }
   }
 
@@ -652,7 +698,10 @@ bool verify_tc_supported(int D, int R, int batch) {
   return D == tc::kD && verify_tc_npad(R) != 0 && batch <= tc::kMaxBatch;
 }
 
-int verify_tc_chunk() { return tc::kMaxTiles * tc::kPos; }
+int verify_tc_chunk(int R) {
+  const int np = verify_tc_npad(R);
+  return np == 16 ? tc::Cfg<16>::kChunk : tc::Cfg<32>::kChunk;
+}
 
 int launch_verify_tc(const CUtensorMap& tk, const CUtensorMap& tv, const VerifyParams& p,
                      int batch, int num_sms, cudaStream_t stream) {

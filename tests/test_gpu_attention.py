@@ -60,6 +60,7 @@ def test_verify_matches_oracle(Hq, Hkv, d, k, lens):
     (32, 8, 6, [2500, 1025, 4000]),     # 28 rows
     (16, 8, 6, [3000, 900]),            # 14 rows
     (32, 8, 0, [1200, 2100]),           # 4 rows (prefill pass)
+    (32, 8, 6, [9000, 12000, 7000, 10000, 11000, 8000, 9500, 10500]),   # several chunks per CTA
 ])
 def test_verify_kernels_agree_with_oracle(Hq, Hkv, k, lens):
     """The tcgen05 tensor-memory kernel and the mma.sync kernel on the same case."""
