@@ -136,6 +136,16 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// 4-D TMA tiled load global -> shared (coordinates innermost first).
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            int z, int w, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3, %4, %5}], [%6];\n" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(bar)
+      : "memory");
+}
+
 // Byte offset of 16-byte chunk `c` (0 .. d/8-1) of tile row `row` in a stage laid out as
 // [d/64 halves][kTile rows][128 B] with the 128-byte swizzle (chunk ^= row % 8), the layout a
 // TMA load with CU_TENSOR_MAP_SWIZZLE_128B writes into a 1024-byte aligned buffer.

@@ -139,6 +139,31 @@ int make_pool_map(CUtensorMap* map, void* pool, const s3r_kv_cache* c) {
   return S3R_OK;
 }
 
+// 4-D view of a pool (d, slot, kv head, page) with boxes of 64 columns x 16 slots x 1 head x
+// `pages` pages: `pages` consecutive page ids of one head land as one [pages*16][128 B] block
+// (128-byte swizzle), the layout of the 2-D map's 16-row boxes stacked.
+int make_paged_map(CUtensorMap* map, void* pool, const s3r_kv_cache* c, int pages) {
+  auto fn = encode_fn();
+  if (!fn) {
+    std::snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled unavailable");
+    return S3R_ERR_CUDA;
+  }
+  const cuuint64_t row = (cuuint64_t)c->head_dim * 2;
+  cuuint64_t dims[4] = {(cuuint64_t)c->head_dim, (cuuint64_t)S3R_PAGE_SIZE,
+                        (cuuint64_t)c->num_kv_heads, (cuuint64_t)c->num_pages};
+  cuuint64_t strides[3] = {row, row * S3R_PAGE_SIZE, row * S3R_PAGE_SIZE * c->num_kv_heads};
+  cuuint32_t box[4] = {64, (cuuint32_t)S3R_PAGE_SIZE, 1, (cuuint32_t)pages};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, pool, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    std::snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled (4-D): error %d", (int)r);
+    return S3R_ERR_CUDA;
+  }
+  return S3R_OK;
+}
+
 size_t verify_need(const s3r_kv_cache* c, int num_requests, int cap, int k) {
   const int G = c->num_q_heads / c->num_kv_heads;
   return head_bytes(num_requests) +
@@ -241,7 +266,12 @@ int s3r_verify_attn(const s3r_kv_cache* cache, const s3r_batch* batch, int32_t k
     p.Rp = verify_tc_npad(R);
     p.chunk = verify_tc_chunk(R);
     p.nchunk_max = (cap + p.chunk - 1) / p.chunk;
-    st = launch_verify_tc(tk, tv, p, batch->batch, sm_count(), (cudaStream_t)stream);
+    CUtensorMap k1, v1, k8, v8;
+    S3R_TRY(make_paged_map(&k1, cache->k_pool, cache, 1));
+    S3R_TRY(make_paged_map(&v1, cache->v_pool, cache, 1));
+    S3R_TRY(make_paged_map(&k8, cache->k_pool, cache, 8));
+    S3R_TRY(make_paged_map(&v8, cache->v_pool, cache, 8));
+    st = launch_verify_tc(k1, v1, k8, v8, p, batch->batch, sm_count(), (cudaStream_t)stream);
   } else {
     st = launch_verify(tk, tv, p, cache->head_dim, batch->batch, (cudaStream_t)stream);
   }

@@ -9,9 +9,10 @@
 // Organisation (one persistent CTA per SM, 6 warps):
 //   warp 0     producer: per work item (request, KV head, chunk of up to 8 tiles of 128
 //              positions) it copies the item's Q rows into shared memory, then streams the
-//              chunk's K tiles and then its V tiles through a 4-stage ring with 2-D TMA (one
-//              16-row box per page and 64-column half, 128-byte swizzle). The tile holding
-//              the block (positions >= L) is patched after its TMA lands.
+//              chunk's K tiles and then its V tiles through a 4-stage ring with 4-D TMA over
+//              (d, slot, head, page): a tile of 8 consecutive page ids is 2 boxes (one per
+//              64-column half, 128-byte swizzle), otherwise one box per page and half. The
+//              tile holding the block (positions >= L) is patched after its TMA lands.
 //   warp 1     MMA issuer: S^T tile t (128 positions x N rows, fp32) = K_t . Q^T into tensor
 //              memory columns [t*N, t*N+N) for every tile of the chunk, then, once the
 //              softmax warps have written P^T, O^T (128 d x N) = sum_t V_t^T . P_t^T into the
@@ -36,7 +37,7 @@ constexpr int kD = 128;                     // head_dim of this path
 constexpr int kStages = 4;
 constexpr int kThreads = 320;          // producer, MMA, 8 softmax warps
 constexpr int kTileBytes = kPos * kD * 2;   // 32 KB: [2 halves][128 rows][128 B]
-constexpr int kMaxBatch = 2048;             // requests per launch on this path
+constexpr int kMaxBatch = 1024;             // requests per launch on this path
 
 // --------------------------------------------------------------- tcgen05 wrappers -------
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
@@ -130,7 +131,10 @@ struct Cfg {
   static constexpr int kRedOff = kPOff + kPBytes;            // redM, redL [8 warps][NP]; cm, cl [2][NP]
   static constexpr int kRedBytes = (2 * 8 * NP + 4 * NP) * 4;
   static constexpr int kPrefOff = kRedOff + kRedBytes;       // request prefix [kMaxBatch+1]
-  static constexpr int kBarOff = (kPrefOff + (kMaxBatch + 1) * 4 + 63) / 64 * 64;
+  static constexpr int kLenOff = kPrefOff + (kMaxBatch + 1) * 4;   // L per request [kMaxBatch]
+  static constexpr int kRidOff = kLenOff + kMaxBatch * 4;          // request id [kMaxBatch]
+  static constexpr int kIdsOff = kRidOff + kMaxBatch * 4;          // page ids [2 items][64]
+  static constexpr int kBarOff = (kIdsOff + 2 * 64 * 4 + 63) / 64 * 64;
   static constexpr int kSmem = kBarOff + 256 + 1024;         // + barriers + alignment slack
 };
 
@@ -194,12 +198,13 @@ struct Item {
 };
 
 template <int NP>
-__device__ __forceinline__ Item make_item(int it, const int* pref, int batch, const VerifyParams& p) {
+__device__ __forceinline__ Item make_item(int it, const int* pref, const int* lens_s,
+                                          const int* rid_s, int batch, const VerifyParams& p) {
   Item x;
   int bl;
   item_of(it, pref, batch, p.Hkv, bl, x.kvh, x.c);
-  x.r = p.req_ids ? p.req_ids[bl] : bl;
-  x.L = p.seq_lens[x.r];
+  x.r = rid_s[bl];
+  x.L = lens_s[bl];
   x.Lc = x.L + p.T;
   x.start = x.c * Cfg<NP>::kChunk;
   x.end = min(x.start + Cfg<NP>::kChunk, x.Lc);
@@ -210,12 +215,16 @@ __device__ __forceinline__ Item make_item(int it, const int* pref, int batch, co
 template <int NP>
 __global__ void __launch_bounds__(kThreads, 1)
     verify_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                     const __grid_constant__ CUtensorMap tmK8, const __grid_constant__ CUtensorMap tmV8,
                      const VerifyParams p, int batch) {
   using C = Cfg<NP>;
   extern __shared__ uint8_t smem_dyn[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) &
                                              ~uintptr_t(1023));
   int* pref = reinterpret_cast<int*>(smem + C::kPrefOff);
+  int* lens_s = reinterpret_cast<int*>(smem + C::kLenOff);
+  int* rid_s = reinterpret_cast<int*>(smem + C::kRidOff);
+  int* ids_s = reinterpret_cast<int*>(smem + C::kIdsOff);
   float* redM = reinterpret_cast<float*>(smem + C::kRedOff);   // [8][NP]
   float* redL = redM + 8 * NP;                                  // [8][NP]
   float* cm = redL + 8 * NP;                                    // [2][NP] chunk max (log2)
@@ -234,6 +243,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = p.req_ids ? p.req_ids[b] : b;
     const int L = p.seq_lens[r];
     const int Lc = L + T;
+    rid_s[b] = r;
+    lens_s[b] = L;
     int items = 0;
     if (L >= 0 && Lc <= p.cap) items = Hkv * ((Lc + chunk - 1) / chunk);
     else if (blockIdx.x == 0) set_error(p.err, S3R_ERR_DEVICE_BOUNDS);
@@ -294,14 +305,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ===================================================================== producer ====
+    if (lane == 0) {
+      asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&tmK)) : "memory");
+      asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&tmV)) : "memory");
+      asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&tmK8)) : "memory");
+      asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&tmV8)) : "memory");
+    }
     // ring order: K(0), then per item n: K(n+1), V(n) -- the MMA warp consumes in this order
     int g = 0;
     uint32_t tma_phase = 0;   // bit s: phase of tma[s]
     bool stop = false;
-    auto load_tiles = [&](const Item& x, bool is_v) {
+    auto load_tiles = [&](const Item& x, bool is_v, const int* ids_item) {
       const CUtensorMap* map = is_v ? &tmV : &tmK;
+      const CUtensorMap* map8 = is_v ? &tmV8 : &tmK8;
       const __nv_bfloat16* blk = is_v ? p.v_new : p.k_new;
-      const int* ptab = p.page_table + (size_t)x.r * p.max_pages;
       for (int t = 0; t < x.ntile && !stop; ++t, ++g) {
         const int s = g % kStages;
         if (g >= kStages &&
@@ -316,11 +333,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool tail = (t0 + kPos > x.L);
         int ids[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int pg = (t0 >> 4) + i;
-          ids[i] = -1;
-          if (pg * kPage < x.L) ids[i] = ptab[pg];
-        }
+        for (int i = 0; i < 8; ++i) ids[i] = ids_item[t * 8 + i];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const int pg = (t0 >> 4) + i;
@@ -335,15 +348,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         const uint32_t landing = smem_u32(tail ? &B->tma[s] : &B->full[s]);
-        if (lane == 0) {
-          mbar_arrive_expect_tx(landing, (uint32_t)(nload * kPage * kD * 2));
+        if (lane == 0) mbar_arrive_expect_tx(landing, (uint32_t)(nload * kPage * kD * 2));
+        __syncwarp();
+        bool run = okmask == 0xFFu && !tail;   // 8 consecutive page ids: 2 boxes of 8 pages
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            if (!(okmask & (1u << i))) continue;
-            const int y = (int)(((int64_t)ids[i] * Hkv + x.kvh) * kPage);
-            tma_load_2d(dst + i * kPage * 128, map, 0, y, landing);
-            tma_load_2d(dst + kPos * 128 + i * kPage * 128, map, 64, y, landing);
-          }
+        for (int i = 1; i < 8; ++i) run = run && ids[i] == ids[0] + i;
+        if (run) {
+          if (lane < 2) tma_load_4d(dst + lane * kPos * 128, map8, lane * 64, 0, x.kvh, ids[0], landing);
+        } else if (lane < 16) {
+          // one page per lane pair (page lane/2, half lane%2)
+          const int i = lane >> 1, h = lane & 1;
+          if (okmask & (1u << i))
+            tma_load_4d(dst + h * kPos * 128 + i * kPage * 128, map, h * 64, 0, x.kvh, ids[i], landing);
         }
         if (tail) {
           // wait for the committed rows, then write block rows / zeros over the rest
@@ -370,8 +386,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     };
     auto load_q_and_k = [&](int m) {
-      const Item x = make_item<NP>(blockIdx.x + m * gridDim.x, pref, batch, p);
+      const Item x = make_item<NP>(blockIdx.x + m * gridDim.x, pref, lens_s, rid_s, batch, p);
       const int* ptab = p.page_table + (size_t)x.r * p.max_pages;
+      // page ids of the item's committed pages (-1 past L), read once for its K and V tiles
+      int* ids_item = ids_s + (m & 1) * 64;
+      {
+        const int npg = x.ntile * 8;
+        const int pg0 = x.start >> 4;
+        const int a = lane < npg && (pg0 + lane) * kPage < x.L ? ptab[pg0 + lane] : -1;
+        const int b = lane + 32 < npg && (pg0 + lane + 32) * kPage < x.L ? ptab[pg0 + lane + 32] : -1;
+        ids_item[lane] = a;
+        ids_item[lane + 32] = b;
+      }
       if (x.c == 0) {   // the block's K/V enter the cache once per (request, head)
         for (int idx = lane; idx < T * (kD / 8); idx += 32) {
           const int t = idx / (kD / 8), ch = idx - t * (kD / 8);
@@ -415,13 +441,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&B->q_full));
-      load_tiles(x, false);
+      load_tiles(x, false, ids_item);
     };
     if (my_items > 0) load_q_and_k(0);
     for (int n = 0; n < my_items && !stop && !aborted(abort_flag); ++n) {
       if (n + 1 < my_items) load_q_and_k(n + 1);
       if (stop) break;
-      load_tiles(make_item<NP>(blockIdx.x + n * gridDim.x, pref, batch, p), true);
+      load_tiles(make_item<NP>(blockIdx.x + n * gridDim.x, pref, lens_s, rid_s, batch, p), true,
+                 ids_s + (n & 1) * 64);
     }
   } else if (warp == 1) {
     // ====================================================================== MMA warp ===
@@ -430,7 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int g = 0;
     bool ok = true;
     auto qk = [&](int m) {
-      const Item x = make_item<NP>(blockIdx.x + m * gridDim.x, pref, batch, p);
+      const Item x = make_item<NP>(blockIdx.x + m * gridDim.x, pref, lens_s, rid_s, batch, p);
       ok = wait_bar(smem_u32(&B->q_full), m & 1, abort_flag, p.err);
       if (ok && m >= 2) ok = wait_bar(smem_u32(&B->s_empty[m & 1]), ((m - 2) >> 1) & 1, abort_flag, p.err);
       if (!ok) return;
@@ -460,7 +487,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
     };
     auto pv = [&](int n) {
-      const Item x = make_item<NP>(blockIdx.x + n * gridDim.x, pref, batch, p);
+      const Item x = make_item<NP>(blockIdx.x + n * gridDim.x, pref, lens_s, rid_s, batch, p);
       ok = wait_bar(smem_u32(&B->p_full), n & 1, abort_flag, p.err);
       if (ok && n >= 2) ok = wait_bar(smem_u32(&B->o_empty[n & 1]), ((n - 2) >> 1) & 1, abort_flag, p.err);
       if (!ok) return;
@@ -510,7 +537,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // record of chunk m: O^T buffer m&1 -> workspace, with its row max / sum from cm / cl
     auto epilogue = [&](int m) -> bool {
-      const Item x = make_item<NP>(blockIdx.x + m * gridDim.x, pref, batch, p);
+      const Item x = make_item<NP>(blockIdx.x + m * gridDim.x, pref, lens_s, rid_s, batch, p);
       if (!wait_bar(smem_u32(&B->o_full[m & 1]), (m >> 1) & 1, abort_flag, p.err)) return false;
       tc_fence_after();
       const size_t rec_floats = (size_t)p.Rp * (kD + 2);
@@ -535,7 +562,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     bool ok = true;
     for (int n = 0; n < my_items && !aborted(abort_flag); ++n) {
-      const Item x = make_item<NP>(blockIdx.x + n * gridDim.x, pref, batch, p);
+      const Item x = make_item<NP>(blockIdx.x + n * gridDim.x, pref, lens_s, rid_s, batch, p);
       const int L = x.L, start = x.start, end = x.end;
       float* scores = p.scores ? p.scores + ((size_t)x.r * Hkv + x.kvh) * (size_t)p.cap * R : nullptr;
       if (!wait_bar(smem_u32(&B->s_full[n & 1]), (n >> 1) & 1, abort_flag, p.err)) {
@@ -679,8 +706,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 int verify_tc_npad(int R) { return R <= 16 ? 16 : (R <= 32 ? 32 : 0); }
 
 template <int NP>
-static int launch_tc(const CUtensorMap& tk, const CUtensorMap& tv, const VerifyParams& p,
-                     int batch, int num_sms, cudaStream_t stream) {
+static int launch_tc(const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tk8,
+                     const CUtensorMap& tv8, const VerifyParams& p, int batch, int num_sms,
+                     cudaStream_t stream) {
   using C = tc::Cfg<NP>;
   static bool attr_done = false;
   if (!attr_done) {
@@ -690,7 +718,7 @@ static int launch_tc(const CUtensorMap& tk, const CUtensorMap& tv, const VerifyP
       return S3R_ERR_CUDA;
     attr_done = true;
   }
-  tc::verify_tc_kernel<NP><<<num_sms, tc::kThreads, C::kSmem, stream>>>(tk, tv, p, batch);
+  tc::verify_tc_kernel<NP><<<num_sms, tc::kThreads, C::kSmem, stream>>>(tk, tv, tk8, tv8, p, batch);
   return cuda_status(cudaGetLastError(), __func__);
 }
 
@@ -703,11 +731,12 @@ int verify_tc_chunk(int R) {
   return np == 16 ? tc::Cfg<16>::kChunk : tc::Cfg<32>::kChunk;
 }
 
-int launch_verify_tc(const CUtensorMap& tk, const CUtensorMap& tv, const VerifyParams& p,
-                     int batch, int num_sms, cudaStream_t stream) {
+int launch_verify_tc(const CUtensorMap& k1, const CUtensorMap& v1, const CUtensorMap& k8,
+                     const CUtensorMap& v8, const VerifyParams& p, int batch, int num_sms,
+                     cudaStream_t stream) {
   const int np = verify_tc_npad(p.R);
-  if (np == 16) return launch_tc<16>(tk, tv, p, batch, num_sms, stream);
-  if (np == 32) return launch_tc<32>(tk, tv, p, batch, num_sms, stream);
+  if (np == 16) return launch_tc<16>(k1, v1, k8, v8, p, batch, num_sms, stream);
+  if (np == 32) return launch_tc<32>(k1, v1, k8, v8, p, batch, num_sms, stream);
   return S3R_ERR_UNSUPPORTED;
 }
 
