@@ -173,6 +173,29 @@ S3R_API int s3r_draft_sample(const s3r_batch* batch, const int32_t* draft_step, 
                      const float* q_logits, int32_t vocab, uint64_t seed, int32_t* draft_tokens,
                      void* ws, size_t ws_bytes, s3r_stream_t stream);
 
+/* s3r_draft_sample without a workspace. The paper has no counterpart: this is a
+ * library convenience for callers that cannot hand the library device memory at the
+ * point of the call: a host program that drives the library from plain C without an
+ * allocator of its own, or a server that has given all free HBM to the KV pool and must
+ * not allocate between rounds. Same arguments, arithmetic and outputs as
+ * s3r_draft_sample, bit for bit; the scratch (arrival tickets and per-chunk partials)
+ * lives in a static device array inside the library, 8 KiB + 1 MiB per device, so
+ *   - num_requests <= S3R_NOALLOC_MAX_REQUESTS and vocab <= S3R_NOALLOC_MAX_VOCAB, else
+ *     S3R_ERR_UNSUPPORTED with a message in s3r_last_error_message() and no launch;
+ *   - err_word (device int32, caller-owned, zeroed by the caller before first use)
+ *     receives the device-side status bits that the workspace's error word would get;
+ *   - the first call on a device (the current device) looks the array up and zeroes its
+ *     tickets with a synchronous cudaMemset, so it belongs before any stream capture
+ *     begins. Later calls issue one kernel launch and nothing else.
+ *   - the array is shared by every call on a device: two calls that may overlap (other
+ *     streams, other host threads) race on it and give wrong tokens; order them.
+ * The library calls no allocation routine on this path. */
+#define S3R_NOALLOC_MAX_REQUESTS 2048
+#define S3R_NOALLOC_MAX_VOCAB 262144
+S3R_API int s3r_draft_sample_noalloc(const s3r_batch* batch, const int32_t* draft_step,
+                             int32_t k, const float* q_logits, int32_t vocab, uint64_t seed,
+                             int32_t* draft_tokens, int32_t* err_word, s3r_stream_t stream);
+
 /* Exact speculative sampling ([News] Interpretation; [Explainer] Jargon, exact speculative
  * sampling). p_j = softmax(p_logits[r][j]) (j = 0..k), q_j = softmax(q_logits[r][j])
  * (j < k) are the target / draft distributions of the token at position L+j+1.

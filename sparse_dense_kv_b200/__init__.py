@@ -17,6 +17,7 @@ from ._lib import (  # noqa: F401
     new_workspace,
     s3r_commit,
     s3r_draft_sample,
+    s3r_draft_sample_noalloc,
     s3r_get_error,
     s3r_launch_count,
     s3r_philox,

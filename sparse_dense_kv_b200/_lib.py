@@ -59,6 +59,7 @@ def _load():
         "s3r_select_from_scores": (ctypes.c_int, [C, B, P, I32, I32, I32, P, I32, P, P, SZ, P]),
         "s3r_sparse_draft_attn": (ctypes.c_int, [C, B, P, P, I32, P, P, I32, P, I32, P, P, P, P, SZ, P]),
         "s3r_draft_sample": (ctypes.c_int, [B, P, I32, P, I32, U64, P, P, SZ, P]),
+        "s3r_draft_sample_noalloc": (ctypes.c_int, [B, P, I32, P, I32, U64, P, P, P]),
         "s3r_spec_sample": (ctypes.c_int, [B, I32, P, P, P, I32, U64, P, P, P, SZ, P]),
         "s3r_commit": (ctypes.c_int, [B, I32, P, P, P, P]),
         "s3r_philox": (ctypes.c_int, [U64, I32, P, P, I64, P, P, P]),
@@ -220,6 +221,20 @@ def s3r_draft_sample(batch, draft_step, k, q_logits, vocab, seed, draft_tokens, 
         _ptr(q_logits, torch.float32, "q_logits"), vocab, seed,
         _ptr(draft_tokens, torch.int32, "draft_tokens"), _ptr(ws, torch.uint8, "ws"), ws.numel(),
         _stream(stream)), "s3r_draft_sample")
+
+
+def s3r_draft_sample_noalloc(batch, draft_step, k, q_logits, vocab, seed, draft_tokens, err_word,
+                             stream=None):
+    """s3r_draft_sample with the library's static scratch instead of a workspace; err_word
+    is a device int32 tensor of one element that receives the device-side status bits."""
+    st = _lib.s3r_draft_sample_noalloc(
+        ctypes.byref(batch), _ptr(draft_step, torch.int32, "draft_step"), k,
+        _ptr(q_logits, torch.float32, "q_logits"), vocab, seed,
+        _ptr(draft_tokens, torch.int32, "draft_tokens"), _ptr(err_word, torch.int32, "err_word"),
+        _stream(stream))
+    if st == 2 and _lib.s3r_last_error_message():
+        raise S3RError(st, "s3r_draft_sample_noalloc: " + _lib.s3r_last_error_message().decode())
+    _check(st, "s3r_draft_sample_noalloc")
 
 
 def s3r_spec_sample(batch, k, p_logits, q_logits, draft_tokens, vocab, seed, out_tokens, n_out,

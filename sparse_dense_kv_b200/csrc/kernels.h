@@ -123,6 +123,8 @@ int launch_select(const SelectParams& p, int batch, cudaStream_t stream);
 
 int launch_draft_sample(const SampleParams& p, int batch, cudaStream_t stream);
 int launch_spec_sample(const SampleParams& p, int batch, cudaStream_t stream, int* launches);
+// Bytes of one per-(request, vocabulary chunk) partial of the samplers.
+constexpr int kSamplePartialBytes = 16;
 size_t sample_partial_bytes(int num_requests, int k, int vocab);
 void spec_offsets(int num_requests, int k, int vocab, size_t* plan_off, size_t* draw_off);
 

@@ -3,6 +3,7 @@
 #include <atomic>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include <cudaTypedefs.h>
 
@@ -178,6 +179,50 @@ size_t draft_need(const s3r_kv_cache* c, int num_requests, int sel_stride) {
 
 size_t sample_need(int num_requests, int hkv, int k, int vocab) {
   return head_bytes(num_requests) + sample_partial_bytes(num_requests, k, vocab);
+}
+
+// ---------------------------------------------------- draft sampling without a workspace
+// Scratch of s3r_draft_sample_noalloc, a file-scope device array instead of a caller's
+// workspace: one arrival ticket per request (must start at zero; the last block of a
+// request puts it back to zero) followed by one partial record per (request, vocabulary
+// chunk). It is sized for S3R_NOALLOC_MAX_REQUESTS requests and vocabularies of at most
+// S3R_NOALLOC_MAX_VOCAB entries: 8 KiB of tickets + 1 MiB of partials per device.
+constexpr int kNoAllocChunks = S3R_NOALLOC_MAX_VOCAB / kVocabChunk;
+constexpr size_t kNoAllocTicketBytes = (size_t)S3R_NOALLOC_MAX_REQUESTS * sizeof(int);
+constexpr size_t kNoAllocBytes =
+    kNoAllocTicketBytes + (size_t)S3R_NOALLOC_MAX_REQUESTS * kNoAllocChunks * kSamplePartialBytes;
+static_assert(S3R_NOALLOC_MAX_VOCAB % kVocabChunk == 0, "whole vocabulary chunks");
+static_assert(kNoAllocTicketBytes % 256 == 0, "partials start 256-byte aligned");
+
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
+
+namespace {
+
+// Device address of the scratch on the current device. The first call on a device looks
+// the symbol up and zeroes its tickets (a synchronous cudaMemset, no allocation); later
+// calls only read the cached address.
+int noalloc_scratch(unsigned char** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cuda_status(cudaGetLastError(), "cudaGetDevice");
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return S3R_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    const int st = cuda_status(cudaGetSymbolAddress(&p, g_noalloc_scratch), "cudaGetSymbolAddress");
+    if (st != S3R_OK) return st;
+    if ((reinterpret_cast<uintptr_t>(p) & 255u) != 0) return S3R_ERR_WORKSPACE;
+    const int zs = cuda_status(cudaMemset(p, 0, kNoAllocTicketBytes), "cudaMemset");
+    if (zs != S3R_OK) return zs;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = static_cast<unsigned char*>(g_noalloc_ptr[dev]);
+  return S3R_OK;
 }
 
 #define S3R_TRY(x)              \
@@ -423,6 +468,43 @@ int s3r_draft_sample(const s3r_batch* batch, const int32_t* draft_step, int32_t 
   p.err = w.err;
   p.tickets = w.tickets;
   p.part = w.part;
+  return finish(launch_draft_sample(p, batch->batch, (cudaStream_t)stream), 1);
+}
+
+int s3r_draft_sample_noalloc(const s3r_batch* batch, const int32_t* draft_step, int32_t k,
+                             const float* q_logits, int32_t vocab, uint64_t seed,
+                             int32_t* draft_tokens, int32_t* err_word, s3r_stream_t stream) {
+  g_last_error[0] = '\0';
+  S3R_TRY(check_batch(batch, false));
+  if (k < 1 || k > S3R_MAX_K) return S3R_ERR_UNSUPPORTED;
+  if (vocab < 1) return S3R_ERR_UNSUPPORTED;
+  if (!draft_step || !q_logits || !draft_tokens || !err_word || !aligned4(draft_step) ||
+      !aligned4(q_logits) || !aligned4(draft_tokens) || !aligned4(err_word))
+    return S3R_ERR_INVALID_ARG;
+  if (batch->num_requests > S3R_NOALLOC_MAX_REQUESTS || vocab > S3R_NOALLOC_MAX_VOCAB) {
+    std::snprintf(g_last_error, sizeof(g_last_error),
+                  "s3r_draft_sample_noalloc: %d requests / vocab %d exceed the static scratch "
+                  "(at most %d requests, vocab %d)",
+                  batch->num_requests, vocab, S3R_NOALLOC_MAX_REQUESTS, S3R_NOALLOC_MAX_VOCAB);
+    return S3R_ERR_UNSUPPORTED;
+  }
+  if (batch->batch == 0) return S3R_OK;
+  unsigned char* scratch = nullptr;
+  S3R_TRY(noalloc_scratch(&scratch));
+  SampleParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.req_ids = batch->req_ids;
+  p.seq_lens = batch->seq_lens;
+  p.draft_step = draft_step;
+  p.k = k;
+  p.vocab = vocab;
+  p.nvch = nvch_of(vocab);
+  p.q_logits = q_logits;
+  p.draft_out = draft_tokens;
+  p.seed = seed;
+  p.err = err_word;
+  p.tickets = reinterpret_cast<int*>(scratch);
+  p.part = scratch + kNoAllocTicketBytes;
   return finish(launch_draft_sample(p, batch->batch, (cudaStream_t)stream), 1);
 }
 

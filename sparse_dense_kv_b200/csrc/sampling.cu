@@ -24,6 +24,7 @@ struct MS {
   float pad;
   double s;
 };
+static_assert(sizeof(MS) == kSamplePartialBytes, "partial record size");
 
 struct SpecPlan {
   int type;      // 0: residual of row j, 1: target row j

@@ -90,3 +90,22 @@ def test_host_validation_rejects_before_launch():
     # an empty batch is a no-op that succeeds
     e = s3r.BatchDesc(0, 0, None, None, None, 0)
     assert L.s3r_commit(ctypes.byref(e), 6, 0x10, 0x10, None, null) == 0
+
+
+def test_noalloc_draft_sample_validates_on_the_host():
+    """The static-scratch draft sampler checks its size limits before touching the device."""
+    import sparse_dense_kv_b200 as s3r
+    L = s3r.lib
+    null = ctypes.c_void_p(0)
+    big = s3r.BatchDesc(1, 2049, None, 0x1000, None, 0)
+    assert L.s3r_draft_sample_noalloc(ctypes.byref(big), 0x10, 6, 0x10, 1000, 1, 0x10, 0x10,
+                                      null) == 2
+    assert b"static scratch" in L.s3r_last_error_message()
+    b = s3r.BatchDesc(1, 8, None, 0x1000, None, 0)
+    assert L.s3r_draft_sample_noalloc(ctypes.byref(b), 0x10, 6, 0x10, 262145, 1, 0x10, 0x10,
+                                      null) == 2
+    # the caller's error word is required
+    assert L.s3r_draft_sample_noalloc(ctypes.byref(b), 0x10, 6, 0x10, 1000, 1, 0x10, None,
+                                      null) == 1
+    assert L.s3r_draft_sample_noalloc(ctypes.byref(b), 0x10, 9, 0x10, 1000, 1, 0x10, 0x10,
+                                      null) == 2
