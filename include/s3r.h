@@ -113,11 +113,12 @@ S3R_API int s3r_workspace_init(void* ws, size_t ws_bytes, s3r_stream_t stream);
  *              of positions L..L+k (which must be allocated) and used for the block.
  *   out        bf16 [num_requests][T][H_q][d], softmax(q K^T / sqrt(d)) V rounded once.
  *   lse        fp32 [num_requests][T][H_q], natural-log log-sum-exp of the logits.
- *   score_logits fp32 [num_requests][H_kv][capacity][G*T] or NULL: logit q.k/sqrt(d) of
- *              row t*G+g of each KV head at every committed position j < L, the G*T logits
- *              of one position contiguous (entries at j >= L are not written). With lse it
+ *   score_logits fp32 [num_requests][H_kv][G*T][capacity] or NULL: logit q.k/sqrt(d) of
+ *              row t*G+g of each KV head at every committed position j < L, the positions
+ *              of one row contiguous (entries at j >= L are not written). With lse it
  *              defines the scores of s3r_select_kv.
- * Needs L + T <= capacity (device check). */
+ * q, k_new, v_new, out and score_logits must be 16-byte aligned, lse 4-byte aligned
+ * (S3R_ERR_INVALID_ARG otherwise). Needs L + T <= capacity (device check). */
 S3R_API int s3r_verify_attn(const s3r_kv_cache* cache, const s3r_batch* batch, int32_t k,
                     const void* q, const void* k_new, const void* v_new, void* out,
                     float* lse, float* score_logits, void* ws, size_t ws_bytes,
@@ -130,7 +131,9 @@ S3R_API int s3r_verify_attn(const s3r_kv_cache* cache, const s3r_batch* batch, i
  * is the W' newest positions plus the n - W' positions j < L - W' of highest score
  *   sigma_j = sum over the G*(k_prev+1) rows of exp(score_logits[row][j] - lse[row]),
  * ties to the lower j, written ascending to sel_idx[r][h][0..n-1]; sel_count[r][h] = n.
- *   score_logits, lse  as written by the previous s3r_verify_attn with k = k_prev.
+ *   score_logits, lse  as written by the previous s3r_verify_attn with k = k_prev
+ *              (score_logits 16-byte aligned). The exponentials are formed as
+ *              2^(x log2(e) - lse log2(e)) in fp32 (relative error about 1e-6).
  *   sel_idx    int32 [num_requests][H_kv][sel_stride]; n > sel_stride is a device bounds
  *              error. sel_count int32 [num_requests][H_kv].
  * Needs 1 <= budget_bp <= 10000 and window >= k_prev + 1 (so that every scored non-window

@@ -31,4 +31,4 @@ from ._lib import (  # noqa: F401
     s3r_workspace_init,
     s3r_workspace_size,
 )
-from .engine import RoundBuffers, S3REngine  # noqa: F401
+from .engine import MixedPhaseDriver, RoundBuffers, S3REngine  # noqa: F401

@@ -15,7 +15,12 @@
 
 namespace s3r {
 
-template <int D, int NTW>
+// Shared-memory layouts of a KV stage: byte offset of 16-byte chunk c of tile row `row`.
+// Swz128: [d/64][64 rows][128 B] with the 128-byte swizzle (what a swizzled TMA box writes).
+struct Swz128Layout {
+  __device__ __forceinline__ static uint32_t off(int row, int c) { return swz(row, c); }
+};
+template <int D, int NTW, class Layout = Swz128Layout>
 struct WarpAttn {
   uint32_t qf[NTW][D / 16][2];  // Q^T B-fragments
   float o[D / 16][NTW][4];      // O^T accumulators: (d = dm*16 + lane/4 (+8), row pair)
@@ -71,7 +76,7 @@ struct WarpAttn {
 #pragma unroll
     for (int ks = 0; ks < D / 16; ++ks) {
       uint32_t a[4];
-      ldsm_x4(kb + swz(krow, 2 * ks + (mi >> 1)), a);
+      ldsm_x4(kb + Layout::off(krow, 2 * ks + (mi >> 1)), a);
 #pragma unroll
       for (int nt = 0; nt < NTW; ++nt) mma_bf16(s[nt], a, qf[nt][ks][0], qf[nt][ks][1]);
     }
@@ -132,7 +137,7 @@ struct WarpAttn {
 #pragma unroll
     for (int dm = 0; dm < D / 16; ++dm) {
       uint32_t a[4];
-      ldsm_x4_t(vb + swz(vrow, 2 * dm + (mi & 1)), a);
+      ldsm_x4_t(vb + Layout::off(vrow, 2 * dm + (mi & 1)), a);
 #pragma unroll
       for (int nt = 0; nt < NTW; ++nt) mma_bf16(o[dm][nt], a, b[nt][0], b[nt][1]);
     }
@@ -184,13 +189,14 @@ struct WarpAttn {
 // Merge the 4 position-slice warps of each row group in shared scratch into one chunk
 // record in global memory: rec = [m: Rp][l: Rp][O: Rp][D] (floats, m in log2 units).
 // Warp w = group*4 + slice; group g covers rows g*RW .. g*RW+RW-1.
+// Threads tid = 0..nthreads-1 share the work.
 template <int D, int RW>
 __device__ __forceinline__ void merge_slices_to_record(const float* redO, const float* redM,
                                                        const float* redL, int ngroups,
-                                                       float* rec, int Rp) {
+                                                       float* rec, int Rp, int tid, int nthreads) {
   constexpr int DS = D + 4;
   const int rows = ngroups * RW;
-  for (int idx = threadIdx.x; idx < rows * D; idx += blockDim.x) {
+  for (int idx = tid; idx < rows * D; idx += nthreads) {
     const int grow = idx / D, d = idx - grow * D;
     const int g = grow / RW, rl = grow - g * RW;
     float M = -INFINITY;
@@ -211,6 +217,13 @@ __device__ __forceinline__ void merge_slices_to_record(const float* redO, const 
       rec[Rp + grow] = lsum;
     }
   }
+}
+
+template <int D, int RW>
+__device__ __forceinline__ void merge_slices_to_record(const float* redO, const float* redM,
+                                                       const float* redL, int ngroups,
+                                                       float* rec, int Rp) {
+  merge_slices_to_record<D, RW>(redO, redM, redL, ngroups, rec, Rp, threadIdx.x, blockDim.x);
 }
 
 // Combine `nch` chunk records of `R` rows into normalised outputs: for row < R and d < D,

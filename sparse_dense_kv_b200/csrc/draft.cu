@@ -35,7 +35,7 @@ __global__ void __launch_bounds__(128) draft_kernel(const DraftParams p) {
   const int i = p.draft_step[r];
   const int Hkv = p.Hkv, G = p.G;
   const int n = p.sel_count[(size_t)r * Hkv + kvh];
-  if (L < 0 || i < 0 || L + i >= p.cap || n < 0 || n > p.sel_stride) {
+  if (L < 0 || i < 0 || i >= S3R_MAX_K || L + i >= p.cap || n < 0 || n > p.sel_stride) {
     if (c == 0 && tid == 0) set_error(p.err, S3R_ERR_DEVICE_BOUNDS);
     return;
   }
@@ -184,7 +184,7 @@ static int launch_draft_d(const DraftParams& p, int batch, cudaStream_t stream) 
   return cuda_status(cudaGetLastError(), __func__);
 }
 
-int launch_draft(const DraftParams& p, int D, int batch, cudaStream_t stream) {
+int launch_draft(const DraftParams& p, int D, int batch, int /*num_sms*/, cudaStream_t stream) {
   if (D == 128) return launch_draft_d<128>(p, batch, stream);
   if (D == 64) return launch_draft_d<64>(p, batch, stream);
   return S3R_ERR_UNSUPPORTED;

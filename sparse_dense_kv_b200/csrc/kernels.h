@@ -112,11 +112,11 @@ int launch_verify_combine(const VerifyParams& p, int D, int batch, cudaStream_t 
 bool verify_tc_supported(int D, int R, int batch);
 int verify_tc_npad(int R);
 int verify_tc_chunk(int R);
-int launch_verify_tc(const CUtensorMap& k1, const CUtensorMap& v1, const CUtensorMap& k8,
-                     const CUtensorMap& v8, const VerifyParams& p, int batch, int num_sms,
-                     cudaStream_t stream);
+int launch_verify_tc(const CUtensorMap& qm, const CUtensorMap& k1, const CUtensorMap& v1,
+                     const CUtensorMap& k8, const CUtensorMap& v8, const VerifyParams& p,
+                     int batch, int num_sms, cudaStream_t stream);
 
-int launch_draft(const DraftParams& p, int D, int batch, cudaStream_t stream);
+int launch_draft(const DraftParams& p, int D, int batch, int num_sms, cudaStream_t stream);
 size_t draft_partial_bytes(int num_requests, int Hkv, int sel_stride, int D);
 
 int launch_select(const SelectParams& p, int batch, cudaStream_t stream);

@@ -165,6 +165,32 @@ int make_paged_map(CUtensorMap* map, void* pool, const s3r_kv_cache* c, int page
   return S3R_OK;
 }
 
+// 3-D view of the query rows q [num_requests][T][H_q][d] as (d, q head, request * T + t)
+// with boxes of 64 columns x G heads x T rows: the G*T rows of one (request, KV head) land
+// as one [T*G][128 B] block (row t*G + g, 128-byte swizzle) per 64-column half.
+int make_q_map(CUtensorMap* map, const void* q, const s3r_kv_cache* c, int num_requests, int T) {
+  auto fn = encode_fn();
+  if (!fn) {
+    std::snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled unavailable");
+    return S3R_ERR_CUDA;
+  }
+  const int G = c->num_q_heads / c->num_kv_heads;
+  const cuuint64_t row = (cuuint64_t)c->head_dim * 2;
+  cuuint64_t dims[3] = {(cuuint64_t)c->head_dim, (cuuint64_t)c->num_q_heads,
+                        (cuuint64_t)num_requests * T};
+  cuuint64_t strides[2] = {row, row * c->num_q_heads};
+  cuuint32_t box[3] = {64, (cuuint32_t)G, (cuuint32_t)T};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    std::snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled (q): error %d", (int)r);
+    return S3R_ERR_CUDA;
+  }
+  return S3R_OK;
+}
+
 size_t verify_need(const s3r_kv_cache* c, int num_requests, int cap, int k) {
   const int G = c->num_q_heads / c->num_kv_heads;
   return head_bytes(num_requests) +
@@ -269,7 +295,7 @@ int s3r_verify_attn(const s3r_kv_cache* cache, const s3r_batch* batch, int32_t k
   if (R > S3R_MAX_ROWS) return S3R_ERR_UNSUPPORTED;
   if (!q || !k_new || !v_new || !out || !lse) return S3R_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(out) ||
-      !aligned4(lse) || (score_logits && !aligned4(score_logits)))
+      !aligned4(lse) || (score_logits && !aligned16(score_logits)))
     return S3R_ERR_INVALID_ARG;
   if (batch->batch == 0) return S3R_OK;
   const int cap = batch->max_pages_per_req * S3R_PAGE_SIZE;
@@ -311,12 +337,13 @@ int s3r_verify_attn(const s3r_kv_cache* cache, const s3r_batch* batch, int32_t k
     p.Rp = verify_tc_npad(R);
     p.chunk = verify_tc_chunk(R);
     p.nchunk_max = (cap + p.chunk - 1) / p.chunk;
-    CUtensorMap k1, v1, k8, v8;
+    CUtensorMap k1, v1, k8, v8, qm;
+    S3R_TRY(make_q_map(&qm, q, cache, batch->num_requests, k + 1));
     S3R_TRY(make_paged_map(&k1, cache->k_pool, cache, 1));
     S3R_TRY(make_paged_map(&v1, cache->v_pool, cache, 1));
     S3R_TRY(make_paged_map(&k8, cache->k_pool, cache, 8));
     S3R_TRY(make_paged_map(&v8, cache->v_pool, cache, 8));
-    st = launch_verify_tc(k1, v1, k8, v8, p, batch->batch, sm_count(), (cudaStream_t)stream);
+    st = launch_verify_tc(qm, k1, v1, k8, v8, p, batch->batch, sm_count(), (cudaStream_t)stream);
   } else {
     st = launch_verify(tk, tv, p, cache->head_dim, batch->batch, (cudaStream_t)stream);
   }
@@ -357,7 +384,7 @@ int s3r_select_kv(const s3r_kv_cache* cache, const s3r_batch* batch, const float
   S3R_TRY(check_batch(batch, true));
   if (k_prev < 0 || k_prev > S3R_MAX_K) return S3R_ERR_UNSUPPORTED;
   if (window < k_prev + 1) return S3R_ERR_INVALID_ARG;
-  if (!score_logits || !lse || !aligned4(score_logits) || !aligned4(lse))
+  if (!score_logits || !lse || !aligned16(score_logits) || !aligned4(lse))
     return S3R_ERR_INVALID_ARG;
   const int G = cache->num_q_heads / cache->num_kv_heads;
   if (G * (k_prev + 1) > S3R_MAX_ROWS) return S3R_ERR_UNSUPPORTED;
@@ -439,7 +466,7 @@ int s3r_sparse_draft_attn(const s3r_kv_cache* cache, const s3r_batch* batch,
   p.err = w.err;
   p.tickets = w.tickets;
   p.part = reinterpret_cast<float*>(w.part);
-  return finish(launch_draft(p, cache->head_dim, batch->batch, (cudaStream_t)stream), 1);
+  return finish(launch_draft(p, cache->head_dim, batch->batch, sm_count(), (cudaStream_t)stream), 1);
 }
 
 int s3r_draft_sample(const s3r_batch* batch, const int32_t* draft_step, int32_t k,

@@ -8,9 +8,10 @@
 //
 // One CTA of 1024 threads per (KV head, request). Scores sigma_j = sum over the G*(k+1)
 // verify rows of exp(logit - lse) are computed once into shared memory as order-preserving
-// uint32 keys; four 8-bit MSB-first histogram passes (warp-aggregated shared atomics) find
-// the exact key of the M-th largest score and how many ties at that key to keep; a final
-// pass compacts the chosen indices in increasing order with ballot-based block scans.
+// uint32 keys; three MSB-first histogram passes of 11, 11 and 10 bits (warp-aggregated
+// shared atomics, one block scan over the bins per pass) find the exact key of the M-th
+// largest score and how many ties at that key to keep; a final pass compacts the chosen
+// indices in increasing order, each warp over its own contiguous run of positions.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -18,6 +19,7 @@ namespace s3r {
 
 constexpr int kSelectThreads = 1024;
 constexpr int kSelectMaxN = 49152;   // non-window positions held in shared memory
+constexpr int kSelectBins = 2048;    // 11-bit digits: bits 31..21, 20..10, 9..0
 
 __device__ __forceinline__ uint32_t order_key(float f) {
   if (f == 0.f) f = 0.f;              // -0 and +0 compare equal
@@ -25,34 +27,43 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Exclusive block-wide prefix count of `flag`; also returns the block total.
-__device__ __forceinline__ int block_excl_count(bool flag, int* warp_tot, int& total) {
+// Block-wide exclusive prefix sum of `v` in thread order (1024 threads); `wsum` holds 32
+// ints of scratch. Ends with a barrier.
+__device__ __forceinline__ int block_excl_scan(int v, int* wsum) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const unsigned b = __ballot_sync(kFull, flag);
-  const int in_warp = __popc(b & ((1u << lane) - 1u));
-  if (lane == 0) warp_tot[warp] = __popc(b);
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(kFull, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) wsum[warp] = incl;
   __syncthreads();
-  int before = 0, tot = 0;
-  const int nw = blockDim.x >> 5;
-  for (int w = 0; w < nw; ++w) {
-    const int v = warp_tot[w];
-    before += (w < warp) ? v : 0;
-    tot += v;
+  if (warp == 0) {
+    const int t = wsum[lane];
+    int ti = t;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(kFull, ti, o);
+      if (lane >= o) ti += n;
+    }
+    wsum[lane] = ti - t;
   }
   __syncthreads();
-  total = tot;
-  return before + in_warp;
+  const int r = wsum[warp] + incl - v;
+  __syncthreads();
+  return r;
 }
 
-__global__ void __launch_bounds__(kSelectThreads) select_kernel(const SelectParams p) {
+__global__ void __launch_bounds__(kSelectThreads, 2) select_kernel(const SelectParams p) {
   extern __shared__ uint32_t keys[];
-  __shared__ uint32_t hist[256];
+  __shared__ uint32_t hist[kSelectBins];
   __shared__ float lse_s[S3R_MAX_ROWS];
-  __shared__ int warp_tot[32];
+  __shared__ int wsum[32], wa[32], wb[32];
   __shared__ uint32_t s_prefix;
   __shared__ int s_remaining;
 
-  const int tid = threadIdx.x, lane = tid & 31;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int kvh = blockIdx.x, bl = blockIdx.y;
   const int r = p.req_ids ? p.req_ids[bl] : bl;
   const int L = p.seq_lens[r];
@@ -78,116 +89,167 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const SelectPara
   if (tid == 0) p.sel_count[(size_t)r * p.Hkv + kvh] = n;
   if (M == 0) return;
 
-  // ---- scores -> keys
+  // ---- scores -> order-preserving keys in shared memory
+  bool bad = false;
   if (p.logits) {
+    // sigma_j = sum over rows of 2^(logit * log2(e) - lse * log2(e)); the logits of one row
+    // are contiguous over positions ([..][R][cap]), so every thread takes 4 consecutive
+    // positions with one 16-byte load per row, four rows in flight at a time
     for (int row = tid; row < p.R; row += blockDim.x) {
       const int t = row / p.G, g = row - t * p.G;
-      lse_s[row] = p.lse[((size_t)r * p.T + t) * p.Hq + kvh * p.G + g];
+      lse_s[row] = p.lse[((size_t)r * p.T + t) * p.Hq + kvh * p.G + g] * kLog2e;
     }
     __syncthreads();
-  }
-  bool bad = false;
-  for (int j = tid; j < N; j += blockDim.x) {
-    float sigma;
-    if (p.logits) {
-      // the G*(k+1) logits of position j are contiguous: [..][cap][R]
-      const float* lg = p.logits + (((size_t)r * p.Hkv + kvh) * p.cap + j) * p.R;
-      float acc = 0.f;
-      if ((p.R & 3) == 0) {
-        for (int row = 0; row < p.R; row += 4) {
-          const float4 x = __ldg(reinterpret_cast<const float4*>(lg + row));
-          acc += expf(x.x - lse_s[row]) + expf(x.y - lse_s[row + 1]) +
-                 expf(x.z - lse_s[row + 2]) + expf(x.w - lse_s[row + 3]);
+    const float* base = p.logits + ((size_t)r * p.Hkv + kvh) * (size_t)p.R * p.cap;
+    for (int j4 = 4 * tid; j4 < N; j4 += 4 * blockDim.x) {
+      float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+      int row = 0;
+      for (; row + 4 <= p.R; row += 4) {
+        float4 x[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          x[u] = __ldg(reinterpret_cast<const float4*>(base + (size_t)(row + u) * p.cap + j4));
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float l2 = lse_s[row + u];
+          acc0 += ex2(fmaf(x[u].x, kLog2e, -l2));
+          acc1 += ex2(fmaf(x[u].y, kLog2e, -l2));
+          acc2 += ex2(fmaf(x[u].z, kLog2e, -l2));
+          acc3 += ex2(fmaf(x[u].w, kLog2e, -l2));
         }
-      } else if ((p.R & 1) == 0) {
-        for (int row = 0; row < p.R; row += 2) {
-          const float2 x = __ldg(reinterpret_cast<const float2*>(lg + row));
-          acc += expf(x.x - lse_s[row]) + expf(x.y - lse_s[row + 1]);
-        }
-      } else {
-        for (int row = 0; row < p.R; ++row) acc += expf(__ldg(lg + row) - lse_s[row]);
       }
-      sigma = acc;
-    } else {
-      sigma = p.scores[((size_t)r * p.Hkv + kvh) * p.score_stride + j];
+      for (; row < p.R; ++row) {
+        const float4 x = __ldg(reinterpret_cast<const float4*>(base + (size_t)row * p.cap + j4));
+        const float l2 = lse_s[row];
+        acc0 += ex2(fmaf(x.x, kLog2e, -l2));
+        acc1 += ex2(fmaf(x.y, kLog2e, -l2));
+        acc2 += ex2(fmaf(x.z, kLog2e, -l2));
+        acc3 += ex2(fmaf(x.w, kLog2e, -l2));
+      }
+      const float sg[4] = {acc0, acc1, acc2, acc3};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (j4 + q >= N) break;
+        float sigma = sg[q];
+        if (!isfinite(sigma)) {
+          bad = true;
+          sigma = -INFINITY;
+        }
+        keys[j4 + q] = order_key(sigma);
+      }
     }
-    if (!isfinite(sigma)) {
-      bad = true;
-      sigma = -INFINITY;
+  } else {
+    for (int j = tid; j < N; j += blockDim.x) {
+      float sigma = p.scores[((size_t)r * p.Hkv + kvh) * p.score_stride + j];
+      if (!isfinite(sigma)) {
+        bad = true;
+        sigma = -INFINITY;
+      }
+      keys[j] = order_key(sigma);
     }
-    keys[j] = order_key(sigma);
   }
   if (bad) set_error(p.err, S3R_ERR_NONFINITE);
   __syncthreads();
 
-  // ---- radix select of the M-th largest key
+  // ---- radix select of the M-th largest key: three MSB-first passes of 11, 11, 10 bits.
+  // Each pass histograms the digit of the keys still matching the prefix (warp-aggregated
+  // shared atomics), then one block scan over the bins from the top finds the bin holding
+  // the remaining-th largest.
   uint32_t prefix = 0, mask = 0;
   int remaining = M;
   const int Nround = (N + blockDim.x - 1) / blockDim.x * blockDim.x;
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    if (tid < 256) hist[tid] = 0;
+#pragma unroll 1
+  for (int pass = 0; pass < 3; ++pass) {
+    const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+    const int nb = pass == 2 ? 1024 : 2048;
+    for (int b = tid; b < nb; b += blockDim.x) hist[b] = 0;
     __syncthreads();
     for (int j = tid; j < Nround; j += blockDim.x) {
       const uint32_t key = j < N ? keys[j] : 0u;
       const bool part = j < N && (key & mask) == prefix;
-      const uint32_t digit = (key >> shift) & 255u;
-      const unsigned peers = __match_any_sync(kFull, part ? digit : (0x100u + lane));
+      const uint32_t digit = (key >> shift) & (uint32_t)(nb - 1);
+      const unsigned peers = __match_any_sync(kFull, part ? digit : (0x10000u + lane));
       if (part && lane == __ffs(peers) - 1) atomicAdd(&hist[digit], (uint32_t)__popc(peers));
     }
     __syncthreads();
-    if (tid < 32) {
-      // lane l owns bins 255-8l .. 248-8l (descending)
-      uint32_t loc = 0;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) loc += hist[255 - 8 * lane - q];
-      uint32_t incl = loc;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t v = __shfl_up_sync(kFull, incl, o);
-        if (lane >= o) incl += v;
-      }
-      const uint32_t excl = incl - loc;
-      const unsigned hit = __ballot_sync(kFull, incl >= (uint32_t)remaining);
-      const int owner = __ffs(hit) - 1;
-      if (lane == owner) {
-        uint32_t cum = excl;
-        int dsel = 248 - 8 * lane;
-        for (int q = 0; q < 8; ++q) {
-          const int bin = 255 - 8 * lane - q;
-          if (cum + hist[bin] >= (uint32_t)remaining) {
-            dsel = bin;
-            break;
-          }
-          cum += hist[bin];
+    // thread t owns the bins nb-1-per*t .. nb-per*(t+1) (descending)
+    const int per = nb / kSelectThreads;
+    int h[2] = {0, 0}, local = 0;
+    for (int q = 0; q < per; ++q) {
+      h[q] = (int)hist[nb - 1 - per * tid - q];
+      local += h[q];
+    }
+    const int before = block_excl_scan(local, wsum);
+    if (before < remaining && remaining <= before + local) {
+      int cum = before;
+      for (int q = 0; q < per; ++q) {
+        if (cum + h[q] >= remaining) {
+          s_prefix = prefix | ((uint32_t)(nb - 1 - per * tid - q) << shift);
+          s_remaining = remaining - cum;
+          break;
         }
-        s_prefix = prefix | ((uint32_t)dsel << shift);
-        s_remaining = remaining - (int)cum;
+        cum += h[q];
       }
     }
     __syncthreads();
     prefix = s_prefix;
     remaining = s_remaining;
-    mask |= 255u << shift;
+    mask |= (uint32_t)(nb - 1) << shift;
   }
-  // prefix is the key of the M-th largest score; `remaining` keys equal to it are kept.
+  // prefix is the key of the M-th largest score; the first `remaining` keys equal to it (in
+  // position order) are kept.
   const uint32_t thr = prefix;
   const int need_eq = remaining;
 
-  // ---- ordered compaction
-  int base = 0, eq_seen = 0;
-  for (int j0 = 0; j0 < N && base < M; j0 += blockDim.x) {
-    const int j = j0 + tid;
-    const uint32_t key = j < N ? keys[j] : 0u;
-    const bool gt = j < N && key > thr;
-    const bool eq = j < N && key == thr;
-    int eq_tot, take_tot;
-    const int eq_rank = eq_seen + block_excl_count(eq, warp_tot, eq_tot);
-    const bool take = gt || (eq && eq_rank < need_eq);
-    const int at = base + block_excl_count(take, warp_tot, take_tot);
-    if (take) out[at] = j;
-    base += take_tot;
-    eq_seen += eq_tot;
+  // ---- ordered compaction: warp w owns a contiguous run of positions; counts per warp, one
+  // scan over the 32 warps, then every warp writes its picks in order
+  const int seg = ((N + 31) / 32 + 31) / 32 * 32;
+  const int j0 = warp * seg, j1 = min(N, j0 + seg);
+  const unsigned lt = (1u << lane) - 1u;
+  int gt_w = 0, eq_w = 0;
+  for (int jb = j0; jb < j1; jb += 32) {
+    const int j = jb + lane;
+    const uint32_t key = j < j1 ? keys[j] : 0u;
+    gt_w += __popc(__ballot_sync(kFull, j < j1 && key > thr));
+    eq_w += __popc(__ballot_sync(kFull, j < j1 && key == thr));
+  }
+  if (lane == 0) {
+    wa[warp] = gt_w;
+    wb[warp] = eq_w;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const int e = wb[lane];
+    int ei = e;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(kFull, ei, o);
+      if (lane >= o) ei += v;
+    }
+    const int eq_before = ei - e;
+    const int take = wa[lane] + min(max(need_eq - eq_before, 0), e);
+    int ti = take;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(kFull, ti, o);
+      if (lane >= o) ti += v;
+    }
+    wa[lane] = ti - take;   // picks before this warp's run
+    wb[lane] = eq_before;   // equal keys before this warp's run
+  }
+  __syncthreads();
+  int base = wa[warp], eqb = wb[warp];
+  for (int jb = j0; jb < j1; jb += 32) {
+    const int j = jb + lane;
+    const uint32_t key = j < j1 ? keys[j] : 0u;
+    const bool gt = j < j1 && key > thr;
+    const bool eq = j < j1 && key == thr;
+    const unsigned em = __ballot_sync(kFull, eq);
+    const bool take = gt || (eq && eqb + __popc(em & lt) < need_eq);
+    const unsigned tm = __ballot_sync(kFull, take);
+    if (take) out[base + __popc(tm & lt)] = j;
+    base += __popc(tm);
+    eqb += __popc(em);
   }
 }
 

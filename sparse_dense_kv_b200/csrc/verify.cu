@@ -180,14 +180,10 @@ __global__ void __launch_bounds__(MAXT) verify_kernel(const __grid_constant__ CU
       auto cap_fn = [&](int tr, int nt, float lg0, float lg1) {
         const int pos = t0 + tr;
         const int row = grp * RW + nt * 8 + 2 * (lane & 3);
-        if (scores && row < R && pos < L) {
-          float* dst = scores + score_base + (size_t)pos * R + row;
-          if (!(R & 1)) {
-            *reinterpret_cast<float2*>(dst) = make_float2(lg0, lg1);
-          } else {
-            dst[0] = lg0;
-            if (row + 1 < R) dst[1] = lg1;
-          }
+        if (scores && row < R && pos < L) {   // [row][position]
+          float* dst = scores + score_base + (size_t)row * p.cap + pos;
+          dst[0] = lg0;
+          if (row + 1 < R) dst[p.cap] = lg1;
         }
       };
       if (t0 + kTile <= L && t0 + kTile <= end)

@@ -34,8 +34,10 @@ namespace tc {
 
 constexpr int kPos = 128;                   // positions per tile (MMA M)
 constexpr int kD = 128;                     // head_dim of this path
-constexpr int kStages = 4;
-constexpr int kThreads = 320;          // producer, MMA, 8 softmax warps
+constexpr int kKStages = 2;                 // K ring
+constexpr int kVStages = 2;                 // V ring
+constexpr int kThreads = 352;               // K producer, V producer, MMA, 8 softmax warps
+constexpr int kSoftWarp0 = 3;
 constexpr int kTileBytes = kPos * kD * 2;   // 32 KB: [2 halves][128 rows][128 B]
 constexpr int kMaxBatch = 1024;             // requests per launch on this path
 
@@ -117,7 +119,7 @@ template <int NP>
 struct Cfg {
   static constexpr int kTiles = NP == 32 ? 7 : 8;            // tiles per chunk
   static constexpr int kChunk = kTiles * kPos;
-  static constexpr int kQBytes = 2 * NP * 128;               // [2 halves][NP rows][128 B]
+  static constexpr int kQBytes = 2 * NP * 128;               // one Q buffer: [2 halves][NP rows][128 B]
   static constexpr int kPTile = kPos * NP * 2;               // P^T tile: [128 pos][NP rows] bf16
   static constexpr int kPBytes = kTiles * kPTile;
   static constexpr uint32_t kPSwz = NP == 16 ? 6u : 4u;      // 32- / 64-byte swizzle
@@ -125,53 +127,36 @@ struct Cfg {
   static constexpr int kSCols = kTiles * NP;                 // one S buffer
   static constexpr int kOCol = 2 * kSCols;                   // two O buffers after two S buffers
   static_assert(kOCol + 2 * NP <= kTmemCols, "tensor memory budget");
-  static constexpr int kRingOff = 0;
-  static constexpr int kQOff = kStages * kTileBytes;
-  static constexpr int kPOff = kQOff + kQBytes;
+  static constexpr int kSmemMax = 227 * 1024;
+  static constexpr int kKRingOff = 0;
+  static constexpr int kVRingOff = kKStages * kTileBytes;
+  static constexpr int kQOff = (kKStages + kVStages) * kTileBytes;
+  static constexpr int kPOff = kQOff + 2 * kQBytes;         // two Q buffers (item parity)
   static constexpr int kRedOff = kPOff + kPBytes;            // redM, redL [8 warps][NP]; cm, cl [2][NP]
   static constexpr int kRedBytes = (2 * 8 * NP + 4 * NP) * 4;
   static constexpr int kPrefOff = kRedOff + kRedBytes;       // request prefix [kMaxBatch+1]
   static constexpr int kLenOff = kPrefOff + (kMaxBatch + 1) * 4;   // L per request [kMaxBatch]
   static constexpr int kRidOff = kLenOff + kMaxBatch * 4;          // request id [kMaxBatch]
-  static constexpr int kIdsOff = kRidOff + kMaxBatch * 4;          // page ids [2 items][64]
+  static constexpr int kIdsOff = kRidOff + kMaxBatch * 4;          // page ids [K, V producer][64]
   static constexpr int kBarOff = (kIdsOff + 2 * 64 * 4 + 63) / 64 * 64;
   static constexpr int kSmem = kBarOff + 256 + 1024;         // + barriers + alignment slack
+  static_assert(kSmem <= kSmemMax, "shared memory budget");
+  static_assert(kQOff % 1024 == 0 && kPOff % 1024 == 0 && kRedOff % 16 == 0 && kBarOff % 64 == 0,
+                "alignment of the swizzled operands, the reduction scratch and the barriers");
 };
 
 struct Bars {
-  uint64_t full[kStages], empty[kStages], tma[kStages];
+  uint64_t kfull[kKStages], kempty[kKStages], ktma[kKStages];
+  uint64_t vfull[kVStages], vempty[kVStages], vtma[kVStages];
   // one barrier pair per tensor-memory buffer (chunk parity), so that no barrier ever runs
   // two phases ahead of a waiter
-  uint64_t q_full, q_empty, p_full, fin;
+  uint64_t q_full[2], q_empty[2], p_full, fin;
   uint64_t s_full[2], s_empty[2], o_full[2], o_empty[2];
   uint32_t tmem_base;
   int abort_flag;
 };
 static_assert(sizeof(Bars) <= 256, "barrier block");
 
-// Warp-uniform bounded wait on an mbarrier phase (every lane observes the phase itself).
-// Gives up when another role raised the abort flag, or after kWaitLimit polls (then raises
-// it, with S3R_ERR_TIMEOUT in the error word).
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                         int* err) {
-  for (int i = 0; i < kWaitLimit; ++i) {
-    const bool done = mbar_try_wait(bar, parity);
-    if (__all_sync(kFull, done)) return true;
-    if ((i & 255) == 255 && __any_sync(kFull, *abort_flag != 0)) return false;
-  }
-  if ((threadIdx.x & 31) == 0) {
-    *abort_flag = 1;
-    set_error(err, S3R_ERR_TIMEOUT);
-  }
-  __syncwarp();
-  return false;
-}
-__device__ __forceinline__ bool aborted(volatile int* abort_flag) {
-  return __any_sync(kFull, *abort_flag != 0);
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
-}
 __device__ __forceinline__ void named_sync_softmax() {
   asm volatile("bar.sync 1, 256;\n" ::: "memory");
 }
@@ -214,7 +199,8 @@ __device__ __forceinline__ Item make_item(int it, const int* pref, const int* le
 
 template <int NP>
 __global__ void __launch_bounds__(kThreads, 1)
-    verify_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+    verify_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
+                     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      const __grid_constant__ CUtensorMap tmK8, const __grid_constant__ CUtensorMap tmV8,
                      const VerifyParams p, int batch) {
   using C = Cfg<NP>;
@@ -272,13 +258,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (tid < NP) trow[tid] = tid / G;
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(smem_u32(&B->full[s]), 1);
-      mbar_init(smem_u32(&B->empty[s]), 1);
-      mbar_init(smem_u32(&B->tma[s]), 1);
+    for (int s = 0; s < kKStages; ++s) {
+      mbar_init(smem_u32(&B->kfull[s]), 1);
+      mbar_init(smem_u32(&B->kempty[s]), 1);
+      mbar_init(smem_u32(&B->ktma[s]), 1);
     }
-    mbar_init(smem_u32(&B->q_full), 1);
-    mbar_init(smem_u32(&B->q_empty), 1);
+    for (int s = 0; s < kVStages; ++s) {
+      mbar_init(smem_u32(&B->vfull[s]), 1);
+      mbar_init(smem_u32(&B->vempty[s]), 1);
+      mbar_init(smem_u32(&B->vtma[s]), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&B->q_full[b]), 1);
+      mbar_init(smem_u32(&B->q_empty[b]), 1);
+    }
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&B->s_full[b]), 1);
       mbar_init(smem_u32(&B->s_empty[b]), 8);
@@ -291,7 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
     fence_proxy_async();
   }
-  if (warp == 1) {
+  if (warp == 2) {
     tmem_alloc(smem_u32(&B->tmem_base), C::kTmemCols);
     tmem_relinquish();
   }
@@ -303,37 +296,43 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int my_items = nitems > (int)blockIdx.x ? (nitems - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
   const uint32_t qbuf = sbase + C::kQOff, pbuf = sbase + C::kPOff;
 
-  if (warp == 0) {
-    // ===================================================================== producer ====
+  if (warp <= 1) {
+    // ============================================================ producers ====
+    // warp 0 streams the K tiles of every item (and its Q rows), warp 1 the V tiles, each
+    // through its own ring, so the two streams never wait on each other
+    const bool is_v = warp == 1;
     if (lane == 0) {
-      asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&tmK)) : "memory");
-      asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&tmV)) : "memory");
-      asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&tmK8)) : "memory");
-      asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&tmV8)) : "memory");
+      asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(is_v ? &tmV : &tmK)) : "memory");
+      asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(is_v ? &tmV8 : &tmK8)) : "memory");
+      if (!is_v) asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&tmQ)) : "memory");
     }
-    // ring order: K(0), then per item n: K(n+1), V(n) -- the MMA warp consumes in this order
+    const int nst = is_v ? kVStages : kKStages;
+    const int roff = is_v ? C::kVRingOff : C::kKRingOff;
+    uint64_t* full = is_v ? B->vfull : B->kfull;
+    uint64_t* empty = is_v ? B->vempty : B->kempty;
+    uint64_t* tmab = is_v ? B->vtma : B->ktma;
+    const CUtensorMap* map = is_v ? &tmV : &tmK;
+    const CUtensorMap* map8 = is_v ? &tmV8 : &tmK8;
+    const __nv_bfloat16* blk = is_v ? p.v_new : p.k_new;
+    int* ids_own = ids_s + (is_v ? 64 : 0);
     int g = 0;
     uint32_t tma_phase = 0;   // bit s: phase of tma[s]
     bool stop = false;
-    auto load_tiles = [&](const Item& x, bool is_v, const int* ids_item) {
-      const CUtensorMap* map = is_v ? &tmV : &tmK;
-      const CUtensorMap* map8 = is_v ? &tmV8 : &tmK8;
-      const __nv_bfloat16* blk = is_v ? p.v_new : p.k_new;
+    auto load_tiles = [&](const Item& x) {
       for (int t = 0; t < x.ntile && !stop; ++t, ++g) {
-        const int s = g % kStages;
-        if (g >= kStages &&
-            !wait_bar(smem_u32(&B->empty[s]), ((g / kStages) - 1) & 1, abort_flag, p.err)) {
+        const int s = g % nst;
+        if (g >= nst && !wait_bar(smem_u32(&empty[s]), ((g / nst) - 1) & 1, abort_flag, p.err)) {
           stop = true;
           break;
         }
         const int t0 = x.start + t * kPos;
-        const uint32_t dst = sbase + C::kRingOff + s * kTileBytes;
+        const uint32_t dst = sbase + roff + s * kTileBytes;
         uint32_t okmask = 0;
         int nload = 0;
         bool tail = (t0 + kPos > x.L);
         int ids[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) ids[i] = ids_item[t * 8 + i];
+        for (int i = 0; i < 8; ++i) ids[i] = ids_own[t * 8 + i];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const int pg = (t0 >> 4) + i;
@@ -347,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        const uint32_t landing = smem_u32(tail ? &B->tma[s] : &B->full[s]);
+        const uint32_t landing = smem_u32(tail ? &tmab[s] : &full[s]);
         if (lane == 0) mbar_arrive_expect_tx(landing, (uint32_t)(nload * kPage * kD * 2));
         __syncwarp();
         bool run = okmask == 0xFFu && !tail;   // 8 consecutive page ids: 2 boxes of 8 pages
@@ -363,7 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (tail) {
           // wait for the committed rows, then write block rows / zeros over the rest
-          if (!wait_bar(smem_u32(&B->tma[s]), (tma_phase >> s) & 1, abort_flag, p.err)) {
+          if (!wait_bar(smem_u32(&tmab[s]), (tma_phase >> s) & 1, abort_flag, p.err)) {
             stop = true;
             break;
           }
@@ -376,29 +375,60 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (pos >= x.L && pos < x.Lc)
               v = *reinterpret_cast<const uint4*>(blk + (((size_t)x.r * T + (pos - x.L)) * Hkv + x.kvh) * kD + ch * 8);
             const uint32_t off = (ch >> 3) * (kPos * 128) + row * 128 + (((ch & 7) ^ (row & 7)) << 4);
-            *reinterpret_cast<uint4*>(smem + C::kRingOff + s * kTileBytes + off) = v;
+            *reinterpret_cast<uint4*>(smem + roff + s * kTileBytes + off) = v;
           }
           fence_proxy_async();
           __syncwarp();
-          if (lane == 0) mbar_arrive(smem_u32(&B->full[s]));
+          if (lane == 0) mbar_arrive(smem_u32(&full[s]));
         }
         __syncwarp();
       }
     };
-    auto load_q_and_k = [&](int m) {
-      const Item x = make_item<NP>(blockIdx.x + m * gridDim.x, pref, lens_s, rid_s, batch, p);
-      const int* ptab = p.page_table + (size_t)x.r * p.max_pages;
-      // page ids of the item's committed pages (-1 past L), read once for its K and V tiles
-      int* ids_item = ids_s + (m & 1) * 64;
-      {
-        const int npg = x.ntile * 8;
-        const int pg0 = x.start >> 4;
-        const int a = lane < npg && (pg0 + lane) * kPage < x.L ? ptab[pg0 + lane] : -1;
-        const int b = lane + 32 < npg && (pg0 + lane + 32) * kPage < x.L ? ptab[pg0 + lane + 32] : -1;
-        ids_item[lane] = a;
-        ids_item[lane + 32] = b;
+    if (!is_v) {
+      // Q padding rows R..NP-1 of both halves of both buffers stay zero: the Q copies
+      // write rows < R only
+      for (int idx = lane; idx < 4 * (NP - R) * 8; idx += 32) {
+        const int h = idx / ((NP - R) * 8), rem = idx - h * (NP - R) * 8;   // h: buffer*2 + half
+        *reinterpret_cast<uint4*>(smem + C::kQOff + h * (NP * 128) + (R + (rem >> 3)) * 128 +
+                                  ((rem & 7) << 4)) = make_uint4(0, 0, 0, 0);
       }
-      if (x.c == 0) {   // the block's K/V enter the cache once per (request, head)
+      fence_proxy_async();
+      __syncwarp();
+    }
+    // page ids of an item's committed pages (-1 past L), two per lane, loaded one item ahead
+    auto fetch_ids = [&](const Item& x, int& a, int& b) {
+      const int* ptab = p.page_table + (size_t)x.r * p.max_pages;
+      const int npg = x.ntile * 8;
+      const int pg0 = x.start >> 4;
+      a = lane < npg && (pg0 + lane) * kPage < x.L ? ptab[pg0 + lane] : -1;
+      b = lane + 32 < npg && (pg0 + lane + 32) * kPage < x.L ? ptab[pg0 + lane + 32] : -1;
+    };
+    int next_a = -1, next_b = -1;
+    for (int m = 0; m < my_items && !stop && !aborted(abort_flag); ++m) {
+      const Item x = make_item<NP>(blockIdx.x + m * gridDim.x, pref, lens_s, rid_s, batch, p);
+      int a = next_a, b = next_b;
+      if (m == 0) fetch_ids(x, a, b);
+      __syncwarp();   // every lane is done with the previous item's ids
+      ids_own[lane] = a;
+      ids_own[lane + 32] = b;
+      if (m + 1 < my_items)
+        fetch_ids(make_item<NP>(blockIdx.x + (m + 1) * gridDim.x, pref, lens_s, rid_s, batch, p),
+                  next_a, next_b);
+      __syncwarp();
+      if (!is_v) {
+        // Q rows -> Q buffer m&1 by TMA (K-major, 128-byte swizzle) once QK(m-2) has read it
+        const int qb = m & 1;
+        if (m >= 2 && !wait_bar(smem_u32(&B->q_empty[qb]), ((m - 2) >> 1) & 1, abort_flag, p.err)) break;
+        if (lane == 0) mbar_arrive_expect_tx(smem_u32(&B->q_full[qb]), (uint32_t)(2 * R * 128));
+        __syncwarp();
+        if (lane < 2)
+          tma_load_3d(qbuf + qb * C::kQBytes + lane * (NP * 128), &tmQ, lane * 64, x.kvh * G,
+                      x.r * T, smem_u32(&B->q_full[qb]));
+        __syncwarp();
+      }
+      load_tiles(x);
+      if (!is_v && x.c == 0 && !stop) {   // the block's K/V enter the cache once per (request, head)
+        const int* ptab = p.page_table + (size_t)x.r * p.max_pages;
         for (int idx = lane; idx < T * (kD / 8); idx += 32) {
           const int t = idx / (kD / 8), ch = idx - t * (kD / 8);
           const int pos = x.L + t;
@@ -413,112 +443,119 @@ __global__ void __launch_bounds__(kThreads, 1)
           *reinterpret_cast<uint4*>(p.v_pool + dst) = *reinterpret_cast<const uint4*>(p.v_new + src);
         }
       }
-      // Q rows -> qbuf (K-major, 128-byte swizzle, zero padding rows), once QK(m-1) is done
-      constexpr int kPer = NP * (kD / 8) / 32;
-      uint4 qv[kPer];
-#pragma unroll
-      for (int i = 0; i < kPer; ++i) {
-        const int idx = lane + 32 * i;
-        const int row = idx / (kD / 8), ch = idx - row * (kD / 8);
-        qv[i] = make_uint4(0, 0, 0, 0);
-        if (row < R) {
-          const int t = row / G, gg = row - t * G;
-          qv[i] = __ldg(reinterpret_cast<const uint4*>(
-              p.q + (((size_t)x.r * T + t) * Hq + x.kvh * G + gg) * kD + ch * 8));
-        }
-      }
-      if (m > 0 && !wait_bar(smem_u32(&B->q_empty), (m - 1) & 1, abort_flag, p.err)) {
-        stop = true;
-        return;
-      }
-#pragma unroll
-      for (int i = 0; i < kPer; ++i) {
-        const int idx = lane + 32 * i;
-        const int row = idx / (kD / 8), ch = idx - row * (kD / 8);
-        const uint32_t off = (ch >> 3) * (NP * 128) + row * 128 + (((ch & 7) ^ (row & 7)) << 4);
-        *reinterpret_cast<uint4*>(smem + C::kQOff + off) = qv[i];
-      }
-      fence_proxy_async();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&B->q_full));
-      load_tiles(x, false, ids_item);
-    };
-    if (my_items > 0) load_q_and_k(0);
-    for (int n = 0; n < my_items && !stop && !aborted(abort_flag); ++n) {
-      if (n + 1 < my_items) load_q_and_k(n + 1);
-      if (stop) break;
-      load_tiles(make_item<NP>(blockIdx.x + n * gridDim.x, pref, lens_s, rid_s, batch, p), true,
-                 ids_s + (n & 1) * 64);
     }
-  } else if (warp == 1) {
+    // nothing may still be landing in this ring when the CTA exits
+    for (int q = g - nst > 0 ? g - nst : 0; q < g; ++q) mbar_wait(smem_u32(&full[q % nst]), (q / nst) & 1);
+  } else if (warp == 2) {
     // ====================================================================== MMA warp ===
+    // Two queues in issue order: QK of item m (its K tiles) and PV of item n < m (its V
+    // tiles, once the softmax has written P^T). Whichever has its next tile ready is issued,
+    // so a V tile never waits behind K tiles of the next item, nor the reverse.
     constexpr uint32_t kIdQK = idesc_bf16(kPos, NP, false, false);
     constexpr uint32_t kIdPV = idesc_bf16(kD, NP, true, true);
-    int g = 0;
-    bool ok = true;
-    auto qk = [&](int m) {
-      const Item x = make_item<NP>(blockIdx.x + m * gridDim.x, pref, lens_s, rid_s, batch, p);
-      ok = wait_bar(smem_u32(&B->q_full), m & 1, abort_flag, p.err);
-      if (ok && m >= 2) ok = wait_bar(smem_u32(&B->s_empty[m & 1]), ((m - 2) >> 1) & 1, abort_flag, p.err);
-      if (!ok) return;
-      tc_fence_after();
-      const uint32_t sd = tmem + (m & 1) * C::kSCols;
-      for (int t = 0; t < x.ntile; ++t, ++g) {
-        const int s = g % kStages;
-        ok = wait_bar(smem_u32(&B->full[s]), (g / kStages) & 1, abort_flag, p.err);
-        if (!ok) return;
-        tc_fence_after();
-        if (lane == 0) {
-          const uint32_t kt = sbase + C::kRingOff + s * kTileBytes;
-#pragma unroll
-          for (int kk = 0; kk < kD / 16; ++kk) {
-            const uint64_t ad = sdesc(kt + (kk >> 2) * (kPos * 128) + (kk & 3) * 32, 16, 1024, 2);
-            const uint64_t bd = sdesc(qbuf + (kk >> 2) * (NP * 128) + (kk & 3) * 32, 16, 1024, 2);
-            tc_mma(sd + t * NP, ad, bd, kIdQK, kk > 0 ? 1u : 0u);
-          }
-          tc_commit(smem_u32(&B->empty[s]));
-        }
-        __syncwarp();
-      }
-      if (lane == 0) {
-        tc_commit(smem_u32(&B->s_full[m & 1]));
-        tc_commit(smem_u32(&B->q_empty));
-      }
-      __syncwarp();
+    auto ready = [&](uint64_t* bar, uint32_t parity) -> bool {   // warp-uniform test
+      const bool r = lane == 0 ? mbar_test(smem_u32(bar), parity) : false;
+      return __shfl_sync(kFull, r ? 1 : 0, 0) != 0;
     };
-    auto pv = [&](int n) {
-      const Item x = make_item<NP>(blockIdx.x + n * gridDim.x, pref, lens_s, rid_s, batch, p);
-      ok = wait_bar(smem_u32(&B->p_full), n & 1, abort_flag, p.err);
-      if (ok && n >= 2) ok = wait_bar(smem_u32(&B->o_empty[n & 1]), ((n - 2) >> 1) & 1, abort_flag, p.err);
-      if (!ok) return;
-      tc_fence_after();
-      const uint32_t od = tmem + C::kOCol + (n & 1) * NP;
-      for (int t = 0; t < x.ntile; ++t, ++g) {
-        const int s = g % kStages;
-        ok = wait_bar(smem_u32(&B->full[s]), (g / kStages) & 1, abort_flag, p.err);
-        if (!ok) return;
-        tc_fence_after();
-        if (lane == 0) {
-          const uint32_t vt = sbase + C::kRingOff + s * kTileBytes;
-          const uint32_t pt = pbuf + t * C::kPTile;
-#pragma unroll
-          for (int kk = 0; kk < kPos / 16; ++kk) {
-            const uint64_t ad = sdesc(vt + kk * 2048, kPos * 128, 1024, 2);
-            const uint64_t bd = sdesc(pt + kk * 16 * NP * 2, NP * 2 * 8, 8 * NP * 2, C::kPSwz);
-            tc_mma(od, ad, bd, kIdPV, (t > 0 || kk > 0) ? 1u : 0u);
-          }
-          tc_commit(smem_u32(&B->empty[s]));
+    int mk = 0, tk = 0, gk = 0, nv = 0, tv = 0, gv = 0;
+    bool kgo = false, vgo = false, ok = true;
+    Item xk{}, xv{};
+    if (my_items > 0) {
+      xk = make_item<NP>(blockIdx.x, pref, lens_s, rid_s, batch, p);
+      xv = xk;
+    }
+    uint32_t idle = 0;
+    while (ok && (mk < my_items || nv < my_items)) {
+      bool did = false;
+      if (mk < my_items) {
+        if (!kgo) {
+          kgo = ready(&B->q_full[mk & 1], (mk >> 1) & 1) &&
+                (mk < 2 || ready(&B->s_empty[mk & 1], ((mk - 2) >> 1) & 1));
+          if (kgo) tc_fence_after();
         }
-        __syncwarp();
+        if (kgo) {
+          const int s = gk % kKStages;
+          if (ready(&B->kfull[s], (gk / kKStages) & 1)) {
+            tc_fence_after();
+            if (lane == 0) {
+              const uint32_t kt = sbase + C::kKRingOff + s * kTileBytes;
+              const uint32_t sd = tmem + (mk & 1) * C::kSCols + tk * NP;
+#pragma unroll
+              for (int kk = 0; kk < kD / 16; ++kk) {
+                const uint64_t ad = sdesc(kt + (kk >> 2) * (kPos * 128) + (kk & 3) * 32, 16, 1024, 2);
+                const uint64_t bd = sdesc(qbuf + (mk & 1) * C::kQBytes + (kk >> 2) * (NP * 128) +
+                                              (kk & 3) * 32, 16, 1024, 2);
+                tc_mma(sd, ad, bd, kIdQK, kk > 0 ? 1u : 0u);
+              }
+              tc_commit(smem_u32(&B->kempty[s]));
+            }
+            __syncwarp();
+            ++tk;
+            ++gk;
+            did = true;
+            if (tk == xk.ntile) {
+              if (lane == 0) {
+                tc_commit(smem_u32(&B->s_full[mk & 1]));
+                tc_commit(smem_u32(&B->q_empty[mk & 1]));
+              }
+              __syncwarp();
+              ++mk;
+              tk = 0;
+              kgo = false;
+              if (mk < my_items) xk = make_item<NP>(blockIdx.x + mk * gridDim.x, pref, lens_s, rid_s, batch, p);
+            }
+          }
+        }
       }
-      if (lane == 0) tc_commit(smem_u32(&B->o_full[n & 1]));
-      __syncwarp();
-    };
-    if (my_items > 0) qk(0);
-    for (int n = 0; n < my_items && ok && !aborted(abort_flag); ++n) {
-      if (n + 1 < my_items) qk(n + 1);
-      if (!ok) break;
-      pv(n);
+      if (nv < mk) {
+        if (!vgo) {
+          vgo = ready(&B->p_full, nv & 1) &&
+                (nv < 2 || ready(&B->o_empty[nv & 1], ((nv - 2) >> 1) & 1));
+          if (vgo) tc_fence_after();
+        }
+        if (vgo) {
+          const int s = gv % kVStages;
+          if (ready(&B->vfull[s], (gv / kVStages) & 1)) {
+            tc_fence_after();
+            if (lane == 0) {
+              const uint32_t vt = sbase + C::kVRingOff + s * kTileBytes;
+              const uint32_t pt = pbuf + tv * C::kPTile;
+              const uint32_t od = tmem + C::kOCol + (nv & 1) * NP;
+#pragma unroll
+              for (int kk = 0; kk < kPos / 16; ++kk) {
+                const uint64_t ad = sdesc(vt + kk * 2048, kPos * 128, 1024, 2);
+                const uint64_t bd = sdesc(pt + kk * 16 * NP * 2, NP * 2 * 8, 8 * NP * 2, C::kPSwz);
+                tc_mma(od, ad, bd, kIdPV, (tv > 0 || kk > 0) ? 1u : 0u);
+              }
+              tc_commit(smem_u32(&B->vempty[s]));
+            }
+            __syncwarp();
+            ++tv;
+            ++gv;
+            did = true;
+            if (tv == xv.ntile) {
+              if (lane == 0) tc_commit(smem_u32(&B->o_full[nv & 1]));
+              __syncwarp();
+              ++nv;
+              tv = 0;
+              vgo = false;
+              if (nv < my_items) xv = make_item<NP>(blockIdx.x + nv * gridDim.x, pref, lens_s, rid_s, batch, p);
+            }
+          }
+        }
+      }
+      if (did) {
+        idle = 0;
+      } else if (++idle >= (uint32_t)kWaitLimit) {
+        if (lane == 0) {
+          *abort_flag = 1;
+          set_error(p.err, S3R_ERR_TIMEOUT);
+        }
+        ok = false;
+      } else {
+        if ((idle & 1023) == 0 && aborted(abort_flag)) ok = false;
+        __nanosleep(32);
+      }
     }
     // make sure nothing issued is still running before the tensor memory goes away
     if (lane == 0) tc_commit(smem_u32(&B->fin));
@@ -526,10 +563,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     wait_bar(smem_u32(&B->fin), 0, abort_flag, p.err);
   } else {
     // ================================================================ softmax warps ===
-    const int sw8 = warp - 2;                // 0..7
+    const int sw8 = warp - kSoftWarp0;       // 0..7
     const int sg = sw8 >> 2;                 // warpgroup: tiles t with t % 2 == sg
     const int q4 = warp & 3;                 // tensor-memory lane quarter of this warp
-    const int st = tid - 64;                 // 0..255 within the softmax warps
+    const int st = tid - 32 * kSoftWarp0;    // 0..255 within the softmax warps
     const int lrow = q4 * 32 + lane;         // tile position (S) or d (O) of this thread
     const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
     const float scale = p.scale, scale2 = p.scale * kLog2e;
@@ -564,7 +601,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int n = 0; n < my_items && !aborted(abort_flag); ++n) {
       const Item x = make_item<NP>(blockIdx.x + n * gridDim.x, pref, lens_s, rid_s, batch, p);
       const int L = x.L, start = x.start, end = x.end;
-      float* scores = p.scores ? p.scores + ((size_t)x.r * Hkv + x.kvh) * (size_t)p.cap * R : nullptr;
+      float* scores = p.scores ? p.scores + ((size_t)x.r * Hkv + x.kvh) * (size_t)R * p.cap : nullptr;
       if (!wait_bar(smem_u32(&B->s_full[n & 1]), (n >> 1) & 1, abort_flag, p.err)) {
         ok = false;
         break;
@@ -583,18 +620,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int t0 = start + t * kPos;
         const int pos = t0 + lrow;
         if (scores && pos < L) {
-          float* dst = scores + (size_t)pos * R;
-          if ((R & 3) == 0) {
+          // committed logits, [row][position]: the warp's 32 lanes write 32 consecutive
+          // positions of one row per store, one whole 128-byte line
 #pragma unroll
-            for (int j = 0; j < NP; j += 4)
-              if (j < R)
-                *reinterpret_cast<float4*>(dst + j) =
-                    make_float4(v[j] * scale, v[j + 1] * scale, v[j + 2] * scale, v[j + 3] * scale);
-          } else {
-#pragma unroll
-            for (int j = 0; j < NP; ++j)
-              if (j < R) dst[j] = v[j] * scale;
-          }
+          for (int j = 0; j < NP; ++j)
+            if (j < R) scores[(size_t)j * p.cap + pos] = v[j] * scale;
         }
         if (t0 + kPos <= min(L, end)) {
 #pragma unroll
@@ -695,7 +725,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 2) {
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
   }
@@ -706,9 +736,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 int verify_tc_npad(int R) { return R <= 16 ? 16 : (R <= 32 ? 32 : 0); }
 
 template <int NP>
-static int launch_tc(const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tk8,
-                     const CUtensorMap& tv8, const VerifyParams& p, int batch, int num_sms,
-                     cudaStream_t stream) {
+static int launch_tc(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                     const CUtensorMap& tk8, const CUtensorMap& tv8, const VerifyParams& p,
+                     int batch, int num_sms, cudaStream_t stream) {
   using C = tc::Cfg<NP>;
   static bool attr_done = false;
   if (!attr_done) {
@@ -718,7 +748,8 @@ static int launch_tc(const CUtensorMap& tk, const CUtensorMap& tv, const CUtenso
       return S3R_ERR_CUDA;
     attr_done = true;
   }
-  tc::verify_tc_kernel<NP><<<num_sms, tc::kThreads, C::kSmem, stream>>>(tk, tv, tk8, tv8, p, batch);
+  tc::verify_tc_kernel<NP><<<num_sms, tc::kThreads, C::kSmem, stream>>>(tq, tk, tv, tk8, tv8, p,
+                                                                        batch);
   return cuda_status(cudaGetLastError(), __func__);
 }
 
@@ -731,12 +762,12 @@ int verify_tc_chunk(int R) {
   return np == 16 ? tc::Cfg<16>::kChunk : tc::Cfg<32>::kChunk;
 }
 
-int launch_verify_tc(const CUtensorMap& k1, const CUtensorMap& v1, const CUtensorMap& k8,
-                     const CUtensorMap& v8, const VerifyParams& p, int batch, int num_sms,
-                     cudaStream_t stream) {
+int launch_verify_tc(const CUtensorMap& qm, const CUtensorMap& k1, const CUtensorMap& v1,
+                     const CUtensorMap& k8, const CUtensorMap& v8, const VerifyParams& p,
+                     int batch, int num_sms, cudaStream_t stream) {
   const int np = verify_tc_npad(p.R);
-  if (np == 16) return launch_tc<16>(k1, v1, k8, v8, p, batch, num_sms, stream);
-  if (np == 32) return launch_tc<32>(k1, v1, k8, v8, p, batch, num_sms, stream);
+  if (np == 16) return launch_tc<16>(qm, k1, v1, k8, v8, p, batch, num_sms, stream);
+  if (np == 32) return launch_tc<32>(qm, k1, v1, k8, v8, p, batch, num_sms, stream);
   return S3R_ERR_UNSUPPORTED;
 }
 

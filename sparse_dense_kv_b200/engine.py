@@ -27,7 +27,7 @@ class RoundBuffers:
                  sel_stride, device="cuda"):
         G = num_q_heads // num_kv_heads
         f32, bf, i32 = torch.float32, torch.bfloat16, torch.int32
-        self.scores = torch.empty((num_requests, num_kv_heads, cap, G * (k + 1)), dtype=f32, device=device)
+        self.scores = torch.empty((num_requests, num_kv_heads, G * (k + 1), cap), dtype=f32, device=device)
         self.lse = torch.empty((num_requests, k + 1, num_q_heads), dtype=f32, device=device)
         self.prefill_lse = torch.empty((num_requests, 1, num_q_heads), dtype=f32, device=device)
         self.sel_idx = torch.zeros((num_requests, num_kv_heads, sel_stride), dtype=i32, device=device)
@@ -87,15 +87,21 @@ class S3REngine:
         L.s3r_select_kv(self.cache, self.batch, b.scores, lse, self.k_prev, self.budget_bp,
                         self.window, b.sel_idx, b.sel_count, self.ws)
 
-    def draft_step(self, i, q_block, k_block, v_block, q_logits, draft_logits_fn=None):
+    def draft_attn(self, i, q_block, k_block, v_block):
         b = self.buf
         L.s3r_sparse_draft_attn(self.cache, self.batch, b.steps[i], q_block[:, i], k_block[:, i],
                                 v_block[:, i], b.sel_idx, b.sel_count, b.draft_out, b.draft_lse,
                                 self.ws)
+
+    def draft_sample(self, i, q_logits):
+        L.s3r_draft_sample(self.batch, self.buf.steps[i], self.k, q_logits, self.vocab, self.seed,
+                           self.buf.draft_tokens, self.ws)
+
+    def draft_step(self, i, q_block, k_block, v_block, q_logits, draft_logits_fn=None):
+        self.draft_attn(i, q_block, k_block, v_block)
         if draft_logits_fn is not None:
-            draft_logits_fn(i, b.draft_out, q_logits)
-        L.s3r_draft_sample(self.batch, b.steps[i], self.k, q_logits, self.vocab, self.seed,
-                           b.draft_tokens, self.ws)
+            draft_logits_fn(i, self.buf.draft_out, q_logits)
+        self.draft_sample(i, q_logits)
 
     def verify(self, q_block, k_block, v_block):
         b = self.buf
@@ -129,3 +135,96 @@ class S3REngine:
     def check_errors(self) -> int:
         """Synchronise and return (and clear) the device error bitmask."""
         return L.s3r_get_error(self.ws)
+
+    def capture(self, step):
+        """Record `step()` (library calls on fixed device buffers) into a CUDA graph once;
+        replaying it issues the same launches with no host work per launch. `step` runs once
+        eagerly on a side stream first, so one-time host set-up (kernel attributes) is done
+        before capture. Returns (graph, launches recorded per replay)."""
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            step()
+        torch.cuda.current_stream().wait_stream(side)
+        g = torch.cuda.CUDAGraph()
+        before = L.s3r_launch_count()
+        with torch.cuda.graph(g):
+            step()
+        return g, L.s3r_launch_count() - before
+
+
+class MixedPhaseDriver:
+    """Requests at different points of their rounds, advanced one phase per iteration with
+    launches over request subsets (req_ids): phase i < k is draft step i, phase k is the
+    verify, speculative sampling and commit, followed at once by the selection of the
+    request's next round. One iteration issues one draft-attention and one draft-sampling
+    launch for every drafting request (each reads its own step from the step array), one
+    verify, one speculative-sampling pass, one commit and one selection for the verifying
+    requests.
+
+    Which request is in which phase is host bookkeeping (a numpy array); the kernels see only
+    the request-id lists and the per-request step array.
+    """
+
+    def __init__(self, engine: S3REngine, phases):
+        import numpy as np
+        self.e = engine
+        self.phases = np.asarray(phases, dtype=np.int64).copy()
+        if self.phases.shape != (engine.num_requests,) or self.phases.min() < 0 or \
+                self.phases.max() > engine.k:
+            raise ValueError("one phase in 0..k per request")
+        dev = engine.k_pool.device
+        self.step = torch.zeros((engine.num_requests,), dtype=torch.int32, device=dev)
+        self._dev = dev
+
+    def _batch(self, ids):
+        t = torch.as_tensor(ids, dtype=torch.int32, device=self._dev)
+        return L.make_batch(self.e.seq_lens, self.e.page_table, req_ids=t)
+
+    def start(self, q_block, k_block, v_block, q_logits):
+        """After prefill: every request selects its first sparse set from the prefill scores,
+        then drafts the steps before its phase (a request at phase p has drafted 0..p-1)."""
+        import numpy as np
+        e = self.e
+        e.select()
+        for i in range(e.k):
+            ids = np.nonzero(self.phases > i)[0]
+            if ids.size:
+                self._draft(ids, np.full(ids.size, i), q_block, k_block, v_block, q_logits)
+
+    def _draft(self, ids, steps, q_block, k_block, v_block, q_logits):
+        import numpy as np
+        e, b = self.e, self.e.buf
+        st = np.zeros(e.num_requests, dtype=np.int32)
+        st[ids] = steps
+        self.step.copy_(torch.as_tensor(st), non_blocking=False)
+        rows = torch.as_tensor(st, dtype=torch.long, device=self._dev)
+        ar = torch.arange(e.num_requests, device=self._dev)
+        # the current token of each request (its own step) -- model output in a real system
+        qc = q_block[ar, rows].contiguous()
+        kc = k_block[ar, rows].contiguous()
+        vc = v_block[ar, rows].contiguous()
+        batch = self._batch(ids)
+        L.s3r_sparse_draft_attn(e.cache, batch, self.step, qc, kc, vc, b.sel_idx, b.sel_count,
+                                b.draft_out, b.draft_lse, e.ws)
+        L.s3r_draft_sample(batch, self.step, e.k, q_logits, e.vocab, e.seed, b.draft_tokens, e.ws)
+
+    def iterate(self, q_block, k_block, v_block, p_logits, q_logits):
+        """Advance every request by one phase; returns the ids that completed a round."""
+        import numpy as np
+        e, b = self.e, self.e.buf
+        d_ids = np.nonzero(self.phases < e.k)[0]
+        v_ids = np.nonzero(self.phases == e.k)[0]
+        if d_ids.size:
+            self._draft(d_ids, self.phases[d_ids], q_block, k_block, v_block, q_logits)
+        if v_ids.size:
+            batch = self._batch(v_ids)
+            L.s3r_verify_attn(e.cache, batch, e.k, q_block, k_block, v_block, b.verify_out, b.lse,
+                              b.scores, e.ws)
+            L.s3r_spec_sample(batch, e.k, p_logits, q_logits, b.draft_tokens, e.vocab, e.seed,
+                              b.out_tokens, b.n_out, e.ws)
+            L.s3r_commit(batch, e.k, b.n_out, e.seq_lens, b.stats)
+            L.s3r_select_kv(e.cache, batch, b.scores, b.lse, e.k, e.budget_bp, e.window,
+                            b.sel_idx, b.sel_count, e.ws)
+        self.phases = (self.phases + 1) % (e.k + 1)
+        return v_ids

@@ -22,7 +22,7 @@ def run_verify(case, k, seed, scores=True):
     lse = torch.empty((NR, T, Hq), dtype=torch.float32, device="cuda")
     cap = case.cache.capacity
     G = Hq // Hkv
-    sc = torch.full((NR, Hkv, cap, G * T), float("nan"), device="cuda") if scores else None
+    sc = torch.full((NR, Hkv, G * T, cap), float("nan"), device="cuda") if scores else None
     cache = s3r.make_cache(case.k_pool, case.v_pool, Hq)
     batch = s3r.make_batch(case.seq_lens, case.page_table)
     ws = s3r.new_workspace(s3r.s3r_workspace_size(cache, NR, case.cache.max_pages, k, 64, 64))
@@ -52,8 +52,9 @@ def test_verify_matches_oracle(Hq, Hkv, d, k, lens):
         o, l, sigma, logits = O.verify_attention(f64(q[r]), K, V, int(L))
         assert_attention_close(f64(out[r]), o, f"out r={r}")
         np.testing.assert_allclose(f64(lse[r]), l, rtol=0, atol=2e-4)
-        got = f64(sc[r][:, :L, :])                      # [H_kv][position][row]
-        np.testing.assert_allclose(got, logits[:, :, :L].transpose(0, 2, 1), rtol=1e-5, atol=1e-4)
+        got = f64(sc[r][:, :, :L])                      # [H_kv][row][position]
+        np.testing.assert_allclose(got, logits[:, :, :L], rtol=1e-5, atol=1e-4)
+        assert torch.isnan(sc[r][:, :, L:]).all()       # nothing written past L
 
 
 @pytest.mark.parametrize("Hq,Hkv,k,lens", [
@@ -80,8 +81,7 @@ def test_verify_kernels_agree_with_oracle(Hq, Hkv, k, lens):
             o, l, _, logits = O.verify_attention(f64(q[r]), K, V, int(L))
             assert_attention_close(f64(out[r]), o, f"kernel {which} out r={r}")
             np.testing.assert_allclose(f64(lse[r]), l, rtol=0, atol=2e-4)
-            np.testing.assert_allclose(f64(sc[r][:, :L, :]), logits[:, :, :L].transpose(0, 2, 1),
-                                       rtol=1e-5, atol=1e-4)
+            np.testing.assert_allclose(f64(sc[r][:, :, :L]), logits[:, :, :L], rtol=1e-5, atol=1e-4)
     (o1, l1, s1), (o0, l0, s0) = outs
     assert (o1.float() - o0.float()).abs().max().item() < 2e-2
     assert (l1 - l0).abs().max().item() < 1e-3
@@ -99,8 +99,9 @@ def test_verify_without_score_capture_and_full_capacity():
         assert_attention_close(f64(out[r]), o, f"out r={r}")
 
 
-def draft_case(Hq, Hkv, d, lens, steps, budget_bp, window, seed):
-    spec = spec_for(Hq, Hkv, d, lens, budget_bp=budget_bp, window=window, seed=seed)
+def draft_case(Hq, Hkv, d, lens, steps, budget_bp, window, seed, shuffle=False, req_ids=None):
+    spec = spec_for(Hq, Hkv, d, lens, budget_bp=budget_bp, window=window, seed=seed,
+                    shuffle=shuffle)
     case = Case(spec, extra_tokens=16)
     NR = len(lens)
     rng = np.random.default_rng(seed)
@@ -117,10 +118,11 @@ def draft_case(Hq, Hkv, d, lens, steps, budget_bp, window, seed):
     kn = synth.randn_bf16((NR, Hkv, d), seed + 2, "cuda")
     vn = synth.randn_bf16((NR, Hkv, d), seed + 3, "cuda")
     step = torch.as_tensor(steps, dtype=torch.int32).cuda()
-    out = torch.empty_like(q)
-    lse = torch.empty((NR, Hq), dtype=torch.float32, device="cuda")
+    out = torch.full_like(q, float("nan"))
+    lse = torch.full((NR, Hq), float("nan"), dtype=torch.float32, device="cuda")
     cache = s3r.make_cache(case.k_pool, case.v_pool, Hq)
-    batch = s3r.make_batch(case.seq_lens, case.page_table)
+    rid = None if req_ids is None else torch.as_tensor(req_ids, dtype=torch.int32).cuda()
+    batch = s3r.make_batch(case.seq_lens, case.page_table, req_ids=rid)
     ws = s3r.new_workspace(s3r.s3r_workspace_size(cache, NR, case.cache.max_pages, 8, 64, stride))
     s3r.s3r_sparse_draft_attn(cache, batch, step, q, kn, vn, sel_idx.cuda(), sel_cnt.cuda(), out,
                               lse, ws)
@@ -145,6 +147,41 @@ def test_sparse_draft_matches_oracle(Hq, Hkv, d, lens, steps, bp, W):
         o, l = O.sparse_draft_attention(f64(q[r]), K, V, sels[r], int(L), i)
         assert_attention_close(f64(out[r]), o, f"draft r={r}")
         np.testing.assert_allclose(f64(lse[r]), l, rtol=0, atol=2e-4)
+
+
+def test_sparse_draft_many_items_per_cta():
+    """More (request, head, chunk) items than SMs, so each persistent CTA walks several items
+    and reuses its ring and tables; shuffled pages, ragged budgets, mixed steps."""
+    rng = np.random.default_rng(8)
+    lens = rng.integers(1200, 4200, size=48).tolist()
+    steps = rng.integers(0, 6, size=48).tolist()
+    case, sels, q, kn, vn, out, lse = draft_case(16, 8, 128, lens, steps, 2000, 64, seed=31,
+                                                 shuffle=True)
+    kp, vp = case.host_pools()
+    for r, L in enumerate(case.lens):
+        i = steps[r]
+        K, V = case.dense(r, L + i + 1, (kp, vp))
+        o, l = O.sparse_draft_attention(f64(q[r]), K, V, sels[r], int(L), i)
+        assert_attention_close(f64(out[r]), o, f"draft r={r}")
+        np.testing.assert_allclose(f64(lse[r]), l, rtol=0, atol=2e-4)
+
+
+def test_sparse_draft_request_subset():
+    """A launch over req_ids (a mixed-phase batch) writes only those requests."""
+    lens = [900, 2500, 1700, 3100, 640, 2000]
+    steps = [2, 0, 5, 1, 3, 4]
+    ids = [5, 1, 3]
+    case, sels, q, kn, vn, out, lse = draft_case(32, 8, 128, lens, steps, 1000, 64, seed=13,
+                                                 req_ids=ids)
+    kp, vp = case.host_pools()
+    for r, L in enumerate(case.lens):
+        if r not in ids:
+            assert torch.isnan(out[r].float()).all() and torch.isnan(lse[r]).all()
+            continue
+        i = steps[r]
+        K, V = case.dense(r, L + i + 1, (kp, vp))
+        o, l = O.sparse_draft_attention(f64(q[r]), K, V, sels[r], int(L), i)
+        assert_attention_close(f64(out[r]), o, f"draft r={r}")
 
 
 def test_sparse_draft_full_budget_equals_verify_row():

@@ -1,0 +1,149 @@
+"""Whole-workload GPU runs against the oracle: the mixed-phase ragged batch (requests at
+different points of their rounds, launches over request subsets, shuffled pages) and the
+full-size Qwen3-shaped workloads on sampled requests.
+
+Per request the GPU's round must equal the oracle's round on the same inputs: attention
+outputs within 2e-2 + 1e-2 |oracle|, selections, drafts and emitted tokens bit-exact unless
+the oracle's margin to a decision boundary is below 1e-5 (counted)."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+import sparse_dense_kv_b200 as s3r
+from oracle import s3r_oracle as O
+from tests.s3r_testlib import MARGIN, assert_attention_close, f64
+
+pytestmark = pytest.mark.gpu
+
+
+def _inputs(spec, lens, device="cuda"):
+    """q/k/v of each request's block L..L+k and the logits of positions L+1..L+k+1."""
+    q, k, v, pl, ql = [], [], [], [], []
+    for r, L in enumerate(lens):
+        a, b, c = synth.token_qkv(spec, r, range(int(L), int(L) + spec.k + 1))
+        p_log, q_log = synth.token_logits(spec, r, range(int(L) + 1, int(L) + spec.k + 2))
+        q.append(a), k.append(b), v.append(c), pl.append(p_log), ql.append(q_log[: spec.k])
+    cu = lambda t: torch.stack(t).to(device)  # noqa: E731
+    return (cu(q), cu(k), cu(v), torch.as_tensor(np.stack(pl)).to(device),
+            torch.as_tensor(np.stack(ql)).to(device))
+
+
+def _oracle_state(spec, kp, vp, pt, r, L):
+    cap = int((pt[r] >= 0).sum()) * 16
+    K = np.stack([O.gather_positions(kp, pt[r], h, np.arange(cap)) for h in range(spec.num_kv_heads)])
+    V = np.stack([O.gather_positions(vp, pt[r], h, np.arange(cap)) for h in range(spec.num_kv_heads)])
+    return O.RequestState(K, V, int(L))
+
+
+def _compare_round(spec, r, res, sel, cnt, sig_prev, L, verify_out, lse, out_tokens, n_out):
+    """Returns True if the request's emitted tokens were compared exactly, False if a
+    boundary decision (oracle margin < 1e-5) let them differ."""
+    for h in range(spec.num_kv_heads):
+        near = set(O.selection_margin_cases(sig_prev[h], L, spec.budget_bp, spec.window, MARGIN).tolist())
+        diff = set(sel[h, : cnt[h]].tolist()) ^ set(res["sel"][h].tolist())
+        assert diff <= near, (r, h)
+    assert_attention_close(verify_out, res["verify_out"], f"verify r={r}")
+    np.testing.assert_allclose(lse, res["lse"], atol=2e-4, rtol=0)
+    near_decision = min(res["draft_margin"].min(), res["margins"].min()) < MARGIN
+    same = n_out == res["n_out"] and out_tokens[:n_out].tolist() == res["tokens"].tolist()
+    if not same:
+        assert near_decision, r
+    return same
+
+
+def test_mixed_phase_batch_matches_oracle():
+    """Ragged batch at mixed round phases (the high-concurrency workload's shape, fewer and
+    shorter requests so the oracle stays quick): each iteration drafts every request that is
+    mid-round with one launch over its ids and verifies the others with another; after k+1
+    iterations every request has finished the round it was in, which must equal the
+    oracle's round for that request."""
+    spec = synth.CONFIGS[3].with_(num_requests=24, lengths=("loguniform", 1024, 3072))
+    k = spec.k
+    lens = synth.make_lengths(spec)
+    cache = synth.build_cache(spec, lens, extra_tokens=2 * (k + 1) + 16)
+    kp, vp = cache.k_pool.float().numpy(), cache.v_pool.float().numpy()
+    pt = cache.page_table.numpy()
+    seq = torch.as_tensor(lens, dtype=torch.int32).cuda()
+    eng = s3r.S3REngine(cache.k_pool.cuda(), cache.v_pool.cuda(), cache.page_table.cuda(), seq,
+                        spec.num_q_heads, k=k, budget_bp=spec.budget_bp, window=spec.window,
+                        vocab=spec.vocab, seed=spec.sample_seed)
+    q, kb, vb, pl, ql = _inputs(spec, lens)
+    eng.prefill(q[:, :1].contiguous(), kb[:, :1].contiguous(), vb[:, :1].contiguous())
+    phases = synth.initial_phases(spec)
+    assert len(set(phases.tolist())) > 1
+    drv = s3r.MixedPhaseDriver(eng, phases)
+    drv.start(q, kb, vb, ql)
+    sel = eng.buf.sel_idx.cpu().numpy()
+    cnt = eng.buf.sel_count.cpu().numpy()
+    done = np.zeros(spec.num_requests, dtype=bool)
+    for _ in range(k + 1):
+        ids = drv.iterate(q, kb, vb, pl, ql)
+        assert not done[ids].any()
+        done[ids] = True
+    assert done.all()
+    assert eng.check_errors() == 0
+    b = eng.buf
+    exact = 0
+    for r in range(spec.num_requests):
+        L = int(lens[r])
+        st = _oracle_state(spec, kp, vp, pt, r, L)
+        O.prefill_scores(st, f64(q[r, 0]), f64(kb[r, 0]), f64(vb[r, 0]))
+        sig_prev = st.sigma
+        res = O.run_round(st, r, spec.sample_seed, k, spec.budget_bp, spec.window, f64(q[r]),
+                          f64(kb[r]), f64(vb[r]), ql[r].cpu().numpy(), pl[r].cpu().numpy())
+        exact += _compare_round(spec, r, res, sel[r], cnt[r], sig_prev, L, f64(b.verify_out[r]),
+                                f64(b.lse[r]), b.out_tokens[r].cpu().numpy(), int(b.n_out[r]))
+        assert int(eng.seq_lens[r]) == L + int(b.n_out[r])
+    assert exact >= spec.num_requests - 2
+    st = b.stats.cpu().numpy()
+    assert st[1] == spec.num_requests
+
+
+@pytest.mark.parametrize("config", [1, 2])
+def test_full_size_round_on_sampled_requests(config):
+    """One round of the whole Qwen3-shaped batch at full size (the benchmark's launch
+    configuration); the oracle replays two sampled requests."""
+    spec = synth.CONFIGS[config]
+    k = spec.k
+    lens = synth.make_lengths(spec)
+    cache = synth.build_cache(spec, lens, extra_tokens=k + 1 + 16, device="cuda")
+    seq = torch.as_tensor(lens, dtype=torch.int32, device="cuda")
+    NR, Hq, Hkv, d, V = spec.num_requests, spec.num_q_heads, spec.num_kv_heads, spec.head_dim, spec.vocab
+    q = synth.randn_bf16((NR, k + 1, Hq, d), 100, "cuda")
+    kb = synth.randn_bf16((NR, k + 1, Hkv, d), 101, "cuda")
+    vb = synth.randn_bf16((NR, k + 1, Hkv, d), 102, "cuda")
+    pl = synth.randn_f32((NR, k + 1, V), 103, "cuda", scale=spec.logit_std)
+    ql = (pl[:, :k] + synth.randn_f32((NR, k, V), 104, "cuda", scale=spec.draft_noise_std)).contiguous()
+    rng = np.random.default_rng(config)
+    picks = sorted(rng.choice(NR, size=2, replace=False).tolist())
+    pt = cache.page_table.cpu().numpy()
+    host = {}
+    for r in picks:    # the requests' pages before the round writes its block
+        ids = pt[r][pt[r] >= 0]
+        host[r] = (cache.k_pool[ids].float().cpu().numpy(), cache.v_pool[ids].float().cpu().numpy())
+    eng = s3r.S3REngine(cache.k_pool, cache.v_pool, cache.page_table, seq, Hq, k=k,
+                        budget_bp=spec.budget_bp, window=spec.window, vocab=V, seed=spec.sample_seed)
+    eng.prefill(q[:, :1].contiguous(), kb[:, :1].contiguous(), vb[:, :1].contiguous())
+    eng.select()
+    sel = eng.buf.sel_idx.cpu().numpy()
+    cnt = eng.buf.sel_count.cpu().numpy()
+    for i in range(k):
+        eng.draft_step(i, q, kb, vb, ql)
+    eng.verify(q, kb, vb)
+    eng.sample_and_commit(pl, ql)
+    assert eng.check_errors() == 0
+    b = eng.buf
+    for r in picks:
+        kpr, vpr = host[r]
+        local = np.arange(kpr.shape[0], dtype=np.int32)
+        K = np.stack([O.gather_positions(kpr, local, h, np.arange(len(local) * 16)) for h in range(Hkv)])
+        Vv = np.stack([O.gather_positions(vpr, local, h, np.arange(len(local) * 16)) for h in range(Hkv)])
+        st = O.RequestState(K, Vv, int(lens[r]))
+        O.prefill_scores(st, f64(q[r, 0]), f64(kb[r, 0]), f64(vb[r, 0]))
+        sig_prev = st.sigma
+        res = O.run_round(st, r, spec.sample_seed, k, spec.budget_bp, spec.window, f64(q[r]),
+                          f64(kb[r]), f64(vb[r]), ql[r].cpu().numpy(), pl[r].cpu().numpy())
+        _compare_round(spec, r, res, sel[r], cnt[r], sig_prev, int(lens[r]), f64(b.verify_out[r]),
+                       f64(b.lse[r]), b.out_tokens[r].cpu().numpy(), int(b.n_out[r]))
+        assert_attention_close(f64(b.draft_out[r]), res["draft_out"][k - 1], f"last draft r={r}")

@@ -76,7 +76,7 @@ def test_select_from_verify_scores_matches_oracle():
     cap = case.cache.capacity
     out = torch.empty_like(q)
     lse = torch.empty((NR, k + 1, Hq), dtype=torch.float32, device="cuda")
-    sc = torch.empty((NR, Hkv, cap, 4 * (k + 1)), device="cuda")
+    sc = torch.empty((NR, Hkv, 4 * (k + 1), cap), device="cuda")
     stride = 512
     ws = s3r.new_workspace(s3r.s3r_workspace_size(cache, NR, case.cache.max_pages, k, 64, stride))
     s3r.s3r_verify_attn(cache, batch, k, q, kn, vn, out, lse, sc, ws)
