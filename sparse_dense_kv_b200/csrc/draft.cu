@@ -16,7 +16,7 @@
 
 namespace s3r {
 
-constexpr int kDraftStages = 3;
+constexpr int kDraftStages = 2;
 
 template <int D>
 __global__ void __launch_bounds__(128) draft_kernel(const DraftParams p) {

@@ -101,6 +101,30 @@ __device__ MS block_ms(float m, float s) {
   return r;
 }
 
+// Merge one row's chunk partials with one warp: lane q loads partial q (and q + 32), so
+// the loads are one round trip, not one per chunk. Writes the chunk weights
+// csum[q] = s_q 2^((m_q - M) log2 e) (fp64) and returns the row maximum M on every lane.
+__device__ __forceinline__ float merge_partials_warp(const MS* part, int nvch, double* csum) {
+  const int lane = threadIdx.x & 31;
+  float mq[2] = {-INFINITY, -INFINITY};
+  double sq[2] = {0.0, 0.0};
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int q = lane + 32 * h;
+    if (q < nvch) {
+      mq[h] = __ldcg(&part[q].m);
+      sq[h] = __ldcg(&part[q].s);
+    }
+  }
+  const float M = warp_max(fmaxf(mq[0], mq[1]));
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int q = lane + 32 * h;
+    if (q < nvch) csum[q] = (mq[h] == -INFINITY) ? 0.0 : sq[h] * (double)exp2f((mq[h] - M) * kLog2e);
+  }
+  return M;
+}
+
 __device__ double block_sum_d(double v) {
   __shared__ double sd[kSampThreads / 32];
   __shared__ double tot;
@@ -251,14 +275,9 @@ __global__ void __launch_bounds__(kSampThreads) draft_sample_kernel(const Sample
   if (threadIdx.x == 0) part[c] = tot;
   if (!last_of(p.tickets + r, p.nvch, &s_flag)) return;
 
-  if (threadIdx.x == 0) {
-    float M = -INFINITY;
-    for (int q = 0; q < p.nvch; ++q) M = fmaxf(M, __ldcg(&part[q].m));
-    for (int q = 0; q < p.nvch; ++q) {
-      const float mq = __ldcg(&part[q].m);
-      csum[q] = (mq == -INFINITY) ? 0.0 : __ldcg(&part[q].s) * (double)exp2f((mq - M) * kLog2e);
-    }
-    s_M = M;
+  if (threadIdx.x < 32) {
+    const float M = merge_partials_warp(part, p.nvch, csum);
+    if (threadIdx.x == 0) s_M = M;
   }
   __syncthreads();
   const float M = s_M;
@@ -294,45 +313,46 @@ __global__ void __launch_bounds__(kSampThreads) spec_norm_kernel(const SamplePar
   if (threadIdx.x == 0) part[rw * p.nvch + c] = tot;
   if (!last_of(p.tickets + r, nrows * p.nvch, &s_flag)) return;
 
-  // normalisers of every row
-  if (threadIdx.x < nrows) {
-    const MS* pr = part + threadIdx.x * p.nvch;
-    float M = -INFINITY;
-    for (int q = 0; q < p.nvch; ++q) M = fmaxf(M, __ldcg(&pr[q].m));
-    double Z = 0.0;
-    for (int q = 0; q < p.nvch; ++q) {
-      const float mq = __ldcg(&pr[q].m);
-      if (mq != -INFINITY) Z += __ldcg(&pr[q].s) * (double)exp2f((mq - M) * kLog2e);
+  // normalisers of every row: one warp per row, the row's chunk partials loaded in parallel
+  __shared__ double s_cs[8][64];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int row = warp; row < nrows; row += kSampThreads / 32) {
+    const float M = merge_partials_warp(part + row * p.nvch, p.nvch, s_cs[warp]);
+    __syncwarp();
+    double z = 0.0;
+    for (int q = lane; q < p.nvch; q += 32) z += s_cs[warp][q];
+    z = warp_sum_d(z);
+    if (lane == 0) {
+      sM[row] = M;
+      sZ[row] = z;
     }
-    sM[threadIdx.x] = M;
-    sZ[threadIdx.x] = Z;
+    __syncwarp();
   }
   __syncthreads();
-  if (threadIdx.x != 0) return;
+  if (warp != 0) return;
 
+  // the k accept tests at once (lane j tests draft j), then the first rejection by ballot
   const int L = p.seq_lens[r];
   const size_t pbase = (size_t)r * (k + 1) * V, qbase = (size_t)r * k * V;
-  int a = 0, type = 1, jrow = k;
-  for (int j = 0; j < k; ++j) {
-    const int d = p.draft_tokens[(size_t)r * k + j];
-    bool accept = false;
+  bool acc = false;
+  int d = -1;
+  if (lane < k) {
+    d = p.draft_tokens[(size_t)r * k + lane];
     if (d < 0 || d >= V) {
       set_error(p.err, S3R_ERR_DEVICE_BOUNDS);
     } else {
-      const double pj = exp((double)p.p_logits[pbase + (size_t)j * V + d] - (double)sM[j]) / sZ[j];
-      const double qj =
-          exp((double)p.q_logits[qbase + (size_t)j * V + d] - (double)sM[k + 1 + j]) / sZ[k + 1 + j];
-      const double u = philox_u(p.seed, (uint32_t)(L + j + 1), (uint32_t)r, 1u);
-      accept = u * qj < pj;
+      const double pj = exp((double)p.p_logits[pbase + (size_t)lane * V + d] - (double)sM[lane]) / sZ[lane];
+      const double qj = exp((double)p.q_logits[qbase + (size_t)lane * V + d] - (double)sM[k + 1 + lane]) /
+                        sZ[k + 1 + lane];
+      const double u = philox_u(p.seed, (uint32_t)(L + lane + 1), (uint32_t)r, 1u);
+      acc = u * qj < pj;
     }
-    if (!accept) {
-      type = 0;
-      jrow = j;
-      break;
-    }
-    p.out_tokens[(size_t)r * (k + 1) + j] = d;
-    ++a;
   }
+  const unsigned rej = ~__ballot_sync(kFull, acc) & ((1u << k) - 1u);
+  const int a = rej ? __ffs(rej) - 1 : k;      // drafts accepted before the first rejection
+  if (lane < a) p.out_tokens[(size_t)r * (k + 1) + lane] = d;
+  if (lane != 0) return;
+  const int type = a < k ? 0 : 1, jrow = a;
   SpecPlan* plan = reinterpret_cast<SpecPlan*>(p.part + p.plan_off) + r;
   SpecPlan pl;
   pl.type = type;
@@ -386,12 +406,19 @@ __global__ void __launch_bounds__(kSampThreads) spec_draw_kernel(const SamplePar
   if (threadIdx.x == 0) part[c] = make_double2(sr, sp);
   if (!last_of(p.tickets + r, p.nvch, &s_flag)) return;
 
-  if (threadIdx.x == 0) {
-    double zr = 0.0;
-    for (int q = 0; q < p.nvch; ++q) zr += __ldcg(&part[q].x);
+  if (threadIdx.x < 32) {
+    // chunk sums loaded by the lanes at once; the residual mass decides which row is drawn
+    const int lane = threadIdx.x;
+    double2 pq[2] = {make_double2(0.0, 0.0), make_double2(0.0, 0.0)};
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+      if (lane + 32 * h < p.nvch) pq[h] = __ldcg(&part[lane + 32 * h]);
+    const double zr = warp_sum_d(pq[0].x + pq[1].x);
     const int use_res = resid && zr > 0.0;
-    for (int q = 0; q < p.nvch; ++q) csum[q] = use_res ? __ldcg(&part[q].x) : __ldcg(&part[q].y);
-    s_use_res = use_res;
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+      if (lane + 32 * h < p.nvch) csum[lane + 32 * h] = use_res ? pq[h].x : pq[h].y;
+    if (lane == 0) s_use_res = use_res;
   }
   __syncthreads();
   double Z = 0.0;

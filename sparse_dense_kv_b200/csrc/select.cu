@@ -8,9 +8,9 @@
 //
 // One CTA of 1024 threads per (KV head, request). Scores sigma_j = sum over the G*(k+1)
 // verify rows of exp(logit - lse) are computed once into shared memory as order-preserving
-// uint32 keys; three MSB-first histogram passes of 11, 11 and 10 bits (warp-aggregated
-// shared atomics, one block scan over the bins per pass) find the exact key of the M-th
-// largest score and how many ties at that key to keep; a final pass compacts the chosen
+// uint32 keys; MSB-first histogram passes of up to 11 bits over the bits in which the keys
+// differ (shared atomics, one block scan over the bins per pass) find the exact key of the
+// M-th largest score and how many ties at that key to keep; a final pass compacts the chosen
 // indices in increasing order, each warp over its own contiguous run of positions.
 #include "common.cuh"
 #include "kernels.h"
@@ -19,7 +19,7 @@ namespace s3r {
 
 constexpr int kSelectThreads = 1024;
 constexpr int kSelectMaxN = 49152;   // non-window positions held in shared memory
-constexpr int kSelectBins = 2048;    // 11-bit digits: bits 31..21, 20..10, 9..0
+constexpr int kSelectBins = 2048;    // digits of up to 11 bits
 
 __device__ __forceinline__ uint32_t order_key(float f) {
   if (f == 0.f) f = 0.f;              // -0 and +0 compare equal
@@ -151,40 +151,60 @@ __global__ void __launch_bounds__(kSelectThreads, 2) select_kernel(const SelectP
   if (bad) set_error(p.err, S3R_ERR_NONFINITE);
   __syncthreads();
 
-  // ---- radix select of the M-th largest key: three MSB-first passes of 11, 11, 10 bits.
-  // Each pass histograms the digit of the keys still matching the prefix (warp-aggregated
-  // shared atomics), then one block scan over the bins from the top finds the bin holding
-  // the remaining-th largest.
-  uint32_t prefix = 0, mask = 0;
+  // ---- radix select of the M-th largest key over the bits in which the keys differ: the
+  // block's smallest and largest key fix the common high bits, the rest is taken MSB-first
+  // in digits of up to 11 bits. Each pass histograms the digit of the keys that still
+  // match the prefix (shared atomics; the keys are spread over the bins, so contention
+  // stays low), then one block scan over the bins from the top finds the bin holding the
+  // remaining-th largest.
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+  for (int j = tid; j < N; j += blockDim.x) {
+    const uint32_t key = keys[j];
+    kmin = min(kmin, key);
+    kmax = max(kmax, key);
+  }
+  kmin = __reduce_min_sync(kFull, kmin);
+  kmax = __reduce_max_sync(kFull, kmax);
+  if (lane == 0) {
+    wa[warp] = (int)kmin;
+    wb[warp] = (int)kmax;
+  }
+  __syncthreads();
+  kmin = __reduce_min_sync(kFull, (uint32_t)wa[lane]);
+  kmax = __reduce_max_sync(kFull, (uint32_t)wb[lane]);
+  __syncthreads();
+  int nbits = 32 - __clz((int)(kmin ^ kmax));    // low bits in which keys differ (0: all equal)
+  uint32_t mask = nbits >= 32 ? 0u : ~((1u << nbits) - 1u);
+  uint32_t prefix = kmin & mask;
   int remaining = M;
-  const int Nround = (N + blockDim.x - 1) / blockDim.x * blockDim.x;
 #pragma unroll 1
-  for (int pass = 0; pass < 3; ++pass) {
-    const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
-    const int nb = pass == 2 ? 1024 : 2048;
-    for (int b = tid; b < nb; b += blockDim.x) hist[b] = 0;
+  while (nbits > 0) {
+    const int width = nbits < 11 ? nbits : 11;
+    const int shift = nbits - width;
+    const int nb = 1 << width;
+    for (int b = tid; b < kSelectBins; b += blockDim.x) hist[b] = 0;
     __syncthreads();
-    for (int j = tid; j < Nround; j += blockDim.x) {
-      const uint32_t key = j < N ? keys[j] : 0u;
-      const bool part = j < N && (key & mask) == prefix;
-      const uint32_t digit = (key >> shift) & (uint32_t)(nb - 1);
-      const unsigned peers = __match_any_sync(kFull, part ? digit : (0x10000u + lane));
-      if (part && lane == __ffs(peers) - 1) atomicAdd(&hist[digit], (uint32_t)__popc(peers));
+    for (int j = tid; j < N; j += blockDim.x) {
+      const uint32_t key = keys[j];
+      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & (uint32_t)(nb - 1)], 1u);
     }
     __syncthreads();
-    // thread t owns the bins nb-1-per*t .. nb-per*(t+1) (descending)
-    const int per = nb / kSelectThreads;
-    int h[2] = {0, 0}, local = 0;
-    for (int q = 0; q < per; ++q) {
-      h[q] = (int)hist[nb - 1 - per * tid - q];
+    // thread t owns bins 2047-2t and 2046-2t of the 2048-bin view (descending); bins at or
+    // above nb are empty
+    int h[2], local = 0;
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const int bin = kSelectBins - 1 - 2 * tid - q;
+      h[q] = bin < nb ? (int)hist[bin] : 0;
       local += h[q];
     }
     const int before = block_excl_scan(local, wsum);
     if (before < remaining && remaining <= before + local) {
       int cum = before;
-      for (int q = 0; q < per; ++q) {
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
         if (cum + h[q] >= remaining) {
-          s_prefix = prefix | ((uint32_t)(nb - 1 - per * tid - q) << shift);
+          s_prefix = prefix | ((uint32_t)(kSelectBins - 1 - 2 * tid - q) << shift);
           s_remaining = remaining - cum;
           break;
         }
@@ -195,6 +215,7 @@ __global__ void __launch_bounds__(kSelectThreads, 2) select_kernel(const SelectP
     prefix = s_prefix;
     remaining = s_remaining;
     mask |= (uint32_t)(nb - 1) << shift;
+    nbits = shift;
   }
   // prefix is the key of the M-th largest score; the first `remaining` keys equal to it (in
   // position order) are kept.
