@@ -521,6 +521,8 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--requests", type=int, default=0,
+                    help="override the workload's request count (small cases for profiling)")
     ap.add_argument("--sweep", action="store_true",
                     help="budget / draft-length sweep (one JSON line per point)")
     ap.add_argument("--sweep-rounds", type=int, default=3)
@@ -531,6 +533,8 @@ def main(argv=None):
         run_sweep(args)
         return
     spec = synth.CONFIGS[args.config]
+    if args.requests > 0:
+        spec = spec.with_(num_requests=args.requests)
     if spec.projection_logits or spec.mixed_phases:
         raise SystemExit("config 3 (mixed phases) and 4 (sweep) are parity / sweep cases, not bench lines")
     if args.impl == "reference":

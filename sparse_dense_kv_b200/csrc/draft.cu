@@ -20,6 +20,7 @@ constexpr int kDraftStages = 2;
 
 template <int D>
 __global__ void __launch_bounds__(128) draft_kernel(const DraftParams p) {
+  static_assert(kDraftChunk % 128 == 0, "128 threads resolve the chunk's rows");
   constexpr int NTW = 1, RW = 8, STAGE = 2 * kTile * D * 2, CPR = D / 8;
   extern __shared__ uint8_t smem_dyn[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) &
@@ -64,37 +65,46 @@ __global__ void __launch_bounds__(128) draft_kernel(const DraftParams p) {
     }
   }
 
-  // Element offsets of the chunk's rows: >= 0 pool offset, -1 zeros, -2 this step's token.
-  for (int e = tid; e < kDraftChunk; e += blockDim.x) {
-    const int a = start + e;
-    int64_t off = -1;
-    if (a < end) {
-      int pos;
-      bool ok = true;
-      if (a < n) {
-        pos = sel[a];
-        ok = pos >= 0 && pos < L;
-      } else {
-        pos = L + (a - n);
-      }
-      if (!ok) {
-        set_error(p.err, S3R_ERR_DEVICE_BOUNDS);
-      } else if (pos == L + i) {
-        off = -2;
-      } else {
-        const int page = ptab[pos >> 4];
-        if (page < 0 || page >= npages) set_error(p.err, S3R_ERR_DEVICE_BOUNDS);
-        else off = (((int64_t)page * Hkv + kvh) * kPage + (pos & 15)) * D;
-      }
-    }
-    rowoff[e] = off;
-  }
-
+  // The query rows first (their loads overlap the index work below).
   WarpAttn<D, NTW> wa;
   wa.init();
   wa.load_q(0, lane, [&](int rr) -> const __nv_bfloat16* {
     return rr < G ? p.q + (size_t)r * p.q_stride + (size_t)(kvh * G + rr) * D : nullptr;
   });
+
+  // Element offsets of the chunk's rows: >= 0 pool offset, -1 zeros, -2 this step's token.
+  // All selected indices are loaded at once, then all page ids: two dependent round trips.
+  constexpr int kPer = kDraftChunk / 128;
+  int pos[kPer];
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    const int a = start + tid + 128 * u;
+    pos[u] = a < end ? (a < n ? sel[a] : L + (a - n)) : -1;
+  }
+  int page[kPer];
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    const int a = start + tid + 128 * u;
+    const bool look = a < end && pos[u] >= 0 && pos[u] < L + i;   // a committed position
+    page[u] = look ? ptab[pos[u] >> 4] : -1;
+  }
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    const int a = start + tid + 128 * u;
+    int64_t off = -1;
+    if (a < end) {
+      if (a < n && (pos[u] < 0 || pos[u] >= L)) {
+        set_error(p.err, S3R_ERR_DEVICE_BOUNDS);
+      } else if (pos[u] == L + i) {
+        off = -2;
+      } else if (page[u] < 0 || page[u] >= npages) {
+        set_error(p.err, S3R_ERR_DEVICE_BOUNDS);
+      } else {
+        off = (((int64_t)page[u] * Hkv + kvh) * kPage + (pos[u] & 15)) * D;
+      }
+    }
+    rowoff[tid + 128 * u] = off;
+  }
   __syncthreads();
 
   const int ntiles = (end - start + kTile - 1) / kTile;

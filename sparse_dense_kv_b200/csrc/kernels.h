@@ -34,6 +34,7 @@ struct VerifyParams {
   int* err;
   int* tickets;
   float* part;
+  int req_off;             // launch covers requests req_ids[req_off + b] (or req_off + b)
 };
 
 struct DraftParams {
@@ -107,14 +108,17 @@ int launch_verify(const CUtensorMap& tk, const CUtensorMap& tv, const VerifyPara
                   int batch, cudaStream_t stream);
 size_t verify_partial_bytes(int num_requests, int Hkv, int cap, int R, int D, int chunk);
 int launch_verify_combine(const VerifyParams& p, int D, int batch, cudaStream_t stream);
+// Whether the chunk merge of a verify with these chunk counts fits in shared memory.
+bool verify_combine_fits(int nchunk_max, int R);
 
-// tcgen05 verify (head_dim 128, G*(k+1) <= 32 rows, <= 2048 requests per launch)
+// tcgen05 verify (head_dim 128, G*(k+1) <= 32 rows; batches beyond the per-launch request
+// table are split into several launches)
 bool verify_tc_supported(int D, int R, int batch);
 int verify_tc_npad(int R);
 int verify_tc_chunk(int R);
 int launch_verify_tc(const CUtensorMap& qm, const CUtensorMap& k1, const CUtensorMap& v1,
                      const CUtensorMap& k8, const CUtensorMap& v8, const VerifyParams& p,
-                     int batch, int num_sms, cudaStream_t stream);
+                     int batch, int num_sms, cudaStream_t stream, int* launches);
 
 int launch_draft(const DraftParams& p, int D, int batch, int num_sms, cudaStream_t stream);
 size_t draft_partial_bytes(int num_requests, int Hkv, int sel_stride, int D);

@@ -333,7 +333,12 @@ int s3r_verify_attn(const s3r_kv_cache* cache, const s3r_batch* batch, int32_t k
   p.tickets = w.tickets;
   p.part = reinterpret_cast<float*>(w.part);
   int st;
-  if (g_verify_kernel.load() == 0 && verify_tc_supported(cache->head_dim, R, batch->batch)) {
+  const bool tc = g_verify_kernel.load() == 0 && verify_tc_supported(cache->head_dim, R, batch->batch);
+  {
+    const int chunk = tc ? verify_tc_chunk(R) : kVerifyChunk;
+    if (!verify_combine_fits((cap + chunk - 1) / chunk, R)) return S3R_ERR_UNSUPPORTED;
+  }
+  if (tc) {
     p.Rp = verify_tc_npad(R);
     p.chunk = verify_tc_chunk(R);
     p.nchunk_max = (cap + p.chunk - 1) / p.chunk;
@@ -343,12 +348,14 @@ int s3r_verify_attn(const s3r_kv_cache* cache, const s3r_batch* batch, int32_t k
     S3R_TRY(make_paged_map(&v1, cache->v_pool, cache, 1));
     S3R_TRY(make_paged_map(&k8, cache->k_pool, cache, 8));
     S3R_TRY(make_paged_map(&v8, cache->v_pool, cache, 8));
-    st = launch_verify_tc(qm, k1, v1, k8, v8, p, batch->batch, sm_count(), (cudaStream_t)stream);
+    int nl = 0;
+    st = launch_verify_tc(qm, k1, v1, k8, v8, p, batch->batch, sm_count(), (cudaStream_t)stream, &nl);
+    g_launches.fetch_add((uint64_t)nl, std::memory_order_relaxed);
   } else {
     st = launch_verify(tk, tv, p, cache->head_dim, batch->batch, (cudaStream_t)stream);
+    if (st == S3R_OK) g_launches.fetch_add(1, std::memory_order_relaxed);
   }
   if (st != S3R_OK) return st;
-  g_launches.fetch_add(1, std::memory_order_relaxed);
   return finish(launch_verify_combine(p, cache->head_dim, batch->batch, (cudaStream_t)stream), 1);
 }
 

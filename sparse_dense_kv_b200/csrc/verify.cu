@@ -297,9 +297,13 @@ __global__ void __launch_bounds__(256) verify_combine_kernel(const VerifyParams 
   (void)Ms;
 }
 
+bool verify_combine_fits(int nchunk_max, int R) {
+  return ((size_t)3 * nchunk_max * R + R) * 4 <= 200 * 1024;
+}
+
 int launch_verify_combine(const VerifyParams& p, int D, int batch, cudaStream_t stream) {
   const size_t smem = ((size_t)3 * p.nchunk_max * p.R + p.R) * 4;
-  if (smem > 200 * 1024) return S3R_ERR_UNSUPPORTED;
+  if (!verify_combine_fits(p.nchunk_max, p.R)) return S3R_ERR_UNSUPPORTED;
   dim3 grid(p.Hkv, batch);
   if (D == 128) {
     static size_t attr = 0;

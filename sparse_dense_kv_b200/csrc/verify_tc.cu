@@ -34,12 +34,12 @@ namespace tc {
 
 constexpr int kPos = 128;                   // positions per tile (MMA M)
 constexpr int kD = 128;                     // head_dim of this path
-constexpr int kKStages = 2;                 // K ring
-constexpr int kVStages = 2;                 // V ring
+constexpr int kMaxStages = 4;               // ring barriers per stream
 constexpr int kThreads = 352;               // K producer, V producer, MMA, 8 softmax warps
 constexpr int kSoftWarp0 = 3;
+constexpr int kBarBytes = 512;              // mbarriers and flags
 constexpr int kTileBytes = kPos * kD * 2;   // 32 KB: [2 halves][128 rows][128 B]
-constexpr int kMaxBatch = 1024;             // requests per launch on this path
+constexpr int kMaxBatch = 256;              // requests per launch (larger batches: several launches)
 
 // --------------------------------------------------------------- tcgen05 wrappers -------
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
@@ -90,6 +90,31 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
+// This warp's 32 lanes x 8 consecutive columns.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float* v) {
+  uint32_t r[8];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                 "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+// N (8 or a multiple of 16) consecutive columns.
+template <int N>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float (&v)[N]) {
+  if constexpr (N == 8) {
+    tmem_ld8(taddr, v);
+  } else {
+#pragma unroll
+    for (int c = 0; c < N; c += 16) {
+      float w[16];
+      tmem_ld16(taddr + c, w);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) v[c + i] = w[i];
+    }
+  }
+}
 template <int N>
 __device__ __forceinline__ void tmem_ld(uint32_t taddr, float (&v)[N]) {
 #pragma unroll
@@ -118,6 +143,8 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool 
 template <int NP>
 struct Cfg {
   static constexpr int kTiles = NP == 32 ? 7 : 8;            // tiles per chunk
+  static constexpr int kKSt = 2;                             // K ring stages
+  static constexpr int kVSt = 2;                             // V ring stages
   static constexpr int kChunk = kTiles * kPos;
   static constexpr int kQBytes = 2 * NP * 128;               // one Q buffer: [2 halves][NP rows][128 B]
   static constexpr int kPTile = kPos * NP * 2;               // P^T tile: [128 pos][NP rows] bf16
@@ -127,10 +154,11 @@ struct Cfg {
   static constexpr int kSCols = kTiles * NP;                 // one S buffer
   static constexpr int kOCol = 2 * kSCols;                   // two O buffers after two S buffers
   static_assert(kOCol + 2 * NP <= kTmemCols, "tensor memory budget");
+  static_assert(kKSt <= kMaxStages && kVSt <= kMaxStages && kTiles <= 8, "barrier arrays");
   static constexpr int kSmemMax = 227 * 1024;
   static constexpr int kKRingOff = 0;
-  static constexpr int kVRingOff = kKStages * kTileBytes;
-  static constexpr int kQOff = (kKStages + kVStages) * kTileBytes;
+  static constexpr int kVRingOff = kKSt * kTileBytes;
+  static constexpr int kQOff = (kKSt + kVSt) * kTileBytes;
   static constexpr int kPOff = kQOff + 2 * kQBytes;         // two Q buffers (item parity)
   static constexpr int kRedOff = kPOff + kPBytes;            // redM, redL [8 warps][NP]; cm, cl [2][NP]
   static constexpr int kRedBytes = (2 * 8 * NP + 4 * NP) * 4;
@@ -139,26 +167,28 @@ struct Cfg {
   static constexpr int kRidOff = kLenOff + kMaxBatch * 4;          // request id [kMaxBatch]
   static constexpr int kIdsOff = kRidOff + kMaxBatch * 4;          // page ids [K, V producer][64]
   static constexpr int kBarOff = (kIdsOff + 2 * 64 * 4 + 63) / 64 * 64;
-  static constexpr int kSmem = kBarOff + 256 + 1024;         // + barriers + alignment slack
+  static constexpr int kSmem = kBarOff + kBarBytes + 1024;   // + barriers + alignment slack
   static_assert(kSmem <= kSmemMax, "shared memory budget");
   static_assert(kQOff % 1024 == 0 && kPOff % 1024 == 0 && kRedOff % 16 == 0 && kBarOff % 64 == 0,
                 "alignment of the swizzled operands, the reduction scratch and the barriers");
 };
 
 struct Bars {
-  uint64_t kfull[kKStages], kempty[kKStages], ktma[kKStages];
-  uint64_t vfull[kVStages], vempty[kVStages], vtma[kVStages];
+  uint64_t kfull[kMaxStages], kempty[kMaxStages], ktma[kMaxStages];
+  uint64_t vfull[kMaxStages], vempty[kMaxStages], vtma[kMaxStages];
   // one barrier pair per tensor-memory buffer (chunk parity), so that no barrier ever runs
   // two phases ahead of a waiter
   uint64_t q_full[2], q_empty[2], p_full, fin;
   uint64_t s_full[2], s_empty[2], o_full[2], o_empty[2];
+  uint64_t p_free[8];   // P^T tile t has been read by the PV of the previous chunk
   uint32_t tmem_base;
   int abort_flag;
 };
-static_assert(sizeof(Bars) <= 256, "barrier block");
+static_assert(sizeof(Bars) <= kBarBytes, "barrier block");
 
-__device__ __forceinline__ void named_sync_softmax() {
-  asm volatile("bar.sync 1, 256;\n" ::: "memory");
+// Barrier of one softmax warpgroup (named barriers 1 and 2, 128 threads each).
+__device__ __forceinline__ void wg_sync(int sg) {
+  asm volatile("bar.sync %0, 128;\n" ::"r"(1 + sg) : "memory");
 }
 
 // Work item i of the launch -> (launch-local request, KV head, chunk), from the prefix of
@@ -226,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ---- set-up: request prefix (items), barriers, tensor memory
   for (int b = tid; b < batch; b += blockDim.x) {
-    const int r = p.req_ids ? p.req_ids[b] : b;
+    const int r = p.req_ids ? p.req_ids[p.req_off + b] : p.req_off + b;
     const int L = p.seq_lens[r];
     const int Lc = L + T;
     rid_s[b] = r;
@@ -258,12 +288,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (tid < NP) trow[tid] = tid / G;
   if (tid == 0) {
-    for (int s = 0; s < kKStages; ++s) {
+    for (int s = 0; s < C::kKSt; ++s) {
       mbar_init(smem_u32(&B->kfull[s]), 1);
       mbar_init(smem_u32(&B->kempty[s]), 1);
       mbar_init(smem_u32(&B->ktma[s]), 1);
     }
-    for (int s = 0; s < kVStages; ++s) {
+    for (int s = 0; s < C::kVSt; ++s) {
       mbar_init(smem_u32(&B->vfull[s]), 1);
       mbar_init(smem_u32(&B->vempty[s]), 1);
       mbar_init(smem_u32(&B->vtma[s]), 1);
@@ -279,6 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&B->o_empty[b]), 8);
     }
     mbar_init(smem_u32(&B->p_full), 8);
+    for (int t = 0; t < 8; ++t) mbar_init(smem_u32(&B->p_free[t]), 1);
     mbar_init(smem_u32(&B->fin), 1);
     B->abort_flag = 0;
     fence_mbar_init();
@@ -306,7 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(is_v ? &tmV8 : &tmK8)) : "memory");
       if (!is_v) asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&tmQ)) : "memory");
     }
-    const int nst = is_v ? kVStages : kKStages;
+    const int nst = is_v ? C::kVSt : C::kKSt;
     const int roff = is_v ? C::kVRingOff : C::kKRingOff;
     uint64_t* full = is_v ? B->vfull : B->kfull;
     uint64_t* empty = is_v ? B->vempty : B->kempty;
@@ -474,8 +505,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (kgo) tc_fence_after();
         }
         if (kgo) {
-          const int s = gk % kKStages;
-          if (ready(&B->kfull[s], (gk / kKStages) & 1)) {
+          const int s = gk % C::kKSt;
+          if (ready(&B->kfull[s], (gk / C::kKSt) & 1)) {
             tc_fence_after();
             if (lane == 0) {
               const uint32_t kt = sbase + C::kKRingOff + s * kTileBytes;
@@ -514,8 +545,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (vgo) tc_fence_after();
         }
         if (vgo) {
-          const int s = gv % kVStages;
-          if (ready(&B->vfull[s], (gv / kVStages) & 1)) {
+          const int s = gv % C::kVSt;
+          if (ready(&B->vfull[s], (gv / C::kVSt) & 1)) {
             tc_fence_after();
             if (lane == 0) {
               const uint32_t vt = sbase + C::kVRingOff + s * kTileBytes;
@@ -528,13 +559,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_mma(od, ad, bd, kIdPV, (tv > 0 || kk > 0) ? 1u : 0u);
               }
               tc_commit(smem_u32(&B->vempty[s]));
+              tc_commit(smem_u32(&B->p_free[tv]));
             }
             __syncwarp();
             ++tv;
             ++gv;
             did = true;
             if (tv == xv.ntile) {
-              if (lane == 0) tc_commit(smem_u32(&B->o_full[nv & 1]));
+              if (lane == 0) {
+                // every P^T tile's barrier completes once per chunk, used or not
+                for (int t = xv.ntile; t < C::kTiles; ++t) tc_commit(smem_u32(&B->p_free[t]));
+                tc_commit(smem_u32(&B->o_full[nv & 1]));
+              }
               __syncwarp();
               ++nv;
               tv = 0;
@@ -563,36 +599,40 @@ __global__ void __launch_bounds__(kThreads, 1)
     wait_bar(smem_u32(&B->fin), 0, abort_flag, p.err);
   } else {
     // ================================================================ softmax warps ===
+    // Warpgroup sg owns rows (columns of S and O^T) [sg*NH, sg*NH + NH) of every tile; the
+    // two warpgroups only meet at the chunk's barriers for the MMA warp.
+    constexpr int NH = NP / 2;               // rows per warpgroup
+    constexpr int BT = NP == 32 ? 2 : 4;     // tiles per tensor-memory wait (no spills)
     const int sw8 = warp - kSoftWarp0;       // 0..7
-    const int sg = sw8 >> 2;                 // warpgroup: tiles t with t % 2 == sg
+    const int sg = sw8 >> 2;                 // warpgroup
+    const int sw4 = sw8 & 3;                 // warp within the warpgroup
     const int q4 = warp & 3;                 // tensor-memory lane quarter of this warp
-    const int st = tid - 32 * kSoftWarp0;    // 0..255 within the softmax warps
+    const int gt = (tid - 32 * kSoftWarp0) & 127;   // thread within the warpgroup
     const int lrow = q4 * 32 + lane;         // tile position (S) or d (O) of this thread
+    const int c0 = sg * NH;                  // first row of this warpgroup
     const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
     const float scale = p.scale, scale2 = p.scale * kLog2e;
     const int swz_row = (NP == 16) ? ((lrow >> 2) & 1) : ((lrow >> 1) & 3);
 
-    // record of chunk m: O^T buffer m&1 -> workspace, with its row max / sum from cm / cl
+    // record of chunk m (this warpgroup's rows): O^T buffer m&1 -> workspace, with the rows'
+    // max / sum from cm / cl
     auto epilogue = [&](int m) -> bool {
       const Item x = make_item<NP>(blockIdx.x + m * gridDim.x, pref, lens_s, rid_s, batch, p);
       if (!wait_bar(smem_u32(&B->o_full[m & 1]), (m >> 1) & 1, abort_flag, p.err)) return false;
       tc_fence_after();
       const size_t rec_floats = (size_t)p.Rp * (kD + 2);
       float* rec = p.part + (((size_t)x.r * Hkv + x.kvh) * p.nchunk_max + x.c) * rec_floats;
-      constexpr int kHalf = NP / 2 >= 16 ? NP / 2 : 16;    // columns per warpgroup
-      if (sg * kHalf < NP) {
-        float o[16];
-        tmem_ld16(tl + C::kOCol + (m & 1) * NP + sg * kHalf, o);
-        tmem_wait_ld();
+      float o[NH];
+      tmem_ld_cols<NH>(tl + C::kOCol + (m & 1) * NP + c0, o);
+      tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 16; ++j) rec[2 * p.Rp + (size_t)(sg * kHalf + j) * kD + lrow] = o[j];
-      }
+      for (int j = 0; j < NH; ++j) rec[2 * p.Rp + (size_t)(c0 + j) * kD + lrow] = o[j];
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&B->o_empty[m & 1]));
-      if (st < NP) {
-        rec[st] = cm[(m & 1) * NP + st];
-        rec[p.Rp + st] = cl[(m & 1) * NP + st];
+      if (gt < NH) {
+        rec[c0 + gt] = cm[(m & 1) * NP + c0 + gt];
+        rec[p.Rp + c0 + gt] = cl[(m & 1) * NP + c0 + gt];
       }
       return true;
     };
@@ -607,93 +647,110 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      const uint32_t sbuf = tl + (n & 1) * C::kSCols;
+      const uint32_t sbuf = tl + (n & 1) * C::kSCols + c0;
 
-      // pass 1 over this warpgroup's tiles: committed logits out, max per row (raw units)
-      float mrow[NP];
+      // pass 1 over every tile: committed logits out, max per row (raw units)
+      float mrow[NH];
 #pragma unroll
-      for (int j = 0; j < NP; ++j) mrow[j] = -INFINITY;
-      for (int t = sg; t < x.ntile; t += 2) {
-        float v[NP];
-        tmem_ld<NP>(sbuf + t * NP, v);
+      for (int j = 0; j < NH; ++j) mrow[j] = -INFINITY;
+      for (int tb = 0; tb < x.ntile; tb += BT) {
+        float vv[BT][NH];
+#pragma unroll
+        for (int u = 0; u < BT; ++u)   // past the last tile: reload the last tile (unused)
+          tmem_ld_cols<NH>(sbuf + min(tb + u, x.ntile - 1) * NP, vv[u]);
         tmem_wait_ld();
-        const int t0 = start + t * kPos;
-        const int pos = t0 + lrow;
-        if (scores && pos < L) {
-          // committed logits, [row][position]: the warp's 32 lanes write 32 consecutive
-          // positions of one row per store, one whole 128-byte line
 #pragma unroll
-          for (int j = 0; j < NP; ++j)
-            if (j < R) scores[(size_t)j * p.cap + pos] = v[j] * scale;
-        }
-        if (t0 + kPos <= min(L, end)) {
+        for (int u = 0; u < BT; ++u) {
+          if (tb + u >= x.ntile) break;
+          const int t0 = start + (tb + u) * kPos;
+          const int pos = t0 + lrow;
+          if (scores && pos < L) {
+            // committed logits, [row][position]: the warp's 32 lanes write 32 consecutive
+            // positions of one row per store, one whole 128-byte line
 #pragma unroll
-          for (int j = 0; j < NP; ++j) mrow[j] = fmaxf(mrow[j], v[j]);
-        } else {
+            for (int j = 0; j < NH; ++j)
+              if (c0 + j < R) scores[(size_t)(c0 + j) * p.cap + pos] = vv[u][j] * scale;
+          }
+          if (t0 + kPos <= min(L, end)) {
 #pragma unroll
-          for (int j = 0; j < NP; ++j) {
-            const bool vis = pos < end && j < R && (pos < L || pos - L <= trow[j]);
-            if (vis) mrow[j] = fmaxf(mrow[j], v[j]);
+            for (int j = 0; j < NH; ++j) mrow[j] = fmaxf(mrow[j], vv[u][j]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < NH; ++j) {
+              const int row = c0 + j;
+              const bool vis = pos < end && row < R && (pos < L || pos - L <= trow[row]);
+              if (vis) mrow[j] = fmaxf(mrow[j], vv[u][j]);
+            }
           }
         }
       }
 #pragma unroll
-      for (int j = 0; j < NP; ++j) {
+      for (int j = 0; j < NH; ++j) {
         float m = mrow[j];
 #pragma unroll
         for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
-        if (lane == j) redM[sw8 * NP + j] = m;
+        if (lane == j) redM[(sg * 4 + sw4) * NH + j] = m;
       }
-      named_sync_softmax();
-      if (st < NP) {
-        float m = redM[st];
+      wg_sync(sg);
+      if (gt < NH) {
+        float m = redM[(sg * 4) * NH + gt];
 #pragma unroll
-        for (int w = 1; w < 8; ++w) m = fmaxf(m, redM[w * NP + st]);
-        cm[(n & 1) * NP + st] = scale2 * m;
+        for (int w = 1; w < 4; ++w) m = fmaxf(m, redM[(sg * 4 + w) * NH + gt]);
+        cm[(n & 1) * NP + c0 + gt] = scale2 * m;
       }
-      named_sync_softmax();
+      wg_sync(sg);
 #pragma unroll
-      for (int j = 0; j < NP; ++j) mrow[j] = cm[(n & 1) * NP + j];
+      for (int j = 0; j < NH; ++j) mrow[j] = cm[(n & 1) * NP + c0 + j];
 
-      // the previous chunk's output leaves tensor memory before P^T is overwritten
-      if (n > 0 && !epilogue(n - 1)) {
-        ok = false;
-        break;
-      }
-
-      // pass 2: P = 2^(s - max) as bf16 P^T tiles (MN-major, NP values per position) + sums
-      float lsum[NP];
+      // pass 2: P = 2^(s - max) as bf16 P^T tiles (MN-major, NP values per position; this
+      // warpgroup writes its NH of them) + sums. P^T tile t is overwritten once the previous
+      // chunk's PV has read it (its own barrier), so this pass runs alongside that PV.
+      float lsum[NH];
 #pragma unroll
-      for (int j = 0; j < NP; ++j) lsum[j] = 0.f;
-      for (int t = sg; t < x.ntile; t += 2) {
-        float v[NP];
-        tmem_ld<NP>(sbuf + t * NP, v);
+      for (int j = 0; j < NH; ++j) lsum[j] = 0.f;
+      for (int tb = 0; tb < x.ntile && ok; tb += BT) {
+        float vv[BT][NH];
+#pragma unroll
+        for (int u = 0; u < BT; ++u)   // past the last tile: reload the last tile (unused)
+          tmem_ld_cols<NH>(sbuf + min(tb + u, x.ntile - 1) * NP, vv[u]);
         tmem_wait_ld();
-        const int t0 = start + t * kPos;
-        const int pos = t0 + lrow;
-        const bool interior = t0 + kPos <= min(L, end);
-        uint32_t pk[NP / 2];
 #pragma unroll
-        for (int j = 0; j < NP; j += 2) {
-          float e0 = ex2(fmaf(v[j], scale2, -mrow[j]));
-          float e1 = ex2(fmaf(v[j + 1], scale2, -mrow[j + 1]));
-          if (!interior) {
-            const bool v0 = pos < end && j < R && (pos < L || pos - L <= trow[j]) && mrow[j] != -INFINITY;
-            const bool v1 = pos < end && j + 1 < R && (pos < L || pos - L <= trow[j + 1]) &&
-                            mrow[j + 1] != -INFINITY;
-            e0 = v0 ? e0 : 0.f;
-            e1 = v1 ? e1 : 0.f;
+        for (int u = 0; u < BT; ++u) {
+          if (tb + u >= x.ntile) break;
+          const int t = tb + u;
+          const int t0 = start + t * kPos;
+          const int pos = t0 + lrow;
+          const bool interior = t0 + kPos <= min(L, end);
+          uint32_t pk[NH / 2];
+#pragma unroll
+          for (int j = 0; j < NH; j += 2) {
+            float e0 = ex2(fmaf(vv[u][j], scale2, -mrow[j]));
+            float e1 = ex2(fmaf(vv[u][j + 1], scale2, -mrow[j + 1]));
+            if (!interior) {
+              const int r0 = c0 + j, r1 = c0 + j + 1;
+              const bool v0 = pos < end && r0 < R && (pos < L || pos - L <= trow[r0]) && mrow[j] != -INFINITY;
+              const bool v1 = pos < end && r1 < R && (pos < L || pos - L <= trow[r1]) && mrow[j + 1] != -INFINITY;
+              e0 = v0 ? e0 : 0.f;
+              e1 = v1 ? e1 : 0.f;
+            }
+            lsum[j] += e0;
+            lsum[j + 1] += e1;
+            pk[j / 2] = pack_bf16(e0, e1);
           }
-          lsum[j] += e0;
-          lsum[j + 1] += e1;
-          pk[j / 2] = pack_bf16(e0, e1);
-        }
-        uint8_t* prow = smem + C::kPOff + t * C::kPTile + lrow * (NP * 2);
+          if (n > 0 && !wait_bar(smem_u32(&B->p_free[t]), (n - 1) & 1, abort_flag, p.err)) {
+            ok = false;
+            break;
+          }
+          uint8_t* prow = smem + C::kPOff + t * C::kPTile + lrow * (NP * 2);
 #pragma unroll
-        for (int cc = 0; cc < NP / 8; ++cc)
-          *reinterpret_cast<uint4*>(prow + ((cc ^ swz_row) << 4)) =
-              make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
+          for (int i = 0; i < NH / 8; ++i) {
+            const int cc = sg * (NH / 8) + i;
+            *reinterpret_cast<uint4*>(prow + ((cc ^ swz_row) << 4)) =
+                make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          }
+        }
       }
+      if (!ok) break;
       fence_proxy_async();
       tc_fence_before();
       __syncwarp();
@@ -701,24 +758,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(smem_u32(&B->s_empty[n & 1]));
         mbar_arrive(smem_u32(&B->p_full));
       }
+      // the previous chunk's output leaves tensor memory (its PV has finished by now or
+      // soon: this pass already waited for each of its tiles)
+      if (n > 0 && !epilogue(n - 1)) {
+        ok = false;
+        break;
+      }
 #pragma unroll
-      for (int j = 0; j < NP; ++j) {
+      for (int j = 0; j < NH; ++j) {
         float sacc = lsum[j];
 #pragma unroll
         for (int o = 16; o; o >>= 1) sacc += __shfl_xor_sync(kFull, sacc, o);
-        if (lane == j) redL[sw8 * NP + j] = sacc;
+        if (lane == j) redL[(sg * 4 + sw4) * NH + j] = sacc;
       }
-      named_sync_softmax();
-      if (st < NP) {
+      wg_sync(sg);
+      if (gt < NH) {
         float l = 0.f;
 #pragma unroll
-        for (int w = 0; w < 8; ++w) l += redL[w * NP + st];
-        cl[(n & 1) * NP + st] = l;
+        for (int w = 0; w < 4; ++w) l += redL[(sg * 4 + w) * NH + gt];
+        cl[(n & 1) * NP + c0 + gt] = l;
       }
       // (cl / redL reuse is ordered by the barriers of the next chunk)
     }
     if (ok && my_items > 0 && !aborted(abort_flag)) {
-      named_sync_softmax();   // cl of the last chunk complete
+      wg_sync(sg);   // cl of the last chunk complete
       epilogue(my_items - 1);
     }
   }
@@ -753,8 +816,8 @@ static int launch_tc(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
   return cuda_status(cudaGetLastError(), __func__);
 }
 
-bool verify_tc_supported(int D, int R, int batch) {
-  return D == tc::kD && verify_tc_npad(R) != 0 && batch <= tc::kMaxBatch;
+bool verify_tc_supported(int D, int R, int /*batch*/) {
+  return D == tc::kD && verify_tc_npad(R) != 0;
 }
 
 int verify_tc_chunk(int R) {
@@ -764,11 +827,22 @@ int verify_tc_chunk(int R) {
 
 int launch_verify_tc(const CUtensorMap& qm, const CUtensorMap& k1, const CUtensorMap& v1,
                      const CUtensorMap& k8, const CUtensorMap& v8, const VerifyParams& p,
-                     int batch, int num_sms, cudaStream_t stream) {
+                     int batch, int num_sms, cudaStream_t stream, int* launches) {
   const int np = verify_tc_npad(p.R);
-  if (np == 16) return launch_tc<16>(qm, k1, v1, k8, v8, p, batch, num_sms, stream);
-  if (np == 32) return launch_tc<32>(qm, k1, v1, k8, v8, p, batch, num_sms, stream);
-  return S3R_ERR_UNSUPPORTED;
+  *launches = 0;
+  if (np != 16 && np != 32) return S3R_ERR_UNSUPPORTED;
+  // the per-launch request tables hold kMaxBatch requests; a larger batch is several
+  // launches over consecutive slices of it (each chunk record still lands in its slot)
+  for (int b0 = 0; b0 < batch; b0 += tc::kMaxBatch) {
+    VerifyParams q = p;
+    q.req_off = p.req_off + b0;
+    const int nb = batch - b0 < tc::kMaxBatch ? batch - b0 : tc::kMaxBatch;
+    const int st = np == 16 ? launch_tc<16>(qm, k1, v1, k8, v8, q, nb, num_sms, stream)
+                            : launch_tc<32>(qm, k1, v1, k8, v8, q, nb, num_sms, stream);
+    if (st != S3R_OK) return st;
+    ++*launches;
+  }
+  return S3R_OK;
 }
 
 }  // namespace s3r

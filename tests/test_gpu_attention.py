@@ -200,3 +200,24 @@ def test_sparse_draft_full_budget_equals_verify_row():
                         vo, vl, None, ws)
     torch.cuda.synchronize()
     assert_attention_close(f64(out), f64(vo[:, 0]), "draft vs verify row")
+
+
+def test_verify_batch_larger_than_one_launch():
+    """300 requests: the tensor-memory verify splits the batch into several launches over
+    consecutive request slices; every request must still match the oracle."""
+    rng = np.random.default_rng(12)
+    lens = rng.integers(100, 700, size=300).tolist()
+    k = 6
+    spec = spec_for(32, 8, 128, lens, k=k, seed=19)
+    case = Case(spec, extra_tokens=k + 1 + 8)
+    before = s3r.s3r_launch_count()
+    q, kn, vn, out, lse, sc = run_verify(case, k, seed=41)
+    assert s3r.s3r_launch_count() - before == 3      # two verify launches + the merge
+    kp, vp = case.host_pools()
+    for r in rng.choice(len(lens), size=12, replace=False).tolist() + [0, 255, 256, 299]:
+        L = case.lens[r]
+        K, V = case.dense(r, L + k + 1, (kp, vp))
+        o, l, _, logits = O.verify_attention(f64(q[r]), K, V, int(L))
+        assert_attention_close(f64(out[r]), o, f"out r={r}")
+        np.testing.assert_allclose(f64(lse[r]), l, rtol=0, atol=2e-4)
+        np.testing.assert_allclose(f64(sc[r][:, :, :L]), logits[:, :, :L], rtol=1e-5, atol=1e-4)

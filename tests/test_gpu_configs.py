@@ -147,3 +147,94 @@ def test_full_size_round_on_sampled_requests(config):
         _compare_round(spec, r, res, sel[r], cnt[r], sig_prev, int(lens[r]), f64(b.verify_out[r]),
                        f64(b.lse[r]), b.out_tokens[r].cpu().numpy(), int(b.n_out[r]))
         assert_attention_close(f64(b.draft_out[r]), res["draft_out"][k - 1], f"last draft r={r}")
+
+
+def test_projection_logits_round_matches_oracle():
+    """The budget-sweep workload's logit model (a seeded bf16 projection of the
+    head-concatenated attention outputs, fewer and shorter requests so the oracle stays
+    quick): attention outputs of every draft step and of the verify match the oracle's, and
+    the GPU samplers, given the oracle's own logits, take the oracle's decisions."""
+    spec = synth.CONFIGS[4].with_(num_requests=3, lengths=("fixed", (3000, 4100, 2500)))
+    k, V = spec.k, spec.vocab
+    NR, Hq, Hkv, d = spec.num_requests, spec.num_q_heads, spec.num_kv_heads, spec.head_dim
+    lens = synth.make_lengths(spec)
+    cache = synth.build_cache(spec, lens, extra_tokens=k + 1 + 16)
+    kp, vp = cache.k_pool.float().numpy(), cache.v_pool.float().numpy()
+    pt = cache.page_table.numpy()
+    W = synth.projection_matrix(spec, "cuda")
+    W64 = W.double().cpu().numpy()
+    gamma = 3.0
+    seq = torch.as_tensor(lens, dtype=torch.int32).cuda()
+    eng = s3r.S3REngine(cache.k_pool.cuda(), cache.v_pool.cuda(), cache.page_table.cuda(), seq,
+                        Hq, k=k, budget_bp=spec.budget_bp, window=spec.window, vocab=V,
+                        seed=spec.sample_seed)
+    q, kb, vb, _, _ = _inputs(spec.with_(vocab=8), lens)
+    eng.prefill(q[:, :1].contiguous(), kb[:, :1].contiguous(), vb[:, :1].contiguous())
+    ql = torch.empty((NR, k, V), device="cuda")
+    pl = torch.empty((NR, k + 1, V), device="cuda")
+    draft_outs = []
+
+    def draft_fn(i, out, q_logits):
+        draft_outs.append(out.clone())
+        q_logits[:, i] = gamma * (out.float().reshape(NR, -1) @ W.float())
+
+    def target_fn(vout, p_logits):
+        p_logits.copy_((gamma * (vout.float().reshape(NR * (k + 1), -1) @ W.float())).view(NR, k + 1, V))
+
+    eng.round(q, kb, vb, pl, ql, draft_logits_fn=draft_fn, target_logits_fn=target_fn)
+    assert eng.check_errors() == 0
+    n_out = eng.buf.n_out.cpu().numpy()
+    assert ((n_out >= 1) & (n_out <= k + 1)).all()
+    gsel, gcnt = eng.buf.sel_idx.cpu().numpy(), eng.buf.sel_count.cpu().numpy()
+    # the oracle's round, with logits from its own attention outputs
+    oq = np.zeros((NR, k, V), np.float32)
+    op = np.zeros((NR, k + 1, V), np.float32)
+    odrafts = np.zeros((NR, k), np.int32)
+    res_tok = []
+    for r in range(NR):
+        L = int(lens[r])
+        st = _oracle_state(spec, kp, vp, pt, r, L)
+        O.prefill_scores(st, f64(q[r, 0]), f64(kb[r, 0]), f64(vb[r, 0]))
+        sel = [O.select_positions(st.sigma[h], L, spec.budget_bp, spec.window) for h in range(Hkv)]
+        same_sel = True
+        for h in range(Hkv):
+            got = set(gsel[r, h, : gcnt[r, h]].tolist())
+            near = set(O.selection_margin_cases(st.sigma[h], L, spec.budget_bp, spec.window, MARGIN).tolist())
+            assert (got ^ set(sel[h].tolist())) <= near, (r, h)
+            same_sel &= got == set(sel[h].tolist())
+        for i in range(k):
+            st.write([L + i], [f64(kb[r, i])], [f64(vb[r, i])])
+            o, _ = O.sparse_draft_attention(f64(q[r, i]), st.K, st.V, sel, L, i)
+            if same_sel:
+                assert_attention_close(f64(draft_outs[i][r]), o, f"draft r={r} i={i}")
+            oq[r, i] = gamma * (o.reshape(-1) @ W64)
+            u0 = float(O.uniform(spec.sample_seed, r, L + i + 1, O.STREAM_DRAFT))
+            odrafts[r, i], _ = O.draft_sample(oq[r, i], u0)
+        st.write(list(range(L, L + k + 1)), f64(kb[r]), f64(vb[r]))
+        vo, _, _, _ = O.verify_attention(f64(q[r]), st.K, st.V, L)
+        assert_attention_close(f64(eng.buf.verify_out[r]), vo, f"verify r={r}")
+        op[r] = gamma * (vo.reshape(k + 1, -1) @ W64)
+        res_tok.append(O.spec_sample(op[r], oq[r], odrafts[r], spec.sample_seed, r, L))
+    # the GPU samplers on the oracle's logits
+    batch = s3r.make_batch(torch.as_tensor(lens, dtype=torch.int32).cuda())
+    cdesc = s3r.KVCacheDesc(8, 8, 128, 16, 1, 16, 16)
+    ws = s3r.new_workspace(s3r.s3r_workspace_size(cdesc, NR, 1, k, V, 1))
+    qd, pd = torch.as_tensor(oq).cuda(), torch.as_tensor(op).cuda()
+    gd = torch.zeros((NR, k), dtype=torch.int32, device="cuda")
+    for i in range(k):
+        s3r.s3r_draft_sample(batch, torch.full((NR,), i, dtype=torch.int32, device="cuda"), k, qd,
+                             V, spec.sample_seed, gd, ws)
+    out = torch.full((NR, k + 1), -1, dtype=torch.int32, device="cuda")
+    nout = torch.zeros(NR, dtype=torch.int32, device="cuda")
+    s3r.s3r_spec_sample(batch, k, pd, qd, torch.as_tensor(odrafts).cuda(), V, spec.sample_seed,
+                        out, nout, ws)
+    assert s3r.s3r_get_error(ws) == 0
+    gd, out, nout = gd.cpu().numpy(), out.cpu().numpy(), nout.cpu().numpy()
+    for r in range(NR):
+        toks, n, margins = res_tok[r]
+        for i in range(k):
+            if gd[r, i] != odrafts[r, i]:
+                u0 = float(O.uniform(spec.sample_seed, r, int(lens[r]) + i + 1, O.STREAM_DRAFT))
+                assert O.draft_sample(oq[r, i], u0)[1] < MARGIN, (r, i)
+        if not (nout[r] == n and out[r, :n].tolist() == toks.tolist()):
+            assert margins.min() < MARGIN, r
