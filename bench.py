@@ -73,8 +73,9 @@ def kernel_source_hash(files):
     return h.hexdigest()[:16]
 
 
-VERIFY_SOURCES = ["sparse_dense_kv_b200/csrc/verify.cu", "sparse_dense_kv_b200/csrc/attention.cuh",
-                  "sparse_dense_kv_b200/csrc/common.cuh"]
+VERIFY_SOURCES = ["sparse_dense_kv_b200/csrc/verify_tc.cu", "sparse_dense_kv_b200/csrc/verify.cu",
+                  "sparse_dense_kv_b200/csrc/attention.cuh", "sparse_dense_kv_b200/csrc/common.cuh",
+                  "sparse_dense_kv_b200/csrc/kernels.h"]
 
 
 def verify_traffic_per_launch(workload: str):
