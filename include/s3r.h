@@ -134,6 +134,8 @@ S3R_API int s3r_verify_attn(const s3r_kv_cache* cache, const s3r_batch* batch, i
  *   score_logits, lse  as written by the previous s3r_verify_attn with k = k_prev
  *              (score_logits 16-byte aligned). The exponentials are formed as
  *              2^(x log2(e) - lse log2(e)) in fp32 (relative error about 1e-6).
+ *   Two launches: the scores of every (request, KV head) into the workspace (4 bytes per
+ *   position of the page-table capacity, counted by s3r_workspace_size), then the selection.
  *   sel_idx    int32 [num_requests][H_kv][sel_stride]; n > sel_stride is a device bounds
  *              error. sel_count int32 [num_requests][H_kv].
  * Needs 1 <= budget_bp <= 10000 and window >= k_prev + 1 (so that every scored non-window

@@ -80,6 +80,7 @@ struct SelectParams {
   int sel_stride;
   int32_t* sel_count;
   int* err;
+  float* sigma_buf;        // workspace: sigma [NR][Hkv][cap] of the logits path
 };
 
 struct SampleParams {
@@ -123,7 +124,8 @@ int launch_verify_tc(const CUtensorMap& qm, const CUtensorMap& k1, const CUtenso
 int launch_draft(const DraftParams& p, int D, int batch, int num_sms, cudaStream_t stream);
 size_t draft_partial_bytes(int num_requests, int Hkv, int sel_stride, int D);
 
-int launch_select(const SelectParams& p, int batch, cudaStream_t stream);
+int launch_select(const SelectParams& p, int batch, cudaStream_t stream, int* launches);
+size_t select_sigma_bytes(int num_requests, int Hkv, int cap);
 
 int launch_draft_sample(const SampleParams& p, int batch, cudaStream_t stream);
 int launch_spec_sample(const SampleParams& p, int batch, cudaStream_t stream, int* launches);

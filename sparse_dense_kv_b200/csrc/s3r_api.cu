@@ -272,6 +272,8 @@ size_t s3r_workspace_size(const s3r_kv_cache* cache, int32_t num_requests,
   size_t a = verify_need(cache, num_requests, cap, max_k);
   size_t b = draft_need(cache, num_requests, sel_stride);
   size_t c = sample_need(num_requests, cache->num_kv_heads, max_k, vocab > 0 ? vocab : 1);
+  const size_t d = head_bytes(num_requests) + select_sigma_bytes(num_requests, cache->num_kv_heads, cap);
+  if (d > need) need = d;
   if (a > need) need = a;
   if (b > need) need = b;
   if (c > need) need = c;
@@ -367,8 +369,11 @@ static int select_common(const s3r_kv_cache* cache, const s3r_batch* batch, Sele
     return S3R_ERR_INVALID_ARG;
   if (batch->batch > 65535) return S3R_ERR_UNSUPPORTED;   // grid.y
   if (batch->batch == 0) return S3R_OK;
-  S3R_TRY(check_ws(ws, ws_bytes, head_bytes(batch->num_requests)));
+  const size_t need = head_bytes(batch->num_requests) +
+                      (p.logits ? select_sigma_bytes(batch->num_requests, cache->num_kv_heads, p.cap) : 0);
+  S3R_TRY(check_ws(ws, ws_bytes, need));
   const Carve w = carve(ws, batch->num_requests);
+  if (p.logits) p.sigma_buf = reinterpret_cast<float*>(w.part);
   p.req_ids = batch->req_ids;
   p.seq_lens = batch->seq_lens;
   p.Hq = cache->num_q_heads;
@@ -380,7 +385,10 @@ static int select_common(const s3r_kv_cache* cache, const s3r_batch* batch, Sele
   p.sel_stride = sel_stride;
   p.sel_count = sel_count;
   p.err = w.err;
-  return finish(launch_select(p, batch->batch, (cudaStream_t)stream), 1);
+  int nl = 0;
+  const int st = launch_select(p, batch->batch, (cudaStream_t)stream, &nl);
+  g_launches.fetch_add((uint64_t)nl, std::memory_order_relaxed);
+  return st;
 }
 
 int s3r_select_kv(const s3r_kv_cache* cache, const s3r_batch* batch, const float* score_logits,

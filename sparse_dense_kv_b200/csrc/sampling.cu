@@ -8,16 +8,14 @@
 // The vocabulary is split into chunks of 8192 entries. A pass over (chunk, row, request)
 // produces (max, sum exp(x - max)) per chunk with fp32 exponentials and fp64 sums; the last
 // CTA of a request merges the chunks (ticket, no spinning) and decides. A draw first finds
-// the chunk holding u * Z from the chunk sums, then splits that chunk into 256 segments of
-// 32 entries, one per thread, scans the segment sums and lets the owning thread walk its
-// 32 entries.
+// the chunk holding u * Z from the chunk sums, then the warp holding it (warp totals in
+// order), then, inside that warp's 1024 entries, the row of 32 and the entry.
 #include "common.cuh"
 #include "kernels.h"
 
 namespace s3r {
 
 constexpr int kSampThreads = 256;
-constexpr int kSeg = kVocabChunk / kSampThreads;   // 32 entries per thread in a draw
 
 struct MS {
   float m;
@@ -143,67 +141,88 @@ __device__ double block_sum_d(double v) {
   return r;
 }
 
-// Exclusive block scan of doubles (fixed order: warp shuffles, then warps in order).
-__device__ double block_excl_scan_d(double v, double& total) {
-  __shared__ double sd[kSampThreads / 32];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  double incl = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const double t = __shfl_up_sync(kFull, incl, o);
-    if (lane >= o) incl += t;
-  }
-  if (lane == 31) sd[warp] = incl;
-  __syncthreads();
-  double before = 0.0, tot = 0.0;
-  for (int w = 0; w < kSampThreads / 32; ++w) {
-    before += (w < warp) ? sd[w] : 0.0;
-    tot += sd[w];
-  }
-  __syncthreads();
-  total = tot;
-  return before + incl - v;
-}
-
-// Inverse-CDF search inside [v0, v1): smallest v with target < base + C_v, C the inclusive
-// running sum of weight(v). The chunk is cut into one 32-entry segment per thread; segment
-// bounds come from one block scan and are shared through shared memory, so the segments
-// partition [base, base + total) exactly and at most one thread owns the target.
-// Returns -1 if the target lies past the chunk; `base` then moves to the chunk's end.
+// Inverse-CDF search inside [v0, v1) (at most kVocabChunk entries): smallest v with
+// target < base + C_v, C the inclusive running sum of weight(v). Warp w takes the 1024
+// entries v0 + 1024 w + 32 m + lane (m = 0..31: coalesced loads, weights kept in
+// registers); the warps' totals, in order, find the warp holding the target; that warp
+// reduces its 32 rows of 32 entries with a butterfly (lane m ends with row m's sum),
+// scans the rows, then the lanes of the chosen row. Returns -1 if the target lies past the
+// chunk; `base` then moves to the chunk's end.
 template <class W>
 __device__ int chunk_search(int v0, int v1, double target, double& base, W weight) {
-  __shared__ double hi_s[kSampThreads];
+  __shared__ double wtot_s[kSampThreads / 32];
   __shared__ int s_tok;
-  const int t = threadIdx.x;
-  const int a = v0 + t * kSeg;
-  const int b = min(a + kSeg, v1);
-  float segf = 0.f;
-  for (int v = a; v < b; ++v) segf += weight(v);
-  const double seg = segf;
-  double total;
-  const double excl = block_excl_scan_d(seg, total);
-  hi_s[t] = base + (excl + seg);
-  if (t == 0) s_tok = -1;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int wb = v0 + warp * 1024;
+  float w[32];
+  float part = 0.f;
+#pragma unroll
+  for (int m = 0; m < 32; ++m) {
+    const int v = wb + 32 * m + lane;
+    w[m] = v < v1 ? weight(v) : 0.f;
+    part += w[m];
+  }
+  const double wt = warp_sum_d((double)part);
+  if (lane == 0) wtot_s[warp] = wt;
+  if (threadIdx.x == 0) s_tok = -1;
   __syncthreads();
-  const double lo = t ? hi_s[t - 1] : base;
-  const double hi = hi_s[t];
-  if (seg > 0.0 && target >= lo && target < hi) {
-    double c = lo;
-    int tok = -1, last_nz = -1;
-    for (int v = a; v < b; ++v) {
-      const double wv = weight(v);
-      if (wv > 0.0) last_nz = v;
-      c += wv;
-      if (target < c) {
-        tok = v;
-        break;
+  double lo = base, total = 0.0;
+  for (int q = 0; q < kSampThreads / 32; ++q) {
+    if (q < warp) lo += wtot_s[q];
+    total += wtot_s[q];
+  }
+  if (wt > 0.0 && target >= lo && target < lo + wt) {
+    // butterfly (in place): afterwards lane l holds row l's total in w[0]
+#pragma unroll
+    for (int k = 16; k >= 1; k >>= 1) {
+      const bool up = (lane & k) != 0;
+#pragma unroll
+      for (int i = 0; i < k; ++i) {
+        const float send = up ? w[i] : w[i + k];
+        const float keep = up ? w[i + k] : w[i];
+        w[i] = keep + __shfl_xor_sync(kFull, send, k);
       }
     }
-    atomicMax(&s_tok, tok < 0 ? last_nz : tok);
+    const double rs = w[0];
+    double incl = rs;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const double t = __shfl_up_sync(kFull, incl, o);
+      if (lane >= o) incl += t;
+    }
+    // row: the first with target < lo + (rows up to and including it)
+    const unsigned rowhit = __ballot_sync(kFull, rs > 0.0 && target < lo + incl);
+    int tok = -1;
+    if (rowhit) {
+      const int mr = __ffs(rowhit) - 1;
+      const double rbase = lo + __shfl_sync(kFull, incl - rs, mr);
+      const int vx = wb + 32 * mr + lane;   // the row's weights again (same values)
+      const float x = vx < v1 ? weight(vx) : 0.f;
+      double li = x;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const double t = __shfl_up_sync(kFull, li, o);
+        if (lane >= o) li += t;
+      }
+      const unsigned hit = __ballot_sync(kFull, x > 0.f && target < rbase + li);
+      // rounding past the row's last entry: its last non-zero entry
+      const unsigned nz = __ballot_sync(kFull, x > 0.f);
+      const int ln = hit ? __ffs(hit) - 1 : 31 - __clz((int)nz);
+      tok = wb + 32 * mr + ln;
+    } else {
+      // rounding past the warp's last row: the last non-zero entry of the warp
+      const unsigned nzr = __ballot_sync(kFull, rs > 0.0);
+      const int mr = 31 - __clz((int)nzr);
+      const int vx = wb + 32 * mr + lane;
+      const float x = vx < v1 ? weight(vx) : 0.f;
+      const unsigned nz = __ballot_sync(kFull, x > 0.f);
+      tok = wb + 32 * mr + (31 - __clz((int)nz));
+    }
+    if (lane == 0) s_tok = tok;
   }
   __syncthreads();
   const int tok = s_tok;
-  base = hi_s[kSampThreads - 1];
+  base += total;
   __syncthreads();
   return tok;
 }

@@ -58,7 +58,6 @@ __device__ __forceinline__ int block_excl_scan(int v, int* wsum) {
 __global__ void __launch_bounds__(kSelectThreads, 2) select_kernel(const SelectParams p) {
   extern __shared__ uint32_t keys[];
   __shared__ uint32_t hist[kSelectBins];
-  __shared__ float lse_s[S3R_MAX_ROWS];
   __shared__ int wsum[32], wa[32], wb[32];
   __shared__ uint32_t s_prefix;
   __shared__ int s_remaining;
@@ -67,8 +66,7 @@ __global__ void __launch_bounds__(kSelectThreads, 2) select_kernel(const SelectP
   const int kvh = blockIdx.x, bl = blockIdx.y;
   const int r = p.req_ids ? p.req_ids[bl] : bl;
   const int L = p.seq_lens[r];
-  const int lim = p.logits ? p.cap : p.score_stride;
-  if (L < 0 || L > lim) {
+  if (L < 0 || L > p.score_stride) {
     if (tid == 0) set_error(p.err, S3R_ERR_DEVICE_BOUNDS);
     return;
   }
@@ -91,62 +89,13 @@ __global__ void __launch_bounds__(kSelectThreads, 2) select_kernel(const SelectP
 
   // ---- scores -> order-preserving keys in shared memory
   bool bad = false;
-  if (p.logits) {
-    // sigma_j = sum over rows of 2^(logit * log2(e) - lse * log2(e)); the logits of one row
-    // are contiguous over positions ([..][R][cap]), so every thread takes 4 consecutive
-    // positions with one 16-byte load per row, four rows in flight at a time
-    for (int row = tid; row < p.R; row += blockDim.x) {
-      const int t = row / p.G, g = row - t * p.G;
-      lse_s[row] = p.lse[((size_t)r * p.T + t) * p.Hq + kvh * p.G + g] * kLog2e;
+  for (int j = tid; j < N; j += blockDim.x) {
+    float sigma = p.scores[((size_t)r * p.Hkv + kvh) * p.score_stride + j];
+    if (!isfinite(sigma)) {
+      bad = true;
+      sigma = -INFINITY;
     }
-    __syncthreads();
-    const float* base = p.logits + ((size_t)r * p.Hkv + kvh) * (size_t)p.R * p.cap;
-    for (int j4 = 4 * tid; j4 < N; j4 += 4 * blockDim.x) {
-      float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
-      int row = 0;
-      for (; row + 4 <= p.R; row += 4) {
-        float4 x[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-          x[u] = __ldg(reinterpret_cast<const float4*>(base + (size_t)(row + u) * p.cap + j4));
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float l2 = lse_s[row + u];
-          acc0 += ex2(fmaf(x[u].x, kLog2e, -l2));
-          acc1 += ex2(fmaf(x[u].y, kLog2e, -l2));
-          acc2 += ex2(fmaf(x[u].z, kLog2e, -l2));
-          acc3 += ex2(fmaf(x[u].w, kLog2e, -l2));
-        }
-      }
-      for (; row < p.R; ++row) {
-        const float4 x = __ldg(reinterpret_cast<const float4*>(base + (size_t)row * p.cap + j4));
-        const float l2 = lse_s[row];
-        acc0 += ex2(fmaf(x.x, kLog2e, -l2));
-        acc1 += ex2(fmaf(x.y, kLog2e, -l2));
-        acc2 += ex2(fmaf(x.z, kLog2e, -l2));
-        acc3 += ex2(fmaf(x.w, kLog2e, -l2));
-      }
-      const float sg[4] = {acc0, acc1, acc2, acc3};
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        if (j4 + q >= N) break;
-        float sigma = sg[q];
-        if (!isfinite(sigma)) {
-          bad = true;
-          sigma = -INFINITY;
-        }
-        keys[j4 + q] = order_key(sigma);
-      }
-    }
-  } else {
-    for (int j = tid; j < N; j += blockDim.x) {
-      float sigma = p.scores[((size_t)r * p.Hkv + kvh) * p.score_stride + j];
-      if (!isfinite(sigma)) {
-        bad = true;
-        sigma = -INFINITY;
-      }
-      keys[j] = order_key(sigma);
-    }
+    keys[j] = order_key(sigma);
   }
   if (bad) set_error(p.err, S3R_ERR_NONFINITE);
   __syncthreads();
@@ -274,8 +223,73 @@ __global__ void __launch_bounds__(kSelectThreads, 2) select_kernel(const SelectP
   }
 }
 
-int launch_select(const SelectParams& p, int batch, cudaStream_t stream) {
-  const int lim = p.logits ? p.cap : p.score_stride;
+// ---- scores from a verify's logits: sigma_j = sum over the G*(k+1) rows of
+// 2^(logit * log2(e) - lse * log2(e)) for every non-window position j < L - min(W, L),
+// written as fp32 [NR][Hkv][cap]. A flat grid over (block of 1024 positions, KV head,
+// request) at full occupancy: the logits of one row are contiguous over positions, each
+// thread takes 4 positions and keeps 8 rows' 16-byte loads in flight.
+constexpr int kSigmaThreads = 256;
+constexpr int kSigmaPos = 4 * kSigmaThreads;
+
+__global__ void __launch_bounds__(kSigmaThreads) sigma_kernel(const SelectParams p) {
+  __shared__ float lse2[S3R_MAX_ROWS];
+  const int kvh = blockIdx.y, bl = blockIdx.z;
+  const int r = p.req_ids ? p.req_ids[bl] : bl;
+  const int L = p.seq_lens[r];
+  if (L < 0 || L > p.cap) return;   // reported by the select kernel
+  const int N = L - min(p.window, L);
+  const int j0 = blockIdx.x * kSigmaPos;
+  if (j0 >= N) return;
+  for (int row = threadIdx.x; row < p.R; row += blockDim.x) {
+    const int t = row / p.G, g = row - t * p.G;
+    lse2[row] = p.lse[((size_t)r * p.T + t) * p.Hq + kvh * p.G + g] * kLog2e;
+  }
+  __syncthreads();
+  const int j4 = j0 + 4 * (int)threadIdx.x;
+  if (j4 >= N) return;
+  const float* base = p.logits + ((size_t)r * p.Hkv + kvh) * (size_t)p.R * p.cap + j4;
+  float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+  for (int row0 = 0; row0 < p.R; row0 += 8) {
+    float4 x[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (row0 + u < p.R) x[u] = __ldg(reinterpret_cast<const float4*>(base + (size_t)(row0 + u) * p.cap));
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (row0 + u >= p.R) break;
+      const float l2 = lse2[row0 + u];
+      acc0 += ex2(fmaf(x[u].x, kLog2e, -l2));
+      acc1 += ex2(fmaf(x[u].y, kLog2e, -l2));
+      acc2 += ex2(fmaf(x[u].z, kLog2e, -l2));
+      acc3 += ex2(fmaf(x[u].w, kLog2e, -l2));
+    }
+  }
+  float* out = p.sigma_buf + ((size_t)r * p.Hkv + kvh) * p.cap + j4;
+  if (j4 + 4 <= N) {
+    *reinterpret_cast<float4*>(out) = make_float4(acc0, acc1, acc2, acc3);
+  } else {
+    const float sg[4] = {acc0, acc1, acc2, acc3};
+    for (int q = 0; q < N - j4; ++q) out[q] = sg[q];
+  }
+}
+
+size_t select_sigma_bytes(int num_requests, int Hkv, int cap) {
+  return align_up((size_t)num_requests * Hkv * cap * 4, 256);
+}
+
+int launch_select(const SelectParams& p, int batch, cudaStream_t stream, int* launches) {
+  *launches = 0;
+  SelectParams q = p;
+  if (p.logits) {
+    dim3 g((p.cap + kSigmaPos - 1) / kSigmaPos, p.Hkv, batch);
+    sigma_kernel<<<g, kSigmaThreads, 0, stream>>>(p);
+    if (cuda_status(cudaGetLastError(), "sigma_kernel") != S3R_OK) return S3R_ERR_CUDA;
+    ++*launches;
+    q.logits = nullptr;
+    q.scores = p.sigma_buf;
+    q.score_stride = p.cap;
+  }
+  const int lim = q.score_stride;
   const int nmax = lim < kSelectMaxN ? lim : kSelectMaxN;
   const size_t smem = (size_t)(nmax > 0 ? nmax : 1) * 4;
   static bool attr_done = false;
@@ -286,9 +300,11 @@ int launch_select(const SelectParams& p, int batch, cudaStream_t stream) {
       return S3R_ERR_CUDA;
     attr_done = true;
   }
-  dim3 grid(p.Hkv, batch);
-  select_kernel<<<grid, kSelectThreads, smem, stream>>>(p);
-  return cuda_status(cudaGetLastError(), __func__);
+  dim3 grid(q.Hkv, batch);
+  select_kernel<<<grid, kSelectThreads, smem, stream>>>(q);
+  const int st = cuda_status(cudaGetLastError(), __func__);
+  if (st == S3R_OK) ++*launches;
+  return st;
 }
 
 }  // namespace s3r

@@ -6,24 +6,32 @@
 // comes from the verifier's last attention pass): rows (t, g) at positions L+t attend
 // positions 0..L+t; out, lse and every committed logit are written.
 //
-// Organisation (one persistent CTA per SM, 6 warps):
-//   warp 0     producer: per work item (request, KV head, chunk of up to 8 tiles of 128
-//              positions) it copies the item's Q rows into shared memory, then streams the
-//              chunk's K tiles and then its V tiles through a 4-stage ring with 4-D TMA over
-//              (d, slot, head, page): a tile of 8 consecutive page ids is 2 boxes (one per
-//              64-column half, 128-byte swizzle), otherwise one box per page and half. The
-//              tile holding the block (positions >= L) is patched after its TMA lands.
-//   warp 1     MMA issuer: S^T tile t (128 positions x N rows, fp32) = K_t . Q^T into tensor
-//              memory columns [t*N, t*N+N) for every tile of the chunk, then, once the
-//              softmax warps have written P^T, O^T (128 d x N) = sum_t V_t^T . P_t^T into the
-//              columns after them. K and Q are K-major operands (128-byte swizzle); V^T is
-//              MN-major (the V tile as it arrives, 128-byte swizzle) and so is P^T (one row of
-//              N values per position, 32- or 64-byte swizzle).
-//   warps 2-5  softmax / epilogue (one thread per tensor-memory lane = position or d):
-//              pass 1 reads every S tile, writes the committed logits and takes the chunk
-//              maximum per row; pass 2 re-reads them and writes P = 2^(s - max) as bf16 P^T
-//              tiles; then the chunk record (max, sum, O) goes to the workspace, and a small
-//              second kernel merges the chunks of every (request, KV head).
+// Organisation (one persistent CTA per SM, 11 warps). A work item is (request, KV head,
+// chunk of up to 7 or 8 tiles of 128 positions).
+//   warp 0     K producer: per item it loads the item's Q rows into one of two Q buffers
+//              (3-D TMA box, rows t*G+g), then streams the chunk's K tiles through a
+//              2-stage ring with 4-D TMA over (d, slot, head, page): a tile of 8
+//              consecutive page ids is 2 boxes (one per 64-column half, 128-byte swizzle),
+//              otherwise one box per page and half. The tile holding the block (positions
+//              >= L) is patched after its TMA lands. It also writes the block into the cache.
+//   warp 1     V producer: the same for the V tiles, through its own 2-stage ring, so the
+//              K stream of item n+1 and the V stream of item n run side by side.
+//   warp 2     MMA issuer: two queues in order, S^T tile t (128 positions x N rows, fp32) =
+//              K_t . Q^T into tensor memory for the QK of item m, and O^T (128 d x N) +=
+//              V_t^T . P_t^T for the PV of item n < m; whichever has its next tile ready is
+//              issued. K and Q are K-major operands (128-byte swizzle); V^T is MN-major (the V
+//              tile as it arrives) and so is P^T (one row of N values per position, 32- or
+//              64-byte swizzle). S and O are double-buffered in tensor memory.
+//   warps 3-10 softmax / epilogue, two warpgroups each owning half of the rows (one thread
+//              per tensor-memory lane = position or d): pass 1 reads every S tile, writes the
+//              committed logits and takes the chunk maximum per row; pass 2 re-reads them and
+//              writes P = 2^(s - max) as bf16 P^T tiles. P^T is single-buffered: a tile is
+//              rewritten for item n+1 once the PV of item n has read it (a barrier per
+//              tile), so that PV and pass 2 of item n+1 overlap; the PV of an item starts
+//              once its whole P^T is written. Then the chunk record (max, sum, O) goes to the
+//              workspace, and a small second kernel merges the chunks of every (request, KV
+//              head).
+// Every wait is bounded (an expired wait sets S3R_ERR_TIMEOUT and the CTA winds down).
 // The softmax is exact per chunk (two passes over logits resident in tensor memory), so no
 // running rescale exists; chunks merge by their (max, sum) as in the CUDA-core kernel.
 #include "attention.cuh"
@@ -181,15 +189,13 @@ struct Bars {
   uint64_t q_full[2], q_empty[2], p_full, fin;
   uint64_t s_full[2], s_empty[2], o_full[2], o_empty[2];
   uint64_t p_free[8];   // P^T tile t has been read by the PV of the previous chunk
+  uint64_t wg[2];       // barrier of each softmax warpgroup (4 warps)
   uint32_t tmem_base;
   int abort_flag;
 };
 static_assert(sizeof(Bars) <= kBarBytes, "barrier block");
 
-// Barrier of one softmax warpgroup (named barriers 1 and 2, 128 threads each).
-__device__ __forceinline__ void wg_sync(int sg) {
-  asm volatile("bar.sync %0, 128;\n" ::"r"(1 + sg) : "memory");
-}
+
 
 // Work item i of the launch -> (launch-local request, KV head, chunk), from the prefix of
 // per-request item counts (items of request b = Hkv * chunks_b).
@@ -250,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ int trow[NP];   // block row t of query row j (j / G)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int T = p.T, G = p.G, R = p.R, Hkv = p.Hkv, Hq = p.Hq;
+  const int T = p.T, G = p.G, R = p.R, Hkv = p.Hkv;
   const int chunk = C::kChunk;
   const uint32_t sbase = smem_u32(smem);
 
@@ -310,6 +316,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(smem_u32(&B->p_full), 8);
     for (int t = 0; t < 8; ++t) mbar_init(smem_u32(&B->p_free[t]), 1);
+    mbar_init(smem_u32(&B->wg[0]), 4);
+    mbar_init(smem_u32(&B->wg[1]), 4);
     mbar_init(smem_u32(&B->fin), 1);
     B->abort_flag = 0;
     fence_mbar_init();
@@ -613,6 +621,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
     const float scale = p.scale, scale2 = p.scale * kLog2e;
     const int swz_row = (NP == 16) ? ((lrow >> 2) & 1) : ((lrow >> 1) & 3);
+    // Warpgroup barrier on an mbarrier (bounded wait, unlike bar.sync): if a wait anywhere
+    // gives up, the other warps of the group give up here too instead of hanging.
+    uint32_t wg_phase = 0;
+    auto wg_sync = [&]() -> bool {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&B->wg[sg]));
+      const bool r = wait_bar(smem_u32(&B->wg[sg]), wg_phase, abort_flag, p.err);
+      wg_phase ^= 1u;
+      return r;
+    };
 
     // record of chunk m (this warpgroup's rows): O^T buffer m&1 -> workspace, with the rows'
     // max / sum from cm / cl
@@ -691,14 +709,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
         if (lane == j) redM[(sg * 4 + sw4) * NH + j] = m;
       }
-      wg_sync(sg);
+      if (!wg_sync()) {
+        ok = false;
+        break;
+      }
       if (gt < NH) {
         float m = redM[(sg * 4) * NH + gt];
 #pragma unroll
         for (int w = 1; w < 4; ++w) m = fmaxf(m, redM[(sg * 4 + w) * NH + gt]);
         cm[(n & 1) * NP + c0 + gt] = scale2 * m;
       }
-      wg_sync(sg);
+      if (!wg_sync()) {
+        ok = false;
+        break;
+      }
 #pragma unroll
       for (int j = 0; j < NH; ++j) mrow[j] = cm[(n & 1) * NP + c0 + j];
 
@@ -771,7 +795,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int o = 16; o; o >>= 1) sacc += __shfl_xor_sync(kFull, sacc, o);
         if (lane == j) redL[(sg * 4 + sw4) * NH + j] = sacc;
       }
-      wg_sync(sg);
+      if (!wg_sync()) {
+        ok = false;
+        break;
+      }
       if (gt < NH) {
         float l = 0.f;
 #pragma unroll
@@ -781,8 +808,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // (cl / redL reuse is ordered by the barriers of the next chunk)
     }
     if (ok && my_items > 0 && !aborted(abort_flag)) {
-      wg_sync(sg);   // cl of the last chunk complete
-      epilogue(my_items - 1);
+      if (wg_sync()) epilogue(my_items - 1);   // cl of the last chunk complete
     }
   }
 

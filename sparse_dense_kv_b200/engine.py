@@ -68,7 +68,7 @@ class S3REngine:
 
     @property
     def launches_per_round(self) -> int:
-        return 1 + 2 * self.k + 2 + 2 + 1   # select, k x (draft, sample), verify (+merge), spec (2), commit
+        return 2 + 2 * self.k + 2 + 2 + 1   # select (sigma + select), k x (draft, sample), verify (+merge), spec (2), commit
 
     def prefill(self, q_x, k_x, v_x):
         """One-row dense pass of each request's pending token at position L (the last step of
