@@ -10,7 +10,7 @@ namespace s3r {
 
 constexpr int kVerifyChunk = 1024;   // positions per verify CTA (multiple of 64)
 constexpr int kVerifyChunkMin = 896; // smallest verify chunk of any kernel (workspace sizing)
-constexpr int kDraftChunk = 256;     // positions per draft CTA (multiple of 64)
+constexpr int kDraftChunk = 512;     // positions per draft CTA (multiple of 128)
 constexpr int kVocabChunk = 8192;    // vocabulary entries per sampler CTA
 
 struct VerifyParams {

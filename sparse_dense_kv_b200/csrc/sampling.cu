@@ -415,9 +415,41 @@ __global__ void __launch_bounds__(kSampThreads) spec_draw_kernel(const SamplePar
 
   const int v0 = c * kVocabChunk, v1 = min(V, (c + 1) * kVocabChunk);
   float srf = 0.f, spf = 0.f;
-  for (int v = v0 + threadIdx.x; v < v1; v += blockDim.x) {
-    spf += w_p(v);
-    if (resid) srf += w_res(v);
+  auto wp_x = [&](float x) -> float {
+    return (isnan(x) || x == INFINITY) ? 0.f : ex2(fmaf(x, kLog2e, -mpb));
+  };
+  auto wres_xy = [&](float x, float y) -> float {
+    const float pv = (isnan(x) || x == INFINITY) ? 0.f : ex2(fmaf(x, kLog2e, -mpb)) * izp;
+    const float qv = (isnan(y) || y == INFINITY) ? 0.f : ex2(fmaf(y, kLog2e, -mqb)) * izq;
+    return fmaxf(pv - qv, 0.f);
+  };
+  const bool vec = ((reinterpret_cast<uintptr_t>(prow + v0) & 15u) == 0) &&
+                   ((reinterpret_cast<uintptr_t>(qrow + v0) & 15u) == 0) && (((v1 - v0) & 3) == 0);
+  if (vec) {
+    // 32 entries per thread as eight 16-byte loads of each row, all in flight at once
+    float4 xp[8], xq[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int v = v0 + 4 * ((int)threadIdx.x + kSampThreads * j);
+      xp[j] = v < v1 ? __ldg(reinterpret_cast<const float4*>(prow + v)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      xq[j] = (resid && v < v1) ? __ldg(reinterpret_cast<const float4*>(qrow + v))
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int v = v0 + 4 * ((int)threadIdx.x + kSampThreads * j);
+      if (v < v1) {
+        spf += wp_x(xp[j].x) + wp_x(xp[j].y) + wp_x(xp[j].z) + wp_x(xp[j].w);
+        if (resid)
+          srf += wres_xy(xp[j].x, xq[j].x) + wres_xy(xp[j].y, xq[j].y) +
+                 wres_xy(xp[j].z, xq[j].z) + wres_xy(xp[j].w, xq[j].w);
+      }
+    }
+  } else {
+    for (int v = v0 + threadIdx.x; v < v1; v += blockDim.x) {
+      spf += w_p(v);
+      if (resid) srf += w_res(v);
+    }
   }
   double sr = srf, sp = spf;
   sp = block_sum_d(sp);
