@@ -331,6 +331,34 @@ def spec_sample(p_logits, q_logits, drafts, seed: int, request: int, L: int):
 
 
 # ----------------------------------------------------------------------------------------
+# Greedy (temperature 0) mode. [Listing] Table 4 setting (component measurements decode
+# greedily): the draft token is the draft row's argmax, a draft is kept while it equals the
+# target row's argmax, the first mismatch is replaced by the target argmax, and when all k
+# agree the bonus token is the last target row's argmax. Ties go to the lowest token id;
+# NaN logits count as -inf.
+# ----------------------------------------------------------------------------------------
+def argmax_token(logits_row) -> int:
+    x = np.asarray(logits_row, dtype=np.float64)
+    x = np.where(np.isnan(x), -np.inf, x)
+    return int(np.argmax(x))   # numpy returns the first (lowest) index of the maximum
+
+
+def greedy_verify(p_logits, drafts):
+    """Tokens emitted by greedy verification: (tokens [a+1], n_out = a+1)."""
+    k = len(drafts)
+    tokens = []
+    for j in range(k):
+        t = argmax_token(p_logits[j])
+        if t == int(drafts[j]):
+            tokens.append(t)
+            continue
+        tokens.append(t)
+        return np.asarray(tokens, dtype=np.int32), len(tokens)
+    tokens.append(argmax_token(p_logits[k]))
+    return np.asarray(tokens, dtype=np.int32), len(tokens)
+
+
+# ----------------------------------------------------------------------------------------
 # O-round: one draft+verify round of one request, composed from the steps above.
 # [Explainer] walkthrough: draft k tokens from the sparse set, check all at once with one
 # full pass, keep the agreeing prefix, replace the first mismatch, drop the rest.
