@@ -214,6 +214,21 @@ S3R_API int s3r_spec_sample(const s3r_batch* batch, int32_t k, const float* p_lo
                     uint64_t seed, int32_t* out_tokens, int32_t* n_out, void* ws,
                     size_t ws_bytes, s3r_stream_t stream);
 
+/* Greedy (temperature 0) mode ([Listing] Table 4 setting: component measurements decode
+ * greedily). s3r_draft_argmax: draft_tokens[r][i] = argmax of q_logits[r][i], i =
+ * draft_step[r]. s3r_greedy_verify: with t_j = argmax of p_logits[r][j], drafts are kept
+ * while draft_tokens[r][j] == t_j; out_tokens[r][0..a] = t_0..t_a (a = drafts kept, the
+ * last one the replacement of the first mismatch or, when all k agree, the bonus t_k);
+ * n_out[r] = a + 1. Ties go to the lowest token id; NaN logits count as -inf and set
+ * S3R_ERR_NONFINITE. Layouts, workspace and limits as s3r_draft_sample / s3r_spec_sample;
+ * one launch each. */
+S3R_API int s3r_draft_argmax(const s3r_batch* batch, const int32_t* draft_step, int32_t k,
+                     const float* q_logits, int32_t vocab, int32_t* draft_tokens, void* ws,
+                     size_t ws_bytes, s3r_stream_t stream);
+S3R_API int s3r_greedy_verify(const s3r_batch* batch, int32_t k, const float* p_logits,
+                     const int32_t* draft_tokens, int32_t vocab, int32_t* out_tokens,
+                     int32_t* n_out, void* ws, size_t ws_bytes, s3r_stream_t stream);
+
 /* Commit a round ([Explainer] Jargon, block efficiency: tokens per round): for each
  * request of the batch, seq_lens[r] += n_out[r]. stats (int64, may be NULL) accumulates
  * [0] tokens emitted, [1] request-rounds, [2+j] drafts accepted at position j and

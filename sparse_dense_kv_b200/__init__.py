@@ -16,9 +16,11 @@ from ._lib import (  # noqa: F401
     make_cache,
     new_workspace,
     s3r_commit,
+    s3r_draft_argmax,
     s3r_draft_sample,
     s3r_draft_sample_noalloc,
     s3r_get_error,
+    s3r_greedy_verify,
     s3r_launch_count,
     s3r_philox,
     s3r_select_from_scores,

@@ -61,6 +61,8 @@ def _load():
         "s3r_draft_sample": (ctypes.c_int, [B, P, I32, P, I32, U64, P, P, SZ, P]),
         "s3r_draft_sample_noalloc": (ctypes.c_int, [B, P, I32, P, I32, U64, P, P, P]),
         "s3r_spec_sample": (ctypes.c_int, [B, I32, P, P, P, I32, U64, P, P, P, SZ, P]),
+        "s3r_draft_argmax": (ctypes.c_int, [B, P, I32, P, I32, P, P, SZ, P]),
+        "s3r_greedy_verify": (ctypes.c_int, [B, I32, P, P, I32, P, P, P, SZ, P]),
         "s3r_commit": (ctypes.c_int, [B, I32, P, P, P, P]),
         "s3r_philox": (ctypes.c_int, [U64, I32, P, P, I64, P, P, P]),
         "s3r_get_error": (ctypes.c_int, [P, P, P]),
@@ -246,6 +248,23 @@ def s3r_spec_sample(batch, k, p_logits, q_logits, draft_tokens, vocab, seed, out
         _ptr(draft_tokens, i32, "draft_tokens", allow_none=(k == 0)), vocab, seed,
         _ptr(out_tokens, i32, "out_tokens"), _ptr(n_out, i32, "n_out"),
         _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)), "s3r_spec_sample")
+
+
+def s3r_draft_argmax(batch, draft_step, k, q_logits, vocab, draft_tokens, ws, stream=None):
+    _check(_lib.s3r_draft_argmax(
+        ctypes.byref(batch), _ptr(draft_step, torch.int32, "draft_step"), k,
+        _ptr(q_logits, torch.float32, "q_logits"), vocab,
+        _ptr(draft_tokens, torch.int32, "draft_tokens"), _ptr(ws, torch.uint8, "ws"), ws.numel(),
+        _stream(stream)), "s3r_draft_argmax")
+
+
+def s3r_greedy_verify(batch, k, p_logits, draft_tokens, vocab, out_tokens, n_out, ws, stream=None):
+    i32 = torch.int32
+    _check(_lib.s3r_greedy_verify(
+        ctypes.byref(batch), k, _ptr(p_logits, torch.float32, "p_logits"),
+        _ptr(draft_tokens, i32, "draft_tokens", allow_none=(k == 0)), vocab,
+        _ptr(out_tokens, i32, "out_tokens"), _ptr(n_out, i32, "n_out"),
+        _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)), "s3r_greedy_verify")
 
 
 def s3r_commit(batch, k, n_out, seq_lens, stats=None, stream=None):

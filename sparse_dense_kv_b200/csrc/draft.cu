@@ -6,11 +6,11 @@
 // query rows of each KV head attend A_i = S ∪ {L, .., L+i}, S the selected positions.
 //
 // Layout of the work: grid (chunk of A_i, kv_head, request), 128 threads. The CTA first
-// resolves the element offsets of its <= 256 positions (index -> page -> slot), then
-// gathers 256-byte K and V rows with 16-byte cp.async (16 lanes per row, coalesced) into a
-// 3-stage pipeline laid out like the TMA tiles of the verify (128-byte swizzle), so the
-// same tensor-core step (one n-tile of 8 rows per warp) serves both. Chunks merge through
-// the workspace in the last CTA of the (request, head).
+// resolves the element offsets of its <= kDraftChunk (512) positions (index -> page ->
+// slot), then gathers 256-byte K and V rows with 16-byte cp.async (16 lanes per row,
+// coalesced) into a 2-stage pipeline laid out like the TMA tiles of the verify (128-byte
+// swizzle), so the same tensor-core step (one n-tile of 8 rows per warp) serves both.
+// Chunks merge through the workspace in the last CTA of the (request, head).
 #include "attention.cuh"
 #include "kernels.h"
 

@@ -129,6 +129,8 @@ size_t select_sigma_bytes(int num_requests, int Hkv, int cap);
 
 int launch_draft_sample(const SampleParams& p, int batch, cudaStream_t stream);
 int launch_spec_sample(const SampleParams& p, int batch, cudaStream_t stream, int* launches);
+// Greedy mode: mode 0 draft argmax, mode 1 greedy verification.
+int launch_argmax(const SampleParams& p, int batch, int mode, cudaStream_t stream);
 // Bytes of one per-(request, vocabulary chunk) partial of the samplers.
 constexpr int kSamplePartialBytes = 16;
 size_t sample_partial_bytes(int num_requests, int k, int vocab);

@@ -589,6 +589,64 @@ int s3r_spec_sample(const s3r_batch* batch, int32_t k, const float* p_logits,
   return st;
 }
 
+int s3r_draft_argmax(const s3r_batch* batch, const int32_t* draft_step, int32_t k,
+                     const float* q_logits, int32_t vocab, int32_t* draft_tokens, void* ws,
+                     size_t ws_bytes, s3r_stream_t stream) {
+  S3R_TRY(check_batch(batch, false));
+  if (k < 1 || k > S3R_MAX_K) return S3R_ERR_UNSUPPORTED;
+  if (vocab < 1 || vocab > 64 * kVocabChunk) return S3R_ERR_UNSUPPORTED;
+  if (!draft_step || !q_logits || !draft_tokens || !aligned4(draft_step) ||
+      !aligned4(q_logits) || !aligned4(draft_tokens))
+    return S3R_ERR_INVALID_ARG;
+  if (batch->batch == 0) return S3R_OK;
+  S3R_TRY(check_ws(ws, ws_bytes, sample_need(batch->num_requests, 1, k, vocab)));
+  const Carve w = carve(ws, batch->num_requests);
+  SampleParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.req_ids = batch->req_ids;
+  p.seq_lens = batch->seq_lens;
+  p.draft_step = draft_step;
+  p.k = k;
+  p.vocab = vocab;
+  p.nvch = nvch_of(vocab);
+  p.q_logits = q_logits;
+  p.draft_out = draft_tokens;
+  p.err = w.err;
+  p.tickets = w.tickets;
+  p.part = w.part;
+  return finish(launch_argmax(p, batch->batch, 0, (cudaStream_t)stream), 1);
+}
+
+int s3r_greedy_verify(const s3r_batch* batch, int32_t k, const float* p_logits,
+                      const int32_t* draft_tokens, int32_t vocab, int32_t* out_tokens,
+                      int32_t* n_out, void* ws, size_t ws_bytes, s3r_stream_t stream) {
+  S3R_TRY(check_batch(batch, false));
+  if (k < 0 || k > S3R_MAX_K) return S3R_ERR_UNSUPPORTED;
+  if (vocab < 1 || vocab > 64 * kVocabChunk) return S3R_ERR_UNSUPPORTED;
+  if (!p_logits || !out_tokens || !n_out || !aligned4(p_logits) || !aligned4(out_tokens) ||
+      !aligned4(n_out))
+    return S3R_ERR_INVALID_ARG;
+  if (k > 0 && (!draft_tokens || !aligned4(draft_tokens))) return S3R_ERR_INVALID_ARG;
+  if (batch->batch == 0) return S3R_OK;
+  S3R_TRY(check_ws(ws, ws_bytes, sample_need(batch->num_requests, 1, k, vocab)));
+  const Carve w = carve(ws, batch->num_requests);
+  SampleParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.req_ids = batch->req_ids;
+  p.seq_lens = batch->seq_lens;
+  p.k = k;
+  p.vocab = vocab;
+  p.nvch = nvch_of(vocab);
+  p.p_logits = p_logits;
+  p.draft_tokens = draft_tokens;
+  p.out_tokens = out_tokens;
+  p.n_out = n_out;
+  p.err = w.err;
+  p.tickets = w.tickets;
+  p.part = w.part;
+  return finish(launch_argmax(p, batch->batch, 1, (cudaStream_t)stream), 1);
+}
+
 int s3r_commit(const s3r_batch* batch, int32_t k, const int32_t* n_out, int32_t* seq_lens,
                int64_t* stats, s3r_stream_t stream) {
   S3R_TRY(check_batch(batch, false));

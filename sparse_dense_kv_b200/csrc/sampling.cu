@@ -10,6 +10,8 @@
 // CTA of a request merges the chunks (ticket, no spinning) and decides. A draw first finds
 // the chunk holding u * Z from the chunk sums, then the warp holding it (warp totals in
 // order), then, inside that warp's 1024 entries, the row of 32 and the entry.
+#include <climits>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -479,6 +481,118 @@ __global__ void __launch_bounds__(kSampThreads) spec_draw_kernel(const SamplePar
   if (s_use_res) tok = draw_token(V, p.nvch, csum, target, w_res);
   else tok = draw_token(V, p.nvch, csum, target, w_p);
   if (threadIdx.x == 0) p.out_tokens[(size_t)r * (k + 1) + pl.a] = tok;
+}
+
+// ------------------------------------------------------------ greedy (temperature 0) ----
+// Argmax of logit rows, ties to the lowest token id, NaN counted as -inf (and flagged).
+// mode 0: one row per request, the draft row of its step -> draft_tokens.
+// mode 1: the k+1 target rows of each request -> drafts kept while they equal the target
+//         argmax, the first mismatch replaced by it, the bonus token when all k agree.
+// Grid (request, row, vocabulary chunk); the last CTA of a request merges and decides.
+struct ArgMax {
+  float v;
+  int i;
+};
+static_assert(sizeof(ArgMax) <= sizeof(MS), "argmax partials reuse the (m, s) partial slots");
+__device__ __forceinline__ ArgMax better(ArgMax a, ArgMax b) {
+  return (b.v > a.v || (b.v == a.v && b.i < a.i)) ? b : a;
+}
+__device__ __forceinline__ ArgMax warp_argmax(ArgMax a) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    ArgMax b;
+    b.v = __shfl_xor_sync(kFull, a.v, o);
+    b.i = __shfl_xor_sync(kFull, a.i, o);
+    a = better(a, b);
+  }
+  return a;
+}
+
+__global__ void __launch_bounds__(kSampThreads) argmax_kernel(const SampleParams p, int mode) {
+  __shared__ int s_flag;
+  __shared__ ArgMax s_w[kSampThreads / 32];
+  __shared__ ArgMax s_part[(S3R_MAX_K + 1) * 64];
+  __shared__ ArgMax s_row[S3R_MAX_K + 1];
+  const int bl = blockIdx.x, j = blockIdx.y, c = blockIdx.z;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int r = p.req_ids ? p.req_ids[bl] : bl;
+  const int k = p.k, V = p.vocab;
+  const int nrows = mode == 0 ? 1 : k + 1;
+  const float* row;
+  int i = 0;
+  if (mode == 0) {
+    i = p.draft_step[r];
+    if (i < 0 || i >= k) {
+      if (c == 0 && threadIdx.x == 0) set_error(p.err, S3R_ERR_DEVICE_BOUNDS);
+      return;
+    }
+    row = p.q_logits + ((size_t)r * k + i) * V;
+  } else {
+    row = p.p_logits + ((size_t)r * (k + 1) + j) * V;
+  }
+  const int v0 = c * kVocabChunk, v1 = min(V, (c + 1) * kVocabChunk);
+  ArgMax best{-INFINITY, INT_MAX};
+  bool bad = false;
+#pragma unroll 8
+  for (int q = 0; q < kVocabChunk / kSampThreads; ++q) {
+    const int v = v0 + (int)threadIdx.x + kSampThreads * q;
+    if (v < v1) {
+      float x = __ldg(row + v);
+      if (isnan(x)) {
+        bad = true;
+        x = -INFINITY;
+      }
+      best = better(best, ArgMax{x, v});
+    }
+  }
+  if (bad) set_error(p.err, S3R_ERR_NONFINITE);
+  best = warp_argmax(best);
+  if (lane == 0) s_w[warp] = best;
+  __syncthreads();
+  ArgMax* part = reinterpret_cast<ArgMax*>(p.part) + (size_t)r * nrows * p.nvch;
+  if (threadIdx.x == 0) {
+    ArgMax b = s_w[0];
+    for (int w = 1; w < kSampThreads / 32; ++w) b = better(b, s_w[w]);
+    part[j * p.nvch + c] = b;
+  }
+  if (!last_of(p.tickets + r, nrows * p.nvch, &s_flag)) return;
+
+  // every (row, chunk) partial at once, then one warp per row
+  for (int t = threadIdx.x; t < nrows * p.nvch; t += blockDim.x) {
+    ArgMax a;
+    a.v = __ldcg(&part[t].v);
+    a.i = __ldcg(&part[t].i);
+    s_part[t] = a;
+  }
+  __syncthreads();
+  for (int rr = warp; rr < nrows; rr += kSampThreads / 32) {
+    ArgMax b{-INFINITY, INT_MAX};
+    for (int q = lane; q < p.nvch; q += 32) b = better(b, s_part[rr * p.nvch + q]);
+    b = warp_argmax(b);
+    if (lane == 0) s_row[rr] = b;
+  }
+  __syncthreads();
+  if (threadIdx.x != 0) return;
+  // a row of only -inf has no maximum above -inf: its argmax is token 0 (lowest id)
+  auto tok = [&](int rr) { return s_row[rr].i == INT_MAX ? 0 : s_row[rr].i; };
+  if (mode == 0) {
+    p.draft_out[(size_t)r * k + i] = tok(0);
+    return;
+  }
+  int a = 0;
+  while (a < k) {
+    const int d = p.draft_tokens[(size_t)r * k + a];
+    if (d != tok(a)) break;
+    ++a;
+  }
+  for (int t = 0; t <= a; ++t) p.out_tokens[(size_t)r * (k + 1) + t] = tok(t);
+  p.n_out[r] = a + 1;
+}
+
+int launch_argmax(const SampleParams& p, int batch, int mode, cudaStream_t stream) {
+  dim3 grid(batch, mode == 0 ? 1 : p.k + 1, p.nvch);
+  argmax_kernel<<<grid, kSampThreads, 0, stream>>>(p, mode);
+  return cuda_status(cudaGetLastError(), __func__);
 }
 
 // ------------------------------------------------------------------------- commit ----

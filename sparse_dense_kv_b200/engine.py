@@ -46,10 +46,11 @@ class S3REngine:
     """S3R rounds for a batch of requests over one paged KV cache on one GPU."""
 
     def __init__(self, k_pool, v_pool, page_table, seq_lens, num_q_heads, *, k, budget_bp,
-                 window, vocab, seed, sel_stride=None):
+                 window, vocab, seed, sel_stride=None, greedy=False):
         if not (1 <= k <= L.MAX_K):
             raise ValueError("k must be in 1..8")
         self.k, self.budget_bp, self.window, self.vocab, self.seed = k, budget_bp, window, vocab, seed
+        self.greedy = greedy   # temperature 0: argmax drafts, greedy verification
         self.k_pool, self.v_pool = k_pool, v_pool
         self.page_table = page_table
         self.seq_lens = seq_lens
@@ -68,7 +69,8 @@ class S3REngine:
 
     @property
     def launches_per_round(self) -> int:
-        return 2 + 2 * self.k + 2 + 2 + 1   # select (sigma + select), k x (draft, sample), verify (+merge), spec (2), commit
+        # select (sigma + select), k x (draft, sample), verify (+merge), spec (2 / 1 greedy), commit
+        return 2 + 2 * self.k + 2 + (1 if self.greedy else 2) + 1
 
     def prefill(self, q_x, k_x, v_x):
         """One-row dense pass of each request's pending token at position L (the last step of
@@ -94,6 +96,10 @@ class S3REngine:
                                 self.ws)
 
     def draft_sample(self, i, q_logits):
+        if self.greedy:
+            L.s3r_draft_argmax(self.batch, self.buf.steps[i], self.k, q_logits, self.vocab,
+                               self.buf.draft_tokens, self.ws)
+            return
         L.s3r_draft_sample(self.batch, self.buf.steps[i], self.k, q_logits, self.vocab, self.seed,
                            self.buf.draft_tokens, self.ws)
 
@@ -111,8 +117,12 @@ class S3REngine:
 
     def sample_and_commit(self, p_logits, q_logits):
         b = self.buf
-        L.s3r_spec_sample(self.batch, self.k, p_logits, q_logits, b.draft_tokens, self.vocab,
-                          self.seed, b.out_tokens, b.n_out, self.ws)
+        if self.greedy:
+            L.s3r_greedy_verify(self.batch, self.k, p_logits, b.draft_tokens, self.vocab,
+                                b.out_tokens, b.n_out, self.ws)
+        else:
+            L.s3r_spec_sample(self.batch, self.k, p_logits, q_logits, b.draft_tokens, self.vocab,
+                              self.seed, b.out_tokens, b.n_out, self.ws)
         L.s3r_commit(self.batch, self.k, b.n_out, self.seq_lens, b.stats)
 
     def round(self, q_block, k_block, v_block, p_logits, q_logits, draft_logits_fn=None,

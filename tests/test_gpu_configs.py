@@ -238,3 +238,51 @@ def test_projection_logits_round_matches_oracle():
                 assert O.draft_sample(oq[r, i], u0)[1] < MARGIN, (r, i)
         if not (nout[r] == n and out[r, :n].tolist() == toks.tolist()):
             assert margins.min() < MARGIN, r
+
+
+def test_full_size_mixed_phase_batch_on_sampled_requests():
+    """The high-concurrency workload at full size: 256 requests, contexts log-uniform in
+    [1024, 16384], shuffled pages, mixed round phases; k+1 driver iterations complete one
+    round per request, and the oracle replays four sampled requests."""
+    spec = synth.CONFIGS[3]
+    k = spec.k
+    lens = synth.make_lengths(spec)
+    cache = synth.build_cache(spec, lens, extra_tokens=2 * (k + 1) + 16, device="cuda")
+    NR, Hq, Hkv, d, V = spec.num_requests, spec.num_q_heads, spec.num_kv_heads, spec.head_dim, spec.vocab
+    q = synth.randn_bf16((NR, k + 1, Hq, d), 200, "cuda")
+    kb = synth.randn_bf16((NR, k + 1, Hkv, d), 201, "cuda")
+    vb = synth.randn_bf16((NR, k + 1, Hkv, d), 202, "cuda")
+    pl = synth.randn_f32((NR, k + 1, V), 203, "cuda", scale=spec.logit_std)
+    ql = (pl[:, :k] + synth.randn_f32((NR, k, V), 204, "cuda", scale=spec.draft_noise_std)).contiguous()
+    picks = sorted(np.random.default_rng(3).choice(NR, size=4, replace=False).tolist())
+    pt = cache.page_table.cpu().numpy()
+    host = {}
+    for r in picks:
+        ids = pt[r][pt[r] >= 0]
+        host[r] = (cache.k_pool[ids].float().cpu().numpy(), cache.v_pool[ids].float().cpu().numpy())
+    seq = torch.as_tensor(lens, dtype=torch.int32, device="cuda")
+    eng = s3r.S3REngine(cache.k_pool, cache.v_pool, cache.page_table, seq, Hq, k=k,
+                        budget_bp=spec.budget_bp, window=spec.window, vocab=V, seed=spec.sample_seed)
+    eng.prefill(q[:, :1].contiguous(), kb[:, :1].contiguous(), vb[:, :1].contiguous())
+    drv = s3r.MixedPhaseDriver(eng, synth.initial_phases(spec))
+    drv.start(q, kb, vb, ql)
+    sel = eng.buf.sel_idx.cpu().numpy()
+    cnt = eng.buf.sel_count.cpu().numpy()
+    for _ in range(k + 1):
+        drv.iterate(q, kb, vb, pl, ql)
+    assert eng.check_errors() == 0
+    b = eng.buf
+    for r in picks:
+        kpr, vpr = host[r]
+        local = np.arange(kpr.shape[0], dtype=np.int32)
+        K = np.stack([O.gather_positions(kpr, local, h, np.arange(len(local) * 16)) for h in range(Hkv)])
+        Vv = np.stack([O.gather_positions(vpr, local, h, np.arange(len(local) * 16)) for h in range(Hkv)])
+        L = int(lens[r])
+        st = O.RequestState(K, Vv, L)
+        O.prefill_scores(st, f64(q[r, 0]), f64(kb[r, 0]), f64(vb[r, 0]))
+        sig_prev = st.sigma
+        res = O.run_round(st, r, spec.sample_seed, k, spec.budget_bp, spec.window, f64(q[r]),
+                          f64(kb[r]), f64(vb[r]), ql[r].cpu().numpy(), pl[r].cpu().numpy())
+        _compare_round(spec, r, res, sel[r], cnt[r], sig_prev, L, f64(b.verify_out[r]),
+                       f64(b.lse[r]), b.out_tokens[r].cpu().numpy(), int(b.n_out[r]))
+        assert int(eng.seq_lens[r]) == L + int(b.n_out[r])
