@@ -177,6 +177,63 @@ def selection_margin_cases(sigma: np.ndarray, L: int, budget_bp: int, window: in
 
 
 # ----------------------------------------------------------------------------------------
+# O3p: page-granular selection (the second reading of the selection rule).
+# [Explainer] walkthrough: the draft reads the newest window plus the top-scoring *pages*
+# from the verifier's last attention pass (the Jargon entry says positions). Reading: a
+# page's score is the sum of its positions' scores, added in position order in the dtype of
+# the scores given; the pages holding the W' newest positions are always kept (whole, so up
+# to 15 older positions ride along); the budget is ceil(n / P) pages for the token budget n
+# of budget_count and page size P; the remaining pages are the top-scoring pages wholly
+# before the window, ties to the lower page; the set is every position of the chosen pages
+# below L, ascending. With P = 1 this is select_positions.
+# ----------------------------------------------------------------------------------------
+
+
+def page_scores(sigma: np.ndarray, npages: int, page: int) -> np.ndarray:
+    """Score of pages 0 .. npages-1: sigma[P*q] + sigma[P*q+1] + ... in that order, each add
+    rounded to sigma's dtype (float32 scores give float32 sums)."""
+    s = np.asarray(sigma)
+    if npages == 0:
+        return np.zeros(0, dtype=s.dtype)
+    blocks = s[: npages * page].reshape(npages, page)
+    acc = blocks[:, 0].copy()
+    for t in range(1, page):
+        acc = acc + blocks[:, t]
+    return acc
+
+
+def select_pages(sigma: np.ndarray, L: int, budget_bp: int, window: int, page: int = 16) -> np.ndarray:
+    """Sorted positions of the page-granular sparse set for committed length L."""
+    n, w = budget_count(L, budget_bp, window)
+    first_win = (L - w) // page                  # first page holding a window position
+    win_pages = -(-L // page) - first_win
+    m = max(-(-n // page) - win_pages, 0)        # candidate pages to choose
+    chosen = np.zeros(0, dtype=np.int64)
+    if m > 0:
+        ps = page_scores(sigma, first_win, page)
+        thr = np.sort(ps)[::-1][m - 1]
+        above = np.nonzero(ps > thr)[0]
+        ties = np.nonzero(ps == thr)[0][: m - above.size]
+        chosen = np.sort(np.concatenate([above, ties]))
+    pos = (chosen[:, None] * page + np.arange(page)[None, :]).reshape(-1)
+    return np.concatenate([pos, np.arange(first_win * page, L)]).astype(np.int32)
+
+
+def page_selection_margin_cases(sigma: np.ndarray, L: int, budget_bp: int, window: int,
+                                page: int = 16, rel: float = 1e-5) -> np.ndarray:
+    """Candidate pages whose score lies within rel * threshold of the threshold (their
+    selection may differ between two correct implementations; counted, not compared)."""
+    n, w = budget_count(L, budget_bp, window)
+    first_win = (L - w) // page
+    m = max(-(-n // page) - (-(-L // page) - first_win), 0)
+    if m <= 0:
+        return np.zeros(0, dtype=np.int64)
+    ps = np.asarray(page_scores(sigma, first_win, page), dtype=np.float64)
+    thr = np.sort(ps)[::-1][m - 1]
+    return np.nonzero(np.abs(ps - thr) <= rel * thr)[0]
+
+
+# ----------------------------------------------------------------------------------------
 # O4: sparse self-draft attention.
 # [News] Interpretation and [Explainer] "How is this different": the draft uses the same
 # weights, reading only the selected subset of the KV cache. Draft step i (token at
