@@ -158,9 +158,10 @@ def build_workload(spec, rank, device):
     return lens, cache, seq, inp
 
 
-def algorithmic_bytes(spec, lens):
+def algorithmic_bytes(spec, lens, sel_counts=None):
     """KV bytes per launch: verify reads (L+k+1) positions, draft step i reads n+i+1 positions
-    (+4 B per selected index), 2*d*2 bytes per position and KV head."""
+    (+4 B per selected index), 2*d*2 bytes per position and KV head. sel_counts [NR][Hkv]
+    (the set sizes the select kernel wrote) replaces the token budget n when given."""
     from sparse_dense_kv_b200.engine import budget_count
     Hkv, d, k = spec.num_kv_heads, spec.head_dim, spec.k
     per_pos = 2 * d * 2 * Hkv
@@ -168,9 +169,12 @@ def algorithmic_bytes(spec, lens):
     draft = []
     for i in range(k):
         tot = 0
-        for L in lens:
-            n = budget_count(int(L), spec.budget_bp, spec.window)
-            tot += (n + i + 1) * per_pos + 4 * n * Hkv
+        for r, L in enumerate(lens):
+            if sel_counts is None:
+                ns = [budget_count(int(L), spec.budget_bp, spec.window)] * Hkv
+            else:
+                ns = [int(x) for x in sel_counts[r]]
+            tot += sum((n + i + 1) * 2 * d * 2 + 4 * n for n in ns)
         draft.append(tot)
     G = spec.num_q_heads // Hkv
     scores = int(sum(lens)) * Hkv * G * (k + 1) * 4
@@ -192,7 +196,8 @@ def run_ours(args, spec):
     k = spec.k
     eng = s3r.S3REngine(cache.k_pool, cache.v_pool, cache.page_table, seq, spec.num_q_heads,
                         k=k, budget_bp=spec.budget_bp, window=spec.window, vocab=spec.vocab,
-                        seed=spec.sample_seed + rank)
+                        seed=spec.sample_seed + rank, page_select=args.select == "pages",
+                        greedy=args.greedy)
     seq0 = seq.clone()
     eng.prefill(inp["q"][:, :1].contiguous(), inp["k"][:, :1].contiguous(), inp["v"][:, :1].contiguous())
     stream = torch.cuda.current_stream()
@@ -268,7 +273,7 @@ def run_ours(args, spec):
     ds_ms = [avg(lambda e: e["dm"][i], lambda e: e["d1"][i]) for i in range(k)]
     sel_ms = avg(lambda e: e["s0"], lambda e: e["d0"][0])
     spec_ms = avg(lambda e: e["v1"], lambda e: e["c1"])
-    vb, db, sb = algorithmic_bytes(spec, lens)
+    vb, db, sb = algorithmic_bytes(spec, lens, eng.buf.sel_count.cpu().numpy())
     peak, peak_kind = measured_peaks()
     v_gbs = vb / (v_ms * 1e-3) / 1e9
     d_gbs = sum(db) / (sum(d_ms) * 1e-3) / 1e9
@@ -330,6 +335,8 @@ def run_ours(args, spec):
                                f"d {spec.head_dim}, k {k}, s {spec.budget_bp / 1e4}, window {spec.window}, "
                                f"vocab {spec.vocab}",
                    "requests_per_gpu": spec.num_requests, "parallelism": f"replicas x{world}",
+                   "selection": args.select,
+                   "verification": "greedy" if args.greedy else "speculative sampling",
                    "l2": "inputs larger than L2 (KV 2.1 GB, logits 0.25 GB per round)"},
         "roofline": {"bound": "hbm", "achieved": v_gbs, "peak": peak, "unit": "GB/s",
                      "frac": v_gbs / peak, "traffic": verify_traffic_per_launch(spec.name),
@@ -346,7 +353,8 @@ def run_ours(args, spec):
         "execution": "CUDA graph of one round, replayed per step", "clocks": clocks, "e2e": e2e,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(spec, lens, cache, inp, budget_s=args.cpu_seconds)
+        result["cpu_baseline"] = cpu_baseline(spec, lens, cache, inp, budget_s=args.cpu_seconds,
+                                              mode=oracle_mode(args))
     if rank == 0:
         print(json.dumps(result), flush=True)
     if world > 1:
@@ -445,7 +453,12 @@ def oracle_threads():
         return 1
 
 
-def oracle_round_sample(spec, lens, pools, page_table, inp_host, reqs):
+def oracle_mode(args):
+    """Keyword arguments of the oracle's round for the bench's selection / verification."""
+    return {"page": 16 if args.select == "pages" else 1, "greedy": bool(args.greedy)}
+
+
+def oracle_round_sample(spec, lens, pools, page_table, inp_host, reqs, mode=None):
     """Oracle rounds for the requests `reqs` (dense copies built outside the timing)."""
     from oracle import s3r_oracle as O
     k = spec.k
@@ -465,7 +478,7 @@ def oracle_round_sample(spec, lens, pools, page_table, inp_host, reqs):
     for r, st in prepared:
         res = O.run_round(st, r, spec.sample_seed, k, spec.budget_bp, spec.window,
                           inp_host["q"][r], inp_host["k"][r], inp_host["v"][r],
-                          inp_host["qlog"][r], inp_host["p"][r])
+                          inp_host["qlog"][r], inp_host["p"][r], **(mode or {}))
         tokens += res["n_out"]
     return tokens, time.perf_counter() - t0
 
@@ -474,7 +487,7 @@ def host_inputs(inp, reqs):
     return {n: {r: t[r].float().cpu().numpy() for r in reqs} for n, t in inp.items()}
 
 
-def cpu_baseline(spec, lens, cache, inp, budget_s=15.0):
+def cpu_baseline(spec, lens, cache, inp, budget_s=15.0, mode=None):
     """The oracle on this host's cores on a bounded sample of the same workload."""
     reqs, tokens, secs = [], 0, 0.0
     pools = (cache.k_pool.float().cpu().numpy(), cache.v_pool.float().cpu().numpy())
@@ -482,7 +495,7 @@ def cpu_baseline(spec, lens, cache, inp, budget_s=15.0):
     r = 0
     while secs < budget_s and r < spec.num_requests:
         hi = host_inputs(inp, [r])
-        t, s = oracle_round_sample(spec, lens, pools, pt, hi, [r])
+        t, s = oracle_round_sample(spec, lens, pools, pt, hi, [r], mode)
         tokens, secs = tokens + t, secs + s
         reqs.append(r)
         r += 1
@@ -514,7 +527,7 @@ def run_reference(args, spec):
     for s in range(args.warmup + args.steps):
         r = s % NR
         hi = host_inputs(inp, [r])
-        t, dt = oracle_round_sample(spec, lens, pools, pt, hi, [r])
+        t, dt = oracle_round_sample(spec, lens, pools, pt, hi, [r], oracle_mode(args))
         if s >= args.warmup:
             tok, secs = tok + t, secs + dt
     v = tok / secs
@@ -523,7 +536,8 @@ def run_reference(args, spec):
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
            "data": "synthetic",
            "config": {"workload": f"{spec.name} (config {args.config}), one request-round per step",
-                      "requests_sampled": NR},
+                      "requests_sampled": NR, "selection": args.select,
+                      "verification": "greedy" if args.greedy else "speculative sampling"},
            "cpu_baseline": {"value": v, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
                             "sample": f"{args.steps} request-rounds over {NR} requests of the workload"},
            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -546,6 +560,10 @@ def main(argv=None):
     ap.add_argument("--sweep", action="store_true",
                     help="budget / draft-length sweep (one JSON line per point)")
     ap.add_argument("--sweep-rounds", type=int, default=3)
+    ap.add_argument("--select", choices=["positions", "pages"], default="positions",
+                    help="selection unit: positions, or whole 16-position pages")
+    ap.add_argument("--greedy", action="store_true",
+                    help="temperature 0: argmax drafts and greedy verification")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

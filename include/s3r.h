@@ -13,6 +13,7 @@
  *
  * One round of one request with committed length L and pending token x at position L:
  *   s3r_select_kv          sparse set S (n = ceil(s*L) positions) from the last verify's scores
+ *   s3r_select_kv_pages    the same budget in whole 16-position pages
  *   k x s3r_sparse_draft_attn + s3r_draft_sample     draft tokens d_1..d_k
  *   s3r_verify_attn        dense attention of the k+1 rows at L..L+k, with score capture
  *   s3r_spec_sample        exact speculative sampling -> a accepted drafts + 1 token
@@ -151,6 +152,31 @@ S3R_API int s3r_select_from_scores(const s3r_kv_cache* cache, const s3r_batch* b
                            const float* scores, int32_t score_stride, int32_t budget_bp,
                            int32_t window, int32_t* sel_idx, int32_t sel_stride,
                            int32_t* sel_count, void* ws, size_t ws_bytes, s3r_stream_t stream);
+
+/* Page-granular selection ([Explainer] walkthrough: the newest window plus the top-scoring
+ * pages from the verifier's last attention pass). The units are the 16-position pages
+ * wholly before the window, page q scored by sigma_16q + sigma_16q+1 + ... + sigma_16q+15
+ * added in that order in fp32 (one rounding per add), sigma_j as for s3r_select_kv; the
+ * pages that hold any of the W' newest positions are always kept, whole; the budget is
+ * ceil(n / 16) pages in all (never fewer than the window's), the rest the highest-scored
+ * candidate pages, ties to the lower page. Every position below L of a chosen page is
+ * written, ascending: sel_count = 16 * (chosen candidate pages) + (L - 16 * first window
+ * page) <= n + 15, so sel_stride must hold n + 15 positions (a larger count is a device
+ * bounds error). Arguments, launches, workspace and errors as s3r_select_kv; the set is a
+ * list of positions, so s3r_sparse_draft_attn reads it unchanged (whole pages are 4 KB
+ * contiguous runs at d = 128). Needs (L - W') / 16 <= 49152. */
+S3R_API int s3r_select_kv_pages(const s3r_kv_cache* cache, const s3r_batch* batch,
+                        const float* score_logits, const float* lse, int32_t k_prev,
+                        int32_t budget_bp, int32_t window, int32_t* sel_idx, int32_t sel_stride,
+                        int32_t* sel_count, void* ws, size_t ws_bytes, s3r_stream_t stream);
+
+/* Page-granular selection from caller-given scores (layout as s3r_select_from_scores; a
+ * non-finite score in a page makes that page's score -inf and sets S3R_ERR_NONFINITE). */
+S3R_API int s3r_select_pages_from_scores(const s3r_kv_cache* cache, const s3r_batch* batch,
+                                 const float* scores, int32_t score_stride, int32_t budget_bp,
+                                 int32_t window, int32_t* sel_idx, int32_t sel_stride,
+                                 int32_t* sel_count, void* ws, size_t ws_bytes,
+                                 s3r_stream_t stream);
 
 /* Sparse self-draft attention ([News] Interpretation; [Explainer] "How is this different":
  * the same weights reading a sparse subset of the KV cache). Draft step i = draft_step[r]

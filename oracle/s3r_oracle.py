@@ -447,29 +447,42 @@ def prefill_scores(state: RequestState, q_x, k_x, v_x):
 
 
 def run_round(state: RequestState, request: int, seed: int, k: int, budget_bp: int,
-              window: int, q_rows, k_rows, v_rows, draft_logits, target_logits):
+              window: int, q_rows, k_rows, v_rows, draft_logits, target_logits, page: int = 1,
+              greedy: bool = False):
     """One round for one request.
 
     q_rows [k+1][H_q][d], k_rows/v_rows [k+1][H_kv][d]: projections of the tokens at
     positions L .. L+k (identical in draft and verify). draft_logits [k][V] give q_j,
-    target_logits [k+1][V] give p_j for the token at position L+j+1.
+    target_logits [k+1][V] give p_j for the token at position L+j+1. page > 1 selects whole
+    pages of that size (O3p) instead of positions; greedy drafts and verifies by argmax
+    (temperature 0) and has no sampling margins.
     """
     L = state.L
     Hkv = state.K.shape[0]
     q_rows = np.asarray(q_rows, np.float64)
-    sel = [select_positions(state.sigma[h], L, budget_bp, window) for h in range(Hkv)]
+    if page > 1:
+        sel = [select_pages(state.sigma[h], L, budget_bp, window, page) for h in range(Hkv)]
+    else:
+        sel = [select_positions(state.sigma[h], L, budget_bp, window) for h in range(Hkv)]
     drafts, draft_out, draft_margin = [], [], []
     for i in range(k):
         state.write([L + i], [k_rows[i]], [v_rows[i]])
         o, _ = sparse_draft_attention(q_rows[i], state.K, state.V, sel, L, i)
         draft_out.append(o)
-        u0 = float(uniform(seed, request, L + i + 1, STREAM_DRAFT))
-        tok, mg = draft_sample(draft_logits[i], u0)
+        if greedy:
+            tok, mg = argmax_token(draft_logits[i]), np.inf
+        else:
+            u0 = float(uniform(seed, request, L + i + 1, STREAM_DRAFT))
+            tok, mg = draft_sample(draft_logits[i], u0)
         drafts.append(tok)
         draft_margin.append(mg)
     state.write(list(range(L, L + k + 1)), k_rows, v_rows)
     v_out, lse, sigma, logits = verify_attention(q_rows, state.K, state.V, L)
-    tokens, n_out, margins = spec_sample(target_logits, draft_logits, drafts, seed, request, L)
+    if greedy:
+        tokens, n_out = greedy_verify(target_logits, drafts)
+        margins = np.array([np.inf])
+    else:
+        tokens, n_out, margins = spec_sample(target_logits, draft_logits, drafts, seed, request, L)
     state.sigma = sigma
     state.L = L + n_out
     return dict(sel=sel, drafts=np.asarray(drafts, np.int32), draft_out=np.asarray(draft_out),

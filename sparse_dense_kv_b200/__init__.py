@@ -24,6 +24,8 @@ from ._lib import (  # noqa: F401
     s3r_launch_count,
     s3r_philox,
     s3r_select_from_scores,
+    s3r_select_kv_pages,
+    s3r_select_pages_from_scores,
     s3r_select_kv,
     s3r_set_verify_kernel,
     s3r_sparse_draft_attn,

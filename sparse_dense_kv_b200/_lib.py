@@ -57,6 +57,8 @@ def _load():
         "s3r_verify_attn": (ctypes.c_int, [C, B, I32, P, P, P, P, P, P, P, SZ, P]),
         "s3r_select_kv": (ctypes.c_int, [C, B, P, P, I32, I32, I32, P, I32, P, P, SZ, P]),
         "s3r_select_from_scores": (ctypes.c_int, [C, B, P, I32, I32, I32, P, I32, P, P, SZ, P]),
+        "s3r_select_kv_pages": (ctypes.c_int, [C, B, P, P, I32, I32, I32, P, I32, P, P, SZ, P]),
+        "s3r_select_pages_from_scores": (ctypes.c_int, [C, B, P, I32, I32, I32, P, I32, P, P, SZ, P]),
         "s3r_sparse_draft_attn": (ctypes.c_int, [C, B, P, P, I32, P, P, I32, P, I32, P, P, P, P, SZ, P]),
         "s3r_draft_sample": (ctypes.c_int, [B, P, I32, P, I32, U64, P, P, SZ, P]),
         "s3r_draft_sample_noalloc": (ctypes.c_int, [B, P, I32, P, I32, U64, P, P, P]),
@@ -170,24 +172,48 @@ def s3r_verify_attn(cache, batch, k, q, k_new, v_new, out, lse, score_logits, ws
         ws.numel(), _stream(stream)), "s3r_verify_attn")
 
 
-def s3r_select_kv(cache, batch, score_logits, lse, k_prev, budget_bp, window, sel_idx,
-                  sel_count, ws, stream=None):
+def _select_kv(fn, cache, batch, score_logits, lse, k_prev, budget_bp, window, sel_idx,
+               sel_count, ws, stream):
     f32, i32 = torch.float32, torch.int32
-    _check(_lib.s3r_select_kv(
+    _check(getattr(_lib, fn)(
         ctypes.byref(cache), ctypes.byref(batch), _ptr(score_logits, f32, "score_logits"),
         _ptr(lse, f32, "lse"), k_prev, budget_bp, window, _ptr(sel_idx, i32, "sel_idx"),
         sel_idx.shape[-1], _ptr(sel_count, i32, "sel_count"), _ptr(ws, torch.uint8, "ws"),
-        ws.numel(), _stream(stream)), "s3r_select_kv")
+        ws.numel(), _stream(stream)), fn)
+
+
+def _select_from_scores(fn, cache, batch, scores, budget_bp, window, sel_idx, sel_count, ws,
+                        stream):
+    f32, i32 = torch.float32, torch.int32
+    _check(getattr(_lib, fn)(
+        ctypes.byref(cache), ctypes.byref(batch), _ptr(scores, f32, "scores"), scores.shape[-1],
+        budget_bp, window, _ptr(sel_idx, i32, "sel_idx"), sel_idx.shape[-1],
+        _ptr(sel_count, i32, "sel_count"), _ptr(ws, torch.uint8, "ws"), ws.numel(),
+        _stream(stream)), fn)
+
+
+def s3r_select_kv(cache, batch, score_logits, lse, k_prev, budget_bp, window, sel_idx,
+                  sel_count, ws, stream=None):
+    _select_kv("s3r_select_kv", cache, batch, score_logits, lse, k_prev, budget_bp, window,
+               sel_idx, sel_count, ws, stream)
+
+
+def s3r_select_kv_pages(cache, batch, score_logits, lse, k_prev, budget_bp, window, sel_idx,
+                        sel_count, ws, stream=None):
+    _select_kv("s3r_select_kv_pages", cache, batch, score_logits, lse, k_prev, budget_bp,
+               window, sel_idx, sel_count, ws, stream)
 
 
 def s3r_select_from_scores(cache, batch, scores, budget_bp, window, sel_idx, sel_count, ws,
                            stream=None):
-    f32, i32 = torch.float32, torch.int32
-    _check(_lib.s3r_select_from_scores(
-        ctypes.byref(cache), ctypes.byref(batch), _ptr(scores, f32, "scores"), scores.shape[-1],
-        budget_bp, window, _ptr(sel_idx, i32, "sel_idx"), sel_idx.shape[-1],
-        _ptr(sel_count, i32, "sel_count"), _ptr(ws, torch.uint8, "ws"), ws.numel(),
-        _stream(stream)), "s3r_select_from_scores")
+    _select_from_scores("s3r_select_from_scores", cache, batch, scores, budget_bp, window,
+                        sel_idx, sel_count, ws, stream)
+
+
+def s3r_select_pages_from_scores(cache, batch, scores, budget_bp, window, sel_idx, sel_count,
+                                 ws, stream=None):
+    _select_from_scores("s3r_select_pages_from_scores", cache, batch, scores, budget_bp,
+                        window, sel_idx, sel_count, ws, stream)
 
 
 def _rows(t, inner, what):

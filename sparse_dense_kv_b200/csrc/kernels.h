@@ -81,6 +81,7 @@ struct SelectParams {
   int32_t* sel_count;
   int* err;
   float* sigma_buf;        // workspace: sigma [NR][Hkv][cap] of the logits path
+  int page;                // selection unit: 1 (positions) or S3R_PAGE_SIZE (pages)
 };
 
 struct SampleParams {

@@ -363,7 +363,8 @@ int s3r_verify_attn(const s3r_kv_cache* cache, const s3r_batch* batch, int32_t k
 
 static int select_common(const s3r_kv_cache* cache, const s3r_batch* batch, SelectParams& p,
                          int32_t budget_bp, int32_t window, int32_t* sel_idx, int32_t sel_stride,
-                         int32_t* sel_count, void* ws, size_t ws_bytes, s3r_stream_t stream) {
+                         int32_t* sel_count, void* ws, size_t ws_bytes, s3r_stream_t stream,
+                         int page = 1) {
   if (budget_bp < 1 || budget_bp > 10000 || window < 1) return S3R_ERR_INVALID_ARG;
   if (!sel_idx || !sel_count || sel_stride < 1 || !aligned4(sel_idx) || !aligned4(sel_count))
     return S3R_ERR_INVALID_ARG;
@@ -385,16 +386,18 @@ static int select_common(const s3r_kv_cache* cache, const s3r_batch* batch, Sele
   p.sel_stride = sel_stride;
   p.sel_count = sel_count;
   p.err = w.err;
+  p.page = page;
   int nl = 0;
   const int st = launch_select(p, batch->batch, (cudaStream_t)stream, &nl);
   g_launches.fetch_add((uint64_t)nl, std::memory_order_relaxed);
   return st;
 }
 
-int s3r_select_kv(const s3r_kv_cache* cache, const s3r_batch* batch, const float* score_logits,
-                  const float* lse, int32_t k_prev, int32_t budget_bp, int32_t window,
-                  int32_t* sel_idx, int32_t sel_stride, int32_t* sel_count, void* ws,
-                  size_t ws_bytes, s3r_stream_t stream) {
+static int select_kv_impl(const s3r_kv_cache* cache, const s3r_batch* batch,
+                          const float* score_logits, const float* lse, int32_t k_prev,
+                          int32_t budget_bp, int32_t window, int32_t* sel_idx, int32_t sel_stride,
+                          int32_t* sel_count, void* ws, size_t ws_bytes, s3r_stream_t stream,
+                          int page) {
   S3R_TRY(check_cache(cache));
   S3R_TRY(check_batch(batch, true));
   if (k_prev < 0 || k_prev > S3R_MAX_K) return S3R_ERR_UNSUPPORTED;
@@ -411,13 +414,14 @@ int s3r_select_kv(const s3r_kv_cache* cache, const s3r_batch* batch, const float
   p.T = k_prev + 1;
   p.R = G * (k_prev + 1);
   return select_common(cache, batch, p, budget_bp, window, sel_idx, sel_stride, sel_count, ws,
-                       ws_bytes, stream);
+                       ws_bytes, stream, page);
 }
 
-int s3r_select_from_scores(const s3r_kv_cache* cache, const s3r_batch* batch,
-                           const float* scores, int32_t score_stride, int32_t budget_bp,
-                           int32_t window, int32_t* sel_idx, int32_t sel_stride,
-                           int32_t* sel_count, void* ws, size_t ws_bytes, s3r_stream_t stream) {
+static int select_from_scores_impl(const s3r_kv_cache* cache, const s3r_batch* batch,
+                                   const float* scores, int32_t score_stride, int32_t budget_bp,
+                                   int32_t window, int32_t* sel_idx, int32_t sel_stride,
+                                   int32_t* sel_count, void* ws, size_t ws_bytes,
+                                   s3r_stream_t stream, int page) {
   S3R_TRY(check_cache(cache));
   S3R_TRY(check_batch(batch, false));
   if (!scores || !aligned4(scores) || score_stride < 1) return S3R_ERR_INVALID_ARG;
@@ -426,7 +430,40 @@ int s3r_select_from_scores(const s3r_kv_cache* cache, const s3r_batch* batch,
   p.scores = scores;
   p.score_stride = score_stride;
   return select_common(cache, batch, p, budget_bp, window, sel_idx, sel_stride, sel_count, ws,
-                       ws_bytes, stream);
+                       ws_bytes, stream, page);
+}
+
+int s3r_select_kv(const s3r_kv_cache* cache, const s3r_batch* batch, const float* score_logits,
+                  const float* lse, int32_t k_prev, int32_t budget_bp, int32_t window,
+                  int32_t* sel_idx, int32_t sel_stride, int32_t* sel_count, void* ws,
+                  size_t ws_bytes, s3r_stream_t stream) {
+  return select_kv_impl(cache, batch, score_logits, lse, k_prev, budget_bp, window, sel_idx,
+                        sel_stride, sel_count, ws, ws_bytes, stream, 1);
+}
+
+int s3r_select_kv_pages(const s3r_kv_cache* cache, const s3r_batch* batch,
+                        const float* score_logits, const float* lse, int32_t k_prev,
+                        int32_t budget_bp, int32_t window, int32_t* sel_idx, int32_t sel_stride,
+                        int32_t* sel_count, void* ws, size_t ws_bytes, s3r_stream_t stream) {
+  return select_kv_impl(cache, batch, score_logits, lse, k_prev, budget_bp, window, sel_idx,
+                        sel_stride, sel_count, ws, ws_bytes, stream, S3R_PAGE_SIZE);
+}
+
+int s3r_select_from_scores(const s3r_kv_cache* cache, const s3r_batch* batch,
+                           const float* scores, int32_t score_stride, int32_t budget_bp,
+                           int32_t window, int32_t* sel_idx, int32_t sel_stride,
+                           int32_t* sel_count, void* ws, size_t ws_bytes, s3r_stream_t stream) {
+  return select_from_scores_impl(cache, batch, scores, score_stride, budget_bp, window, sel_idx,
+                                 sel_stride, sel_count, ws, ws_bytes, stream, 1);
+}
+
+int s3r_select_pages_from_scores(const s3r_kv_cache* cache, const s3r_batch* batch,
+                                 const float* scores, int32_t score_stride, int32_t budget_bp,
+                                 int32_t window, int32_t* sel_idx, int32_t sel_stride,
+                                 int32_t* sel_count, void* ws, size_t ws_bytes,
+                                 s3r_stream_t stream) {
+  return select_from_scores_impl(cache, batch, scores, score_stride, budget_bp, window, sel_idx,
+                                 sel_stride, sel_count, ws, ws_bytes, stream, S3R_PAGE_SIZE);
 }
 
 int s3r_sparse_draft_attn(const s3r_kv_cache* cache, const s3r_batch* batch,

@@ -6,6 +6,12 @@
 // positions, W' = min(W, L): the W' newest plus the n - W' highest-scored positions
 // j < L - W', ties to the lower j, ascending.
 //
+// Page-granular variant ([Explainer] walkthrough: "top-scoring pages"): the units are the
+// 16-position pages wholly before the window, each scored by the fp32 sum of its positions'
+// scores added in position order; the pages holding the W' newest positions are kept whole;
+// ceil(n / 16) pages in all (at least the window's); every position of a chosen page below L
+// is emitted, ascending, so the count is at most n + 15.
+//
 // One CTA of 1024 threads per (KV head, request). Scores sigma_j = sum over the G*(k+1)
 // verify rows of exp(logit - lse) are computed once into shared memory as order-preserving
 // uint32 keys; MSB-first histogram passes of up to 11 bits over the bits in which the keys
@@ -55,6 +61,7 @@ __device__ __forceinline__ int block_excl_scan(int v, int* wsum) {
   return r;
 }
 
+template <int P>
 __global__ void __launch_bounds__(kSelectThreads, 2) select_kernel(const SelectParams p) {
   extern __shared__ uint32_t keys[];
   __shared__ uint32_t hist[kSelectBins];
@@ -73,27 +80,57 @@ __global__ void __launch_bounds__(kSelectThreads, 2) select_kernel(const SelectP
   int n = (int)(((int64_t)L * p.budget_bp + 9999) / 10000);
   const int w = min(p.window, L);
   n = min(max(n, w), L);
-  if (n > p.sel_stride) {
+  // units: positions (P = 1) or pages (P = 16); M of the N candidate units are chosen, the
+  // window's units start at position wstart, cnt positions are emitted
+  int M, N, wstart;
+  if constexpr (P == 1) {
+    M = n - w;
+    N = L - w;
+    wstart = N;
+  } else {
+    N = (L - w) / P;
+    const int win_pages = (L + P - 1) / P - N;
+    M = max((n + P - 1) / P - win_pages, 0);
+    wstart = N * P;
+  }
+  const int cnt = M * P + (L - wstart);
+  if (cnt > p.sel_stride) {
     if (tid == 0) set_error(p.err, S3R_ERR_DEVICE_BOUNDS);
     return;
   }
-  const int M = n - w, N = L - w;
   if (M > 0 && N > kSelectMaxN) {
     if (tid == 0) set_error(p.err, S3R_ERR_DEVICE_BOUNDS);
     return;
   }
   int32_t* out = p.sel_idx + ((size_t)r * p.Hkv + kvh) * p.sel_stride;
-  for (int j = tid; j < w; j += blockDim.x) out[M + j] = N + j;
-  if (tid == 0) p.sel_count[(size_t)r * p.Hkv + kvh] = n;
+  for (int j = tid; j < L - wstart; j += blockDim.x) out[M * P + j] = wstart + j;
+  if (tid == 0) p.sel_count[(size_t)r * p.Hkv + kvh] = cnt;
   if (M == 0) return;
 
   // ---- scores -> order-preserving keys in shared memory
   bool bad = false;
+  const float* srow = p.scores + ((size_t)r * p.Hkv + kvh) * p.score_stride;
   for (int j = tid; j < N; j += blockDim.x) {
-    float sigma = p.scores[((size_t)r * p.Hkv + kvh) * p.score_stride + j];
-    if (!isfinite(sigma)) {
-      bad = true;
-      sigma = -INFINITY;
+    float sigma;
+    if constexpr (P == 1) {
+      sigma = srow[j];
+      if (!isfinite(sigma)) {
+        bad = true;
+        sigma = -INFINITY;
+      }
+    } else {
+      const float* sp = srow + (size_t)j * P;
+      sigma = sp[0];
+      bool fin = isfinite(sigma);
+      for (int t = 1; t < P; ++t) {
+        const float x = sp[t];
+        fin = fin && isfinite(x);
+        sigma = __fadd_rn(sigma, x);   // position order, one rounding per add
+      }
+      if (!fin) {
+        bad = true;
+        sigma = -INFINITY;
+      }
     }
     keys[j] = order_key(sigma);
   }
@@ -217,7 +254,10 @@ __global__ void __launch_bounds__(kSelectThreads, 2) select_kernel(const SelectP
     const unsigned em = __ballot_sync(kFull, eq);
     const bool take = gt || (eq && eqb + __popc(em & lt) < need_eq);
     const unsigned tm = __ballot_sync(kFull, take);
-    if (take) out[base + __popc(tm & lt)] = j;
+    if (take) {
+      int32_t* o = out + (size_t)(base + __popc(tm & lt)) * P;
+      for (int t = 0; t < P; ++t) o[t] = j * P + t;
+    }
     base += __popc(tm);
     eqb += __popc(em);
   }
@@ -294,14 +334,19 @@ int launch_select(const SelectParams& p, int batch, cudaStream_t stream, int* la
   const size_t smem = (size_t)(nmax > 0 ? nmax : 1) * 4;
   static bool attr_done = false;
   if (!attr_done) {
-    if (cuda_status(cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kSelectMaxN * 4), "cudaFuncSetAttribute") != S3R_OK)
-
+    if (cuda_status(cudaFuncSetAttribute(select_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kSelectMaxN * 4), "cudaFuncSetAttribute") != S3R_OK ||
+        cuda_status(cudaFuncSetAttribute(select_kernel<S3R_PAGE_SIZE>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSelectMaxN * 4),
+                    "cudaFuncSetAttribute") != S3R_OK)
       return S3R_ERR_CUDA;
     attr_done = true;
   }
   dim3 grid(q.Hkv, batch);
-  select_kernel<<<grid, kSelectThreads, smem, stream>>>(q);
+  if (p.page == S3R_PAGE_SIZE)
+    select_kernel<S3R_PAGE_SIZE><<<grid, kSelectThreads, smem, stream>>>(q);
+  else
+    select_kernel<1><<<grid, kSelectThreads, smem, stream>>>(q);
   const int st = cuda_status(cudaGetLastError(), __func__);
   if (st == S3R_OK) ++*launches;
   return st;

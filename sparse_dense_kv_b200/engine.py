@@ -46,18 +46,21 @@ class S3REngine:
     """S3R rounds for a batch of requests over one paged KV cache on one GPU."""
 
     def __init__(self, k_pool, v_pool, page_table, seq_lens, num_q_heads, *, k, budget_bp,
-                 window, vocab, seed, sel_stride=None, greedy=False):
+                 window, vocab, seed, sel_stride=None, greedy=False, page_select=False):
         if not (1 <= k <= L.MAX_K):
             raise ValueError("k must be in 1..8")
         self.k, self.budget_bp, self.window, self.vocab, self.seed = k, budget_bp, window, vocab, seed
         self.greedy = greedy   # temperature 0: argmax drafts, greedy verification
+        self.page_select = page_select   # whole 16-position pages instead of positions
         self.k_pool, self.v_pool = k_pool, v_pool
         self.page_table = page_table
         self.seq_lens = seq_lens
         self.cache = L.make_cache(k_pool, v_pool, num_q_heads)
         self.num_requests, self.max_pages = page_table.shape
         self.cap = self.max_pages * L.PAGE_SIZE
-        self.sel_stride = sel_stride or budget_count(self.cap, budget_bp, window)
+        # a page-granular set holds up to 15 positions more than the token budget
+        self.sel_stride = sel_stride or (budget_count(self.cap, budget_bp, window)
+                                         + (L.PAGE_SIZE - 1 if page_select else 0))
         self.buf = RoundBuffers(self.num_requests, num_q_heads, self.cache.num_kv_heads,
                                 self.cache.head_dim, self.cap, k, vocab, self.sel_stride,
                                 k_pool.device)
@@ -86,8 +89,9 @@ class S3REngine:
     def select(self):
         b = self.buf
         lse = b.prefill_lse if self.k_prev == 0 else b.lse
-        L.s3r_select_kv(self.cache, self.batch, b.scores, lse, self.k_prev, self.budget_bp,
-                        self.window, b.sel_idx, b.sel_count, self.ws)
+        fn = L.s3r_select_kv_pages if self.page_select else L.s3r_select_kv
+        fn(self.cache, self.batch, b.scores, lse, self.k_prev, self.budget_bp, self.window,
+           b.sel_idx, b.sel_count, self.ws)
 
     def draft_attn(self, i, q_block, k_block, v_block):
         b = self.buf
@@ -217,7 +221,11 @@ class MixedPhaseDriver:
         batch = self._batch(ids)
         L.s3r_sparse_draft_attn(e.cache, batch, self.step, qc, kc, vc, b.sel_idx, b.sel_count,
                                 b.draft_out, b.draft_lse, e.ws)
-        L.s3r_draft_sample(batch, self.step, e.k, q_logits, e.vocab, e.seed, b.draft_tokens, e.ws)
+        if e.greedy:
+            L.s3r_draft_argmax(batch, self.step, e.k, q_logits, e.vocab, b.draft_tokens, e.ws)
+        else:
+            L.s3r_draft_sample(batch, self.step, e.k, q_logits, e.vocab, e.seed, b.draft_tokens,
+                               e.ws)
 
     def iterate(self, q_block, k_block, v_block, p_logits, q_logits):
         """Advance every request by one phase; returns the ids that completed a round."""
@@ -231,10 +239,15 @@ class MixedPhaseDriver:
             batch = self._batch(v_ids)
             L.s3r_verify_attn(e.cache, batch, e.k, q_block, k_block, v_block, b.verify_out, b.lse,
                               b.scores, e.ws)
-            L.s3r_spec_sample(batch, e.k, p_logits, q_logits, b.draft_tokens, e.vocab, e.seed,
-                              b.out_tokens, b.n_out, e.ws)
+            if e.greedy:
+                L.s3r_greedy_verify(batch, e.k, p_logits, b.draft_tokens, e.vocab, b.out_tokens,
+                                    b.n_out, e.ws)
+            else:
+                L.s3r_spec_sample(batch, e.k, p_logits, q_logits, b.draft_tokens, e.vocab,
+                                  e.seed, b.out_tokens, b.n_out, e.ws)
             L.s3r_commit(batch, e.k, b.n_out, e.seq_lens, b.stats)
-            L.s3r_select_kv(e.cache, batch, b.scores, b.lse, e.k, e.budget_bp, e.window,
-                            b.sel_idx, b.sel_count, e.ws)
+            sel = L.s3r_select_kv_pages if e.page_select else L.s3r_select_kv
+            sel(e.cache, batch, b.scores, b.lse, e.k, e.budget_bp, e.window, b.sel_idx,
+                b.sel_count, e.ws)
         self.phases = (self.phases + 1) % (e.k + 1)
         return v_ids

@@ -13,13 +13,14 @@ from tests.test_oracle_round import make_states
 pytestmark = pytest.mark.gpu
 
 
-def gpu_engine(spec, rounds):
+def gpu_engine(spec, rounds, page_select=False, greedy=False):
     lens = synth.make_lengths(spec)
     cache = synth.build_cache(spec, lens, extra_tokens=800)
     seq = torch.as_tensor(lens, dtype=torch.int32).cuda()
     eng = s3r.S3REngine(cache.k_pool.cuda(), cache.v_pool.cuda(), cache.page_table.cuda(), seq,
                         spec.num_q_heads, k=spec.k, budget_bp=spec.budget_bp, window=spec.window,
-                        vocab=spec.vocab, seed=spec.sample_seed)
+                        vocab=spec.vocab, seed=spec.sample_seed, page_select=page_select,
+                        greedy=greedy)
     qs, ks, vs = zip(*[synth.token_qkv(spec, r, [int(lens[r])]) for r in range(spec.num_requests)])
     eng.prefill(torch.stack(qs).cuda(), torch.stack(ks).cuda(), torch.stack(vs).cuda())
     return eng
@@ -35,13 +36,23 @@ def round_inputs(spec, lengths):
     return cu(q), cu(k), cu(v), torch.as_tensor(np.stack(pl)).cuda(), torch.as_tensor(np.stack(ql)).cuda()
 
 
-def test_rounds_match_oracle_tiny():
+def near_threshold(sigma, L, spec, page):
+    """Positions whose selection may go either way (oracle margin below 1e-5)."""
+    if page == 1:
+        return set(O.selection_margin_cases(sigma, L, spec.budget_bp, spec.window, MARGIN).tolist())
+    pages = O.page_selection_margin_cases(sigma, L, spec.budget_bp, spec.window, page, MARGIN)
+    return {int(q) * page + t for q in pages for t in range(page)}
+
+
+@pytest.mark.parametrize("page,greedy", [(1, False), (16, False), (1, True), (16, True)])
+def test_rounds_match_oracle_tiny(page, greedy):
     """Rounds are compared request by request. A decision whose oracle margin is below 1e-5
     may go either way; if the GPU then differs, that request's later rounds are no longer
-    comparable and it leaves the comparison (counted)."""
+    comparable and it leaves the comparison (counted). page 16: page-granular selection;
+    greedy: argmax drafts and greedy verification (no sampling margins: tokens must match)."""
     spec = synth.CONFIGS[0]
     n_rounds = 40
-    eng = gpu_engine(spec, n_rounds)
+    eng = gpu_engine(spec, n_rounds, page_select=page > 1, greedy=greedy)
     states = make_states(spec)
     alive = [True] * spec.num_requests
     compared = diverged = boundary = 0
@@ -61,9 +72,10 @@ def test_rounds_match_oracle_tiny():
                 continue
             sig_prev, L = st.sigma, st.L
             res = O.run_round(st, r, spec.sample_seed, spec.k, spec.budget_bp, spec.window,
-                              f64(q[r]), f64(k[r]), f64(v[r]), ql[r].cpu().numpy(), pl[r].cpu().numpy())
+                              f64(q[r]), f64(k[r]), f64(v[r]), ql[r].cpu().numpy(), pl[r].cpu().numpy(),
+                              page=page, greedy=greedy)
             for h in range(spec.num_kv_heads):
-                near = set(O.selection_margin_cases(sig_prev[h], L, spec.budget_bp, spec.window, MARGIN).tolist())
+                near = near_threshold(sig_prev[h], L, spec, page)
                 diff = set(sel[r, h, : cnt[r, h]].tolist()) ^ set(res["sel"][h].tolist())
                 assert diff <= near
             assert_attention_close(f64(b.verify_out[r]), res["verify_out"], f"verify r={r}")

@@ -33,3 +33,22 @@ def test_greedy_verify_round():
     # with identical draft and target rows, greedy drafting is always fully accepted
     drafts = [O.argmax_token(p[j]) for j in range(k)]
     assert O.greedy_verify(p, drafts)[1] == k + 1
+
+
+def test_greedy_round_with_equal_logits_accepts_every_draft():
+    """A whole greedy oracle round: identical draft and target logits emit k + 1 tokens,
+    the argmax of each target row."""
+    rng = np.random.default_rng(5)
+    k, L, Hkv, G, d, V = 4, 40, 1, 2, 8, 32
+    K = rng.normal(size=(Hkv, L + k + 1, d))
+    Vv = rng.normal(size=(Hkv, L + k + 1, d))
+    st = O.RequestState(K.copy(), Vv.copy(), L)
+    O.prefill_scores(st, rng.normal(size=(Hkv * G, d)), K[:, L], Vv[:, L])
+    p = rng.normal(size=(k + 1, V))
+    res = O.run_round(st, 0, 1, k, 2500, 8, rng.normal(size=(k + 1, Hkv * G, d)),
+                      K[:, L:L + k + 1].transpose(1, 0, 2), Vv[:, L:L + k + 1].transpose(1, 0, 2),
+                      p[:k], p, greedy=True)
+    assert res["n_out"] == k + 1
+    assert res["tokens"].tolist() == [int(np.argmax(p[j])) for j in range(k + 1)]
+    assert res["drafts"].tolist() == [int(np.argmax(p[j])) for j in range(k)]
+    assert st.L == L + k + 1
