@@ -20,11 +20,13 @@ constexpr unsigned kFull = 0xffffffffu;
 constexpr int kWaitLimit = 1 << 24;       // bounded spin on an mbarrier phase
 
 // ---------------------------------------------------------------- workspace layout ----
-// [0, 256)      error word (int32 bitmask of 1 << s3r_status) + reserved
+// [0, 256)      error word (int32 bitmask of 1 << s3r_status) at 0; at 64 the dense verify's
+//               work counter and exit counter (zero between calls); the rest reserved
 // [256, T)      tickets: int32 [num_requests][kMaxKvHeads] (zero between calls); the same
 //               region for every call, whatever its head count
 // [T, ...)      per-call partials, overwritten by each call
 constexpr size_t kWsHeader = 256;
+constexpr size_t kWsSchedOff = 64;
 constexpr int kMaxKvHeads = 64;
 __host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 __host__ __device__ inline size_t ws_tickets_bytes(int num_requests) {

@@ -35,6 +35,7 @@ struct VerifyParams {
   int* tickets;
   float* part;
   int req_off;             // launch covers requests req_ids[req_off + b] (or req_off + b)
+  int* sched;              // [2] work counter, exited CTAs (zero between launches)
 };
 
 struct DraftParams {

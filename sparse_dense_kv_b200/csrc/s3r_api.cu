@@ -80,6 +80,7 @@ int check_ws(void* ws, size_t ws_bytes, size_t need) {
 
 struct Carve {
   int* err;
+  int* sched;
   int* tickets;
   uint8_t* part;
 };
@@ -88,6 +89,7 @@ Carve carve(void* ws, int num_requests) {
   uint8_t* b = static_cast<uint8_t*>(ws);
   Carve c;
   c.err = reinterpret_cast<int*>(b);
+  c.sched = reinterpret_cast<int*>(b + kWsSchedOff);
   c.tickets = reinterpret_cast<int*>(b + kWsHeader);
   c.part = b + kWsHeader + ws_tickets_bytes(num_requests);
   return c;
@@ -333,6 +335,7 @@ int s3r_verify_attn(const s3r_kv_cache* cache, const s3r_batch* batch, int32_t k
   p.nchunk_max = (cap + kVerifyChunk - 1) / kVerifyChunk;
   p.err = w.err;
   p.tickets = w.tickets;
+  p.sched = w.sched;
   p.part = reinterpret_cast<float*>(w.part);
   int st;
   const bool tc = g_verify_kernel.load() == 0 && verify_tc_supported(cache->head_dim, R, batch->batch);

@@ -214,118 +214,120 @@ __global__ void __launch_bounds__(MAXT) verify_kernel(const __grid_constant__ CU
 
 }
 
-// Merge the chunk records of every (request, KV head) of a verify launch into out / lse:
-// one CTA per (KV head, request), weights from all chunk maxima / sums, then 16-byte loads
-// of the chunk outputs with several independent accumulators per thread.
+// Merge the chunk records of every (request, KV head) of a verify launch into out / lse.
+// Grid (group of kCombRows rows, KV head, request), so a launch has a few CTAs per SM and
+// every merge runs at once: the group's chunk maxima / sums are loaded in one round, the
+// weights of each row are formed in shared memory, then every thread accumulates two
+// 16-byte output slices over the chunks in chunk order with 8 chunks' loads in flight.
+constexpr int kCombRows = 8;
+constexpr int kCombThreads = 128;
+constexpr int kCombBatch = 8;   // chunks whose loads are issued together
+
 template <int D>
-__global__ void __launch_bounds__(256) verify_combine_kernel(const VerifyParams p) {
-  extern __shared__ float cw[];   // [nchunk_max][R] m, then l, then weights
-  const int kvh = blockIdx.x, bl = blockIdx.y;
+__global__ void __launch_bounds__(kCombThreads) verify_combine_kernel(const VerifyParams p) {
+  extern __shared__ float cw[];   // m, l, weights: [nch][kCombRows] each
+  const int j0 = blockIdx.x * kCombRows, kvh = blockIdx.y, bl = blockIdx.z;
   const int r = p.req_ids ? p.req_ids[bl] : bl;
   const int L = p.seq_lens[r];
   const int T = p.T, G = p.G, R = p.R, Rp = p.Rp, Lc = L + T;
-  if (L < 0 || Lc > p.cap) return;   // reported by the attention kernel
+  if (L < 0 || Lc > p.cap || j0 >= R) return;   // bad lengths are reported by the attention kernel
+  const int nr = min(kCombRows, R - j0);
   const int nch = (Lc + p.chunk - 1) / p.chunk;
   const size_t rec_floats = (size_t)Rp * (D + 2);
   const float* recs = p.part + ((size_t)r * p.Hkv + kvh) * p.nchunk_max * rec_floats;
   float* mm = cw;
-  float* ll = cw + (size_t)nch * R;
-  float* ww = ll + (size_t)nch * R;
-  float* Ms = ww + (size_t)nch * R;
-  for (int i = threadIdx.x; i < nch * R; i += blockDim.x) {
-    const int c = i / R, row = i - c * R;
-    mm[i] = __ldcg(recs + c * rec_floats + row);
-    ll[i] = __ldcg(recs + c * rec_floats + Rp + row);
+  float* ll = cw + (size_t)nch * kCombRows;
+  float* ww = ll + (size_t)nch * kCombRows;
+  for (int i = threadIdx.x; i < nch * nr; i += blockDim.x) {
+    const int c = i / nr, j = i - c * nr;
+    mm[c * kCombRows + j] = __ldcg(recs + c * rec_floats + j0 + j);
+    ll[c * kCombRows + j] = __ldcg(recs + c * rec_floats + Rp + j0 + j);
   }
   __syncthreads();
-  for (int row = threadIdx.x; row < R; row += blockDim.x) {
+  if (threadIdx.x < nr) {
+    const int j = threadIdx.x, row = j0 + j;
     float M = -INFINITY;
-    for (int c = 0; c < nch; ++c) M = fmaxf(M, mm[c * R + row]);
+    for (int c = 0; c < nch; ++c) M = fmaxf(M, mm[c * kCombRows + j]);
     float lsum = 0.f;
     for (int c = 0; c < nch; ++c) {
-      const float mc = mm[c * R + row];
-      lsum += (mc == -INFINITY) ? 0.f : exp2f(mc - M) * ll[c * R + row];
+      const float mc = mm[c * kCombRows + j];
+      lsum += (mc == -INFINITY) ? 0.f : exp2f(mc - M) * ll[c * kCombRows + j];
     }
     const float inv = 1.f / lsum;
     for (int c = 0; c < nch; ++c) {
-      const float mc = mm[c * R + row];
-      ww[c * R + row] = (mc == -INFINITY) ? 0.f : exp2f(mc - M) * inv;
+      const float mc = mm[c * kCombRows + j];
+      ww[c * kCombRows + j] = (mc == -INFINITY) ? 0.f : exp2f(mc - M) * inv;
     }
     const int t = row / G, g = row - t * G;
     p.lse[((size_t)r * T + t) * p.Hq + kvh * G + g] = (M + log2f(lsum)) * kLn2;
-    Ms[row] = M;
   }
   __syncthreads();
-  constexpr int kV = 4;   // (row, 4 d) items per thread per pass
-  const int nvec = R * (D / 4);
-  for (int v0 = threadIdx.x; v0 < nvec; v0 += kV * blockDim.x) {
-    float4 acc[kV];
-    int rows[kV];
+  constexpr int kQ = D / 4;       // float4 slices per row
+  const int nvec = nr * kQ;
+  for (int v0 = threadIdx.x; v0 < nvec; v0 += 2 * blockDim.x) {
+    const int v1 = v0 + blockDim.x;
+    const bool has1 = v1 < nvec;
+    const int ja = v0 / kQ, jb = has1 ? v1 / kQ : ja;
+    const float4* pa = reinterpret_cast<const float4*>(recs + 2 * Rp + (size_t)j0 * D) + v0;
+    const float4* pb = reinterpret_cast<const float4*>(recs + 2 * Rp + (size_t)j0 * D) + (has1 ? v1 : v0);
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+    for (int c0 = 0; c0 < nch; c0 += kCombBatch) {
+      const int nb = min(kCombBatch, nch - c0);
+      float4 xa[kCombBatch], xb[kCombBatch];
 #pragma unroll
-    for (int s = 0; s < kV; ++s) {
-      acc[s] = make_float4(0.f, 0.f, 0.f, 0.f);
-      const int v = v0 + s * blockDim.x;
-      rows[s] = v < nvec ? v / (D / 4) : 0;
-    }
-    for (int c = 0; c < nch; ++c) {
-      const float* oc = recs + c * rec_floats + 2 * Rp;
+      for (int u = 0; u < kCombBatch; ++u) {
+        if (u < nb) {
+          const size_t off = (size_t)(c0 + u) * rec_floats / 4;
+          xa[u] = __ldcg(pa + off);
+          xb[u] = __ldcg(pb + off);
+        }
+      }
 #pragma unroll
-      for (int s = 0; s < kV; ++s) {
-        const int v = v0 + s * blockDim.x;
-        if (v < nvec) {
-          const float w = ww[c * R + rows[s]];
-          const float4 x = __ldcg(reinterpret_cast<const float4*>(oc) + v);
-          acc[s].x += w * x.x;
-          acc[s].y += w * x.y;
-          acc[s].z += w * x.z;
-          acc[s].w += w * x.w;
+      for (int u = 0; u < kCombBatch; ++u) {
+        if (u < nb) {
+          const float wa = ww[(c0 + u) * kCombRows + ja], wb = ww[(c0 + u) * kCombRows + jb];
+          a.x += wa * xa[u].x;
+          a.y += wa * xa[u].y;
+          a.z += wa * xa[u].z;
+          a.w += wa * xa[u].w;
+          b.x += wb * xb[u].x;
+          b.y += wb * xb[u].y;
+          b.z += wb * xb[u].z;
+          b.w += wb * xb[u].w;
         }
       }
     }
-#pragma unroll
-    for (int s = 0; s < kV; ++s) {
-      const int v = v0 + s * blockDim.x;
-      if (v >= nvec) continue;
-      const int row = rows[s], d4 = v - row * (D / 4);
+    auto store = [&](int v, int j, const float4& acc) {
+      const int row = j0 + j, d4 = v - j * kQ;
       const int t = row / G, g = row - t * G;
       __nv_bfloat162* o = reinterpret_cast<__nv_bfloat162*>(
           p.out + (((size_t)r * T + t) * p.Hq + kvh * G + g) * D + d4 * 4);
-      o[0] = __floats2bfloat162_rn(acc[s].x, acc[s].y);
-      o[1] = __floats2bfloat162_rn(acc[s].z, acc[s].w);
-    }
+      o[0] = __floats2bfloat162_rn(acc.x, acc.y);
+      o[1] = __floats2bfloat162_rn(acc.z, acc.w);
+    };
+    store(v0, ja, a);
+    if (has1) store(v1, jb, b);
   }
-  (void)Ms;
 }
 
-bool verify_combine_fits(int nchunk_max, int R) {
-  return ((size_t)3 * nchunk_max * R + R) * 4 <= 200 * 1024;
+bool verify_combine_fits(int nchunk_max, int /*R*/) {
+  return (size_t)3 * nchunk_max * kCombRows * 4 <= 200 * 1024;
 }
 
 int launch_verify_combine(const VerifyParams& p, int D, int batch, cudaStream_t stream) {
-  const size_t smem = ((size_t)3 * p.nchunk_max * p.R + p.R) * 4;
+  const size_t smem = (size_t)3 * p.nchunk_max * kCombRows * 4;
   if (!verify_combine_fits(p.nchunk_max, p.R)) return S3R_ERR_UNSUPPORTED;
-  dim3 grid(p.Hkv, batch);
-  if (D == 128) {
-    static size_t attr = 0;
-    if (smem > 48 * 1024 && smem > attr) {
-      if (cuda_status(cudaFuncSetAttribute(verify_combine_kernel<128>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem),
-                      "cudaFuncSetAttribute") != S3R_OK)
-        return S3R_ERR_CUDA;
-      attr = smem;
-    }
-    verify_combine_kernel<128><<<grid, 256, smem, stream>>>(p);
-  } else {
-    static size_t attr = 0;
-    if (smem > 48 * 1024 && smem > attr) {
-      if (cuda_status(cudaFuncSetAttribute(verify_combine_kernel<64>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem),
-                      "cudaFuncSetAttribute") != S3R_OK)
-        return S3R_ERR_CUDA;
-      attr = smem;
-    }
-    verify_combine_kernel<64><<<grid, 256, smem, stream>>>(p);
+  dim3 grid((p.R + kCombRows - 1) / kCombRows, p.Hkv, batch);
+  auto kern = D == 128 ? verify_combine_kernel<128> : verify_combine_kernel<64>;
+  static size_t attr[2] = {0, 0};
+  size_t& a = attr[D == 128 ? 0 : 1];
+  if (smem > 48 * 1024 && smem > a) {
+    if (cuda_status(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem),
+                    "cudaFuncSetAttribute") != S3R_OK)
+      return S3R_ERR_CUDA;
+    a = smem;
   }
+  kern<<<grid, kCombThreads, smem, stream>>>(p);
   return cuda_status(cudaGetLastError(), __func__);
 }
 

@@ -7,7 +7,9 @@
 // positions 0..L+t; out, lse and every committed logit are written.
 //
 // Organisation (one persistent CTA per SM, 11 warps). A work item is (request, KV head,
-// chunk of up to 7 or 8 tiles of 128 positions).
+// chunk of up to 7 or 8 tiles of 128 positions). Items are claimed from a counter in the
+// workspace as CTAs progress (the K producer claims, a ring in shared memory tells the
+// other roles), so faster SMs take more of them.
 //   warp 0     K producer: per item it loads the item's Q rows into one of two Q buffers
 //              (3-D TMA box, rows t*G+g), then streams the chunk's K tiles through a
 //              2-stage ring with 4-D TMA over (d, slot, head, page): a tile of 8
@@ -29,8 +31,7 @@
 //              rewritten for item n+1 once the PV of item n has read it (a barrier per
 //              tile), so that PV and pass 2 of item n+1 overlap; the PV of an item starts
 //              once its whole P^T is written. Then the chunk record (max, sum, O) goes to the
-//              workspace, and a small second kernel merges the chunks of every (request, KV
-//              head).
+//              workspace, and a second kernel merges the chunks of every (request, KV head).
 // Every wait is bounded (an expired wait sets S3R_ERR_TIMEOUT and the CTA winds down).
 // The softmax is exact per chunk (two passes over logits resident in tensor memory), so no
 // running rescale exists; chunks merge by their (max, sum) as in the CUDA-core kernel.
@@ -45,7 +46,8 @@ constexpr int kD = 128;                     // head_dim of this path
 constexpr int kMaxStages = 4;               // ring barriers per stream
 constexpr int kThreads = 352;               // K producer, V producer, MMA, 8 softmax warps
 constexpr int kSoftWarp0 = 3;
-constexpr int kBarBytes = 512;              // mbarriers and flags
+constexpr int kBarBytes = 768;              // mbarriers and flags
+constexpr int kRing = 16;                   // item ids published by the K producer
 constexpr int kTileBytes = kPos * kD * 2;   // 32 KB: [2 halves][128 rows][128 B]
 constexpr int kMaxBatch = 256;              // requests per launch (larger batches: several launches)
 
@@ -190,6 +192,8 @@ struct Bars {
   uint64_t s_full[2], s_empty[2], o_full[2], o_empty[2];
   uint64_t p_free[8];   // P^T tile t has been read by the PV of the previous chunk
   uint64_t wg[2];       // barrier of each softmax warpgroup (4 warps)
+  uint64_t item_bar[kRing];   // item id of the CTA's m-th item published in item_id[m % kRing]
+  int item_id[kRing];
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -316,6 +320,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(smem_u32(&B->p_full), 8);
     for (int t = 0; t < 8; ++t) mbar_init(smem_u32(&B->p_free[t]), 1);
+    for (int i = 0; i < kRing; ++i) mbar_init(smem_u32(&B->item_bar[i]), 1);
     mbar_init(smem_u32(&B->wg[0]), 4);
     mbar_init(smem_u32(&B->wg[1]), 4);
     mbar_init(smem_u32(&B->fin), 1);
@@ -332,7 +337,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = B->tmem_base;
   const int nitems = pref[batch];
-  const int my_items = nitems > (int)blockIdx.x ? (nitems - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  // Work is claimed, not dealt: a CTA's first item is blockIdx.x, every later one comes from
+  // the launch's counter (item gridDim.x + counter), claimed by the K producer one item
+  // ahead of its own progress and published in the ring (item id nitems: no more work), so
+  // CTAs on faster SMs take more chunks and all finish within about one chunk of each other.
+  auto ring_id = [&](int m) -> int {   // warp-uniform; -1 if the wait gave up
+    const int slot = m & (kRing - 1);
+    if (!wait_bar(smem_u32(&B->item_bar[slot]), (uint32_t)(m / kRing) & 1u, abort_flag, p.err)) return -1;
+    return *reinterpret_cast<volatile int*>(&B->item_id[slot]);
+  };
   const uint32_t qbuf = sbase + C::kQOff, pbuf = sbase + C::kPOff;
 
   if (warp <= 1) {
@@ -442,17 +455,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       a = lane < npg && (pg0 + lane) * kPage < x.L ? ptab[pg0 + lane] : -1;
       b = lane + 32 < npg && (pg0 + lane + 32) * kPage < x.L ? ptab[pg0 + lane + 32] : -1;
     };
+    // id of the CTA's m-th item: the K producer claims and publishes it, the V producer
+    // reads it from the ring
+    auto item_id = [&](int m) -> int {
+      if (is_v) return ring_id(m);
+      int id = (int)blockIdx.x;
+      if (m > 0) {
+        int v = 0;
+        if (lane == 0) v = atomicAdd(p.sched, 1);
+        id = __shfl_sync(kFull, v, 0) + (int)gridDim.x;
+      }
+      id = min(id, nitems);
+      if (lane == 0) {
+        B->item_id[m & (kRing - 1)] = id;
+        mbar_arrive(smem_u32(&B->item_bar[m & (kRing - 1)]));   // release: the id is visible
+      }
+      __syncwarp();
+      return id;
+    };
     int next_a = -1, next_b = -1;
-    for (int m = 0; m < my_items && !stop && !aborted(abort_flag); ++m) {
-      const Item x = make_item<NP>(blockIdx.x + m * gridDim.x, pref, lens_s, rid_s, batch, p);
+    int cur = item_id(0);
+    for (int m = 0; cur >= 0 && cur < nitems && !stop && !aborted(abort_flag); ++m) {
+      const int nxt = item_id(m + 1);
+      if (nxt < 0) break;
+      const Item x = make_item<NP>(cur, pref, lens_s, rid_s, batch, p);
+      cur = nxt;
       int a = next_a, b = next_b;
       if (m == 0) fetch_ids(x, a, b);
       __syncwarp();   // every lane is done with the previous item's ids
       ids_own[lane] = a;
       ids_own[lane + 32] = b;
-      if (m + 1 < my_items)
-        fetch_ids(make_item<NP>(blockIdx.x + (m + 1) * gridDim.x, pref, lens_s, rid_s, batch, p),
-                  next_a, next_b);
+      if (nxt < nitems) fetch_ids(make_item<NP>(nxt, pref, lens_s, rid_s, batch, p), next_a, next_b);
       __syncwarp();
       if (!is_v) {
         // Q rows -> Q buffer m&1 by TMA (K-major, 128-byte swizzle) once QK(m-2) has read it
@@ -497,16 +530,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       return __shfl_sync(kFull, r ? 1 : 0, 0) != 0;
     };
     int mk = 0, tk = 0, gk = 0, nv = 0, tv = 0, gv = 0;
+    int kend = -1;           // number of items, once the ring has said "no more"
+    bool kknown = false;     // xk holds item mk
+    int xv_of = -1;          // xv holds item xv_of
     bool kgo = false, vgo = false, ok = true;
     Item xk{}, xv{};
-    if (my_items > 0) {
-      xk = make_item<NP>(blockIdx.x, pref, lens_s, rid_s, batch, p);
-      xv = xk;
-    }
     uint32_t idle = 0;
-    while (ok && (mk < my_items || nv < my_items)) {
+    while (ok && (kend < 0 || nv < kend)) {
       bool did = false;
-      if (mk < my_items) {
+      if (kend < 0 && !kknown) {
+        const int slot = mk & (kRing - 1);
+        if (ready(&B->item_bar[slot], (uint32_t)(mk / kRing) & 1u)) {
+          // lane 0 made the acquiring test: it reads the id and hands it to the warp
+          int id = lane == 0 ? *reinterpret_cast<volatile int*>(&B->item_id[slot]) : 0;
+          id = __shfl_sync(kFull, id, 0);
+          if (id >= nitems) {
+            kend = mk;
+          } else {
+            xk = make_item<NP>(id, pref, lens_s, rid_s, batch, p);
+            kknown = true;
+          }
+          did = true;
+        }
+      }
+      if (kknown) {
         if (!kgo) {
           kgo = ready(&B->q_full[mk & 1], (mk >> 1) & 1) &&
                 (mk < 2 || ready(&B->s_empty[mk & 1], ((mk - 2) >> 1) & 1));
@@ -541,12 +588,18 @@ __global__ void __launch_bounds__(kThreads, 1)
               ++mk;
               tk = 0;
               kgo = false;
-              if (mk < my_items) xk = make_item<NP>(blockIdx.x + mk * gridDim.x, pref, lens_s, rid_s, batch, p);
+              kknown = false;
             }
           }
         }
       }
       if (nv < mk) {
+        if (xv_of != nv) {   // item nv's id was read from the ring when its QK started
+          int id = lane == 0 ? *reinterpret_cast<volatile int*>(&B->item_id[nv & (kRing - 1)]) : 0;
+          id = __shfl_sync(kFull, id, 0);
+          xv = make_item<NP>(id, pref, lens_s, rid_s, batch, p);
+          xv_of = nv;
+        }
         if (!vgo) {
           vgo = ready(&B->p_full, nv & 1) &&
                 (nv < 2 || ready(&B->o_empty[nv & 1], ((nv - 2) >> 1) & 1));
@@ -583,7 +636,6 @@ __global__ void __launch_bounds__(kThreads, 1)
               ++nv;
               tv = 0;
               vgo = false;
-              if (nv < my_items) xv = make_item<NP>(blockIdx.x + nv * gridDim.x, pref, lens_s, rid_s, batch, p);
             }
           }
         }
@@ -634,8 +686,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // record of chunk m (this warpgroup's rows): O^T buffer m&1 -> workspace, with the rows'
     // max / sum from cm / cl
-    auto epilogue = [&](int m) -> bool {
-      const Item x = make_item<NP>(blockIdx.x + m * gridDim.x, pref, lens_s, rid_s, batch, p);
+    auto epilogue = [&](int m, const Item& x) -> bool {
       if (!wait_bar(smem_u32(&B->o_full[m & 1]), (m >> 1) & 1, abort_flag, p.err)) return false;
       tc_fence_after();
       const size_t rec_floats = (size_t)p.Rp * (kD + 2);
@@ -656,8 +707,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
 
     bool ok = true;
-    for (int n = 0; n < my_items && !aborted(abort_flag); ++n) {
-      const Item x = make_item<NP>(blockIdx.x + n * gridDim.x, pref, lens_s, rid_s, batch, p);
+    int n = 0;
+    Item xprev{};
+    for (; !aborted(abort_flag); ++n) {
+      const int id = ring_id(n);
+      if (id < 0) {
+        ok = false;
+        break;
+      }
+      if (id >= nitems) break;
+      const Item x = make_item<NP>(id, pref, lens_s, rid_s, batch, p);
       const int L = x.L, start = x.start, end = x.end;
       float* scores = p.scores ? p.scores + ((size_t)x.r * Hkv + x.kvh) * (size_t)R * p.cap : nullptr;
       if (!wait_bar(smem_u32(&B->s_full[n & 1]), (n >> 1) & 1, abort_flag, p.err)) {
@@ -784,7 +843,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // the previous chunk's output leaves tensor memory (its PV has finished by now or
       // soon: this pass already waited for each of its tiles)
-      if (n > 0 && !epilogue(n - 1)) {
+      if (n > 0 && !epilogue(n - 1, xprev)) {
         ok = false;
         break;
       }
@@ -806,9 +865,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         cl[(n & 1) * NP + c0 + gt] = l;
       }
       // (cl / redL reuse is ordered by the barriers of the next chunk)
+      xprev = x;
     }
-    if (ok && my_items > 0 && !aborted(abort_flag)) {
-      if (wg_sync()) epilogue(my_items - 1);   // cl of the last chunk complete
+    if (ok && n > 0 && !aborted(abort_flag)) {
+      if (wg_sync()) epilogue(n - 1, xprev);   // cl of the last chunk complete
     }
   }
 
@@ -817,6 +877,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 2) {
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
+  }
+  // the last CTA out returns the counters to zero for the next launch
+  if (tid == 0) __threadfence();   // this CTA's claims are performed before its exit count
+  if (tid == 0 && atomicAdd(p.sched + 1, 1) == (int)gridDim.x - 1) {
+    p.sched[0] = 0;
+    p.sched[1] = 0;
   }
 }
 

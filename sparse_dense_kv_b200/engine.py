@@ -69,11 +69,13 @@ class S3REngine:
         self.ws = L.new_workspace(nbytes, k_pool.device)
         self.batch = L.make_batch(seq_lens, page_table)
         self.k_prev = None
+        self._verify_launches = 2
 
     @property
     def launches_per_round(self) -> int:
-        # select (sigma + select), k x (draft, sample), verify (+merge), spec (2 / 1 greedy), commit
-        return 2 + 2 * self.k + 2 + (1 if self.greedy else 2) + 1
+        # select (sigma + select), k x (draft, sample), verify (attention launches + the chunk
+        # merge, as counted at the last verify), spec (2 / 1 greedy), commit
+        return 2 + 2 * self.k + self._verify_launches + (1 if self.greedy else 2) + 1
 
     def prefill(self, q_x, k_x, v_x):
         """One-row dense pass of each request's pending token at position L (the last step of
@@ -115,8 +117,10 @@ class S3REngine:
 
     def verify(self, q_block, k_block, v_block):
         b = self.buf
+        before = L.s3r_launch_count()
         L.s3r_verify_attn(self.cache, self.batch, self.k, q_block, k_block, v_block, b.verify_out,
                           b.lse, b.scores, self.ws)
+        self._verify_launches = L.s3r_launch_count() - before
         self.k_prev = self.k
 
     def sample_and_commit(self, p_logits, q_logits):
