@@ -273,28 +273,89 @@ __device__ int draw_token(int V, int nvch, const double* csum, double target, W 
 }
 
 // ------------------------------------------------------------------ draft sampling ----
+// Draft sampling: a CTA takes kDsSpan logits of one request's draft row (two vocabulary
+// chunks), staged in shared memory by one bulk copy (so no registers are held by loads in
+// flight and a launch over 32 requests x 151,936 logits is one wave), and writes the two
+// chunks' (max, sum) partials; the last CTA of the request merges them and draws.
+constexpr int kDsPer = 2;
+constexpr int kDsSpan = kDsPer * kVocabChunk;
+
+// (max, sum) of this thread's entries t + 256 q of a staged chunk of n <= kVocabChunk, all
+// 32 read from shared memory at once (no load latency per entry).
+__device__ __forceinline__ void smem_ms(const float* xs, int n, float& m, float& s, bool& bad) {
+  static_assert(kVocabChunk == 32 * kSampThreads, "32 entries per thread");
+  float x[32];
+#pragma unroll
+  for (int q = 0; q < 32; ++q) {
+    const int j = (int)threadIdx.x + kSampThreads * q;
+    float v = j < n ? xs[j] : -INFINITY;
+    if (isnan(v) || v == INFINITY) {
+      bad = true;
+      v = -INFINITY;
+    }
+    x[q] = v;
+  }
+  m = -INFINITY;
+#pragma unroll
+  for (int q = 0; q < 32; ++q) m = fmaxf(m, x[q]);
+  s = 0.f;
+  if (m != -INFINITY) {
+    const float mb = m * kLog2e;
+#pragma unroll
+    for (int q = 0; q < 32; ++q) s += ex2(fmaf(x[q], kLog2e, -mb));
+  }
+}
+
 __global__ void __launch_bounds__(kSampThreads) draft_sample_kernel(const SampleParams p) {
+  extern __shared__ float4 xs4[];   // [kDsSpan] logits of this CTA's span
+  float* xs = reinterpret_cast<float*>(xs4);
+  __shared__ __align__(8) uint64_t bar;
   __shared__ int s_flag;
   __shared__ double csum[64];
   __shared__ float s_M;
-  const int c = blockIdx.y, bl = blockIdx.x;
+  const int cb = blockIdx.y, bl = blockIdx.x;
   const int r = p.req_ids ? p.req_ids[bl] : bl;
   const int i = p.draft_step[r];
   const int V = p.vocab;
   if (i < 0 || i >= p.k) {
-    if (c == 0 && threadIdx.x == 0) set_error(p.err, S3R_ERR_DEVICE_BOUNDS);
+    if (cb == 0 && threadIdx.x == 0) set_error(p.err, S3R_ERR_DEVICE_BOUNDS);
     return;
   }
   const float* row = p.q_logits + ((size_t)r * p.k + i) * V;
   MS* part = reinterpret_cast<MS*>(p.part) + (size_t)r * p.nvch;
+  const int v0 = cb * kDsSpan, n = min(V - v0, kDsSpan);
 
-  float m, s;
+  // stage the span: one bulk copy when it is 16-byte aligned and sized, else plain loads
+  const bool bulk = ((reinterpret_cast<uintptr_t>(row + v0) & 15u) == 0) && ((n & 3) == 0);
+  if (bulk) {
+    if (threadIdx.x == 0) {
+      mbar_init(smem_u32(&bar), 1);
+      fence_mbar_init();
+    }
+    __syncthreads();   // the barrier is initialised before the copy and before anyone polls it
+    if (threadIdx.x == 0) {
+      mbar_arrive_expect_tx(smem_u32(&bar), (uint32_t)n * 4u);
+      bulk_load(smem_u32(xs), row + v0, (uint32_t)n * 4u, smem_u32(&bar));
+    }
+    if (!mbar_wait(smem_u32(&bar), 0) && threadIdx.x == 0) set_error(p.err, S3R_ERR_TIMEOUT);
+  } else {
+    for (int j = threadIdx.x; j < n; j += kSampThreads) xs[j] = __ldg(row + v0 + j);
+    __syncthreads();
+  }
+
   bool bad = false;
-  thread_ms(row, c * kVocabChunk, min(V, (c + 1) * kVocabChunk), m, s, bad);
+#pragma unroll
+  for (int h = 0; h < kDsPer; ++h) {
+    const int c = cb * kDsPer + h;
+    if (c >= p.nvch) break;
+    float m, s;
+    smem_ms(xs + h * kVocabChunk, min(n - h * kVocabChunk, kVocabChunk), m, s, bad);
+    const MS tot = block_ms(m, s);
+    if (threadIdx.x == 0) part[c] = tot;
+    __syncthreads();   // block_ms's scratch is reused by the next chunk
+  }
   if (bad) set_error(p.err, S3R_ERR_NONFINITE);
-  const MS tot = block_ms(m, s);
-  if (threadIdx.x == 0) part[c] = tot;
-  if (!last_of(p.tickets + r, p.nvch, &s_flag)) return;
+  if (!last_of(p.tickets + r, (int)gridDim.y, &s_flag)) return;
 
   if (threadIdx.x < 32) {
     const float M = merge_partials_warp(part, p.nvch, csum);
@@ -307,10 +368,52 @@ __global__ void __launch_bounds__(kSampThreads) draft_sample_kernel(const Sample
   const int L = p.seq_lens[r];
   const double u = philox_u(p.seed, (uint32_t)(L + i + 1), (uint32_t)r, 0u);
   const float Mb = M * kLog2e;
-  const int tok = draw_token(V, p.nvch, csum, u * Z, [&](int v) -> float {
-    const float x = row[v];
-    return (isnan(x) || x == INFINITY) ? 0.f : ex2(fmaf(x, kLog2e, -Mb));
-  });
+  const double target = u * Z;
+  // the chunk holding the target (thread 0 over the chunk sums), then that chunk staged in
+  // shared memory, so that the search reads its 8192 logits at shared-memory latency
+  __shared__ int s_c;
+  __shared__ double s_base;
+  if (threadIdx.x == 0) {
+    double cum = 0.0;
+    int c = p.nvch;
+    for (int q = 0; q < p.nvch; ++q) {
+      if (target < cum + csum[q]) {
+        c = q;
+        break;
+      }
+      cum += csum[q];
+    }
+    s_c = c;
+    s_base = cum;
+  }
+  __syncthreads();
+  double base = s_base;
+  uint32_t phase = bulk ? 1u : 0u;   // phase 0 of the barrier was the span's copy
+  int tok = -1;
+  for (int c = s_c; c < p.nvch && tok < 0; ++c) {
+    const int c0 = c * kVocabChunk, cn = min(V - c0, kVocabChunk);
+    __syncthreads();   // every thread is done with the shared buffer
+    if (bulk && (cn & 3) == 0) {   // the barrier is set up and its phase 0 is done
+      if (threadIdx.x == 0) {
+        mbar_arrive_expect_tx(smem_u32(&bar), (uint32_t)cn * 4u);
+        bulk_load(smem_u32(xs), row + c0, (uint32_t)cn * 4u, smem_u32(&bar));
+      }
+      if (!mbar_wait(smem_u32(&bar), phase & 1u) && threadIdx.x == 0) set_error(p.err, S3R_ERR_TIMEOUT);
+      ++phase;
+    } else {
+      for (int j = threadIdx.x; j < cn; j += kSampThreads) xs[j] = __ldg(row + c0 + j);
+      __syncthreads();
+    }
+    tok = chunk_search(c0, c0 + cn, target, base, [&](int v) -> float {
+      const float x = xs[v - c0];
+      return (isnan(x) || x == INFINITY) ? 0.f : ex2(fmaf(x, kLog2e, -Mb));
+    });
+  }
+  if (tok < 0)   // rounding past the last chunk: the last token of nonzero probability
+    tok = last_nonzero(V, [&](int v) -> float {
+      const float x = row[v];
+      return (isnan(x) || x == INFINITY) ? 0.f : ex2(fmaf(x, kLog2e, -Mb));
+    });
   if (threadIdx.x == 0) p.draft_out[(size_t)r * p.k + i] = tok;
 }
 
@@ -630,8 +733,16 @@ __global__ void philox_kernel(uint64_t seed, int stream_id, const int32_t* reque
 
 // ------------------------------------------------------------------------ launchers ----
 int launch_draft_sample(const SampleParams& p, int batch, cudaStream_t stream) {
-  dim3 grid(batch, p.nvch);
-  draft_sample_kernel<<<grid, kSampThreads, 0, stream>>>(p);
+  constexpr int smem = kDsSpan * 4;
+  static bool attr_done = false;
+  if (!attr_done) {
+    if (cuda_status(cudaFuncSetAttribute(draft_sample_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         smem), "cudaFuncSetAttribute") != S3R_OK)
+      return S3R_ERR_CUDA;
+    attr_done = true;
+  }
+  dim3 grid(batch, (p.vocab + kDsSpan - 1) / kDsSpan);
+  draft_sample_kernel<<<grid, kSampThreads, smem, stream>>>(p);
   return cuda_status(cudaGetLastError(), __func__);
 }
 
