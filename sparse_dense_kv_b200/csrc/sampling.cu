@@ -244,8 +244,13 @@ __device__ int last_nonzero(int V, W weight) {
 }
 
 // Draw with target u * Z over weights whose chunk sums are csum[0..nvch).
-template <class W>
-__device__ int draw_token(int V, int nvch, const double* csum, double target, W weight) {
+// Inverse-CDF draw of target = u * Z from the chunk sums csum: thread 0 finds the chunk,
+// stage(c0, n) brings that chunk's inputs into shared memory (ending with a barrier), and
+// the search reads them there through sweight(v, c0); if rounding carries the target past
+// the last chunk, the last token of nonzero weight (gweight reads global memory) is taken.
+template <class Stage, class SW, class GW>
+__device__ int draw_staged(int V, int nvch, const double* csum, double target, Stage stage,
+                           SW sweight, GW gweight) {
   __shared__ int s_c;
   __shared__ double s_base;
   if (threadIdx.x == 0) {
@@ -262,14 +267,15 @@ __device__ int draw_token(int V, int nvch, const double* csum, double target, W 
     s_base = cum;
   }
   __syncthreads();
-  int c = s_c;
   double base = s_base;
-  __syncthreads();
-  for (; c < nvch; ++c) {
-    const int tok = chunk_search(c * kVocabChunk, min(V, (c + 1) * kVocabChunk), target, base, weight);
-    if (tok >= 0) return tok;
+  int tok = -1;
+  for (int c = s_c; c < nvch && tok < 0; ++c) {
+    const int c0 = c * kVocabChunk, cn = min(V - c0, kVocabChunk);
+    __syncthreads();   // every thread is done with the shared buffers
+    stage(c0, cn);
+    tok = chunk_search(c0, c0 + cn, target, base, [&](int v) -> float { return sweight(v, c0); });
   }
-  return last_nonzero(V, weight);
+  return tok >= 0 ? tok : last_nonzero(V, gweight);
 }
 
 // ------------------------------------------------------------------ draft sampling ----
@@ -368,32 +374,11 @@ __global__ void __launch_bounds__(kSampThreads) draft_sample_kernel(const Sample
   const int L = p.seq_lens[r];
   const double u = philox_u(p.seed, (uint32_t)(L + i + 1), (uint32_t)r, 0u);
   const float Mb = M * kLog2e;
-  const double target = u * Z;
-  // the chunk holding the target (thread 0 over the chunk sums), then that chunk staged in
-  // shared memory, so that the search reads its 8192 logits at shared-memory latency
-  __shared__ int s_c;
-  __shared__ double s_base;
-  if (threadIdx.x == 0) {
-    double cum = 0.0;
-    int c = p.nvch;
-    for (int q = 0; q < p.nvch; ++q) {
-      if (target < cum + csum[q]) {
-        c = q;
-        break;
-      }
-      cum += csum[q];
-    }
-    s_c = c;
-    s_base = cum;
-  }
-  __syncthreads();
-  double base = s_base;
-  uint32_t phase = bulk ? 1u : 0u;   // phase 0 of the barrier was the span's copy
-  int tok = -1;
-  for (int c = s_c; c < p.nvch && tok < 0; ++c) {
-    const int c0 = c * kVocabChunk, cn = min(V - c0, kVocabChunk);
-    __syncthreads();   // every thread is done with the shared buffer
-    if (bulk && (cn & 3) == 0) {   // the barrier is set up and its phase 0 is done
+  // the chunk holding u * Z is staged in shared memory (the span's buffer, by a bulk copy
+  // on the same barrier, whose phase 0 was the span's copy), then searched there
+  uint32_t phase = 1;
+  auto stage = [&](int c0, int cn) {
+    if (bulk && (cn & 3) == 0) {
       if (threadIdx.x == 0) {
         mbar_arrive_expect_tx(smem_u32(&bar), (uint32_t)cn * 4u);
         bulk_load(smem_u32(xs), row + c0, (uint32_t)cn * 4u, smem_u32(&bar));
@@ -404,16 +389,11 @@ __global__ void __launch_bounds__(kSampThreads) draft_sample_kernel(const Sample
       for (int j = threadIdx.x; j < cn; j += kSampThreads) xs[j] = __ldg(row + c0 + j);
       __syncthreads();
     }
-    tok = chunk_search(c0, c0 + cn, target, base, [&](int v) -> float {
-      const float x = xs[v - c0];
-      return (isnan(x) || x == INFINITY) ? 0.f : ex2(fmaf(x, kLog2e, -Mb));
-    });
-  }
-  if (tok < 0)   // rounding past the last chunk: the last token of nonzero probability
-    tok = last_nonzero(V, [&](int v) -> float {
-      const float x = row[v];
-      return (isnan(x) || x == INFINITY) ? 0.f : ex2(fmaf(x, kLog2e, -Mb));
-    });
+  };
+  auto wq = [&](float x) -> float { return (isnan(x) || x == INFINITY) ? 0.f : ex2(fmaf(x, kLog2e, -Mb)); };
+  const int tok = draw_staged(
+      V, p.nvch, csum, u * Z, stage, [&](int v, int c0) { return wq(xs[v - c0]); },
+      [&](int v) { return wq(row[v]); });
   if (threadIdx.x == 0) p.draft_out[(size_t)r * p.k + i] = tok;
 }
 
@@ -494,6 +474,9 @@ __global__ void __launch_bounds__(kSampThreads) spec_norm_kernel(const SamplePar
 
 // ------------------------------------------------------- speculative sampling: pass 2 --
 __global__ void __launch_bounds__(kSampThreads) spec_draw_kernel(const SampleParams p) {
+  extern __shared__ float4 xs4[];   // the drawn chunk: p logits, then q logits
+  float* xps = reinterpret_cast<float*>(xs4);
+  float* xqs = xps + kVocabChunk;
   __shared__ int s_flag;
   __shared__ double csum[64];
   __shared__ int s_use_res;
@@ -580,9 +563,44 @@ __global__ void __launch_bounds__(kSampThreads) spec_draw_kernel(const SamplePar
   double Z = 0.0;
   for (int q = 0; q < p.nvch; ++q) Z += csum[q];
   const double target = pl.u * Z;
+  const bool use_res = s_use_res != 0;
+  // the drawn chunk of the p row (and the q row for a residual) staged in shared memory by
+  // bulk copies (or plain loads when unaligned), then searched there
+  __shared__ __align__(8) uint64_t bar;
+  uint32_t phase = 0;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  auto stage = [&](int c0, int cn) {
+    const bool v4 = ((reinterpret_cast<uintptr_t>(prow + c0) & 15u) == 0) &&
+                    ((reinterpret_cast<uintptr_t>(qrow + c0) & 15u) == 0) && ((cn & 3) == 0);
+    if (v4) {
+      if (threadIdx.x == 0) {
+        const uint32_t bytes = (uint32_t)cn * 4u;
+        mbar_arrive_expect_tx(smem_u32(&bar), use_res ? 2u * bytes : bytes);
+        bulk_load(smem_u32(xps), prow + c0, bytes, smem_u32(&bar));
+        if (use_res) bulk_load(smem_u32(xqs), qrow + c0, bytes, smem_u32(&bar));
+      }
+      if (!mbar_wait(smem_u32(&bar), phase & 1u) && threadIdx.x == 0) set_error(p.err, S3R_ERR_TIMEOUT);
+      ++phase;
+      return;
+    } else {
+      for (int j = threadIdx.x; j < cn; j += kSampThreads) {
+        xps[j] = __ldg(prow + c0 + j);
+        if (use_res) xqs[j] = __ldg(qrow + c0 + j);
+      }
+    }
+    __syncthreads();
+  };
   int tok;
-  if (s_use_res) tok = draw_token(V, p.nvch, csum, target, w_res);
-  else tok = draw_token(V, p.nvch, csum, target, w_p);
+  if (use_res)
+    tok = draw_staged(V, p.nvch, csum, target, stage,
+                      [&](int v, int c0) { return wres_xy(xps[v - c0], xqs[v - c0]); }, w_res);
+  else
+    tok = draw_staged(V, p.nvch, csum, target, stage,
+                      [&](int v, int c0) { return wp_x(xps[v - c0]); }, w_p);
   if (threadIdx.x == 0) p.out_tokens[(size_t)r * (k + 1) + pl.a] = tok;
 }
 
@@ -750,8 +768,16 @@ int launch_spec_sample(const SampleParams& p, int batch, cudaStream_t stream, in
   dim3 g1(batch, 2 * p.k + 1, p.nvch);
   spec_norm_kernel<<<g1, kSampThreads, 0, stream>>>(p);
   if (cuda_status(cudaGetLastError(), __func__) != S3R_OK) return S3R_ERR_CUDA;
+  constexpr int smem2 = 2 * kVocabChunk * 4;
+  static bool attr_done = false;
+  if (!attr_done) {
+    if (cuda_status(cudaFuncSetAttribute(spec_draw_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         smem2), "cudaFuncSetAttribute") != S3R_OK)
+      return S3R_ERR_CUDA;
+    attr_done = true;
+  }
   dim3 g2(batch, p.nvch);
-  spec_draw_kernel<<<g2, kSampThreads, 0, stream>>>(p);
+  spec_draw_kernel<<<g2, kSampThreads, smem2, stream>>>(p);
   *launches = 2;
   return cuda_status(cudaGetLastError(), __func__);
 }
