@@ -3,6 +3,8 @@
 // workspace layout.
 #pragma once
 
+#include <utility>
+
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -161,6 +163,30 @@ __device__ __forceinline__ bool aborted(volatile int* abort_flag) {
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
 }
+// Programmatic dependent launch: every kernel of the library is launched with the
+// programmatic-stream-serialization attribute and waits here, before its first access to
+// global memory, until the preceding kernel of the stream has completed and its writes are
+// visible. Stream order is therefore unchanged; what overlaps is the next launch's set-up
+// (grid launch, CTA placement) with the previous kernel's tail. Without a preceding
+// programmatic launch the wait returns at once.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline void launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  (void)cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);   // errors: cudaGetLastError
+}
+
 // Untiled bulk copy global -> shared of `bytes` (both addresses 16-byte aligned, bytes a
 // multiple of 16), completion counted on `bar` (bytes).
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {

@@ -20,6 +20,7 @@ constexpr int kDraftStages = 2;
 
 template <int D>
 __global__ void __launch_bounds__(128) draft_kernel(const DraftParams p) {
+  pdl_wait();
   static_assert(kDraftChunk % 128 == 0, "128 threads resolve the chunk's rows");
   constexpr int NTW = 1, RW = 8, STAGE = 2 * kTile * D * 2, CPR = D / 8;
   extern __shared__ uint8_t smem_dyn[];
@@ -190,7 +191,7 @@ static int launch_draft_d(const DraftParams& p, int batch, cudaStream_t stream) 
     attr_done = true;
   }
   dim3 grid(p.nchunk_max, p.Hkv, batch);
-  draft_kernel<D><<<grid, 128, smem, stream>>>(p);
+  launch_pdl(draft_kernel<D>, grid, 128, smem, stream, p);
   return cuda_status(cudaGetLastError(), __func__);
 }
 

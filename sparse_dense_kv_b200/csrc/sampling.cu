@@ -313,6 +313,7 @@ __device__ __forceinline__ void smem_ms(const float* xs, int n, float& m, float&
 }
 
 __global__ void __launch_bounds__(kSampThreads) draft_sample_kernel(const SampleParams p) {
+  pdl_wait();
   extern __shared__ float4 xs4[];   // [kDsSpan] logits of this CTA's span
   float* xs = reinterpret_cast<float*>(xs4);
   __shared__ __align__(8) uint64_t bar;
@@ -399,6 +400,7 @@ __global__ void __launch_bounds__(kSampThreads) draft_sample_kernel(const Sample
 
 // ------------------------------------------------------- speculative sampling: pass 1 --
 __global__ void __launch_bounds__(kSampThreads) spec_norm_kernel(const SampleParams p) {
+  pdl_wait();
   __shared__ int s_flag;
   __shared__ float sM[2 * S3R_MAX_K + 1];
   __shared__ double sZ[2 * S3R_MAX_K + 1];
@@ -474,6 +476,7 @@ __global__ void __launch_bounds__(kSampThreads) spec_norm_kernel(const SamplePar
 
 // ------------------------------------------------------- speculative sampling: pass 2 --
 __global__ void __launch_bounds__(kSampThreads) spec_draw_kernel(const SampleParams p) {
+  pdl_wait();
   extern __shared__ float4 xs4[];   // the drawn chunk: p logits, then q logits
   float* xps = reinterpret_cast<float*>(xs4);
   float* xqs = xps + kVocabChunk;
@@ -630,6 +633,7 @@ __device__ __forceinline__ ArgMax warp_argmax(ArgMax a) {
 }
 
 __global__ void __launch_bounds__(kSampThreads) argmax_kernel(const SampleParams p, int mode) {
+  pdl_wait();
   __shared__ int s_flag;
   __shared__ ArgMax s_w[kSampThreads / 32];
   __shared__ ArgMax s_part[(S3R_MAX_K + 1) * 64];
@@ -712,13 +716,14 @@ __global__ void __launch_bounds__(kSampThreads) argmax_kernel(const SampleParams
 
 int launch_argmax(const SampleParams& p, int batch, int mode, cudaStream_t stream) {
   dim3 grid(batch, mode == 0 ? 1 : p.k + 1, p.nvch);
-  argmax_kernel<<<grid, kSampThreads, 0, stream>>>(p, mode);
+  launch_pdl(argmax_kernel, grid, kSampThreads, 0, stream, p, mode);
   return cuda_status(cudaGetLastError(), __func__);
 }
 
 // ------------------------------------------------------------------------- commit ----
 __global__ void commit_kernel(const int32_t* req_ids, int batch, int k, const int32_t* n_out,
                               int32_t* seq_lens, long long* stats) {
+  pdl_wait();
   const int bl = blockIdx.x * blockDim.x + threadIdx.x;
   if (bl >= batch) return;
   const int r = req_ids ? req_ids[bl] : bl;
@@ -736,6 +741,7 @@ __global__ void commit_kernel(const int32_t* req_ids, int batch, int k, const in
 
 __global__ void philox_kernel(uint64_t seed, int stream_id, const int32_t* request,
                               const int32_t* position, int64_t n, uint32_t* words, float* u) {
+  pdl_wait();
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= n) return;
   uint32_t c[4] = {(uint32_t)position[i], (uint32_t)request[i], (uint32_t)stream_id, 0u};
@@ -760,13 +766,13 @@ int launch_draft_sample(const SampleParams& p, int batch, cudaStream_t stream) {
     attr_done = true;
   }
   dim3 grid(batch, (p.vocab + kDsSpan - 1) / kDsSpan);
-  draft_sample_kernel<<<grid, kSampThreads, smem, stream>>>(p);
+  launch_pdl(draft_sample_kernel, grid, kSampThreads, smem, stream, p);
   return cuda_status(cudaGetLastError(), __func__);
 }
 
 int launch_spec_sample(const SampleParams& p, int batch, cudaStream_t stream, int* launches) {
   dim3 g1(batch, 2 * p.k + 1, p.nvch);
-  spec_norm_kernel<<<g1, kSampThreads, 0, stream>>>(p);
+  launch_pdl(spec_norm_kernel, g1, kSampThreads, 0, stream, p);
   if (cuda_status(cudaGetLastError(), __func__) != S3R_OK) return S3R_ERR_CUDA;
   constexpr int smem2 = 2 * kVocabChunk * 4;
   static bool attr_done = false;
@@ -777,7 +783,7 @@ int launch_spec_sample(const SampleParams& p, int batch, cudaStream_t stream, in
     attr_done = true;
   }
   dim3 g2(batch, p.nvch);
-  spec_draw_kernel<<<g2, kSampThreads, smem2, stream>>>(p);
+  launch_pdl(spec_draw_kernel, g2, kSampThreads, smem2, stream, p);
   *launches = 2;
   return cuda_status(cudaGetLastError(), __func__);
 }
@@ -798,14 +804,14 @@ void spec_offsets(int num_requests, int k, int vocab, size_t* plan_off, size_t* 
 
 int launch_commit(const int32_t* req_ids, int batch, int k, const int32_t* n_out,
                   int32_t* seq_lens, int64_t* stats, cudaStream_t stream) {
-  commit_kernel<<<(batch + 255) / 256, 256, 0, stream>>>(req_ids, batch, k, n_out, seq_lens,
+  launch_pdl(commit_kernel, (batch + 255) / 256, 256, 0, stream, req_ids, batch, k, n_out, seq_lens,
                                                         reinterpret_cast<long long*>(stats));
   return cuda_status(cudaGetLastError(), __func__);
 }
 
 int launch_philox(uint64_t seed, int stream_id, const int32_t* request, const int32_t* position,
                   int64_t n, uint32_t* words, float* u, cudaStream_t stream) {
-  philox_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(seed, stream_id, request, position,
+  launch_pdl(philox_kernel, (unsigned)((n + 255) / 256), 256, 0, stream, seed, stream_id, request, position,
                                                                  n, words, u);
   return cuda_status(cudaGetLastError(), __func__);
 }

@@ -63,6 +63,7 @@ __device__ __forceinline__ int block_excl_scan(int v, int* wsum) {
 
 template <int P>
 __global__ void __launch_bounds__(kSelectThreads, 2) select_kernel(const SelectParams p) {
+  pdl_wait();
   extern __shared__ uint32_t keys[];
   __shared__ uint32_t hist[kSelectBins];
   __shared__ int wsum[32], wa[32], wb[32];
@@ -272,6 +273,7 @@ constexpr int kSigmaThreads = 256;
 constexpr int kSigmaPos = 4 * kSigmaThreads;
 
 __global__ void __launch_bounds__(kSigmaThreads) sigma_kernel(const SelectParams p) {
+  pdl_wait();
   __shared__ float lse2[S3R_MAX_ROWS];
   const int kvh = blockIdx.y, bl = blockIdx.z;
   const int r = p.req_ids ? p.req_ids[bl] : bl;
@@ -322,7 +324,7 @@ int launch_select(const SelectParams& p, int batch, cudaStream_t stream, int* la
   SelectParams q = p;
   if (p.logits) {
     dim3 g((p.cap + kSigmaPos - 1) / kSigmaPos, p.Hkv, batch);
-    sigma_kernel<<<g, kSigmaThreads, 0, stream>>>(p);
+    launch_pdl(sigma_kernel, g, kSigmaThreads, 0, stream, p);
     if (cuda_status(cudaGetLastError(), "sigma_kernel") != S3R_OK) return S3R_ERR_CUDA;
     ++*launches;
     q.logits = nullptr;
@@ -344,9 +346,9 @@ int launch_select(const SelectParams& p, int batch, cudaStream_t stream, int* la
   }
   dim3 grid(q.Hkv, batch);
   if (p.page == S3R_PAGE_SIZE)
-    select_kernel<S3R_PAGE_SIZE><<<grid, kSelectThreads, smem, stream>>>(q);
+    launch_pdl(select_kernel<S3R_PAGE_SIZE>, grid, kSelectThreads, smem, stream, q);
   else
-    select_kernel<1><<<grid, kSelectThreads, smem, stream>>>(q);
+    launch_pdl(select_kernel<1>, grid, kSelectThreads, smem, stream, q);
   const int st = cuda_status(cudaGetLastError(), __func__);
   if (st == S3R_OK) ++*launches;
   return st;

@@ -27,6 +27,7 @@ template <int D, int MAXT>
 __global__ void __launch_bounds__(MAXT) verify_kernel(const __grid_constant__ CUtensorMap tmK,
                                                      const __grid_constant__ CUtensorMap tmV,
                                                      const VerifyParams p) {
+  pdl_wait();
   constexpr int NTW = 2, RW = 16, STAGE = verify_stage_bytes<D>();
   extern __shared__ uint8_t smem_dyn[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) &
@@ -225,6 +226,7 @@ constexpr int kCombBatch = 8;   // chunks whose loads are issued together
 
 template <int D>
 __global__ void __launch_bounds__(kCombThreads) verify_combine_kernel(const VerifyParams p) {
+  pdl_wait();
   extern __shared__ float cw[];   // m, l, weights: [nch][kCombRows] each
   const int j0 = blockIdx.x * kCombRows, kvh = blockIdx.y, bl = blockIdx.z;
   const int r = p.req_ids ? p.req_ids[bl] : bl;
@@ -327,7 +329,7 @@ int launch_verify_combine(const VerifyParams& p, int D, int batch, cudaStream_t 
       return S3R_ERR_CUDA;
     a = smem;
   }
-  kern<<<grid, kCombThreads, smem, stream>>>(p);
+  launch_pdl(kern, grid, kCombThreads, smem, stream, p);
   return cuda_status(cudaGetLastError(), __func__);
 }
 
@@ -348,7 +350,7 @@ static int launch_verify_t(const CUtensorMap& tk, const CUtensorMap& tv, const V
     attr_bytes = need;
   }
   dim3 grid(p.nchunk_max, p.Hkv, batch);
-  verify_kernel<D, MAXT><<<grid, threads, need, stream>>>(tk, tv, p);
+  launch_pdl(verify_kernel<D, MAXT>, grid, threads, need, stream, tk, tv, p);
   return cuda_status(cudaGetLastError(), __func__);
 }
 

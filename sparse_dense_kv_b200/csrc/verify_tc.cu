@@ -243,6 +243,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                      const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                      const __grid_constant__ CUtensorMap tmK8, const __grid_constant__ CUtensorMap tmV8,
                      const VerifyParams p, int batch) {
+  pdl_wait();
   using C = Cfg<NP>;
   extern __shared__ uint8_t smem_dyn[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) &
@@ -903,7 +904,7 @@ static int launch_tc(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
       return S3R_ERR_CUDA;
     attr_done = true;
   }
-  tc::verify_tc_kernel<NP><<<num_sms, tc::kThreads, C::kSmem, stream>>>(tq, tk, tv, tk8, tv8, p,
+  launch_pdl(tc::verify_tc_kernel<NP>, num_sms, tc::kThreads, C::kSmem, stream, tq, tk, tv, tk8, tv8, p,
                                                                         batch);
   return cuda_status(cudaGetLastError(), __func__);
 }
