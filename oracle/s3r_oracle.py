@@ -506,6 +506,39 @@ def expected_tau(alpha) -> float:
     return tau
 
 
+# ----------------------------------------------------------------------------------------
+# O-horizon: adaptive draft length.
+# [Wispaper] position-dependent acceptance: acceptance falls with the draft position and
+# over training, and the authors propose shortening the draft horizon when the later
+# positions' acceptance deteriorates (left to future work). [Listing] Table 7 prices a
+# round under sequential stage accounting as k draft steps plus one verify (6 T_q + T_V at
+# k = 6). Reading: estimate each position's acceptance from the counts so far, smoothed
+# toward a prior, alpha_j = (accepted_j + w * alpha0) / (decided_j + w); take the k in
+# [1, k_max] with the most expected tokens per unit round cost,
+# expected_tau(alpha_1..alpha_k) / (k * c_draft + c_verify), the smallest k on ties.
+# ----------------------------------------------------------------------------------------
+
+
+def acceptance_estimate(accepted, decided, prior_alpha: float, prior_weight: float):
+    """Smoothed per-position acceptance (a_j + w alpha0) / (d_j + w); the prior alone for a
+    position never decided (w > 0)."""
+    a = [float(x) for x in accepted]
+    d = [float(x) for x in decided]
+    return [(a[j] + prior_weight * prior_alpha) / (d[j] + prior_weight) for j in range(len(a))]
+
+
+def choose_horizon(accepted, decided, c_draft: float, c_verify: float, k_max: int,
+                   prior_alpha: float = 0.5, prior_weight: float = 4.0) -> int:
+    """Draft length for the next rounds (see the block comment above)."""
+    alpha = acceptance_estimate(accepted[:k_max], decided[:k_max], prior_alpha, prior_weight)
+    best_k, best = 1, -1.0
+    for k in range(1, k_max + 1):
+        rate = expected_tau(alpha[:k]) / (k * c_draft + c_verify)
+        if rate > best:
+            best_k, best = k, rate
+    return best_k
+
+
 def break_even_acceptance(total_ms: float, ar_ms: float, k: int) -> float:
     """Acceptance at which a round (draft + verify = total) costs as much per token as AR.
 
