@@ -324,7 +324,7 @@ def run_ours(args, spec):
     del graph
 
     st = eng.buf.stats.cpu().numpy()
-    acc = [float(st[2 + j] / max(st[2 + k + j], 1)) for j in range(k)]
+    acc = [float(st[2 + j] / max(st[2 + s3r.MAX_K + j], 1)) for j in range(k)]
     result = {
         "metric": METRIC, "value": tokens_all / (ms_max * 1e-3), "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -360,6 +360,132 @@ def run_ours(args, spec):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------ adaptive horizon ----
+
+
+def run_adaptive(args, spec):
+    """Rounds whose draft length an AdaptiveHorizon controller picks every --interval rounds
+    from the measured acceptance by position, against the same procedure at the fixed k of
+    the workload. Each length has its own CUDA graph: k draft steps, verify, speculative
+    sampling, commit, and the selection of the next round from this verify's scores (so a
+    graph never reads scores of another length); lengths grow from round to round. The
+    costs of a draft step and of the rest of a round come from replaying the graphs of two
+    lengths."""
+    import torch
+    import sparse_dense_kv_b200 as s3r
+
+    rank, world, local = dist_env()
+    if world > 1:
+        raise SystemExit("--adaptive runs on one GPU")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    k_max, k0 = args.k_max, spec.k
+    rounds_total = 2 * (args.warmup + args.steps) + 40
+    spec_m = spec.with_(k=k_max)
+    lens = synth.make_lengths(spec)
+    cache = synth.build_cache(spec_m, lens, extra_tokens=rounds_total * (k_max + 1) + 16, device=dev,
+                              seed=spec.data_seed)
+    NR, Hq, Hkv, d, V = spec.num_requests, spec.num_q_heads, spec.num_kv_heads, spec.head_dim, spec.vocab
+    base = dict(q=synth.randn_bf16((NR, k_max + 1, Hq, d), 100, dev),
+                k=synth.randn_bf16((NR, k_max + 1, Hkv, d), 101, dev),
+                v=synth.randn_bf16((NR, k_max + 1, Hkv, d), 102, dev),
+                p=synth.randn_f32((NR, k_max + 1, V), 103, dev, scale=spec.logit_std))
+    base["qlog"] = base["p"][:, :k_max] + synth.randn_f32((NR, k_max, V), 104, dev, scale=spec.draft_noise_std)
+    inputs = {k: dict(q=base["q"][:, : k + 1].contiguous(), k=base["k"][:, : k + 1].contiguous(),
+                      v=base["v"][:, : k + 1].contiguous(), p=base["p"][:, : k + 1].contiguous(),
+                      qlog=base["qlog"][:, :k].contiguous()) for k in range(1, k_max + 1)}
+    seq0 = torch.as_tensor(lens, dtype=torch.int32, device=dev)
+
+    def fresh_engine():
+        seq = seq0.clone()
+        eng = s3r.S3REngine(cache.k_pool, cache.v_pool, cache.page_table, seq, Hq, k=k0,
+                            budget_bp=spec.budget_bp, window=max(spec.window, k_max + 1),
+                            vocab=V, seed=spec.sample_seed, k_max=k_max)
+        x = inputs[k_max]
+        eng.prefill(x["q"][:, :1].contiguous(), x["k"][:, :1].contiguous(), x["v"][:, :1].contiguous())
+        eng.select()
+        graphs = {}
+        for k in range(1, k_max + 1):
+            eng.set_k(k)
+            xk = inputs[k]
+
+            def step(xk=xk, k=k):
+                for i in range(k):
+                    eng.draft_attn(i, xk["q"], xk["k"], xk["v"])
+                    eng.draft_sample(i, xk["qlog"])
+                eng.verify(xk["q"], xk["k"], xk["v"])
+                eng.sample_and_commit(xk["p"], xk["qlog"])
+                eng.select()
+            graphs[k], _ = eng.capture(step)
+        return eng, graphs
+
+    E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+
+    def replay_ms(graphs, k, n=8):
+        a, b = E(), E()
+        a.record()
+        for _ in range(n):
+            graphs[k].replay()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / n
+
+    def run(adaptive: bool):
+        eng, graphs = fresh_engine()
+        eng.set_k(k0)
+        for _ in range(args.warmup):
+            graphs[k0].replay()
+        # costs per round: t(k) = c_verify + k c_draft from two lengths
+        ka, kb = 2, k_max
+        ta, tb = replay_ms(graphs, ka), replay_ms(graphs, kb)
+        c_draft = max((tb - ta) / (kb - ka), 1e-4)
+        c_verify = max(ta - ka * c_draft, 1e-4)
+        ctl = s3r.AdaptiveHorizon(eng, c_draft, c_verify, decay=args.decay) if adaptive else None
+        assert eng.check_errors() == 0, "device error in warm-up"
+        tok0 = int(eng.buf.stats[0].item())
+        ks = []
+        torch.cuda.synchronize()
+        a, b = E(), E()
+        a.record()
+        k = k0
+        for st_ in range(args.steps):
+            if ctl is not None and st_ % args.interval == 0:
+                k = ctl.step()
+            ks.append(k)
+            graphs[k].replay()
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b)
+        tokens = int(eng.buf.stats[0].item()) - tok0
+        assert eng.check_errors() == 0, "device error in the timed rounds"
+        st = eng.buf.stats.cpu().numpy()
+        acc = [float(st[2 + j] / max(st[2 + s3r.MAX_K + j], 1)) for j in range(k_max)]
+        del graphs
+        return dict(ms=ms, tokens=tokens, ks=ks, c_draft=c_draft, c_verify=c_verify, acc=acc)
+
+    fixed = run(False)
+    adapt = run(True)
+    hist = {str(k): adapt["ks"].count(k) for k in range(1, k_max + 1) if k in adapt["ks"]}
+    value = adapt["tokens"] / (adapt["ms"] * 1e-3)
+    result = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": adapt["ms"] / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{spec.name} (config {args.config}): {NR} requests, L {spec.lengths} growing "
+                               f"by the emitted tokens, {Hq}/{Hkv} heads, d {d}, s {spec.budget_bp / 1e4}, "
+                               f"vocab {V}, adaptive draft length in 1..{k_max}",
+                   "requests_per_gpu": NR, "parallelism": "replicas x1", "horizon": "adaptive",
+                   "interval": args.interval, "decay": args.decay},
+        "adaptive": {"k_histogram": hist, "c_draft_ms": adapt["c_draft"], "c_verify_ms": adapt["c_verify"],
+                     "acceptance_by_position": adapt["acc"][:k_max],
+                     "tau": adapt["tokens"] / max(1, args.steps * NR)},
+        "fixed_k": {"k": k0, "value": fixed["tokens"] / (fixed["ms"] * 1e-3), "ms_per_step": fixed["ms"] / args.steps,
+                    "tau": fixed["tokens"] / max(1, args.steps * NR)},
+        "execution": "one CUDA graph per draft length, chosen on the host every interval rounds",
+    }
+    print(json.dumps(result), flush=True)
 
 
 # -------------------------------------------------------------------------- sweep -------
@@ -433,7 +559,7 @@ def run_sweep(args):
                     timed += 1
             assert eng.check_errors() == 0
             st = eng.buf.stats.cpu().numpy()
-            acc = [float(st[2 + j] / max(st[2 + k + j], 1)) for j in range(k)]
+            acc = [float(st[2 + j] / max(st[2 + s3r.MAX_K + j], 1)) for j in range(k)]
             print(json.dumps({
                 "sweep_point": {"budget": bp / 1e4, "k": k}, "workload": spec.name,
                 "rounds": timed, "requests": NR, "context": int(lens[0]),
@@ -564,6 +690,12 @@ def main(argv=None):
                     help="selection unit: positions, or whole 16-position pages")
     ap.add_argument("--greedy", action="store_true",
                     help="temperature 0: argmax drafts and greedy verification")
+    ap.add_argument("--adaptive", action="store_true",
+                    help="draft length chosen from the measured acceptance (one line, with the fixed-k run)")
+    ap.add_argument("--k-max", type=int, default=7,
+                    help="largest adaptive draft length (7: the verify stays on the tensor-memory kernel at G = 4)")
+    ap.add_argument("--interval", type=int, default=4)
+    ap.add_argument("--decay", type=float, default=0.8)
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -577,6 +709,8 @@ def main(argv=None):
         raise SystemExit("config 3 (mixed phases) and 4 (sweep) are parity / sweep cases, not bench lines")
     if args.impl == "reference":
         run_reference(args, spec)
+    elif args.adaptive:
+        run_adaptive(args, spec)
     else:
         run_ours(args, spec)
 

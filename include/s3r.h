@@ -18,6 +18,7 @@
  *   s3r_verify_attn        dense attention of the k+1 rows at L..L+k, with score capture
  *   s3r_spec_sample        exact speculative sampling -> a accepted drafts + 1 token
  *   s3r_commit             L <- L + a + 1, acceptance counters
+ *   s3r_choose_horizon     (host) draft length for the next rounds from those counters
  *
  * Conventions shared by every call
  *   - Every pointer argument is a DEVICE pointer owned by the caller, unless it is marked
@@ -258,9 +259,27 @@ S3R_API int s3r_greedy_verify(const s3r_batch* batch, int32_t k, const float* p_
 /* Commit a round ([Explainer] Jargon, block efficiency: tokens per round): for each
  * request of the batch, seq_lens[r] += n_out[r]. stats (int64, may be NULL) accumulates
  * [0] tokens emitted, [1] request-rounds, [2+j] drafts accepted at position j and
- * [2+k+j] drafts decided at position j (j < k); it has 2 + 2k entries. */
+ * [2+S3R_MAX_K+j] drafts decided at position j (j < k); it has 2 + 2*S3R_MAX_K entries, laid
+ * out alike whatever k, so rounds of different draft lengths count into the same array. */
 S3R_API int s3r_commit(const s3r_batch* batch, int32_t k, const int32_t* n_out, int32_t* seq_lens,
                int64_t* stats, s3r_stream_t stream);
+
+/* Adaptive draft length ([Wispaper] position-dependent acceptance: shorten the draft
+ * horizon when the later positions' acceptance falls; [Listing] Table 7: a round costs k
+ * draft steps plus one verify). HOST function, no device work: with the smoothed
+ * acceptance alpha_j = (accepted[j] + prior_weight * prior_alpha) / (decided[j] +
+ * prior_weight) for positions j < k_max, writes to *k_out the k in [1, k_max] that
+ * maximises (1 + sum_{i<=k} prod_{j<=i} alpha_j) / (k * c_draft + c_verify), the smallest
+ * k on ties (all arithmetic in double, in that order).
+ *   accepted, decided  host double [k_max]: counts per draft position (for instance the
+ *                      stats of s3r_commit, possibly decayed over time); not kept.
+ *   c_draft, c_verify  cost of one draft step and of the rest of a round (any unit, > 0).
+ * S3R_ERR_INVALID_ARG for NULL pointers, k_max outside 1..S3R_MAX_K, a cost <= 0 or not
+ * finite, prior_alpha outside [0, 1], prior_weight < 0, a negative count, or a position with
+ * decided + prior_weight == 0. */
+S3R_API int s3r_choose_horizon(const double* accepted, const double* decided, int32_t k_max,
+                       double c_draft, double c_verify, double prior_alpha,
+                       double prior_weight, int32_t* k_out);
 
 /* Philox4x32-10 words and uniforms for n counters (position[i], request[i], stream_id, 0)
  * under key = seed: words uint32 [n][4] (may be NULL), u fp32 [n] (may be NULL). */

@@ -15,6 +15,7 @@ from ._lib import (  # noqa: F401
     make_batch,
     make_cache,
     new_workspace,
+    s3r_choose_horizon,
     s3r_commit,
     s3r_draft_argmax,
     s3r_draft_sample,
@@ -35,4 +36,4 @@ from ._lib import (  # noqa: F401
     s3r_workspace_init,
     s3r_workspace_size,
 )
-from .engine import MixedPhaseDriver, RoundBuffers, S3REngine  # noqa: F401
+from .engine import AdaptiveHorizon, MixedPhaseDriver, RoundBuffers, S3REngine  # noqa: F401

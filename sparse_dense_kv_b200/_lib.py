@@ -64,6 +64,8 @@ def _load():
         "s3r_draft_sample_noalloc": (ctypes.c_int, [B, P, I32, P, I32, U64, P, P, P]),
         "s3r_spec_sample": (ctypes.c_int, [B, I32, P, P, P, I32, U64, P, P, P, SZ, P]),
         "s3r_draft_argmax": (ctypes.c_int, [B, P, I32, P, I32, P, P, SZ, P]),
+        "s3r_choose_horizon": (ctypes.c_int, [P, P, I32, ctypes.c_double, ctypes.c_double,
+                                              ctypes.c_double, ctypes.c_double, P]),
         "s3r_greedy_verify": (ctypes.c_int, [B, I32, P, P, I32, P, P, P, SZ, P]),
         "s3r_commit": (ctypes.c_int, [B, I32, P, P, P, P]),
         "s3r_philox": (ctypes.c_int, [U64, I32, P, P, I64, P, P, P]),
@@ -298,6 +300,21 @@ def s3r_commit(batch, k, n_out, seq_lens, stats=None, stream=None):
         ctypes.byref(batch), k, _ptr(n_out, torch.int32, "n_out"),
         _ptr(seq_lens, torch.int32, "seq_lens"), _ptr(stats, torch.int64, "stats", allow_none=True),
         _stream(stream)), "s3r_commit")
+
+
+def s3r_choose_horizon(accepted, decided, c_draft, c_verify, prior_alpha=0.5, prior_weight=4.0):
+    """Host call: draft length in [1, len(accepted)] from per-position counts (sequences of
+    float; the first len(accepted) positions)."""
+    k_max = len(accepted)
+    if len(decided) != k_max:
+        raise ValueError("accepted and decided differ in length")
+    arr = ctypes.c_double * max(k_max, 1)
+    a, d, out = arr(*accepted), arr(*decided), ctypes.c_int32(0)
+    _check(_lib.s3r_choose_horizon(ctypes.cast(a, ctypes.c_void_p), ctypes.cast(d, ctypes.c_void_p),
+                                   k_max, float(c_draft), float(c_verify), float(prior_alpha),
+                                   float(prior_weight), ctypes.cast(ctypes.pointer(out), ctypes.c_void_p)),
+           "s3r_choose_horizon")
+    return int(out.value)
 
 
 def s3r_philox(seed, stream_id, request, position, words=None, u=None, stream=None):

@@ -2,6 +2,7 @@
 // descriptors and kernel launches. Nothing here allocates device memory.
 #include <atomic>
 #include <cstdio>
+#include <cmath>
 #include <cstring>
 #include <mutex>
 
@@ -697,6 +698,36 @@ int s3r_commit(const s3r_batch* batch, int32_t k, const int32_t* n_out, int32_t*
   return finish(launch_commit(batch->req_ids, batch->batch, k, n_out, seq_lens, stats,
                               (cudaStream_t)stream),
                 1);
+}
+
+int s3r_choose_horizon(const double* accepted, const double* decided, int32_t k_max,
+                       double c_draft, double c_verify, double prior_alpha, double prior_weight,
+                       int32_t* k_out) {
+  if (!accepted || !decided || !k_out || k_max < 1 || k_max > S3R_MAX_K) return S3R_ERR_INVALID_ARG;
+  if (!(c_draft > 0.0) || !(c_verify > 0.0) || !std::isfinite(c_draft) || !std::isfinite(c_verify))
+    return S3R_ERR_INVALID_ARG;
+  if (!(prior_alpha >= 0.0 && prior_alpha <= 1.0) || !(prior_weight >= 0.0) || !std::isfinite(prior_weight))
+    return S3R_ERR_INVALID_ARG;
+  double alpha[S3R_MAX_K];
+  for (int j = 0; j < k_max; ++j) {
+    if (!(accepted[j] >= 0.0) || !(decided[j] >= 0.0) || !std::isfinite(accepted[j]) ||
+        !std::isfinite(decided[j]) || decided[j] + prior_weight == 0.0)
+      return S3R_ERR_INVALID_ARG;
+    alpha[j] = (accepted[j] + prior_weight * prior_alpha) / (decided[j] + prior_weight);
+  }
+  int best_k = 1;
+  double best = -1.0, tau = 1.0, run = 1.0;
+  for (int k = 1; k <= k_max; ++k) {
+    run *= alpha[k - 1];
+    tau += run;
+    const double rate = tau / ((double)k * c_draft + c_verify);
+    if (rate > best) {
+      best = rate;
+      best_k = k;
+    }
+  }
+  *k_out = best_k;
+  return S3R_OK;
 }
 
 int s3r_philox(uint64_t seed, int32_t stream_id, const int32_t* request, const int32_t* position,

@@ -733,7 +733,7 @@ __global__ void commit_kernel(const int32_t* req_ids, int batch, int k, const in
     atomicAdd(reinterpret_cast<unsigned long long*>(&stats[0]), (unsigned long long)n);
     atomicAdd(reinterpret_cast<unsigned long long*>(&stats[1]), 1ull);
     for (int j = 0; j < k && j < n; ++j) {
-      atomicAdd(reinterpret_cast<unsigned long long*>(&stats[2 + k + j]), 1ull);
+      atomicAdd(reinterpret_cast<unsigned long long*>(&stats[2 + S3R_MAX_K + j]), 1ull);
       if (j < n - 1) atomicAdd(reinterpret_cast<unsigned long long*>(&stats[2 + j]), 1ull);
     }
   }

@@ -21,34 +21,53 @@ def budget_count(length: int, budget_bp: int, window: int) -> int:
 
 
 class RoundBuffers:
-    """Device buffers of one batch: selection, attention outputs, tokens and statistics."""
+    """Device buffers of one batch: selection, attention outputs, tokens and statistics.
 
-    def __init__(self, num_requests, num_q_heads, num_kv_heads, head_dim, cap, k, vocab,
+    The buffers whose layout depends on the draft length hold k_max drafts; set_k(k) makes
+    the attributes contiguous views laid out for k (the layouts the library's calls use), so
+    the draft length can change between rounds."""
+
+    def __init__(self, num_requests, num_q_heads, num_kv_heads, head_dim, cap, k_max, vocab,
                  sel_stride, device="cuda"):
+        self.dims = (num_requests, num_q_heads, num_kv_heads, head_dim, cap)
         G = num_q_heads // num_kv_heads
         f32, bf, i32 = torch.float32, torch.bfloat16, torch.int32
-        self.scores = torch.empty((num_requests, num_kv_heads, G * (k + 1), cap), dtype=f32, device=device)
-        self.lse = torch.empty((num_requests, k + 1, num_q_heads), dtype=f32, device=device)
+        T = k_max + 1
+        self.k_max = k_max
+        self._scores = torch.empty(num_requests * num_kv_heads * G * T * cap, dtype=f32, device=device)
+        self._lse = torch.empty(num_requests * T * num_q_heads, dtype=f32, device=device)
+        self._verify_out = torch.empty(num_requests * T * num_q_heads * head_dim, dtype=bf, device=device)
+        self._draft_tokens = torch.zeros(num_requests * k_max, dtype=i32, device=device)
+        self._out_tokens = torch.full((num_requests * T,), -1, dtype=i32, device=device)
         self.prefill_lse = torch.empty((num_requests, 1, num_q_heads), dtype=f32, device=device)
         self.sel_idx = torch.zeros((num_requests, num_kv_heads, sel_stride), dtype=i32, device=device)
         self.sel_count = torch.zeros((num_requests, num_kv_heads), dtype=i32, device=device)
-        self.steps = [torch.full((num_requests,), i, dtype=i32, device=device) for i in range(max(k, 1))]
+        self.steps = [torch.full((num_requests,), i, dtype=i32, device=device) for i in range(k_max)]
         self.draft_out = torch.empty((num_requests, num_q_heads, head_dim), dtype=bf, device=device)
         self.draft_lse = torch.empty((num_requests, num_q_heads), dtype=f32, device=device)
-        self.verify_out = torch.empty((num_requests, k + 1, num_q_heads, head_dim), dtype=bf, device=device)
-        self.draft_tokens = torch.zeros((num_requests, max(k, 1)), dtype=i32, device=device)
-        self.out_tokens = torch.full((num_requests, k + 1), -1, dtype=i32, device=device)
         self.n_out = torch.zeros((num_requests,), dtype=i32, device=device)
-        self.stats = torch.zeros((2 + 2 * k,), dtype=torch.int64, device=device)
+        # [0] tokens, [1] request-rounds, [2 + j] accepted / [2 + MAX_K + j] decided at position j
+        self.stats = torch.zeros((2 + 2 * L.MAX_K,), dtype=torch.int64, device=device)
+        self.set_k(k_max)
+
+    def set_k(self, k: int):
+        NR, Hq, Hkv, d, cap = self.dims
+        G, T = Hq // Hkv, k + 1
+        self.scores = self._scores[: NR * Hkv * G * T * cap].view(NR, Hkv, G * T, cap)
+        self.lse = self._lse[: NR * T * Hq].view(NR, T, Hq)
+        self.verify_out = self._verify_out[: NR * T * Hq * d].view(NR, T, Hq, d)
+        self.draft_tokens = self._draft_tokens[: NR * k].view(NR, k)
+        self.out_tokens = self._out_tokens[: NR * T].view(NR, T)
 
 
 class S3REngine:
     """S3R rounds for a batch of requests over one paged KV cache on one GPU."""
 
     def __init__(self, k_pool, v_pool, page_table, seq_lens, num_q_heads, *, k, budget_bp,
-                 window, vocab, seed, sel_stride=None, greedy=False, page_select=False):
-        if not (1 <= k <= L.MAX_K):
-            raise ValueError("k must be in 1..8")
+                 window, vocab, seed, sel_stride=None, greedy=False, page_select=False, k_max=None):
+        k_max = k if k_max is None else k_max
+        if not (1 <= k <= k_max <= L.MAX_K):
+            raise ValueError("need 1 <= k <= k_max <= 8")
         self.k, self.budget_bp, self.window, self.vocab, self.seed = k, budget_bp, window, vocab, seed
         self.greedy = greedy   # temperature 0: argmax drafts, greedy verification
         self.page_select = page_select   # whole 16-position pages instead of positions
@@ -62,14 +81,23 @@ class S3REngine:
         self.sel_stride = sel_stride or (budget_count(self.cap, budget_bp, window)
                                          + (L.PAGE_SIZE - 1 if page_select else 0))
         self.buf = RoundBuffers(self.num_requests, num_q_heads, self.cache.num_kv_heads,
-                                self.cache.head_dim, self.cap, k, vocab, self.sel_stride,
+                                self.cache.head_dim, self.cap, k_max, vocab, self.sel_stride,
                                 k_pool.device)
-        nbytes = L.s3r_workspace_size(self.cache, self.num_requests, self.max_pages, k, vocab,
+        self.buf.set_k(k)
+        nbytes = L.s3r_workspace_size(self.cache, self.num_requests, self.max_pages, k_max, vocab,
                                       self.sel_stride)
         self.ws = L.new_workspace(nbytes, k_pool.device)
         self.batch = L.make_batch(seq_lens, page_table)
         self.k_prev = None
         self._verify_launches = 2
+
+    def set_k(self, k: int):
+        """Draft length of the next rounds (1 <= k <= k_max). The selection of the next round
+        still reads the last verify's scores with that verify's length (k_prev)."""
+        if not (1 <= k <= self.buf.k_max):
+            raise ValueError("k outside 1..k_max")
+        self.k = k
+        self.buf.set_k(k)
 
     @property
     def launches_per_round(self) -> int:
@@ -255,3 +283,45 @@ class MixedPhaseDriver:
                 b.sel_count, e.ws)
         self.phases = (self.phases + 1) % (e.k + 1)
         return v_ids
+
+
+class AdaptiveHorizon:
+    """Draft length from the measured acceptance by position: the engine's counters are read
+    every call of step() (one device-to-host copy), added to exponentially decayed counts,
+    and s3r_choose_horizon picks the k with the most expected tokens per unit round cost
+    (c_draft per draft step, c_verify for the rest of the round). Positions not drafted for
+    a while decay toward the prior, so longer horizons are tried again when it is good; with
+    prior_alpha="pooled" the prior is the acceptance pooled over all positions so far (the
+    plain expectation for a position without evidence of its own)."""
+
+    def __init__(self, engine: S3REngine, c_draft: float, c_verify: float, *, decay: float = 0.8,
+                 prior_alpha="pooled", prior_weight: float = 4.0, k_max: int | None = None):
+        self.e = engine
+        self.c_draft, self.c_verify = c_draft, c_verify
+        self.decay, self.prior_alpha, self.prior_weight = decay, prior_alpha, prior_weight
+        self.k_max = k_max or engine.buf.k_max
+        self.acc = [0.0] * L.MAX_K
+        self.dec = [0.0] * L.MAX_K
+        self.last = engine.buf.stats.cpu().tolist()
+        self.history = []
+
+    def observe(self):
+        st = self.e.buf.stats.cpu().tolist()
+        for j in range(L.MAX_K):
+            self.acc[j] = self.decay * self.acc[j] + (st[2 + j] - self.last[2 + j])
+            self.dec[j] = self.decay * self.dec[j] + (st[2 + L.MAX_K + j] - self.last[2 + L.MAX_K + j])
+        self.last = st
+
+    def prior(self) -> float:
+        if self.prior_alpha != "pooled":
+            return float(self.prior_alpha)
+        d = sum(self.dec[: self.k_max])
+        return sum(self.acc[: self.k_max]) / d if d > 0 else 0.5
+
+    def step(self) -> int:
+        self.observe()
+        k = L.s3r_choose_horizon(self.acc[: self.k_max], self.dec[: self.k_max], self.c_draft,
+                                 self.c_verify, self.prior(), self.prior_weight)
+        self.e.set_k(k)
+        self.history.append(k)
+        return k

@@ -13,14 +13,14 @@ from tests.test_oracle_round import make_states
 pytestmark = pytest.mark.gpu
 
 
-def gpu_engine(spec, rounds, page_select=False, greedy=False):
+def gpu_engine(spec, rounds, page_select=False, greedy=False, k_max=None):
     lens = synth.make_lengths(spec)
     cache = synth.build_cache(spec, lens, extra_tokens=800)
     seq = torch.as_tensor(lens, dtype=torch.int32).cuda()
     eng = s3r.S3REngine(cache.k_pool.cuda(), cache.v_pool.cuda(), cache.page_table.cuda(), seq,
                         spec.num_q_heads, k=spec.k, budget_bp=spec.budget_bp, window=spec.window,
                         vocab=spec.vocab, seed=spec.sample_seed, page_select=page_select,
-                        greedy=greedy)
+                        greedy=greedy, k_max=k_max)
     qs, ks, vs = zip(*[synth.token_qkv(spec, r, [int(lens[r])]) for r in range(spec.num_requests)])
     eng.prefill(torch.stack(qs).cuda(), torch.stack(ks).cuda(), torch.stack(vs).cuda())
     return eng
@@ -44,19 +44,27 @@ def near_threshold(sigma, L, spec, page):
     return {int(q) * page + t for q in pages for t in range(page)}
 
 
-@pytest.mark.parametrize("page,greedy", [(1, False), (16, False), (1, True), (16, True)])
-def test_rounds_match_oracle_tiny(page, greedy):
+K_SCHEDULE = [6, 3, 1, 5, 2, 6, 4, 1, 1, 6]
+
+
+@pytest.mark.parametrize("page,greedy,vary_k", [(1, False, False), (16, False, False), (1, True, False),
+                                                (16, True, False), (1, False, True), (16, True, True)])
+def test_rounds_match_oracle_tiny(page, greedy, vary_k):
     """Rounds are compared request by request. A decision whose oracle margin is below 1e-5
     may go either way; if the GPU then differs, that request's later rounds are no longer
     comparable and it leaves the comparison (counted). page 16: page-granular selection;
-    greedy: argmax drafts and greedy verification (no sampling margins: tokens must match)."""
-    spec = synth.CONFIGS[0]
+    greedy: argmax drafts and greedy verification (no sampling margins: tokens must match);
+    vary_k: the draft length changes from round to round (adaptive horizon), the selection
+    reading the scores of a verify of another length."""
+    spec0 = synth.CONFIGS[0]
     n_rounds = 40
-    eng = gpu_engine(spec, n_rounds, page_select=page > 1, greedy=greedy)
-    states = make_states(spec)
-    alive = [True] * spec.num_requests
+    eng = gpu_engine(spec0, n_rounds, page_select=page > 1, greedy=greedy, k_max=spec0.k)
+    states = make_states(spec0)
+    alive = [True] * spec0.num_requests
     compared = diverged = boundary = 0
     for rnd in range(n_rounds):
+        spec = spec0.with_(k=K_SCHEDULE[rnd % len(K_SCHEDULE)]) if vary_k else spec0
+        eng.set_k(spec.k)
         lengths = eng.seq_lens.cpu().numpy().tolist()
         for r, st in enumerate(states):
             if alive[r]:
@@ -95,6 +103,33 @@ def test_rounds_match_oracle_tiny(page, greedy):
     st = b.stats.cpu().numpy()
     assert st[1] > 0 and st[0] >= st[1]
     print(f"compared {compared} request-rounds, boundary decisions {boundary}, diverged {diverged}")
+
+
+def test_adaptive_horizon_follows_acceptance_and_costs():
+    """The controller on whole rounds: with every draft accepted (draft logits equal to the
+    target's) and verify far dearer than a draft step it keeps the longest horizon; once a
+    draft step is made dear it drops to one draft; rounds at the chosen lengths stay
+    error-free and count decisions only at the positions drafted."""
+    spec = synth.CONFIGS[0]
+    eng = gpu_engine(spec, 0, k_max=spec.k)
+    ctl = s3r.AdaptiveHorizon(eng, c_draft=1.0, c_verify=1000.0, prior_weight=1.0)
+
+    def rounds(n):
+        for _ in range(n):
+            lengths = eng.seq_lens.cpu().numpy().tolist()
+            q, k, v, pl, ql = round_inputs(spec.with_(k=eng.k), lengths)
+            eng.round(q, k, v, pl, pl[:, : eng.k].contiguous())
+            assert eng.check_errors() == 0
+
+    rounds(3)
+    assert ctl.step() == spec.k and eng.k == spec.k
+    ctl.c_draft = 1e6
+    assert ctl.step() == 1 and eng.k == 1
+    before = eng.buf.stats.cpu().numpy()
+    rounds(2)
+    after = eng.buf.stats.cpu().numpy()
+    dec = after[2 + s3r.MAX_K: 2 + 2 * s3r.MAX_K] - before[2 + s3r.MAX_K: 2 + 2 * s3r.MAX_K]
+    assert dec[0] == 2 * spec.num_requests and not dec[1:].any()
 
 
 def test_device_errors_are_reported_not_faulted():
