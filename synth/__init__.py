@@ -18,3 +18,4 @@ from .workload import (  # noqa: F401
     randn_bf16,
     randn_f32,
 )
+from .rollouts import RolloutSpec, make_rollouts  # noqa: F401,E402
