@@ -19,6 +19,7 @@
  *   s3r_spec_sample        exact speculative sampling -> a accepted drafts + 1 token
  *   s3r_commit             L <- L + a + 1, acceptance counters
  *   s3r_choose_horizon     (host) draft length for the next rounds from those counters
+ *   s3r_sched_simulate     (host) KV-aware AIMD admission of requests to a replica
  *
  * Conventions shared by every call
  *   - Every pointer argument is a DEVICE pointer owned by the caller, unless it is marked
@@ -263,6 +264,62 @@ S3R_API int s3r_greedy_verify(const s3r_batch* batch, int32_t k, const float* p_
  * out alike whatever k, so rounds of different draft lengths count into the same array. */
 S3R_API int s3r_commit(const s3r_batch* batch, int32_t k, const int32_t* n_out, int32_t* seq_lens,
                int64_t* stats, s3r_stream_t stream);
+
+/* KV-aware admission of requests to one rollout replica ([News] summary: a KV-aware AIMD
+ * scheduler adapts admission to limit repeated KV offloading and restoring while keeping
+ * rollout parallelism; [Explainer] Jargon, AIMD scheduler: admit one more request when
+ * GPU KV memory has room, halve the limit under pressure; [Explainer] "Where it earns its
+ * keep": back off when pressure or the restore backlog grows; [Wispaper] "dense
+ * verification still needs the complete KV cache": utilisation and the paused requests'
+ * backlog drive it). HOST function, no device work: a discrete-event model of the
+ * replica, one iteration per draft-and-verify round of all active requests:
+ *   1. capacity C_t = capacity - pressure[t] pages (pressure may be NULL; t >= pressure_len:
+ *      0), the injected memory-pressure events;
+ *   2. each active request, in admission order, emits min(tau[r][j], left) tokens, j its
+ *      own round count; finished requests free their pages;
+ *   3. U = sum of ceil((prompt + generated) / 16) over active requests;
+ *   4. while U > C_t the most recently admitted request is evicted to the FIFO paused
+ *      queue (evict 0: its pages are offloaded to host memory, transferred += pages;
+ *      evict 1: dropped, recomputed when restored);
+ *   5. policy 0 (AIMD): cap = max(cap_min, cap / 2) if anything was evicted, U > u_high C_t
+ *      or the paused requests' pages > b_high C_t; else cap = min(cap_max, cap + 1) if the
+ *      cap binds (active >= cap) and U < u_low C_t. Policy 1 keeps cap = cap0;
+ *   6. while active < cap: restore the head of the paused queue (transferred, or
+ *      recomputed, += its pages), else admit the next new request (prefilled += its prompt
+ *      pages), each only if U + pages <= C_t, else stop for this iteration;
+ *   7. time += c0 + c_tok tokens_t + c_kv U + c_xfer transferred_t + c_rec recomputed_t +
+ *      c_pre prefilled_t (in double, in that order).
+ * The run ends when all requests are done, after max_iters, or when no progress is
+ * possible (nothing active and the head of the queues cannot fit; result.stalled = 1).
+ *   prompt_len, resp_len  host int32 [num_requests] (>= 0): prompt tokens, tokens to emit.
+ *   tau                   host uint8 [num_requests][tau_stride]: tokens one round emits
+ *                         for request r at its j-th active round (a run that needs more
+ *                         than tau_stride rounds of one request is S3R_ERR_INVALID_ARG).
+ *   pressure              host int32 [pressure_len] (0 <= pressure < capacity) or NULL.
+ *   out                   totals; trace (host int32 [trace_cap][8], may be NULL): per
+ *                         iteration cap, active, paused, U, transferred, recomputed,
+ *                         prefilled, tokens, for the first trace_cap iterations.
+ * S3R_ERR_INVALID_ARG for NULL inputs, sizes or parameters out of range. */
+typedef struct {
+  int32_t capacity;   /* GPU KV pages (16 tokens each) of the replica */
+  int32_t policy;     /* 0 AIMD, 1 fixed cap */
+  int32_t evict;      /* 0 offload to host memory, 1 recompute on restore */
+  int32_t cap0, cap_min, cap_max;
+  double u_low, u_high, b_high;
+  double c0, c_tok, c_kv, c_xfer, c_rec, c_pre;
+  int64_t max_iters;
+} s3r_sched_config;
+
+typedef struct {
+  int64_t tokens, transferred, recomputed, prefilled, evictions, iterations;
+  int32_t max_active, done, stalled, reserved;
+  double time;
+} s3r_sched_result;
+
+S3R_API int s3r_sched_simulate(const s3r_sched_config* cfg, int32_t num_requests,
+                       const int32_t* prompt_len, const int32_t* resp_len, const uint8_t* tau,
+                       int64_t tau_stride, const int32_t* pressure, int64_t pressure_len,
+                       s3r_sched_result* out, int32_t* trace, int64_t trace_cap);
 
 /* Adaptive draft length ([Wispaper] position-dependent acceptance: shorten the draft
  * horizon when the later positions' acceptance falls; [Listing] Table 7: a round costs k

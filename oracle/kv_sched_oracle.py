@@ -15,7 +15,9 @@ GPU KV utilisation measures resident pressure, the restore backlog the unmet dem
 paused requests, which keep their tokens and proposal state).
 
 The reading taken (every step below is fixed so that two implementations agree exactly):
-one iteration is one draft-and-verify round of every active request.
+one iteration is one draft-and-verify round of every active request. The default backlog
+mark b_high = 1 reads "too large a backlog" as more paused pages than the whole replica
+holds; at half of it the cap collapses to a few requests during a long pressure event.
   1. capacity of this iteration C_t = capacity - pressure[t] pages (injected pressure).
   2. every active request, in admission order, emits min(tau[r][j], left) tokens, j its
      own round count; a request with nothing left is done and frees its pages.
@@ -49,7 +51,7 @@ def pages(prompt: int, generated: int) -> int:
 
 def simulate(prompt_len, resp_len, tau, *, capacity: int, policy: str = "aimd",
              evict: str = "offload", cap0: int = 16, cap_min: int = 1, cap_max: int = 4096,
-             u_low: float = 0.85, u_high: float = 0.97, b_high: float = 0.5,
+             u_low: float = 0.85, u_high: float = 0.97, b_high: float = 1.0,
              costs=(10.0, 0.0, 0.00074, 0.094, 0.5, 0.5), pressure=None, max_iters: int = 1 << 20):
     """Runs the scheduler; returns (totals dict, trace list of per-iteration tuples
     (cap, active, paused, U, transferred, recomputed, prefilled, tokens))."""

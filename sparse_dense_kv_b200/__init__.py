@@ -17,6 +17,7 @@ from ._lib import (  # noqa: F401
     new_workspace,
     s3r_choose_horizon,
     s3r_commit,
+    s3r_sched_simulate,
     s3r_draft_argmax,
     s3r_draft_sample,
     s3r_draft_sample_noalloc,

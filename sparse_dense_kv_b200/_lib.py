@@ -45,6 +45,23 @@ class BatchDesc(ctypes.Structure):
                 ("page_table", ctypes.c_void_p), ("max_pages_per_req", ctypes.c_int32)]
 
 
+class SchedConfig(ctypes.Structure):
+    _fields_ = [("capacity", ctypes.c_int32), ("policy", ctypes.c_int32), ("evict", ctypes.c_int32),
+                ("cap0", ctypes.c_int32), ("cap_min", ctypes.c_int32), ("cap_max", ctypes.c_int32),
+                ("u_low", ctypes.c_double), ("u_high", ctypes.c_double), ("b_high", ctypes.c_double),
+                ("c0", ctypes.c_double), ("c_tok", ctypes.c_double), ("c_kv", ctypes.c_double),
+                ("c_xfer", ctypes.c_double), ("c_rec", ctypes.c_double), ("c_pre", ctypes.c_double),
+                ("max_iters", ctypes.c_int64)]
+
+
+class SchedResult(ctypes.Structure):
+    _fields_ = [("tokens", ctypes.c_int64), ("transferred", ctypes.c_int64),
+                ("recomputed", ctypes.c_int64), ("prefilled", ctypes.c_int64),
+                ("evictions", ctypes.c_int64), ("iterations", ctypes.c_int64),
+                ("max_active", ctypes.c_int32), ("done", ctypes.c_int32), ("stalled", ctypes.c_int32),
+                ("reserved", ctypes.c_int32), ("time", ctypes.c_double)]
+
+
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"libs3r.so is not built ({LIB_PATH}); run python sparse_dense_kv_b200/build.py")
@@ -64,6 +81,9 @@ def _load():
         "s3r_draft_sample_noalloc": (ctypes.c_int, [B, P, I32, P, I32, U64, P, P, P]),
         "s3r_spec_sample": (ctypes.c_int, [B, I32, P, P, P, I32, U64, P, P, P, SZ, P]),
         "s3r_draft_argmax": (ctypes.c_int, [B, P, I32, P, I32, P, P, SZ, P]),
+        "s3r_sched_simulate": (ctypes.c_int, [ctypes.POINTER(SchedConfig), I32, P, P, P, ctypes.c_int64,
+                                              P, ctypes.c_int64, ctypes.POINTER(SchedResult), P,
+                                              ctypes.c_int64]),
         "s3r_choose_horizon": (ctypes.c_int, [P, P, I32, ctypes.c_double, ctypes.c_double,
                                               ctypes.c_double, ctypes.c_double, P]),
         "s3r_greedy_verify": (ctypes.c_int, [B, I32, P, P, I32, P, P, P, SZ, P]),
@@ -315,6 +335,33 @@ def s3r_choose_horizon(accepted, decided, c_draft, c_verify, prior_alpha=0.5, pr
                                    float(prior_weight), ctypes.cast(ctypes.pointer(out), ctypes.c_void_p)),
            "s3r_choose_horizon")
     return int(out.value)
+
+
+def s3r_sched_simulate(prompt_len, resp_len, tau, *, capacity, policy="aimd", evict="offload",
+                       cap0=16, cap_min=1, cap_max=4096, u_low=0.85, u_high=0.97, b_high=1.0,
+                       costs=(10.0, 0.0, 0.00074, 0.094, 0.5, 0.5), pressure=None,
+                       max_iters=1 << 20, trace=True):
+    """Host call: the KV-aware admission model over numpy inputs; returns (totals dict,
+    trace int32 [iterations][8] or None)."""
+    import numpy as np
+    prompt = np.ascontiguousarray(prompt_len, dtype=np.int32)
+    resp = np.ascontiguousarray(resp_len, dtype=np.int32)
+    tau = np.ascontiguousarray(tau, dtype=np.uint8)
+    if tau.ndim != 2 or tau.shape[0] != prompt.size or resp.size != prompt.size:
+        raise ValueError("tau must be [num_requests][rounds]")
+    pr = None if pressure is None else np.ascontiguousarray(pressure, dtype=np.int32)
+    cfg = SchedConfig(capacity, {"aimd": 0, "fixed": 1}[policy], {"offload": 0, "recompute": 1}[evict],
+                      cap0, cap_min, cap_max, u_low, u_high, b_high, *costs, max_iters)
+    res = SchedResult()
+    cap_rows = int(max_iters) if trace else 0
+    cap_rows = min(cap_rows, 1 << 22)
+    tr = np.zeros((cap_rows, 8), dtype=np.int32) if cap_rows else None
+    vp = lambda a: None if a is None else a.ctypes.data_as(ctypes.c_void_p)  # noqa: E731
+    _check(_lib.s3r_sched_simulate(ctypes.byref(cfg), prompt.size, vp(prompt), vp(resp), vp(tau),
+                                   tau.shape[1], vp(pr), 0 if pr is None else pr.size,
+                                   ctypes.byref(res), vp(tr), cap_rows), "s3r_sched_simulate")
+    tot = {f: getattr(res, f) for f, _ in SchedResult._fields_ if f != "reserved"}
+    return tot, (tr[: min(res.iterations, cap_rows)] if tr is not None else None)
 
 
 def s3r_philox(seed, stream_id, request, position, words=None, u=None, stream=None):

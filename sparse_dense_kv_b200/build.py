@@ -16,7 +16,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libs3r.so")
-SOURCES = ["s3r_api.cu", "verify.cu", "verify_tc.cu", "draft.cu", "select.cu", "sampling.cu"]
+SOURCES = ["s3r_api.cu", "verify.cu", "verify_tc.cu", "draft.cu", "select.cu", "sampling.cu", "sched.cpp"]
 HEADERS = ["common.cuh", "attention.cuh", "kernels.h"]
 
 

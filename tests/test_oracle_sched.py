@@ -53,7 +53,7 @@ def test_recompute_counts_restores_not_transfers():
 def test_aimd_halves_on_eviction_and_backlog():
     # 4 requests of 1-page prompts, 48 tokens, 16 per round, capacity 6 (high mark 5.82,
     # low mark 5.1, backlog mark 3), AIMD from cap 4
-    tot, tr = K.simulate([16] * 4, [48] * 4, tau_const(4, 16), capacity=6, cap0=4)
+    tot, tr = K.simulate([16] * 4, [48] * 4, tau_const(4, 16), capacity=6, cap0=4, b_high=0.5)
     assert tr == [
         (4, 4, 0, 4, 0, 0, 4, 0),    # cap does not bind yet (0 active): admit 4
         (2, 3, 1, 6, 2, 0, 0, 64),   # 2 pages each, U 8 > 6: evict r3 (U 6 fits); cap 4 -> 2
