@@ -431,8 +431,8 @@ def run_adaptive(args, spec):
     the workload. Each length has its own CUDA graph: k draft steps, verify, speculative
     sampling, commit, and the selection of the next round from this verify's scores (so a
     graph never reads scores of another length); lengths grow from round to round. The
-    costs of a draft step and of the rest of a round come from replaying the graphs of two
-    lengths."""
+    costs of a draft step and of the rest of a round come from a line fitted to replays of
+    the graphs of k = 3 .. k_max."""
     import torch
     import sparse_dense_kv_b200 as s3r
 
@@ -497,11 +497,15 @@ def run_adaptive(args, spec):
         eng.set_k(k0)
         for _ in range(args.warmup):
             graphs[k0].replay()
-        # costs per round: t(k) = c_verify + k c_draft from two lengths
-        ka, kb = 2, k_max
-        ta, tb = replay_ms(graphs, ka), replay_ms(graphs, kb)
-        c_draft = max((tb - ta) / (kb - ka), 1e-4)
-        c_verify = max(ta - ka * c_draft, 1e-4)
+        # costs per round: t(k) = c_verify + k c_draft, a least-squares line through the
+        # replayed graphs of k = 3 .. k_max (one verify configuration: 32-row tiles at G = 4)
+        kk = np.arange(min(3, k_max), k_max + 1, dtype=np.float64)
+        tt = np.array([replay_ms(graphs, int(k)) for k in kk])
+        if kk.size >= 2:
+            c_draft, c_verify = (float(x) for x in np.polyfit(kk, tt, 1))
+        else:
+            c_draft, c_verify = tt[0] / 2, tt[0] / 2
+        c_draft, c_verify = max(c_draft, 1e-4), max(c_verify, 1e-4)
         ctl = s3r.AdaptiveHorizon(eng, c_draft, c_verify, decay=args.decay) if adaptive else None
         assert eng.check_errors() == 0, "device error in warm-up"
         tok0 = int(eng.buf.stats[0].item())
