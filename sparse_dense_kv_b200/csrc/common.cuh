@@ -1,6 +1,6 @@
 // Device helpers shared by the S3R kernels: PTX wrappers for sm_100a (ldmatrix, mma.sync,
-// movmatrix, cp.async, mbarrier, TMA tiled loads), warp reductions, Philox4x32-10 and the
-// workspace layout.
+// movmatrix, cp.async, mbarrier, TMA tiled and untiled bulk loads, programmatic dependent
+// launch), warp reductions, Philox4x32-10 and the workspace layout.
 #pragma once
 
 #include <utility>
