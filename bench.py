@@ -1,6 +1,6 @@
 """Benchmark of the S3R per-round hot path on B200 (one process per GPU).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config 2]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload qwen3-8b]
 
 A step is one whole S3R round over the batch of the chosen synthetic workload (default:
 the Qwen3-8B-shaped single attention layer, 32 requests with contexts uniform in
@@ -330,7 +330,7 @@ def run_ours(args, spec):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": f"{spec.name} (config {args.config}): {spec.num_requests} requests, "
+        "config": {"workload": f"{spec.name}: {spec.num_requests} requests, "
                                f"L {spec.lengths}, {spec.num_q_heads}/{spec.num_kv_heads} heads, "
                                f"d {spec.head_dim}, k {k}, s {spec.budget_bp / 1e4}, window {spec.window}, "
                                f"vocab {spec.vocab}",
@@ -537,7 +537,7 @@ def run_adaptive(args, spec):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": adapt["ms"] / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": f"{spec.name} (config {args.config}): {NR} requests, L {spec.lengths} growing "
+        "config": {"workload": f"{spec.name}: {NR} requests, L {spec.lengths} growing "
                                f"by the emitted tokens, {Hq}/{Hkv} heads, d {d}, s {spec.budget_bp / 1e4}, "
                                f"vocab {V}, adaptive draft length in 1..{k_max}",
                    "requests_per_gpu": NR, "parallelism": "replicas x1", "horizon": "adaptive",
@@ -562,7 +562,7 @@ def run_sweep(args):
     import torch
     import sparse_dense_kv_b200 as s3r
     from sparse_dense_kv_b200.engine import budget_count
-    spec = synth.CONFIGS[4]
+    spec = synth.WORKLOADS["sweep"]
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     lens = synth.make_lengths(spec)
@@ -725,7 +725,7 @@ def run_reference(args, spec):
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
            "data": "synthetic",
-           "config": {"workload": f"{spec.name} (config {args.config}), one request-round per step",
+           "config": {"workload": f"{spec.name}, one request-round per step",
                       "requests_sampled": NR, "selection": args.select,
                       "verification": "greedy" if args.greedy else "speculative sampling"},
            "cpu_baseline": {"value": v, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
@@ -741,7 +741,8 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", type=int, default=2)
+    ap.add_argument("--workload", default="qwen3-8b", choices=["tiny", "qwen3-1.7b", "qwen3-8b"],
+                    help="synthetic workload (the ragged mixed-phase and sweep workloads are test / sweep cases)")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -771,11 +772,11 @@ def main(argv=None):
     if args.sched:
         run_sched(args)
         return
-    spec = synth.CONFIGS[args.config]
+    spec = synth.WORKLOADS[args.workload]
     if args.requests > 0:
         spec = spec.with_(num_requests=args.requests)
     if spec.projection_logits or spec.mixed_phases:
-        raise SystemExit("config 3 (mixed phases) and 4 (sweep) are parity / sweep cases, not bench lines")
+        raise SystemExit("the mixed-phase and sweep workloads are parity / sweep cases, not bench lines")
     if args.impl == "reference":
         run_reference(args, spec)
     elif args.adaptive:

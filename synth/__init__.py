@@ -5,7 +5,7 @@ sampling, no Philox): it only draws the synthetic KV cache, the per-token q/k/v 
 synthetic logits from seeded generators, with the shapes of the Qwen3-shaped workloads.
 """
 from .workload import (  # noqa: F401
-    CONFIGS,
+    WORKLOADS,
     WorkloadSpec,
     KVCache,
     make_lengths,

@@ -5,15 +5,15 @@ pages (Qwen3-shaped head counts; the pages' own runs used Qwen3-1.7B / Qwen3-8B 
 rollouts on DAPO-MATH prompts, which are not available here, so random tensors with the
 stated distributions stand in for them):
 
-  0 tiny      2 requests, L in {256, 300}, 2 q-heads / 1 kv-head, d 64, k 6, s 0.25,
+  tiny        2 requests, L in {256, 300}, 2 q-heads / 1 kv-head, d 64, k 6, s 0.25,
               window 16, vocab 64, target logits N(0, 2), draft = target + N(0, 0.3^2)
-  1 qwen3-1.7b  64 requests, L ~ U[4096, 16384], 16/8 heads, d 128, k 6, s 0.05,
+  qwen3-1.7b  64 requests, L ~ U[4096, 16384], 16/8 heads, d 128, k 6, s 0.05,
               window 64, 32 heavy-hitter keys (x4) per (request, kv-head), vocab 151936,
               draft noise N(0, 0.5^2)
-  2 qwen3-8b  32 requests, L ~ U[8192, 24576], 32/8 heads, otherwise as 1
-  3 ragged    256 requests, L log-uniform in [1024, 16384], 16/8 heads, mixed round
-              phases, shuffled page tables, otherwise as 1
-  4 sweep     32 requests at L = 24576, 32/8 heads, s in {.02,.05,.1,.2} x k in
+  qwen3-8b    32 requests, L ~ U[8192, 24576], 32/8 heads, otherwise as qwen3-1.7b
+  ragged      256 requests, L log-uniform in [1024, 16384], 16/8 heads, mixed round
+              phases, shuffled page tables, otherwise as qwen3-1.7b
+  sweep       32 requests at L = 24576, 32/8 heads, s in {.02,.05,.1,.2} x k in
               {2,4,6,8}, vocab 32768, logits from a seeded bf16 projection of the
               head-concatenated attention outputs
 
@@ -62,7 +62,7 @@ class WorkloadSpec:
         return replace(self, **kw)
 
 
-CONFIGS = [
+_SPECS = [
     WorkloadSpec("tiny", 2, 2, 1, 64, ("fixed", (256, 300)), k=6, budget_bp=2500, window=16,
                  vocab=64, logit_std=math.sqrt(2.0), draft_noise_std=0.3,
                  data_seed=0, sample_seed=1000),
@@ -81,6 +81,7 @@ CONFIGS = [
                  heavy_hitters=32, projection_logits=True, data_seed=4, sample_seed=1004,
                  sweep_budgets_bp=(200, 500, 1000, 2000), sweep_ks=(2, 4, 6, 8)),
 ]
+WORKLOADS = {spec.name: spec for spec in _SPECS}
 
 
 def bf16_round(x) -> np.ndarray:

@@ -14,7 +14,7 @@ MARGIN = 1e-5                     # decisions closer than this to a boundary are
 
 def spec_for(H_q, H_kv, d, lens, k=6, budget_bp=500, window=64, vocab=64, seed=0, heavy=0,
              shuffle=False):
-    return synth.CONFIGS[0].with_(num_requests=len(lens), num_q_heads=H_q, num_kv_heads=H_kv,
+    return synth.WORKLOADS["tiny"].with_(num_requests=len(lens), num_q_heads=H_q, num_kv_heads=H_kv,
                                   head_dim=d, lengths=("fixed", tuple(int(x) for x in lens)),
                                   k=k, budget_bp=budget_bp, window=window, vocab=vocab,
                                   data_seed=seed, heavy_hitters=heavy, shuffle_pages=shuffle)

@@ -54,7 +54,7 @@ def test_ranks_build_same_shaped_disjoint_work():
     import torch
     import bench
     import synth
-    spec = synth.CONFIGS[0]
+    spec = synth.WORKLOADS["tiny"]
     l0, c0, s0, i0 = bench.build_workload(spec, 0, "cpu")
     l1, c1, s1, i1 = bench.build_workload(spec, 1, "cpu")
     assert (l0 == l1).all() and torch.equal(s0, s1)

@@ -58,7 +58,7 @@ def test_mixed_phase_batch_matches_oracle():
     mid-round with one launch over its ids and verifies the others with another; after k+1
     iterations every request has finished the round it was in, which must equal the
     oracle's round for that request."""
-    spec = synth.CONFIGS[3].with_(num_requests=24, lengths=("loguniform", 1024, 3072))
+    spec = synth.WORKLOADS["ragged"].with_(num_requests=24, lengths=("loguniform", 1024, 3072))
     k = spec.k
     lens = synth.make_lengths(spec)
     cache = synth.build_cache(spec, lens, extra_tokens=2 * (k + 1) + 16)
@@ -100,11 +100,11 @@ def test_mixed_phase_batch_matches_oracle():
     assert st[1] == spec.num_requests
 
 
-@pytest.mark.parametrize("config", [1, 2])
-def test_full_size_round_on_sampled_requests(config):
+@pytest.mark.parametrize("workload", ["qwen3-1.7b", "qwen3-8b"])
+def test_full_size_round_on_sampled_requests(workload):
     """One round of the whole Qwen3-shaped batch at full size (the benchmark's launch
     configuration); the oracle replays two sampled requests."""
-    spec = synth.CONFIGS[config]
+    spec = synth.WORKLOADS[workload]
     k = spec.k
     lens = synth.make_lengths(spec)
     cache = synth.build_cache(spec, lens, extra_tokens=k + 1 + 16, device="cuda")
@@ -115,7 +115,7 @@ def test_full_size_round_on_sampled_requests(config):
     vb = synth.randn_bf16((NR, k + 1, Hkv, d), 102, "cuda")
     pl = synth.randn_f32((NR, k + 1, V), 103, "cuda", scale=spec.logit_std)
     ql = (pl[:, :k] + synth.randn_f32((NR, k, V), 104, "cuda", scale=spec.draft_noise_std)).contiguous()
-    rng = np.random.default_rng(config)
+    rng = np.random.default_rng(spec.data_seed)
     picks = sorted(rng.choice(NR, size=2, replace=False).tolist())
     pt = cache.page_table.cpu().numpy()
     host = {}
@@ -154,7 +154,7 @@ def test_projection_logits_round_matches_oracle():
     head-concatenated attention outputs, fewer and shorter requests so the oracle stays
     quick): attention outputs of every draft step and of the verify match the oracle's, and
     the GPU samplers, given the oracle's own logits, take the oracle's decisions."""
-    spec = synth.CONFIGS[4].with_(num_requests=3, lengths=("fixed", (3000, 4100, 2500)))
+    spec = synth.WORKLOADS["sweep"].with_(num_requests=3, lengths=("fixed", (3000, 4100, 2500)))
     k, V = spec.k, spec.vocab
     NR, Hq, Hkv, d = spec.num_requests, spec.num_q_heads, spec.num_kv_heads, spec.head_dim
     lens = synth.make_lengths(spec)
@@ -244,7 +244,7 @@ def test_full_size_mixed_phase_batch_on_sampled_requests():
     """The high-concurrency workload at full size: 256 requests, contexts log-uniform in
     [1024, 16384], shuffled pages, mixed round phases; k+1 driver iterations complete one
     round per request, and the oracle replays four sampled requests."""
-    spec = synth.CONFIGS[3]
+    spec = synth.WORKLOADS["ragged"]
     k = spec.k
     lens = synth.make_lengths(spec)
     cache = synth.build_cache(spec, lens, extra_tokens=2 * (k + 1) + 16, device="cuda")

@@ -52,7 +52,7 @@ def test_greedy_draft_and_verify_match_oracle(V):
 def test_greedy_rounds_through_the_engine():
     """Whole greedy rounds on the tiny workload; identical draft and target logits must
     accept every draft (k + 1 tokens per round)."""
-    spec = synth.CONFIGS[0]
+    spec = synth.WORKLOADS["tiny"]
     lens = synth.make_lengths(spec)
     cache = synth.build_cache(spec, lens, extra_tokens=200)
     seq = torch.as_tensor(lens, dtype=torch.int32).cuda()

@@ -56,7 +56,7 @@ def test_rounds_match_oracle_tiny(page, greedy, vary_k):
     greedy: argmax drafts and greedy verification (no sampling margins: tokens must match);
     vary_k: the draft length changes from round to round (adaptive horizon), the selection
     reading the scores of a verify of another length."""
-    spec0 = synth.CONFIGS[0]
+    spec0 = synth.WORKLOADS["tiny"]
     n_rounds = 40
     eng = gpu_engine(spec0, n_rounds, page_select=page > 1, greedy=greedy, k_max=spec0.k)
     states = make_states(spec0)
@@ -110,7 +110,7 @@ def test_adaptive_horizon_follows_acceptance_and_costs():
     target's) and verify far dearer than a draft step it keeps the longest horizon; once a
     draft step is made dear it drops to one draft; rounds at the chosen lengths stay
     error-free and count decisions only at the positions drafted."""
-    spec = synth.CONFIGS[0]
+    spec = synth.WORKLOADS["tiny"]
     eng = gpu_engine(spec, 0, k_max=spec.k)
     ctl = s3r.AdaptiveHorizon(eng, c_draft=1.0, c_verify=1000.0, prior_weight=1.0)
 
@@ -133,7 +133,7 @@ def test_adaptive_horizon_follows_acceptance_and_costs():
 
 
 def test_device_errors_are_reported_not_faulted():
-    spec = synth.CONFIGS[0]
+    spec = synth.WORKLOADS["tiny"]
     lens = synth.make_lengths(spec)
     cache = synth.build_cache(spec, lens, extra_tokens=32)
     pt = cache.page_table.clone()

@@ -44,7 +44,7 @@ def run_rounds(spec, n_rounds):
 
 
 def test_hundred_rounds_tiny_is_fast_and_deterministic():
-    spec = synth.CONFIGS[0]
+    spec = synth.WORKLOADS["tiny"]
     t0 = time.time()
     states, log = run_rounds(spec, 100)
     assert time.time() - t0 < 120
