@@ -39,3 +39,51 @@ def test_choose_horizon_hand_worked_case():
 def test_choose_horizon_rejects_bad_arguments(args):
     with pytest.raises(s3r.S3RError):
         s3r.s3r_choose_horizon(*args)
+
+
+class _FakeBuf:
+    def __init__(self, k_max):
+        import torch
+        self.k_max = k_max
+        self.stats = torch.zeros(2 + 2 * s3r.MAX_K, dtype=torch.int64)
+
+
+class _FakeEngine:
+    """The controller's view of an engine: the commit counters, k_max and set_k."""
+
+    def __init__(self, k_max):
+        self.buf = _FakeBuf(k_max)
+        self.k = k_max
+
+    def set_k(self, k):
+        self.k = k
+
+    def commit(self, accepted, decided):
+        for j, (a, d) in enumerate(zip(accepted, decided)):
+            self.buf.stats[2 + j] += a
+            self.buf.stats[2 + s3r.MAX_K + j] += d
+
+
+def test_controller_decays_counts_and_pools_the_prior():
+    eng = _FakeEngine(6)
+    ctl = s3r.AdaptiveHorizon(eng, c_draft=57.0, c_verify=730.0, decay=0.5, prior_weight=4.0)
+    eng.commit([80, 60, 40, 0, 0, 0], [100, 80, 60, 0, 0, 0])
+    k1 = ctl.step()
+    assert ctl.acc[:3] == [80.0, 60.0, 40.0] and ctl.dec[:3] == [100.0, 80.0, 60.0]
+    pooled = 180.0 / 240.0
+    assert ctl.prior() == pooled
+    want = O.choose_horizon(ctl.acc[:6], ctl.dec[:6], 57.0, 730.0, 6, pooled, 4.0)
+    assert k1 == want == eng.k
+    # a second window halves the first and adds the new counts
+    eng.commit([10, 0, 0, 0, 0, 0], [20, 0, 0, 0, 0, 0])
+    ctl.step()
+    assert ctl.acc[0] == 0.5 * 80 + 10 and ctl.dec[0] == 0.5 * 100 + 20 and ctl.dec[1] == 40.0
+    assert ctl.history == [k1, eng.k]
+
+
+def test_controller_fixed_prior():
+    eng = _FakeEngine(4)
+    ctl = s3r.AdaptiveHorizon(eng, c_draft=1.0, c_verify=1000.0, prior_alpha=0.0, prior_weight=4.0)
+    eng.commit([50, 0, 0, 0], [50, 0, 0, 0])
+    # position 1 always accepted, later positions never drafted and a prior of 0: k = 1
+    assert ctl.step() == 1
