@@ -86,3 +86,20 @@ def test_full_size_invariants(policy, cap0):
         for a, b in zip(caps, caps[1:]):
             assert b <= a + 1                        # additive increase: +1 at most
             assert b >= a or b == max(1, a // 2)     # a decrease is a halving
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_offload_moves_twice_what_recompute_recomputes(seed):
+    """The evict mode only changes the counters, never a decision: on the same population
+    the traces agree in cap, active, paused and resident pages, and every evicted request's
+    pages go out and come back once (offload) or are recomputed once (recompute)."""
+    spec = synth.RolloutSpec(num_requests=96, seed=100 + seed)
+    p, r, tau = synth.make_rollouts(spec)
+    pressure = np.zeros(1500, dtype=np.int32)
+    pressure[500:900] = 2500
+    kw = dict(capacity=9000, pressure=pressure, policy=["aimd", "fixed"][seed % 2], cap0=[16, 128][seed % 2])
+    off, t_off = K.simulate(p, r, tau, evict="offload", **kw)
+    rec, t_rec = K.simulate(p, r, tau, evict="recompute", **kw)
+    assert [x[:4] for x in t_off] == [x[:4] for x in t_rec]
+    assert off["done"] == rec["done"] == 96 and off["evictions"] == rec["evictions"] > 0
+    assert off["transferred"] == 2 * rec["recomputed"] and rec["transferred"] == 0
