@@ -109,3 +109,47 @@ def test_noalloc_draft_sample_validates_on_the_host():
                                       null) == 1
     assert L.s3r_draft_sample_noalloc(ctypes.byref(b), 0x10, 9, 0x10, 1000, 1, 0x10, 0x10,
                                       null) == 2
+
+
+C_PROGRAM = r"""
+#include <stdio.h>
+#include "s3r.h"
+int main(void) {
+  double a[2] = {9.0, 8.0}, d[2] = {10.0, 10.0};
+  int32_t k = 0;
+  int st = s3r_choose_horizon(a, d, 2, 1.0, 100.0, 0.5, 1.0, &k);
+  s3r_sched_config cfg = {50, 0, 0, 4, 1, 64, 0.85, 0.97, 1.0, 10.0, 0.0, 0.001, 0.1, 0.5, 0.5, 1000};
+  int32_t prompt[1] = {16}, resp[1] = {32};
+  uint8_t tau[64];
+  for (int i = 0; i < 64; ++i) tau[i] = 4;
+  s3r_sched_result res;
+  int st2 = s3r_sched_simulate(&cfg, 1, prompt, resp, tau, 64, NULL, 0, &res, NULL, 0);
+  size_t ws = s3r_workspace_size(NULL, 1, 1, 6, 64, 64);
+  printf("%d %d %d %lld %lld %zu\n", st, k, st2, (long long)res.tokens, (long long)res.done, ws);
+  return 0;
+}
+"""
+
+
+def test_header_is_plain_c_and_host_calls_run_from_c(tmp_path):
+    """The boundary as a C user sees it: the header compiles as strict C99, a C program
+    links the library and runs its host-only calls (no GPU needed)."""
+    import shutil
+    import subprocess
+    import sparse_dense_kv_b200 as s3r
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "abi.c"
+    src.write_text(C_PROGRAM)
+    exe = tmp_path / "abi"
+    libdir = os.path.dirname(s3r.LIB_PATH)
+    res = subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I",
+                          os.path.join(ROOT, "include"), str(src), "-o", str(exe), "-L", libdir, "-ls3r",
+                          f"-Wl,-rpath,{libdir}"], capture_output=True, text=True)
+    assert res.returncode == 0, res.stderr
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0, out.stderr
+    st, k, st2, tokens, done, ws = out.stdout.split()
+    assert (st, k, st2, tokens, done) == ("0", "2", "0", "32", "1")
+    assert ws == "0"   # a NULL cache descriptor is rejected (size 0)
