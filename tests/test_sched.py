@@ -121,3 +121,38 @@ def test_two_replicas_as_gloo_ranks():
         assert res[0][key] == shards[0][key] + shards[1][key]
     assert res[0]["time"] == max(shards[0]["time"], shards[1]["time"])
     assert res[0]["tokens"] == int(r.sum())
+
+
+def _dying_replica_worker(rank, world, port, out):
+    import torch.distributed as dist
+    from datetime import timedelta
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=10))
+    if rank == 1:
+        out.put((rank, "left"))
+        out.close()
+        out.join_thread()              # the message is out before the process goes
+        os._exit(3)                    # the replica dies before the collective, no cleanup
+    from sparse_dense_kv_b200.replicas import simulate_replicas
+    p, r, tau = synth.make_rollouts(synth.RolloutSpec(num_requests=16, seed=5))
+    try:
+        simulate_replicas(p, r, tau, capacity=4000, cap0=8)
+        out.put((rank, "no error"))
+    except Exception as exc:           # the collective fails instead of waiting for good
+        out.put((rank, f"error: {type(exc).__name__}"))
+
+
+def test_a_dead_replica_fails_the_others_fast():
+    """A replica that dies before the totals' all-reduce: the survivor's collective ends
+    with an error (peer gone, or the process group's 10 s timeout) rather than a hang."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_dying_replica_worker, args=(k, 2, port, q)) for k in range(2)]
+    for pr in procs:
+        pr.start()
+    res = dict(q.get(timeout=120) for _ in procs)
+    for pr in procs:
+        pr.join(timeout=60)
+    assert res[1] == "left"
+    assert res[0].startswith("error"), res[0]
