@@ -87,3 +87,23 @@ def test_controller_fixed_prior():
     eng.commit([50, 0, 0, 0], [50, 0, 0, 0])
     # position 1 always accepted, later positions never drafted and a prior of 0: k = 1
     assert ctl.step() == 1
+
+
+def test_round_buffers_views_share_their_storage_across_lengths():
+    """set_k lays the length-dependent buffers out for k in the same storage: every view
+    starts at the same address whatever k (graphs captured per length keep valid
+    pointers) and has the contiguous layout the library's calls use for that k."""
+    from sparse_dense_kv_b200.engine import RoundBuffers
+    NR, Hq, Hkv, d, cap = 3, 8, 2, 16, 64
+    b = RoundBuffers(NR, Hq, Hkv, d, cap, 6, 64, 32, device="cpu")
+    ptrs = {name: getattr(b, name).data_ptr() for name in
+            ("scores", "lse", "verify_out", "draft_tokens", "out_tokens")}
+    for k in (1, 3, 6):
+        b.set_k(k)
+        G, T = Hq // Hkv, k + 1
+        assert b.scores.shape == (NR, Hkv, G * T, cap) and b.scores.is_contiguous()
+        assert b.lse.shape == (NR, T, Hq) and b.verify_out.shape == (NR, T, Hq, d)
+        assert b.draft_tokens.shape == (NR, k) and b.out_tokens.shape == (NR, T)
+        for name, p in ptrs.items():
+            assert getattr(b, name).data_ptr() == p, (name, k)
+    assert b.stats.numel() == 2 + 2 * s3r.MAX_K and len(b.steps) == 6
