@@ -34,9 +34,11 @@
  *   - KV pools: bf16 [num_pages][num_kv_heads][16][head_dim]; head_dim is 64 or 128.
  *     Query head h reads KV head h / G, G = num_q_heads / num_kv_heads <= 8.
  *   - Requests: a launch covers `batch` requests; with req_ids == NULL they are requests
- *     0..batch-1, else req_ids[0..batch-1]. Every per-request array is indexed by the
- *     request id (size num_requests), so a launch can cover a subset of a larger batch
- *     (mixed round phases).
+ *     0..batch-1, else req_ids[0..batch-1], which must be distinct and in [0, num_requests)
+ *     (the samplers check the range on the device: an id outside it sets
+ *     S3R_ERR_DEVICE_BOUNDS and that request is skipped). Every per-request array is indexed
+ *     by the request id (size num_requests), so a launch can cover a subset of a larger
+ *     batch (mixed round phases).
  *     Attention and selection calls cover at most 65535 requests per launch.
  *   - Page table: int32 [num_requests][max_pages_per_req]; position j of request r is
  *     slot j % 16 of page page_table[r][j / 16]. capacity = 16 * max_pages_per_req.
@@ -201,27 +203,33 @@ S3R_API int s3r_sparse_draft_attn(const s3r_kv_cache* cache, const s3r_batch* ba
  * counter = (L+i+1, r, 0, 0)) word 0 >> 8, times 2^-24; the token is the smallest v with
  * u * Z < C_v (C inclusive cumulative sum of exp(x - max), Z its total), written to
  * draft_tokens[r][i].  q_logits fp32 [num_requests][k][vocab]; draft_tokens int32
- * [num_requests][k]. */
+ * [num_requests][k]. margins (fp32 [num_requests][k], may be NULL) receives the draw's
+ * distance to the nearer edge of the drawn token's cell, min(u - C_{v-1}/Z, C_v/Z - u),
+ * as this call computed the sums: a draw with a margin below the rounding of those sums
+ * may go either way in another correct implementation. */
 S3R_API int s3r_draft_sample(const s3r_batch* batch, const int32_t* draft_step, int32_t k,
                      const float* q_logits, int32_t vocab, uint64_t seed, int32_t* draft_tokens,
-                     void* ws, size_t ws_bytes, s3r_stream_t stream);
+                     float* margins, void* ws, size_t ws_bytes, s3r_stream_t stream);
 
 /* s3r_draft_sample without a workspace. The paper has no counterpart: this is a
  * library convenience for callers that cannot hand the library device memory at the
  * point of the call: a host program that drives the library from plain C without an
  * allocator of its own, or a server that has given all free HBM to the KV pool and must
  * not allocate between rounds. Same arguments, arithmetic and outputs as
- * s3r_draft_sample, bit for bit; the scratch (arrival tickets and per-chunk partials)
- * lives in a static device array inside the library, 8 KiB + 1 MiB per device, so
+ * s3r_draft_sample (without margins), bit for bit; the scratch (arrival tickets and
+ * per-chunk partials) lives in a static device array inside the library, 8 KiB + 1 MiB
+ * per device that loads the library, held until the process exits, so
  *   - num_requests <= S3R_NOALLOC_MAX_REQUESTS and vocab <= S3R_NOALLOC_MAX_VOCAB, else
  *     S3R_ERR_UNSUPPORTED with a message in s3r_last_error_message() and no launch;
  *   - err_word (device int32, caller-owned, zeroed by the caller before first use)
  *     receives the device-side status bits that the workspace's error word would get;
- *   - the first call on a device (the current device) looks the array up and zeroes its
- *     tickets with a synchronous cudaMemset, so it belongs before any stream capture
- *     begins. Later calls issue one kernel launch and nothing else.
- *   - the array is shared by every call on a device: two calls that may overlap (other
- *     streams, other host threads) race on it and give wrong tokens; order them.
+ *   - the first call on a device (the current device) looks the array's device address
+ *     up (cudaGetSymbolAddress), so it belongs before any stream capture begins. Every
+ *     call then clears the tickets of its num_requests requests with a cudaMemsetAsync on
+ *     `stream` and launches one kernel on it;
+ *   - the array is shared by every call on a device and keeps the last call's contents:
+ *     two calls that may overlap on the GPU (other streams, other host threads) race on
+ *     it and give wrong tokens; order them.
  * The library calls no allocation routine on this path. */
 #define S3R_NOALLOC_MAX_REQUESTS 2048
 #define S3R_NOALLOC_MAX_VOCAB 262144
@@ -236,11 +244,16 @@ S3R_API int s3r_draft_sample_noalloc(const s3r_batch* batch, const int32_t* draf
  * first rejection the token is drawn from max(0, p_j - q_j) normalised (from p_j if that is
  * all zero) with u2 from counter (L+j+1, r, 2, 0); if all k pass, from p_k with
  * counter (L+k+1, r, 2, 0).  out_tokens int32 [num_requests][k+1] receives the a accepted
- * drafts and the drawn token (entries after them untouched); n_out[r] = a + 1. */
+ * drafts and the drawn token (entries after them untouched); n_out[r] = a + 1.
+ * margins (fp32 [num_requests][k+1], may be NULL) receives the decisions' distances to
+ * their boundaries, in decision order: |u1 - p_j(d)/q_j(d)| for each decided draft (the a
+ * accepted ones and the rejected one, if any), then the draw's distance to the nearer edge
+ * of the drawn token's cell (as for s3r_draft_sample); min(a + 1, k) + 1 entries are
+ * written, the rest untouched. */
 S3R_API int s3r_spec_sample(const s3r_batch* batch, int32_t k, const float* p_logits,
                     const float* q_logits, const int32_t* draft_tokens, int32_t vocab,
-                    uint64_t seed, int32_t* out_tokens, int32_t* n_out, void* ws,
-                    size_t ws_bytes, s3r_stream_t stream);
+                    uint64_t seed, int32_t* out_tokens, int32_t* n_out, float* margins,
+                    void* ws, size_t ws_bytes, s3r_stream_t stream);
 
 /* Greedy (temperature 0) mode ([Listing] Table 4 setting: component measurements decode
  * greedily). s3r_draft_argmax: draft_tokens[r][i] = argmax of q_logits[r][i], i =
@@ -358,6 +371,14 @@ S3R_API uint64_t s3r_launch_count(void);
  * requests, otherwise the mma.sync kernel), 1 = always the mma.sync kernel. Both compute
  * the same function. */
 S3R_API int s3r_set_verify_kernel(int32_t which);
+
+/* Bound, in polls, on every wait of the tcgen05 verify kernel's roles for one another's
+ * progress (process-wide, for later calls; 0 restores the default of 2^24 polls). A wait
+ * that runs out sets S3R_ERR_TIMEOUT in the error word and the kernel winds down: each role
+ * still waits, without this bound, for its own copies and tensor-core work in flight,
+ * frees its tensor memory and returns, so the context stays usable. A diagnostic knob: a
+ * small bound makes a correct launch time out on purpose. S3R_ERR_INVALID_ARG if polls < 0. */
+S3R_API int s3r_set_wait_limit(int32_t polls);
 
 /* Text of the CUDA error behind the last S3R_ERR_CUDA status returned on this thread
  * ("" if none). */

@@ -30,6 +30,7 @@ from ._lib import (  # noqa: F401
     s3r_select_pages_from_scores,
     s3r_select_kv,
     s3r_set_verify_kernel,
+    s3r_set_wait_limit,
     s3r_sparse_draft_attn,
     s3r_spec_sample,
     s3r_status_string,

@@ -77,9 +77,9 @@ def _load():
         "s3r_select_kv_pages": (ctypes.c_int, [C, B, P, P, I32, I32, I32, P, I32, P, P, SZ, P]),
         "s3r_select_pages_from_scores": (ctypes.c_int, [C, B, P, I32, I32, I32, P, I32, P, P, SZ, P]),
         "s3r_sparse_draft_attn": (ctypes.c_int, [C, B, P, P, I32, P, P, I32, P, I32, P, P, P, P, SZ, P]),
-        "s3r_draft_sample": (ctypes.c_int, [B, P, I32, P, I32, U64, P, P, SZ, P]),
+        "s3r_draft_sample": (ctypes.c_int, [B, P, I32, P, I32, U64, P, P, P, SZ, P]),
         "s3r_draft_sample_noalloc": (ctypes.c_int, [B, P, I32, P, I32, U64, P, P, P]),
-        "s3r_spec_sample": (ctypes.c_int, [B, I32, P, P, P, I32, U64, P, P, P, SZ, P]),
+        "s3r_spec_sample": (ctypes.c_int, [B, I32, P, P, P, I32, U64, P, P, P, P, SZ, P]),
         "s3r_draft_argmax": (ctypes.c_int, [B, P, I32, P, I32, P, P, SZ, P]),
         "s3r_sched_simulate": (ctypes.c_int, [ctypes.POINTER(SchedConfig), I32, P, P, P, ctypes.c_int64,
                                               P, ctypes.c_int64, ctypes.POINTER(SchedResult), P,
@@ -94,6 +94,7 @@ def _load():
         "s3r_launch_count": (U64, []),
         "s3r_last_error_message": (ctypes.c_char_p, []),
         "s3r_set_verify_kernel": (ctypes.c_int, [I32]),
+        "s3r_set_wait_limit": (ctypes.c_int, [I32]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -265,12 +266,15 @@ def s3r_sparse_draft_attn(cache, batch, draft_step, q, k_new, v_new, sel_idx, se
         _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)), "s3r_sparse_draft_attn")
 
 
-def s3r_draft_sample(batch, draft_step, k, q_logits, vocab, seed, draft_tokens, ws, stream=None):
+def s3r_draft_sample(batch, draft_step, k, q_logits, vocab, seed, draft_tokens, ws, stream=None,
+                     margins=None):
+    """margins: optional fp32 [NR][k] tensor receiving each draw's boundary margin."""
     _check(_lib.s3r_draft_sample(
         ctypes.byref(batch), _ptr(draft_step, torch.int32, "draft_step"), k,
         _ptr(q_logits, torch.float32, "q_logits"), vocab, seed,
-        _ptr(draft_tokens, torch.int32, "draft_tokens"), _ptr(ws, torch.uint8, "ws"), ws.numel(),
-        _stream(stream)), "s3r_draft_sample")
+        _ptr(draft_tokens, torch.int32, "draft_tokens"),
+        _ptr(margins, torch.float32, "margins", allow_none=True), _ptr(ws, torch.uint8, "ws"),
+        ws.numel(), _stream(stream)), "s3r_draft_sample")
 
 
 def s3r_draft_sample_noalloc(batch, draft_step, k, q_logits, vocab, seed, draft_tokens, err_word,
@@ -288,13 +292,15 @@ def s3r_draft_sample_noalloc(batch, draft_step, k, q_logits, vocab, seed, draft_
 
 
 def s3r_spec_sample(batch, k, p_logits, q_logits, draft_tokens, vocab, seed, out_tokens, n_out,
-                    ws, stream=None):
+                    ws, stream=None, margins=None):
+    """margins: optional fp32 [NR][k+1] tensor receiving the decisions' boundary margins."""
     f32, i32 = torch.float32, torch.int32
     _check(_lib.s3r_spec_sample(
         ctypes.byref(batch), k, _ptr(p_logits, f32, "p_logits"),
         _ptr(q_logits, f32, "q_logits", allow_none=(k == 0)),
         _ptr(draft_tokens, i32, "draft_tokens", allow_none=(k == 0)), vocab, seed,
         _ptr(out_tokens, i32, "out_tokens"), _ptr(n_out, i32, "n_out"),
+        _ptr(margins, f32, "margins", allow_none=True),
         _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)), "s3r_spec_sample")
 
 
@@ -386,6 +392,11 @@ def s3r_status_string(status: int) -> str:
 def s3r_set_verify_kernel(which: int):
     """0: automatic (tcgen05 kernel where supported), 1: mma.sync kernel."""
     _check(_lib.s3r_set_verify_kernel(which), "s3r_set_verify_kernel")
+
+
+def s3r_set_wait_limit(polls: int):
+    """Bound on the tcgen05 verify's waits of one role for another (0: the default)."""
+    _check(_lib.s3r_set_wait_limit(polls), "s3r_set_wait_limit")
 
 
 def s3r_launch_count() -> int:

@@ -3,6 +3,7 @@
 // launch), warp reductions, Philox4x32-10 and the workspace layout.
 #pragma once
 
+#include <atomic>
 #include <utility>
 
 #include <cuda.h>
@@ -19,7 +20,7 @@ constexpr int kTile = 64;                 // KV positions per pipeline stage
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr unsigned kFull = 0xffffffffu;
-constexpr int kWaitLimit = 1 << 24;       // bounded spin on an mbarrier phase
+constexpr int kWaitLimit = 1 << 24;       // bounded spin on an mbarrier phase (default)
 
 // ---------------------------------------------------------------- workspace layout ----
 // [0, 256)      error word (int32 bitmask of 1 << s3r_status) at 0; at 64 the dense verify's
@@ -141,11 +142,13 @@ __device__ __forceinline__ void fence_proxy_async() {
 }
 
 // Warp-uniform bounded wait on an mbarrier phase (every lane observes the phase itself).
-// Gives up when another role raised the abort flag, or after kWaitLimit polls (then raises
-// it, with S3R_ERR_TIMEOUT in the error word).
+// Gives up when another role raised the abort flag, or after `limit` polls (then raises
+// it, with S3R_ERR_TIMEOUT in the error word). For waits on another role's progress; a
+// wait for this thread's own copies or tensor-core work in flight uses mbar_wait, which
+// no abort cuts short.
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                         int* err) {
-  for (int i = 0; i < kWaitLimit; ++i) {
+                                         int* err, int limit = kWaitLimit) {
+  for (int i = 0; i < limit; ++i) {
     const bool done = mbar_try_wait(bar, parity);
     if (__all_sync(kFull, done)) return true;
     if ((i & 255) == 255 && __any_sync(kFull, *abort_flag != 0)) return false;
@@ -185,6 +188,22 @@ inline void launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   (void)cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);   // errors: cudaGetLastError
+}
+
+// Raise `kern`'s dynamic shared-memory limit to `bytes` on the current device, once per
+// device: the attribute belongs to the device, so a process that drives several GPUs sets
+// it on each. `done` is the caller's record (bit d: device d done; devices >= 64 set it on
+// every call). Returns the CUDA error of the attribute call.
+template <typename... KArgs>
+inline cudaError_t ensure_smem_attr(void (*kern)(KArgs...), int bytes, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = dev < 64 ? (uint64_t)1 << dev : 0;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_release);
+  return e;
 }
 
 // Untiled bulk copy global -> shared of `bytes` (both addresses 16-byte aligned, bytes a

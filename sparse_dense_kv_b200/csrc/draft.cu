@@ -182,14 +182,9 @@ __global__ void __launch_bounds__(128) draft_kernel(const DraftParams p) {
 template <int D>
 static int launch_draft_d(const DraftParams& p, int batch, cudaStream_t stream) {
   const size_t smem = 1024 + kDraftStages * 2 * kTile * D * 2 + kDraftChunk * 8 + 64;
-  static bool attr_done = false;
-  if (!attr_done) {
-    if (cuda_status(cudaFuncSetAttribute(draft_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem), "cudaFuncSetAttribute") != S3R_OK)
-
-      return S3R_ERR_CUDA;
-    attr_done = true;
-  }
+  static std::atomic<uint64_t> attr_done{0};
+  if (cuda_status(ensure_smem_attr(draft_kernel<D>, (int)smem, attr_done), "cudaFuncSetAttribute") != S3R_OK)
+    return S3R_ERR_CUDA;
   dim3 grid(p.nchunk_max, p.Hkv, batch);
   launch_pdl(draft_kernel<D>, grid, 128, smem, stream, p);
   return cuda_status(cudaGetLastError(), __func__);

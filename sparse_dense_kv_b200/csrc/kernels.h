@@ -36,6 +36,7 @@ struct VerifyParams {
   float* part;
   int req_off;             // launch covers requests req_ids[req_off + b] (or req_off + b)
   int* sched;              // [2] work counter, exited CTAs (zero between launches)
+  int wait_limit;          // polls before a wait on another role's progress gives up
 };
 
 struct DraftParams {
@@ -101,6 +102,8 @@ struct SampleParams {
   int* tickets;
   uint8_t* part;
   size_t plan_off, draw_off;   // spec sampling: byte offsets of the plans / draw partials
+  int num_requests;            // size of every per-request array (request ids are checked)
+  float* margins;              // optional: draft [NR][k], spec [NR][k+1] decision margins
 };
 
 // Record the CUDA error behind an S3R_ERR_CUDA status (readable by s3r_last_error_message)

@@ -27,6 +27,7 @@ namespace {
 
 std::atomic<uint64_t> g_launches{0};
 std::atomic<int> g_verify_kernel{0};   // 0 auto, 1 CUDA-core mma.sync kernel
+std::atomic<int> g_wait_limit{kWaitLimit};   // polls of the verify roles' waits on each other
 
 int sm_count() {
   int dev = 0, n = 0;
@@ -234,8 +235,8 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
 namespace {
 
 // Device address of the scratch on the current device. The first call on a device looks
-// the symbol up and zeroes its tickets (a synchronous cudaMemset, no allocation); later
-// calls only read the cached address.
+// the symbol up (cudaGetSymbolAddress, no allocation); later calls only read the cached
+// address.
 int noalloc_scratch(unsigned char** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return cuda_status(cudaGetLastError(), "cudaGetDevice");
@@ -246,8 +247,6 @@ int noalloc_scratch(unsigned char** out) {
     const int st = cuda_status(cudaGetSymbolAddress(&p, g_noalloc_scratch), "cudaGetSymbolAddress");
     if (st != S3R_OK) return st;
     if ((reinterpret_cast<uintptr_t>(p) & 255u) != 0) return S3R_ERR_WORKSPACE;
-    const int zs = cuda_status(cudaMemset(p, 0, kNoAllocTicketBytes), "cudaMemset");
-    if (zs != S3R_OK) return zs;
     g_noalloc_ptr[dev] = p;
   }
   *out = static_cast<unsigned char*>(g_noalloc_ptr[dev]);
@@ -338,6 +337,7 @@ int s3r_verify_attn(const s3r_kv_cache* cache, const s3r_batch* batch, int32_t k
   p.tickets = w.tickets;
   p.sched = w.sched;
   p.part = reinterpret_cast<float*>(w.part);
+  p.wait_limit = g_wait_limit.load();
   int st;
   const bool tc = g_verify_kernel.load() == 0 && verify_tc_supported(cache->head_dim, R, batch->batch);
   {
@@ -527,12 +527,12 @@ int s3r_sparse_draft_attn(const s3r_kv_cache* cache, const s3r_batch* batch,
 
 int s3r_draft_sample(const s3r_batch* batch, const int32_t* draft_step, int32_t k,
                      const float* q_logits, int32_t vocab, uint64_t seed, int32_t* draft_tokens,
-                     void* ws, size_t ws_bytes, s3r_stream_t stream) {
+                     float* margins, void* ws, size_t ws_bytes, s3r_stream_t stream) {
   S3R_TRY(check_batch(batch, false));
   if (k < 1 || k > S3R_MAX_K) return S3R_ERR_UNSUPPORTED;
   if (vocab < 1 || vocab > 64 * kVocabChunk) return S3R_ERR_UNSUPPORTED;
   if (!draft_step || !q_logits || !draft_tokens || !aligned4(draft_step) ||
-      !aligned4(q_logits) || !aligned4(draft_tokens))
+      !aligned4(q_logits) || !aligned4(draft_tokens) || (margins && !aligned4(margins)))
     return S3R_ERR_INVALID_ARG;
   if (batch->batch == 0) return S3R_OK;
   S3R_TRY(check_ws(ws, ws_bytes, sample_need(batch->num_requests, 1, k, vocab)));
@@ -551,6 +551,8 @@ int s3r_draft_sample(const s3r_batch* batch, const int32_t* draft_step, int32_t 
   p.err = w.err;
   p.tickets = w.tickets;
   p.part = w.part;
+  p.num_requests = batch->num_requests;
+  p.margins = margins;
   return finish(launch_draft_sample(p, batch->batch, (cudaStream_t)stream), 1);
 }
 
@@ -588,18 +590,23 @@ int s3r_draft_sample_noalloc(const s3r_batch* batch, const int32_t* draft_step, 
   p.err = err_word;
   p.tickets = reinterpret_cast<int*>(scratch);
   p.part = scratch + kNoAllocTicketBytes;
+  p.num_requests = batch->num_requests;
+  // the tickets of this call's requests start at zero whatever an earlier call left there,
+  // cleared on the call's own stream (so ordered with the launch below)
+  S3R_TRY(cuda_status(cudaMemsetAsync(scratch, 0, (size_t)batch->num_requests * sizeof(int),
+                                      (cudaStream_t)stream), "cudaMemsetAsync"));
   return finish(launch_draft_sample(p, batch->batch, (cudaStream_t)stream), 1);
 }
 
 int s3r_spec_sample(const s3r_batch* batch, int32_t k, const float* p_logits,
                     const float* q_logits, const int32_t* draft_tokens, int32_t vocab,
-                    uint64_t seed, int32_t* out_tokens, int32_t* n_out, void* ws,
-                    size_t ws_bytes, s3r_stream_t stream) {
+                    uint64_t seed, int32_t* out_tokens, int32_t* n_out, float* margins,
+                    void* ws, size_t ws_bytes, s3r_stream_t stream) {
   S3R_TRY(check_batch(batch, false));
   if (k < 0 || k > S3R_MAX_K) return S3R_ERR_UNSUPPORTED;
   if (vocab < 1 || vocab > 64 * kVocabChunk) return S3R_ERR_UNSUPPORTED;
   if (!p_logits || !out_tokens || !n_out || !aligned4(p_logits) || !aligned4(out_tokens) ||
-      !aligned4(n_out))
+      !aligned4(n_out) || (margins && !aligned4(margins)))
     return S3R_ERR_INVALID_ARG;
   if (k > 0 && (!q_logits || !draft_tokens || !aligned4(q_logits) || !aligned4(draft_tokens)))
     return S3R_ERR_INVALID_ARG;
@@ -622,6 +629,8 @@ int s3r_spec_sample(const s3r_batch* batch, int32_t k, const float* p_logits,
   p.err = w.err;
   p.tickets = w.tickets;
   p.part = w.part;
+  p.num_requests = batch->num_requests;
+  p.margins = margins;
   spec_offsets(batch->num_requests, k, vocab, &p.plan_off, &p.draw_off);
   int launches = 0;
   const int st = launch_spec_sample(p, batch->batch, (cudaStream_t)stream, &launches);
@@ -655,6 +664,7 @@ int s3r_draft_argmax(const s3r_batch* batch, const int32_t* draft_step, int32_t 
   p.err = w.err;
   p.tickets = w.tickets;
   p.part = w.part;
+  p.num_requests = batch->num_requests;
   return finish(launch_argmax(p, batch->batch, 0, (cudaStream_t)stream), 1);
 }
 
@@ -685,6 +695,7 @@ int s3r_greedy_verify(const s3r_batch* batch, int32_t k, const float* p_logits,
   p.err = w.err;
   p.tickets = w.tickets;
   p.part = w.part;
+  p.num_requests = batch->num_requests;
   return finish(launch_argmax(p, batch->batch, 1, (cudaStream_t)stream), 1);
 }
 
@@ -773,6 +784,12 @@ const char* s3r_last_error_message(void) { return g_last_error; }
 int s3r_set_verify_kernel(int32_t which) {
   if (which < 0 || which > 1) return S3R_ERR_INVALID_ARG;
   g_verify_kernel.store(which);
+  return S3R_OK;
+}
+
+int s3r_set_wait_limit(int32_t polls) {
+  if (polls < 0) return S3R_ERR_INVALID_ARG;
+  g_wait_limit.store(polls == 0 ? kWaitLimit : polls);
   return S3R_OK;
 }
 

@@ -150,10 +150,13 @@ __device__ double block_sum_d(double v) {
 // reduces its 32 rows of 32 entries with a butterfly (lane m ends with row m's sum),
 // scans the rows, then the lanes of the chosen row. Returns -1 if the target lies past the
 // chunk; `base` then moves to the chunk's end.
+// `mrg` receives the distance of the target to the nearer edge of the drawn token's cell
+// [C_{v-1}, C_v) (0 where rounding carried the target past the last entry).
 template <class W>
-__device__ int chunk_search(int v0, int v1, double target, double& base, W weight) {
+__device__ int chunk_search(int v0, int v1, double target, double& base, double& mrg, W weight) {
   __shared__ double wtot_s[kSampThreads / 32];
   __shared__ int s_tok;
+  __shared__ double s_mrg;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int wb = v0 + warp * 1024;
   float w[32];
@@ -166,7 +169,10 @@ __device__ int chunk_search(int v0, int v1, double target, double& base, W weigh
   }
   const double wt = warp_sum_d((double)part);
   if (lane == 0) wtot_s[warp] = wt;
-  if (threadIdx.x == 0) s_tok = -1;
+  if (threadIdx.x == 0) {
+    s_tok = -1;
+    s_mrg = 0.0;
+  }
   __syncthreads();
   double lo = base, total = 0.0;
   for (int q = 0; q < kSampThreads / 32; ++q) {
@@ -195,6 +201,7 @@ __device__ int chunk_search(int v0, int v1, double target, double& base, W weigh
     // row: the first with target < lo + (rows up to and including it)
     const unsigned rowhit = __ballot_sync(kFull, rs > 0.0 && target < lo + incl);
     int tok = -1;
+    double m = 0.0;
     if (rowhit) {
       const int mr = __ffs(rowhit) - 1;
       const double rbase = lo + __shfl_sync(kFull, incl - rs, mr);
@@ -211,6 +218,9 @@ __device__ int chunk_search(int v0, int v1, double target, double& base, W weigh
       const unsigned nz = __ballot_sync(kFull, x > 0.f);
       const int ln = hit ? __ffs(hit) - 1 : 31 - __clz((int)nz);
       tok = wb + 32 * mr + ln;
+      const double hi_e = rbase + li, lo_e = hi_e - (double)x;   // the lane's cell
+      const double mine = fmin(target - lo_e, hi_e - target);
+      m = hit ? __shfl_sync(kFull, mine, ln) : 0.0;
     } else {
       // rounding past the warp's last row: the last non-zero entry of the warp
       const unsigned nzr = __ballot_sync(kFull, rs > 0.0);
@@ -220,10 +230,14 @@ __device__ int chunk_search(int v0, int v1, double target, double& base, W weigh
       const unsigned nz = __ballot_sync(kFull, x > 0.f);
       tok = wb + 32 * mr + (31 - __clz((int)nz));
     }
-    if (lane == 0) s_tok = tok;
+    if (lane == 0) {
+      s_tok = tok;
+      s_mrg = m;
+    }
   }
   __syncthreads();
   const int tok = s_tok;
+  if (tok >= 0) mrg = s_mrg;
   base += total;
   __syncthreads();
   return tok;
@@ -249,8 +263,8 @@ __device__ int last_nonzero(int V, W weight) {
 // the search reads them there through sweight(v, c0); if rounding carries the target past
 // the last chunk, the last token of nonzero weight (gweight reads global memory) is taken.
 template <class Stage, class SW, class GW>
-__device__ int draw_staged(int V, int nvch, const double* csum, double target, Stage stage,
-                           SW sweight, GW gweight) {
+__device__ int draw_staged(int V, int nvch, const double* csum, double target, double& mrg,
+                           Stage stage, SW sweight, GW gweight) {
   __shared__ int s_c;
   __shared__ double s_base;
   if (threadIdx.x == 0) {
@@ -269,11 +283,12 @@ __device__ int draw_staged(int V, int nvch, const double* csum, double target, S
   __syncthreads();
   double base = s_base;
   int tok = -1;
+  mrg = 0.0;
   for (int c = s_c; c < nvch && tok < 0; ++c) {
     const int c0 = c * kVocabChunk, cn = min(V - c0, kVocabChunk);
     __syncthreads();   // every thread is done with the shared buffers
     stage(c0, cn);
-    tok = chunk_search(c0, c0 + cn, target, base, [&](int v) -> float { return sweight(v, c0); });
+    tok = chunk_search(c0, c0 + cn, target, base, mrg, [&](int v) -> float { return sweight(v, c0); });
   }
   return tok >= 0 ? tok : last_nonzero(V, gweight);
 }
@@ -322,6 +337,10 @@ __global__ void __launch_bounds__(kSampThreads) draft_sample_kernel(const Sample
   __shared__ float s_M;
   const int cb = blockIdx.y, bl = blockIdx.x;
   const int r = p.req_ids ? p.req_ids[bl] : bl;
+  if (r < 0 || r >= p.num_requests) {   // every CTA of the row returns: no ticket is touched
+    if (cb == 0 && threadIdx.x == 0) set_error(p.err, S3R_ERR_DEVICE_BOUNDS);
+    return;
+  }
   const int i = p.draft_step[r];
   const int V = p.vocab;
   if (i < 0 || i >= p.k) {
@@ -392,10 +411,14 @@ __global__ void __launch_bounds__(kSampThreads) draft_sample_kernel(const Sample
     }
   };
   auto wq = [&](float x) -> float { return (isnan(x) || x == INFINITY) ? 0.f : ex2(fmaf(x, kLog2e, -Mb)); };
+  double mrg;
   const int tok = draw_staged(
-      V, p.nvch, csum, u * Z, stage, [&](int v, int c0) { return wq(xs[v - c0]); },
+      V, p.nvch, csum, u * Z, mrg, stage, [&](int v, int c0) { return wq(xs[v - c0]); },
       [&](int v) { return wq(row[v]); });
-  if (threadIdx.x == 0) p.draft_out[(size_t)r * p.k + i] = tok;
+  if (threadIdx.x == 0) {
+    p.draft_out[(size_t)r * p.k + i] = tok;
+    if (p.margins) p.margins[(size_t)r * p.k + i] = Z > 0.0 ? (float)(mrg / Z) : 0.f;
+  }
 }
 
 // ------------------------------------------------------- speculative sampling: pass 1 --
@@ -406,6 +429,10 @@ __global__ void __launch_bounds__(kSampThreads) spec_norm_kernel(const SamplePar
   __shared__ double sZ[2 * S3R_MAX_K + 1];
   const int bl = blockIdx.x, rw = blockIdx.y, c = blockIdx.z;
   const int r = p.req_ids ? p.req_ids[bl] : bl;
+  if (r < 0 || r >= p.num_requests) {   // every CTA of the request returns
+    if (rw == 0 && c == 0 && threadIdx.x == 0) set_error(p.err, S3R_ERR_DEVICE_BOUNDS);
+    return;
+  }
   const int k = p.k, V = p.vocab, nrows = 2 * k + 1;
   const float* row = (rw <= k) ? p.p_logits + ((size_t)r * (k + 1) + rw) * V
                                : p.q_logits + ((size_t)r * k + (rw - k - 1)) * V;
@@ -442,6 +469,7 @@ __global__ void __launch_bounds__(kSampThreads) spec_norm_kernel(const SamplePar
   const size_t pbase = (size_t)r * (k + 1) * V, qbase = (size_t)r * k * V;
   bool acc = false;
   int d = -1;
+  double margin = 0.0;   // |u - p/q| of this lane's draft
   if (lane < k) {
     d = p.draft_tokens[(size_t)r * k + lane];
     if (d < 0 || d >= V) {
@@ -452,11 +480,14 @@ __global__ void __launch_bounds__(kSampThreads) spec_norm_kernel(const SamplePar
                         sZ[k + 1 + lane];
       const double u = philox_u(p.seed, (uint32_t)(L + lane + 1), (uint32_t)r, 1u);
       acc = u * qj < pj;
+      margin = qj > 0.0 ? fabs(u - pj / qj) : INFINITY;
     }
   }
   const unsigned rej = ~__ballot_sync(kFull, acc) & ((1u << k) - 1u);
   const int a = rej ? __ffs(rej) - 1 : k;      // drafts accepted before the first rejection
   if (lane < a) p.out_tokens[(size_t)r * (k + 1) + lane] = d;
+  // the decided drafts' margins: the accepted ones and the first rejected one
+  if (p.margins && lane < k && lane <= a) p.margins[(size_t)r * (k + 1) + lane] = (float)margin;
   if (lane != 0) return;
   const int type = a < k ? 0 : 1, jrow = a;
   SpecPlan* plan = reinterpret_cast<SpecPlan*>(p.part + p.plan_off) + r;
@@ -485,6 +516,7 @@ __global__ void __launch_bounds__(kSampThreads) spec_draw_kernel(const SamplePar
   __shared__ int s_use_res;
   const int c = blockIdx.y, bl = blockIdx.x;
   const int r = p.req_ids ? p.req_ids[bl] : bl;
+  if (r < 0 || r >= p.num_requests) return;   // reported by the first pass
   const int k = p.k, V = p.vocab;
   const SpecPlan pl = reinterpret_cast<const SpecPlan*>(p.part + p.plan_off)[r];
   const float* prow = p.p_logits + ((size_t)r * (k + 1) + pl.row) * V;
@@ -598,13 +630,18 @@ __global__ void __launch_bounds__(kSampThreads) spec_draw_kernel(const SamplePar
     __syncthreads();
   };
   int tok;
+  double mrg;
   if (use_res)
-    tok = draw_staged(V, p.nvch, csum, target, stage,
+    tok = draw_staged(V, p.nvch, csum, target, mrg, stage,
                       [&](int v, int c0) { return wres_xy(xps[v - c0], xqs[v - c0]); }, w_res);
   else
-    tok = draw_staged(V, p.nvch, csum, target, stage,
+    tok = draw_staged(V, p.nvch, csum, target, mrg, stage,
                       [&](int v, int c0) { return wp_x(xps[v - c0]); }, w_p);
-  if (threadIdx.x == 0) p.out_tokens[(size_t)r * (k + 1) + pl.a] = tok;
+  if (threadIdx.x == 0) {
+    p.out_tokens[(size_t)r * (k + 1) + pl.a] = tok;
+    // the draw's margin follows the decided drafts' margins
+    if (p.margins) p.margins[(size_t)r * (k + 1) + (pl.a < k ? pl.a + 1 : k)] = Z > 0.0 ? (float)(mrg / Z) : 0.f;
+  }
 }
 
 // ------------------------------------------------------------ greedy (temperature 0) ----
@@ -641,6 +678,10 @@ __global__ void __launch_bounds__(kSampThreads) argmax_kernel(const SampleParams
   const int bl = blockIdx.x, j = blockIdx.y, c = blockIdx.z;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int r = p.req_ids ? p.req_ids[bl] : bl;
+  if (r < 0 || r >= p.num_requests) {   // every CTA of the request returns
+    if (j == 0 && c == 0 && threadIdx.x == 0) set_error(p.err, S3R_ERR_DEVICE_BOUNDS);
+    return;
+  }
   const int k = p.k, V = p.vocab;
   const int nrows = mode == 0 ? 1 : k + 1;
   const float* row;
@@ -758,13 +799,9 @@ __global__ void philox_kernel(uint64_t seed, int stream_id, const int32_t* reque
 // ------------------------------------------------------------------------ launchers ----
 int launch_draft_sample(const SampleParams& p, int batch, cudaStream_t stream) {
   constexpr int smem = kDsSpan * 4;
-  static bool attr_done = false;
-  if (!attr_done) {
-    if (cuda_status(cudaFuncSetAttribute(draft_sample_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         smem), "cudaFuncSetAttribute") != S3R_OK)
-      return S3R_ERR_CUDA;
-    attr_done = true;
-  }
+  static std::atomic<uint64_t> attr_done{0};
+  if (cuda_status(ensure_smem_attr(draft_sample_kernel, smem, attr_done), "cudaFuncSetAttribute") != S3R_OK)
+    return S3R_ERR_CUDA;
   dim3 grid(batch, (p.vocab + kDsSpan - 1) / kDsSpan);
   launch_pdl(draft_sample_kernel, grid, kSampThreads, smem, stream, p);
   return cuda_status(cudaGetLastError(), __func__);
@@ -775,13 +812,9 @@ int launch_spec_sample(const SampleParams& p, int batch, cudaStream_t stream, in
   launch_pdl(spec_norm_kernel, g1, kSampThreads, 0, stream, p);
   if (cuda_status(cudaGetLastError(), __func__) != S3R_OK) return S3R_ERR_CUDA;
   constexpr int smem2 = 2 * kVocabChunk * 4;
-  static bool attr_done = false;
-  if (!attr_done) {
-    if (cuda_status(cudaFuncSetAttribute(spec_draw_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         smem2), "cudaFuncSetAttribute") != S3R_OK)
-      return S3R_ERR_CUDA;
-    attr_done = true;
-  }
+  static std::atomic<uint64_t> attr_done{0};
+  if (cuda_status(ensure_smem_attr(spec_draw_kernel, smem2, attr_done), "cudaFuncSetAttribute") != S3R_OK)
+    return S3R_ERR_CUDA;
   dim3 g2(batch, p.nvch);
   launch_pdl(spec_draw_kernel, g2, kSampThreads, smem2, stream, p);
   *launches = 2;

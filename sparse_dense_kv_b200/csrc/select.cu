@@ -334,16 +334,11 @@ int launch_select(const SelectParams& p, int batch, cudaStream_t stream, int* la
   const int lim = q.score_stride;
   const int nmax = lim < kSelectMaxN ? lim : kSelectMaxN;
   const size_t smem = (size_t)(nmax > 0 ? nmax : 1) * 4;
-  static bool attr_done = false;
-  if (!attr_done) {
-    if (cuda_status(cudaFuncSetAttribute(select_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kSelectMaxN * 4), "cudaFuncSetAttribute") != S3R_OK ||
-        cuda_status(cudaFuncSetAttribute(select_kernel<S3R_PAGE_SIZE>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSelectMaxN * 4),
-                    "cudaFuncSetAttribute") != S3R_OK)
-      return S3R_ERR_CUDA;
-    attr_done = true;
-  }
+  static std::atomic<uint64_t> attr_tok{0}, attr_page{0};
+  if (cuda_status(ensure_smem_attr(select_kernel<1>, kSelectMaxN * 4, attr_tok), "cudaFuncSetAttribute") != S3R_OK ||
+      cuda_status(ensure_smem_attr(select_kernel<S3R_PAGE_SIZE>, kSelectMaxN * 4, attr_page),
+                  "cudaFuncSetAttribute") != S3R_OK)
+    return S3R_ERR_CUDA;
   dim3 grid(q.Hkv, batch);
   if (p.page == S3R_PAGE_SIZE)
     launch_pdl(select_kernel<S3R_PAGE_SIZE>, grid, kSelectThreads, smem, stream, q);

@@ -321,14 +321,11 @@ int launch_verify_combine(const VerifyParams& p, int D, int batch, cudaStream_t 
   if (!verify_combine_fits(p.nchunk_max, p.R)) return S3R_ERR_UNSUPPORTED;
   dim3 grid((p.R + kCombRows - 1) / kCombRows, p.Hkv, batch);
   auto kern = D == 128 ? verify_combine_kernel<128> : verify_combine_kernel<64>;
-  static size_t attr[2] = {0, 0};
-  size_t& a = attr[D == 128 ? 0 : 1];
-  if (smem > 48 * 1024 && smem > a) {
-    if (cuda_status(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem),
-                    "cudaFuncSetAttribute") != S3R_OK)
-      return S3R_ERR_CUDA;
-    a = smem;
-  }
+  // the limit is raised once per device to the largest merge that verify_combine_fits admits
+  static std::atomic<uint64_t> attr_done[2];
+  if (smem > 48 * 1024 &&
+      cuda_status(ensure_smem_attr(kern, 200 * 1024, attr_done[D == 128 ? 0 : 1]), "cudaFuncSetAttribute") != S3R_OK)
+    return S3R_ERR_CUDA;
   launch_pdl(kern, grid, kCombThreads, smem, stream, p);
   return cuda_status(cudaGetLastError(), __func__);
 }
@@ -341,14 +338,13 @@ static int launch_verify_t(const CUtensorMap& tk, const CUtensorMap& tv, const V
   const size_t smem = 1024 + kVerifyStages * verify_stage_bytes<D>() + 64;
   const size_t red = (size_t)(threads / 32) * 16 * (D + 4 + 2) * 4;
   const size_t need = smem > red + 1024 + 64 ? smem : red + 1024 + 64;
-  static size_t attr_bytes = 0;
-  if (need > attr_bytes) {
-    if (cuda_status(cudaFuncSetAttribute(verify_kernel<D, MAXT>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)need),
-                    "cudaFuncSetAttribute") != S3R_OK)
-      return S3R_ERR_CUDA;
-    attr_bytes = need;
-  }
+  // raised once per device to what the largest row count (S3R_MAX_ROWS: 4 row groups) needs
+  const size_t red_max = (size_t)(128 * ((S3R_MAX_ROWS + 15) / 16) / 32) * 16 * (D + 4 + 2) * 4;
+  const size_t need_max = smem > red_max + 1024 + 64 ? smem : red_max + 1024 + 64;
+  static std::atomic<uint64_t> attr_done{0};
+  if (cuda_status(ensure_smem_attr(verify_kernel<D, MAXT>, (int)need_max, attr_done), "cudaFuncSetAttribute") !=
+      S3R_OK)
+    return S3R_ERR_CUDA;
   dim3 grid(p.nchunk_max, p.Hkv, batch);
   launch_pdl(verify_kernel<D, MAXT>, grid, threads, need, stream, tk, tv, p);
   return cuda_status(cudaGetLastError(), __func__);

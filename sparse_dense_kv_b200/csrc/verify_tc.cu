@@ -344,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // CTAs on faster SMs take more chunks and all finish within about one chunk of each other.
   auto ring_id = [&](int m) -> int {   // warp-uniform; -1 if the wait gave up
     const int slot = m & (kRing - 1);
-    if (!wait_bar(smem_u32(&B->item_bar[slot]), (uint32_t)(m / kRing) & 1u, abort_flag, p.err)) return -1;
+    if (!wait_bar(smem_u32(&B->item_bar[slot]), (uint32_t)(m / kRing) & 1u, abort_flag, p.err, p.wait_limit)) return -1;
     return *reinterpret_cast<volatile int*>(&B->item_id[slot]);
   };
   const uint32_t qbuf = sbase + C::kQOff, pbuf = sbase + C::kPOff;
@@ -374,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto load_tiles = [&](const Item& x) {
       for (int t = 0; t < x.ntile && !stop; ++t, ++g) {
         const int s = g % nst;
-        if (g >= nst && !wait_bar(smem_u32(&empty[s]), ((g / nst) - 1) & 1, abort_flag, p.err)) {
+        if (g >= nst && !wait_bar(smem_u32(&empty[s]), ((g / nst) - 1) & 1, abort_flag, p.err, p.wait_limit)) {
           stop = true;
           break;
         }
@@ -415,7 +415,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (tail) {
           // wait for the committed rows, then write block rows / zeros over the rest
-          if (!wait_bar(smem_u32(&tmab[s]), (tma_phase >> s) & 1, abort_flag, p.err)) {
+          if (!wait_bar(smem_u32(&tmab[s]), (tma_phase >> s) & 1, abort_flag, p.err, p.wait_limit)) {
+            mbar_wait(smem_u32(&tmab[s]), (tma_phase >> s) & 1);   // its copies land before exit
             stop = true;
             break;
           }
@@ -475,6 +476,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       return id;
     };
     int next_a = -1, next_b = -1;
+    int q_issued = 0;   // Q loads issued (item m's load lands on q_full[m & 1], phase (m >> 1) & 1)
     int cur = item_id(0);
     for (int m = 0; cur >= 0 && cur < nitems && !stop && !aborted(abort_flag); ++m) {
       const int nxt = item_id(m + 1);
@@ -491,12 +493,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!is_v) {
         // Q rows -> Q buffer m&1 by TMA (K-major, 128-byte swizzle) once QK(m-2) has read it
         const int qb = m & 1;
-        if (m >= 2 && !wait_bar(smem_u32(&B->q_empty[qb]), ((m - 2) >> 1) & 1, abort_flag, p.err)) break;
+        if (m >= 2 && !wait_bar(smem_u32(&B->q_empty[qb]), ((m - 2) >> 1) & 1, abort_flag, p.err, p.wait_limit)) break;
         if (lane == 0) mbar_arrive_expect_tx(smem_u32(&B->q_full[qb]), (uint32_t)(2 * R * 128));
         __syncwarp();
         if (lane < 2)
           tma_load_3d(qbuf + qb * C::kQBytes + lane * (NP * 128), &tmQ, lane * 64, x.kvh * G,
                       x.r * T, smem_u32(&B->q_full[qb]));
+        q_issued = m + 1;
         __syncwarp();
       }
       load_tiles(x);
@@ -517,8 +520,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    // nothing may still be landing in this ring when the CTA exits
+    // nothing may still be landing in this ring (or a Q buffer) when the CTA exits, also after
+    // an abort: these waits are for this warp's own copies and are not cut short
     for (int q = g - nst > 0 ? g - nst : 0; q < g; ++q) mbar_wait(smem_u32(&full[q % nst]), (q / nst) & 1);
+    for (int m = q_issued - 2 > 0 ? q_issued - 2 : 0; m < q_issued; ++m)
+      mbar_wait(smem_u32(&B->q_full[m & 1]), (uint32_t)(m >> 1) & 1u);
   } else if (warp == 2) {
     // ====================================================================== MMA warp ===
     // Two queues in issue order: QK of item m (its K tiles) and PV of item n < m (its V
@@ -643,7 +649,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (did) {
         idle = 0;
-      } else if (++idle >= (uint32_t)kWaitLimit) {
+      } else if (++idle >= (uint32_t)p.wait_limit) {
         if (lane == 0) {
           *abort_flag = 1;
           set_error(p.err, S3R_ERR_TIMEOUT);
@@ -657,7 +663,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // make sure nothing issued is still running before the tensor memory goes away
     if (lane == 0) tc_commit(smem_u32(&B->fin));
     __syncwarp();
-    wait_bar(smem_u32(&B->fin), 0, abort_flag, p.err);
+    mbar_wait(smem_u32(&B->fin), 0);   // not cut short by an abort: the work is in flight
   } else {
     // ================================================================ softmax warps ===
     // Warpgroup sg owns rows (columns of S and O^T) [sg*NH, sg*NH + NH) of every tile; the
@@ -680,7 +686,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto wg_sync = [&]() -> bool {
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&B->wg[sg]));
-      const bool r = wait_bar(smem_u32(&B->wg[sg]), wg_phase, abort_flag, p.err);
+      const bool r = wait_bar(smem_u32(&B->wg[sg]), wg_phase, abort_flag, p.err, p.wait_limit);
       wg_phase ^= 1u;
       return r;
     };
@@ -688,7 +694,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // record of chunk m (this warpgroup's rows): O^T buffer m&1 -> workspace, with the rows'
     // max / sum from cm / cl
     auto epilogue = [&](int m, const Item& x) -> bool {
-      if (!wait_bar(smem_u32(&B->o_full[m & 1]), (m >> 1) & 1, abort_flag, p.err)) return false;
+      if (!wait_bar(smem_u32(&B->o_full[m & 1]), (m >> 1) & 1, abort_flag, p.err, p.wait_limit)) return false;
       tc_fence_after();
       const size_t rec_floats = (size_t)p.Rp * (kD + 2);
       float* rec = p.part + (((size_t)x.r * Hkv + x.kvh) * p.nchunk_max + x.c) * rec_floats;
@@ -720,7 +726,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Item x = make_item<NP>(id, pref, lens_s, rid_s, batch, p);
       const int L = x.L, start = x.start, end = x.end;
       float* scores = p.scores ? p.scores + ((size_t)x.r * Hkv + x.kvh) * (size_t)R * p.cap : nullptr;
-      if (!wait_bar(smem_u32(&B->s_full[n & 1]), (n >> 1) & 1, abort_flag, p.err)) {
+      if (!wait_bar(smem_u32(&B->s_full[n & 1]), (n >> 1) & 1, abort_flag, p.err, p.wait_limit)) {
         ok = false;
         break;
       }
@@ -821,7 +827,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             lsum[j + 1] += e1;
             pk[j / 2] = pack_bf16(e0, e1);
           }
-          if (n > 0 && !wait_bar(smem_u32(&B->p_free[t]), (n - 1) & 1, abort_flag, p.err)) {
+          if (n > 0 && !wait_bar(smem_u32(&B->p_free[t]), (n - 1) & 1, abort_flag, p.err, p.wait_limit)) {
             ok = false;
             break;
           }
@@ -896,14 +902,10 @@ static int launch_tc(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
                      const CUtensorMap& tk8, const CUtensorMap& tv8, const VerifyParams& p,
                      int batch, int num_sms, cudaStream_t stream) {
   using C = tc::Cfg<NP>;
-  static bool attr_done = false;
-  if (!attr_done) {
-    if (cuda_status(cudaFuncSetAttribute(tc::verify_tc_kernel<NP>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem),
-                    "cudaFuncSetAttribute") != S3R_OK)
-      return S3R_ERR_CUDA;
-    attr_done = true;
-  }
+  static std::atomic<uint64_t> attr_done{0};
+  if (cuda_status(ensure_smem_attr(tc::verify_tc_kernel<NP>, C::kSmem, attr_done), "cudaFuncSetAttribute") !=
+      S3R_OK)
+    return S3R_ERR_CUDA;
   launch_pdl(tc::verify_tc_kernel<NP>, num_sms, tc::kThreads, C::kSmem, stream, tq, tk, tv, tk8, tv8, p,
                                                                         batch);
   return cuda_status(cudaGetLastError(), __func__);

@@ -39,6 +39,9 @@ class RoundBuffers:
         self._verify_out = torch.empty(num_requests * T * num_q_heads * head_dim, dtype=bf, device=device)
         self._draft_tokens = torch.zeros(num_requests * k_max, dtype=i32, device=device)
         self._out_tokens = torch.full((num_requests * T,), -1, dtype=i32, device=device)
+        # decision margins the samplers report (draft draws; accept tests and the final draw)
+        self._draft_margins = torch.zeros(num_requests * k_max, dtype=f32, device=device)
+        self._spec_margins = torch.zeros(num_requests * T, dtype=f32, device=device)
         self.prefill_lse = torch.empty((num_requests, 1, num_q_heads), dtype=f32, device=device)
         self.sel_idx = torch.zeros((num_requests, num_kv_heads, sel_stride), dtype=i32, device=device)
         self.sel_count = torch.zeros((num_requests, num_kv_heads), dtype=i32, device=device)
@@ -58,6 +61,8 @@ class RoundBuffers:
         self.verify_out = self._verify_out[: NR * T * Hq * d].view(NR, T, Hq, d)
         self.draft_tokens = self._draft_tokens[: NR * k].view(NR, k)
         self.out_tokens = self._out_tokens[: NR * T].view(NR, T)
+        self.draft_margins = self._draft_margins[: NR * k].view(NR, k)
+        self.spec_margins = self._spec_margins[: NR * T].view(NR, T)
 
 
 class S3REngine:
@@ -135,7 +140,7 @@ class S3REngine:
                                self.buf.draft_tokens, self.ws)
             return
         L.s3r_draft_sample(self.batch, self.buf.steps[i], self.k, q_logits, self.vocab, self.seed,
-                           self.buf.draft_tokens, self.ws)
+                           self.buf.draft_tokens, self.ws, margins=self.buf.draft_margins)
 
     def draft_step(self, i, q_block, k_block, v_block, q_logits, draft_logits_fn=None):
         self.draft_attn(i, q_block, k_block, v_block)
@@ -158,7 +163,7 @@ class S3REngine:
                                 b.out_tokens, b.n_out, self.ws)
         else:
             L.s3r_spec_sample(self.batch, self.k, p_logits, q_logits, b.draft_tokens, self.vocab,
-                              self.seed, b.out_tokens, b.n_out, self.ws)
+                              self.seed, b.out_tokens, b.n_out, self.ws, margins=b.spec_margins)
         L.s3r_commit(self.batch, self.k, b.n_out, self.seq_lens, b.stats)
 
     def round(self, q_block, k_block, v_block, p_logits, q_logits, draft_logits_fn=None,
@@ -257,7 +262,7 @@ class MixedPhaseDriver:
             L.s3r_draft_argmax(batch, self.step, e.k, q_logits, e.vocab, b.draft_tokens, e.ws)
         else:
             L.s3r_draft_sample(batch, self.step, e.k, q_logits, e.vocab, e.seed, b.draft_tokens,
-                               e.ws)
+                               e.ws, margins=b.draft_margins)
 
     def iterate(self, q_block, k_block, v_block, p_logits, q_logits):
         """Advance every request by one phase; returns the ids that completed a round."""
@@ -276,7 +281,7 @@ class MixedPhaseDriver:
                                     b.n_out, e.ws)
             else:
                 L.s3r_spec_sample(batch, e.k, p_logits, q_logits, b.draft_tokens, e.vocab,
-                                  e.seed, b.out_tokens, b.n_out, e.ws)
+                                  e.seed, b.out_tokens, b.n_out, e.ws, margins=b.spec_margins)
             L.s3r_commit(batch, e.k, b.n_out, e.seq_lens, b.stats)
             sel = L.s3r_select_kv_pages if e.page_select else L.s3r_select_kv
             sel(e.cache, batch, b.scores, b.lse, e.k, e.budget_bp, e.window, b.sel_idx,

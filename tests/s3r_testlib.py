@@ -57,3 +57,39 @@ def assert_attention_close(gpu, ref, what=""):
     bound = ATOL + RTOL * np.abs(ref)
     bad = err > bound
     assert not bad.any(), f"{what}: {bad.sum()} of {bad.size} outside tolerance, max err {err.max():.3g}"
+
+
+def compare_round_decisions(res, drafts, tokens, n_out, k):
+    """Compare one request's sampled decisions of a round with the oracle's round `res`.
+
+    Decisions are taken in order: the k draft draws, then the accept tests of the drafts up
+    to the first rejection, then the final draw. Everything before the first decision that
+    differs must be identical, and that decision must be a boundary case: its own oracle
+    margin (|u - C_edge / Z| for a draw, |u - p/q| for an accept test) below MARGIN.
+    Returns True if the whole round was identical, False for an excused boundary case."""
+    od = np.asarray(res["drafts"])
+    for i in range(k):
+        if int(drafts[i]) != int(od[i]):
+            assert res["draft_margin"][i] < MARGIN, ("draft", i, float(res["draft_margin"][i]))
+            return False   # later decisions follow other drafts
+    ot, on, om = list(res["tokens"]), int(res["n_out"]), np.asarray(res["margins"])
+    gt = [int(x) for x in tokens[:n_out]]
+    if n_out == on and gt == ot:
+        return True
+    a_o, a_g = on - 1, int(n_out) - 1     # drafts each side accepted
+    j = min(a_o, a_g)
+    assert gt[:j] == ot[:j] == [int(x) for x in od[:j]], ("accepted prefix", j)
+    if a_o != a_g:                         # the accept test of draft j went both ways
+        assert om[j] < MARGIN, ("accept", j, om.tolist())
+    else:                                  # same accepts, the final draw differs
+        assert om[-1] < MARGIN, ("draw", j, om.tolist())
+    return False
+
+
+def check_sampler_margins(gpu_margins, oracle_margins, count):
+    """The first `count` margins the GPU reported agree with the oracle's to 1e-5 (plus
+    1e-5 relative): both measure the same distance, the GPU from fp32 weights."""
+    g = np.asarray(gpu_margins, dtype=np.float64)[:count]
+    o = np.asarray(oracle_margins, dtype=np.float64)[:count]
+    fin = np.isfinite(o)
+    assert np.all(np.abs(g[fin] - o[fin]) <= 1e-5 + 1e-5 * np.abs(o[fin])), (g, o)

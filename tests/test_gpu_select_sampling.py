@@ -9,7 +9,7 @@ from scipy import stats
 import synth
 import sparse_dense_kv_b200 as s3r
 from oracle import s3r_oracle as O
-from tests.s3r_testlib import MARGIN, Case, f64, spec_for
+from tests.s3r_testlib import MARGIN, Case, check_sampler_margins, f64, spec_for
 
 pytestmark = pytest.mark.gpu
 
@@ -137,21 +137,24 @@ def test_draft_and_spec_sampling_match_oracle(V):
     batch = s3r.make_batch(seq)
     pd, qd = torch.as_tensor(p).cuda(), torch.as_tensor(qn).cuda()
     gdrafts = torch.zeros((NR, k), dtype=torch.int32, device="cuda")
+    gdm = torch.full((NR, k), -1.0, dtype=torch.float32, device="cuda")
     cache = s3r.KVCacheDesc(8, 8, 128, 16, 1, 16, 16)
     ws = s3r.new_workspace(s3r.s3r_workspace_size(cache, NR, 1, k, V, 1))
     for i in range(k):
         step = torch.full((NR,), i, dtype=torch.int32, device="cuda")
-        s3r.s3r_draft_sample(batch, step, k, qd, V, seed, gdrafts, ws)
+        s3r.s3r_draft_sample(batch, step, k, qd, V, seed, gdrafts, ws, margins=gdm)
     # the oracle's drafts drive the speculative sampler on both sides
     odrafts = np.zeros((NR, k), dtype=np.int32)
     exact = near = 0
     gd = gdrafts.cpu().numpy()
+    gdm = gdm.cpu().numpy()
     for r in range(NR):
         for i in range(k):
             u = float(O.uniform(seed, r, int(lens[r]) + i + 1, O.STREAM_DRAFT))
             t, mg = O.draft_sample(qn[r, i], u)
             odrafts[r, i] = t
             if gd[r, i] == t:
+                check_sampler_margins([gdm[r, i]], [mg], 1)   # the GPU reports the same margin
                 exact += 1
             else:
                 assert mg < MARGIN and draw_is_valid(O.softmax64(qn[r, i]), u, gd[r, i]), (r, i)
@@ -159,9 +162,11 @@ def test_draft_and_spec_sampling_match_oracle(V):
     assert exact >= 0.99 * NR * k
     out = torch.full((NR, k + 1), -1, dtype=torch.int32, device="cuda")
     n_out = torch.zeros(NR, dtype=torch.int32, device="cuda")
-    s3r.s3r_spec_sample(batch, k, pd, qd, torch.as_tensor(odrafts).cuda(), V, seed, out, n_out, ws)
+    smg = torch.full((NR, k + 1), -1.0, dtype=torch.float32, device="cuda")
+    s3r.s3r_spec_sample(batch, k, pd, qd, torch.as_tensor(odrafts).cuda(), V, seed, out, n_out, ws,
+                        margins=smg)
     assert s3r.s3r_get_error(ws) == 0
-    out, n_out = out.cpu().numpy(), n_out.cpu().numpy()
+    out, n_out, smg = out.cpu().numpy(), n_out.cpu().numpy(), smg.cpu().numpy()
     same = 0
     P, Q = O.softmax64(p), O.softmax64(qn)
     for r in range(NR):
@@ -169,6 +174,11 @@ def test_draft_and_spec_sampling_match_oracle(V):
         toks, n, margins = O.spec_sample(p[r], qn[r], odrafts[r], seed, r, L)
         g = out[r, : n_out[r]].tolist()
         if n_out[r] == n and g == toks.tolist():
+            # decided drafts' |u - p/q| and the draw's cell-edge distance, in decision order;
+            # entries past them are untouched
+            assert len(margins) == min(n, k) + 1
+            check_sampler_margins(smg[r], margins, len(margins))
+            assert (smg[r, len(margins):] == -1.0).all()
             same += 1
             continue
         # the first decision that differs must be a boundary case

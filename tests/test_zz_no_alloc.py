@@ -92,3 +92,36 @@ def test_noalloc_rejects_sizes_beyond_the_static_scratch():
     with pytest.raises(s3r.S3RError, match="static scratch"):
         s3r.s3r_draft_sample_noalloc(small, step, k, q, 262145, 1, out, err)
     assert s3r.s3r_launch_count() == before
+
+
+def test_noalloc_out_of_range_request_id_is_reported_and_skipped():
+    """A request id outside [0, num_requests) sets the device-bounds bit and that row is
+    skipped by every CTA (no ticket or partial outside the scratch is touched); the other
+    rows are drawn, and a clean call afterwards still matches the workspace path."""
+    NR, k, V = 40, 4, 30000
+    q, lens, step = _inputs(NR, k, V, seed=8)
+    cache = s3r.KVCacheDesc(8, 8, 128, 16, 1, 16, 16)
+    ws = s3r.new_workspace(s3r.s3r_workspace_size(cache, NR, 1, k, V, 1))
+    ids = torch.arange(0, NR, 2, dtype=torch.int32, device="cuda")
+    ref = torch.full((NR, k), -1, dtype=torch.int32, device="cuda")
+    s3r.s3r_draft_sample(s3r.make_batch(lens, req_ids=ids), step, k, q, V, 3, ref, ws)
+    assert s3r.s3r_get_error(ws) == 0
+    bad_ids = ids.clone()
+    bad_ids[1] = NR                      # one past the last request
+    bad_ids[2] = -1
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    got = torch.full((NR, k), -1, dtype=torch.int32, device="cuda")
+    s3r.s3r_draft_sample_noalloc(s3r.make_batch(lens, req_ids=bad_ids), step, k, q, V, 3, got, err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 1 << 5     # S3R_ERR_DEVICE_BOUNDS
+    keep = torch.ones(ids.numel(), dtype=torch.bool)
+    keep[1:3] = False
+    good = ids[keep.cuda()].long()
+    assert torch.equal(got[good], ref[good])
+    assert bool((got[ids[1:3].long()] == -1).all())
+    err.zero_()
+    again = torch.full((NR, k), -1, dtype=torch.int32, device="cuda")
+    s3r.s3r_draft_sample_noalloc(s3r.make_batch(lens, req_ids=ids), step, k, q, V, 3, again, err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert torch.equal(again, ref)
