@@ -10,7 +10,7 @@ namespace s3r {
 
 constexpr int kVerifyChunk = 1024;   // positions per verify CTA (multiple of 64)
 constexpr int kVerifyChunkMin = 896; // smallest verify chunk of any kernel (workspace sizing)
-constexpr int kSegMax = 4;           // draft: segments (chunk records) per (request, KV head)
+constexpr int kDraftChunk = 512;     // positions per draft CTA (multiple of 128)
 constexpr int kVocabChunk = 8192;    // vocabulary entries per sampler CTA
 
 struct VerifyParams {
@@ -62,10 +62,9 @@ struct DraftParams {
   float scale;
   int* err;
   int* tickets;
-  float* part;             // [num_requests][Hkv][kSegMax] chunk records
-  int req_off;             // launch covers requests req_ids[req_off + b] (or req_off + b)
+  float* part;             // [num_requests][Hkv][nchunk_max] chunk records
+  int nchunk_max;
   int num_requests;        // size of every per-request array (request ids are checked)
-  int wait_limit;          // polls before a wait on another warp role gives up
 };
 
 struct SelectParams {
@@ -128,8 +127,7 @@ int launch_verify_tc(const CUtensorMap& qm, const CUtensorMap& k1, const CUtenso
                      const CUtensorMap& k8, const CUtensorMap& v8, const VerifyParams& p,
                      int batch, int num_sms, cudaStream_t stream, int* launches);
 
-// Persistent draft kernel over all pairs of the batch (several launches beyond 4096
-// (request, KV head) pairs); *launches receives the number of launches issued.
+// *launches receives the number of launches issued.
 int launch_draft(const DraftParams& p, int D, int batch, int num_sms, cudaStream_t stream, int* launches);
 size_t draft_partial_bytes(int num_requests, int Hkv, int sel_stride, int D);
 

@@ -521,9 +521,8 @@ int s3r_sparse_draft_attn(const s3r_kv_cache* cache, const s3r_batch* batch,
   p.err = w.err;
   p.tickets = w.tickets;
   p.part = reinterpret_cast<float*>(w.part);
-  p.req_off = 0;
+  p.nchunk_max = (sel_stride + S3R_MAX_K + 1 + kDraftChunk - 1) / kDraftChunk;
   p.num_requests = batch->num_requests;
-  p.wait_limit = g_wait_limit.load();
   int nl = 0;
   const int st = launch_draft(p, cache->head_dim, batch->batch, sm_count(), (cudaStream_t)stream, &nl);
   g_launches.fetch_add((uint64_t)nl, std::memory_order_relaxed);
