@@ -181,6 +181,66 @@ def algorithmic_bytes(spec, lens, sel_counts=None):
     return verify, draft, scores
 
 
+def projection_logits_round(eng, spec, inp, seq, seq0, o_prefill):
+    """Fill inp["p"] / inp["qlog"] from a round whose logits are gamma * (head-concatenated
+    attention output) @ W, W the workload's seeded bf16 projection; gamma is one scalar
+    calibrated on the prefill outputs so that dense logits have standard deviation sqrt(2).
+    Returns (gamma, the round's emitted-token count)."""
+    import math as _m
+    import torch
+    NR, k = spec.num_requests, spec.k
+    W = synth.projection_matrix(spec, seq.device).float()
+    gamma = float(_m.sqrt(2.0) / (o_prefill.float().reshape(NR, -1) @ W).std().item())
+
+    def draft_fn(i, out, q_logits):
+        q_logits[:, i] = gamma * (out.float().reshape(NR, -1) @ W)
+
+    def target_fn(vout, p_logits):
+        p_logits.copy_((gamma * (vout.float().reshape(NR * (k + 1), -1) @ W)).view(NR, k + 1, -1))
+
+    seq.copy_(seq0)
+    before = int(eng.buf.stats[0].item())
+    eng.round(inp["q"], inp["k"], inp["v"], inp["p"], inp["qlog"], draft_logits_fn=draft_fn,
+              target_logits_fn=target_fn)
+    torch.cuda.synchronize()
+    return gamma, int(eng.buf.stats[0].item()) - before
+
+
+def boundary_cases(eng, k, margin=1e-5, tight=1e-7):
+    """Decisions of the last round whose margin to their boundary (as the samplers computed
+    it) is below `margin` (the stated 1e-5) and below `tight` (about the rounding of the
+    samplers' fp32 cumulative sums, the margins that can flip a decision): draft draws, and
+    the accept tests and final draws of the speculative sampler (min(n_out, k) + 1 decisions
+    per request). With a 151936-token vocabulary the mean cell of a draw is 6.6e-6 wide, so
+    most draws lie within 1e-5 of a cell edge."""
+    dm = eng.buf.draft_margins.cpu().numpy()
+    sm = eng.buf.spec_margins.cpu().numpy()
+    n_out = eng.buf.n_out.cpu().numpy()
+    spec_dec = [sm[r, : min(int(n_out[r]), k) + 1] for r in range(len(n_out))]
+    n_spec = int(sum(x.size for x in spec_dec))
+    count = lambda th: {"draft_draws": int((dm < th).sum()),  # noqa: E731
+                        "spec_decisions": int(sum((x < th).sum() for x in spec_dec))}
+    return {"threshold": margin, **count(margin), "draft_of": int(dm.size), "spec_of": n_spec,
+            "tight_threshold": tight, "tight": count(tight),
+            "note": "counted from the samplers' margin outputs of the last timed round"}
+
+
+def round_bytes(spec, lens, vb, db, sb, greedy=False):
+    """Algorithmic HBM bytes of one round: verify K/V reads and score-logit writes, the
+    selection's score-logit reads and its per-position score array (written, read), the
+    draft K/V and index reads, and the samplers' logit reads (draft sampling: one row per
+    request and step; speculative sampling: 2k+1 rows, plus the drawn row again)."""
+    NR, Hkv, V, k = spec.num_requests, spec.num_kv_heads, spec.vocab, spec.k
+    pos = int(sum(lens))
+    select = sb + 2 * 4 * pos * Hkv
+    draft_sampling = k * NR * V * 4
+    spec_sampling = NR * (2 * k + 1) * V * 4 + NR * V * 4 * (1 if greedy else 2)
+    parts = {"verify_kv": int(vb), "verify_scores": int(sb), "select": int(select),
+             "draft_kv": int(sum(db)), "draft_sampling": int(draft_sampling),
+             "spec_sampling": int(spec_sampling)}
+    return {"total": int(sum(parts.values())), "parts": parts}
+
+
 def run_ours(args, spec):
     import torch
     import torch.distributed as dist
@@ -199,7 +259,7 @@ def run_ours(args, spec):
                         seed=spec.sample_seed + rank, page_select=args.select == "pages",
                         greedy=args.greedy)
     seq0 = seq.clone()
-    eng.prefill(inp["q"][:, :1].contiguous(), inp["k"][:, :1].contiguous(), inp["v"][:, :1].contiguous())
+    o0 = eng.prefill(inp["q"][:, :1].contiguous(), inp["k"][:, :1].contiguous(), inp["v"][:, :1].contiguous())
     stream = torch.cuda.current_stream()
 
     def step(ev=None, x=inp):
@@ -223,6 +283,14 @@ def run_ours(args, spec):
     for _ in range(args.warmup):
         step()
     assert eng.check_errors() == 0, "device error during warm-up"
+    gamma = None
+    if spec.projection_logits:
+        # the logits of the round come from a seeded bf16 projection of the attention outputs
+        # (the rest of the model, off the timed path): one round from the committed lengths,
+        # in the steady state the warm-up reached, computes them; the timed rounds replay the
+        # same round with these logits, so acceptance follows draft / verify fidelity
+        gamma, _ = projection_logits_round(eng, spec, inp, seq, seq0, o0)
+        assert eng.check_errors() == 0, "device error in the projection round"
 
     # the round as one CUDA graph: the same launches on the same buffers, no host work per
     # launch; the timed steps are graph replays
@@ -255,6 +323,7 @@ def run_ours(args, spec):
     tokens = int(eng.buf.stats[0].item()) - tok0
     assert eng.check_errors() == 0, "device error in the timed region"
     ms_max, tokens_all = reduce_results(ms, tokens)
+    boundary = boundary_cases(eng, k)
 
     # per-kernel device times: eager steps with events between the library calls, each
     # enqueued behind a sleeping kernel so that the host is ahead and the kernels run back to
@@ -273,10 +342,22 @@ def run_ours(args, spec):
     ds_ms = [avg(lambda e: e["dm"][i], lambda e: e["d1"][i]) for i in range(k)]
     sel_ms = avg(lambda e: e["s0"], lambda e: e["d0"][0])
     spec_ms = avg(lambda e: e["v1"], lambda e: e["c1"])
+    # the verify call without score capture (score_logits = NULL): its K/V stream alone
+    evn = [(E(), E()) for _ in range(nb)]
+    for a_, b_ in evn:
+        torch.cuda._sleep(30_000_000)
+        a_.record(stream)
+        s3r.s3r_verify_attn(eng.cache, eng.batch, k, inp["q"], inp["k"], inp["v"], eng.buf.verify_out,
+                            eng.buf.lse, None, eng.ws)
+        b_.record(stream)
+    torch.cuda.synchronize()
+    assert eng.check_errors() == 0, "device error in the no-capture verify pass"
+    vn_ms = sum(a_.elapsed_time(b_) for a_, b_ in evn) / nb
     vb, db, sb = algorithmic_bytes(spec, lens, eng.buf.sel_count.cpu().numpy())
     peak, peak_kind = measured_peaks()
     v_gbs = vb / (v_ms * 1e-3) / 1e9
     d_gbs = sum(db) / (sum(d_ms) * 1e-3) / 1e9
+    rb = round_bytes(spec, lens, vb, db, sb, greedy=args.greedy)
 
     # end to end through the public API: pinned host inputs in, tokens out, every round. The
     # inputs are double-buffered: while the graph of round s runs on the compute stream, the
@@ -344,14 +425,26 @@ def run_ours(args, spec):
                      "algorithmic_bytes_per_launch": vb},
         "kernels": {"verify_ms": v_ms, "verify_kv_gbs": v_gbs,
                     "verify_gbs_with_scores": (vb + sb) / (v_ms * 1e-3) / 1e9,
+                    "verify_no_capture_ms": vn_ms,
+                    "verify_no_capture_kv_gbs": vb / (vn_ms * 1e-3) / 1e9,
+                    "verify_no_capture_frac": vb / (vn_ms * 1e-3) / 1e9 / peak,
                     "draft_attn_ms_per_step": sum(d_ms) / k, "draft_kv_gbs": d_gbs,
                     "draft_sample_ms_per_step": sum(ds_ms) / k, "select_ms": sel_ms,
                     "spec_sample_commit_ms": spec_ms,
                     "frac_of_8tbs": {"verify": v_gbs / 8000.0, "draft": d_gbs / 8000.0}},
+        "round_roofline": {"bytes": rb["total"], "parts": rb["parts"],
+                           "ms_at_peak": rb["total"] / (peak * 1e9) * 1e3,
+                           "achieved_gbs": rb["total"] / (ms_max / args.steps * 1e-3) / 1e9,
+                           "frac": rb["total"] / (ms_max / args.steps * 1e-3) / 1e9 / peak},
+        "boundary_cases": boundary,
         "tau": float(st[0] / max(st[1], 1)), "acceptance_by_position": acc,
         "gpu_launches": int(launches), "launches_per_step": int(launches_per_step),
         "execution": "CUDA graph of one round, replayed per step", "clocks": clocks, "e2e": e2e,
     }
+    if spec.projection_logits:
+        result["config"]["logits"] = (f"seeded bf16 projection (vocab {spec.vocab}) of the attention "
+                                      f"outputs, gamma {gamma:.3f}, computed off the timed path")
+        result["config"]["l2"] = "inputs larger than L2 (KV 3.2 GB)"
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(spec, lens, cache, inp, budget_s=args.cpu_seconds,
                                               mode=oracle_mode(args))
@@ -360,6 +453,220 @@ def run_ours(args, spec):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+# ----------------------------------------------------------- mixed-phase ragged batch ----
+def run_ragged(args, spec):
+    """The high-concurrency ragged workload: requests at mixed round phases over shuffled
+    page tables. A step is one iteration of the mixed-phase schedule: the requests in the
+    middle of a round draft their next token (one draft-attention and one draft-sampling
+    launch over their ids, each request at its own step) and the others verify, sample,
+    commit and select their next set (one launch each over their ids); k+1 steps give every
+    request one round. The k+1 iteration patterns repeat, so each is captured once as a
+    CUDA graph and the timed steps replay them in order; the drafting requests' current
+    q/k/v rows (the model's output in a real system) are gathered per pattern outside the
+    timed region. value = tokens emitted by the steps' commits / device time."""
+    import torch
+    import torch.distributed as dist
+    import sparse_dense_kv_b200 as s3r
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1 and not dist.is_initialized():
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    k, NR = spec.k, spec.num_requests
+    # iterations the cache must absorb: warm-up, the capture's eager pass, timed steps, the
+    # per-kernel pass and the end-to-end steps, each advancing a request by <= k+1 tokens a round
+    iters = args.warmup + 2 * (k + 1) + args.steps + (k + 1) + args.e2e_steps
+    extra = (iters // (k + 1) + 3) * (k + 1) + 16
+    lens = synth.make_lengths(spec)
+    cache = synth.build_cache(spec, lens, extra_tokens=extra, device=dev, seed=spec.data_seed + 7919 * rank)
+    Hq, Hkv, d, V = spec.num_q_heads, spec.num_kv_heads, spec.head_dim, spec.vocab
+    s0 = 100 + 13 * rank
+    inp = dict(q=synth.randn_bf16((NR, k + 1, Hq, d), s0, dev), k=synth.randn_bf16((NR, k + 1, Hkv, d), s0 + 1, dev),
+               v=synth.randn_bf16((NR, k + 1, Hkv, d), s0 + 2, dev),
+               p=synth.randn_f32((NR, k + 1, V), s0 + 3, dev, scale=spec.logit_std))
+    inp["qlog"] = (inp["p"][:, :k] + synth.randn_f32((NR, k, V), s0 + 4, dev, scale=spec.draft_noise_std)).contiguous()
+    seq = torch.as_tensor(lens, dtype=torch.int32, device=dev)
+    eng = s3r.S3REngine(cache.k_pool, cache.v_pool, cache.page_table, seq, Hq, k=k, budget_bp=spec.budget_bp,
+                        window=spec.window, vocab=V, seed=spec.sample_seed + rank,
+                        page_select=args.select == "pages", greedy=args.greedy)
+    eng.prefill(inp["q"][:, :1].contiguous(), inp["k"][:, :1].contiguous(), inp["v"][:, :1].contiguous())
+    drv = s3r.MixedPhaseDriver(eng, synth.initial_phases(spec, seed=spec.data_seed + rank))
+    drv.start(inp["q"], inp["k"], inp["v"], inp["qlog"])
+    its = drv.cycle(inp["q"], inp["k"], inp["v"], inp["p"], inp["qlog"])
+    n = len(its)
+    stream = torch.cuda.current_stream()
+    for w in range(args.warmup):
+        its[w % n]()
+    # finish the cycle, so the graphs are captured (each after one eager pass of its own
+    # iteration) in cycle order from pattern 0
+    for w in range(args.warmup, -(-args.warmup // n) * n):
+        its[w % n]()
+    assert eng.check_errors() == 0, "device error during warm-up"
+    graphs, lpi = [], []
+    for it in its:
+        g, nl = eng.capture(it)
+        graphs.append(g)
+        lpi.append(nl)
+
+    E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    start, end = E(), E()
+    tok0 = int(eng.buf.stats[0].item())
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = time.time()
+    start.record(stream)
+    for st_ in range(args.steps):
+        graphs[st_ % n].replay()
+    end.record(stream)
+    torch.cuda.synchronize()
+    t1 = time.time()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop(t0, t1)
+    ms = start.elapsed_time(end)
+    tokens = int(eng.buf.stats[0].item()) - tok0
+    assert eng.check_errors() == 0, "device error in the timed region"
+    ms_max, tokens_all = reduce_results(ms, tokens)
+    launches = sum(lpi[st_ % n] for st_ in range(args.steps))
+    boundary = boundary_cases(eng, k)
+    # the timed steps end on a cycle boundary only if steps % n == 0: finish the cycle so the
+    # per-kernel pass starts at pattern 0
+    for st_ in range(args.steps, -(-args.steps // n) * n):
+        graphs[st_ % n].replay()
+
+    # per-kernel device times over one eager cycle, behind a sleeping kernel; the lengths and
+    # set sizes each iteration saw are copied aside on the device for the byte counts
+    evs = [{n_: E() for n_ in ("d0", "dm", "d1", "v0", "v1", "c1", "s1")} for _ in range(n)]
+    L_hist = torch.empty((n, NR), dtype=torch.int32, device=dev)
+    C_hist = torch.empty((n, NR, Hkv), dtype=torch.int32, device=dev)
+    torch.cuda._sleep(60_000_000)
+    for c, it in enumerate(its):
+        L_hist[c].copy_(eng.seq_lens)
+        C_hist[c].copy_(eng.buf.sel_count)
+        it(evs[c])
+    torch.cuda.synchronize()
+    assert eng.check_errors() == 0, "device error in the per-kernel pass"
+    L_hist, C_hist = L_hist.cpu().numpy().astype(np.int64), C_hist.cpu().numpy().astype(np.int64)
+    per_pos = 2 * d * 2 * Hkv
+    v_ms = d_ms = ds_ms = sp_ms = sel_ms = 0.0
+    vb = db = 0
+    for c, it in enumerate(its):
+        e = evs[c]
+        d_ms += e["d0"].elapsed_time(e["dm"])
+        ds_ms += e["dm"].elapsed_time(e["d1"])
+        v_ms += e["v0"].elapsed_time(e["v1"])
+        sp_ms += e["v1"].elapsed_time(e["c1"])
+        sel_ms += e["c1"].elapsed_time(e["s1"])
+        info = it.info
+        vb += int(sum(L_hist[c, r] + k + 1 for r in info["v_ids"])) * per_pos
+        for r in info["d_ids"]:
+            i = int(info["steps"][r])
+            db += int(sum((C_hist[c, r, h] + i + 1) * 2 * d * 2 + 4 * C_hist[c, r, h] for h in range(Hkv)))
+    peak, peak_kind = measured_peaks()
+    v_gbs = vb / (v_ms * 1e-3) / 1e9
+    d_gbs = db / (d_ms * 1e-3) / 1e9
+
+    # end to end: every step copies the rows its launches read from pinned host memory
+    # (drafting requests: their current q/k/v rows and draft-logit row; verifying requests:
+    # their q/k/v blocks, target and draft logits) and reads the emitted tokens back
+    e2e = None
+    if args.e2e_steps > 0:
+        hp = {n_: t.cpu().pin_memory() for n_, t in inp.items()}
+        plan = []
+        for it in its:
+            info = it.info
+            di = torch.as_tensor(info["d_ids"], dtype=torch.long)
+            vi = torch.as_tensor(info["v_ids"], dtype=torch.long)
+            st_h = torch.as_tensor(info["steps"], dtype=torch.long)[di]
+            host = {"qc": it.info["qc"].cpu()[di].pin_memory(), "kc": it.info["kc"].cpu()[di].pin_memory(),
+                    "vc": it.info["vc"].cpu()[di].pin_memory(), "qd": hp["qlog"][di, st_h].pin_memory()}
+            for n_ in ("q", "k", "v", "p", "qlog"):
+                host["v_" + n_] = hp[n_][vi].pin_memory()
+            devb = {n_: torch.empty_like(t, device=dev) for n_, t in host.items()}
+            plan.append((di.to(dev), vi.to(dev), st_h.to(dev), host, devb))
+        out_h = torch.empty((NR, k + 1), dtype=torch.int32).pin_memory()
+        n_h = torch.empty((NR,), dtype=torch.int32).pin_memory()
+        h2d = d2h = 0
+        e0, e1 = E(), E()
+        tok_e = int(eng.buf.stats[0].item())
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for st_ in range(args.e2e_steps):
+            c = st_ % n
+            di, vi, st_d, host, devb = plan[c]
+            for n_, t in host.items():
+                devb[n_].copy_(t, non_blocking=True)
+                h2d += t.numel() * t.element_size()
+            it = its[c].info
+            it["qc"].index_copy_(0, di, devb["qc"])
+            it["kc"].index_copy_(0, di, devb["kc"])
+            it["vc"].index_copy_(0, di, devb["vc"])
+            inp["qlog"][di, st_d] = devb["qd"]
+            for n_ in ("q", "k", "v", "p", "qlog"):
+                inp[n_].index_copy_(0, vi, devb["v_" + n_])
+            graphs[c].replay()
+            out_h.copy_(eng.buf.out_tokens, non_blocking=True)
+            n_h.copy_(eng.buf.n_out, non_blocking=True)
+            d2h += out_h.numel() * 4 + n_h.numel() * 4
+        e1.record(stream)
+        torch.cuda.synchronize()
+        tok_e = int(eng.buf.stats[0].item()) - tok_e
+        ems, etok = reduce_results(e0.elapsed_time(e1), tok_e)
+        e2e = {"value": etok / (ems * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d // args.e2e_steps,
+               "d2h_bytes_per_step": d2h // args.e2e_steps, "steps": args.e2e_steps,
+               "overlap": "none: each step's rows are copied, scattered into place, then the step runs"}
+    del graphs
+
+    st = eng.buf.stats.cpu().numpy()
+    acc = [float(st[2 + j] / max(st[2 + s3r.MAX_K + j], 1)) for j in range(k)]
+    result = {
+        "metric": METRIC, "value": tokens_all / (ms_max * 1e-3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{spec.name}: {NR} requests, L {spec.lengths}, {Hq}/{Hkv} heads, d {d}, k {k}, "
+                               f"s {spec.budget_bp / 1e4}, window {spec.window}, vocab {V}, mixed round phases, "
+                               "shuffled page tables",
+                   "step": "one iteration of the mixed-phase schedule (k+1 iterations = one round per request)",
+                   "requests_per_gpu": NR, "parallelism": f"replicas x{world}", "selection": args.select,
+                   "verification": "greedy" if args.greedy else "speculative sampling",
+                   "l2": "inputs larger than L2 (KV 5.8 GB, logits 2.0 GB)"},
+        "roofline": {"bound": "hbm", "achieved": v_gbs, "peak": peak, "unit": "GB/s", "frac": v_gbs / peak,
+                     "traffic": None, "kernel": "s3r_verify_attn", "peak_kind": peak_kind,
+                     "algorithmic_bytes_per_launch": vb // n},
+        "kernels": {"verify_ms_per_cycle": v_ms, "verify_kv_gbs": v_gbs, "draft_attn_ms_per_cycle": d_ms,
+                    "draft_kv_gbs": d_gbs, "draft_sample_ms_per_cycle": ds_ms,
+                    "spec_sample_commit_ms_per_cycle": sp_ms, "select_ms_per_cycle": sel_ms,
+                    "frac_of_8tbs": {"verify": v_gbs / 8000.0, "draft": d_gbs / 8000.0},
+                    "draft_frac": d_gbs / peak},
+        "boundary_cases": boundary,
+        "tau": float(st[0] / max(st[1], 1)), "acceptance_by_position": acc,
+        "gpu_launches": int(launches), "launches_per_step": float(sum(lpi)) / n,
+        "execution": f"{n} CUDA graphs (one per iteration pattern), replayed in order", "clocks": clocks,
+        "e2e": e2e,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline_ragged(spec, lens, cache, inp, budget_s=args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def cpu_baseline_ragged(spec, lens, cache, inp, budget_s=15.0):
+    """The oracle's rounds of the first requests of the ragged workload (each request's round
+    is what one cycle of iterations computes for it), on this host's cores."""
+    base = cpu_baseline(spec.with_(mixed_phases=False), lens, cache, inp, budget_s=budget_s)
+    base["sample"] += "; the oracle runs whole rounds (a cycle of k+1 iterations per request)"
+    return base
 
 
 # ---------------------------------------------------------------- admission scheduler ----
@@ -648,8 +955,9 @@ def oracle_mode(args):
     return {"page": 16 if args.select == "pages" else 1, "greedy": bool(args.greedy)}
 
 
-def oracle_round_sample(spec, lens, pools, page_table, inp_host, reqs, mode=None):
-    """Oracle rounds for the requests `reqs` (dense copies built outside the timing)."""
+def oracle_round_sample(spec, lens, pools, page_table, inp_host, reqs, mode=None, timings=None):
+    """Oracle rounds for the requests `reqs` (dense copies built outside the timing);
+    `timings` accumulates the seconds of each step of the round."""
     from oracle import s3r_oracle as O
     k = spec.k
     kp, vp = pools
@@ -668,7 +976,7 @@ def oracle_round_sample(spec, lens, pools, page_table, inp_host, reqs, mode=None
     for r, st in prepared:
         res = O.run_round(st, r, spec.sample_seed, k, spec.budget_bp, spec.window,
                           inp_host["q"][r], inp_host["k"][r], inp_host["v"][r],
-                          inp_host["qlog"][r], inp_host["p"][r], **(mode or {}))
+                          inp_host["qlog"][r], inp_host["p"][r], timings=timings, **(mode or {}))
         tokens += res["n_out"]
     return tokens, time.perf_counter() - t0
 
@@ -678,20 +986,48 @@ def host_inputs(inp, reqs):
 
 
 def cpu_baseline(spec, lens, cache, inp, budget_s=15.0, mode=None):
-    """The oracle on this host's cores on a bounded sample of the same workload."""
+    """The oracle on this host's cores on a bounded sample of the same workload, with the
+    seconds of each step of its rounds, and the first sampled request's round again with
+    the BLAS thread pool limited to one thread."""
     reqs, tokens, secs = [], 0, 0.0
-    pools = (cache.k_pool.float().cpu().numpy(), cache.v_pool.float().cpu().numpy())
-    pt = cache.page_table.cpu().numpy()
+    pt_all = cache.page_table.cpu().numpy()
+    timings = {}
+
+    def request_pools(r):
+        # the request's own pages only (its page-table row renumbered), in float32 on the host
+        import torch
+        ids = pt_all[r][pt_all[r] >= 0]
+        idx = torch.as_tensor(ids, dtype=torch.long, device=cache.k_pool.device)
+        kp = cache.k_pool.index_select(0, idx).float().cpu().numpy()
+        vp = cache.v_pool.index_select(0, idx).float().cpu().numpy()
+        pt = np.full_like(pt_all, -1)
+        pt[r, : ids.size] = np.arange(ids.size)
+        return (kp, vp), pt
+
     r = 0
     while secs < budget_s and r < spec.num_requests:
         hi = host_inputs(inp, [r])
-        t, s = oracle_round_sample(spec, lens, pools, pt, hi, [r], mode)
+        pools, pt = request_pools(r)
+        t, s = oracle_round_sample(spec, lens, pools, pt, hi, [r], mode, timings)
         tokens, secs = tokens + t, secs + s
         reqs.append(r)
         r += 1
+    one = None
+    try:
+        from threadpoolctl import threadpool_limits
+        hi = host_inputs(inp, [reqs[0]])
+        pools, pt = request_pools(reqs[0])
+        with threadpool_limits(limits=1):
+            t1, s1 = oracle_round_sample(spec, lens, pools, pt, hi, [reqs[0]], mode)
+        one = {"value": t1 / s1, "unit": UNIT, "cores": 1, "sample": f"one round of request {reqs[0]}",
+               "seconds": s1}
+    except ImportError:
+        pass
     return {"value": tokens / secs, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
             "sample": f"one round of requests {reqs[0]}..{reqs[-1]} ({len(reqs)} of "
-                      f"{spec.num_requests}), float64 numpy, {secs:.1f} s"}
+                      f"{spec.num_requests}), float64 numpy, {secs:.1f} s",
+            "step_seconds": {n_: round(v_, 4) for n_, v_ in timings.items()},
+            "single_thread": one}
 
 
 def run_reference(args, spec):
@@ -741,8 +1077,11 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="qwen3-8b", choices=["tiny", "qwen3-1.7b", "qwen3-8b"],
-                    help="synthetic workload (the ragged mixed-phase and sweep workloads are test / sweep cases)")
+    ap.add_argument("--workload", default="qwen3-8b", choices=["tiny", "qwen3-1.7b", "qwen3-8b", "ragged", "sweep"],
+                    help="synthetic workload (ragged: mixed-phase iterations; sweep: one (s, k) point of the "
+                         "budget / draft-length sweep, --budget-bp / --k)")
+    ap.add_argument("--budget-bp", type=int, default=0, help="sparse budget s in 1e-4 units (sweep point)")
+    ap.add_argument("--k", type=int, default=0, help="draft length (sweep point)")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -774,13 +1113,19 @@ def main(argv=None):
         return
     spec = synth.WORKLOADS[args.workload]
     if args.requests > 0:
-        spec = spec.with_(num_requests=args.requests)
-    if spec.projection_logits or spec.mixed_phases:
-        raise SystemExit("the mixed-phase and sweep workloads are parity / sweep cases, not bench lines")
+        spec = spec.with_(num_requests=args.requests,
+                          lengths=spec.lengths if spec.lengths[0] != "fixed"
+                          else ("fixed", spec.lengths[1][: args.requests]))
+    if args.budget_bp > 0 or args.k > 0:
+        if not spec.projection_logits:
+            raise SystemExit("--budget-bp / --k choose a point of the sweep workload")
+        spec = spec.with_(budget_bp=args.budget_bp or spec.budget_bp, k=args.k or spec.k)
     if args.impl == "reference":
         run_reference(args, spec)
     elif args.adaptive:
         run_adaptive(args, spec)
+    elif spec.mixed_phases:
+        run_ragged(args, spec)
     else:
         run_ours(args, spec)
 

@@ -448,15 +448,26 @@ def prefill_scores(state: RequestState, q_x, k_x, v_x):
 
 def run_round(state: RequestState, request: int, seed: int, k: int, budget_bp: int,
               window: int, q_rows, k_rows, v_rows, draft_logits, target_logits, page: int = 1,
-              greedy: bool = False):
+              greedy: bool = False, timings: dict | None = None):
     """One round for one request.
 
     q_rows [k+1][H_q][d], k_rows/v_rows [k+1][H_kv][d]: projections of the tokens at
     positions L .. L+k (identical in draft and verify). draft_logits [k][V] give q_j,
     target_logits [k+1][V] give p_j for the token at position L+j+1. page > 1 selects whole
     pages of that size (O3p) instead of positions; greedy drafts and verifies by argmax
-    (temperature 0) and has no sampling margins.
+    (temperature 0) and has no sampling margins. `timings`, if given, accumulates the wall
+    seconds of each step (select, draft_attn, draft_sample, verify, spec_sample) for the
+    benchmark's CPU baseline; it does not change what is computed.
     """
+    import time
+    clock = [time.perf_counter()]
+
+    def lap(name):
+        if timings is not None:
+            now = time.perf_counter()
+            timings[name] = timings.get(name, 0.0) + now - clock[0]
+            clock[0] = now
+
     L = state.L
     Hkv = state.K.shape[0]
     q_rows = np.asarray(q_rows, np.float64)
@@ -464,11 +475,13 @@ def run_round(state: RequestState, request: int, seed: int, k: int, budget_bp: i
         sel = [select_pages(state.sigma[h], L, budget_bp, window, page) for h in range(Hkv)]
     else:
         sel = [select_positions(state.sigma[h], L, budget_bp, window) for h in range(Hkv)]
+    lap("select")
     drafts, draft_out, draft_margin = [], [], []
     for i in range(k):
         state.write([L + i], [k_rows[i]], [v_rows[i]])
         o, _ = sparse_draft_attention(q_rows[i], state.K, state.V, sel, L, i)
         draft_out.append(o)
+        lap("draft_attn")
         if greedy:
             tok, mg = argmax_token(draft_logits[i]), np.inf
         else:
@@ -476,13 +489,16 @@ def run_round(state: RequestState, request: int, seed: int, k: int, budget_bp: i
             tok, mg = draft_sample(draft_logits[i], u0)
         drafts.append(tok)
         draft_margin.append(mg)
+        lap("draft_sample")
     state.write(list(range(L, L + k + 1)), k_rows, v_rows)
     v_out, lse, sigma, logits = verify_attention(q_rows, state.K, state.V, L)
+    lap("verify")
     if greedy:
         tokens, n_out = greedy_verify(target_logits, drafts)
         margins = np.array([np.inf])
     else:
         tokens, n_out, margins = spec_sample(target_logits, draft_logits, drafts, seed, request, L)
+    lap("spec_sample")
     state.sigma = sigma
     state.L = L + n_out
     return dict(sel=sel, drafts=np.asarray(drafts, np.int32), draft_out=np.asarray(draft_out),

@@ -264,6 +264,74 @@ class MixedPhaseDriver:
             L.s3r_draft_sample(batch, self.step, e.k, q_logits, e.vocab, e.seed, b.draft_tokens,
                                e.ws, margins=b.draft_margins)
 
+    def cycle(self, q_block, k_block, v_block, p_logits, q_logits):
+        """The k+1 iterations of one cycle from the current phases, as callables that issue
+        only library launches on fixed device buffers (so each can be captured in a CUDA
+        graph and replayed): iteration c drafts every request at phase (phase0 + c) % (k+1)
+        < k and verifies, samples, commits and reselects the others. The request lists, the
+        step arrays and each drafting request's current q/k/v rows are gathered here, once,
+        on the device. Calling them in order 0..k advances every request by one round and
+        returns the phases to where they were. Each callable takes an optional dict of
+        CUDA events ("d0", "dm", "d1", "v0", "v1", "c1", "s1") recorded between its calls."""
+        import numpy as np
+        e, b = self.e, self.e.buf
+        k, NR, dev = e.k, e.num_requests, self._dev
+        ar = torch.arange(NR, device=dev)
+        its = []
+        for c in range(k + 1):
+            ph = (self.phases + c) % (k + 1)
+            d_ids = np.nonzero(ph < k)[0]
+            v_ids = np.nonzero(ph == k)[0]
+            st = np.zeros(NR, dtype=np.int32)
+            st[d_ids] = ph[d_ids]
+            st_d = torch.as_tensor(st, device=dev)
+            rows = st_d.long()
+            it = dict(n_draft=int(d_ids.size), n_verify=int(v_ids.size), d_ids=d_ids, v_ids=v_ids,
+                      steps=st, step=st_d, qc=q_block[ar, rows].contiguous(),
+                      kc=k_block[ar, rows].contiguous(), vc=v_block[ar, rows].contiguous(),
+                      d_batch=self._batch(d_ids) if d_ids.size else None,
+                      v_batch=self._batch(v_ids) if v_ids.size else None)
+            its.append(it)
+
+        def make(it):
+            def run(ev=None):
+                rec = (lambda n: ev[n].record()) if ev is not None else (lambda n: None)
+                rec("d0")
+                if it["n_draft"]:
+                    L.s3r_sparse_draft_attn(e.cache, it["d_batch"], it["step"], it["qc"], it["kc"], it["vc"],
+                                            b.sel_idx, b.sel_count, b.draft_out, b.draft_lse, e.ws)
+                rec("dm")
+                if it["n_draft"]:
+                    if e.greedy:
+                        L.s3r_draft_argmax(it["d_batch"], it["step"], k, q_logits, e.vocab, b.draft_tokens, e.ws)
+                    else:
+                        L.s3r_draft_sample(it["d_batch"], it["step"], k, q_logits, e.vocab, e.seed,
+                                           b.draft_tokens, e.ws, margins=b.draft_margins)
+                rec("d1")
+                rec("v0")
+                if it["n_verify"]:
+                    vb = it["v_batch"]
+                    L.s3r_verify_attn(e.cache, vb, k, q_block, k_block, v_block, b.verify_out, b.lse,
+                                      b.scores, e.ws)
+                    rec("v1")
+                    if e.greedy:
+                        L.s3r_greedy_verify(vb, k, p_logits, b.draft_tokens, e.vocab, b.out_tokens, b.n_out, e.ws)
+                    else:
+                        L.s3r_spec_sample(vb, k, p_logits, q_logits, b.draft_tokens, e.vocab, e.seed,
+                                          b.out_tokens, b.n_out, e.ws, margins=b.spec_margins)
+                    L.s3r_commit(vb, k, b.n_out, e.seq_lens, b.stats)
+                    rec("c1")
+                    sel = L.s3r_select_kv_pages if e.page_select else L.s3r_select_kv
+                    sel(e.cache, vb, b.scores, b.lse, k, e.budget_bp, e.window, b.sel_idx, b.sel_count, e.ws)
+                else:
+                    rec("v1")
+                    rec("c1")
+                rec("s1")
+            run.info = it
+            return run
+
+        return [make(it) for it in its]
+
     def iterate(self, q_block, k_block, v_block, p_logits, q_logits):
         """Advance every request by one phase; returns the ids that completed a round."""
         import numpy as np
