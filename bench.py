@@ -1097,7 +1097,7 @@ def main(argv=None):
     ap.add_argument("--adaptive", action="store_true",
                     help="draft length chosen from the measured acceptance (one line, with the fixed-k run)")
     ap.add_argument("--k-max", type=int, default=7,
-                    help="largest adaptive draft length (7: the verify stays on the tensor-memory kernel at G = 4)")
+                    help="largest adaptive draft length")
     ap.add_argument("--interval", type=int, default=4)
     ap.add_argument("--decay", type=float, default=0.8)
     ap.add_argument("--sched", action="store_true",

@@ -367,9 +367,9 @@ S3R_API const char* s3r_status_string(int status);
 S3R_API uint64_t s3r_launch_count(void);
 
 /* Choose the kernel behind s3r_verify_attn for later calls (process-wide): 0 = automatic
- * (the tcgen05 tensor-memory kernel for head_dim 128 with G*(k+1) <= 32 and <= 2048
- * requests, otherwise the mma.sync kernel), 1 = always the mma.sync kernel. Both compute
- * the same function. */
+ * (the tcgen05 tensor-memory kernel for head_dim 128, G*(k+1) <= 64 rows padded to 16, 32
+ * or 64; the mma.sync kernel for head_dim 64), 1 = always the mma.sync kernel. Both
+ * compute the same function. */
 S3R_API int s3r_set_verify_kernel(int32_t which);
 
 /* Bound, in polls, on every wait of the tcgen05 verify kernel's roles for one another's

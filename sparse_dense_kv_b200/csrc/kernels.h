@@ -9,7 +9,7 @@
 namespace s3r {
 
 constexpr int kVerifyChunk = 1024;   // positions per verify CTA (multiple of 64)
-constexpr int kVerifyChunkMin = 896; // smallest verify chunk of any kernel (workspace sizing)
+constexpr int kVerifyChunkMin = 384; // smallest verify chunk of any kernel (workspace sizing)
 constexpr int kDraftChunk = 512;     // positions per draft CTA (multiple of 128)
 constexpr int kVocabChunk = 8192;    // vocabulary entries per sampler CTA
 
@@ -118,11 +118,12 @@ int launch_verify_combine(const VerifyParams& p, int D, int batch, cudaStream_t 
 // Whether the chunk merge of a verify with these chunk counts fits in shared memory.
 bool verify_combine_fits(int nchunk_max, int R);
 
-// tcgen05 verify (head_dim 128, G*(k+1) <= 32 rows; batches beyond the per-launch request
+// tcgen05 verify (head_dim 128, G*(k+1) <= 64 rows; batches beyond the per-launch request
 // table are split into several launches)
 bool verify_tc_supported(int D, int R, int batch);
 int verify_tc_npad(int R);
 int verify_tc_chunk(int R);
+int verify_tc_rec_rows(int R);   // row pitch of its chunk records
 int launch_verify_tc(const CUtensorMap& qm, const CUtensorMap& k1, const CUtensorMap& v1,
                      const CUtensorMap& k8, const CUtensorMap& v8, const VerifyParams& p,
                      int batch, int num_sms, cudaStream_t stream, int* launches);

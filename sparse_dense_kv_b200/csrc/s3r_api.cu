@@ -345,7 +345,7 @@ int s3r_verify_attn(const s3r_kv_cache* cache, const s3r_batch* batch, int32_t k
     if (!verify_combine_fits((cap + chunk - 1) / chunk, R)) return S3R_ERR_UNSUPPORTED;
   }
   if (tc) {
-    p.Rp = verify_tc_npad(R);
+    p.Rp = verify_tc_rec_rows(R);
     p.chunk = verify_tc_chunk(R);
     p.nchunk_max = (cap + p.chunk - 1) / p.chunk;
     CUtensorMap k1, v1, k8, v8, qm;

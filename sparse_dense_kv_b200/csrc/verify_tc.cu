@@ -1,5 +1,6 @@
 // Dense verify attention with score capture on the 5th-generation tensor cores (tcgen05,
-// accumulators in tensor memory), head_dim 128, up to 32 rows per KV head.
+// accumulators in tensor memory), head_dim 128, up to 64 rows per KV head (padded to 16, 32
+// or 64 rows: N of both products).
 //
 // What it computes is what verify.cu computes ([News] Interpretation: the proposed block is
 // recomputed against the complete historical KV; [Explainer] walkthrough: the sparse set
@@ -7,7 +8,8 @@
 // positions 0..L+t; out, lse and every committed logit are written.
 //
 // Organisation (one persistent CTA per SM, 11 warps). A work item is (request, KV head,
-// chunk of up to 7 or 8 tiles of 128 positions). Items are claimed from a counter in the
+// chunk of up to 8, 7 or 3 tiles of 128 positions at 16, 32 or 64 rows: two S buffers of a
+// chunk and two O buffers fill the 512 columns of tensor memory). Items are claimed from a counter in the
 // workspace as CTAs progress (the K producer claims, a ring in shared memory tells the
 // other roles), so faster SMs take more of them.
 //   warp 0     K producer: per item it loads the item's Q rows into one of two Q buffers
@@ -22,8 +24,8 @@
 //              K_t . Q^T into tensor memory for the QK of item m, and O^T (128 d x N) +=
 //              V_t^T . P_t^T for the PV of item n < m; whichever has its next tile ready is
 //              issued. K and Q are K-major operands (128-byte swizzle); V^T is MN-major (the V
-//              tile as it arrives) and so is P^T (one row of N values per position, 32- or
-//              64-byte swizzle). S and O are double-buffered in tensor memory.
+//              tile as it arrives) and so is P^T (one row of N values per position, 32-,
+//              64- or 128-byte swizzle). S and O are double-buffered in tensor memory.
 //   warps 3-10 softmax / epilogue, two warpgroups each owning half of the rows (one thread
 //              per tensor-memory lane = position or d): pass 1 reads every S tile, writes the
 //              committed logits and takes the chunk maximum per row; pass 2 re-reads them and
@@ -152,14 +154,14 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool 
 
 template <int NP>
 struct Cfg {
-  static constexpr int kTiles = NP == 32 ? 7 : 8;            // tiles per chunk
+  static constexpr int kTiles = NP == 64 ? 3 : (NP == 32 ? 7 : 8);   // tiles per chunk
   static constexpr int kKSt = 2;                             // K ring stages
   static constexpr int kVSt = 2;                             // V ring stages
   static constexpr int kChunk = kTiles * kPos;
   static constexpr int kQBytes = 2 * NP * 128;               // one Q buffer: [2 halves][NP rows][128 B]
   static constexpr int kPTile = kPos * NP * 2;               // P^T tile: [128 pos][NP rows] bf16
   static constexpr int kPBytes = kTiles * kPTile;
-  static constexpr uint32_t kPSwz = NP == 16 ? 6u : 4u;      // 32- / 64-byte swizzle
+  static constexpr uint32_t kPSwz = NP == 16 ? 6u : (NP == 32 ? 4u : 2u);   // 32- / 64- / 128-byte swizzle
   static constexpr int kTmemCols = 512;
   static constexpr int kSCols = kTiles * NP;                 // one S buffer
   static constexpr int kOCol = 2 * kSCols;                   // two O buffers after two S buffers
@@ -669,7 +671,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Warpgroup sg owns rows (columns of S and O^T) [sg*NH, sg*NH + NH) of every tile; the
     // two warpgroups only meet at the chunk's barriers for the MMA warp.
     constexpr int NH = NP / 2;               // rows per warpgroup
-    constexpr int BT = NP == 32 ? 2 : 4;     // tiles per tensor-memory wait (no spills)
+    constexpr int BT = NP == 64 ? 1 : (NP == 32 ? 2 : 4);   // tiles per tensor-memory wait (no spills)
     const int sw8 = warp - kSoftWarp0;       // 0..7
     const int sg = sw8 >> 2;                 // warpgroup
     const int sw4 = sw8 & 3;                 // warp within the warpgroup
@@ -679,7 +681,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int c0 = sg * NH;                  // first row of this warpgroup
     const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
     const float scale = p.scale, scale2 = p.scale * kLog2e;
-    const int swz_row = (NP == 16) ? ((lrow >> 2) & 1) : ((lrow >> 1) & 3);
+    // the row's 16-byte chunk is XORed with address bits 7.. of its P^T row (32-, 64-, 128-byte swizzle)
+    const int swz_row = (NP == 16) ? ((lrow >> 2) & 1) : (NP == 32 ? ((lrow >> 1) & 3) : (lrow & 7));
     // Warpgroup barrier on an mbarrier (bounded wait, unlike bar.sync): if a wait anywhere
     // gives up, the other warps of the group give up here too instead of hanging.
     uint32_t wg_phase = 0;
@@ -701,12 +704,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       float o[NH];
       tmem_ld_cols<NH>(tl + C::kOCol + (m & 1) * NP + c0, o);
       tmem_wait_ld();
+      // records hold the R real rows (row pitch p.Rp >= R)
 #pragma unroll
-      for (int j = 0; j < NH; ++j) rec[2 * p.Rp + (size_t)(c0 + j) * kD + lrow] = o[j];
+      for (int j = 0; j < NH; ++j)
+        if (c0 + j < R) rec[2 * p.Rp + (size_t)(c0 + j) * kD + lrow] = o[j];
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&B->o_empty[m & 1]));
-      if (gt < NH) {
+      if (gt < NH && c0 + gt < R) {
         rec[c0 + gt] = cm[(m & 1) * NP + c0 + gt];
         rec[p.Rp + c0 + gt] = cl[(m & 1) * NP + c0 + gt];
       }
@@ -895,7 +900,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace tc
 
-int verify_tc_npad(int R) { return R <= 16 ? 16 : (R <= 32 ? 32 : 0); }
+int verify_tc_npad(int R) { return R <= 16 ? 16 : (R <= 32 ? 32 : (R <= 64 ? 64 : 0)); }
 
 template <int NP>
 static int launch_tc(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
@@ -917,7 +922,15 @@ bool verify_tc_supported(int D, int R, int /*batch*/) {
 
 int verify_tc_chunk(int R) {
   const int np = verify_tc_npad(R);
-  return np == 16 ? tc::Cfg<16>::kChunk : tc::Cfg<32>::kChunk;
+  return np == 16 ? tc::Cfg<16>::kChunk : (np == 32 ? tc::Cfg<32>::kChunk : tc::Cfg<64>::kChunk);
+}
+
+// Row pitch of the chunk records: the padded rows for 16 / 32 (as the merge has always read
+// them), the real rows (rounded to 4 for 16-byte loads) for 64, where padding would add a
+// third to the records' traffic.
+int verify_tc_rec_rows(int R) {
+  const int np = verify_tc_npad(R);
+  return np == 64 ? (R + 3) / 4 * 4 : np;
 }
 
 int launch_verify_tc(const CUtensorMap& qm, const CUtensorMap& k1, const CUtensorMap& v1,
@@ -925,15 +938,16 @@ int launch_verify_tc(const CUtensorMap& qm, const CUtensorMap& k1, const CUtenso
                      int batch, int num_sms, cudaStream_t stream, int* launches) {
   const int np = verify_tc_npad(p.R);
   *launches = 0;
-  if (np != 16 && np != 32) return S3R_ERR_UNSUPPORTED;
+  if (np != 16 && np != 32 && np != 64) return S3R_ERR_UNSUPPORTED;
   // the per-launch request tables hold kMaxBatch requests; a larger batch is several
   // launches over consecutive slices of it (each chunk record still lands in its slot)
   for (int b0 = 0; b0 < batch; b0 += tc::kMaxBatch) {
     VerifyParams q = p;
     q.req_off = p.req_off + b0;
     const int nb = batch - b0 < tc::kMaxBatch ? batch - b0 : tc::kMaxBatch;
-    const int st = np == 16 ? launch_tc<16>(qm, k1, v1, k8, v8, q, nb, num_sms, stream)
-                            : launch_tc<32>(qm, k1, v1, k8, v8, q, nb, num_sms, stream);
+    const int st = np == 16   ? launch_tc<16>(qm, k1, v1, k8, v8, q, nb, num_sms, stream)
+                   : np == 32 ? launch_tc<32>(qm, k1, v1, k8, v8, q, nb, num_sms, stream)
+                              : launch_tc<64>(qm, k1, v1, k8, v8, q, nb, num_sms, stream);
     if (st != S3R_OK) return st;
     ++*launches;
   }
