@@ -351,6 +351,24 @@ S3R_API int s3r_choose_horizon(const double* accepted, const double* decided, in
                        double c_draft, double c_verify, double prior_alpha,
                        double prior_weight, int32_t* k_out);
 
+/* One decision of the adaptive draft length from the commit counters (HOST function, no
+ * device work; [Wispaper] position-dependent acceptance). With the counters of s3r_commit
+ * now and at the last decision (host int64 [2 + 2*S3R_MAX_K] each, that layout), for every
+ * position j < S3R_MAX_K, in double:
+ *   accepted[j] = decay * accepted[j] + (stats_now[2+j] - stats_last[2+j])
+ *   decided[j]  = decay * decided[j]  + (stats_now[2+S3R_MAX_K+j] - stats_last[2+S3R_MAX_K+j])
+ * then stats_last = stats_now; the prior is prior_alpha, or (prior_alpha < 0) the acceptance
+ * pooled over positions j < k_max, sum accepted / sum decided added in position order (0.5
+ * when nothing was decided), written to *prior_out (may be NULL); *k_out is then what
+ * s3r_choose_horizon picks from accepted / decided [0, k_max) with that prior.
+ *   accepted, decided  host double [S3R_MAX_K], the caller's decayed counts (start at 0).
+ * S3R_ERR_INVALID_ARG for NULL pointers, decay outside [0, 1], a counter that went down, or
+ * any argument s3r_choose_horizon rejects (then nothing is updated). */
+S3R_API int s3r_horizon_step(const int64_t* stats_now, int64_t* stats_last, double* accepted,
+                     double* decided, int32_t k_max, double decay, double c_draft,
+                     double c_verify, double prior_alpha, double prior_weight,
+                     double* prior_out, int32_t* k_out);
+
 /* Philox4x32-10 words and uniforms for n counters (position[i], request[i], stream_id, 0)
  * under key = seed: words uint32 [n][4] (may be NULL), u fp32 [n] (may be NULL). */
 S3R_API int s3r_philox(uint64_t seed, int32_t stream_id, const int32_t* request, const int32_t* position,

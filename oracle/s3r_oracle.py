@@ -555,6 +555,35 @@ def choose_horizon(accepted, decided, c_draft: float, c_verify: float, k_max: in
     return best_k
 
 
+def horizon_update(acc, dec, accepted_new, decided_new, decay: float):
+    """Decayed counts per position: acc_j <- decay * acc_j + accepted_new_j, the same for the
+    decided counts (positions that stop being drafted fade toward the prior)."""
+    acc = [decay * float(a) + float(n) for a, n in zip(acc, accepted_new)]
+    dec = [decay * float(d) + float(n) for d, n in zip(dec, decided_new)]
+    return acc, dec
+
+
+def pooled_prior(acc, dec, k_max: int, default: float = 0.5) -> float:
+    """Acceptance pooled over positions 1..k_max (the plain expectation for a position with
+    no evidence of its own): sum of accepted / sum of decided, summed in position order;
+    `default` when nothing was decided."""
+    sa, sd = 0.0, 0.0
+    for j in range(k_max):
+        sa += float(acc[j])
+        sd += float(dec[j])
+    return sa / sd if sd > 0 else default
+
+
+def horizon_step(acc, dec, accepted_new, decided_new, decay: float, c_draft: float,
+                 c_verify: float, k_max: int, prior_alpha=None, prior_weight: float = 4.0):
+    """One decision of the adaptive draft length: decay the counts, add the new ones, take
+    the prior (pooled when prior_alpha is None) and choose k. Returns (acc, dec, prior, k)."""
+    acc, dec = horizon_update(acc, dec, accepted_new, decided_new, decay)
+    prior = pooled_prior(acc, dec, k_max) if prior_alpha is None else float(prior_alpha)
+    return acc, dec, prior, choose_horizon(acc[:k_max], dec[:k_max], c_draft, c_verify, k_max, prior,
+                                           prior_weight)
+
+
 def break_even_acceptance(total_ms: float, ar_ms: float, k: int) -> float:
     """Acceptance at which a round (draft + verify = total) costs as much per token as AR.
 

@@ -23,6 +23,7 @@ from ._lib import (  # noqa: F401
     s3r_draft_sample_noalloc,
     s3r_get_error,
     s3r_greedy_verify,
+    s3r_horizon_step,
     s3r_launch_count,
     s3r_philox,
     s3r_select_from_scores,

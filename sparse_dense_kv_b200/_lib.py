@@ -86,6 +86,8 @@ def _load():
                                               ctypes.c_int64]),
         "s3r_choose_horizon": (ctypes.c_int, [P, P, I32, ctypes.c_double, ctypes.c_double,
                                               ctypes.c_double, ctypes.c_double, P]),
+        "s3r_horizon_step": (ctypes.c_int, [P, P, P, P, I32, ctypes.c_double, ctypes.c_double,
+                                            ctypes.c_double, ctypes.c_double, ctypes.c_double, P, P]),
         "s3r_greedy_verify": (ctypes.c_int, [B, I32, P, P, I32, P, P, P, SZ, P]),
         "s3r_commit": (ctypes.c_int, [B, I32, P, P, P, P]),
         "s3r_philox": (ctypes.c_int, [U64, I32, P, P, I64, P, P, P]),
@@ -341,6 +343,27 @@ def s3r_choose_horizon(accepted, decided, c_draft, c_verify, prior_alpha=0.5, pr
                                    float(prior_weight), ctypes.cast(ctypes.pointer(out), ctypes.c_void_p)),
            "s3r_choose_horizon")
     return int(out.value)
+
+
+def s3r_horizon_step(stats_now, stats_last, accepted, decided, k_max, decay, c_draft, c_verify,
+                     prior_alpha=-1.0, prior_weight=4.0):
+    """Host call: decay / add the counts and choose k. stats_now, stats_last: numpy int64
+    [2 + 2*MAX_K] (stats_last is updated); accepted, decided: numpy float64 [MAX_K] (updated).
+    prior_alpha < 0 pools the prior. Returns (k, prior used)."""
+    import numpy as np
+    now = np.ascontiguousarray(stats_now, dtype=np.int64)
+    for a, dt in ((stats_last, np.int64), (accepted, np.float64), (decided, np.float64)):
+        if not (isinstance(a, np.ndarray) and a.dtype == dt and a.flags.c_contiguous):
+            raise TypeError("stats_last / accepted / decided must be contiguous numpy arrays")
+    if now.size != 2 + 2 * MAX_K or stats_last.size != now.size or accepted.size != MAX_K or decided.size != MAX_K:
+        raise ValueError("counter arrays of the s3r_commit layout")
+    k, prior = ctypes.c_int32(0), ctypes.c_double(0.0)
+    vp = lambda a: a.ctypes.data_as(ctypes.c_void_p)  # noqa: E731
+    _check(_lib.s3r_horizon_step(vp(now), vp(stats_last), vp(accepted), vp(decided), k_max, float(decay),
+                                 float(c_draft), float(c_verify), float(prior_alpha), float(prior_weight),
+                                 ctypes.cast(ctypes.pointer(prior), ctypes.c_void_p),
+                                 ctypes.cast(ctypes.pointer(k), ctypes.c_void_p)), "s3r_horizon_step")
+    return int(k.value), float(prior.value)
 
 
 def s3r_sched_simulate(prompt_len, resp_len, tau, *, capacity, policy="aimd", evict="offload",

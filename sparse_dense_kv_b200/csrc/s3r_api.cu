@@ -745,6 +745,42 @@ int s3r_choose_horizon(const double* accepted, const double* decided, int32_t k_
   return S3R_OK;
 }
 
+int s3r_horizon_step(const int64_t* stats_now, int64_t* stats_last, double* accepted,
+                     double* decided, int32_t k_max, double decay, double c_draft,
+                     double c_verify, double prior_alpha, double prior_weight,
+                     double* prior_out, int32_t* k_out) {
+  if (!stats_now || !stats_last || !accepted || !decided || !k_out) return S3R_ERR_INVALID_ARG;
+  if (k_max < 1 || k_max > S3R_MAX_K || !(decay >= 0.0 && decay <= 1.0)) return S3R_ERR_INVALID_ARG;
+  double acc[S3R_MAX_K], dec[S3R_MAX_K];
+  for (int j = 0; j < S3R_MAX_K; ++j) {
+    const int64_t da = stats_now[2 + j] - stats_last[2 + j];
+    const int64_t dd = stats_now[2 + S3R_MAX_K + j] - stats_last[2 + S3R_MAX_K + j];
+    if (da < 0 || dd < 0) return S3R_ERR_INVALID_ARG;
+    acc[j] = decay * accepted[j] + (double)da;
+    dec[j] = decay * decided[j] + (double)dd;
+  }
+  double prior = prior_alpha;
+  if (prior_alpha < 0.0) {
+    double sa = 0.0, sd = 0.0;
+    for (int j = 0; j < k_max; ++j) {
+      sa += acc[j];
+      sd += dec[j];
+    }
+    prior = sd > 0.0 ? sa / sd : 0.5;
+  }
+  int32_t k = 0;
+  const int st = s3r_choose_horizon(acc, dec, k_max, c_draft, c_verify, prior, prior_weight, &k);
+  if (st != S3R_OK) return st;
+  for (int j = 0; j < S3R_MAX_K; ++j) {
+    accepted[j] = acc[j];
+    decided[j] = dec[j];
+  }
+  for (int j = 0; j < 2 + 2 * S3R_MAX_K; ++j) stats_last[j] = stats_now[j];
+  if (prior_out) *prior_out = prior;
+  *k_out = k;
+  return S3R_OK;
+}
+
 int s3r_philox(uint64_t seed, int32_t stream_id, const int32_t* request, const int32_t* position,
                int64_t n, uint32_t* words, float* u, s3r_stream_t stream) {
   if (n < 0 || (n > 0 && (!request || !position))) return S3R_ERR_INVALID_ARG;

@@ -359,42 +359,32 @@ class MixedPhaseDriver:
 
 
 class AdaptiveHorizon:
-    """Draft length from the measured acceptance by position: the engine's counters are read
-    every call of step() (one device-to-host copy), added to exponentially decayed counts,
-    and s3r_choose_horizon picks the k with the most expected tokens per unit round cost
-    (c_draft per draft step, c_verify for the rest of the round). Positions not drafted for
-    a while decay toward the prior, so longer horizons are tried again when it is good; with
-    prior_alpha="pooled" the prior is the acceptance pooled over all positions so far (the
-    plain expectation for a position without evidence of its own)."""
+    """Draft length from the measured acceptance by position: every call of step() reads the
+    engine's counters (one device-to-host copy) and s3r_horizon_step decays the kept counts,
+    adds the new ones, takes the prior and picks the k with the most expected tokens per unit
+    round cost (c_draft per draft step, c_verify for the rest of the round). Positions not
+    drafted for a while decay toward the prior, so longer horizons are tried again when it is
+    good; with prior_alpha="pooled" the prior is the acceptance pooled over all positions so
+    far (the plain expectation for a position without evidence of its own)."""
 
     def __init__(self, engine: S3REngine, c_draft: float, c_verify: float, *, decay: float = 0.8,
                  prior_alpha="pooled", prior_weight: float = 4.0, k_max: int | None = None):
+        import numpy as np
         self.e = engine
         self.c_draft, self.c_verify = c_draft, c_verify
         self.decay, self.prior_alpha, self.prior_weight = decay, prior_alpha, prior_weight
         self.k_max = k_max or engine.buf.k_max
-        self.acc = [0.0] * L.MAX_K
-        self.dec = [0.0] * L.MAX_K
-        self.last = engine.buf.stats.cpu().tolist()
+        self.acc = np.zeros(L.MAX_K, dtype=np.float64)
+        self.dec = np.zeros(L.MAX_K, dtype=np.float64)
+        self.last = engine.buf.stats.cpu().numpy().astype(np.int64)
+        self.last_prior = None
         self.history = []
 
-    def observe(self):
-        st = self.e.buf.stats.cpu().tolist()
-        for j in range(L.MAX_K):
-            self.acc[j] = self.decay * self.acc[j] + (st[2 + j] - self.last[2 + j])
-            self.dec[j] = self.decay * self.dec[j] + (st[2 + L.MAX_K + j] - self.last[2 + L.MAX_K + j])
-        self.last = st
-
-    def prior(self) -> float:
-        if self.prior_alpha != "pooled":
-            return float(self.prior_alpha)
-        d = sum(self.dec[: self.k_max])
-        return sum(self.acc[: self.k_max]) / d if d > 0 else 0.5
-
     def step(self) -> int:
-        self.observe()
-        k = L.s3r_choose_horizon(self.acc[: self.k_max], self.dec[: self.k_max], self.c_draft,
-                                 self.c_verify, self.prior(), self.prior_weight)
+        now = self.e.buf.stats.cpu().numpy()
+        pa = -1.0 if self.prior_alpha == "pooled" else float(self.prior_alpha)
+        k, self.last_prior = L.s3r_horizon_step(now, self.last, self.acc, self.dec, self.k_max, self.decay,
+                                                self.c_draft, self.c_verify, pa, self.prior_weight)
         self.e.set_k(k)
         self.history.append(k)
         return k

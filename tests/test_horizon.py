@@ -64,15 +64,55 @@ class _FakeEngine:
             self.buf.stats[2 + s3r.MAX_K + j] += d
 
 
+@pytest.mark.parametrize("seed", range(200))
+def test_horizon_step_matches_oracle(seed):
+    """The library's decay, pooled prior and choice against the oracle's, in double, on
+    random counters, decays, costs and priors."""
+    rng = np.random.default_rng(1000 + seed)
+    M = s3r.MAX_K
+    k_max = int(rng.integers(1, M + 1))
+    acc0 = np.floor(rng.random(M) * 50) * (seed % 2) + 0.0
+    dec0 = acc0 + np.floor(rng.random(M) * 30) + 0.0
+    last = np.zeros(2 + 2 * M, dtype=np.int64)
+    last[2: 2 + M] = rng.integers(0, 100, M)
+    last[2 + M:] = last[2: 2 + M] + rng.integers(0, 50, M)
+    now = last.copy()
+    new_a = rng.integers(0, 60, M)
+    now[2: 2 + M] += new_a
+    now[2 + M:] += new_a + rng.integers(0, 40, M)
+    decay = float(rng.choice([0.0, 0.5, 0.8, 1.0]))
+    c_d, c_v = float(rng.uniform(1, 100)), float(rng.uniform(1, 2000))
+    pa = None if seed % 3 else float(rng.uniform(0, 1))
+    oa, od, oprior, ok = O.horizon_step(acc0.tolist(), dec0.tolist(), (now - last)[2: 2 + M].tolist(),
+                                        (now - last)[2 + M:].tolist(), decay, c_d, c_v, k_max, pa, 4.0)
+    acc, dec, lst = acc0.copy(), dec0.copy(), last.copy()
+    k, prior = s3r.s3r_horizon_step(now, lst, acc, dec, k_max, decay, c_d, c_v, -1.0 if pa is None else pa, 4.0)
+    assert (k, prior) == (ok, oprior)
+    assert acc.tolist() == oa and dec.tolist() == od and lst.tolist() == now.tolist()
+
+
+def test_horizon_step_rejects_bad_arguments_and_leaves_state():
+    M = s3r.MAX_K
+    now = np.zeros(2 + 2 * M, dtype=np.int64)
+    last = now.copy()
+    last[2] = 5                                   # a counter that went down
+    acc, dec = np.ones(M), np.ones(M)
+    with pytest.raises(s3r.S3RError):
+        s3r.s3r_horizon_step(now, last, acc, dec, 4, 0.5, 1.0, 1.0)
+    assert last[2] == 5 and acc.tolist() == [1.0] * M
+    with pytest.raises(s3r.S3RError):
+        s3r.s3r_horizon_step(now, now.copy(), acc, dec, 4, 1.5, 1.0, 1.0)   # decay > 1
+
+
 def test_controller_decays_counts_and_pools_the_prior():
     eng = _FakeEngine(6)
     ctl = s3r.AdaptiveHorizon(eng, c_draft=57.0, c_verify=730.0, decay=0.5, prior_weight=4.0)
     eng.commit([80, 60, 40, 0, 0, 0], [100, 80, 60, 0, 0, 0])
     k1 = ctl.step()
-    assert ctl.acc[:3] == [80.0, 60.0, 40.0] and ctl.dec[:3] == [100.0, 80.0, 60.0]
+    assert ctl.acc[:3].tolist() == [80.0, 60.0, 40.0] and ctl.dec[:3].tolist() == [100.0, 80.0, 60.0]
     pooled = 180.0 / 240.0
-    assert ctl.prior() == pooled
-    want = O.choose_horizon(ctl.acc[:6], ctl.dec[:6], 57.0, 730.0, 6, pooled, 4.0)
+    assert ctl.last_prior == pooled
+    want = O.choose_horizon(ctl.acc[:6].tolist(), ctl.dec[:6].tolist(), 57.0, 730.0, 6, pooled, 4.0)
     assert k1 == want == eng.k
     # a second window halves the first and adds the new counts
     eng.commit([10, 0, 0, 0, 0, 0], [20, 0, 0, 0, 0, 0])

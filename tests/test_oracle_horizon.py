@@ -54,3 +54,22 @@ def test_prior_fills_undecided_positions():
     assert abs(est[0] - (90 + 2) / 104) < 1e-15
     # with a pessimistic prior the extra positions are not worth drafting
     assert O.choose_horizon(acc, dec, 57.0, 730.0, 8, prior_alpha=0.0, prior_weight=4.0) <= 6
+
+
+def test_decayed_counts_and_pooled_prior_hand_worked():
+    # decay 1/2: accepted (4, 2) -> (4/2 + 2, 2/2 + 0) = (4, 1); decided (8, 8) -> (6, 6)
+    acc, dec, prior, k = O.horizon_step([4.0, 2.0], [8.0, 8.0], [2, 0], [2, 2], 0.5, 1.0, 4.0, 2,
+                                        prior_alpha=None, prior_weight=4.0)
+    assert acc == [4.0, 1.0] and dec == [6.0, 6.0]
+    assert prior == 5.0 / 12.0                      # (4 + 1) / (6 + 6)
+    # alpha = ((4 + 4 * 5/12) / 10, (1 + 4 * 5/12) / 10) = (17/30, 8/30)
+    # c_draft 1, c_verify 4: k=1 (47/30)/5 = .31333 > k=2 (1546/900)/6 = .28630
+    assert k == 1
+    # c_verify 40: k=1 (47/30)/41 = .038211 < k=2 (1546/900)/42 = .040899
+    assert O.horizon_step([4.0, 2.0], [8.0, 8.0], [2, 0], [2, 2], 0.5, 1.0, 40.0, 2)[3] == 2
+    # a fixed prior replaces the pooled one; decay 1 keeps every count
+    acc, dec, prior, _ = O.horizon_step([4.0, 2.0], [8.0, 8.0], [2, 0], [2, 2], 1.0, 1.0, 4.0, 2,
+                                        prior_alpha=0.25)
+    assert acc == [6.0, 2.0] and dec == [10.0, 10.0] and prior == 0.25
+    # nothing decided yet: the pooled prior is one half
+    assert O.pooled_prior([0.0] * 4, [0.0] * 4, 4) == 0.5
