@@ -216,9 +216,9 @@ S3R_API int s3r_draft_sample(const s3r_batch* batch, const int32_t* draft_step, 
  * point of the call: a host program that drives the library from plain C without an
  * allocator of its own, or a server that has given all free HBM to the KV pool and must
  * not allocate between rounds. Same arguments, arithmetic and outputs as
- * s3r_draft_sample (without margins), bit for bit; the scratch (arrival tickets and
- * per-chunk partials) lives in a static device array inside the library, 8 KiB + 1 MiB
- * per device that loads the library, held until the process exits, so
+ * s3r_draft_sample (without margins), bit for bit; the scratch (arrival tickets, per-chunk
+ * partials and sub-block sums) lives in a static device array inside the library, 8 KiB +
+ * 3 MiB per device that loads the library, held until the process exits, so
  *   - num_requests <= S3R_NOALLOC_MAX_REQUESTS and vocab <= S3R_NOALLOC_MAX_VOCAB, else
  *     S3R_ERR_UNSUPPORTED with a message in s3r_last_error_message() and no launch;
  *   - err_word (device int32, caller-owned, zeroed by the caller before first use)

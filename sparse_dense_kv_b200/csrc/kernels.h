@@ -103,6 +103,7 @@ struct SampleParams {
   int* tickets;
   uint8_t* part;
   size_t plan_off, draw_off;   // spec sampling: byte offsets of the plans / draw partials
+  size_t sub_off;              // byte offset of the sub-block sums (draft or spec draw)
   int num_requests;            // size of every per-request array (request ids are checked)
   float* margins;              // optional: draft [NR][k], spec [NR][k+1] decision margins
 };
@@ -142,7 +143,9 @@ int launch_argmax(const SampleParams& p, int batch, int mode, cudaStream_t strea
 // Bytes of one per-(request, vocabulary chunk) partial of the samplers.
 constexpr int kSamplePartialBytes = 16;
 size_t sample_partial_bytes(int num_requests, int k, int vocab);
-void spec_offsets(int num_requests, int k, int vocab, size_t* plan_off, size_t* draw_off);
+void spec_offsets(int num_requests, int k, int vocab, size_t* plan_off, size_t* draw_off, size_t* sub_off);
+// Byte offset of draft sampling's sub-block sums in its partials area.
+size_t draft_sub_offset(int num_requests, int vocab);
 
 int launch_commit(const int32_t* req_ids, int batch, int k, const int32_t* n_out,
                   int32_t* seq_lens, int64_t* stats, cudaStream_t stream);

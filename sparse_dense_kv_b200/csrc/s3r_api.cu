@@ -213,14 +213,16 @@ size_t sample_need(int num_requests, int hkv, int k, int vocab) {
 
 // ---------------------------------------------------- draft sampling without a workspace
 // Scratch of s3r_draft_sample_noalloc, a file-scope device array instead of a caller's
-// workspace: one arrival ticket per request (must start at zero; the last block of a
-// request puts it back to zero) followed by one partial record per (request, vocabulary
-// chunk). It is sized for S3R_NOALLOC_MAX_REQUESTS requests and vocabularies of at most
-// S3R_NOALLOC_MAX_VOCAB entries: 8 KiB of tickets + 1 MiB of partials per device.
+// workspace: one arrival ticket per request (cleared by every call for its requests; the
+// last block of a request puts it back to zero) followed by one partial record per
+// (request, vocabulary chunk) and the eight sub-block sums of each chunk. It is sized for
+// S3R_NOALLOC_MAX_REQUESTS requests and vocabularies of at most S3R_NOALLOC_MAX_VOCAB
+// entries: 8 KiB of tickets + 1 MiB of partials + 2 MiB of sub-block sums per device.
 constexpr int kNoAllocChunks = S3R_NOALLOC_MAX_VOCAB / kVocabChunk;
 constexpr size_t kNoAllocTicketBytes = (size_t)S3R_NOALLOC_MAX_REQUESTS * sizeof(int);
 constexpr size_t kNoAllocBytes =
-    kNoAllocTicketBytes + (size_t)S3R_NOALLOC_MAX_REQUESTS * kNoAllocChunks * kSamplePartialBytes;
+    kNoAllocTicketBytes + (size_t)S3R_NOALLOC_MAX_REQUESTS * kNoAllocChunks * kSamplePartialBytes +
+    (size_t)S3R_NOALLOC_MAX_REQUESTS * kNoAllocChunks * 8 * sizeof(float);
 static_assert(S3R_NOALLOC_MAX_VOCAB % kVocabChunk == 0, "whole vocabulary chunks");
 static_assert(kNoAllocTicketBytes % 256 == 0, "partials start 256-byte aligned");
 
@@ -557,6 +559,7 @@ int s3r_draft_sample(const s3r_batch* batch, const int32_t* draft_step, int32_t 
   p.part = w.part;
   p.num_requests = batch->num_requests;
   p.margins = margins;
+  p.sub_off = draft_sub_offset(batch->num_requests, vocab);
   return finish(launch_draft_sample(p, batch->batch, (cudaStream_t)stream), 1);
 }
 
@@ -595,6 +598,7 @@ int s3r_draft_sample_noalloc(const s3r_batch* batch, const int32_t* draft_step, 
   p.tickets = reinterpret_cast<int*>(scratch);
   p.part = scratch + kNoAllocTicketBytes;
   p.num_requests = batch->num_requests;
+  p.sub_off = draft_sub_offset(batch->num_requests, vocab);
   // the tickets of this call's requests start at zero whatever an earlier call left there,
   // cleared on the call's own stream (so ordered with the launch below)
   S3R_TRY(cuda_status(cudaMemsetAsync(scratch, 0, (size_t)batch->num_requests * sizeof(int),
@@ -635,7 +639,7 @@ int s3r_spec_sample(const s3r_batch* batch, int32_t k, const float* p_logits,
   p.part = w.part;
   p.num_requests = batch->num_requests;
   p.margins = margins;
-  spec_offsets(batch->num_requests, k, vocab, &p.plan_off, &p.draw_off);
+  spec_offsets(batch->num_requests, k, vocab, &p.plan_off, &p.draw_off, &p.sub_off);
   int launches = 0;
   const int st = launch_spec_sample(p, batch->batch, (cudaStream_t)stream, &launches);
   if (st != S3R_OK && launches == 0) return st;

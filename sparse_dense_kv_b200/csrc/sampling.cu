@@ -7,9 +7,11 @@
 //
 // The vocabulary is split into chunks of 8192 entries. A pass over (chunk, row, request)
 // produces (max, sum exp(x - max)) per chunk with fp32 exponentials and fp64 sums; the last
-// CTA of a request merges the chunks (ticket, no spinning) and decides. A draw first finds
-// the chunk holding u * Z from the chunk sums, then the warp holding it (warp totals in
-// order), then, inside that warp's 1024 entries, the row of 32 and the entry.
+// CTA of a request merges the chunks (ticket, no spinning) and decides. For a draw the pass
+// also writes the sums of the chunk's eight sub-blocks of 1024 entries, so the last CTA
+// finds the chunk and then the sub-block holding u * Z from sums alone, and reads and
+// searches only that sub-block's 1024 logits (one 16-byte load per thread, a block-wide
+// prefix sum in fp64).
 #include <climits>
 
 #include "common.cuh"
@@ -125,296 +127,255 @@ __device__ __forceinline__ float merge_partials_warp(const MS* part, int nvch, d
   return M;
 }
 
-__device__ double block_sum_d(double v) {
-  __shared__ double sd[kSampThreads / 32];
-  __shared__ double tot;
+// ----------------------------------------------------------------- sub-block draws ----
+constexpr int kSub = 1024;                     // entries per sub-block sum
+constexpr int kSubPer = kVocabChunk / kSub;    // sub-blocks per vocabulary chunk (8)
+static_assert(kSub == 4 * kSampThreads, "one 16-byte load of a sub-block per thread");
+
+// Sum over the block of each thread's kSubPer values; out[0..kSubPer) valid after return
+// in every thread (fp32 warp sums, fp32 across the warps).
+__device__ __forceinline__ void block_sum_sub(float (&v)[kSubPer], float* out) {
+  __shared__ float sw[kSampThreads / 32][kSubPer];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  v = warp_sum_d(v);
-  if (lane == 0) sd[warp] = v;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    double t = 0.0;
-    for (int w = 0; w < kSampThreads / 32; ++w) t += sd[w];
-    tot = t;
+#pragma unroll
+  for (int b = 0; b < kSubPer; ++b) {
+    float x = v[b];
+#pragma unroll
+    for (int o = 16; o; o >>= 1) x += __shfl_xor_sync(kFull, x, o);
+    if (lane == 0) sw[warp][b] = x;
   }
   __syncthreads();
-  const double r = tot;
+  if (threadIdx.x < kSubPer) {
+    float t = 0.f;
+    for (int w = 0; w < kSampThreads / 32; ++w) t += sw[w][threadIdx.x];
+    out[threadIdx.x] = t;
+  }
   __syncthreads();
-  return r;
 }
 
-// Inverse-CDF search inside [v0, v1) (at most kVocabChunk entries): smallest v with
-// target < base + C_v, C the inclusive running sum of weight(v). Warp w takes the 1024
-// entries v0 + 1024 w + 32 m + lane (m = 0..31: coalesced loads, weights kept in
-// registers); the warps' totals, in order, find the warp holding the target; that warp
-// reduces its 32 rows of 32 entries with a butterfly (lane m ends with row m's sum),
-// scans the rows, then the lanes of the chosen row. Returns -1 if the target lies past the
-// chunk; `base` then moves to the chunk's end.
-// `mrg` receives the distance of the target to the nearer edge of the drawn token's cell
-// [C_{v-1}, C_v) (0 where rounding carried the target past the last entry).
-template <class W>
-__device__ int chunk_search(int v0, int v1, double target, double& base, double& mrg, W weight) {
-  __shared__ double wtot_s[kSampThreads / 32];
-  __shared__ int s_tok;
-  __shared__ double s_mrg;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int wb = v0 + warp * 1024;
-  float w[32];
-  float part = 0.f;
-#pragma unroll
-  for (int m = 0; m < 32; ++m) {
-    const int v = wb + 32 * m + lane;
-    w[m] = v < v1 ? weight(v) : 0.f;
-    part += w[m];
-  }
-  const double wt = warp_sum_d((double)part);
-  if (lane == 0) wtot_s[warp] = wt;
+// The draw of the last CTA of a request: target = u * Z on the weights' common scale, the
+// chunk sums csum[0..nvch) (that scale), sub(c, b) the sum of sub-block b of chunk c (that
+// scale). Thread 0 walks the chunk sums, then the chosen chunk's sub-block sums; then every
+// thread takes 4 consecutive entries of the sub-block (weight4(v0, w) fills w[0..3] on the
+// common scale, 0 past the vocabulary), and a block-wide fp64 prefix sum finds the smallest v
+// with target < C_v. `mrg` receives the target's distance to the nearer edge of v's cell
+// (0 where rounding carried the target past the sub-block: its last non-zero entry is taken).
+template <class Sub, class W4>
+__device__ int subblock_draw(int V, int nvch, const double* csum, double target, double& mrg, Sub sub,
+                             W4 weight4) {
+  __shared__ int s_c, s_b, s_tok, s_last;
+  __shared__ double s_base, s_mrg;
+  __shared__ double s_wt[kSampThreads / 32];
   if (threadIdx.x == 0) {
-    s_tok = -1;
+    double cum = 0.0;
+    int c = -1, lastc = -1;
+    for (int i = 0; i < nvch; ++i) {
+      if (csum[i] > 0.0) lastc = i;
+      if (c < 0 && target < cum + csum[i]) c = i;
+      if (c < 0) cum += csum[i];
+    }
+    int b = -1;
+    if (c < 0) {                      // rounding past the last chunk: its last sub-block
+      c = lastc < 0 ? 0 : lastc;
+      cum = 0.0;
+      for (int i = 0; i < c; ++i) cum += csum[i];
+      for (int j = 0; j < kSubPer; ++j)
+        if (sub(c, j) > 0.0) b = j;
+      for (int j = 0; j < b; ++j) cum += sub(c, j);
+    } else {
+      int lastb = 0;
+      for (int j = 0; j < kSubPer && b < 0; ++j) {
+        const double sj = sub(c, j);
+        if (sj > 0.0) lastb = j;
+        if (target < cum + sj) b = j;
+        else cum += sj;
+      }
+      if (b < 0) {                    // rounding past the chunk's last sub-block
+        b = lastb;
+        cum = 0.0;
+        for (int i = 0; i < c; ++i) cum += csum[i];
+        for (int j = 0; j < b; ++j) cum += sub(c, j);
+      }
+    }
+    s_c = c;
+    s_b = b < 0 ? 0 : b;
+    s_base = cum;
+    s_tok = INT_MAX;
+    s_last = -1;
     s_mrg = 0.0;
   }
   __syncthreads();
-  double lo = base, total = 0.0;
-  for (int q = 0; q < kSampThreads / 32; ++q) {
-    if (q < warp) lo += wtot_s[q];
-    total += wtot_s[q];
+  const int v0 = s_c * kVocabChunk + s_b * kSub + 4 * (int)threadIdx.x;
+  double w[4];
+  weight4(v0, w);
+  const double mine = (w[0] + w[1]) + (w[2] + w[3]);
+  // block exclusive prefix of the threads' sums (fp64)
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  double incl = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const double t = __shfl_up_sync(kFull, incl, o);
+    if (lane >= o) incl += t;
   }
-  if (wt > 0.0 && target >= lo && target < lo + wt) {
-    // butterfly (in place): afterwards lane l holds row l's total in w[0]
-#pragma unroll
-    for (int k = 16; k >= 1; k >>= 1) {
-      const bool up = (lane & k) != 0;
-#pragma unroll
-      for (int i = 0; i < k; ++i) {
-        const float send = up ? w[i] : w[i + k];
-        const float keep = up ? w[i + k] : w[i];
-        w[i] = keep + __shfl_xor_sync(kFull, send, k);
-      }
-    }
-    const double rs = w[0];
-    double incl = rs;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const double t = __shfl_up_sync(kFull, incl, o);
-      if (lane >= o) incl += t;
-    }
-    // row: the first with target < lo + (rows up to and including it)
-    const unsigned rowhit = __ballot_sync(kFull, rs > 0.0 && target < lo + incl);
-    int tok = -1;
-    double m = 0.0;
-    if (rowhit) {
-      const int mr = __ffs(rowhit) - 1;
-      const double rbase = lo + __shfl_sync(kFull, incl - rs, mr);
-      const int vx = wb + 32 * mr + lane;   // the row's weights again (same values)
-      const float x = vx < v1 ? weight(vx) : 0.f;
-      double li = x;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const double t = __shfl_up_sync(kFull, li, o);
-        if (lane >= o) li += t;
-      }
-      const unsigned hit = __ballot_sync(kFull, x > 0.f && target < rbase + li);
-      // rounding past the row's last entry: its last non-zero entry
-      const unsigned nz = __ballot_sync(kFull, x > 0.f);
-      const int ln = hit ? __ffs(hit) - 1 : 31 - __clz((int)nz);
-      tok = wb + 32 * mr + ln;
-      const double hi_e = rbase + li, lo_e = hi_e - (double)x;   // the lane's cell
-      const double mine = fmin(target - lo_e, hi_e - target);
-      m = hit ? __shfl_sync(kFull, mine, ln) : 0.0;
-    } else {
-      // rounding past the warp's last row: the last non-zero entry of the warp
-      const unsigned nzr = __ballot_sync(kFull, rs > 0.0);
-      const int mr = 31 - __clz((int)nzr);
-      const int vx = wb + 32 * mr + lane;
-      const float x = vx < v1 ? weight(vx) : 0.f;
-      const unsigned nz = __ballot_sync(kFull, x > 0.f);
-      tok = wb + 32 * mr + (31 - __clz((int)nz));
-    }
-    if (lane == 0) {
-      s_tok = tok;
-      s_mrg = m;
-    }
-  }
+  if (lane == 31) s_wt[warp] = incl;
   __syncthreads();
-  const int tok = s_tok;
-  if (tok >= 0) mrg = s_mrg;
-  base += total;
+  double before = s_base;
+  for (int q = 0; q < warp; ++q) before += s_wt[q];
+  double c0 = before + incl - mine;
+  int last_nz = -1;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    if (w[e] > 0.0) {
+      last_nz = v0 + e;
+      if (target >= c0 && target < c0 + w[e]) {   // cells are disjoint: one entry at most
+        s_tok = v0 + e;
+        s_mrg = fmin(target - c0, c0 + w[e] - target);
+      }
+    }
+    c0 += w[e];
+  }
+  if (last_nz >= 0) atomicMax(&s_last, last_nz);
+  __syncthreads();
+  int tok = s_tok;
+  mrg = s_mrg;
+  if (tok == INT_MAX) {               // rounding past the sub-block: its last non-zero entry
+    tok = s_last >= 0 ? s_last : min(v0, V - 1);
+    mrg = 0.0;
+  }
   __syncthreads();
   return tok;
 }
 
-// Last entry with non-zero weight in [0, V) (rounding fallback of a draw).
-template <class W>
-__device__ int last_nonzero(int V, W weight) {
-  __shared__ int s_last;
-  if (threadIdx.x == 0) s_last = -1;
-  __syncthreads();
-  for (int v = threadIdx.x; v < V; v += blockDim.x)
-    if (weight(v) > 0.f) atomicMax(&s_last, v);
-  __syncthreads();
-  const int r = s_last;
-  __syncthreads();
-  return r < 0 ? V - 1 : r;
-}
-
-// Draw with target u * Z over weights whose chunk sums are csum[0..nvch).
-// Inverse-CDF draw of target = u * Z from the chunk sums csum: thread 0 finds the chunk,
-// stage(c0, n) brings that chunk's inputs into shared memory (ending with a barrier), and
-// the search reads them there through sweight(v, c0); if rounding carries the target past
-// the last chunk, the last token of nonzero weight (gweight reads global memory) is taken.
-template <class Stage, class SW, class GW>
-__device__ int draw_staged(int V, int nvch, const double* csum, double target, double& mrg,
-                           Stage stage, SW sweight, GW gweight) {
-  __shared__ int s_c;
-  __shared__ double s_base;
-  if (threadIdx.x == 0) {
-    double cum = 0.0;
-    int c = nvch;
-    for (int i = 0; i < nvch; ++i) {
-      if (target < cum + csum[i]) {
-        c = i;
-        break;
-      }
-      cum += csum[i];
-    }
-    s_c = c;
-    s_base = cum;
-  }
-  __syncthreads();
-  double base = s_base;
-  int tok = -1;
-  mrg = 0.0;
-  for (int c = s_c; c < nvch && tok < 0; ++c) {
-    const int c0 = c * kVocabChunk, cn = min(V - c0, kVocabChunk);
-    __syncthreads();   // every thread is done with the shared buffers
-    stage(c0, cn);
-    tok = chunk_search(c0, c0 + cn, target, base, mrg, [&](int v) -> float { return sweight(v, c0); });
-  }
-  return tok >= 0 ? tok : last_nonzero(V, gweight);
-}
-
 // ------------------------------------------------------------------ draft sampling ----
-// Draft sampling: a CTA takes kDsSpan logits of one request's draft row (two vocabulary
-// chunks), staged in shared memory by one bulk copy (so no registers are held by loads in
-// flight and a launch over 32 requests x 151,936 logits is one wave), and writes the two
-// chunks' (max, sum) partials; the last CTA of the request merges them and draws.
-constexpr int kDsPer = 2;
-constexpr int kDsSpan = kDsPer * kVocabChunk;
+// Draft sampling: a CTA takes one vocabulary chunk (8192 logits) of one request's draft row,
+// eight 16-byte loads per thread all in flight at once (load j of thread t holds entries
+// 1024 j + 4 t .. + 3, so it lies in sub-block j), and writes the chunk's (max, sum) partial
+// and its sub-block sums; the last CTA of the request merges them and draws from the one
+// sub-block that holds u * Z. At most 51 registers a thread, so five CTAs fit on an SM and a
+// launch over 32 requests x 151,936 logits (608 CTAs) is one wave.
+constexpr int kDsMinBlocks = 5;
 
-// (max, sum) of this thread's entries t + 256 q of a staged chunk of n <= kVocabChunk, all
-// 32 read from shared memory at once (no load latency per entry).
-__device__ __forceinline__ void smem_ms(const float* xs, int n, float& m, float& s, bool& bad) {
-  static_assert(kVocabChunk == 32 * kSampThreads, "32 entries per thread");
-  float x[32];
-#pragma unroll
-  for (int q = 0; q < 32; ++q) {
-    const int j = (int)threadIdx.x + kSampThreads * q;
-    float v = j < n ? xs[j] : -INFINITY;
-    if (isnan(v) || v == INFINITY) {
-      bad = true;
-      v = -INFINITY;
-    }
-    x[q] = v;
-  }
-  m = -INFINITY;
-#pragma unroll
-  for (int q = 0; q < 32; ++q) m = fmaxf(m, x[q]);
-  s = 0.f;
-  if (m != -INFINITY) {
-    const float mb = m * kLog2e;
-#pragma unroll
-    for (int q = 0; q < 32; ++q) s += ex2(fmaf(x[q], kLog2e, -mb));
-  }
-}
-
-__global__ void __launch_bounds__(kSampThreads) draft_sample_kernel(const SampleParams p) {
+__global__ void __launch_bounds__(kSampThreads, kDsMinBlocks) draft_sample_kernel(const SampleParams p) {
   pdl_wait();
-  extern __shared__ float4 xs4[];   // [kDsSpan] logits of this CTA's span
-  float* xs = reinterpret_cast<float*>(xs4);
-  __shared__ __align__(8) uint64_t bar;
   __shared__ int s_flag;
   __shared__ double csum[64];
+  __shared__ float s_mc[64];        // chunk maxima
+  __shared__ float s_red[kSampThreads / 32];
+  __shared__ float s_sub[kSubPer];
+  __shared__ float s_subs[64 * kSubPer];
   __shared__ float s_M;
-  const int cb = blockIdx.y, bl = blockIdx.x;
+  const int c = blockIdx.y, bl = blockIdx.x;
   const int r = p.req_ids ? p.req_ids[bl] : bl;
   if (r < 0 || r >= p.num_requests) {   // every CTA of the row returns: no ticket is touched
-    if (cb == 0 && threadIdx.x == 0) set_error(p.err, S3R_ERR_DEVICE_BOUNDS);
+    if (c == 0 && threadIdx.x == 0) set_error(p.err, S3R_ERR_DEVICE_BOUNDS);
     return;
   }
   const int i = p.draft_step[r];
+  const int L = p.seq_lens[r];      // read now: both loads in flight together
   const int V = p.vocab;
   if (i < 0 || i >= p.k) {
-    if (cb == 0 && threadIdx.x == 0) set_error(p.err, S3R_ERR_DEVICE_BOUNDS);
+    if (c == 0 && threadIdx.x == 0) set_error(p.err, S3R_ERR_DEVICE_BOUNDS);
     return;
   }
   const float* row = p.q_logits + ((size_t)r * p.k + i) * V;
   MS* part = reinterpret_cast<MS*>(p.part) + (size_t)r * p.nvch;
-  const int v0 = cb * kDsSpan, n = min(V - v0, kDsSpan);
+  float* subs = reinterpret_cast<float*>(p.part + p.sub_off) + (size_t)r * p.nvch * kSubPer;
+  const int v0 = c * kVocabChunk, v1 = min(V, v0 + kVocabChunk);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
-  // stage the span: one bulk copy when it is 16-byte aligned and sized, else plain loads
-  const bool bulk = ((reinterpret_cast<uintptr_t>(row + v0) & 15u) == 0) && ((n & 3) == 0);
-  if (bulk) {
-    if (threadIdx.x == 0) {
-      mbar_init(smem_u32(&bar), 1);
-      fence_mbar_init();
-    }
-    __syncthreads();   // the barrier is initialised before the copy and before anyone polls it
-    if (threadIdx.x == 0) {
-      mbar_arrive_expect_tx(smem_u32(&bar), (uint32_t)n * 4u);
-      bulk_load(smem_u32(xs), row + v0, (uint32_t)n * 4u, smem_u32(&bar));
-    }
-    if (!mbar_wait(smem_u32(&bar), 0) && threadIdx.x == 0) set_error(p.err, S3R_ERR_TIMEOUT);
-  } else {
-    for (int j = threadIdx.x; j < n; j += kSampThreads) xs[j] = __ldg(row + v0 + j);
-    __syncthreads();
-  }
-
-  bool bad = false;
+  float4 x[kSubPer];
+  const bool vec = ((reinterpret_cast<uintptr_t>(row + v0) & 15u) == 0) && (((v1 - v0) & 3) == 0);
 #pragma unroll
-  for (int h = 0; h < kDsPer; ++h) {
-    const int c = cb * kDsPer + h;
-    if (c >= p.nvch) break;
-    float m, s;
-    smem_ms(xs + h * kVocabChunk, min(n - h * kVocabChunk, kVocabChunk), m, s, bad);
-    const MS tot = block_ms(m, s);
-    if (threadIdx.x == 0) part[c] = tot;
-    __syncthreads();   // block_ms's scratch is reused by the next chunk
+  for (int j = 0; j < kSubPer; ++j) {
+    const int v = v0 + kSub * j + 4 * (int)threadIdx.x;
+    if (vec) {
+      x[j] = v < v1 ? __ldg(reinterpret_cast<const float4*>(row + v))
+                    : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+    } else {
+      x[j].x = v < v1 ? __ldg(row + v) : -INFINITY;
+      x[j].y = v + 1 < v1 ? __ldg(row + v + 1) : -INFINITY;
+      x[j].z = v + 2 < v1 ? __ldg(row + v + 2) : -INFINITY;
+      x[j].w = v + 3 < v1 ? __ldg(row + v + 3) : -INFINITY;
+    }
+  }
+  bool bad = false;
+  float m = -INFINITY;
+  auto clean = [&](float& v) {
+    if (isnan(v) || v == INFINITY) {
+      bad = true;
+      v = -INFINITY;
+    }
+  };
+#pragma unroll
+  for (int j = 0; j < kSubPer; ++j) {
+    clean(x[j].x);
+    clean(x[j].y);
+    clean(x[j].z);
+    clean(x[j].w);
+    m = fmaxf(fmaxf(m, fmaxf(x[j].x, x[j].y)), fmaxf(x[j].z, x[j].w));
   }
   if (bad) set_error(p.err, S3R_ERR_NONFINITE);
+  m = warp_max(m);
+  if (lane == 0) s_red[warp] = m;
+  __syncthreads();
+  float Mc = s_red[0];
+  for (int w = 1; w < kSampThreads / 32; ++w) Mc = fmaxf(Mc, s_red[w]);
+  float sub[kSubPer];
+  const float mb = Mc * kLog2e;
+#pragma unroll
+  for (int j = 0; j < kSubPer; ++j)
+    sub[j] = Mc == -INFINITY ? 0.f
+                             : (ex2(fmaf(x[j].x, kLog2e, -mb)) + ex2(fmaf(x[j].y, kLog2e, -mb))) +
+                                   (ex2(fmaf(x[j].z, kLog2e, -mb)) + ex2(fmaf(x[j].w, kLog2e, -mb)));
+  block_sum_sub(sub, s_sub);
+  if (threadIdx.x < kSubPer) subs[(size_t)c * kSubPer + threadIdx.x] = s_sub[threadIdx.x];
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int b = 0; b < kSubPer; ++b) t += (double)s_sub[b];
+    MS tot;
+    tot.m = Mc;
+    tot.pad = 0.f;
+    tot.s = t;
+    part[c] = tot;
+  }
   if (!last_of(p.tickets + r, (int)gridDim.y, &s_flag)) return;
 
+  // the last CTA: chunk maxima and weights on the common scale, every sub-block sum
   if (threadIdx.x < 32) {
     const float M = merge_partials_warp(part, p.nvch, csum);
     if (threadIdx.x == 0) s_M = M;
+    for (int q = threadIdx.x; q < p.nvch; q += 32) s_mc[q] = __ldcg(&part[q].m);
   }
+  for (int t = threadIdx.x; t < p.nvch * kSubPer; t += kSampThreads) s_subs[t] = __ldcg(subs + t);
   __syncthreads();
   const float M = s_M;
   double Z = 0.0;
   for (int q = 0; q < p.nvch; ++q) Z += csum[q];
-  const int L = p.seq_lens[r];
   const double u = philox_u(p.seed, (uint32_t)(L + i + 1), (uint32_t)r, 0u);
-  const float Mb = M * kLog2e;
-  // the chunk holding u * Z is staged in shared memory (the span's buffer, by a bulk copy
-  // on the same barrier, whose phase 0 was the span's copy), then searched there
-  uint32_t phase = 1;
-  auto stage = [&](int c0, int cn) {
-    if (bulk && (cn & 3) == 0) {
-      if (threadIdx.x == 0) {
-        mbar_arrive_expect_tx(smem_u32(&bar), (uint32_t)cn * 4u);
-        bulk_load(smem_u32(xs), row + c0, (uint32_t)cn * 4u, smem_u32(&bar));
-      }
-      if (!mbar_wait(smem_u32(&bar), phase & 1u) && threadIdx.x == 0) set_error(p.err, S3R_ERR_TIMEOUT);
-      ++phase;
-    } else {
-      for (int j = threadIdx.x; j < cn; j += kSampThreads) xs[j] = __ldg(row + c0 + j);
-      __syncthreads();
-    }
+  auto scale = [&](int cc) -> double {   // chunk cc's weights -> the common scale
+    return s_mc[cc] == -INFINITY ? 0.0 : (double)exp2f((s_mc[cc] - M) * kLog2e);
   };
-  auto wq = [&](float x) -> float { return (isnan(x) || x == INFINITY) ? 0.f : ex2(fmaf(x, kLog2e, -Mb)); };
   double mrg;
-  const int tok = draw_staged(
-      V, p.nvch, csum, u * Z, mrg, stage, [&](int v, int c0) { return wq(xs[v - c0]); },
-      [&](int v) { return wq(row[v]); });
+  const int tok = subblock_draw(
+      V, p.nvch, csum, u * Z, mrg, [&](int cc, int b) { return (double)s_subs[cc * kSubPer + b] * scale(cc); },
+      [&](int vw, double (&w)[4]) {
+        const int cc = vw / kVocabChunk;
+        const float mbc = s_mc[cc] * kLog2e;
+        const double f = scale(cc);
+        float xv[4];
+        if (vw + 3 < V && ((reinterpret_cast<uintptr_t>(row + vw) & 15u) == 0)) {
+          const float4 t = __ldg(reinterpret_cast<const float4*>(row + vw));
+          xv[0] = t.x; xv[1] = t.y; xv[2] = t.z; xv[3] = t.w;
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) xv[e] = vw + e < V ? __ldg(row + vw + e) : -INFINITY;
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float xe = (isnan(xv[e]) || xv[e] == INFINITY) ? -INFINITY : xv[e];
+          w[e] = (s_mc[cc] == -INFINITY) ? 0.0 : (double)ex2(fmaf(xe, kLog2e, -mbc)) * f;
+        }
+      });
   if (threadIdx.x == 0) {
     p.draft_out[(size_t)r * p.k + i] = tok;
     if (p.margins) p.margins[(size_t)r * p.k + i] = Z > 0.0 ? (float)(mrg / Z) : 0.f;
@@ -506,14 +467,15 @@ __global__ void __launch_bounds__(kSampThreads) spec_norm_kernel(const SamplePar
 }
 
 // ------------------------------------------------------- speculative sampling: pass 2 --
-__global__ void __launch_bounds__(kSampThreads) spec_draw_kernel(const SampleParams p) {
+// The drawn row's chunk sums of the residual max(0, p - q) and of p, with the sums of their
+// sub-blocks; the last CTA draws from the residual (or from p if its mass is zero).
+__global__ void __launch_bounds__(kSampThreads, kDsMinBlocks) spec_draw_kernel(const SampleParams p) {
   pdl_wait();
-  extern __shared__ float4 xs4[];   // the drawn chunk: p logits, then q logits
-  float* xps = reinterpret_cast<float*>(xs4);
-  float* xqs = xps + kVocabChunk;
   __shared__ int s_flag;
   __shared__ double csum[64];
   __shared__ int s_use_res;
+  __shared__ float s_subr[kSubPer], s_subp[kSubPer];
+  __shared__ float s_subs[64 * kSubPer];
   const int c = blockIdx.y, bl = blockIdx.x;
   const int r = p.req_ids ? p.req_ids[bl] : bl;
   if (r < 0 || r >= p.num_requests) return;   // reported by the first pass
@@ -522,22 +484,10 @@ __global__ void __launch_bounds__(kSampThreads) spec_draw_kernel(const SamplePar
   const float* prow = p.p_logits + ((size_t)r * (k + 1) + pl.row) * V;
   const float* qrow = p.q_logits + ((size_t)r * k + (pl.type == 0 ? pl.row : 0)) * V;
   double2* part = reinterpret_cast<double2*>(p.part + p.draw_off) + (size_t)r * p.nvch;
+  float* subs = reinterpret_cast<float*>(p.part + p.sub_off) + (size_t)r * p.nvch * 2 * kSubPer;
   const bool resid = pl.type == 0;
   const float mpb = pl.mp * kLog2e, mqb = pl.mq * kLog2e;
   const float izp = (float)(1.0 / pl.zp), izq = (float)(1.0 / pl.zq);
-  auto w_p = [&](int v) -> float {
-    const float x = prow[v];
-    return (isnan(x) || x == INFINITY) ? 0.f : ex2(fmaf(x, kLog2e, -mpb));
-  };
-  auto w_res = [&](int v) -> float {
-    const float x = prow[v], y = qrow[v];
-    const float pv = (isnan(x) || x == INFINITY) ? 0.f : ex2(fmaf(x, kLog2e, -mpb)) * izp;
-    const float qv = (isnan(y) || y == INFINITY) ? 0.f : ex2(fmaf(y, kLog2e, -mqb)) * izq;
-    return fmaxf(pv - qv, 0.f);
-  };
-
-  const int v0 = c * kVocabChunk, v1 = min(V, (c + 1) * kVocabChunk);
-  float srf = 0.f, spf = 0.f;
   auto wp_x = [&](float x) -> float {
     return (isnan(x) || x == INFINITY) ? 0.f : ex2(fmaf(x, kLog2e, -mpb));
   };
@@ -546,38 +496,60 @@ __global__ void __launch_bounds__(kSampThreads) spec_draw_kernel(const SamplePar
     const float qv = (isnan(y) || y == INFINITY) ? 0.f : ex2(fmaf(y, kLog2e, -mqb)) * izq;
     return fmaxf(pv - qv, 0.f);
   };
+
+  const int v0 = c * kVocabChunk, v1 = min(V, (c + 1) * kVocabChunk);
+  float subr[kSubPer], subp[kSubPer];
+#pragma unroll
+  for (int b = 0; b < kSubPer; ++b) subr[b] = subp[b] = 0.f;
   const bool vec = ((reinterpret_cast<uintptr_t>(prow + v0) & 15u) == 0) &&
                    ((reinterpret_cast<uintptr_t>(qrow + v0) & 15u) == 0) && (((v1 - v0) & 3) == 0);
   if (vec) {
-    // 32 entries per thread as eight 16-byte loads of each row, all in flight at once
-    float4 xp[8], xq[8];
+    // 32 entries per thread as eight 16-byte loads of each row, four of each in flight at a
+    // time (the register budget of five CTAs per SM); load j of every thread covers sub-block j
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int v = v0 + 4 * ((int)threadIdx.x + kSampThreads * j);
-      xp[j] = v < v1 ? __ldg(reinterpret_cast<const float4*>(prow + v)) : make_float4(0.f, 0.f, 0.f, 0.f);
-      xq[j] = (resid && v < v1) ? __ldg(reinterpret_cast<const float4*>(qrow + v))
-                                : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
+    for (int h = 0; h < 2; ++h) {
+      float4 xp[4], xq[4];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int v = v0 + 4 * ((int)threadIdx.x + kSampThreads * j);
-      if (v < v1) {
-        spf += wp_x(xp[j].x) + wp_x(xp[j].y) + wp_x(xp[j].z) + wp_x(xp[j].w);
-        if (resid)
-          srf += wres_xy(xp[j].x, xq[j].x) + wres_xy(xp[j].y, xq[j].y) +
-                 wres_xy(xp[j].z, xq[j].z) + wres_xy(xp[j].w, xq[j].w);
+      for (int jj = 0; jj < 4; ++jj) {
+        const int v = v0 + 4 * ((int)threadIdx.x + kSampThreads * (4 * h + jj));
+        xp[jj] = v < v1 ? __ldg(reinterpret_cast<const float4*>(prow + v)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        xq[jj] = (resid && v < v1) ? __ldg(reinterpret_cast<const float4*>(qrow + v))
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        const int j = 4 * h + jj;
+        const int v = v0 + 4 * ((int)threadIdx.x + kSampThreads * j);
+        if (v < v1) {
+          subp[j] = wp_x(xp[jj].x) + wp_x(xp[jj].y) + wp_x(xp[jj].z) + wp_x(xp[jj].w);
+          if (resid)
+            subr[j] = wres_xy(xp[jj].x, xq[jj].x) + wres_xy(xp[jj].y, xq[jj].y) +
+                      wres_xy(xp[jj].z, xq[jj].z) + wres_xy(xp[jj].w, xq[jj].w);
+        }
       }
     }
   } else {
     for (int v = v0 + threadIdx.x; v < v1; v += blockDim.x) {
-      spf += w_p(v);
-      if (resid) srf += w_res(v);
+      const int b = (v - v0) / kSub;
+      const float x = prow[v];
+      subp[b] += wp_x(x);
+      if (resid) subr[b] += wres_xy(x, qrow[v]);
     }
   }
-  double sr = srf, sp = spf;
-  sp = block_sum_d(sp);
-  sr = block_sum_d(sr);
-  if (threadIdx.x == 0) part[c] = make_double2(sr, sp);
+  block_sum_sub(subr, s_subr);
+  block_sum_sub(subp, s_subp);
+  if (threadIdx.x < kSubPer) {
+    subs[((size_t)c * 2) * kSubPer + threadIdx.x] = s_subr[threadIdx.x];
+    subs[((size_t)c * 2 + 1) * kSubPer + threadIdx.x] = s_subp[threadIdx.x];
+  }
+  if (threadIdx.x == 0) {
+    double sr = 0.0, sp = 0.0;
+    for (int b = 0; b < kSubPer; ++b) {
+      sr += (double)s_subr[b];
+      sp += (double)s_subp[b];
+    }
+    part[c] = make_double2(sr, sp);
+  }
   if (!last_of(p.tickets + r, p.nvch, &s_flag)) return;
 
   if (threadIdx.x < 32) {
@@ -595,48 +567,40 @@ __global__ void __launch_bounds__(kSampThreads) spec_draw_kernel(const SamplePar
     if (lane == 0) s_use_res = use_res;
   }
   __syncthreads();
+  const bool use_res = s_use_res != 0;
+  for (int t = threadIdx.x; t < p.nvch * kSubPer; t += kSampThreads) {
+    const int cc = t / kSubPer, b = t - cc * kSubPer;
+    s_subs[t] = __ldcg(subs + ((size_t)cc * 2 + (use_res ? 0 : 1)) * kSubPer + b);
+  }
+  __syncthreads();
   double Z = 0.0;
   for (int q = 0; q < p.nvch; ++q) Z += csum[q];
   const double target = pl.u * Z;
-  const bool use_res = s_use_res != 0;
-  // the drawn chunk of the p row (and the q row for a residual) staged in shared memory by
-  // bulk copies (or plain loads when unaligned), then searched there
-  __shared__ __align__(8) uint64_t bar;
-  uint32_t phase = 0;
-  if (threadIdx.x == 0) {
-    mbar_init(smem_u32(&bar), 1);
-    fence_mbar_init();
-  }
-  __syncthreads();
-  auto stage = [&](int c0, int cn) {
-    const bool v4 = ((reinterpret_cast<uintptr_t>(prow + c0) & 15u) == 0) &&
-                    ((reinterpret_cast<uintptr_t>(qrow + c0) & 15u) == 0) && ((cn & 3) == 0);
-    if (v4) {
-      if (threadIdx.x == 0) {
-        const uint32_t bytes = (uint32_t)cn * 4u;
-        mbar_arrive_expect_tx(smem_u32(&bar), use_res ? 2u * bytes : bytes);
-        bulk_load(smem_u32(xps), prow + c0, bytes, smem_u32(&bar));
-        if (use_res) bulk_load(smem_u32(xqs), qrow + c0, bytes, smem_u32(&bar));
-      }
-      if (!mbar_wait(smem_u32(&bar), phase & 1u) && threadIdx.x == 0) set_error(p.err, S3R_ERR_TIMEOUT);
-      ++phase;
-      return;
-    } else {
-      for (int j = threadIdx.x; j < cn; j += kSampThreads) {
-        xps[j] = __ldg(prow + c0 + j);
-        if (use_res) xqs[j] = __ldg(qrow + c0 + j);
-      }
-    }
-    __syncthreads();
-  };
-  int tok;
   double mrg;
-  if (use_res)
-    tok = draw_staged(V, p.nvch, csum, target, mrg, stage,
-                      [&](int v, int c0) { return wres_xy(xps[v - c0], xqs[v - c0]); }, w_res);
-  else
-    tok = draw_staged(V, p.nvch, csum, target, mrg, stage,
-                      [&](int v, int c0) { return wp_x(xps[v - c0]); }, w_p);
+  const int tok = subblock_draw(
+      V, p.nvch, csum, target, mrg, [&](int cc, int b) { return (double)s_subs[cc * kSubPer + b]; },
+      [&](int vw, double (&w)[4]) {
+        float xp[4], xq[4];
+        const bool al = vw + 3 < V && ((reinterpret_cast<uintptr_t>(prow + vw) & 15u) == 0) &&
+                        ((reinterpret_cast<uintptr_t>(qrow + vw) & 15u) == 0);
+        if (al) {
+          const float4 a = __ldg(reinterpret_cast<const float4*>(prow + vw));
+          xp[0] = a.x; xp[1] = a.y; xp[2] = a.z; xp[3] = a.w;
+          if (use_res) {
+            const float4 b = __ldg(reinterpret_cast<const float4*>(qrow + vw));
+            xq[0] = b.x; xq[1] = b.y; xq[2] = b.z; xq[3] = b.w;
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            xp[e] = vw + e < V ? __ldg(prow + vw + e) : -INFINITY;
+            xq[e] = (use_res && vw + e < V) ? __ldg(qrow + vw + e) : -INFINITY;
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          w[e] = vw + e >= V ? 0.0 : (double)(use_res ? wres_xy(xp[e], xq[e]) : wp_x(xp[e]));
+      });
   if (threadIdx.x == 0) {
     p.out_tokens[(size_t)r * (k + 1) + pl.a] = tok;
     // the draw's margin follows the decided drafts' margins
@@ -798,12 +762,8 @@ __global__ void philox_kernel(uint64_t seed, int stream_id, const int32_t* reque
 
 // ------------------------------------------------------------------------ launchers ----
 int launch_draft_sample(const SampleParams& p, int batch, cudaStream_t stream) {
-  constexpr int smem = kDsSpan * 4;
-  static std::atomic<uint64_t> attr_done{0};
-  if (cuda_status(ensure_smem_attr(draft_sample_kernel, smem, attr_done), "cudaFuncSetAttribute") != S3R_OK)
-    return S3R_ERR_CUDA;
-  dim3 grid(batch, (p.vocab + kDsSpan - 1) / kDsSpan);
-  launch_pdl(draft_sample_kernel, grid, kSampThreads, smem, stream, p);
+  dim3 grid(batch, p.nvch);
+  launch_pdl(draft_sample_kernel, grid, kSampThreads, 0, stream, p);
   return cuda_status(cudaGetLastError(), __func__);
 }
 
@@ -811,28 +771,36 @@ int launch_spec_sample(const SampleParams& p, int batch, cudaStream_t stream, in
   dim3 g1(batch, 2 * p.k + 1, p.nvch);
   launch_pdl(spec_norm_kernel, g1, kSampThreads, 0, stream, p);
   if (cuda_status(cudaGetLastError(), __func__) != S3R_OK) return S3R_ERR_CUDA;
-  constexpr int smem2 = 2 * kVocabChunk * 4;
-  static std::atomic<uint64_t> attr_done{0};
-  if (cuda_status(ensure_smem_attr(spec_draw_kernel, smem2, attr_done), "cudaFuncSetAttribute") != S3R_OK)
-    return S3R_ERR_CUDA;
   dim3 g2(batch, p.nvch);
-  launch_pdl(spec_draw_kernel, g2, kSampThreads, smem2, stream, p);
+  launch_pdl(spec_draw_kernel, g2, kSampThreads, 0, stream, p);
   *launches = 2;
   return cuda_status(cudaGetLastError(), __func__);
 }
 
+// Speculative sampling's workspace: normaliser partials [NR][2k+1][nvch], plans [NR], draw
+// partials [NR][nvch] (double2), draw sub-block sums [NR][nvch][2][kSubPer] (fp32).
+// Draft sampling's: partials [NR][nvch], then sub-block sums [NR][nvch][kSubPer].
 size_t sample_partial_bytes(int num_requests, int k, int vocab) {
   const size_t nvch = (size_t)((vocab + kVocabChunk - 1) / kVocabChunk);
   const size_t a = align_up((size_t)num_requests * (2 * k + 1) * nvch * sizeof(MS), 256);
   const size_t b = align_up((size_t)num_requests * sizeof(SpecPlan), 256);
   const size_t c = align_up((size_t)num_requests * nvch * sizeof(double2), 256);
-  return a + b + c;
+  const size_t d = align_up((size_t)num_requests * nvch * 2 * kSubPer * sizeof(float), 256);
+  const size_t draft = draft_sub_offset(num_requests, vocab) +
+                       align_up((size_t)num_requests * nvch * kSubPer * sizeof(float), 256);
+  return a + b + c + d > draft ? a + b + c + d : draft;
 }
 
-void spec_offsets(int num_requests, int k, int vocab, size_t* plan_off, size_t* draw_off) {
+void spec_offsets(int num_requests, int k, int vocab, size_t* plan_off, size_t* draw_off, size_t* sub_off) {
   const size_t nvch = (size_t)((vocab + kVocabChunk - 1) / kVocabChunk);
   *plan_off = align_up((size_t)num_requests * (2 * k + 1) * nvch * sizeof(MS), 256);
   *draw_off = *plan_off + align_up((size_t)num_requests * sizeof(SpecPlan), 256);
+  *sub_off = *draw_off + align_up((size_t)num_requests * nvch * sizeof(double2), 256);
+}
+
+size_t draft_sub_offset(int num_requests, int vocab) {
+  const size_t nvch = (size_t)((vocab + kVocabChunk - 1) / kVocabChunk);
+  return align_up((size_t)num_requests * nvch * sizeof(MS), 256);
 }
 
 int launch_commit(const int32_t* req_ids, int batch, int k, const int32_t* n_out,
