@@ -139,11 +139,19 @@ def test_mixed_phase_batch_matches_oracle():
     assert st[1] == spec.num_requests
 
 
-@pytest.mark.parametrize("workload", ["qwen3-1.7b", "qwen3-8b"])
-def test_full_size_round_on_sampled_requests(workload):
+@pytest.mark.parametrize("workload,point,picks", [
+    ("qwen3-1.7b", None, 6), ("qwen3-8b", None, 6),
+    ("sweep", (500, 6), 3),     # the 32 x 24576 budget-sweep shapes at the bench point
+    ("sweep", (2000, 8), 3),    # k = 8: 36 rows per KV head, the 64-row tensor-memory verify
+])
+def test_full_size_round_on_sampled_requests(workload, point, picks):
     """One round of the whole Qwen3-shaped batch at full size (the benchmark's launch
-    configuration); the oracle replays two sampled requests."""
+    configuration); the oracle replays sampled requests. The sweep shapes run with the
+    synthetic logit model here (their projection logits are covered at reduced size below)."""
     spec = synth.WORKLOADS[workload]
+    if point is not None:
+        spec = spec.with_(budget_bp=point[0], k=point[1], vocab=32768, projection_logits=False,
+                          draft_noise_std=0.5)
     k = spec.k
     lens = synth.make_lengths(spec)
     cache = synth.build_cache(spec, lens, extra_tokens=k + 1 + 16, device="cuda")
@@ -154,8 +162,8 @@ def test_full_size_round_on_sampled_requests(workload):
     vb = synth.randn_bf16((NR, k + 1, Hkv, d), 102, "cuda")
     pl = synth.randn_f32((NR, k + 1, V), 103, "cuda", scale=spec.logit_std)
     ql = (pl[:, :k] + synth.randn_f32((NR, k, V), 104, "cuda", scale=spec.draft_noise_std)).contiguous()
-    rng = np.random.default_rng(spec.data_seed)
-    picks = sorted(rng.choice(NR, size=2, replace=False).tolist())
+    rng = np.random.default_rng(spec.data_seed + k)
+    picks = sorted(rng.choice(NR, size=picks, replace=False).tolist())
     pt = cache.page_table.cpu().numpy()
     host = {}
     for r in picks:    # the requests' pages before the round writes its block
@@ -289,7 +297,7 @@ def test_projection_logits_round_matches_oracle():
 def test_full_size_mixed_phase_batch_on_sampled_requests():
     """The high-concurrency workload at full size: 256 requests, contexts log-uniform in
     [1024, 16384], shuffled pages, mixed round phases; k+1 driver iterations complete one
-    round per request, and the oracle replays four sampled requests."""
+    round per request, and the oracle replays twelve sampled requests."""
     spec = synth.WORKLOADS["ragged"]
     k = spec.k
     lens = synth.make_lengths(spec)
@@ -300,7 +308,7 @@ def test_full_size_mixed_phase_batch_on_sampled_requests():
     vb = synth.randn_bf16((NR, k + 1, Hkv, d), 202, "cuda")
     pl = synth.randn_f32((NR, k + 1, V), 203, "cuda", scale=spec.logit_std)
     ql = (pl[:, :k] + synth.randn_f32((NR, k, V), 204, "cuda", scale=spec.draft_noise_std)).contiguous()
-    picks = sorted(np.random.default_rng(3).choice(NR, size=4, replace=False).tolist())
+    picks = sorted(np.random.default_rng(3).choice(NR, size=12, replace=False).tolist())
     pt = cache.page_table.cpu().numpy()
     host = {}
     for r in picks:
