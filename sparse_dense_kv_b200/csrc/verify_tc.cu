@@ -1,6 +1,6 @@
 // Dense verify attention with score capture on the 5th-generation tensor cores (tcgen05,
-// accumulators in tensor memory), head_dim 128, up to 64 rows per KV head (padded to 16, 32
-// or 64 rows: N of both products).
+// accumulators in tensor memory), head_dim 128, up to 64 rows per KV head (padded to 16, 32,
+// 48 or 64 rows: N of both products).
 //
 // What it computes is what verify.cu computes ([News] Interpretation: the proposed block is
 // recomputed against the complete historical KV; [Explainer] walkthrough: the sparse set
@@ -8,8 +8,8 @@
 // positions 0..L+t; out, lse and every committed logit are written.
 //
 // Organisation (one persistent CTA per SM, 11 warps). A work item is (request, KV head,
-// chunk of up to 8, 7 or 3 tiles of 128 positions at 16, 32 or 64 rows: two S buffers of a
-// chunk and two O buffers fill the 512 columns of tensor memory). Items are claimed from a counter in the
+// chunk of up to 8, 7, 4 or 3 tiles of 128 positions at 16, 32, 48 or 64 rows: two S
+// buffers of a chunk and two O buffers fill the 512 columns of tensor memory). Items are claimed from a counter in the
 // workspace as CTAs progress (the K producer claims, a ring in shared memory tells the
 // other roles), so faster SMs take more of them.
 //   warp 0     K producer: per item it loads the item's Q rows into one of two Q buffers
@@ -24,8 +24,9 @@
 //              K_t . Q^T into tensor memory for the QK of item m, and O^T (128 d x N) +=
 //              V_t^T . P_t^T for the PV of item n < m; whichever has its next tile ready is
 //              issued. K and Q are K-major operands (128-byte swizzle); V^T is MN-major (the V
-//              tile as it arrives) and so is P^T (one row of N values per position, 32-,
-//              64- or 128-byte swizzle). S and O are double-buffered in tensor memory.
+//              tile as it arrives) and so is P^T (N values per position in atoms of 16, 32
+//              or 64 rows: 32-, 64- or 128-byte swizzle; 48 rows are three 16-row atoms).
+//              S and O are double-buffered in tensor memory.
 //   warps 3-10 softmax / epilogue, two warpgroups each owning half of the rows (one thread
 //              per tensor-memory lane = position or d): pass 1 reads every S tile, writes the
 //              committed logits and takes the chunk maximum per row; pass 2 re-reads them and
@@ -112,19 +113,31 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float* v) {
 #pragma unroll
   for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
-// N (8 or a multiple of 16) consecutive columns.
+// N (a multiple of 8) consecutive columns in loads of 16 and, if N % 16 == 8, one of 8.
+// Every 16-column load starts on a multiple of 16 columns: lead8 says the first column is
+// 8 past one (the upper half of 48 rows starts at column 24), so the 8-column load goes first.
 template <int N>
-__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float (&v)[N]) {
-  if constexpr (N == 8) {
-    tmem_ld8(taddr, v);
-  } else {
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float (&v)[N], bool lead8 = false) {
+  static_assert(N % 8 == 0, "whole groups of 8 columns");
+  auto run16 = [&](int first) {
 #pragma unroll
-    for (int c = 0; c < N; c += 16) {
+    for (int c = first; c + 16 <= N; c += 16) {
       float w[16];
       tmem_ld16(taddr + c, w);
 #pragma unroll
       for (int i = 0; i < 16; ++i) v[c + i] = w[i];
     }
+  };
+  if constexpr (N % 16 == 8) {
+    if (lead8) {
+      tmem_ld8(taddr, v);
+      run16(8);
+    } else {
+      run16(0);
+      tmem_ld8(taddr + (N - 8), v + (N - 8));
+    }
+  } else {
+    run16(0);
   }
 }
 template <int N>
@@ -154,14 +167,18 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool 
 
 template <int NP>
 struct Cfg {
-  static constexpr int kTiles = NP == 64 ? 3 : (NP == 32 ? 7 : 8);   // tiles per chunk
+  static constexpr int kTiles = NP == 64 ? 3 : (NP == 48 ? 4 : (NP == 32 ? 7 : 8));   // tiles per chunk
   static constexpr int kKSt = 2;                             // K ring stages
   static constexpr int kVSt = 2;                             // V ring stages
   static constexpr int kChunk = kTiles * kPos;
   static constexpr int kQBytes = 2 * NP * 128;               // one Q buffer: [2 halves][NP rows][128 B]
   static constexpr int kPTile = kPos * NP * 2;               // P^T tile: [128 pos][NP rows] bf16
   static constexpr int kPBytes = kTiles * kPTile;
-  static constexpr uint32_t kPSwz = NP == 16 ? 6u : (NP == 32 ? 4u : 2u);   // 32- / 64- / 128-byte swizzle
+  // P^T swizzle: 32 bytes for 16 and 48 rows (one or three 16-row atoms along N), 64 for
+  // 32, 128 for 64 (one atom)
+  static constexpr uint32_t kPSwz = (NP == 16 || NP == 48) ? 6u : (NP == 32 ? 4u : 2u);
+  static constexpr int kPAtomRows = (NP == 16 || NP == 48) ? 16 : NP;       // rows of one atom
+  static constexpr int kPAtomBytes = kPos * kPAtomRows * 2;                 // one atom column of a tile
   static constexpr int kTmemCols = 512;
   static constexpr int kSCols = kTiles * NP;                 // one S buffer
   static constexpr int kOCol = 2 * kSCols;                   // two O buffers after two S buffers
@@ -625,7 +642,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int kk = 0; kk < kPos / 16; ++kk) {
                 const uint64_t ad = sdesc(vt + kk * 2048, kPos * 128, 1024, 2);
-                const uint64_t bd = sdesc(pt + kk * 16 * NP * 2, NP * 2 * 8, 8 * NP * 2, C::kPSwz);
+                // MN-major P^T: LBO = stride between atoms along N, SBO = stride between
+                // groups of 8 positions (one atom row is kPAtomRows * 2 bytes)
+                const uint64_t bd = sdesc(pt + kk * 16 * C::kPAtomRows * 2, C::kPAtomBytes,
+                                          8 * C::kPAtomRows * 2, C::kPSwz);
                 tc_mma(od, ad, bd, kIdPV, (tv > 0 || kk > 0) ? 1u : 0u);
               }
               tc_commit(smem_u32(&B->vempty[s]));
@@ -671,7 +691,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Warpgroup sg owns rows (columns of S and O^T) [sg*NH, sg*NH + NH) of every tile; the
     // two warpgroups only meet at the chunk's barriers for the MMA warp.
     constexpr int NH = NP / 2;               // rows per warpgroup
-    constexpr int BT = NP == 64 ? 1 : (NP == 32 ? 2 : 4);   // tiles per tensor-memory wait (no spills)
+    constexpr int BT = NP >= 48 ? 1 : (NP == 32 ? 2 : 4);   // tiles per tensor-memory wait (no spills)
     const int sw8 = warp - kSoftWarp0;       // 0..7
     const int sg = sw8 >> 2;                 // warpgroup
     const int sw4 = sw8 & 3;                 // warp within the warpgroup
@@ -679,10 +699,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int gt = (tid - 32 * kSoftWarp0) & 127;   // thread within the warpgroup
     const int lrow = q4 * 32 + lane;         // tile position (S) or d (O) of this thread
     const int c0 = sg * NH;                  // first row of this warpgroup
+    const bool lead8 = (c0 & 15) == 8;       // its columns start 8 past a multiple of 16
     const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
     const float scale = p.scale, scale2 = p.scale * kLog2e;
     // the row's 16-byte chunk is XORed with address bits 7.. of its P^T row (32-, 64-, 128-byte swizzle)
-    const int swz_row = (NP == 16) ? ((lrow >> 2) & 1) : (NP == 32 ? ((lrow >> 1) & 3) : (lrow & 7));
+    const int swz_row = (NP == 16 || NP == 48) ? ((lrow >> 2) & 1) : (NP == 32 ? ((lrow >> 1) & 3) : (lrow & 7));
     // Warpgroup barrier on an mbarrier (bounded wait, unlike bar.sync): if a wait anywhere
     // gives up, the other warps of the group give up here too instead of hanging.
     uint32_t wg_phase = 0;
@@ -702,7 +723,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const size_t rec_floats = (size_t)p.Rp * (kD + 2);
       float* rec = p.part + (((size_t)x.r * Hkv + x.kvh) * p.nchunk_max + x.c) * rec_floats;
       float o[NH];
-      tmem_ld_cols<NH>(tl + C::kOCol + (m & 1) * NP + c0, o);
+      tmem_ld_cols<NH>(tl + C::kOCol + (m & 1) * NP + c0, o, lead8);
       tmem_wait_ld();
       // records hold the R real rows (row pitch p.Rp >= R)
 #pragma unroll
@@ -746,7 +767,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float vv[BT][NH];
 #pragma unroll
         for (int u = 0; u < BT; ++u)   // past the last tile: reload the last tile (unused)
-          tmem_ld_cols<NH>(sbuf + min(tb + u, x.ntile - 1) * NP, vv[u]);
+          tmem_ld_cols<NH>(sbuf + min(tb + u, x.ntile - 1) * NP, vv[u], lead8);
         tmem_wait_ld();
 #pragma unroll
         for (int u = 0; u < BT; ++u) {
@@ -807,7 +828,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float vv[BT][NH];
 #pragma unroll
         for (int u = 0; u < BT; ++u)   // past the last tile: reload the last tile (unused)
-          tmem_ld_cols<NH>(sbuf + min(tb + u, x.ntile - 1) * NP, vv[u]);
+          tmem_ld_cols<NH>(sbuf + min(tb + u, x.ntile - 1) * NP, vv[u], lead8);
         tmem_wait_ld();
 #pragma unroll
         for (int u = 0; u < BT; ++u) {
@@ -836,11 +857,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          uint8_t* prow = smem + C::kPOff + t * C::kPTile + lrow * (NP * 2);
+          // 16-byte chunk cc holds rows 8 cc .. 8 cc + 7: atom cc / (kPAtomRows / 8), chunk
+          // cc % (kPAtomRows / 8) of the position's row in that atom
+          constexpr int CPA = C::kPAtomRows / 8;   // chunks per atom row
+          uint8_t* ptile = smem + C::kPOff + t * C::kPTile + lrow * (C::kPAtomRows * 2);
 #pragma unroll
           for (int i = 0; i < NH / 8; ++i) {
             const int cc = sg * (NH / 8) + i;
-            *reinterpret_cast<uint4*>(prow + ((cc ^ swz_row) << 4)) =
+            *reinterpret_cast<uint4*>(ptile + (cc / CPA) * C::kPAtomBytes + (((cc % CPA) ^ swz_row) << 4)) =
                 make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
           }
         }
@@ -900,7 +924,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace tc
 
-int verify_tc_npad(int R) { return R <= 16 ? 16 : (R <= 32 ? 32 : (R <= 64 ? 64 : 0)); }
+int verify_tc_npad(int R) { return R <= 16 ? 16 : (R <= 32 ? 32 : (R <= 48 ? 48 : (R <= 64 ? 64 : 0))); }
 
 template <int NP>
 static int launch_tc(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
@@ -922,15 +946,16 @@ bool verify_tc_supported(int D, int R, int /*batch*/) {
 
 int verify_tc_chunk(int R) {
   const int np = verify_tc_npad(R);
-  return np == 16 ? tc::Cfg<16>::kChunk : (np == 32 ? tc::Cfg<32>::kChunk : tc::Cfg<64>::kChunk);
+  return np == 16 ? tc::Cfg<16>::kChunk
+                   : (np == 32 ? tc::Cfg<32>::kChunk : (np == 48 ? tc::Cfg<48>::kChunk : tc::Cfg<64>::kChunk));
 }
 
 // Row pitch of the chunk records: the padded rows for 16 / 32 (as the merge has always read
-// them), the real rows (rounded to 4 for 16-byte loads) for 64, where padding would add a
-// third to the records' traffic.
+// them), the real rows (rounded to 4 for 16-byte loads) for 48 and 64, where padding would
+// add up to a third to the records' traffic.
 int verify_tc_rec_rows(int R) {
   const int np = verify_tc_npad(R);
-  return np == 64 ? (R + 3) / 4 * 4 : np;
+  return np >= 48 ? (R + 3) / 4 * 4 : np;
 }
 
 int launch_verify_tc(const CUtensorMap& qm, const CUtensorMap& k1, const CUtensorMap& v1,
@@ -938,7 +963,7 @@ int launch_verify_tc(const CUtensorMap& qm, const CUtensorMap& k1, const CUtenso
                      int batch, int num_sms, cudaStream_t stream, int* launches) {
   const int np = verify_tc_npad(p.R);
   *launches = 0;
-  if (np != 16 && np != 32 && np != 64) return S3R_ERR_UNSUPPORTED;
+  if (np != 16 && np != 32 && np != 48 && np != 64) return S3R_ERR_UNSUPPORTED;
   // the per-launch request tables hold kMaxBatch requests; a larger batch is several
   // launches over consecutive slices of it (each chunk record still lands in its slot)
   for (int b0 = 0; b0 < batch; b0 += tc::kMaxBatch) {
@@ -947,6 +972,7 @@ int launch_verify_tc(const CUtensorMap& qm, const CUtensorMap& k1, const CUtenso
     const int nb = batch - b0 < tc::kMaxBatch ? batch - b0 : tc::kMaxBatch;
     const int st = np == 16   ? launch_tc<16>(qm, k1, v1, k8, v8, q, nb, num_sms, stream)
                    : np == 32 ? launch_tc<32>(qm, k1, v1, k8, v8, q, nb, num_sms, stream)
+                   : np == 48 ? launch_tc<48>(qm, k1, v1, k8, v8, q, nb, num_sms, stream)
                               : launch_tc<64>(qm, k1, v1, k8, v8, q, nb, num_sms, stream);
     if (st != S3R_OK) return st;
     ++*launches;
