@@ -390,7 +390,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int g = 0;
     uint32_t tma_phase = 0;   // bit s: phase of tma[s]
     bool stop = false;
-    auto load_tiles = [&](const Item& x) {
+    // after_first() runs once, when the item's first tile is on its way
+    auto load_tiles = [&](const Item& x, auto&& after_first) {
       for (int t = 0; t < x.ntile && !stop; ++t, ++g) {
         const int s = g % nst;
         if (g >= nst && !wait_bar(smem_u32(&empty[s]), ((g / nst) - 1) & 1, abort_flag, p.err, p.wait_limit)) {
@@ -455,6 +456,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) mbar_arrive(smem_u32(&full[s]));
         }
         __syncwarp();
+        if (t == 0) after_first();
       }
     };
     if (!is_v) {
@@ -494,34 +496,52 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       return id;
     };
-    int next_a = -1, next_b = -1;
     int q_issued = 0;   // Q loads issued (item m's load lands on q_full[m & 1], phase (m >> 1) & 1)
-    int cur = item_id(0);
-    for (int m = 0; cur >= 0 && cur < nitems && !stop && !aborted(abort_flag); ++m) {
-      const int nxt = item_id(m + 1);
-      if (nxt < 0) break;
-      const Item x = make_item<NP>(cur, pref, lens_s, rid_s, batch, p);
-      cur = nxt;
-      int a = next_a, b = next_b;
-      if (m == 0) fetch_ids(x, a, b);
-      __syncwarp();   // every lane is done with the previous item's ids
-      ids_own[lane] = a;
-      ids_own[lane + 32] = b;
-      if (nxt < nitems) fetch_ids(make_item<NP>(nxt, pref, lens_s, rid_s, batch, p), next_a, next_b);
+    // K producer: item m's Q rows -> Q buffer m&1 by TMA (K-major, 128-byte swizzle) once the
+    // QK of item m-2 has read that buffer
+    auto load_q = [&](const Item& x, int m) -> bool {
+      const int qb = m & 1;
+      if (m >= 2 && !wait_bar(smem_u32(&B->q_empty[qb]), ((m - 2) >> 1) & 1, abort_flag, p.err, p.wait_limit))
+        return false;
+      if (lane == 0) mbar_arrive_expect_tx(smem_u32(&B->q_full[qb]), (uint32_t)(2 * R * 128));
       __syncwarp();
-      if (!is_v) {
-        // Q rows -> Q buffer m&1 by TMA (K-major, 128-byte swizzle) once QK(m-2) has read it
-        const int qb = m & 1;
-        if (m >= 2 && !wait_bar(smem_u32(&B->q_empty[qb]), ((m - 2) >> 1) & 1, abort_flag, p.err, p.wait_limit)) break;
-        if (lane == 0) mbar_arrive_expect_tx(smem_u32(&B->q_full[qb]), (uint32_t)(2 * R * 128));
-        __syncwarp();
-        if (lane < 2)
-          tma_load_3d(qbuf + qb * C::kQBytes + lane * (NP * 128), &tmQ, lane * 64, x.kvh * G,
-                      x.r * T, smem_u32(&B->q_full[qb]));
-        q_issued = m + 1;
-        __syncwarp();
-      }
-      load_tiles(x);
+      if (lane < 2)
+        tma_load_3d(qbuf + qb * C::kQBytes + lane * (NP * 128), &tmQ, lane * 64, x.kvh * G, x.r * T,
+                    smem_u32(&B->q_full[qb]));
+      q_issued = m + 1;
+      __syncwarp();
+      return true;
+    };
+    int cur = item_id(0);
+    Item x{};
+    int ida = -1, idb = -1;   // page ids of item m (two per lane)
+    if (cur >= 0 && cur < nitems) {
+      x = make_item<NP>(cur, pref, lens_s, rid_s, batch, p);
+      fetch_ids(x, ida, idb);
+      if (!is_v && !load_q(x, 0)) stop = true;
+    }
+    for (int m = 0; cur >= 0 && cur < nitems && !stop && !aborted(abort_flag); ++m) {
+      __syncwarp();   // every lane is done with the previous item's ids
+      ids_own[lane] = ida;
+      ids_own[lane + 32] = idb;
+      __syncwarp();
+      // The next item is claimed (K) or read from the ring (V), its page ids fetched and its
+      // Q rows loaded (K) once this item's first tile is on its way, so those round trips
+      // overlap the ring's waits instead of leaving the stream idle between items.
+      int nxt = -1, na = -1, nb = -1;
+      Item xn{};
+      bool ahead = false;
+      auto next_item = [&]() {
+        ahead = true;
+        nxt = item_id(m + 1);
+        if (nxt >= 0 && nxt < nitems) {
+          xn = make_item<NP>(nxt, pref, lens_s, rid_s, batch, p);
+          fetch_ids(xn, na, nb);
+          if (!is_v && !load_q(xn, m + 1)) stop = true;
+        }
+      };
+      load_tiles(x, next_item);
+      if (!ahead && !stop) next_item();
       if (!is_v && x.c == 0 && !stop) {   // the block's K/V enter the cache once per (request, head)
         const int* ptab = p.page_table + (size_t)x.r * p.max_pages;
         for (int idx = lane; idx < T * (kD / 8); idx += 32) {
@@ -538,6 +558,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           *reinterpret_cast<uint4*>(p.v_pool + dst) = *reinterpret_cast<const uint4*>(p.v_new + src);
         }
       }
+      cur = nxt;
+      x = xn;
+      ida = na;
+      idb = nb;
     }
     // nothing may still be landing in this ring (or a Q buffer) when the CTA exits, also after
     // an abort: these waits are for this warp's own copies and are not cut short
@@ -691,7 +715,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Warpgroup sg owns rows (columns of S and O^T) [sg*NH, sg*NH + NH) of every tile; the
     // two warpgroups only meet at the chunk's barriers for the MMA warp.
     constexpr int NH = NP / 2;               // rows per warpgroup
-    constexpr int BT = NP >= 48 ? 1 : (NP == 32 ? 2 : 4);   // tiles per tensor-memory wait (no spills)
+    // tiles per tensor-memory wait: one from 32 rows up (two tiles' values in flight made the
+    // 32-row pass 2 twice as slow, measured), four at 16
+    constexpr int BT = NP >= 32 ? 1 : 4;
     const int sw8 = warp - kSoftWarp0;       // 0..7
     const int sg = sw8 >> 2;                 // warpgroup
     const int sw4 = sw8 & 3;                 // warp within the warpgroup

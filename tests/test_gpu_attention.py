@@ -62,7 +62,9 @@ def test_verify_matches_oracle(Hq, Hkv, d, k, lens):
     (16, 8, 6, [3000, 900]),            # 14 rows
     (32, 8, 0, [1200, 2100]),           # 4 rows (prefill pass)
     (32, 8, 6, [9000, 12000, 7000, 10000, 11000, 8000, 9500, 10500]),   # several chunks per CTA
-    (32, 8, 8, [2500, 1025, 4000, 383, 385]),    # 36 rows: the 64-row tensor-memory kernel
+    (32, 8, 8, [2500, 1025, 4000, 383, 385]),    # 36 rows: the 48-row tensor-memory kernel
+    (64, 8, 4, [2049, 511, 513, 1700]),          # 40 rows (G = 8, k = 4), 48-row kernel
+    (64, 8, 5, [3000, 127, 129, 2600]),          # 48 rows (G = 8, k = 5): no padding rows
     (64, 8, 7, [1500, 3000, 769]),               # 64 rows (G = 8, k = 7)
 ])
 def test_verify_kernels_agree_with_oracle(Hq, Hkv, k, lens):

@@ -2,8 +2,9 @@
 (sparse_dense_kv_b200/csrc/verify_tc.cu), kept by hand in step with the kernel.
 
 Roles: the K producer (claims chunk ids and publishes them, one ahead of its own progress,
-through a ring of kRing slots with one barrier per slot; loads Q into one of two buffers
-and the K tiles through its 2-stage ring), the V producer (reads the ids from the ring,
+through a ring of kRing slots with one barrier per slot, once the current chunk's first K
+tile is issued; loads Q into one of two buffers one chunk ahead and the K tiles through its
+2-stage ring), the V producer (reads the ids from the ring after its chunk's first V tile,
 V tiles through its own 2-stage ring), the MMA warp (QK of chunk m and PV of chunk n < m,
 whichever has its next tile ready), and 8 softmax warps in two warpgroups (S double
 buffer, per-tile P^T release by the previous chunk's PV, O double buffer, warpgroup
@@ -98,33 +99,41 @@ def run(ntiles, ring, seed, kst=2, vst=2, KT=7, limit=20000):
         return W(f"item{m % ring}", (m // ring) & 1)
 
     def kprod():
+        # item m+1 is claimed and published, and its Q rows loaded, once item m's first K
+        # tile is on its way
         g = 0
         yield publish(0)
+        if M > 0:
+            yield A("qfull0")
         for m in range(M):
-            yield publish(m + 1)
-            if m >= 2:
-                yield W(f"qempty{m & 1}", ((m - 2) >> 1) & 1)
-            yield A(f"qfull{m & 1}")
-            for _ in range(ntiles[m]):
+            for t in range(ntiles[m]):
                 s = g % kst
                 if g >= kst:
                     yield W(f"kempty{s}", ((g // kst) - 1) & 1)
                 yield A(f"kfull{s}")
                 g += 1
+                if t == 0:
+                    yield publish(m + 1)
+                    if m + 1 < M:
+                        if m + 1 >= 2:
+                            yield W(f"qempty{(m + 1) & 1}", ((m - 1) >> 1) & 1)
+                        yield A(f"qfull{(m + 1) & 1}")
 
     def vprod():
+        # the id of item m+1 is read from the ring once item m's first V tile is on its way
         g = 0
         yield W_item(0)
         yield read(0)
         for m in range(M):
-            yield W_item(m + 1)
-            yield read(m + 1)
-            for _ in range(ntiles[m]):
+            for t in range(ntiles[m]):
                 s = g % vst
                 if g >= vst:
                     yield W(f"vempty{s}", ((g // vst) - 1) & 1)
                 yield A(f"vfull{s}")
                 g += 1
+                if t == 0:
+                    yield W_item(m + 1)
+                    yield read(m + 1)
 
     def mma():
         mk = tk = gk = nv = tv = gv = 0
