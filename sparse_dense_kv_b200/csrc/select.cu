@@ -111,7 +111,42 @@ __global__ void __launch_bounds__(kSelectThreads, 2) select_kernel(const SelectP
   // ---- scores -> order-preserving keys in shared memory
   bool bad = false;
   const float* srow = p.scores + ((size_t)r * p.Hkv + kvh) * p.score_stride;
-  for (int j = tid; j < N; j += blockDim.x) {
+  int jv = 0;   // positions below jv were loaded as 16-byte vectors
+  if constexpr (P == 1) {
+    if ((reinterpret_cast<uintptr_t>(srow) & 15u) == 0) {
+      // every thread has kU 16-byte loads in flight before it converts them
+      constexpr int kU = 4;
+      const int n4 = N >> 2;
+      const float4* s4 = reinterpret_cast<const float4*>(srow);
+      for (int b0 = 0; b0 < n4; b0 += kU * kSelectThreads) {
+        float4 v[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          const int i4 = b0 + u * kSelectThreads + tid;
+          v[u] = i4 < n4 ? __ldg(s4 + i4) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          const int i4 = b0 + u * kSelectThreads + tid;
+          if (i4 < n4) {
+            float x[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+            uint32_t kk[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              if (!isfinite(x[e])) {
+                bad = true;
+                x[e] = -INFINITY;
+              }
+              kk[e] = order_key(x[e]);
+            }
+            *reinterpret_cast<uint4*>(keys + 4 * i4) = make_uint4(kk[0], kk[1], kk[2], kk[3]);
+          }
+        }
+      }
+      jv = n4 * 4;
+    }
+  }
+  for (int j = jv + tid; j < N; j += blockDim.x) {
     float sigma;
     if constexpr (P == 1) {
       sigma = srow[j];

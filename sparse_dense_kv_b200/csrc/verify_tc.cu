@@ -7,26 +7,30 @@
 // comes from the verifier's last attention pass): rows (t, g) at positions L+t attend
 // positions 0..L+t; out, lse and every committed logit are written.
 //
-// Organisation (one persistent CTA per SM, 11 warps). A work item is (request, KV head,
+// Organisation (one persistent CTA per SM, 12 warps). A work item is (request, KV head,
 // chunk of up to 8, 7, 4 or 3 tiles of 128 positions at 16, 32, 48 or 64 rows: two S
-// buffers of a chunk and two O buffers fill the 512 columns of tensor memory). Items are claimed from a counter in the
-// workspace as CTAs progress (the K producer claims, a ring in shared memory tells the
-// other roles), so faster SMs take more of them.
+// buffers of a chunk and two O buffers fill the 512 columns of tensor memory). Items are
+// claimed from a counter in the workspace as CTAs progress (the K producer claims, a ring in
+// shared memory tells the other roles), so faster SMs take more of them.
 //   warp 0     K producer: per item it loads the item's Q rows into one of two Q buffers
 //              (3-D TMA box, rows t*G+g), then streams the chunk's K tiles through a
 //              2-stage ring with 4-D TMA over (d, slot, head, page): a tile of 8
 //              consecutive page ids is 2 boxes (one per 64-column half, 128-byte swizzle),
 //              otherwise one box per page and half. The tile holding the block (positions
 //              >= L) is patched after its TMA lands. It also writes the block into the cache.
+//              The next item is claimed, and its page ids and Q rows fetched, once the
+//              current item's first tile is on its way.
 //   warp 1     V producer: the same for the V tiles, through its own 2-stage ring, so the
 //              K stream of item n+1 and the V stream of item n run side by side.
-//   warp 2     MMA issuer: two queues in order, S^T tile t (128 positions x N rows, fp32) =
-//              K_t . Q^T into tensor memory for the QK of item m, and O^T (128 d x N) +=
-//              V_t^T . P_t^T for the PV of item n < m; whichever has its next tile ready is
-//              issued. K and Q are K-major operands (128-byte swizzle); V^T is MN-major (the V
-//              tile as it arrives) and so is P^T (N values per position in atoms of 16, 32
-//              or 64 rows: 32-, 64- or 128-byte swizzle; 48 rows are three 16-row atoms).
-//              S and O are double-buffered in tensor memory.
+//   warp 2     QK issuer: S^T tile t (128 positions x N rows, fp32) = K_t . Q^T into tensor
+//              memory, item after item. K and Q are K-major operands (128-byte swizzle).
+//   warp 11    PV issuer: O^T (128 d x N) += V_t^T . P_t^T, item after item, once the item's
+//              P^T is written. V^T is MN-major (the V tile as it arrives) and so is P^T (N
+//              values per position in atoms of 16, 32 or 64 rows: 32-, 64- or 128-byte
+//              swizzle; 48 rows are three 16-row atoms). S and O are double-buffered in
+//              tensor memory. The two issuers block on their own barriers, so neither
+//              product waits for the other's issue (each tile's eight dependent MMAs take
+//              about half a microsecond to issue).
 //   warps 3-10 softmax / epilogue, two warpgroups each owning half of the rows (one thread
 //              per tensor-memory lane = position or d): pass 1 reads every S tile, writes the
 //              committed logits and takes the chunk maximum per row; pass 2 re-reads them and
@@ -47,8 +51,9 @@ namespace tc {
 constexpr int kPos = 128;                   // positions per tile (MMA M)
 constexpr int kD = 128;                     // head_dim of this path
 constexpr int kMaxStages = 4;               // ring barriers per stream
-constexpr int kThreads = 352;               // K producer, V producer, MMA, 8 softmax warps
+constexpr int kThreads = 384;               // K producer, V producer, QK MMA, 8 softmax, PV MMA warps
 constexpr int kSoftWarp0 = 3;
+constexpr int kPvWarp = 11;
 constexpr int kBarBytes = 768;              // mbarriers and flags
 constexpr int kRing = 16;                   // item ids published by the K producer
 constexpr int kTileBytes = kPos * kD * 2;   // 32 KB: [2 halves][128 rows][128 B]
@@ -207,7 +212,7 @@ struct Bars {
   uint64_t vfull[kMaxStages], vempty[kMaxStages], vtma[kMaxStages];
   // one barrier pair per tensor-memory buffer (chunk parity), so that no barrier ever runs
   // two phases ahead of a waiter
-  uint64_t q_full[2], q_empty[2], p_full, fin;
+  uint64_t q_full[2], q_empty[2], p_full, fin[2];
   uint64_t s_full[2], s_empty[2], o_full[2], o_empty[2];
   uint64_t p_free[8];   // P^T tile t has been read by the PV of the previous chunk
   uint64_t wg[2];       // barrier of each softmax warpgroup (4 warps)
@@ -343,7 +348,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < kRing; ++i) mbar_init(smem_u32(&B->item_bar[i]), 1);
     mbar_init(smem_u32(&B->wg[0]), 4);
     mbar_init(smem_u32(&B->wg[1]), 4);
-    mbar_init(smem_u32(&B->fin), 1);
+    mbar_init(smem_u32(&B->fin[0]), 1);
+    mbar_init(smem_u32(&B->fin[1]), 1);
     B->abort_flag = 0;
     fence_mbar_init();
     fence_proxy_async();
@@ -568,152 +574,108 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int q = g - nst > 0 ? g - nst : 0; q < g; ++q) mbar_wait(smem_u32(&full[q % nst]), (q / nst) & 1);
     for (int m = q_issued - 2 > 0 ? q_issued - 2 : 0; m < q_issued; ++m)
       mbar_wait(smem_u32(&B->q_full[m & 1]), (uint32_t)(m >> 1) & 1u);
-  } else if (warp == 2) {
-    // ====================================================================== MMA warp ===
-    // Two queues in issue order: QK of item m (its K tiles) and PV of item n < m (its V
-    // tiles, once the softmax has written P^T). Whichever has its next tile ready is issued,
-    // so a V tile never waits behind K tiles of the next item, nor the reverse.
+  } else if (warp == 2 || warp == kPvWarp) {
+    // ===================================================================== MMA warps ===
+    // Warp 2 issues the QK products of the CTA's items in order (S^T = K_t . Q^T per tile,
+    // once the tile, the item's Q rows and a free S buffer are there); warp kPvWarp issues
+    // the PV products (O^T += V_t^T . P_t^T, once the softmax has written the item's P^T and
+    // its O buffer is free). Each blocks on its own barriers, so a PV never waits for the
+    // issue of QK tiles of a later item, nor the reverse.
+    const bool is_pv = warp == kPvWarp;
     constexpr uint32_t kIdQK = idesc_bf16(kPos, NP, false, false);
     constexpr uint32_t kIdPV = idesc_bf16(kD, NP, true, true);
-    auto ready = [&](uint64_t* bar, uint32_t parity) -> bool {   // warp-uniform test
-      const bool r = lane == 0 ? mbar_test(smem_u32(bar), parity) : false;
-      return __shfl_sync(kFull, r ? 1 : 0, 0) != 0;
-    };
-    int mk = 0, tk = 0, gk = 0, nv = 0, tv = 0, gv = 0;
-    int kend = -1;           // number of items, once the ring has said "no more"
-    bool kknown = false;     // xk holds item mk
-    int xv_of = -1;          // xv holds item xv_of
-    bool kgo = false, vgo = false, ok = true;
-    Item xk{}, xv{};
-    uint32_t idle = 0;
-    while (ok && (kend < 0 || nv < kend)) {
-      bool did = false;
-      if (kend < 0 && !kknown) {
-        const int slot = mk & (kRing - 1);
-        if (ready(&B->item_bar[slot], (uint32_t)(mk / kRing) & 1u)) {
-          // lane 0 made the acquiring test: it reads the id and hands it to the warp
-          int id = lane == 0 ? *reinterpret_cast<volatile int*>(&B->item_id[slot]) : 0;
-          id = __shfl_sync(kFull, id, 0);
-          if (id >= nitems) {
-            kend = mk;
-          } else {
-            xk = make_item<NP>(id, pref, lens_s, rid_s, batch, p);
-            kknown = true;
-          }
-          did = true;
-        }
-      }
-      if (kknown) {
-        if (!kgo) {
-          kgo = ready(&B->q_full[mk & 1], (mk >> 1) & 1) &&
-                (mk < 2 || ready(&B->s_empty[mk & 1], ((mk - 2) >> 1) & 1));
-          if (kgo) tc_fence_after();
-        }
-        if (kgo) {
+    if (!is_pv) {
+      int gk = 0;
+      for (int mk = 0;; ++mk) {
+        const int id = ring_id(mk);
+        if (id < 0 || id >= nitems) break;
+        const Item xk = make_item<NP>(id, pref, lens_s, rid_s, batch, p);
+        if (!wait_bar(smem_u32(&B->q_full[mk & 1]), (mk >> 1) & 1, abort_flag, p.err, p.wait_limit)) break;
+        if (mk >= 2 &&
+            !wait_bar(smem_u32(&B->s_empty[mk & 1]), ((mk - 2) >> 1) & 1, abort_flag, p.err, p.wait_limit))
+          break;
+        bool ok = true;
+        for (int tk = 0; tk < xk.ntile; ++tk, ++gk) {
           const int s = gk % C::kKSt;
-          if (ready(&B->kfull[s], (gk / C::kKSt) & 1)) {
-            tc_fence_after();
-            if (lane == 0) {
-              const uint32_t kt = sbase + C::kKRingOff + s * kTileBytes;
-              const uint32_t sd = tmem + (mk & 1) * C::kSCols + tk * NP;
-#pragma unroll
-              for (int kk = 0; kk < kD / 16; ++kk) {
-                const uint64_t ad = sdesc(kt + (kk >> 2) * (kPos * 128) + (kk & 3) * 32, 16, 1024, 2);
-                const uint64_t bd = sdesc(qbuf + (mk & 1) * C::kQBytes + (kk >> 2) * (NP * 128) +
-                                              (kk & 3) * 32, 16, 1024, 2);
-                tc_mma(sd, ad, bd, kIdQK, kk > 0 ? 1u : 0u);
-              }
-              tc_commit(smem_u32(&B->kempty[s]));
-            }
-            __syncwarp();
-            ++tk;
-            ++gk;
-            did = true;
-            if (tk == xk.ntile) {
-              if (lane == 0) {
-                tc_commit(smem_u32(&B->s_full[mk & 1]));
-                tc_commit(smem_u32(&B->q_empty[mk & 1]));
-              }
-              __syncwarp();
-              ++mk;
-              tk = 0;
-              kgo = false;
-              kknown = false;
-            }
+          if (!wait_bar(smem_u32(&B->kfull[s]), (gk / C::kKSt) & 1, abort_flag, p.err, p.wait_limit)) {
+            ok = false;
+            break;
           }
-        }
-      }
-      if (nv < mk) {
-        if (xv_of != nv) {   // item nv's id was read from the ring when its QK started
-          int id = lane == 0 ? *reinterpret_cast<volatile int*>(&B->item_id[nv & (kRing - 1)]) : 0;
-          id = __shfl_sync(kFull, id, 0);
-          xv = make_item<NP>(id, pref, lens_s, rid_s, batch, p);
-          xv_of = nv;
-        }
-        if (!vgo) {
-          vgo = ready(&B->p_full, nv & 1) &&
-                (nv < 2 || ready(&B->o_empty[nv & 1], ((nv - 2) >> 1) & 1));
-          if (vgo) tc_fence_after();
-        }
-        if (vgo) {
-          const int s = gv % C::kVSt;
-          if (ready(&B->vfull[s], (gv / C::kVSt) & 1)) {
-            tc_fence_after();
-            if (lane == 0) {
-              const uint32_t vt = sbase + C::kVRingOff + s * kTileBytes;
-              const uint32_t pt = pbuf + tv * C::kPTile;
-              const uint32_t od = tmem + C::kOCol + (nv & 1) * NP;
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t kt = sbase + C::kKRingOff + s * kTileBytes;
+            const uint32_t sd = tmem + (mk & 1) * C::kSCols + tk * NP;
 #pragma unroll
-              for (int kk = 0; kk < kPos / 16; ++kk) {
-                const uint64_t ad = sdesc(vt + kk * 2048, kPos * 128, 1024, 2);
-                // MN-major P^T: LBO = stride between atoms along N, SBO = stride between
-                // groups of 8 positions (one atom row is kPAtomRows * 2 bytes)
-                const uint64_t bd = sdesc(pt + kk * 16 * C::kPAtomRows * 2, C::kPAtomBytes,
-                                          8 * C::kPAtomRows * 2, C::kPSwz);
-                tc_mma(od, ad, bd, kIdPV, (tv > 0 || kk > 0) ? 1u : 0u);
-              }
-              tc_commit(smem_u32(&B->vempty[s]));
-              tc_commit(smem_u32(&B->p_free[tv]));
+            for (int kk = 0; kk < kD / 16; ++kk) {
+              const uint64_t ad = sdesc(kt + (kk >> 2) * (kPos * 128) + (kk & 3) * 32, 16, 1024, 2);
+              const uint64_t bd = sdesc(qbuf + (mk & 1) * C::kQBytes + (kk >> 2) * (NP * 128) +
+                                            (kk & 3) * 32, 16, 1024, 2);
+              tc_mma(sd, ad, bd, kIdQK, kk > 0 ? 1u : 0u);
             }
-            __syncwarp();
-            ++tv;
-            ++gv;
-            did = true;
-            if (tv == xv.ntile) {
-              if (lane == 0) {
-                // every P^T tile's barrier completes once per chunk, used or not
-                for (int t = xv.ntile; t < C::kTiles; ++t) tc_commit(smem_u32(&B->p_free[t]));
-                tc_commit(smem_u32(&B->o_full[nv & 1]));
-              }
-              __syncwarp();
-              ++nv;
-              tv = 0;
-              vgo = false;
-            }
+            tc_commit(smem_u32(&B->kempty[s]));
           }
+          __syncwarp();
         }
-      }
-      if (did) {
-        idle = 0;
-      } else if (++idle >= (uint32_t)p.wait_limit) {
+        if (!ok) break;
         if (lane == 0) {
-          *abort_flag = 1;
-          set_error(p.err, S3R_ERR_TIMEOUT);
+          tc_commit(smem_u32(&B->s_full[mk & 1]));
+          tc_commit(smem_u32(&B->q_empty[mk & 1]));
         }
-        ok = false;
-      } else {
-        if ((idle & 1023) == 0 && aborted(abort_flag)) ok = false;
-        __nanosleep(32);
+        __syncwarp();
+      }
+    } else {
+      int gv = 0;
+      for (int nv = 0;; ++nv) {
+        const int id = ring_id(nv);
+        if (id < 0 || id >= nitems) break;
+        const Item xv = make_item<NP>(id, pref, lens_s, rid_s, batch, p);
+        if (!wait_bar(smem_u32(&B->p_full), nv & 1, abort_flag, p.err, p.wait_limit)) break;
+        if (nv >= 2 &&
+            !wait_bar(smem_u32(&B->o_empty[nv & 1]), ((nv - 2) >> 1) & 1, abort_flag, p.err, p.wait_limit))
+          break;
+        bool ok = true;
+        for (int tv = 0; tv < xv.ntile; ++tv, ++gv) {
+          const int s = gv % C::kVSt;
+          if (!wait_bar(smem_u32(&B->vfull[s]), (gv / C::kVSt) & 1, abort_flag, p.err, p.wait_limit)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t vt = sbase + C::kVRingOff + s * kTileBytes;
+            const uint32_t pt = pbuf + tv * C::kPTile;
+            const uint32_t od = tmem + C::kOCol + (nv & 1) * NP;
+#pragma unroll
+            for (int kk = 0; kk < kPos / 16; ++kk) {
+              const uint64_t ad = sdesc(vt + kk * 2048, kPos * 128, 1024, 2);
+              // MN-major P^T: LBO = stride between atoms along N, SBO = stride between
+              // groups of 8 positions (one atom row is kPAtomRows * 2 bytes)
+              const uint64_t bd = sdesc(pt + kk * 16 * C::kPAtomRows * 2, C::kPAtomBytes,
+                                        8 * C::kPAtomRows * 2, C::kPSwz);
+              tc_mma(od, ad, bd, kIdPV, (tv > 0 || kk > 0) ? 1u : 0u);
+            }
+            tc_commit(smem_u32(&B->vempty[s]));
+            tc_commit(smem_u32(&B->p_free[tv]));
+          }
+          __syncwarp();
+        }
+        if (!ok) break;
+        if (lane == 0) {
+          // every P^T tile's barrier completes once per chunk, used or not
+          for (int t = xv.ntile; t < C::kTiles; ++t) tc_commit(smem_u32(&B->p_free[t]));
+          tc_commit(smem_u32(&B->o_full[nv & 1]));
+        }
+        __syncwarp();
       }
     }
-    // make sure nothing issued is still running before the tensor memory goes away
-    if (lane == 0) tc_commit(smem_u32(&B->fin));
+    // make sure nothing this warp issued is still running before the tensor memory goes away
+    if (lane == 0) tc_commit(smem_u32(&B->fin[is_pv ? 1 : 0]));
     __syncwarp();
-    mbar_wait(smem_u32(&B->fin), 0);   // not cut short by an abort: the work is in flight
+    mbar_wait(smem_u32(&B->fin[is_pv ? 1 : 0]), 0);   // not cut short by an abort: the work is in flight
   } else {
     // ================================================================ softmax warps ===
     // Warpgroup sg owns rows (columns of S and O^T) [sg*NH, sg*NH + NH) of every tile; the
-    // two warpgroups only meet at the chunk's barriers for the MMA warp.
+    // two warpgroups only meet at the chunk's barriers for the MMA warps.
     constexpr int NH = NP / 2;               // rows per warpgroup
     // tiles per tensor-memory wait: one from 32 rows up (two tiles' values in flight made the
     // 32-row pass 2 twice as slow, measured), four at 16

@@ -5,16 +5,15 @@ Roles: the K producer (claims chunk ids and publishes them, one ahead of its own
 through a ring of kRing slots with one barrier per slot, once the current chunk's first K
 tile is issued; loads Q into one of two buffers one chunk ahead and the K tiles through its
 2-stage ring), the V producer (reads the ids from the ring after its chunk's first V tile,
-V tiles through its own 2-stage ring), the MMA warp (QK of chunk m and PV of chunk n < m,
-whichever has its next tile ready), and 8 softmax warps in two warpgroups (S double
-buffer, per-tile P^T release by the previous chunk's PV, O double buffer, warpgroup
-barriers). Each step of each role is an arrive or a wait on a phase-parity barrier, as in
+V tiles through its own 2-stage ring), the QK issuer (chunk after chunk: Q, a free S buffer,
+each K tile) and the PV issuer (chunk after chunk: the whole P^T, a free O buffer, each V
+tile), and 8 softmax warps in two warpgroups (S double buffer, per-tile P^T release by the
+previous chunk's PV, O double buffer, warpgroup barriers). Each step of each role is an arrive or a wait on a phase-parity barrier, as in
 the kernel; a scheduler picks a random role at every step.
 
 Checked over many random schedules and chunk / tile counts: the roles never deadlock, and
 no ring slot is overwritten before every read of its previous id (the V producer reads
-each id once, the MMA warp twice: when the chunk's QK starts and when its PV starts, each
-softmax warp once). Over such schedules the smallest ring that never fails is 6 slots (5
+each id once, the QK and the PV issuer once each, each softmax warp once). Over such schedules the smallest ring that never fails is 6 slots (5
 fails now and then); the kernel has 16. A ring of 4 slots must fail the overwrite check
 (negative control).
 """
@@ -71,7 +70,7 @@ def run(ntiles, ring, seed, kst=2, vst=2, KT=7, limit=20000):
 
     slot_item = {}                 # slot -> id published there last
     reads = {}                     # id -> reads done
-    NEED = 1 + 2 + 8               # V producer, MMA (QK, PV), 8 softmax warps
+    NEED = 1 + 2 + 8               # V producer, the QK and PV issuers, 8 softmax warps
     state = {"overwrite": False}
 
     def W(name, parity):
@@ -135,60 +134,43 @@ def run(ntiles, ring, seed, kst=2, vst=2, KT=7, limit=20000):
                     yield W_item(m + 1)
                     yield read(m + 1)
 
-    def mma():
-        mk = tk = gk = nv = tv = gv = 0
-        kend = None
-        known = kgo = vgo = False
-        xv_of = -1
-        while kend is None or nv < kend:
-            did = False
-            if kend is None and not known and bars[f"item{mk % ring}"].test((mk // ring) & 1):
-                yield read(mk)
-                if mk == M:
-                    kend = M
-                else:
-                    known = True
-                did = True
-            if known:
-                if not kgo:
-                    kgo = bars[f"qfull{mk & 1}"].test((mk >> 1) & 1) and (
-                        mk < 2 or bars[f"sempty{mk & 1}"].test(((mk - 2) >> 1) & 1))
-                if kgo:
-                    s = gk % kst
-                    if bars[f"kfull{s}"].test((gk // kst) & 1):
-                        yield A(f"kempty{s}")
-                        tk += 1
-                        gk += 1
-                        did = True
-                        if tk == ntiles[mk]:
-                            yield A(f"sfull{mk & 1}")
-                            yield A(f"qempty{mk & 1}")
-                            mk += 1
-                            tk = 0
-                            kgo = known = False
-            if nv < mk:
-                if xv_of != nv:
-                    yield read(nv)         # the PV's id, read from the ring again
-                    xv_of = nv
-                if not vgo:
-                    vgo = bars["pfull"].test(nv & 1) and (nv < 2 or bars[f"oempty{nv & 1}"].test(((nv - 2) >> 1) & 1))
-                if vgo:
-                    s = gv % vst
-                    if bars[f"vfull{s}"].test((gv // vst) & 1):
-                        yield A(f"vempty{s}")
-                        yield A(f"pfree{tv}")
-                        tv += 1
-                        gv += 1
-                        did = True
-                        if tv == ntiles[nv]:
-                            for t in range(ntiles[nv], KT):
-                                yield A(f"pfree{t}")
-                            yield A(f"ofull{nv & 1}")
-                            nv += 1
-                            tv = 0
-                            vgo = False
-            if not did:
-                yield ("idle",)
+    def qk():
+        gk = 0
+        for mk in range(M + 1):
+            yield W_item(mk)
+            yield read(mk)
+            if mk == M:
+                return
+            yield W(f"qfull{mk & 1}", (mk >> 1) & 1)
+            if mk >= 2:
+                yield W(f"sempty{mk & 1}", ((mk - 2) >> 1) & 1)
+            for _ in range(ntiles[mk]):
+                s = gk % kst
+                yield W(f"kfull{s}", (gk // kst) & 1)
+                yield A(f"kempty{s}")
+                gk += 1
+            yield A(f"sfull{mk & 1}")
+            yield A(f"qempty{mk & 1}")
+
+    def pv():
+        gv = 0
+        for nv in range(M + 1):
+            yield W_item(nv)
+            yield read(nv)
+            if nv == M:
+                return
+            yield W("pfull", nv & 1)
+            if nv >= 2:
+                yield W(f"oempty{nv & 1}", ((nv - 2) >> 1) & 1)
+            for tv in range(ntiles[nv]):
+                s = gv % vst
+                yield W(f"vfull{s}", (gv // vst) & 1)
+                yield A(f"vempty{s}")
+                yield A(f"pfree{tv}")
+                gv += 1
+            for t in range(ntiles[nv], KT):
+                yield A(f"pfree{t}")
+            yield A(f"ofull{nv & 1}")
 
     def soft(w):
         sg = w // 4
@@ -226,7 +208,7 @@ def run(ntiles, ring, seed, kst=2, vst=2, KT=7, limit=20000):
             yield W(f"ofull{m & 1}", (m >> 1) & 1)
             yield A(f"oempty{m & 1}")
 
-    roles = {"K": kprod(), "V": vprod(), "MMA": mma()}
+    roles = {"K": kprod(), "V": vprod(), "QK": qk(), "PV": pv()}
     for w in range(8):
         roles[f"S{w}"] = soft(w)
     cur = {r: next(g) for r, g in roles.items()}
