@@ -229,12 +229,14 @@ def round_bytes(spec, lens, vb, db, sb, greedy=False):
     """Algorithmic HBM bytes of one round: verify K/V reads and score-logit writes, the
     selection's score-logit reads and its per-position score array (written, read), the
     draft K/V and index reads, and the samplers' logit reads (draft sampling: one row per
-    request and step; speculative sampling: 2k+1 rows, plus the drawn row again)."""
+    request and step, whose normaliser the speculative sampling reuses; speculative sampling:
+    the k+1 target rows, plus the drawn row's target and draft rows again; greedy: the k+1
+    target rows)."""
     NR, Hkv, V, k = spec.num_requests, spec.num_kv_heads, spec.vocab, spec.k
     pos = int(sum(lens))
     select = sb + 2 * 4 * pos * Hkv
     draft_sampling = k * NR * V * 4
-    spec_sampling = NR * (2 * k + 1) * V * 4 + NR * V * 4 * (1 if greedy else 2)
+    spec_sampling = NR * (k + 1) * V * 4 + (0 if greedy else NR * V * 4 * 2)
     parts = {"verify_kv": int(vb), "verify_scores": int(sb), "select": int(select),
              "draft_kv": int(sum(db)), "draft_sampling": int(draft_sampling),
              "spec_sampling": int(spec_sampling)}

@@ -198,6 +198,14 @@ S3R_API int s3r_sparse_draft_attn(const s3r_kv_cache* cache, const s3r_batch* ba
                           const int32_t* sel_count, void* out, float* lse, void* ws,
                           size_t ws_bytes, s3r_stream_t stream);
 
+/* Normaliser of one row of logits x: max = max_v x_v and sum = sum_v exp(x_v - max), so that
+ * softmax(x)_v = exp(x_v - max) / sum (non-finite entries count as -inf). 16 bytes. */
+typedef struct s3r_row_norm {
+  float max;
+  float reserved;
+  double sum;
+} s3r_row_norm;
+
 /* Draft-token sampling (temperature 1). For request r at step i = draft_step[r]:
  * q_i = softmax(q_logits[r][i][0..vocab-1]); u = Philox4x32-10(key = seed,
  * counter = (L+i+1, r, 0, 0)) word 0 >> 8, times 2^-24; the token is the smallest v with
@@ -206,10 +214,13 @@ S3R_API int s3r_sparse_draft_attn(const s3r_kv_cache* cache, const s3r_batch* ba
  * [num_requests][k]. margins (fp32 [num_requests][k], may be NULL) receives the draw's
  * distance to the nearer edge of the drawn token's cell, min(u - C_{v-1}/Z, C_v/Z - u),
  * as this call computed the sums: a draw with a margin below the rounding of those sums
- * may go either way in another correct implementation. */
+ * may go either way in another correct implementation. q_norm (s3r_row_norm
+ * [num_requests][k], may be NULL) receives the normaliser of row i that the draw used, so
+ * that s3r_spec_sample can take it instead of streaming the row again. */
 S3R_API int s3r_draft_sample(const s3r_batch* batch, const int32_t* draft_step, int32_t k,
                      const float* q_logits, int32_t vocab, uint64_t seed, int32_t* draft_tokens,
-                     float* margins, void* ws, size_t ws_bytes, s3r_stream_t stream);
+                     float* margins, s3r_row_norm* q_norm, void* ws, size_t ws_bytes,
+                     s3r_stream_t stream);
 
 /* s3r_draft_sample without a workspace. The paper has no counterpart: this is a
  * library convenience for callers that cannot hand the library device memory at the
@@ -249,11 +260,14 @@ S3R_API int s3r_draft_sample_noalloc(const s3r_batch* batch, const int32_t* draf
  * their boundaries, in decision order: |u1 - p_j(d)/q_j(d)| for each decided draft (the a
  * accepted ones and the rejected one, if any), then the draw's distance to the nearer edge
  * of the drawn token's cell (as for s3r_draft_sample); min(a + 1, k) + 1 entries are
- * written, the rest untouched. */
+ * written, the rest untouched. q_norm (s3r_row_norm [num_requests][k], may be NULL): the
+ * normalisers of the q rows as s3r_draft_sample wrote them for these q_logits; with it the
+ * q rows are read only at the drafted tokens and in the drawn row, not streamed whole
+ * (13 -> 7 rows at k = 6). Without it they are computed here. */
 S3R_API int s3r_spec_sample(const s3r_batch* batch, int32_t k, const float* p_logits,
                     const float* q_logits, const int32_t* draft_tokens, int32_t vocab,
                     uint64_t seed, int32_t* out_tokens, int32_t* n_out, float* margins,
-                    void* ws, size_t ws_bytes, s3r_stream_t stream);
+                    const s3r_row_norm* q_norm, void* ws, size_t ws_bytes, s3r_stream_t stream);
 
 /* Greedy (temperature 0) mode ([Listing] Table 4 setting: component measurements decode
  * greedily). s3r_draft_argmax: draft_tokens[r][i] = argmax of q_logits[r][i], i =

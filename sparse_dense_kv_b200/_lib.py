@@ -77,9 +77,9 @@ def _load():
         "s3r_select_kv_pages": (ctypes.c_int, [C, B, P, P, I32, I32, I32, P, I32, P, P, SZ, P]),
         "s3r_select_pages_from_scores": (ctypes.c_int, [C, B, P, I32, I32, I32, P, I32, P, P, SZ, P]),
         "s3r_sparse_draft_attn": (ctypes.c_int, [C, B, P, P, I32, P, P, I32, P, I32, P, P, P, P, SZ, P]),
-        "s3r_draft_sample": (ctypes.c_int, [B, P, I32, P, I32, U64, P, P, P, SZ, P]),
+        "s3r_draft_sample": (ctypes.c_int, [B, P, I32, P, I32, U64, P, P, P, P, SZ, P]),
         "s3r_draft_sample_noalloc": (ctypes.c_int, [B, P, I32, P, I32, U64, P, P, P]),
-        "s3r_spec_sample": (ctypes.c_int, [B, I32, P, P, P, I32, U64, P, P, P, P, SZ, P]),
+        "s3r_spec_sample": (ctypes.c_int, [B, I32, P, P, P, I32, U64, P, P, P, P, P, SZ, P]),
         "s3r_draft_argmax": (ctypes.c_int, [B, P, I32, P, I32, P, P, SZ, P]),
         "s3r_sched_simulate": (ctypes.c_int, [ctypes.POINTER(SchedConfig), I32, P, P, P, ctypes.c_int64,
                                               P, ctypes.c_int64, ctypes.POINTER(SchedResult), P,
@@ -268,15 +268,30 @@ def s3r_sparse_draft_attn(cache, batch, draft_step, q, k_new, v_new, sel_idx, se
         _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)), "s3r_sparse_draft_attn")
 
 
+def _norms(t, what):
+    """s3r_row_norm [NR][k] as a float64 tensor [NR][k][2] (float max, float unused, double sum)."""
+    if t is not None and (t.dtype != torch.float64 or t.shape[-1] != 2):
+        raise TypeError(f"{what} must be a float64 [NR][k][2] tensor (s3r_row_norm records)")
+    return _ptr(t, torch.float64, what, allow_none=True)
+
+
+def row_norms(t) -> tuple:
+    """(max, sum) arrays of a q_norm tensor written by s3r_draft_sample."""
+    raw = t.detach().cpu().contiguous()
+    mx = raw.view(torch.float32)[..., 0]
+    return mx.numpy(), raw[..., 1].numpy()
+
+
 def s3r_draft_sample(batch, draft_step, k, q_logits, vocab, seed, draft_tokens, ws, stream=None,
-                     margins=None):
-    """margins: optional fp32 [NR][k] tensor receiving each draw's boundary margin."""
+                     margins=None, q_norm=None):
+    """margins: optional fp32 [NR][k] tensor receiving each draw's boundary margin; q_norm:
+    optional float64 [NR][k][2] tensor receiving the rows' normalisers (s3r_row_norm)."""
     _check(_lib.s3r_draft_sample(
         ctypes.byref(batch), _ptr(draft_step, torch.int32, "draft_step"), k,
         _ptr(q_logits, torch.float32, "q_logits"), vocab, seed,
         _ptr(draft_tokens, torch.int32, "draft_tokens"),
-        _ptr(margins, torch.float32, "margins", allow_none=True), _ptr(ws, torch.uint8, "ws"),
-        ws.numel(), _stream(stream)), "s3r_draft_sample")
+        _ptr(margins, torch.float32, "margins", allow_none=True), _norms(q_norm, "q_norm"),
+        _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)), "s3r_draft_sample")
 
 
 def s3r_draft_sample_noalloc(batch, draft_step, k, q_logits, vocab, seed, draft_tokens, err_word,
@@ -294,15 +309,16 @@ def s3r_draft_sample_noalloc(batch, draft_step, k, q_logits, vocab, seed, draft_
 
 
 def s3r_spec_sample(batch, k, p_logits, q_logits, draft_tokens, vocab, seed, out_tokens, n_out,
-                    ws, stream=None, margins=None):
-    """margins: optional fp32 [NR][k+1] tensor receiving the decisions' boundary margins."""
+                    ws, stream=None, margins=None, q_norm=None):
+    """margins: optional fp32 [NR][k+1] tensor receiving the decisions' boundary margins;
+    q_norm: the draft rows' normalisers s3r_draft_sample wrote (optional)."""
     f32, i32 = torch.float32, torch.int32
     _check(_lib.s3r_spec_sample(
         ctypes.byref(batch), k, _ptr(p_logits, f32, "p_logits"),
         _ptr(q_logits, f32, "q_logits", allow_none=(k == 0)),
         _ptr(draft_tokens, i32, "draft_tokens", allow_none=(k == 0)), vocab, seed,
         _ptr(out_tokens, i32, "out_tokens"), _ptr(n_out, i32, "n_out"),
-        _ptr(margins, f32, "margins", allow_none=True),
+        _ptr(margins, f32, "margins", allow_none=True), _norms(q_norm, "q_norm"),
         _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)), "s3r_spec_sample")
 
 

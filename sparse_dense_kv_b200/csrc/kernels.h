@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/s3r.h"
+
 namespace s3r {
 
 constexpr int kVerifyChunk = 1024;   // positions per verify CTA (multiple of 64)
@@ -106,6 +108,7 @@ struct SampleParams {
   size_t sub_off;              // byte offset of the sub-block sums (draft or spec draw)
   int num_requests;            // size of every per-request array (request ids are checked)
   float* margins;              // optional: draft [NR][k], spec [NR][k+1] decision margins
+  s3r_row_norm* q_norm;        // optional: draft rows' normalisers [NR][k] (draft: out, spec: in)
 };
 
 // Record the CUDA error behind an S3R_ERR_CUDA status (readable by s3r_last_error_message)

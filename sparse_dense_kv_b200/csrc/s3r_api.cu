@@ -533,12 +533,14 @@ int s3r_sparse_draft_attn(const s3r_kv_cache* cache, const s3r_batch* batch,
 
 int s3r_draft_sample(const s3r_batch* batch, const int32_t* draft_step, int32_t k,
                      const float* q_logits, int32_t vocab, uint64_t seed, int32_t* draft_tokens,
-                     float* margins, void* ws, size_t ws_bytes, s3r_stream_t stream) {
+                     float* margins, s3r_row_norm* q_norm, void* ws, size_t ws_bytes,
+                     s3r_stream_t stream) {
   S3R_TRY(check_batch(batch, false));
   if (k < 1 || k > S3R_MAX_K) return S3R_ERR_UNSUPPORTED;
   if (vocab < 1 || vocab > 64 * kVocabChunk) return S3R_ERR_UNSUPPORTED;
   if (!draft_step || !q_logits || !draft_tokens || !aligned4(draft_step) ||
-      !aligned4(q_logits) || !aligned4(draft_tokens) || (margins && !aligned4(margins)))
+      !aligned4(q_logits) || !aligned4(draft_tokens) || (margins && !aligned4(margins)) ||
+      (q_norm && (reinterpret_cast<uintptr_t>(q_norm) & 7u)))
     return S3R_ERR_INVALID_ARG;
   if (batch->batch == 0) return S3R_OK;
   S3R_TRY(check_ws(ws, ws_bytes, sample_need(batch->num_requests, 1, k, vocab)));
@@ -559,6 +561,7 @@ int s3r_draft_sample(const s3r_batch* batch, const int32_t* draft_step, int32_t 
   p.part = w.part;
   p.num_requests = batch->num_requests;
   p.margins = margins;
+  p.q_norm = q_norm;
   p.sub_off = draft_sub_offset(batch->num_requests, vocab);
   return finish(launch_draft_sample(p, batch->batch, (cudaStream_t)stream), 1);
 }
@@ -609,12 +612,13 @@ int s3r_draft_sample_noalloc(const s3r_batch* batch, const int32_t* draft_step, 
 int s3r_spec_sample(const s3r_batch* batch, int32_t k, const float* p_logits,
                     const float* q_logits, const int32_t* draft_tokens, int32_t vocab,
                     uint64_t seed, int32_t* out_tokens, int32_t* n_out, float* margins,
-                    void* ws, size_t ws_bytes, s3r_stream_t stream) {
+                    const s3r_row_norm* q_norm, void* ws, size_t ws_bytes, s3r_stream_t stream) {
   S3R_TRY(check_batch(batch, false));
   if (k < 0 || k > S3R_MAX_K) return S3R_ERR_UNSUPPORTED;
   if (vocab < 1 || vocab > 64 * kVocabChunk) return S3R_ERR_UNSUPPORTED;
   if (!p_logits || !out_tokens || !n_out || !aligned4(p_logits) || !aligned4(out_tokens) ||
-      !aligned4(n_out) || (margins && !aligned4(margins)))
+      !aligned4(n_out) || (margins && !aligned4(margins)) ||
+      (q_norm && (reinterpret_cast<uintptr_t>(q_norm) & 7u)))
     return S3R_ERR_INVALID_ARG;
   if (k > 0 && (!q_logits || !draft_tokens || !aligned4(q_logits) || !aligned4(draft_tokens)))
     return S3R_ERR_INVALID_ARG;
@@ -639,6 +643,7 @@ int s3r_spec_sample(const s3r_batch* batch, int32_t k, const float* p_logits,
   p.part = w.part;
   p.num_requests = batch->num_requests;
   p.margins = margins;
+  p.q_norm = const_cast<s3r_row_norm*>(q_norm);
   spec_offsets(batch->num_requests, k, vocab, &p.plan_off, &p.draw_off, &p.sub_off);
   int launches = 0;
   const int st = launch_spec_sample(p, batch->batch, (cudaStream_t)stream, &launches);

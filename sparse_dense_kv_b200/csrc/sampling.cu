@@ -379,6 +379,13 @@ __global__ void __launch_bounds__(kSampThreads, kDsMinBlocks) draft_sample_kerne
   if (threadIdx.x == 0) {
     p.draft_out[(size_t)r * p.k + i] = tok;
     if (p.margins) p.margins[(size_t)r * p.k + i] = Z > 0.0 ? (float)(mrg / Z) : 0.f;
+    if (p.q_norm) {
+      s3r_row_norm nm;
+      nm.max = M;
+      nm.reserved = 0.f;
+      nm.sum = Z;
+      p.q_norm[(size_t)r * p.k + i] = nm;
+    }
   }
 }
 
@@ -395,6 +402,9 @@ __global__ void __launch_bounds__(kSampThreads) spec_norm_kernel(const SamplePar
     return;
   }
   const int k = p.k, V = p.vocab, nrows = 2 * k + 1;
+  // rows 0..k: p, rows k+1..2k: q; with the draft rows' normalisers given, only the p rows
+  // are streamed (the grid's second dimension is k + 1)
+  const int nstream = p.q_norm ? k + 1 : nrows;
   const float* row = (rw <= k) ? p.p_logits + ((size_t)r * (k + 1) + rw) * V
                                : p.q_logits + ((size_t)r * k + (rw - k - 1)) * V;
   MS* part = reinterpret_cast<MS*>(p.part) + (size_t)r * nrows * p.nvch;
@@ -405,12 +415,18 @@ __global__ void __launch_bounds__(kSampThreads) spec_norm_kernel(const SamplePar
   if (bad) set_error(p.err, S3R_ERR_NONFINITE);
   const MS tot = block_ms(m, s);
   if (threadIdx.x == 0) part[rw * p.nvch + c] = tot;
-  if (!last_of(p.tickets + r, nrows * p.nvch, &s_flag)) return;
+  if (!last_of(p.tickets + r, nstream * p.nvch, &s_flag)) return;
 
-  // normalisers of every row: one warp per row, the row's chunk partials loaded in parallel
+  // normalisers of every row: one warp per streamed row, the row's chunk partials loaded in
+  // parallel; the q rows' from q_norm when given
   __shared__ double s_cs[8][64];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int row = warp; row < nrows; row += kSampThreads / 32) {
+  if (p.q_norm && (int)threadIdx.x < k) {
+    const s3r_row_norm nm = p.q_norm[(size_t)r * k + threadIdx.x];
+    sM[k + 1 + threadIdx.x] = nm.max;
+    sZ[k + 1 + threadIdx.x] = nm.sum;
+  }
+  for (int row = warp; row < nstream; row += kSampThreads / 32) {
     const float M = merge_partials_warp(part + row * p.nvch, p.nvch, s_cs[warp]);
     __syncwarp();
     double z = 0.0;
@@ -768,7 +784,7 @@ int launch_draft_sample(const SampleParams& p, int batch, cudaStream_t stream) {
 }
 
 int launch_spec_sample(const SampleParams& p, int batch, cudaStream_t stream, int* launches) {
-  dim3 g1(batch, 2 * p.k + 1, p.nvch);
+  dim3 g1(batch, p.q_norm ? p.k + 1 : 2 * p.k + 1, p.nvch);
   launch_pdl(spec_norm_kernel, g1, kSampThreads, 0, stream, p);
   if (cuda_status(cudaGetLastError(), __func__) != S3R_OK) return S3R_ERR_CUDA;
   dim3 g2(batch, p.nvch);

@@ -42,6 +42,9 @@ class RoundBuffers:
         # decision margins the samplers report (draft draws; accept tests and the final draw)
         self._draft_margins = torch.zeros(num_requests * k_max, dtype=f32, device=device)
         self._spec_margins = torch.zeros(num_requests * T, dtype=f32, device=device)
+        # the draft rows' normalisers (s3r_row_norm), written by the draft sampler and read by
+        # the speculative sampler instead of streaming the q rows again
+        self._q_norm = torch.zeros(num_requests * k_max * 2, dtype=torch.float64, device=device)
         self.prefill_lse = torch.empty((num_requests, 1, num_q_heads), dtype=f32, device=device)
         self.sel_idx = torch.zeros((num_requests, num_kv_heads, sel_stride), dtype=i32, device=device)
         self.sel_count = torch.zeros((num_requests, num_kv_heads), dtype=i32, device=device)
@@ -63,6 +66,7 @@ class RoundBuffers:
         self.out_tokens = self._out_tokens[: NR * T].view(NR, T)
         self.draft_margins = self._draft_margins[: NR * k].view(NR, k)
         self.spec_margins = self._spec_margins[: NR * T].view(NR, T)
+        self.q_norm = self._q_norm[: NR * k * 2].view(NR, k, 2)
 
 
 class S3REngine:
@@ -140,7 +144,8 @@ class S3REngine:
                                self.buf.draft_tokens, self.ws)
             return
         L.s3r_draft_sample(self.batch, self.buf.steps[i], self.k, q_logits, self.vocab, self.seed,
-                           self.buf.draft_tokens, self.ws, margins=self.buf.draft_margins)
+                           self.buf.draft_tokens, self.ws, margins=self.buf.draft_margins,
+                           q_norm=self.buf.q_norm)
 
     def draft_step(self, i, q_block, k_block, v_block, q_logits, draft_logits_fn=None):
         self.draft_attn(i, q_block, k_block, v_block)
@@ -163,7 +168,8 @@ class S3REngine:
                                 b.out_tokens, b.n_out, self.ws)
         else:
             L.s3r_spec_sample(self.batch, self.k, p_logits, q_logits, b.draft_tokens, self.vocab,
-                              self.seed, b.out_tokens, b.n_out, self.ws, margins=b.spec_margins)
+                              self.seed, b.out_tokens, b.n_out, self.ws, margins=b.spec_margins,
+                              q_norm=b.q_norm)
         L.s3r_commit(self.batch, self.k, b.n_out, self.seq_lens, b.stats)
 
     def round(self, q_block, k_block, v_block, p_logits, q_logits, draft_logits_fn=None,
@@ -262,7 +268,7 @@ class MixedPhaseDriver:
             L.s3r_draft_argmax(batch, self.step, e.k, q_logits, e.vocab, b.draft_tokens, e.ws)
         else:
             L.s3r_draft_sample(batch, self.step, e.k, q_logits, e.vocab, e.seed, b.draft_tokens,
-                               e.ws, margins=b.draft_margins)
+                               e.ws, margins=b.draft_margins, q_norm=b.q_norm)
 
     def cycle(self, q_block, k_block, v_block, p_logits, q_logits):
         """The k+1 iterations of one cycle from the current phases, as callables that issue
@@ -306,7 +312,7 @@ class MixedPhaseDriver:
                         L.s3r_draft_argmax(it["d_batch"], it["step"], k, q_logits, e.vocab, b.draft_tokens, e.ws)
                     else:
                         L.s3r_draft_sample(it["d_batch"], it["step"], k, q_logits, e.vocab, e.seed,
-                                           b.draft_tokens, e.ws, margins=b.draft_margins)
+                                           b.draft_tokens, e.ws, margins=b.draft_margins, q_norm=b.q_norm)
                 rec("d1")
                 rec("v0")
                 if it["n_verify"]:
@@ -318,7 +324,7 @@ class MixedPhaseDriver:
                         L.s3r_greedy_verify(vb, k, p_logits, b.draft_tokens, e.vocab, b.out_tokens, b.n_out, e.ws)
                     else:
                         L.s3r_spec_sample(vb, k, p_logits, q_logits, b.draft_tokens, e.vocab, e.seed,
-                                          b.out_tokens, b.n_out, e.ws, margins=b.spec_margins)
+                                          b.out_tokens, b.n_out, e.ws, margins=b.spec_margins, q_norm=b.q_norm)
                     L.s3r_commit(vb, k, b.n_out, e.seq_lens, b.stats)
                     rec("c1")
                     sel = L.s3r_select_kv_pages if e.page_select else L.s3r_select_kv
@@ -349,7 +355,7 @@ class MixedPhaseDriver:
                                     b.n_out, e.ws)
             else:
                 L.s3r_spec_sample(batch, e.k, p_logits, q_logits, b.draft_tokens, e.vocab,
-                                  e.seed, b.out_tokens, b.n_out, e.ws, margins=b.spec_margins)
+                                  e.seed, b.out_tokens, b.n_out, e.ws, margins=b.spec_margins, q_norm=b.q_norm)
             L.s3r_commit(batch, e.k, b.n_out, e.seq_lens, b.stats)
             sel = L.s3r_select_kv_pages if e.page_select else L.s3r_select_kv
             sel(e.cache, batch, b.scores, b.lse, e.k, e.budget_bp, e.window, b.sel_idx,

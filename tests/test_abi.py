@@ -84,13 +84,20 @@ def test_host_validation_rejects_before_launch():
     assert L.s3r_select_kv(ctypes.byref(c), ctypes.byref(b), 0x10, 0x10, 6, 500, 6, 0x10, 100,
                            0x10, 0x100, 1 << 30, null) == 1
     # sampling: vocabulary and k
-    assert L.s3r_spec_sample(ctypes.byref(b), 9, 0x10, 0x10, 0x10, 64, 1, 0x10, 0x10, None, 0x100,
-                             1 << 30, null) == 2
-    assert L.s3r_draft_sample(ctypes.byref(b), 0x10, 6, 0x10, 0, 1, 0x10, None, 0x100, 1 << 30, null) == 2
+    assert L.s3r_spec_sample(ctypes.byref(b), 9, 0x10, 0x10, 0x10, 64, 1, 0x10, 0x10, None, None,
+                             0x100, 1 << 30, null) == 2
+    assert L.s3r_draft_sample(ctypes.byref(b), 0x10, 6, 0x10, 0, 1, 0x10, None, None, 0x100, 1 << 30,
+                              null) == 2
     # a misaligned margins output
-    assert L.s3r_spec_sample(ctypes.byref(b), 6, 0x10, 0x10, 0x10, 64, 1, 0x10, 0x10, 0x11, 0x100,
-                             1 << 30, null) == 1
-    assert L.s3r_draft_sample(ctypes.byref(b), 0x10, 6, 0x10, 64, 1, 0x10, 0x11, 0x100, 1 << 30, null) == 1
+    assert L.s3r_spec_sample(ctypes.byref(b), 6, 0x10, 0x10, 0x10, 64, 1, 0x10, 0x10, 0x11, None,
+                             0x100, 1 << 30, null) == 1
+    assert L.s3r_draft_sample(ctypes.byref(b), 0x10, 6, 0x10, 64, 1, 0x10, 0x11, None, 0x100, 1 << 30,
+                              null) == 1
+    # a misaligned normaliser array (8-byte records)
+    assert L.s3r_spec_sample(ctypes.byref(b), 6, 0x10, 0x10, 0x10, 64, 1, 0x10, 0x10, None, 0x14,
+                             0x100, 1 << 30, null) == 1
+    assert L.s3r_draft_sample(ctypes.byref(b), 0x10, 6, 0x10, 64, 1, 0x10, None, 0x14, 0x100, 1 << 30,
+                              null) == 1
     # the verify's wait bound
     assert L.s3r_set_wait_limit(-1) == 1
     assert L.s3r_set_wait_limit(0) == 0

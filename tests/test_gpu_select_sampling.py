@@ -256,3 +256,45 @@ def test_emitted_tokens_follow_target_distribution_on_gpu():
         assert lo <= alpha[j] <= hi
     # negative control: the drafts themselves do not follow the target
     assert _chi2(drafts[:, 0], P[0]) < 1e-6
+
+
+@pytest.mark.parametrize("NR,k,V", [(64, 6, 151936), (40, 3, 20000)])
+def test_draft_row_normalisers_carry_into_spec_sampling(NR, k, V):
+    """s3r_draft_sample's q_norm output holds each draft row's (max, sum of exp(x - max)), as
+    fp64 arithmetic gives them to fp32-rounding accuracy; s3r_spec_sample given them emits the
+    same tokens as when it streams the q rows itself, except where a decision lies closer to
+    its boundary than that rounding (reported by the margins)."""
+    seed = 5
+    p, qn = _sample_inputs(NR, k, V, seed)
+    pd, qd = torch.as_tensor(p).cuda(), torch.as_tensor(qn).cuda()
+    rng = np.random.default_rng(seed)
+    seq = torch.as_tensor(rng.integers(100, 30000, size=NR).astype(np.int32)).cuda()
+    batch = s3r.make_batch(seq)
+    cache = s3r.KVCacheDesc(8, 8, 128, 16, 1, 16, 16)
+    ws = s3r.new_workspace(s3r.s3r_workspace_size(cache, NR, 1, k, V, 1))
+    drafts = torch.zeros((NR, k), dtype=torch.int32, device="cuda")
+    qnorm = torch.zeros((NR, k, 2), dtype=torch.float64, device="cuda")
+    for i in range(k):
+        s3r.s3r_draft_sample(batch, torch.full((NR,), i, dtype=torch.int32, device="cuda"), k, qd,
+                             V, seed, drafts, ws, q_norm=qnorm)
+    mx, sm = s3r._lib.row_norms(qnorm)
+    ref_m = qn.max(axis=2)
+    ref_s = np.exp(qn.astype(np.float64) - ref_m[..., None]).sum(axis=2)
+    np.testing.assert_array_equal(mx, ref_m.astype(np.float32))
+    np.testing.assert_allclose(sm, ref_s, rtol=1e-5)
+    outs = []
+    for qarg in (None, qnorm):
+        out = torch.full((NR, k + 1), -1, dtype=torch.int32, device="cuda")
+        n_out = torch.zeros(NR, dtype=torch.int32, device="cuda")
+        mg = torch.full((NR, k + 1), float("inf"), dtype=torch.float32, device="cuda")
+        before = s3r.s3r_launch_count()
+        s3r.s3r_spec_sample(batch, k, pd, qd, drafts, V, seed, out, n_out, ws, margins=mg,
+                            q_norm=qarg)
+        assert s3r.s3r_launch_count() - before == 2
+        assert s3r.s3r_get_error(ws) == 0
+        outs.append((out.cpu().numpy(), n_out.cpu().numpy(), mg.cpu().numpy()))
+    (o0, n0, m0), (o1, n1, m1) = outs
+    differ = [r for r in range(NR) if n0[r] != n1[r] or not np.array_equal(o0[r, :n0[r]], o1[r, :n1[r]])]
+    for r in differ:   # only a decision within the rounding of the sums may go the other way
+        assert min(m0[r].min(), m1[r].min()) < 1e-5, r
+    assert len(differ) <= max(1, NR // 20)
