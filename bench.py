@@ -419,6 +419,8 @@ def run_ours(args, spec):
                                f"vocab {spec.vocab}",
                    "requests_per_gpu": spec.num_requests, "parallelism": f"replicas x{world}",
                    "selection": args.select,
+                   "scores": "the next selection's position scores on a second stream, beside "
+                             "speculative sampling and the commit",
                    "verification": "greedy" if args.greedy else "speculative sampling",
                    "l2": "inputs larger than L2 (KV 2.1 GB, logits 0.25 GB per round)"},
         "roofline": {"bound": "hbm", "achieved": v_gbs, "peak": peak, "unit": "GB/s",

@@ -150,6 +150,22 @@ S3R_API int s3r_select_kv(const s3r_kv_cache* cache, const s3r_batch* batch, con
                   int32_t* sel_idx, int32_t sel_stride, int32_t* sel_count, void* ws,
                   size_t ws_bytes, s3r_stream_t stream);
 
+/* The scores s3r_select_kv orders positions by, on their own: for request r (committed length
+ * L at this call) and KV head h, scores[r][h][j] = sum over the G*(k_prev+1) rows of
+ * exp(logit - lse) for every j < L, the same fp32 values s3r_select_kv computes.
+ * s3r_select_from_scores on them makes the same selection as s3r_select_kv. The two halves
+ * split where the round allows it: a selection at committed length L' (at most L + k_prev + 1,
+ * fewer than W positions more) reads only j < L' - W < L, so these scores can be computed
+ * as soon as the verify's logits and lse exist, while speculative sampling and the commit run
+ * on another stream; only the ordering waits for the new lengths.
+ *   scores  fp32 [num_requests][H_kv][score_stride], 16-byte aligned, score_stride a multiple
+ *           of 4 and >= L (a longer context sets S3R_ERR_DEVICE_BOUNDS); entries j >= L are
+ *           not written. Uses only the workspace's error word. */
+S3R_API int s3r_position_scores(const s3r_kv_cache* cache, const s3r_batch* batch,
+                        const float* score_logits, const float* lse, int32_t k_prev,
+                        float* scores, int32_t score_stride, void* ws, size_t ws_bytes,
+                        s3r_stream_t stream);
+
 /* The same selection from caller-given scores: scores fp32 [num_requests][H_kv][score_stride],
  * sigma_j = scores[r][h][j] (any finite float; order by value, ties to the lower j). */
 S3R_API int s3r_select_from_scores(const s3r_kv_cache* cache, const s3r_batch* batch,

@@ -26,6 +26,7 @@ from ._lib import (  # noqa: F401
     s3r_horizon_step,
     s3r_launch_count,
     s3r_philox,
+    s3r_position_scores,
     s3r_select_from_scores,
     s3r_select_kv_pages,
     s3r_select_pages_from_scores,

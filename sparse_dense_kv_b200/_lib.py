@@ -74,6 +74,7 @@ def _load():
         "s3r_verify_attn": (ctypes.c_int, [C, B, I32, P, P, P, P, P, P, P, SZ, P]),
         "s3r_select_kv": (ctypes.c_int, [C, B, P, P, I32, I32, I32, P, I32, P, P, SZ, P]),
         "s3r_select_from_scores": (ctypes.c_int, [C, B, P, I32, I32, I32, P, I32, P, P, SZ, P]),
+        "s3r_position_scores": (ctypes.c_int, [C, B, P, P, I32, P, I32, P, SZ, P]),
         "s3r_select_kv_pages": (ctypes.c_int, [C, B, P, P, I32, I32, I32, P, I32, P, P, SZ, P]),
         "s3r_select_pages_from_scores": (ctypes.c_int, [C, B, P, I32, I32, I32, P, I32, P, P, SZ, P]),
         "s3r_sparse_draft_attn": (ctypes.c_int, [C, B, P, P, I32, P, P, I32, P, I32, P, P, P, P, SZ, P]),
@@ -215,6 +216,15 @@ def _select_from_scores(fn, cache, batch, scores, budget_bp, window, sel_idx, se
         budget_bp, window, _ptr(sel_idx, i32, "sel_idx"), sel_idx.shape[-1],
         _ptr(sel_count, i32, "sel_count"), _ptr(ws, torch.uint8, "ws"), ws.numel(),
         _stream(stream)), fn)
+
+
+def s3r_position_scores(cache, batch, score_logits, lse, k_prev, scores, ws, stream=None):
+    """scores: fp32 [NR][H_kv][stride] receiving sigma_j for every committed j < L."""
+    f32 = torch.float32
+    _check(_lib.s3r_position_scores(
+        ctypes.byref(cache), ctypes.byref(batch), _ptr(score_logits, f32, "score_logits"),
+        _ptr(lse, f32, "lse"), k_prev, _ptr(scores, f32, "scores"), scores.shape[-1],
+        _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)), "s3r_position_scores")
 
 
 def s3r_select_kv(cache, batch, score_logits, lse, k_prev, budget_bp, window, sel_idx,

@@ -85,7 +85,8 @@ struct SelectParams {
   int sel_stride;
   int32_t* sel_count;
   int* err;
-  float* sigma_buf;        // workspace: sigma [NR][Hkv][cap] of the logits path
+  float* sigma_buf;        // sigma [NR][Hkv][sigma_stride]: the workspace's (logits path) or the caller's
+  int sigma_stride;
   int page;                // selection unit: 1 (positions) or S3R_PAGE_SIZE (pages)
 };
 
@@ -137,6 +138,7 @@ int launch_draft(const DraftParams& p, int D, int batch, int num_sms, cudaStream
 size_t draft_partial_bytes(int num_requests, int Hkv, int sel_stride, int D);
 
 int launch_select(const SelectParams& p, int batch, cudaStream_t stream, int* launches);
+int launch_sigma(const SelectParams& p, int batch, cudaStream_t stream);   // scores only
 size_t select_sigma_bytes(int num_requests, int Hkv, int cap);
 
 int launch_draft_sample(const SampleParams& p, int batch, cudaStream_t stream);

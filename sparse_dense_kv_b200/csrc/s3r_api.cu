@@ -455,6 +455,43 @@ int s3r_select_kv_pages(const s3r_kv_cache* cache, const s3r_batch* batch,
                         sel_stride, sel_count, ws, ws_bytes, stream, S3R_PAGE_SIZE);
 }
 
+int s3r_position_scores(const s3r_kv_cache* cache, const s3r_batch* batch,
+                        const float* score_logits, const float* lse, int32_t k_prev,
+                        float* scores, int32_t score_stride, void* ws, size_t ws_bytes,
+                        s3r_stream_t stream) {
+  S3R_TRY(check_cache(cache));
+  S3R_TRY(check_batch(batch, true));
+  if (k_prev < 0 || k_prev > S3R_MAX_K) return S3R_ERR_UNSUPPORTED;
+  const int G = cache->num_q_heads / cache->num_kv_heads;
+  if (G * (k_prev + 1) > S3R_MAX_ROWS) return S3R_ERR_UNSUPPORTED;
+  if (!score_logits || !lse || !scores || !aligned16(score_logits) || !aligned4(lse) ||
+      !aligned16(scores) || score_stride < 1 || (score_stride % 4))
+    return S3R_ERR_INVALID_ARG;
+  if (batch->batch > 65535) return S3R_ERR_UNSUPPORTED;   // grid.z
+  if (batch->batch == 0) return S3R_OK;
+  S3R_TRY(check_ws(ws, ws_bytes, head_bytes(batch->num_requests)));
+  const Carve w = carve(ws, batch->num_requests);
+  SelectParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.req_ids = batch->req_ids;
+  p.seq_lens = batch->seq_lens;
+  p.Hq = cache->num_q_heads;
+  p.Hkv = cache->num_kv_heads;
+  p.G = G;
+  p.cap = batch->max_pages_per_req * S3R_PAGE_SIZE;
+  p.logits = score_logits;
+  p.lse = lse;
+  p.T = k_prev + 1;
+  p.R = G * (k_prev + 1);
+  p.window = 0;   // every committed position
+  p.sigma_buf = scores;
+  p.sigma_stride = score_stride;
+  p.err = w.err;
+  const int st = launch_sigma(p, batch->batch, (cudaStream_t)stream);
+  if (st == S3R_OK) g_launches.fetch_add(1, std::memory_order_relaxed);
+  return st;
+}
+
 int s3r_select_from_scores(const s3r_kv_cache* cache, const s3r_batch* batch,
                            const float* scores, int32_t score_stride, int32_t budget_bp,
                            int32_t window, int32_t* sel_idx, int32_t sel_stride,

@@ -313,7 +313,11 @@ __global__ void __launch_bounds__(kSigmaThreads) sigma_kernel(const SelectParams
   const int kvh = blockIdx.y, bl = blockIdx.z;
   const int r = p.req_ids ? p.req_ids[bl] : bl;
   const int L = p.seq_lens[r];
-  if (L < 0 || L > p.cap) return;   // reported by the select kernel
+  if (L < 0 || L > p.cap || L > p.sigma_stride) {
+    // reported by the select kernel on its path; here for the scores-only call
+    if (p.window == 0 && blockIdx.x == 0 && kvh == 0 && threadIdx.x == 0) set_error(p.err, S3R_ERR_DEVICE_BOUNDS);
+    return;
+  }
   const int N = L - min(p.window, L);
   const int j0 = blockIdx.x * kSigmaPos;
   if (j0 >= N) return;
@@ -341,13 +345,19 @@ __global__ void __launch_bounds__(kSigmaThreads) sigma_kernel(const SelectParams
       acc3 += ex2(fmaf(x[u].w, kLog2e, -l2));
     }
   }
-  float* out = p.sigma_buf + ((size_t)r * p.Hkv + kvh) * p.cap + j4;
+  float* out = p.sigma_buf + ((size_t)r * p.Hkv + kvh) * p.sigma_stride + j4;
   if (j4 + 4 <= N) {
     *reinterpret_cast<float4*>(out) = make_float4(acc0, acc1, acc2, acc3);
   } else {
     const float sg[4] = {acc0, acc1, acc2, acc3};
     for (int q = 0; q < N - j4; ++q) out[q] = sg[q];
   }
+}
+
+int launch_sigma(const SelectParams& p, int batch, cudaStream_t stream) {
+  dim3 g((p.cap + kSigmaPos - 1) / kSigmaPos, p.Hkv, batch);
+  launch_pdl(sigma_kernel, g, kSigmaThreads, 0, stream, p);
+  return cuda_status(cudaGetLastError(), "sigma_kernel");
 }
 
 size_t select_sigma_bytes(int num_requests, int Hkv, int cap) {
@@ -358,8 +368,9 @@ int launch_select(const SelectParams& p, int batch, cudaStream_t stream, int* la
   *launches = 0;
   SelectParams q = p;
   if (p.logits) {
+    q.sigma_stride = p.cap;
     dim3 g((p.cap + kSigmaPos - 1) / kSigmaPos, p.Hkv, batch);
-    launch_pdl(sigma_kernel, g, kSigmaThreads, 0, stream, p);
+    launch_pdl(sigma_kernel, g, kSigmaThreads, 0, stream, q);
     if (cuda_status(cudaGetLastError(), "sigma_kernel") != S3R_OK) return S3R_ERR_CUDA;
     ++*launches;
     q.logits = nullptr;

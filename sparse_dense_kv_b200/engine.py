@@ -73,7 +73,8 @@ class S3REngine:
     """S3R rounds for a batch of requests over one paged KV cache on one GPU."""
 
     def __init__(self, k_pool, v_pool, page_table, seq_lens, num_q_heads, *, k, budget_bp,
-                 window, vocab, seed, sel_stride=None, greedy=False, page_select=False, k_max=None):
+                 window, vocab, seed, sel_stride=None, greedy=False, page_select=False, k_max=None,
+                 overlap_scores=True):
         k_max = k if k_max is None else k_max
         if not (1 <= k <= k_max <= L.MAX_K):
             raise ValueError("need 1 <= k <= k_max <= 8")
@@ -97,6 +98,17 @@ class S3REngine:
                                       self.sel_stride)
         self.ws = L.new_workspace(nbytes, k_pool.device)
         self.batch = L.make_batch(seq_lens, page_table)
+        # The next selection's position scores (s3r_position_scores) are computed on a second
+        # stream while speculative sampling and the commit run on this one; they read the
+        # lengths from a snapshot taken before the fork, so the commit never races them.
+        self.overlap_scores = overlap_scores
+        self._scores_ready = False
+        if overlap_scores:
+            self.pos_scores = torch.empty((self.num_requests, self.cache.num_kv_heads, self.cap),
+                                          dtype=torch.float32, device=k_pool.device)
+            self._len_snap = torch.empty_like(seq_lens)
+            self._snap_batch = L.make_batch(self._len_snap, page_table)
+            self._score_stream = torch.cuda.Stream(k_pool.device)
         self.k_prev = None
         self._verify_launches = 2
 
@@ -110,7 +122,7 @@ class S3REngine:
 
     @property
     def launches_per_round(self) -> int:
-        # select (sigma + select), k x (draft, sample), verify (attention launches + the chunk
+        # select (scores + select), k x (draft, sample), verify (attention launches + the chunk
         # merge, as counted at the last verify), spec (2 / 1 greedy), commit
         return 2 + 2 * self.k + self._verify_launches + (1 if self.greedy else 2) + 1
 
@@ -127,6 +139,11 @@ class S3REngine:
 
     def select(self):
         b = self.buf
+        if self._scores_ready:   # the scores computed beside the last round's sampling
+            fn = L.s3r_select_pages_from_scores if self.page_select else L.s3r_select_from_scores
+            fn(self.cache, self.batch, self.pos_scores, self.budget_bp, self.window, b.sel_idx,
+               b.sel_count, self.ws)
+            return
         lse = b.prefill_lse if self.k_prev == 0 else b.lse
         fn = L.s3r_select_kv_pages if self.page_select else L.s3r_select_kv
         fn(self.cache, self.batch, b.scores, lse, self.k_prev, self.budget_bp, self.window,
@@ -160,9 +177,25 @@ class S3REngine:
                           b.lse, b.scores, self.ws)
         self._verify_launches = L.s3r_launch_count() - before
         self.k_prev = self.k
+        self._scores_ready = False
+
+    def fork_scores(self, batch, snap_batch, k):
+        """The position scores of the verify just run, for the batch's requests, on the second
+        stream (lengths from a snapshot of seq_lens); join_scores() rejoins it."""
+        main = torch.cuda.current_stream()
+        self._len_snap.copy_(self.seq_lens, non_blocking=True)
+        self._score_stream.wait_stream(main)
+        with torch.cuda.stream(self._score_stream):
+            L.s3r_position_scores(self.cache, snap_batch, self.buf.scores, self.buf.lse, k,
+                                  self.pos_scores, self.ws)
+
+    def join_scores(self):
+        torch.cuda.current_stream().wait_stream(self._score_stream)
 
     def sample_and_commit(self, p_logits, q_logits):
         b = self.buf
+        if self.overlap_scores:
+            self.fork_scores(self.batch, self._snap_batch, self.k)
         if self.greedy:
             L.s3r_greedy_verify(self.batch, self.k, p_logits, b.draft_tokens, self.vocab,
                                 b.out_tokens, b.n_out, self.ws)
@@ -171,6 +204,9 @@ class S3REngine:
                               self.seed, b.out_tokens, b.n_out, self.ws, margins=b.spec_margins,
                               q_norm=b.q_norm)
         L.s3r_commit(self.batch, self.k, b.n_out, self.seq_lens, b.stats)
+        if self.overlap_scores:
+            self.join_scores()
+            self._scores_ready = True
 
     def round(self, q_block, k_block, v_block, p_logits, q_logits, draft_logits_fn=None,
               target_logits_fn=None):
@@ -234,9 +270,25 @@ class MixedPhaseDriver:
         self.step = torch.zeros((engine.num_requests,), dtype=torch.int32, device=dev)
         self._dev = dev
 
-    def _batch(self, ids):
+    def _batch(self, ids, snap=False):
         t = torch.as_tensor(ids, dtype=torch.int32, device=self._dev)
-        return L.make_batch(self.e.seq_lens, self.e.page_table, req_ids=t)
+        lens = self.e._len_snap if snap else self.e.seq_lens
+        return L.make_batch(lens, self.e.page_table, req_ids=t)
+
+    def _reselect(self, vb, v_snap, k, commit):
+        """Verify done for the batch vb: position scores (beside the sampling and commit when
+        the engine overlaps them), `commit()`, then the new sparse sets."""
+        e, b = self.e, self.e.buf
+        if e.overlap_scores:
+            e.fork_scores(vb, v_snap, k)
+        commit()
+        if e.overlap_scores:
+            e.join_scores()
+            sel = L.s3r_select_pages_from_scores if e.page_select else L.s3r_select_from_scores
+            sel(e.cache, vb, e.pos_scores, e.budget_bp, e.window, b.sel_idx, b.sel_count, e.ws)
+        else:
+            sel = L.s3r_select_kv_pages if e.page_select else L.s3r_select_kv
+            sel(e.cache, vb, b.scores, b.lse, k, e.budget_bp, e.window, b.sel_idx, b.sel_count, e.ws)
 
     def start(self, q_block, k_block, v_block, q_logits):
         """After prefill: every request selects its first sparse set from the prefill scores,
@@ -296,7 +348,8 @@ class MixedPhaseDriver:
                       steps=st, step=st_d, qc=q_block[ar, rows].contiguous(),
                       kc=k_block[ar, rows].contiguous(), vc=v_block[ar, rows].contiguous(),
                       d_batch=self._batch(d_ids) if d_ids.size else None,
-                      v_batch=self._batch(v_ids) if v_ids.size else None)
+                      v_batch=self._batch(v_ids) if v_ids.size else None,
+                      v_snap=self._batch(v_ids, snap=True) if v_ids.size and e.overlap_scores else None)
             its.append(it)
 
         def make(it):
@@ -320,15 +373,18 @@ class MixedPhaseDriver:
                     L.s3r_verify_attn(e.cache, vb, k, q_block, k_block, v_block, b.verify_out, b.lse,
                                       b.scores, e.ws)
                     rec("v1")
-                    if e.greedy:
-                        L.s3r_greedy_verify(vb, k, p_logits, b.draft_tokens, e.vocab, b.out_tokens, b.n_out, e.ws)
-                    else:
-                        L.s3r_spec_sample(vb, k, p_logits, q_logits, b.draft_tokens, e.vocab, e.seed,
-                                          b.out_tokens, b.n_out, e.ws, margins=b.spec_margins, q_norm=b.q_norm)
-                    L.s3r_commit(vb, k, b.n_out, e.seq_lens, b.stats)
-                    rec("c1")
-                    sel = L.s3r_select_kv_pages if e.page_select else L.s3r_select_kv
-                    sel(e.cache, vb, b.scores, b.lse, k, e.budget_bp, e.window, b.sel_idx, b.sel_count, e.ws)
+
+                    def commit():
+                        if e.greedy:
+                            L.s3r_greedy_verify(vb, k, p_logits, b.draft_tokens, e.vocab, b.out_tokens,
+                                                b.n_out, e.ws)
+                        else:
+                            L.s3r_spec_sample(vb, k, p_logits, q_logits, b.draft_tokens, e.vocab, e.seed,
+                                              b.out_tokens, b.n_out, e.ws, margins=b.spec_margins,
+                                              q_norm=b.q_norm)
+                        L.s3r_commit(vb, k, b.n_out, e.seq_lens, b.stats)
+                        rec("c1")
+                    self._reselect(vb, it["v_snap"], k, commit)
                 else:
                     rec("v1")
                     rec("c1")
@@ -350,16 +406,18 @@ class MixedPhaseDriver:
             batch = self._batch(v_ids)
             L.s3r_verify_attn(e.cache, batch, e.k, q_block, k_block, v_block, b.verify_out, b.lse,
                               b.scores, e.ws)
-            if e.greedy:
-                L.s3r_greedy_verify(batch, e.k, p_logits, b.draft_tokens, e.vocab, b.out_tokens,
-                                    b.n_out, e.ws)
-            else:
-                L.s3r_spec_sample(batch, e.k, p_logits, q_logits, b.draft_tokens, e.vocab,
-                                  e.seed, b.out_tokens, b.n_out, e.ws, margins=b.spec_margins, q_norm=b.q_norm)
-            L.s3r_commit(batch, e.k, b.n_out, e.seq_lens, b.stats)
-            sel = L.s3r_select_kv_pages if e.page_select else L.s3r_select_kv
-            sel(e.cache, batch, b.scores, b.lse, e.k, e.budget_bp, e.window, b.sel_idx,
-                b.sel_count, e.ws)
+
+            def commit():
+                if e.greedy:
+                    L.s3r_greedy_verify(batch, e.k, p_logits, b.draft_tokens, e.vocab, b.out_tokens,
+                                        b.n_out, e.ws)
+                else:
+                    L.s3r_spec_sample(batch, e.k, p_logits, q_logits, b.draft_tokens, e.vocab,
+                                      e.seed, b.out_tokens, b.n_out, e.ws, margins=b.spec_margins,
+                                      q_norm=b.q_norm)
+                L.s3r_commit(batch, e.k, b.n_out, e.seq_lens, b.stats)
+            self._reselect(batch, self._batch(v_ids, snap=True) if e.overlap_scores else None, e.k,
+                           commit)
         self.phases = (self.phases + 1) % (e.k + 1)
         return v_ids
 

@@ -98,6 +98,13 @@ def test_host_validation_rejects_before_launch():
                              0x100, 1 << 30, null) == 1
     assert L.s3r_draft_sample(ctypes.byref(b), 0x10, 6, 0x10, 64, 1, 0x10, None, 0x14, 0x100, 1 << 30,
                               null) == 1
+    # position scores: misaligned output, a stride that is not a multiple of 4, k_prev
+    assert L.s3r_position_scores(ctypes.byref(c), ctypes.byref(b), 0x10, 0x10, 6, 0x18, 1024,
+                                 0x100, 1 << 20, null) == 1
+    assert L.s3r_position_scores(ctypes.byref(c), ctypes.byref(b), 0x10, 0x10, 6, 0x10, 1022,
+                                 0x100, 1 << 20, null) == 1
+    assert L.s3r_position_scores(ctypes.byref(c), ctypes.byref(b), 0x10, 0x10, 9, 0x10, 1024,
+                                 0x100, 1 << 20, null) == 2
     # the verify's wait bound
     assert L.s3r_set_wait_limit(-1) == 1
     assert L.s3r_set_wait_limit(0) == 0

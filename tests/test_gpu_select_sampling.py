@@ -105,6 +105,57 @@ def test_select_from_verify_scores_matches_oracle():
     print(f"select boundary cases: {boundary}")
 
 
+@pytest.mark.parametrize("page", [False, True])
+def test_position_scores_before_the_commit_give_the_same_selection(page):
+    """s3r_position_scores run on the verify's logits before the commit (the lengths then are
+    the verify's L), then s3r_select_from_scores after it: the same sets, bit for bit, as
+    s3r_select_kv after the commit; the scores match the oracle's sigma at every committed
+    position."""
+    k, bp, W = 6, 500, 64
+    spec = spec_for(32, 8, 128, [3000, 5000, 1500, 700], k=k, seed=19, heavy=32)
+    case = Case(spec, extra_tokens=k + 1 + 16)
+    NR, Hq, Hkv, d = 4, 32, 8, 128
+    q = synth.randn_bf16((NR, k + 1, Hq, d), 4, "cuda")
+    kn = synth.randn_bf16((NR, k + 1, Hkv, d), 5, "cuda")
+    vn = synth.randn_bf16((NR, k + 1, Hkv, d), 6, "cuda")
+    cache = s3r.make_cache(case.k_pool, case.v_pool, Hq)
+    batch = s3r.make_batch(case.seq_lens, case.page_table)
+    cap = case.cache.capacity
+    out = torch.empty_like(q)
+    lse = torch.empty((NR, k + 1, Hq), dtype=torch.float32, device="cuda")
+    sc = torch.empty((NR, Hkv, 4 * (k + 1), cap), device="cuda")
+    stride = 512
+    ws = s3r.new_workspace(s3r.s3r_workspace_size(cache, NR, case.cache.max_pages, k, 64, stride))
+    s3r.s3r_verify_attn(cache, batch, k, q, kn, vn, out, lse, sc, ws)
+    lens0 = case.seq_lens.clone()
+    pos = torch.full((NR, Hkv, cap), float("nan"), device="cuda")
+    before = s3r.s3r_launch_count()
+    s3r.s3r_position_scores(cache, batch, sc, lse, k, pos, ws)
+    assert s3r.s3r_launch_count() - before == 1
+    n_out = torch.tensor([1, 7, 3, 5], dtype=torch.int32, device="cuda")
+    s3r.s3r_commit(batch, k, n_out, case.seq_lens)
+    sel_a = torch.zeros((NR, Hkv, stride), dtype=torch.int32, device="cuda")
+    cnt_a = torch.zeros((NR, Hkv), dtype=torch.int32, device="cuda")
+    sel_b, cnt_b = torch.zeros_like(sel_a), torch.zeros_like(cnt_a)
+    fn_kv = s3r.s3r_select_kv_pages if page else s3r.s3r_select_kv
+    fn_sc = s3r.s3r_select_pages_from_scores if page else s3r.s3r_select_from_scores
+    fn_kv(cache, batch, sc, lse, k, bp, W, sel_a, cnt_a, ws)
+    fn_sc(cache, batch, pos, bp, W, sel_b, cnt_b, ws)
+    assert s3r.s3r_get_error(ws) == 0
+    assert torch.equal(cnt_a, cnt_b)
+    for r in range(NR):
+        for h in range(Hkv):
+            n = int(cnt_a[r, h])
+            assert torch.equal(sel_a[r, h, :n], sel_b[r, h, :n]), (r, h)
+    kp, vp = case.host_pools()
+    pos_h = pos.cpu().numpy()
+    for r, L in enumerate(lens0.cpu().tolist()):
+        K, V = case.dense(r, L + k + 1, (kp, vp))
+        _, _, sigma, _ = O.verify_attention(f64(q[r]), K, V, int(L))
+        np.testing.assert_allclose(pos_h[r, :, :L], sigma[:, :L], rtol=1e-4, atol=1e-7)
+        assert np.isnan(pos_h[r, :, L:]).all()          # nothing written past L
+
+
 def _sample_inputs(NR, k, V, seed, same_rows=False):
     rng = np.random.default_rng(seed)
     if same_rows:
