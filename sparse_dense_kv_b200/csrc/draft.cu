@@ -5,9 +5,12 @@
 // request r (token at position L+i) writes that token's K/V into its page and lets the G
 // query rows of each KV head attend A_i = S ∪ {L, .., L+i}, S the selected positions.
 //
-// Layout of the work: grid (chunk of A_i, kv_head, request), 128 threads. The CTA first
-// resolves the element offsets of its <= kDraftChunk (512) positions (index -> page ->
-// slot), then gathers 256-byte K and V rows with 16-byte cp.async (16 lanes per row,
+// Layout of the work: grid (kv_head, request, chunk of A_i), 128 threads: the block
+// scheduler starts every pair's first chunk before any second chunk, so the CTAs that spill
+// past the resident ones are mostly the short last chunks of the largest pairs. Chunks are
+// kDraftChunk (512) positions long, except that the last one also takes a remainder of up to
+// kDraftFold positions instead of leaving it to a CTA of its own. The CTA first resolves the
+// element offsets of its positions (index -> page -> slot), then gathers 256-byte K and V rows with 16-byte cp.async (16 lanes per row,
 // coalesced) into a 2-stage pipeline laid out like the TMA tiles of the verify (128-byte
 // swizzle), so the same tensor-core step (one n-tile of 8 rows per warp) serves both.
 // Chunks merge through the workspace in the last CTA of the (request, head).
@@ -17,11 +20,19 @@
 namespace s3r {
 
 constexpr int kDraftStages = 2;
+constexpr int kDraftFold = 128;
+constexpr int kDraftSpan = kDraftChunk + kDraftFold;   // longest chunk
+
+// Chunks of a set of A positions: ceil(A / kDraftChunk), less one when the last would hold
+// at most kDraftFold positions (that remainder goes to the chunk before it).
+__device__ __forceinline__ int draft_nchunks(int A) {
+  return max(1, (A + kDraftChunk - 1 - kDraftFold) / kDraftChunk);
+}
 
 template <int D>
 __global__ void __launch_bounds__(128) draft_kernel(const DraftParams p) {
   pdl_wait();
-  static_assert(kDraftChunk % 128 == 0, "128 threads resolve the chunk's rows");
+  static_assert(kDraftChunk % 128 == 0 && kDraftSpan % 128 == 0, "128 threads resolve the chunk's rows");
   constexpr int NTW = 1, RW = 8, STAGE = 2 * kTile * D * 2, CPR = D / 8;
   extern __shared__ uint8_t smem_dyn[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) &
@@ -31,7 +42,7 @@ __global__ void __launch_bounds__(128) draft_kernel(const DraftParams p) {
   int* s_flag = &s_flag_mem;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int bl = blockIdx.z, kvh = blockIdx.y, c = blockIdx.x;
+  const int kvh = blockIdx.x, bl = blockIdx.y, c = blockIdx.z;
   const int r = p.req_ids ? p.req_ids[bl] : bl;
   if (r < 0 || r >= p.num_requests) {
     if (c == 0 && kvh == 0 && tid == 0) set_error(p.err, S3R_ERR_DEVICE_BOUNDS);
@@ -46,10 +57,10 @@ __global__ void __launch_bounds__(128) draft_kernel(const DraftParams p) {
     return;
   }
   const int A = n + i + 1;
+  const int nch = draft_nchunks(A);
+  if (c >= nch) return;
   const int start = c * kDraftChunk;
-  if (start >= A) return;
-  const int end = min(start + kDraftChunk, A);
-  const int nch = (A + kDraftChunk - 1) / kDraftChunk;
+  const int end = c == nch - 1 ? A : start + kDraftChunk;
   const int* ptab = p.page_table + (size_t)r * p.max_pages;
   const int* sel = p.sel_idx + ((size_t)r * Hkv + kvh) * p.sel_stride;
   const int64_t npages = p.num_pages;
@@ -79,7 +90,7 @@ __global__ void __launch_bounds__(128) draft_kernel(const DraftParams p) {
 
   // Element offsets of the chunk's rows: >= 0 pool offset, -1 zeros, -2 this step's token.
   // All selected indices are loaded at once, then all page ids: two dependent round trips.
-  constexpr int kPer = kDraftChunk / 128;
+  constexpr int kPer = kDraftSpan / 128;
   int pos[kPer];
 #pragma unroll
   for (int u = 0; u < kPer; ++u) {
@@ -185,11 +196,11 @@ __global__ void __launch_bounds__(128) draft_kernel(const DraftParams p) {
 
 template <int D>
 static int launch_draft_d(const DraftParams& p, int batch, cudaStream_t stream) {
-  const size_t smem = 1024 + kDraftStages * 2 * kTile * D * 2 + kDraftChunk * 8 + 64;
+  const size_t smem = 1024 + kDraftStages * 2 * kTile * D * 2 + kDraftSpan * 8 + 64;
   static std::atomic<uint64_t> attr_done{0};
   if (cuda_status(ensure_smem_attr(draft_kernel<D>, (int)smem, attr_done), "cudaFuncSetAttribute") != S3R_OK)
     return S3R_ERR_CUDA;
-  dim3 grid(p.nchunk_max, p.Hkv, batch);
+  dim3 grid(p.Hkv, batch, p.nchunk_max);
   launch_pdl(draft_kernel<D>, grid, 128, smem, stream, p);
   return cuda_status(cudaGetLastError(), __func__);
 }
