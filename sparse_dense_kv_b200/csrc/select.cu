@@ -14,10 +14,11 @@
 //
 // One CTA of 1024 threads per (KV head, request). Scores sigma_j = sum over the G*(k+1)
 // verify rows of exp(logit - lse) are computed once into shared memory as order-preserving
-// uint32 keys; MSB-first histogram passes of up to 11 bits over the bits in which the keys
-// differ (shared atomics, one block scan over the bins per pass) find the exact key of the
-// M-th largest score and how many ties at that key to keep; a final pass compacts the chosen
-// indices in increasing order, each warp over its own contiguous run of positions.
+// uint32 keys; MSB-first histogram passes over digits of 11, 11 and 10 bits (shared atomics,
+// one block scan over the bins per pass; the first pass is counted while the keys are
+// loaded) find the M-th largest score's digits and how many ties to keep, stopping early
+// once the bin that holds it is taken whole; a final pass compacts the chosen indices in
+// increasing order, each warp over its own contiguous run of positions.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -66,11 +67,11 @@ __global__ void __launch_bounds__(kSelectThreads, 2) select_kernel(const SelectP
   pdl_wait();
   extern __shared__ uint32_t keys[];
   __shared__ uint32_t hist[kSelectBins];
-  __shared__ int wsum[32], wa[32], wb[32];
+  __shared__ int wsum[32];
   __shared__ uint32_t s_prefix;
-  __shared__ int s_remaining;
+  __shared__ int s_remaining, s_whole;
 
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x;
   const int kvh = blockIdx.x, bl = blockIdx.y;
   const int r = p.req_ids ? p.req_ids[bl] : bl;
   const int L = p.seq_lens[r];
@@ -107,8 +108,12 @@ __global__ void __launch_bounds__(kSelectThreads, 2) select_kernel(const SelectP
   for (int j = tid; j < L - wstart; j += blockDim.x) out[M * P + j] = wstart + j;
   if (tid == 0) p.sel_count[(size_t)r * p.Hkv + kvh] = cnt;
   if (M == 0) return;
+  for (int b = tid; b < kSelectBins; b += blockDim.x) hist[b] = 0;
+  __syncthreads();
 
-  // ---- scores -> order-preserving keys in shared memory
+  // ---- scores -> order-preserving keys in shared memory, with the histogram of their top
+  // 11 bits (the first digit)
+  constexpr int kShift0 = 32 - 11;
   bool bad = false;
   const float* srow = p.scores + ((size_t)r * p.Hkv + kvh) * p.score_stride;
   int jv = 0;   // positions below jv were loaded as 16-byte vectors
@@ -138,6 +143,7 @@ __global__ void __launch_bounds__(kSelectThreads, 2) select_kernel(const SelectP
                 x[e] = -INFINITY;
               }
               kk[e] = order_key(x[e]);
+              atomicAdd(&hist[kk[e] >> kShift0], 1u);
             }
             *reinterpret_cast<uint4*>(keys + 4 * i4) = make_uint4(kk[0], kk[1], kk[2], kk[3]);
           }
@@ -168,49 +174,24 @@ __global__ void __launch_bounds__(kSelectThreads, 2) select_kernel(const SelectP
         sigma = -INFINITY;
       }
     }
-    keys[j] = order_key(sigma);
+    const uint32_t key = order_key(sigma);
+    keys[j] = key;
+    atomicAdd(&hist[key >> kShift0], 1u);
   }
   if (bad) set_error(p.err, S3R_ERR_NONFINITE);
   __syncthreads();
 
-  // ---- radix select of the M-th largest key over the bits in which the keys differ: the
-  // block's smallest and largest key fix the common high bits, the rest is taken MSB-first
-  // in digits of up to 11 bits. Each pass histograms the digit of the keys that still
-  // match the prefix (shared atomics; the keys are spread over the bins, so contention
-  // stays low), then one block scan over the bins from the top finds the bin holding the
-  // remaining-th largest.
-  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
-  for (int j = tid; j < N; j += blockDim.x) {
-    const uint32_t key = keys[j];
-    kmin = min(kmin, key);
-    kmax = max(kmax, key);
-  }
-  kmin = __reduce_min_sync(kFull, kmin);
-  kmax = __reduce_max_sync(kFull, kmax);
-  if (lane == 0) {
-    wa[warp] = (int)kmin;
-    wb[warp] = (int)kmax;
-  }
-  __syncthreads();
-  kmin = __reduce_min_sync(kFull, (uint32_t)wa[lane]);
-  kmax = __reduce_max_sync(kFull, (uint32_t)wb[lane]);
-  __syncthreads();
-  int nbits = 32 - __clz((int)(kmin ^ kmax));    // low bits in which keys differ (0: all equal)
-  uint32_t mask = nbits >= 32 ? 0u : ~((1u << nbits) - 1u);
-  uint32_t prefix = kmin & mask;
+  // ---- radix select of the M-th largest key, MSB-first in digits of 11, 11 and 10 bits.
+  // A pass histograms the digit of the keys that match the prefix chosen so far (the first
+  // pass was counted above); one block scan over the bins from the top finds the bin holding
+  // the remaining-th largest. When that bin holds exactly the keys still wanted, all of it is
+  // taken and the lower digits need no pass.
+  uint32_t prefix = 0u, mask = 0u;
   int remaining = M;
+  int shift = kShift0, width = 32 - kShift0;
 #pragma unroll 1
-  while (nbits > 0) {
-    const int width = nbits < 11 ? nbits : 11;
-    const int shift = nbits - width;
+  while (true) {
     const int nb = 1 << width;
-    for (int b = tid; b < kSelectBins; b += blockDim.x) hist[b] = 0;
-    __syncthreads();
-    for (int j = tid; j < N; j += blockDim.x) {
-      const uint32_t key = keys[j];
-      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & (uint32_t)(nb - 1)], 1u);
-    }
-    __syncthreads();
     // thread t owns bins 2047-2t and 2046-2t of the 2048-bin view (descending); bins at or
     // above nb are empty
     int h[2], local = 0;
@@ -228,6 +209,7 @@ __global__ void __launch_bounds__(kSelectThreads, 2) select_kernel(const SelectP
         if (cum + h[q] >= remaining) {
           s_prefix = prefix | ((uint32_t)(kSelectBins - 1 - 2 * tid - q) << shift);
           s_remaining = remaining - cum;
+          s_whole = (remaining - cum == h[q]);
           break;
         }
         cum += h[q];
@@ -237,65 +219,68 @@ __global__ void __launch_bounds__(kSelectThreads, 2) select_kernel(const SelectP
     prefix = s_prefix;
     remaining = s_remaining;
     mask |= (uint32_t)(nb - 1) << shift;
-    nbits = shift;
+    if (shift == 0 || s_whole) break;
+    width = shift < 11 ? shift : 11;
+    shift -= width;
+    for (int b = tid; b < kSelectBins; b += blockDim.x) hist[b] = 0;
+    __syncthreads();
+    const uint32_t dmask = (uint32_t)((1 << width) - 1);
+    const int n4 = N >> 2;
+    const uint4* k4 = reinterpret_cast<const uint4*>(keys);
+    for (int i4 = tid; i4 < n4; i4 += blockDim.x) {
+      const uint4 kv = k4[i4];
+      if ((kv.x & mask) == prefix) atomicAdd(&hist[(kv.x >> shift) & dmask], 1u);
+      if ((kv.y & mask) == prefix) atomicAdd(&hist[(kv.y >> shift) & dmask], 1u);
+      if ((kv.z & mask) == prefix) atomicAdd(&hist[(kv.z >> shift) & dmask], 1u);
+      if ((kv.w & mask) == prefix) atomicAdd(&hist[(kv.w >> shift) & dmask], 1u);
+    }
+    for (int j = 4 * n4 + tid; j < N; j += blockDim.x) {
+      const uint32_t key = keys[j];
+      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & dmask], 1u);
+    }
+    __syncthreads();
   }
-  // prefix is the key of the M-th largest score; the first `remaining` keys equal to it (in
-  // position order) are kept.
+  // Keys whose resolved digits exceed the prefix are taken, and the first `remaining` keys
+  // (in position order) whose resolved digits equal it; unresolved low digits (a bin taken
+  // whole) do not matter.
   const uint32_t thr = prefix;
   const int need_eq = remaining;
 
-  // ---- ordered compaction: warp w owns a contiguous run of positions; counts per warp, one
-  // scan over the 32 warps, then every warp writes its picks in order
-  const int seg = ((N + 31) / 32 + 31) / 32 * 32;
-  const int j0 = warp * seg, j1 = min(N, j0 + seg);
-  const unsigned lt = (1u << lane) - 1u;
-  int gt_w = 0, eq_w = 0;
-  for (int jb = j0; jb < j1; jb += 32) {
-    const int j = jb + lane;
-    const uint32_t key = j < j1 ? keys[j] : 0u;
-    gt_w += __popc(__ballot_sync(kFull, j < j1 && key > thr));
-    eq_w += __popc(__ballot_sync(kFull, j < j1 && key == thr));
-  }
-  if (lane == 0) {
-    wa[warp] = gt_w;
-    wb[warp] = eq_w;
-  }
-  __syncthreads();
-  if (warp == 0) {
-    const int e = wb[lane];
-    int ei = e;
+  // ---- ordered compaction: thread t owns the run of positions [t per, t per + per), read
+  // as 16-byte vectors (per / 4 odd, so the eight threads of a quarter-warp hit distinct
+  // banks); two block scans give each thread the equal keys before its run and its first
+  // output slot, then every thread writes its picks in position order
+  int per = ((N + kSelectThreads - 1) / kSelectThreads + 3) & ~3;
+  if ((per & 7) == 0) per += 4;
+  const int j0 = min(tid * per, N), j1 = min(N, j0 + per);
+  int gt_t = 0, eq_t = 0;
+  for (int jb = j0; jb < j1; jb += 4) {
+    const uint4 kv = *reinterpret_cast<const uint4*>(keys + jb);
+    const uint32_t kk[4] = {kv.x, kv.y, kv.z, kv.w};
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int v = __shfl_up_sync(kFull, ei, o);
-      if (lane >= o) ei += v;
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t key = kk[e] & mask;
+      const bool in = jb + e < j1;
+      gt_t += in && key > thr;
+      eq_t += in && key == thr;
     }
-    const int eq_before = ei - e;
-    const int take = wa[lane] + min(max(need_eq - eq_before, 0), e);
-    int ti = take;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int v = __shfl_up_sync(kFull, ti, o);
-      if (lane >= o) ti += v;
-    }
-    wa[lane] = ti - take;   // picks before this warp's run
-    wb[lane] = eq_before;   // equal keys before this warp's run
   }
-  __syncthreads();
-  int base = wa[warp], eqb = wb[warp];
-  for (int jb = j0; jb < j1; jb += 32) {
-    const int j = jb + lane;
-    const uint32_t key = j < j1 ? keys[j] : 0u;
-    const bool gt = j < j1 && key > thr;
-    const bool eq = j < j1 && key == thr;
-    const unsigned em = __ballot_sync(kFull, eq);
-    const bool take = gt || (eq && eqb + __popc(em & lt) < need_eq);
-    const unsigned tm = __ballot_sync(kFull, take);
-    if (take) {
-      int32_t* o = out + (size_t)(base + __popc(tm & lt)) * P;
-      for (int t = 0; t < P; ++t) o[t] = j * P + t;
+  const int eq_before = block_excl_scan(eq_t, wsum);
+  int base = block_excl_scan(gt_t + min(max(need_eq - eq_before, 0), eq_t), wsum);
+  int eqb = eq_before;
+  for (int jb = j0; jb < j1; jb += 4) {
+    const uint4 kv = *reinterpret_cast<const uint4*>(keys + jb);
+    const uint32_t kk[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t key = kk[e] & mask;
+      if (jb + e < j1 && (key > thr || (key == thr && eqb < need_eq))) {
+        int32_t* o = out + (size_t)base * P;
+        for (int t = 0; t < P; ++t) o[t] = (jb + e) * P + t;
+        ++base;
+      }
+      eqb += (jb + e < j1 && key == thr);
     }
-    base += __popc(tm);
-    eqb += __popc(em);
   }
 }
 
@@ -379,7 +364,8 @@ int launch_select(const SelectParams& p, int batch, cudaStream_t stream, int* la
   }
   const int lim = q.score_stride;
   const int nmax = lim < kSelectMaxN ? lim : kSelectMaxN;
-  const size_t smem = (size_t)(nmax > 0 ? nmax : 1) * 4;
+  // whole 16-byte vectors: the last one may reach 3 keys past the set
+  const size_t smem = align_up((size_t)(nmax > 0 ? nmax : 1), 4) * 4;
   static std::atomic<uint64_t> attr_tok{0}, attr_page{0};
   if (cuda_status(ensure_smem_attr(select_kernel<1>, kSelectMaxN * 4, attr_tok), "cudaFuncSetAttribute") != S3R_OK ||
       cuda_status(ensure_smem_attr(select_kernel<S3R_PAGE_SIZE>, kSelectMaxN * 4, attr_page),

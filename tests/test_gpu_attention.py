@@ -141,6 +141,9 @@ def draft_case(Hq, Hkv, d, lens, steps, budget_bp, window, seed, shuffle=False, 
     (32, 8, 128, [1500, 600], [2, 4], 10000, 64),       # s = 1: every committed position
     (8, 2, 128, [30000], [2], 1000, 64),                # one long pair: six chunks
     (16, 8, 128, [5, 17, 1, 40], [1, 0, 5, 3], 10000, 4),   # very short pairs, many per CTA
+    # s = 1, sets of 512, 513, 640, 641, 1152, 1153 and 640 positions: the edges of the chunk
+    # count where a last remainder of up to 128 positions joins the chunk before it
+    (32, 8, 128, [511, 512, 639, 640, 1151, 1152, 634], [0, 0, 0, 0, 0, 0, 5], 10000, 64),
 ])
 def test_sparse_draft_matches_oracle(Hq, Hkv, d, lens, steps, bp, W):
     case, sels, q, kn, vn, out, lse = draft_case(Hq, Hkv, d, lens, steps, bp, W, seed=21)
