@@ -13,7 +13,8 @@
 // element offsets of its positions (index -> page -> slot), then gathers 256-byte K and V rows with 16-byte cp.async (16 lanes per row,
 // coalesced) into a 2-stage pipeline laid out like the TMA tiles of the verify (128-byte
 // swizzle), so the same tensor-core step (one n-tile of 8 rows per warp) serves both.
-// Chunks merge through the workspace in the last CTA of the (request, head).
+// Chunks merge through the workspace in the last CTA of the (request, head); a set that fits
+// one chunk is normalised by its CTA directly, with no record and no ticket.
 #include "attention.cuh"
 #include "kernels.h"
 
@@ -27,6 +28,44 @@ constexpr int kDraftSpan = kDraftChunk + kDraftFold;   // longest chunk
 // at most kDraftFold positions (that remainder goes to the chunk before it).
 __device__ __forceinline__ int draft_nchunks(int A) {
   return max(1, (A + kDraftChunk - 1 - kDraftFold) / kDraftChunk);
+}
+
+// The G rows of a set held by one CTA: merge the 4 position-slice warps in shared scratch
+// and write the normalised outputs and LSE, with the operations (and their order) of a
+// one-record merge followed by the combine of that single record.
+template <int D, int RW, class OutPtr, class LsePtr>
+__device__ __forceinline__ void normalise_slices(const float* redO, const float* redM, const float* redL,
+                                                 int G, OutPtr out_row, LsePtr lse_row, int tid, int nthreads) {
+  constexpr int DS = D + 4;
+  for (int v = tid; v < G * (D / 4); v += nthreads) {
+    const int row = v / (D / 4), d0 = 4 * (v - row * (D / 4));
+    float M = -INFINITY;
+#pragma unroll
+    for (int s = 0; s < 4; ++s) M = fmaxf(M, redM[s * RW + row]);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f}, lsum = 0.f;
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      const float ms = redM[s * RW + row];
+      const float f = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[e] += f * redO[((size_t)s * RW + row) * DS + d0 + e];
+      lsum += f * redL[s * RW + row];
+    }
+    const float w = (M == -INFINITY) ? 0.f : exp2f(M - M) / lsum;
+    float a[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      a[e] = 0.f;
+      a[e] += w * acc[e];
+    }
+    __nv_bfloat162* o = reinterpret_cast<__nv_bfloat162*>(out_row(row) + d0);
+    o[0] = __floats2bfloat162_rn(a[0], a[1]);
+    o[1] = __floats2bfloat162_rn(a[2], a[3]);
+    if (d0 == 0) {
+      float* lp = lse_row(row);
+      if (lp) *lp = (M + log2f(lsum)) * kLn2;
+    }
+  }
 }
 
 template <int D>
@@ -179,19 +218,19 @@ __global__ void __launch_bounds__(128) draft_kernel(const DraftParams p) {
   float* redL = redM + 4 * RW;
   wa.store_shared(redO, redM, redL, warp, lane);
   __syncthreads();
+  auto out_row = [&](int row) { return p.out + ((size_t)r * p.Hq + kvh * G + row) * D; };
+  auto lse_row = [&](int row) -> float* { return p.lse ? p.lse + (size_t)r * p.Hq + kvh * G + row : nullptr; };
+  if (nch == 1) {
+    normalise_slices<D, RW>(redO, redM, redL, G, out_row, lse_row, tid, blockDim.x);
+    return;
+  }
   const size_t rec_floats = (size_t)RW * (D + 2);
   float* recs = p.part + ((size_t)r * Hkv + kvh) * p.nchunk_max * rec_floats;
   merge_slices_to_record<D, RW>(redO, redM, redL, 1, recs + c * rec_floats, RW);
 
   if (!last_of(p.tickets + (size_t)r * Hkv + kvh, nch, s_flag)) return;
   __shared__ float wts[32 * RW];
-  combine_records<D>(
-      recs, rec_floats, nch, G, RW, wts, 32 * RW,
-      [&](int row) { return p.out + ((size_t)r * p.Hq + kvh * G + row) * D; },
-      [&](int row) -> float* {
-        return p.lse ? p.lse + (size_t)r * p.Hq + kvh * G + row : nullptr;
-      },
-      tid, blockDim.x);
+  combine_records<D>(recs, rec_floats, nch, G, RW, wts, 32 * RW, out_row, lse_row, tid, blockDim.x);
 }
 
 template <int D>
