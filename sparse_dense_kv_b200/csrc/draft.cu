@@ -30,26 +30,75 @@ __device__ __forceinline__ int draft_nchunks(int A) {
   return max(1, (A + kDraftChunk - 1 - kDraftFold) / kDraftChunk);
 }
 
-// The G rows of a set held by one CTA: merge the 4 position-slice warps in shared scratch
-// and write the normalised outputs and LSE, with the operations (and their order) of a
-// one-record merge followed by the combine of that single record.
-template <int D, int RW, class OutPtr, class LsePtr>
-__device__ __forceinline__ void normalise_slices(const float* redO, const float* redM, const float* redL,
-                                                 int G, OutPtr out_row, LsePtr lse_row, int tid, int nthreads) {
+// Merge weights of the 4 position-slice warps of each of the G rows, once per (slice, row):
+// fw[s][row] = 2^(m_s - M) (0 for an empty slice), M the rows' maximum, L = sum_s fw l_s
+// (in slice order). Ends with a barrier.
+template <int RW>
+__device__ __forceinline__ void slice_weights(const float* redM, const float* redL, int G, float* fw,
+                                              float* Mrow, float* Lrow, int tid) {
+  if (tid < G) {
+    float M = -INFINITY;
+#pragma unroll
+    for (int s = 0; s < 4; ++s) M = fmaxf(M, redM[s * RW + tid]);
+    float lsum = 0.f;
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      const float ms = redM[s * RW + tid];
+      const float f = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
+      fw[s * RW + tid] = f;
+      lsum += f * redL[s * RW + tid];
+    }
+    Mrow[tid] = M;
+    Lrow[tid] = lsum;
+  }
+  __syncthreads();
+}
+
+// One chunk's record [m: RW][l: RW][O: RW][D] from the slices (rows below G).
+template <int D, int RW>
+__device__ __forceinline__ void slices_to_record(const float* redO, const float* fw, const float* Mrow,
+                                                 const float* Lrow, int G, float* rec, int tid, int nthreads) {
   constexpr int DS = D + 4;
   for (int v = tid; v < G * (D / 4); v += nthreads) {
     const int row = v / (D / 4), d0 = 4 * (v - row * (D / 4));
-    float M = -INFINITY;
-#pragma unroll
-    for (int s = 0; s < 4; ++s) M = fmaxf(M, redM[s * RW + row]);
-    float acc[4] = {0.f, 0.f, 0.f, 0.f}, lsum = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int s = 0; s < 4; ++s) {
-      const float ms = redM[s * RW + row];
-      const float f = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
+      const float f = fw[s * RW + row];
+      const float4 o = *reinterpret_cast<const float4*>(redO + ((size_t)s * RW + row) * DS + d0);
+      acc.x += f * o.x;
+      acc.y += f * o.y;
+      acc.z += f * o.z;
+      acc.w += f * o.w;
+    }
+    *reinterpret_cast<float4*>(rec + 2 * RW + (size_t)row * D + d0) = acc;
+    if (d0 == 0) {
+      rec[row] = Mrow[row];
+      rec[RW + row] = Lrow[row];
+    }
+  }
+}
+
+// The G rows of a set held by one CTA: normalised outputs and LSE straight from the slices,
+// with the operations (and their order) of a one-record merge followed by the combine of
+// that single record.
+template <int D, int RW, class OutPtr, class LsePtr>
+__device__ __forceinline__ void slices_to_output(const float* redO, const float* fw, const float* Mrow,
+                                                 const float* Lrow, int G, OutPtr out_row, LsePtr lse_row,
+                                                 int tid, int nthreads) {
+  constexpr int DS = D + 4;
+  for (int v = tid; v < G * (D / 4); v += nthreads) {
+    const int row = v / (D / 4), d0 = 4 * (v - row * (D / 4));
+    const float M = Mrow[row], lsum = Lrow[row];
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int e = 0; e < 4; ++e) acc[e] += f * redO[((size_t)s * RW + row) * DS + d0 + e];
-      lsum += f * redL[s * RW + row];
+    for (int s = 0; s < 4; ++s) {
+      const float f = fw[s * RW + row];
+      const float4 o = *reinterpret_cast<const float4*>(redO + ((size_t)s * RW + row) * DS + d0);
+      acc[0] += f * o.x;
+      acc[1] += f * o.y;
+      acc[2] += f * o.z;
+      acc[3] += f * o.w;
     }
     const float w = (M == -INFINITY) ? 0.f : exp2f(M - M) / lsum;
     float a[4];
@@ -87,9 +136,20 @@ __global__ void __launch_bounds__(128) draft_kernel(const DraftParams p) {
     if (c == 0 && kvh == 0 && tid == 0) set_error(p.err, S3R_ERR_DEVICE_BOUNDS);
     return;
   }
+  const int Hkv = p.Hkv, G = p.G;
+  // The chunk's selected indices are loaded before the set size is known (within the set's
+  // row of sel_stride entries; those past the size are not used), so these loads and the
+  // length / step / size loads make one round trip.
+  constexpr int kPer = kDraftSpan / 128;
+  const int* sel = p.sel_idx + ((size_t)r * Hkv + kvh) * p.sel_stride;
+  int selv[kPer];
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    const int a = c * kDraftChunk + tid + 128 * u;
+    selv[u] = a < p.sel_stride ? __ldg(sel + a) : -1;
+  }
   const int L = p.seq_lens[r];
   const int i = p.draft_step[r];
-  const int Hkv = p.Hkv, G = p.G;
   const int n = p.sel_count[(size_t)r * Hkv + kvh];
   if (L < 0 || i < 0 || i >= S3R_MAX_K || L + i >= p.cap || n < 0 || n > p.sel_stride) {
     if (c == 0 && tid == 0) set_error(p.err, S3R_ERR_DEVICE_BOUNDS);
@@ -101,7 +161,6 @@ __global__ void __launch_bounds__(128) draft_kernel(const DraftParams p) {
   const int start = c * kDraftChunk;
   const int end = c == nch - 1 ? A : start + kDraftChunk;
   const int* ptab = p.page_table + (size_t)r * p.max_pages;
-  const int* sel = p.sel_idx + ((size_t)r * Hkv + kvh) * p.sel_stride;
   const int64_t npages = p.num_pages;
   const size_t new_off = (size_t)r * p.kv_stride + (size_t)kvh * D;   // this token in k_new / v_new
 
@@ -128,13 +187,12 @@ __global__ void __launch_bounds__(128) draft_kernel(const DraftParams p) {
   });
 
   // Element offsets of the chunk's rows: >= 0 pool offset, -1 zeros, -2 this step's token.
-  // All selected indices are loaded at once, then all page ids: two dependent round trips.
-  constexpr int kPer = kDraftSpan / 128;
+  // The positions from the indices loaded above, then all page ids in one round trip.
   int pos[kPer];
 #pragma unroll
   for (int u = 0; u < kPer; ++u) {
     const int a = start + tid + 128 * u;
-    pos[u] = a < end ? (a < n ? sel[a] : L + (a - n)) : -1;
+    pos[u] = a < end ? (a < n ? selv[u] : L + (a - n)) : -1;
   }
   int page[kPer];
 #pragma unroll
@@ -220,13 +278,15 @@ __global__ void __launch_bounds__(128) draft_kernel(const DraftParams p) {
   __syncthreads();
   auto out_row = [&](int row) { return p.out + ((size_t)r * p.Hq + kvh * G + row) * D; };
   auto lse_row = [&](int row) -> float* { return p.lse ? p.lse + (size_t)r * p.Hq + kvh * G + row : nullptr; };
+  __shared__ float fw[4 * RW], Mrow[RW], Lrow[RW];
+  slice_weights<RW>(redM, redL, G, fw, Mrow, Lrow, tid);
   if (nch == 1) {
-    normalise_slices<D, RW>(redO, redM, redL, G, out_row, lse_row, tid, blockDim.x);
+    slices_to_output<D, RW>(redO, fw, Mrow, Lrow, G, out_row, lse_row, tid, blockDim.x);
     return;
   }
   const size_t rec_floats = (size_t)RW * (D + 2);
   float* recs = p.part + ((size_t)r * Hkv + kvh) * p.nchunk_max * rec_floats;
-  merge_slices_to_record<D, RW>(redO, redM, redL, 1, recs + c * rec_floats, RW);
+  slices_to_record<D, RW>(redO, fw, Mrow, Lrow, G, recs + c * rec_floats, tid, blockDim.x);
 
   if (!last_of(p.tickets + (size_t)r * Hkv + kvh, nch, s_flag)) return;
   __shared__ float wts[32 * RW];
