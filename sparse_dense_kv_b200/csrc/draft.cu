@@ -117,6 +117,56 @@ __device__ __forceinline__ void slices_to_output(const float* redO, const float*
   }
 }
 
+// The combine of up to kDraftFastMerge chunk records, each thread for 4 consecutive d of one
+// row: the records' maxima, sums and O values are all loaded before any is used (one round
+// trip), then the combine's operations in its order (row maximum, sum of the weighted
+// sums, weights 2^(m_c - M) / sum, weighted sum of O over the chunks).
+constexpr int kDraftFastMerge = 4;
+template <int D, int RW, class OutPtr, class LsePtr>
+__device__ __forceinline__ void combine_few_records(const float* recs, size_t rec_floats, int nch, int G,
+                                                    OutPtr out_row, LsePtr lse_row, int tid, int nthreads) {
+  for (int v = tid; v < G * (D / 4); v += nthreads) {
+    const int row = v / (D / 4), d4 = v - row * (D / 4);
+    float mc[kDraftFastMerge], lc[kDraftFastMerge];
+    float4 x[kDraftFastMerge];
+#pragma unroll
+    for (int c = 0; c < kDraftFastMerge; ++c) {
+      if (c < nch) {
+        const float* rc = recs + c * rec_floats;
+        mc[c] = __ldcg(rc + row);
+        lc[c] = __ldcg(rc + RW + row);
+        x[c] = __ldcg(reinterpret_cast<const float4*>(rc + 2 * RW + (size_t)row * D) + d4);
+      }
+    }
+    float M = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < kDraftFastMerge; ++c)
+      if (c < nch) M = fmaxf(M, mc[c]);
+    float lsum = 0.f;
+#pragma unroll
+    for (int c = 0; c < kDraftFastMerge; ++c)
+      if (c < nch) lsum += (mc[c] == -INFINITY) ? 0.f : exp2f(mc[c] - M) * lc[c];
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int c = 0; c < kDraftFastMerge; ++c) {
+      if (c < nch) {
+        const float w = (mc[c] == -INFINITY) ? 0.f : exp2f(mc[c] - M) / lsum;
+        a.x += w * x[c].x;
+        a.y += w * x[c].y;
+        a.z += w * x[c].z;
+        a.w += w * x[c].w;
+      }
+    }
+    __nv_bfloat162* o = reinterpret_cast<__nv_bfloat162*>(out_row(row) + 4 * d4);
+    o[0] = __floats2bfloat162_rn(a.x, a.y);
+    o[1] = __floats2bfloat162_rn(a.z, a.w);
+    if (d4 == 0) {
+      float* lp = lse_row(row);
+      if (lp) *lp = (M + log2f(lsum)) * kLn2;
+    }
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(128) draft_kernel(const DraftParams p) {
   pdl_wait();
@@ -289,6 +339,10 @@ __global__ void __launch_bounds__(128) draft_kernel(const DraftParams p) {
   slices_to_record<D, RW>(redO, fw, Mrow, Lrow, G, recs + c * rec_floats, tid, blockDim.x);
 
   if (!last_of(p.tickets + (size_t)r * Hkv + kvh, nch, s_flag)) return;
+  if (nch <= kDraftFastMerge) {
+    combine_few_records<D, RW>(recs, rec_floats, nch, G, out_row, lse_row, tid, blockDim.x);
+    return;
+  }
   __shared__ float wts[32 * RW];
   combine_records<D>(recs, rec_floats, nch, G, RW, wts, 32 * RW, out_row, lse_row, tid, blockDim.x);
 }
