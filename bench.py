@@ -959,9 +959,11 @@ def oracle_mode(args):
     return {"page": 16 if args.select == "pages" else 1, "greedy": bool(args.greedy)}
 
 
-def oracle_round_sample(spec, lens, pools, page_table, inp_host, reqs, mode=None, timings=None):
+def oracle_round_sample(spec, lens, pools, page_table, inp_host, reqs, mode=None, timings=None,
+                        dtype=np.float64):
     """Oracle rounds for the requests `reqs` (dense copies built outside the timing);
-    `timings` accumulates the seconds of each step of the round."""
+    `timings` accumulates the seconds of each step of the round; `dtype` is the oracle's
+    attention arithmetic (float64, or the float32 timing variant)."""
     from oracle import s3r_oracle as O
     k = spec.k
     kp, vp = pools
@@ -971,8 +973,8 @@ def oracle_round_sample(spec, lens, pools, page_table, inp_host, reqs, mode=None
         H = spec.num_kv_heads
         K = np.stack([O.gather_positions(kp, page_table[r], h, np.arange(L + k + 1)) for h in range(H)])
         V = np.stack([O.gather_positions(vp, page_table[r], h, np.arange(L + k + 1)) for h in range(H)])
-        st = O.RequestState(K, V, L)
-        q = inp_host["q"][r].astype(np.float64)
+        st = O.RequestState(K, V, L, dtype=dtype)
+        q = inp_host["q"][r].astype(dtype)
         O.prefill_scores(st, q[0], inp_host["k"][r][0], inp_host["v"][r][0])
         prepared.append((r, st))
     t0 = time.perf_counter()
@@ -1027,11 +1029,21 @@ def cpu_baseline(spec, lens, cache, inp, budget_s=15.0, mode=None):
                "seconds": s1}
     except ImportError:
         pass
+    # the same sample with the oracle's attention in float32 (its samplers stay float64)
+    t32, s32, timings32 = 0, 0.0, {}
+    for r in reqs:
+        hi = host_inputs(inp, [r])
+        pools, pt = request_pools(r)
+        t, s_ = oracle_round_sample(spec, lens, pools, pt, hi, [r], mode, timings32, dtype=np.float32)
+        t32, s32 = t32 + t, s32 + s_
+    fp32 = {"value": t32 / s32, "unit": UNIT, "cores": oracle_threads(), "seconds": round(s32, 3),
+            "sample": "the same requests, attention in float32 numpy",
+            "step_seconds": {n_: round(v_, 4) for n_, v_ in timings32.items()}}
     return {"value": tokens / secs, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
             "sample": f"one round of requests {reqs[0]}..{reqs[-1]} ({len(reqs)} of "
                       f"{spec.num_requests}), float64 numpy, {secs:.1f} s",
             "step_seconds": {n_: round(v_, 4) for n_, v_ in timings.items()},
-            "single_thread": one}
+            "single_thread": one, "float32": fp32}
 
 
 def run_reference(args, spec):

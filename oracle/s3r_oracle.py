@@ -424,11 +424,16 @@ def greedy_verify(p_logits, drafts):
 
 
 class RequestState:
-    """Dense per-request copy of the cache (positions in order) and the round state."""
+    """Dense per-request copy of the cache (positions in order) and the round state.
 
-    def __init__(self, K: np.ndarray, V: np.ndarray, L: int, sigma: np.ndarray | None = None):
-        self.K = np.array(K, dtype=np.float64)   # [H_kv][capacity][d]
-        self.V = np.array(V, dtype=np.float64)
+    `dtype` is the attention arithmetic's type: float64 (the default) for every parity
+    use; float32 only for the benchmark's timing of a float32 CPU variant (the samplers
+    stay float64 either way)."""
+
+    def __init__(self, K: np.ndarray, V: np.ndarray, L: int, sigma: np.ndarray | None = None,
+                 dtype=np.float64):
+        self.K = np.array(K, dtype=dtype)   # [H_kv][capacity][d]
+        self.V = np.array(V, dtype=dtype)
         self.L = int(L)
         self.sigma = sigma                       # scores from the last dense pass
 
@@ -441,7 +446,7 @@ class RequestState:
 def prefill_scores(state: RequestState, q_x, k_x, v_x):
     """Scores for round 0: a one-row dense pass of the pending token at position L."""
     state.write([state.L], [k_x], [v_x])
-    _, lse, sigma, _ = verify_attention(np.asarray(q_x, np.float64)[None], state.K, state.V, state.L)
+    _, lse, sigma, _ = verify_attention(np.asarray(q_x, state.K.dtype)[None], state.K, state.V, state.L)
     state.sigma = sigma
     return lse, sigma
 
@@ -470,7 +475,7 @@ def run_round(state: RequestState, request: int, seed: int, k: int, budget_bp: i
 
     L = state.L
     Hkv = state.K.shape[0]
-    q_rows = np.asarray(q_rows, np.float64)
+    q_rows = np.asarray(q_rows, state.K.dtype)
     if page > 1:
         sel = [select_pages(state.sigma[h], L, budget_bp, window, page) for h in range(Hkv)]
     else:

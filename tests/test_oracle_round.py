@@ -88,3 +88,28 @@ def test_expected_tau_closed_form():
     assert O.expected_tau([0.0, 1.0]) == 1.0
     a = 0.8
     assert abs(O.expected_tau([a] * 6) - (1 - a ** 7) / (1 - a)) < 1e-12
+
+
+def test_float32_timing_variant_follows_the_float64_round():
+    """The float32 variant timed by the benchmark's CPU baseline computes the same round: on
+    the tiny workload its attention outputs agree with the float64 oracle to float32
+    rounding, and the emitted tokens agree wherever no sampling decision of the float64 round
+    lies within float32 reach of its boundary."""
+    spec = synth.WORKLOADS["tiny"]
+    states = make_states(spec)
+    for r, st in enumerate(states):
+        st32 = O.RequestState(st.K, st.V, st.L, st.sigma, dtype=np.float32)
+        assert st32.K.dtype == np.float32
+        L = st.L
+        q, k, v = synth.token_qkv(spec, r, range(L, L + spec.k + 1))
+        p_log, q_log = synth.token_logits(spec, r, range(L + 1, L + spec.k + 2))
+        args = (r, spec.sample_seed, spec.k, spec.budget_bp, spec.window,
+                q.float().numpy(), k.float().numpy(), v.float().numpy(), q_log[: spec.k], p_log)
+        a = O.run_round(st, *args)
+        b = O.run_round(st32, *args)
+        assert [s.tolist() for s in a["sel"]] == [s.tolist() for s in b["sel"]]
+        np.testing.assert_allclose(b["draft_out"], a["draft_out"], rtol=1e-4, atol=1e-5)
+        np.testing.assert_allclose(b["verify_out"], a["verify_out"], rtol=1e-4, atol=1e-5)
+        np.testing.assert_allclose(b["sigma"], a["sigma"], rtol=1e-4, atol=1e-6)
+        if min(np.min(a["draft_margin"]), np.min(a["margins"])) > 1e-5:
+            assert a["tokens"].tolist() == b["tokens"].tolist()
