@@ -144,6 +144,9 @@ def draft_case(Hq, Hkv, d, lens, steps, budget_bp, window, seed, shuffle=False, 
     # s = 1, sets of 512, 513, 640, 641, 1152, 1153 and 640 positions: the edges of the chunk
     # count where a last remainder of up to 128 positions joins the chunk before it
     (32, 8, 128, [511, 512, 639, 640, 1151, 1152, 634], [0, 0, 0, 0, 0, 0, 5], 10000, 64),
+    # s = 1, sets of 1801, 2176, 2177 and 2304 positions: four chunks (the last CTA combines
+    # the records in one round trip) and five (the general combine)
+    (32, 8, 128, [1800, 2175, 2176, 2300], [0, 0, 0, 3], 10000, 64),
 ])
 def test_sparse_draft_matches_oracle(Hq, Hkv, d, lens, steps, bp, W):
     case, sels, q, kn, vn, out, lse = draft_case(Hq, Hkv, d, lens, steps, bp, W, seed=21)
