@@ -88,6 +88,8 @@ struct SelectParams {
   float* sigma_buf;        // sigma [NR][Hkv][sigma_stride]: the workspace's (logits path) or the caller's
   int sigma_stride;
   int page;                // selection unit: 1 (positions) or S3R_PAGE_SIZE (pages)
+  int num_requests;        // size of every per-request array (request ids are checked)
+  int num_sms;             // SMs of the device (the select grid's pairing of long and short sets)
 };
 
 struct SampleParams {

@@ -393,6 +393,8 @@ static int select_common(const s3r_kv_cache* cache, const s3r_batch* batch, Sele
   p.sel_count = sel_count;
   p.err = w.err;
   p.page = page;
+  p.num_requests = batch->num_requests;
+  p.num_sms = sm_count();
   int nl = 0;
   const int st = launch_select(p, batch->batch, (cudaStream_t)stream, &nl);
   g_launches.fetch_add((uint64_t)nl, std::memory_order_relaxed);
@@ -487,6 +489,7 @@ int s3r_position_scores(const s3r_kv_cache* cache, const s3r_batch* batch,
   p.sigma_buf = scores;
   p.sigma_stride = score_stride;
   p.err = w.err;
+  p.num_requests = batch->num_requests;
   const int st = launch_sigma(p, batch->batch, (cudaStream_t)stream);
   if (st == S3R_OK) g_launches.fetch_add(1, std::memory_order_relaxed);
   return st;

@@ -27,6 +27,7 @@ namespace s3r {
 constexpr int kSelectThreads = 1024;
 constexpr int kSelectMaxN = 49152;   // non-window positions held in shared memory
 constexpr int kSelectBins = 2048;    // digits of up to 11 bits
+constexpr int kSelectRankMax = 1024; // requests per launch ranked for the CTA pairing
 
 __device__ __forceinline__ uint32_t order_key(float f) {
   if (f == 0.f) f = 0.f;              // -0 and +0 compare equal
@@ -72,8 +73,39 @@ __global__ void __launch_bounds__(kSelectThreads, 2) select_kernel(const SelectP
   __shared__ int s_remaining, s_whole;
 
   const int tid = threadIdx.x;
-  const int kvh = blockIdx.x, bl = blockIdx.y;
+  int kvh = blockIdx.x, bl = blockIdx.y;
+  // Balance: the block scheduler places CTA c (linear index) and CTA c + num_sms on the
+  // same SM, and a CTA's work grows with its request's length. With the requests ranked
+  // by length (longest first, ties to the lower slot) and pairs numbered rank * Hkv + head,
+  // CTA c < num_sms takes pair c and CTA num_sms + j takes pair total - 1 - j, so one SM's
+  // two CTAs hold a long and a short set. Up to kSelectRankMax requests per launch.
+  const int nb = gridDim.y, total = nb * p.Hkv;
+  if (total > p.num_sms && p.num_sms > 0 && nb <= kSelectRankMax) {
+    __shared__ int s_len[kSelectRankMax];
+    __shared__ int s_slot;
+    for (int j = tid; j < nb; j += blockDim.x) {
+      const int rj = p.req_ids ? p.req_ids[j] : j;
+      s_len[j] = (rj >= 0 && rj < p.num_requests) ? p.seq_lens[rj] : -1;
+    }
+    __syncthreads();
+    const int c = blockIdx.x + p.Hkv * blockIdx.y;
+    const int t = c < p.num_sms ? c : total - 1 - (c - p.num_sms);
+    const int want = t / p.Hkv;
+    for (int j = tid; j < nb; j += blockDim.x) {
+      const int Lj = s_len[j];
+      int rank = 0;
+      for (int q = 0; q < nb; ++q) rank += (s_len[q] > Lj) || (s_len[q] == Lj && q < j);
+      if (rank == want) s_slot = j;
+    }
+    __syncthreads();
+    bl = s_slot;
+    kvh = t - want * p.Hkv;
+  }
   const int r = p.req_ids ? p.req_ids[bl] : bl;
+  if (r < 0 || r >= p.num_requests) {
+    if (kvh == 0 && tid == 0) set_error(p.err, S3R_ERR_DEVICE_BOUNDS);
+    return;
+  }
   const int L = p.seq_lens[r];
   if (L < 0 || L > p.score_stride) {
     if (tid == 0) set_error(p.err, S3R_ERR_DEVICE_BOUNDS);
@@ -297,6 +329,11 @@ __global__ void __launch_bounds__(kSigmaThreads) sigma_kernel(const SelectParams
   __shared__ float lse2[S3R_MAX_ROWS];
   const int kvh = blockIdx.y, bl = blockIdx.z;
   const int r = p.req_ids ? p.req_ids[bl] : bl;
+  if (r < 0 || r >= p.num_requests) {
+    // reported by the select kernel on its path; here for the scores-only call
+    if (p.window == 0 && blockIdx.x == 0 && kvh == 0 && threadIdx.x == 0) set_error(p.err, S3R_ERR_DEVICE_BOUNDS);
+    return;
+  }
   const int L = p.seq_lens[r];
   if (L < 0 || L > p.cap || L > p.sigma_stride) {
     // reported by the select kernel on its path; here for the scores-only call

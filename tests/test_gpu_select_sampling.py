@@ -61,6 +61,48 @@ def test_select_from_scores_is_bit_exact(bp, W):
             assert np.array_equal(sel[r, h, : ref.size], ref), (r, h)
 
 
+def test_select_pairs_long_and_short_sets_across_a_grid_larger_than_the_gpu():
+    """More (request, KV head) pairs than SMs, so the select kernel pairs CTAs by request
+    length (the CTA that takes a pair is not the grid position of the pair): every pair of
+    the whole batch, of a shuffled subset and of a subset holding an id outside
+    [0, num_requests) (which sets the device-bounds bit and is skipped) matches the oracle
+    bit for bit; pairs outside a launch are left untouched."""
+    rng = np.random.default_rng(77)
+    NR, H = 48, 8
+    lens = rng.integers(1, 6000, size=NR)
+    lens[5] = lens[6] = lens[7] = lens[20]          # equal lengths: ties in the ranking
+    lens = lens.tolist()
+    case, cache, batch = _select_setup(lens)
+    stride = max(lens) + 8
+    scores = (rng.integers(0, 50, size=(NR, H, stride)) / 7.0).astype(np.float32)
+    sd = torch.as_tensor(scores).cuda()
+    ws = s3r.new_workspace(s3r.s3r_workspace_size(cache, NR, case.cache.max_pages, 6, 64, 64))
+    bp, W = 700, 16
+
+    def check(sel, cnt, reqs):
+        sel, cnt = sel.cpu().numpy(), cnt.cpu().numpy()
+        for r in range(NR):
+            for h in range(H):
+                if r not in reqs:
+                    assert cnt[r, h] == -1 and (sel[r, h] == -1).all(), (r, h)
+                    continue
+                ref = O.select_positions(scores[r, h].astype(np.float64), lens[r], bp, W)
+                assert cnt[r, h] == ref.size, (r, h)
+                assert np.array_equal(sel[r, h, : ref.size], ref), (r, h)
+
+    for ids, bad in ((None, False), (rng.permutation(NR)[:40], False), (None, True)):
+        sel = torch.full((NR, H, stride), -1, dtype=torch.int32, device="cuda")
+        cnt = torch.full((NR, H), -1, dtype=torch.int32, device="cuda")
+        if bad:
+            ids = np.concatenate([rng.permutation(NR)[:30], [NR]])
+        b = batch if ids is None else s3r.make_batch(case.seq_lens, case.page_table,
+                                                    req_ids=torch.as_tensor(ids, dtype=torch.int32).cuda())
+        s3r.s3r_select_from_scores(cache, b, sd, bp, W, sel, cnt, ws)
+        err = s3r.s3r_get_error(ws)
+        assert err == ((1 << 5) if bad else 0), err
+        check(sel, cnt, set(range(NR)) if ids is None else {int(x) for x in ids if 0 <= x < NR})
+
+
 def test_select_from_verify_scores_matches_oracle():
     """Verify writes logits + lse; select turns them into scores and picks the same sets as
     the oracle's selection on the oracle's scores (except near-threshold positions)."""
