@@ -39,6 +39,7 @@ struct VerifyParams {
   int req_off;             // launch covers requests req_ids[req_off + b] (or req_off + b)
   int* sched;              // [2] work counter, exited CTAs (zero between launches)
   int wait_limit;          // polls before a wait on another role's progress gives up
+  int num_requests;        // size of every per-request array (request ids are checked)
 };
 
 struct DraftParams {

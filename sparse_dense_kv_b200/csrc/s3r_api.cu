@@ -314,6 +314,7 @@ int s3r_verify_attn(const s3r_kv_cache* cache, const s3r_batch* batch, int32_t k
   std::memset(&p, 0, sizeof(p));
   p.req_ids = batch->req_ids;
   p.seq_lens = batch->seq_lens;
+  p.num_requests = batch->num_requests;
   p.page_table = batch->page_table;
   p.max_pages = batch->max_pages_per_req;
   p.cap = cap;

@@ -38,6 +38,10 @@ __global__ void __launch_bounds__(MAXT) verify_kernel(const __grid_constant__ CU
   const int grp = warp >> 2, slice = warp & 3;
   const int bl = blockIdx.z, kvh = blockIdx.y, c = blockIdx.x;
   const int r = p.req_ids ? p.req_ids[bl] : bl;
+  if (r < 0 || r >= p.num_requests) {
+    if (c == 0 && kvh == 0 && tid == 0) set_error(p.err, S3R_ERR_DEVICE_BOUNDS);
+    return;
+  }
   const int L = p.seq_lens[r];
   const int T = p.T, G = p.G, Lc = L + T;
   if (L < 0 || Lc > p.cap) {
@@ -230,6 +234,7 @@ __global__ void __launch_bounds__(kCombThreads) verify_combine_kernel(const Veri
   extern __shared__ float cw[];   // m, l, weights: [nch][kCombRows] each
   const int j0 = blockIdx.x * kCombRows, kvh = blockIdx.y, bl = blockIdx.z;
   const int r = p.req_ids ? p.req_ids[bl] : bl;
+  if (r < 0 || r >= p.num_requests) return;     // bad ids are reported by the attention kernel
   const int L = p.seq_lens[r];
   const int T = p.T, G = p.G, R = p.R, Rp = p.Rp, Lc = L + T;
   if (L < 0 || Lc > p.cap || j0 >= R) return;   // bad lengths are reported by the attention kernel

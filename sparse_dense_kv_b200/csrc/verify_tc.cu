@@ -292,9 +292,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ---- set-up: request prefix (items), barriers, tensor memory
   for (int b = tid; b < batch; b += blockDim.x) {
     const int r = p.req_ids ? p.req_ids[p.req_off + b] : p.req_off + b;
-    const int L = p.seq_lens[r];
+    const bool known = r >= 0 && r < p.num_requests;   // else no items, bounds reported
+    const int L = known ? p.seq_lens[r] : -1;
     const int Lc = L + T;
-    rid_s[b] = r;
+    rid_s[b] = known ? r : 0;
     lens_s[b] = L;
     int items = 0;
     if (L >= 0 && Lc <= p.cap) items = Hkv * ((Lc + chunk - 1) / chunk);

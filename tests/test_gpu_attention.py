@@ -251,3 +251,31 @@ def test_verify_batch_larger_than_one_launch():
         assert_attention_close(f64(out[r]), o, f"out r={r}")
         np.testing.assert_allclose(f64(lse[r]), l, rtol=0, atol=2e-4)
         np.testing.assert_allclose(f64(sc[r][:, :, :L]), logits[:, :, :L], rtol=1e-5, atol=1e-4)
+
+
+@pytest.mark.parametrize("Hq,Hkv,d", [(32, 8, 128), (2, 1, 64)])
+def test_verify_skips_a_request_id_outside_the_batch(Hq, Hkv, d):
+    """A verify launch over request ids that include one outside [0, num_requests) sets the
+    device-bounds bit, skips that id and gives the other requests the outputs of a launch
+    without it, bit for bit (tensor-memory kernel at d = 128, mma.sync kernel at d = 64)."""
+    k, lens = 6, [300, 700, 500]
+    spec = spec_for(Hq, Hkv, d, lens, k=k, seed=5)
+    case = Case(spec, extra_tokens=k + 1 + 16)
+    NR, T = len(lens), k + 1
+    q = synth.randn_bf16((NR, T, Hq, d), 11, "cuda")
+    kn = synth.randn_bf16((NR, T, Hkv, d), 12, "cuda")
+    vn = synth.randn_bf16((NR, T, Hkv, d), 13, "cuda")
+    cache = s3r.make_cache(case.k_pool, case.v_pool, Hq)
+    ws = s3r.new_workspace(s3r.s3r_workspace_size(cache, NR, case.cache.max_pages, k, 64, 64))
+    res = []
+    for ids, bit in (([2, 0, NR], 1 << 5), ([2, 0], 0)):
+        out = torch.zeros((NR, T, Hq, d), dtype=torch.bfloat16, device="cuda")
+        lse = torch.zeros((NR, T, Hq), dtype=torch.float32, device="cuda")
+        batch = s3r.make_batch(case.seq_lens, case.page_table,
+                               req_ids=torch.as_tensor(ids, dtype=torch.int32).cuda())
+        s3r.s3r_verify_attn(cache, batch, k, q, kn, vn, out, lse, None, ws)
+        assert s3r.s3r_get_error(ws) == bit
+        res.append((out.cpu(), lse.cpu()))
+    for r in (0, 2):
+        assert torch.equal(res[0][0][r], res[1][0][r]) and torch.equal(res[0][1][r], res[1][1][r])
+    assert not res[0][0][1].any() and not res[0][1][1].any()   # request 1 is in neither launch
