@@ -35,9 +35,9 @@
  *     Query head h reads KV head h / G, G = num_q_heads / num_kv_heads <= 8.
  *   - Requests: a launch covers `batch` requests; with req_ids == NULL they are requests
  *     0..batch-1, else req_ids[0..batch-1], which must be distinct and in [0, num_requests)
- *     (the samplers, the sparse draft attention, the selection and the position scores
- *     check the range on the device: an id outside it sets S3R_ERR_DEVICE_BOUNDS and that
- *     request is skipped; the verify does not check it). Every per-request array is indexed
+ *     (every kernel checks the range on the device: an id outside it sets
+ *     S3R_ERR_DEVICE_BOUNDS and that request is skipped; s3r_commit, which has no error
+ *     word, skips it). Every per-request array is indexed
  *     by the request id (size num_requests), so a launch can cover a subset of a larger
  *     batch (mixed round phases).
  *     Attention and selection calls cover at most 65535 requests per launch.

@@ -155,7 +155,7 @@ void spec_offsets(int num_requests, int k, int vocab, size_t* plan_off, size_t* 
 // Byte offset of draft sampling's sub-block sums in its partials area.
 size_t draft_sub_offset(int num_requests, int vocab);
 
-int launch_commit(const int32_t* req_ids, int batch, int k, const int32_t* n_out,
+int launch_commit(const int32_t* req_ids, int batch, int num_requests, int k, const int32_t* n_out,
                   int32_t* seq_lens, int64_t* stats, cudaStream_t stream);
 int launch_philox(uint64_t seed, int stream_id, const int32_t* request, const int32_t* position,
                   int64_t n, uint32_t* words, float* u, cudaStream_t stream);

@@ -760,7 +760,7 @@ int s3r_commit(const s3r_batch* batch, int32_t k, const int32_t* n_out, int32_t*
   if (!n_out || !seq_lens || !aligned4(n_out) || !aligned4(seq_lens)) return S3R_ERR_INVALID_ARG;
   if (stats && (reinterpret_cast<uintptr_t>(stats) & 7u)) return S3R_ERR_INVALID_ARG;
   if (batch->batch == 0) return S3R_OK;
-  return finish(launch_commit(batch->req_ids, batch->batch, k, n_out, seq_lens, stats,
+  return finish(launch_commit(batch->req_ids, batch->batch, batch->num_requests, k, n_out, seq_lens, stats,
                               (cudaStream_t)stream),
                 1);
 }

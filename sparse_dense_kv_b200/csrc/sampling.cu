@@ -742,12 +742,13 @@ int launch_argmax(const SampleParams& p, int batch, int mode, cudaStream_t strea
 }
 
 // ------------------------------------------------------------------------- commit ----
-__global__ void commit_kernel(const int32_t* req_ids, int batch, int k, const int32_t* n_out,
-                              int32_t* seq_lens, long long* stats) {
+__global__ void commit_kernel(const int32_t* req_ids, int batch, int num_requests, int k,
+                              const int32_t* n_out, int32_t* seq_lens, long long* stats) {
   pdl_wait();
   const int bl = blockIdx.x * blockDim.x + threadIdx.x;
   if (bl >= batch) return;
   const int r = req_ids ? req_ids[bl] : bl;
+  if (r < 0 || r >= num_requests) return;   // skipped (the commit has no error word)
   const int n = n_out[r];
   seq_lens[r] += n;
   if (stats) {
@@ -819,10 +820,10 @@ size_t draft_sub_offset(int num_requests, int vocab) {
   return align_up((size_t)num_requests * nvch * sizeof(MS), 256);
 }
 
-int launch_commit(const int32_t* req_ids, int batch, int k, const int32_t* n_out,
+int launch_commit(const int32_t* req_ids, int batch, int num_requests, int k, const int32_t* n_out,
                   int32_t* seq_lens, int64_t* stats, cudaStream_t stream) {
-  launch_pdl(commit_kernel, (batch + 255) / 256, 256, 0, stream, req_ids, batch, k, n_out, seq_lens,
-                                                        reinterpret_cast<long long*>(stats));
+  launch_pdl(commit_kernel, (batch + 255) / 256, 256, 0, stream, req_ids, batch, num_requests, k, n_out,
+             seq_lens, reinterpret_cast<long long*>(stats));
   return cuda_status(cudaGetLastError(), __func__);
 }
 

@@ -391,3 +391,17 @@ def test_draft_row_normalisers_carry_into_spec_sampling(NR, k, V):
     for r in differ:   # only a decision within the rounding of the sums may go the other way
         assert min(m0[r].min(), m1[r].min()) < 1e-5, r
     assert len(differ) <= max(1, NR // 20)
+
+
+def test_commit_skips_a_request_id_outside_the_batch():
+    """s3r_commit over ids that include one outside [0, num_requests) advances the others by
+    their emitted counts and touches nothing for that id (the commit has no error word)."""
+    NR, k = 6, 6
+    seq = torch.as_tensor([100, 200, 300, 400, 500, 600], dtype=torch.int32).cuda()
+    n_out = torch.as_tensor([1, 2, 3, 4, 5, 6], dtype=torch.int32).cuda()
+    stats = torch.zeros(2 + 2 * 8, dtype=torch.int64, device="cuda")   # 2 + 2 S3R_MAX_K counters
+    ids = torch.as_tensor([4, NR, 1, -1], dtype=torch.int32).cuda()
+    s3r.s3r_commit(s3r.make_batch(seq, req_ids=ids), k, n_out, seq, stats)
+    torch.cuda.synchronize()
+    assert seq.cpu().tolist() == [100, 202, 300, 400, 505, 600]
+    assert int(stats[0].item()) == 7 and int(stats[1].item()) == 2
