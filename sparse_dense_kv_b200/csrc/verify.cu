@@ -221,15 +221,18 @@ __global__ void __launch_bounds__(MAXT) verify_kernel(const __grid_constant__ CU
 
 // Merge the chunk records of every (request, KV head) of a verify launch into out / lse.
 // Grid (group of kCombRows rows, KV head, request), so a launch has a few CTAs per SM and
-// every merge runs at once: the group's chunk maxima / sums are loaded in one round, the
-// weights of each row are formed in shared memory, then every thread accumulates two
-// 16-byte output slices over the chunks in chunk order with 8 chunks' loads in flight.
+// every merge runs at once: the group's chunk maxima / sums are loaded in one round (with
+// the first batch of output slices, which do not depend on them), the weights of each row
+// are formed in shared memory, then every thread accumulates two 16-byte output slices over
+// the chunks in chunk order with kCombBatch chunks' loads in flight. kCombMinBlocks CTAs
+// fit an SM, so the 32-request Qwen3-8B launch (1024 CTAs) is one wave.
 constexpr int kCombRows = 8;
 constexpr int kCombThreads = 128;
-constexpr int kCombBatch = 8;   // chunks whose loads are issued together
+constexpr int kCombBatch = 4;   // chunks whose loads are issued together
+constexpr int kCombMinBlocks = 7;
 
 template <int D>
-__global__ void __launch_bounds__(kCombThreads) verify_combine_kernel(const VerifyParams p) {
+__global__ void __launch_bounds__(kCombThreads, kCombMinBlocks) verify_combine_kernel(const VerifyParams p) {
   pdl_wait();
   extern __shared__ float cw[];   // m, l, weights: [nch][kCombRows] each
   const int j0 = blockIdx.x * kCombRows, kvh = blockIdx.y, bl = blockIdx.z;
@@ -245,6 +248,23 @@ __global__ void __launch_bounds__(kCombThreads) verify_combine_kernel(const Veri
   float* mm = cw;
   float* ll = cw + (size_t)nch * kCombRows;
   float* ww = ll + (size_t)nch * kCombRows;
+  constexpr int kQ = D / 4;       // float4 slices per row
+  const int nvec = nr * kQ;
+  // this thread's first output slices (v0, v0 + blockDim.x) and their first batch of chunks
+  const int v0f = threadIdx.x, v1f = v0f + blockDim.x;
+  const float4* recO = reinterpret_cast<const float4*>(recs + 2 * Rp + (size_t)j0 * D);
+  float4 xa[kCombBatch], xb[kCombBatch];
+  const int nb0 = min(kCombBatch, nch);
+  if (v0f < nvec) {
+#pragma unroll
+    for (int u = 0; u < kCombBatch; ++u) {
+      if (u < nb0) {
+        const size_t off = (size_t)u * rec_floats / 4;
+        xa[u] = __ldcg(recO + v0f + off);
+        xb[u] = __ldcg(recO + (v1f < nvec ? v1f : v0f) + off);
+      }
+    }
+  }
   for (int i = threadIdx.x; i < nch * nr; i += blockDim.x) {
     const int c = i / nr, j = i - c * nr;
     mm[c * kCombRows + j] = __ldcg(recs + c * rec_floats + j0 + j);
@@ -269,24 +289,23 @@ __global__ void __launch_bounds__(kCombThreads) verify_combine_kernel(const Veri
     p.lse[((size_t)r * T + t) * p.Hq + kvh * G + g] = (M + log2f(lsum)) * kLn2;
   }
   __syncthreads();
-  constexpr int kQ = D / 4;       // float4 slices per row
-  const int nvec = nr * kQ;
   for (int v0 = threadIdx.x; v0 < nvec; v0 += 2 * blockDim.x) {
     const int v1 = v0 + blockDim.x;
     const bool has1 = v1 < nvec;
     const int ja = v0 / kQ, jb = has1 ? v1 / kQ : ja;
-    const float4* pa = reinterpret_cast<const float4*>(recs + 2 * Rp + (size_t)j0 * D) + v0;
-    const float4* pb = reinterpret_cast<const float4*>(recs + 2 * Rp + (size_t)j0 * D) + (has1 ? v1 : v0);
+    const float4* pa = recO + v0;
+    const float4* pb = recO + (has1 ? v1 : v0);
     float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
     for (int c0 = 0; c0 < nch; c0 += kCombBatch) {
       const int nb = min(kCombBatch, nch - c0);
-      float4 xa[kCombBatch], xb[kCombBatch];
+      if (v0 != v0f || c0 > 0) {   // the first batch of the first slices was loaded above
 #pragma unroll
-      for (int u = 0; u < kCombBatch; ++u) {
-        if (u < nb) {
-          const size_t off = (size_t)(c0 + u) * rec_floats / 4;
-          xa[u] = __ldcg(pa + off);
-          xb[u] = __ldcg(pb + off);
+        for (int u = 0; u < kCombBatch; ++u) {
+          if (u < nb) {
+            const size_t off = (size_t)(c0 + u) * rec_floats / 4;
+            xa[u] = __ldcg(pa + off);
+            xb[u] = __ldcg(pb + off);
+          }
         }
       }
 #pragma unroll
