@@ -10,11 +10,13 @@
 // past the resident ones are mostly the short last chunks of the largest pairs. Chunks are
 // kDraftChunk (512) positions long, except that the last one also takes a remainder of up to
 // kDraftFold positions instead of leaving it to a CTA of its own. The CTA first resolves the
-// element offsets of its positions (index -> page -> slot), then gathers 256-byte K and V rows with 16-byte cp.async (16 lanes per row,
+// element offsets of its positions (selected index, loaded with the set size -> page ->
+// slot), then gathers 256-byte K and V rows with 16-byte cp.async (16 lanes per row,
 // coalesced) into a 2-stage pipeline laid out like the TMA tiles of the verify (128-byte
 // swizzle), so the same tensor-core step (one n-tile of 8 rows per warp) serves both.
-// Chunks merge through the workspace in the last CTA of the (request, head); a set that fits
-// one chunk is normalised by its CTA directly, with no record and no ticket.
+// Chunks merge through the workspace in the last CTA of the (request, head), up to four
+// records in one round trip; a set that fits one chunk is normalised by its CTA directly,
+// with no record and no ticket.
 #include "attention.cuh"
 #include "kernels.h"
 

@@ -12,13 +12,14 @@
 // ceil(n / 16) pages in all (at least the window's); every position of a chosen page below L
 // is emitted, ascending, so the count is at most n + 15.
 //
-// One CTA of 1024 threads per (KV head, request). Scores sigma_j = sum over the G*(k+1)
+// One CTA of 1024 threads per (KV head, request), the CTAs taking the pairs ranked by
+// request length so that the two on an SM hold a long and a short set. Scores sigma_j = sum over the G*(k+1)
 // verify rows of exp(logit - lse) are computed once into shared memory as order-preserving
 // uint32 keys; MSB-first histogram passes over digits of 11, 11 and 10 bits (shared atomics,
 // one block scan over the bins per pass; the first pass is counted while the keys are
 // loaded) find the M-th largest score's digits and how many ties to keep, stopping early
 // once the bin that holds it is taken whole; a final pass compacts the chosen indices in
-// increasing order, each warp over its own contiguous run of positions.
+// increasing order, each thread over its own contiguous run of positions.
 #include "common.cuh"
 #include "kernels.h"
 
