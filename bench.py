@@ -742,8 +742,8 @@ def run_adaptive(args, spec):
     the workload. Each length has its own CUDA graph: k draft steps, verify, speculative
     sampling, commit, and the selection of the next round from this verify's scores (so a
     graph never reads scores of another length); lengths grow from round to round. The
-    costs of a draft step and of the rest of a round come from a line fitted to replays of
-    the graphs of k = 3 .. k_max."""
+    controller prices a round at each length by replaying that length's graph (the line
+    fitted to the replays of k = 3 .. k_max is reported beside it)."""
     import torch
     import sparse_dense_kv_b200 as s3r
 
@@ -810,14 +810,16 @@ def run_adaptive(args, spec):
             graphs[k0].replay()
         # costs per round: t(k) = c_verify + k c_draft, a least-squares line through the
         # replayed graphs of k = 3 .. k_max (one verify configuration: 32-row tiles at G = 4)
+        round_ms = [replay_ms(graphs, k) for k in range(1, k_max + 1)]
         kk = np.arange(min(3, k_max), k_max + 1, dtype=np.float64)
-        tt = np.array([replay_ms(graphs, int(k)) for k in kk])
+        tt = np.array([round_ms[int(k) - 1] for k in kk])
         if kk.size >= 2:
             c_draft, c_verify = (float(x) for x in np.polyfit(kk, tt, 1))
         else:
             c_draft, c_verify = tt[0] / 2, tt[0] / 2
         c_draft, c_verify = max(c_draft, 1e-4), max(c_verify, 1e-4)
-        ctl = s3r.AdaptiveHorizon(eng, c_draft, c_verify, decay=args.decay) if adaptive else None
+        ctl = s3r.AdaptiveHorizon(eng, decay=args.decay, round_costs=round_ms, stale_counts=True) \
+            if adaptive else None
         assert eng.check_errors() == 0, "device error in warm-up"
         tok0 = int(eng.buf.stats[0].item())
         ks = []
@@ -838,7 +840,7 @@ def run_adaptive(args, spec):
         st = eng.buf.stats.cpu().numpy()
         acc = [float(st[2 + j] / max(st[2 + s3r.MAX_K + j], 1)) for j in range(k_max)]
         del graphs
-        return dict(ms=ms, tokens=tokens, ks=ks, c_draft=c_draft, c_verify=c_verify, acc=acc)
+        return dict(ms=ms, tokens=tokens, ks=ks, c_draft=c_draft, c_verify=c_verify, acc=acc, round_ms=round_ms)
 
     fixed = run(False)
     adapt = run(True)
@@ -853,7 +855,8 @@ def run_adaptive(args, spec):
                                f"vocab {V}, adaptive draft length in 1..{k_max}",
                    "requests_per_gpu": NR, "parallelism": "replicas x1", "horizon": "adaptive",
                    "interval": args.interval, "decay": args.decay},
-        "adaptive": {"k_histogram": hist, "c_draft_ms": adapt["c_draft"], "c_verify_ms": adapt["c_verify"],
+        "adaptive": {"k_histogram": hist, "round_cost_ms": adapt["round_ms"],
+                     "c_draft_ms": adapt["c_draft"], "c_verify_ms": adapt["c_verify"],
                      "acceptance_by_position": adapt["acc"][:k_max],
                      "tau": adapt["tokens"] / max(1, args.steps * NR)},
         "fixed_k": {"k": k0, "value": fixed["tokens"] / (fixed["ms"] * 1e-3), "ms_per_step": fixed["ms"] / args.steps,

@@ -382,6 +382,20 @@ S3R_API int s3r_choose_horizon(const double* accepted, const double* decided, in
                        double c_draft, double c_verify, double prior_alpha,
                        double prior_weight, int32_t* k_out);
 
+/* s3r_choose_horizon with a measured cost per draft length instead of the line
+ * k * c_draft + c_verify (HOST function, no device work): writes to *k_out the k in
+ * [1, k_max] that maximises (1 + sum_{i<=k} prod_{j<=i} alpha_j) / round_cost[k-1], the
+ * smallest k on ties, alpha_j as in s3r_choose_horizon (all arithmetic in double, in that
+ * order). A round's cost need not grow linearly with k (the verify's row count steps, the
+ * launches overlap), so costs taken per length can rank the lengths where a line cannot.
+ *   round_cost  host double [k_max]: cost of one round at draft length k = 1..k_max (any
+ *               unit, > 0); not kept.
+ * S3R_ERR_INVALID_ARG for NULL pointers, a cost <= 0 or not finite, or any other argument
+ * s3r_choose_horizon rejects. */
+S3R_API int s3r_choose_horizon_costs(const double* accepted, const double* decided, int32_t k_max,
+                             const double* round_cost, double prior_alpha, double prior_weight,
+                             int32_t* k_out);
+
 /* One decision of the adaptive draft length from the commit counters (HOST function, no
  * device work; [Wispaper] position-dependent acceptance). With the counters of s3r_commit
  * now and at the last decision (host int64 [2 + 2*S3R_MAX_K] each, that layout), for every
@@ -399,6 +413,11 @@ S3R_API int s3r_horizon_step(const int64_t* stats_now, int64_t* stats_last, doub
                      double* decided, int32_t k_max, double decay, double c_draft,
                      double c_verify, double prior_alpha, double prior_weight,
                      double* prior_out, int32_t* k_out);
+
+/* s3r_horizon_step choosing with s3r_choose_horizon_costs (round_cost host double [k_max]). */
+S3R_API int s3r_horizon_step_costs(const int64_t* stats_now, int64_t* stats_last, double* accepted,
+                           double* decided, int32_t k_max, double decay, const double* round_cost,
+                           double prior_alpha, double prior_weight, double* prior_out, int32_t* k_out);
 
 /* Philox4x32-10 words and uniforms for n counters (position[i], request[i], stream_id, 0)
  * under key = seed: words uint32 [n][4] (may be NULL), u fp32 [n] (may be NULL). */

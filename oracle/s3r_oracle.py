@@ -560,6 +560,20 @@ def choose_horizon(accepted, decided, c_draft: float, c_verify: float, k_max: in
     return best_k
 
 
+def choose_horizon_costs(accepted, decided, round_cost, k_max: int, prior_alpha: float = 0.5,
+                         prior_weight: float = 4.0) -> int:
+    """The same choice with the cost of a round measured per draft length (round_cost[k-1]
+    for length k) instead of the line k * c_draft + c_verify: the k with the most expected
+    tokens per unit cost, the smallest k on ties."""
+    alpha = acceptance_estimate(accepted[:k_max], decided[:k_max], prior_alpha, prior_weight)
+    best_k, best = 1, -1.0
+    for k in range(1, k_max + 1):
+        rate = expected_tau(alpha[:k]) / float(round_cost[k - 1])
+        if rate > best:
+            best_k, best = k, rate
+    return best_k
+
+
 def horizon_update(acc, dec, accepted_new, decided_new, decay: float):
     """Decayed counts per position: acc_j <- decay * acc_j + accepted_new_j, the same for the
     decided counts (positions that stop being drafted fade toward the prior)."""
@@ -587,6 +601,15 @@ def horizon_step(acc, dec, accepted_new, decided_new, decay: float, c_draft: flo
     prior = pooled_prior(acc, dec, k_max) if prior_alpha is None else float(prior_alpha)
     return acc, dec, prior, choose_horizon(acc[:k_max], dec[:k_max], c_draft, c_verify, k_max, prior,
                                            prior_weight)
+
+
+def horizon_step_costs(acc, dec, accepted_new, decided_new, decay: float, round_cost, k_max: int,
+                       prior_alpha=None, prior_weight: float = 4.0):
+    """horizon_step choosing with per-length round costs. Returns (acc, dec, prior, k)."""
+    acc, dec = horizon_update(acc, dec, accepted_new, decided_new, decay)
+    prior = pooled_prior(acc, dec, k_max) if prior_alpha is None else float(prior_alpha)
+    return acc, dec, prior, choose_horizon_costs(acc[:k_max], dec[:k_max], round_cost, k_max, prior,
+                                                 prior_weight)
 
 
 def break_even_acceptance(total_ms: float, ar_ms: float, k: int) -> float:

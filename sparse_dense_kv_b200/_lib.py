@@ -89,6 +89,9 @@ def _load():
                                               ctypes.c_double, ctypes.c_double, P]),
         "s3r_horizon_step": (ctypes.c_int, [P, P, P, P, I32, ctypes.c_double, ctypes.c_double,
                                             ctypes.c_double, ctypes.c_double, ctypes.c_double, P, P]),
+        "s3r_choose_horizon_costs": (ctypes.c_int, [P, P, I32, P, ctypes.c_double, ctypes.c_double, P]),
+        "s3r_horizon_step_costs": (ctypes.c_int, [P, P, P, P, I32, ctypes.c_double, P, ctypes.c_double,
+                                                  ctypes.c_double, P, P]),
         "s3r_greedy_verify": (ctypes.c_int, [B, I32, P, P, I32, P, P, P, SZ, P]),
         "s3r_commit": (ctypes.c_int, [B, I32, P, P, P, P]),
         "s3r_philox": (ctypes.c_int, [U64, I32, P, P, I64, P, P, P]),
@@ -371,6 +374,21 @@ def s3r_choose_horizon(accepted, decided, c_draft, c_verify, prior_alpha=0.5, pr
     return int(out.value)
 
 
+def s3r_choose_horizon_costs(accepted, decided, round_cost, prior_alpha=0.5, prior_weight=4.0):
+    """Host call: draft length in [1, len(accepted)] from per-position counts and the cost of a
+    round at each length 1..len(accepted) (round_cost)."""
+    k_max = len(accepted)
+    if len(decided) != k_max or len(round_cost) != k_max:
+        raise ValueError("accepted, decided and round_cost differ in length")
+    arr = ctypes.c_double * max(k_max, 1)
+    a, d, c, out = arr(*accepted), arr(*decided), arr(*round_cost), ctypes.c_int32(0)
+    _check(_lib.s3r_choose_horizon_costs(ctypes.cast(a, ctypes.c_void_p), ctypes.cast(d, ctypes.c_void_p), k_max,
+                                         ctypes.cast(c, ctypes.c_void_p), float(prior_alpha), float(prior_weight),
+                                         ctypes.cast(ctypes.pointer(out), ctypes.c_void_p)),
+           "s3r_choose_horizon_costs")
+    return int(out.value)
+
+
 def s3r_horizon_step(stats_now, stats_last, accepted, decided, k_max, decay, c_draft, c_verify,
                      prior_alpha=-1.0, prior_weight=4.0):
     """Host call: decay / add the counts and choose k. stats_now, stats_last: numpy int64
@@ -389,6 +407,29 @@ def s3r_horizon_step(stats_now, stats_last, accepted, decided, k_max, decay, c_d
                                  float(c_draft), float(c_verify), float(prior_alpha), float(prior_weight),
                                  ctypes.cast(ctypes.pointer(prior), ctypes.c_void_p),
                                  ctypes.cast(ctypes.pointer(k), ctypes.c_void_p)), "s3r_horizon_step")
+    return int(k.value), float(prior.value)
+
+
+def s3r_horizon_step_costs(stats_now, stats_last, accepted, decided, k_max, decay, round_cost,
+                           prior_alpha=-1.0, prior_weight=4.0):
+    """s3r_horizon_step choosing with the cost of a round at each length 1..k_max
+    (round_cost, a sequence of k_max floats). Returns (k, prior used)."""
+    import numpy as np
+    now = np.ascontiguousarray(stats_now, dtype=np.int64)
+    for a, dt in ((stats_last, np.int64), (accepted, np.float64), (decided, np.float64)):
+        if not (isinstance(a, np.ndarray) and a.dtype == dt and a.flags.c_contiguous):
+            raise TypeError("stats_last / accepted / decided must be contiguous numpy arrays")
+    if now.size != 2 + 2 * MAX_K or stats_last.size != now.size or accepted.size != MAX_K or decided.size != MAX_K:
+        raise ValueError("counter arrays of the s3r_commit layout")
+    if len(round_cost) != k_max:
+        raise ValueError("one round cost per draft length 1..k_max")
+    cost = (ctypes.c_double * max(k_max, 1))(*[float(c) for c in round_cost])
+    k, prior = ctypes.c_int32(0), ctypes.c_double(0.0)
+    vp = lambda a: a.ctypes.data_as(ctypes.c_void_p)  # noqa: E731
+    _check(_lib.s3r_horizon_step_costs(vp(now), vp(stats_last), vp(accepted), vp(decided), k_max, float(decay),
+                                       ctypes.cast(cost, ctypes.c_void_p), float(prior_alpha), float(prior_weight),
+                                       ctypes.cast(ctypes.pointer(prior), ctypes.c_void_p),
+                                       ctypes.cast(ctypes.pointer(k), ctypes.c_void_p)), "s3r_horizon_step_costs")
     return int(k.value), float(prior.value)
 
 

@@ -765,62 +765,99 @@ int s3r_commit(const s3r_batch* batch, int32_t k, const int32_t* n_out, int32_t*
                 1);
 }
 
+// Smoothed acceptance per position (the reading of s3r_choose_horizon), or false for an
+// argument it rejects.
+static bool horizon_alpha(const double* accepted, const double* decided, int32_t k_max, double prior_alpha,
+                          double prior_weight, double* alpha) {
+  if (!(prior_alpha >= 0.0 && prior_alpha <= 1.0) || !(prior_weight >= 0.0) || !std::isfinite(prior_weight))
+    return false;
+  for (int j = 0; j < k_max; ++j) {
+    if (!(accepted[j] >= 0.0) || !(decided[j] >= 0.0) || !std::isfinite(accepted[j]) ||
+        !std::isfinite(decided[j]) || decided[j] + prior_weight == 0.0)
+      return false;
+    alpha[j] = (accepted[j] + prior_weight * prior_alpha) / (decided[j] + prior_weight);
+  }
+  return true;
+}
+
+// The k in [1, k_max] with the most expected tokens per unit cost, cost[k-1] the round's
+// cost at length k; the smallest k on ties.
+static int horizon_pick(const double* alpha, int32_t k_max, const double* cost) {
+  int best_k = 1;
+  double best = -1.0, tau = 1.0, run = 1.0;
+  for (int k = 1; k <= k_max; ++k) {
+    run *= alpha[k - 1];
+    tau += run;
+    const double rate = tau / cost[k - 1];
+    if (rate > best) {
+      best = rate;
+      best_k = k;
+    }
+  }
+  return best_k;
+}
+
+static bool costs_ok(const double* round_cost, int32_t k_max) {
+  for (int k = 0; k < k_max; ++k)
+    if (!(round_cost[k] > 0.0) || !std::isfinite(round_cost[k])) return false;
+  return true;
+}
+
 int s3r_choose_horizon(const double* accepted, const double* decided, int32_t k_max,
                        double c_draft, double c_verify, double prior_alpha, double prior_weight,
                        int32_t* k_out) {
   if (!accepted || !decided || !k_out || k_max < 1 || k_max > S3R_MAX_K) return S3R_ERR_INVALID_ARG;
   if (!(c_draft > 0.0) || !(c_verify > 0.0) || !std::isfinite(c_draft) || !std::isfinite(c_verify))
     return S3R_ERR_INVALID_ARG;
-  if (!(prior_alpha >= 0.0 && prior_alpha <= 1.0) || !(prior_weight >= 0.0) || !std::isfinite(prior_weight))
-    return S3R_ERR_INVALID_ARG;
   double alpha[S3R_MAX_K];
-  for (int j = 0; j < k_max; ++j) {
-    if (!(accepted[j] >= 0.0) || !(decided[j] >= 0.0) || !std::isfinite(accepted[j]) ||
-        !std::isfinite(decided[j]) || decided[j] + prior_weight == 0.0)
-      return S3R_ERR_INVALID_ARG;
-    alpha[j] = (accepted[j] + prior_weight * prior_alpha) / (decided[j] + prior_weight);
-  }
-  int best_k = 1;
-  double best = -1.0, tau = 1.0, run = 1.0;
-  for (int k = 1; k <= k_max; ++k) {
-    run *= alpha[k - 1];
-    tau += run;
-    const double rate = tau / ((double)k * c_draft + c_verify);
-    if (rate > best) {
-      best = rate;
-      best_k = k;
-    }
-  }
-  *k_out = best_k;
+  if (!horizon_alpha(accepted, decided, k_max, prior_alpha, prior_weight, alpha)) return S3R_ERR_INVALID_ARG;
+  double cost[S3R_MAX_K];
+  for (int k = 1; k <= k_max; ++k) cost[k - 1] = (double)k * c_draft + c_verify;
+  *k_out = horizon_pick(alpha, k_max, cost);
   return S3R_OK;
 }
 
-int s3r_horizon_step(const int64_t* stats_now, int64_t* stats_last, double* accepted,
-                     double* decided, int32_t k_max, double decay, double c_draft,
-                     double c_verify, double prior_alpha, double prior_weight,
-                     double* prior_out, int32_t* k_out) {
-  if (!stats_now || !stats_last || !accepted || !decided || !k_out) return S3R_ERR_INVALID_ARG;
-  if (k_max < 1 || k_max > S3R_MAX_K || !(decay >= 0.0 && decay <= 1.0)) return S3R_ERR_INVALID_ARG;
-  double acc[S3R_MAX_K], dec[S3R_MAX_K];
+int s3r_choose_horizon_costs(const double* accepted, const double* decided, int32_t k_max,
+                             const double* round_cost, double prior_alpha, double prior_weight,
+                             int32_t* k_out) {
+  if (!accepted || !decided || !round_cost || !k_out || k_max < 1 || k_max > S3R_MAX_K)
+    return S3R_ERR_INVALID_ARG;
+  if (!costs_ok(round_cost, k_max)) return S3R_ERR_INVALID_ARG;
+  double alpha[S3R_MAX_K];
+  if (!horizon_alpha(accepted, decided, k_max, prior_alpha, prior_weight, alpha)) return S3R_ERR_INVALID_ARG;
+  *k_out = horizon_pick(alpha, k_max, round_cost);
+  return S3R_OK;
+}
+
+// The counter update of s3r_horizon_step into acc / dec / *prior (the caller's arrays are
+// not touched yet); false for an argument it rejects.
+static bool horizon_counts(const int64_t* stats_now, const int64_t* stats_last, const double* accepted,
+                           const double* decided, int32_t k_max, double decay, double prior_alpha, double* acc,
+                           double* dec, double* prior) {
+  if (k_max < 1 || k_max > S3R_MAX_K || !(decay >= 0.0 && decay <= 1.0)) return false;
   for (int j = 0; j < S3R_MAX_K; ++j) {
     const int64_t da = stats_now[2 + j] - stats_last[2 + j];
     const int64_t dd = stats_now[2 + S3R_MAX_K + j] - stats_last[2 + S3R_MAX_K + j];
-    if (da < 0 || dd < 0) return S3R_ERR_INVALID_ARG;
+    if (da < 0 || dd < 0) return false;
     acc[j] = decay * accepted[j] + (double)da;
     dec[j] = decay * decided[j] + (double)dd;
   }
-  double prior = prior_alpha;
+  *prior = prior_alpha;
   if (prior_alpha < 0.0) {
     double sa = 0.0, sd = 0.0;
     for (int j = 0; j < k_max; ++j) {
       sa += acc[j];
       sd += dec[j];
     }
-    prior = sd > 0.0 ? sa / sd : 0.5;
+    *prior = sd > 0.0 ? sa / sd : 0.5;
   }
-  int32_t k = 0;
-  const int st = s3r_choose_horizon(acc, dec, k_max, c_draft, c_verify, prior, prior_weight, &k);
-  if (st != S3R_OK) return st;
+  return true;
+}
+
+// Commit a horizon step: the decayed counts, the counters seen, the prior and the length.
+static void horizon_commit(const int64_t* stats_now, int64_t* stats_last, double* accepted, double* decided,
+                           const double* acc, const double* dec, double prior, int32_t k, double* prior_out,
+                           int32_t* k_out) {
   for (int j = 0; j < S3R_MAX_K; ++j) {
     accepted[j] = acc[j];
     decided[j] = dec[j];
@@ -828,6 +865,34 @@ int s3r_horizon_step(const int64_t* stats_now, int64_t* stats_last, double* acce
   for (int j = 0; j < 2 + 2 * S3R_MAX_K; ++j) stats_last[j] = stats_now[j];
   if (prior_out) *prior_out = prior;
   *k_out = k;
+}
+
+int s3r_horizon_step(const int64_t* stats_now, int64_t* stats_last, double* accepted,
+                     double* decided, int32_t k_max, double decay, double c_draft,
+                     double c_verify, double prior_alpha, double prior_weight,
+                     double* prior_out, int32_t* k_out) {
+  if (!stats_now || !stats_last || !accepted || !decided || !k_out) return S3R_ERR_INVALID_ARG;
+  double acc[S3R_MAX_K], dec[S3R_MAX_K], prior = 0.0;
+  if (!horizon_counts(stats_now, stats_last, accepted, decided, k_max, decay, prior_alpha, acc, dec, &prior))
+    return S3R_ERR_INVALID_ARG;
+  int32_t k = 0;
+  const int st = s3r_choose_horizon(acc, dec, k_max, c_draft, c_verify, prior, prior_weight, &k);
+  if (st != S3R_OK) return st;
+  horizon_commit(stats_now, stats_last, accepted, decided, acc, dec, prior, k, prior_out, k_out);
+  return S3R_OK;
+}
+
+int s3r_horizon_step_costs(const int64_t* stats_now, int64_t* stats_last, double* accepted,
+                           double* decided, int32_t k_max, double decay, const double* round_cost,
+                           double prior_alpha, double prior_weight, double* prior_out, int32_t* k_out) {
+  if (!stats_now || !stats_last || !accepted || !decided || !k_out) return S3R_ERR_INVALID_ARG;
+  double acc[S3R_MAX_K], dec[S3R_MAX_K], prior = 0.0;
+  if (!horizon_counts(stats_now, stats_last, accepted, decided, k_max, decay, prior_alpha, acc, dec, &prior))
+    return S3R_ERR_INVALID_ARG;
+  int32_t k = 0;
+  const int st = s3r_choose_horizon_costs(acc, dec, k_max, round_cost, prior, prior_weight, &k);
+  if (st != S3R_OK) return st;
+  horizon_commit(stats_now, stats_last, accepted, decided, acc, dec, prior, k, prior_out, k_out);
   return S3R_OK;
 }
 

@@ -431,11 +431,17 @@ class AdaptiveHorizon:
     good; with prior_alpha="pooled" the prior is the acceptance pooled over all positions so
     far (the plain expectation for a position without evidence of its own)."""
 
-    def __init__(self, engine: S3REngine, c_draft: float, c_verify: float, *, decay: float = 0.8,
-                 prior_alpha="pooled", prior_weight: float = 4.0, k_max: int | None = None):
+    def __init__(self, engine: S3REngine, c_draft: float = 0.0, c_verify: float = 0.0, *, decay: float = 0.8,
+                 prior_alpha="pooled", prior_weight: float = 4.0, k_max: int | None = None,
+                 round_costs=None, stale_counts: bool = False):
         import numpy as np
         self.e = engine
         self.c_draft, self.c_verify = c_draft, c_verify
+        # round_costs: the cost of a round at each length 1..k_max, used instead of the line
+        # k * c_draft + c_verify when given
+        self.round_costs = None if round_costs is None else [float(c) for c in round_costs]
+        if self.round_costs is None and not (c_draft > 0 and c_verify > 0):
+            raise ValueError("give c_draft and c_verify (> 0) or round_costs")
         self.decay, self.prior_alpha, self.prior_weight = decay, prior_alpha, prior_weight
         self.k_max = k_max or engine.buf.k_max
         self.acc = np.zeros(L.MAX_K, dtype=np.float64)
@@ -443,12 +449,37 @@ class AdaptiveHorizon:
         self.last = engine.buf.stats.cpu().numpy().astype(np.int64)
         self.last_prior = None
         self.history = []
+        # stale_counts: each decision reads the counters copied (asynchronously, into pinned
+        # memory) at the previous decision, so the host never waits for the device; the
+        # decisions then lag the counts by one interval
+        self.stale = stale_counts
+        self._host = None
+        self._copied = None
+
+    def _counters(self):
+        import numpy as np
+        if not self.stale:
+            return self.e.buf.stats.cpu().numpy()
+        if self._host is None:
+            self._host = torch.empty_like(self.e.buf.stats, device="cpu").pin_memory()
+            self._copied = torch.cuda.Event()
+            now = self.last.copy()   # nothing copied yet: no new evidence
+        else:
+            self._copied.synchronize()   # recorded an interval ago: long complete
+            now = self._host.numpy().astype(np.int64)
+        self._host.copy_(self.e.buf.stats, non_blocking=True)
+        self._copied.record()
+        return now
 
     def step(self) -> int:
-        now = self.e.buf.stats.cpu().numpy()
+        now = self._counters()
         pa = -1.0 if self.prior_alpha == "pooled" else float(self.prior_alpha)
-        k, self.last_prior = L.s3r_horizon_step(now, self.last, self.acc, self.dec, self.k_max, self.decay,
-                                                self.c_draft, self.c_verify, pa, self.prior_weight)
+        if self.round_costs is not None:
+            k, self.last_prior = L.s3r_horizon_step_costs(now, self.last, self.acc, self.dec, self.k_max,
+                                                          self.decay, self.round_costs, pa, self.prior_weight)
+        else:
+            k, self.last_prior = L.s3r_horizon_step(now, self.last, self.acc, self.dec, self.k_max, self.decay,
+                                                    self.c_draft, self.c_verify, pa, self.prior_weight)
         self.e.set_k(k)
         self.history.append(k)
         return k

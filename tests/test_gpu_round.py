@@ -174,3 +174,26 @@ def test_device_errors_are_reported_not_faulted():
     with pytest.raises(s3r.S3RError):
         s3r.s3r_select_kv(c, b2, torch.empty((2, 1, 14, 64), device="cuda"), lse, 6, 500, 3, sel, cnt, ws)
     assert s3r.s3r_launch_count() == before
+
+
+def test_adaptive_horizon_with_stale_counts_lags_one_interval():
+    """With stale_counts the controller reads the counters it copied at its previous
+    decision: its first decision sees no new evidence (the prior alone), its second the
+    rounds before the first one, and it never waits for the device in between."""
+    spec = synth.WORKLOADS["tiny"]
+    eng = gpu_engine(spec, 0, k_max=spec.k)
+    ctl = s3r.AdaptiveHorizon(eng, c_draft=1.0, c_verify=1000.0, prior_weight=1.0, prior_alpha=0.0,
+                              stale_counts=True)
+
+    def rounds(n):
+        for _ in range(n):
+            lengths = eng.seq_lens.cpu().numpy().tolist()
+            q, k, v, pl, ql = round_inputs(spec.with_(k=eng.k), lengths)
+            eng.round(q, k, v, pl, pl[:, : eng.k].contiguous())
+            assert eng.check_errors() == 0
+
+    rounds(3)
+    # prior 0 and no counts yet: one draft (every longer horizon is expected to add nothing)
+    assert ctl.step() == 1 and eng.k == 1
+    # now the three rounds before the first decision (every draft accepted) are seen
+    assert ctl.step() == spec.k and eng.k == spec.k

@@ -147,3 +147,69 @@ def test_round_buffers_views_share_their_storage_across_lengths():
         for name, p in ptrs.items():
             assert getattr(b, name).data_ptr() == p, (name, k)
     assert b.stats.numel() == 2 + 2 * s3r.MAX_K and len(b.steps) == 6
+
+
+@pytest.mark.parametrize("seed", range(200))
+def test_choose_horizon_costs_matches_oracle(seed):
+    """The cost-table choice against the oracle on random counts and per-length costs."""
+    rng = np.random.default_rng(1000 + seed)
+    k_max = int(rng.integers(1, 9))
+    dec = rng.integers(0, 200, size=k_max).astype(float)
+    if seed % 3 == 0:
+        dec = dec * rng.random(k_max)
+    acc = np.floor(dec * rng.random(k_max) ** (0.3 if seed % 2 else 3.0))
+    cost = np.cumsum(rng.uniform(0.01, 0.2, size=k_max)) + rng.uniform(0.2, 1.0)
+    if seed % 4 == 0:
+        cost = rng.uniform(0.1, 2.0, size=k_max)               # not monotone at all
+    pa, pw = float(rng.uniform(0, 1)), float(rng.choice([0.5, 4.0, 16.0]))
+    want = O.choose_horizon_costs(acc.tolist(), dec.tolist(), cost.tolist(), k_max, pa, pw)
+    assert s3r.s3r_choose_horizon_costs(acc.tolist(), dec.tolist(), cost.tolist(), pa, pw) == want
+
+
+def test_choose_horizon_costs_hand_worked_cases():
+    """Worked by hand: with acceptance 0.8 at every position the expected tokens for k = 1..6
+    are 1.8, 2.44, 2.952, 3.3616, 3.68928, 3.951424; against round costs 0.52, 0.58, 0.64,
+    0.71, 0.78, 0.80 the rates are 3.46, 4.21, 4.61, 4.735, 4.730, 4.939, so k = 6 (a line
+    through the same costs, 0.058 k + 0.468, would rate k = 6 at 3.951/0.816 = 4.84 and k = 5
+    at 3.689/0.758 = 4.87 and pick k = 5). With every draft accepted the tokens are k + 1,
+    and costs 2, 3, 4, 10 give the rate 1 for k = 1, 2, 3: the smallest k wins the tie."""
+    acc, dec = [0.8e6] * 6, [1e6] * 6
+    cost = [0.52, 0.58, 0.64, 0.71, 0.78, 0.80]
+    assert s3r.s3r_choose_horizon_costs(acc, dec, cost, 0.5, 0.0) == 6
+    assert O.choose_horizon_costs(acc, dec, cost, 6, 0.5, 0.0) == 6
+    assert s3r.s3r_choose_horizon(acc, dec, 0.058, 0.468, 0.5, 0.0) == 5
+    assert s3r.s3r_choose_horizon_costs([5.0] * 4, [5.0] * 4, [2.0, 3.0, 4.0, 10.0], 0.5, 0.0) == 1
+    # the line itself as a table gives the line's choice
+    line = [0.058 * k + 0.468 for k in range(1, 7)]
+    assert s3r.s3r_choose_horizon_costs(acc, dec, line, 0.5, 0.0) == 5
+
+
+@pytest.mark.parametrize("seed", range(50))
+def test_horizon_step_costs_matches_oracle(seed):
+    rng = np.random.default_rng(2000 + seed)
+    k_max = int(rng.integers(1, 9))
+    decay = float(rng.choice([0.0, 0.5, 0.8, 1.0]))
+    cost = (np.cumsum(rng.uniform(0.01, 0.2, size=k_max)) + 0.4).tolist()
+    last = np.zeros(2 + 2 * s3r.MAX_K, dtype=np.int64)
+    acc = np.zeros(s3r.MAX_K, dtype=np.float64)
+    dec = np.zeros(s3r.MAX_K, dtype=np.float64)
+    oacc, odec = [0.0] * s3r.MAX_K, [0.0] * s3r.MAX_K
+    now = last.copy()
+    for _ in range(4):
+        d_new = rng.integers(0, 50, size=s3r.MAX_K)
+        a_new = (d_new * rng.random(s3r.MAX_K)).astype(np.int64)
+        now = now.copy()
+        now[2:2 + s3r.MAX_K] += a_new
+        now[2 + s3r.MAX_K:] += d_new
+        k, prior = s3r.s3r_horizon_step_costs(now, last, acc, dec, k_max, decay, cost)
+        oacc, odec, oprior, ok = O.horizon_step_costs(oacc, odec, a_new.tolist(), d_new.tolist(), decay, cost,
+                                                      k_max)
+        assert k == ok and prior == oprior
+        assert acc.tolist() == oacc and dec.tolist() == odec
+        assert (last == now).all()
+
+
+@pytest.mark.parametrize("cost", [[1.0, 0.0], [1.0, -2.0], [1.0, float("inf")], [float("nan"), 1.0]])
+def test_choose_horizon_costs_rejects_bad_costs(cost):
+    with pytest.raises(s3r.S3RError):
+        s3r.s3r_choose_horizon_costs([1.0, 1.0], [2.0, 2.0], cost, 0.5, 1.0)
