@@ -763,7 +763,15 @@ def run_adaptive(args, spec):
                 k=synth.randn_bf16((NR, k_max + 1, Hkv, d), 101, dev),
                 v=synth.randn_bf16((NR, k_max + 1, Hkv, d), 102, dev),
                 p=synth.randn_f32((NR, k_max + 1, V), 103, dev, scale=spec.logit_std))
-    base["qlog"] = base["p"][:, :k_max] + synth.randn_f32((NR, k_max, V), 104, dev, scale=spec.draft_noise_std)
+    noise = synth.randn_f32((NR, k_max, V), 104, dev, scale=1.0)
+    if args.falling_acceptance:
+        # draft noise growing with the draft position, so acceptance falls from about 0.96 at
+        # the first position to about 0.68 at the sixth (the 8B model's 95.8% -> 67.9% that
+        # [Wispaper] reports by draft position); std 0.11 + 0.142 (i - 1) at position i
+        std = torch.tensor([0.11 + 0.142 * i for i in range(k_max)], device=dev).view(1, k_max, 1)
+    else:
+        std = spec.draft_noise_std
+    base["qlog"] = base["p"][:, :k_max] + noise * std
     inputs = {k: dict(q=base["q"][:, : k + 1].contiguous(), k=base["k"][:, : k + 1].contiguous(),
                       v=base["v"][:, : k + 1].contiguous(), p=base["p"][:, : k + 1].contiguous(),
                       qlog=base["qlog"][:, :k].contiguous()) for k in range(1, k_max + 1)}
@@ -852,7 +860,8 @@ def run_adaptive(args, spec):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": f"{spec.name}: {NR} requests, L {spec.lengths} growing "
                                f"by the emitted tokens, {Hq}/{Hkv} heads, d {d}, s {spec.budget_bp / 1e4}, "
-                               f"vocab {V}, adaptive draft length in 1..{k_max}",
+                               f"vocab {V}, adaptive draft length in 1..{k_max}"
+                               + (", draft noise growing with the position" if args.falling_acceptance else ""),
                    "requests_per_gpu": NR, "parallelism": "replicas x1", "horizon": "adaptive",
                    "interval": args.interval, "decay": args.decay},
         "adaptive": {"k_histogram": hist, "round_cost_ms": adapt["round_ms"],
@@ -1118,6 +1127,8 @@ def main(argv=None):
     ap.add_argument("--k-max", type=int, default=7,
                     help="largest adaptive draft length")
     ap.add_argument("--interval", type=int, default=4)
+    ap.add_argument("--falling-acceptance", action="store_true",
+                    help="with --adaptive: draft noise growing with the position (acceptance 0.96 -> 0.68)")
     ap.add_argument("--decay", type=float, default=0.8)
     ap.add_argument("--sched", action="store_true",
                     help="KV-aware admission scheduler model (host; one line)")
