@@ -405,3 +405,26 @@ def test_commit_skips_a_request_id_outside_the_batch():
     torch.cuda.synchronize()
     assert seq.cpu().tolist() == [100, 202, 300, 400, 505, 600]
     assert int(stats[0].item()) == 7 and int(stats[1].item()) == 2
+
+
+def test_select_with_more_requests_than_the_length_ranking_holds():
+    """1030 requests (more than the 1024 the select kernel ranks for its CTA pairing): the
+    CTAs take their pairs in grid order, and sampled pairs match the oracle bit for bit."""
+    rng = np.random.default_rng(91)
+    NR, H = 1030, 2
+    lens = rng.integers(1, 300, size=NR).tolist()
+    case, cache, batch = _select_setup(lens, Hkv=H, Hq=4)
+    stride = max(lens) + 8
+    scores = (rng.integers(0, 30, size=(NR, H, stride)) / 5.0).astype(np.float32)
+    sel = torch.full((NR, H, stride), -1, dtype=torch.int32, device="cuda")
+    cnt = torch.full((NR, H), -1, dtype=torch.int32, device="cuda")
+    ws = s3r.new_workspace(s3r.s3r_workspace_size(cache, NR, case.cache.max_pages, 6, 64, 64))
+    bp, W = 2500, 8
+    s3r.s3r_select_from_scores(cache, batch, torch.as_tensor(scores).cuda(), bp, W, sel, cnt, ws)
+    assert s3r.s3r_get_error(ws) == 0
+    sel, cnt = sel.cpu().numpy(), cnt.cpu().numpy()
+    for r in rng.choice(NR, size=40, replace=False).tolist() + [0, 1023, 1024, NR - 1]:
+        for h in range(H):
+            ref = O.select_positions(scores[r, h].astype(np.float64), lens[r], bp, W)
+            assert cnt[r, h] == ref.size, (r, h)
+            assert np.array_equal(sel[r, h, : ref.size], ref), (r, h)
