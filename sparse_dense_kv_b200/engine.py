@@ -426,10 +426,14 @@ class AdaptiveHorizon:
     """Draft length from the measured acceptance by position: every call of step() reads the
     engine's counters (one device-to-host copy) and s3r_horizon_step decays the kept counts,
     adds the new ones, takes the prior and picks the k with the most expected tokens per unit
-    round cost (c_draft per draft step, c_verify for the rest of the round). Positions not
-    drafted for a while decay toward the prior, so longer horizons are tried again when it is
-    good; with prior_alpha="pooled" the prior is the acceptance pooled over all positions so
-    far (the plain expectation for a position without evidence of its own)."""
+    round cost: c_draft per draft step plus c_verify for the rest of the round, or, with
+    round_costs, the measured cost of a round at each length 1..k_max
+    (s3r_horizon_step_costs). Positions not drafted for a while decay toward the prior, so
+    longer horizons are tried again when it is good; with prior_alpha="pooled" the prior is
+    the acceptance pooled over all positions so far (the plain expectation for a position
+    without evidence of its own). With stale_counts the counters are copied asynchronously
+    and each decision reads the copy started at the previous one, so the host never waits
+    for the device (the decisions lag the counts by one interval)."""
 
     def __init__(self, engine: S3REngine, c_draft: float = 0.0, c_verify: float = 0.0, *, decay: float = 0.8,
                  prior_alpha="pooled", prior_weight: float = 4.0, k_max: int | None = None,
